@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark of the persistent decode program on B200.
+
+Default workload (N=1): the Llama-3.2-1B-shaped decoder (seeded random bf16
+weights) at batch 1 - prefill of a 496-token uniform-random prompt to the first
+token, then 128 greedy decode steps.  One bench step is that whole job; the
+value is generated tokens per second over it (first token + 128 decode tokens
+per sequence).  Decode-only workloads (batch 16/32/48, already prefilled) time
+the 128 decode steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--mode megakernel|per_op_graph] [--impl ours|reference]
+
+Multi-GPU: the sessions shard across GPUs with no exchange (replicas), one
+process per GPU under torchrun; the value is the sum over ranks divided by the
+slowest rank's time.  `--impl reference` times the float64 CPU oracle on the
+host cores on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode step µs and tokens/s at batch 1–48; achieved HBM GB/s vs 8 TB/s peak"
+KV_BYTES_PER_TOKEN = lambda s: 2 * s.n_layers * s.n_kv_heads * s.head_dim * 2  # K and V, bf16
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama1b_b1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--mode", default="megakernel", choices=["megakernel", "per_op_graph"])
+    ap.add_argument("--regions", default="", help="comma-separated region cuts, e.g. 0,8")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tile-bytes", type=int, default=0)
+    ap.add_argument("--slot-bytes", type=int, default=0)
+    ap.add_argument("--workers-per-sm", type=int, default=0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1645.6)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        load = [s for s, r in zip(sm, rows) if float(r[3]) > 250.0] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------- CPU reference --
+def oracle_sample(wl, weights, n_steps: int = 2):
+    """Time the float64 oracle on host cores: the workload's prefill and a few
+    decode steps for one sequence; tokens/s extrapolated to the whole job."""
+    import oracle
+
+    s = wl.model
+    dec = oracle.Decoder(s, weights)
+    prompts = synth.make_prompts(s.vocab, 1, wl.prompt_len, wl.prompt_seed)
+    cache = dec.new_cache(1, wl.prompt_len + n_steps + 1)
+    t0 = time.perf_counter()
+    lg = dec.prefill(cache, prompts)
+    t_prefill = time.perf_counter() - t0
+    tok = oracle.argmax_lowest(lg)
+    ts = []
+    for _ in range(n_steps):
+        t0 = time.perf_counter()
+        lg = dec.step(cache, tok)
+        ts.append(time.perf_counter() - t0)
+        tok = oracle.argmax_lowest(lg)
+    t_step = statistics.median(ts)
+    return t_prefill, t_step
+
+
+def job_tokens(wl, decode_steps):
+    """Tokens one bench step generates, and whether the prefill is part of it
+    (decode-only workloads start from an already-prefilled prompt)."""
+    with_prefill = not wl.name.startswith("llama1b_decode")
+    return wl.batch * ((1 if with_prefill else 0) + decode_steps), with_prefill
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = synth.WORKLOADS[args.workload]
+    decode_steps = wl.steps if args.decode_steps is None else args.decode_steps
+    weights = synth.cached_weights(wl.model, seed=0)
+    cores = os.cpu_count()
+    # warm-up + timed samples: one decode step each, prefill measured once
+    import oracle
+
+    s = wl.model
+    dec = oracle.Decoder(s, weights)
+    prompts = synth.make_prompts(s.vocab, 1, wl.prompt_len, wl.prompt_seed)
+    cache = dec.new_cache(1, wl.prompt_len + args.warmup + args.steps + 1)
+    t0 = time.perf_counter()
+    tok = oracle.argmax_lowest(dec.prefill(cache, prompts))
+    t_prefill = time.perf_counter() - t0
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        tok = oracle.argmax_lowest(dec.step(cache, tok))
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    t_step = statistics.median(times)
+    tokens, with_prefill = job_tokens(wl, decode_steps)
+    per_seq = (t_prefill if with_prefill else 0.0) + decode_steps * t_step
+    value = tokens / (per_seq * wl.batch)  # the oracle runs the sequences one after another
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "prompt_len": wl.prompt_len, "decode_steps": decode_steps},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"float64 NumPy oracle, one sequence: prefill of {wl.prompt_len} tokens "
+                                   f"({t_prefill:.2f} s) and {args.steps} timed decode steps (median "
+                                   f"{t_step * 1e3:.0f} ms); job time extrapolated to {decode_steps} steps"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- ours --
+def algorithmic_bytes_per_step(shape, weight_bytes, batch, ctx_len):
+    """Weights once + KV read over ctx_len tokens + KV written for 1 token, per sequence."""
+    kv = KV_BYTES_PER_TOKEN(shape)
+    return weight_bytes + batch * (ctx_len * kv + kv)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+
+    from streaming_persistent_sm_b200 import wpk as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    wl = synth.WORKLOADS[args.workload]
+    s = wl.model
+    B, T = wl.batch, wl.prompt_len
+    decode_steps = wl.steps if args.decode_steps is None else args.decode_steps
+    tokens_per_step, with_prefill = job_tokens(wl, decode_steps)
+    ctx = T + max(decode_steps, 1)
+    weights = synth.cached_weights(s, seed=0)
+    mode = W.WPK_MEGAKERNEL if args.mode == "megakernel" else W.WPK_PER_OP_GRAPH
+    plan = dict(mode=mode, tile_bytes=args.tile_bytes, slot_bytes=args.slot_bytes,
+                workers_per_sm=args.workers_per_sm)
+    if args.regions:
+        cuts = [int(x) for x in args.regions.split(",")]
+        plan.update(n_regions=len(cuts), region_cut=tuple(cuts))
+    eng = W.Engine(s, weights, B, ctx, **plan)
+    stats = eng.stats
+    prompts = synth.make_prompts(s.vocab, B, T, wl.prompt_seed + 17 * rank)
+    prompts_dev = torch.as_tensor(prompts, device=dev)
+    out_dev = torch.empty((max(decode_steps, 1) + 1, B), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    launches_per_decode = stats["n_regions"] if mode == W.WPK_MEGAKERNEL else stats["n_ops"]
+
+    def prefill():
+        W.wpk_prefill(eng.h, prompts_dev.data_ptr(), B, T, out_dev[0].data_ptr(), 0, sp)
+
+    def decode(ev=None):
+        for i in range(decode_steps):
+            if ev is not None:
+                ev[i][0].record(stream)
+            W.wpk_step(eng.h, 0, out_dev[i + 1].data_ptr(), 0, sp)
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    def job(ev=None, pev=None):
+        if with_prefill:
+            if pev is not None:
+                pev[0].record(stream)
+            prefill()
+            if pev is not None:
+                pev[1].record(stream)
+        else:
+            prefill()  # untimed part of decode-only workloads is excluded below
+        decode(ev)
+
+    # decode-only workloads: the prompt is prefilled outside the timed region
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        job()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms, dec_us, pre_ms = [], [], []
+    with ClockSampler(local) as clk:
+        if with_prefill:
+            t0, t1 = mk(), mk()
+            evs = [[[mk(), mk()] for _ in range(decode_steps)] for _ in range(args.steps)]
+            pevs = [[mk(), mk()] for _ in range(args.steps)]
+            torch.cuda.synchronize()
+            t0.record(stream)
+            for k in range(args.steps):
+                job(evs[k], pevs[k])
+            t1.record(stream)
+            torch.cuda.synchronize()
+            total_ms = t0.elapsed_time(t1)
+            for k in range(args.steps):
+                pre_ms.append(pevs[k][0].elapsed_time(pevs[k][1]))
+                dec_us += [a.elapsed_time(b) * 1e3 for a, b in evs[k]]
+        else:
+            total_ms = 0.0
+            for k in range(args.steps):
+                prefill()
+                evs = [[mk(), mk()] for _ in range(decode_steps)]
+                t0, t1 = mk(), mk()
+                t0.record(stream)
+                decode(evs)
+                t1.record(stream)
+                torch.cuda.synchronize()
+                total_ms += t0.elapsed_time(t1)
+                dec_us += [a.elapsed_time(b) * 1e3 for a, b in evs]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms_per_step = total_ms / args.steps
+    value = world * tokens_per_step / (ms_per_step / 1e3)
+
+    # roofline of the dominant kernel (the persistent decode program): bytes per
+    # launch over the launch durations measured above
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    kvb = KV_BYTES_PER_TOKEN(s)
+    dec_ctx = [T + i for i in range(decode_steps)]  # tokens already cached at each decode step
+    algo_dec = [algorithmic_bytes_per_step(s, stats["weight_bytes"], B, c) for c in dec_ctx]
+    algo_pre = [algorithmic_bytes_per_step(s, stats["weight_bytes"], B, c) for c in range(T)] if with_prefill else []
+    launch_bytes = sum(algo_dec) + sum(algo_pre)
+    launch_ms = sum(dec_us) / 1e3 / args.steps + (statistics.mean(pre_ms) if pre_ms else 0.0)
+    achieved_gbs = launch_bytes / (launch_ms / 1e3) / 1e9
+    dec_gbs = statistics.mean(algo_dec) / (statistics.median(dec_us) / 1e6) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "accum_dtype": "fp32", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "prompt_len": T, "decode_steps": decode_steps,
+                   "timed": "prefill + decode steps" if with_prefill else "decode steps (prompt prefilled untimed)",
+                   "mode": args.mode, "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
+                   "workers": stats["n_workers"],
+                   "l2": "inputs larger than L2: %.2f GB of weights streamed per step" % (stats["weight_bytes"] / 1e9)},
+        "decode_step_us": {"median": statistics.median(dec_us), "p95": float(np.percentile(dec_us, 95)),
+                           "achieved_gbs": dec_gbs, "frac_of_8tbs": dec_gbs / 8000.0},
+        "ttft_ms": statistics.median(pre_ms) if pre_ms else None,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "traffic": None,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "wpk_persistent_kernel" if mode == W.WPK_MEGAKERNEL else "wpk_per_op_kernel"},
+        "gpu_launches": args.steps * launches_per_decode * ((T if with_prefill else 0) + decode_steps),
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the C ABI with host buffers: pinned prompt -> device,
+    # prefill + decode, tokens -> pinned host, all inside the timed region
+    host_prompt = torch.from_numpy(prompts).pin_memory()
+    host_out = torch.empty((decode_steps + 1, B), dtype=torch.int32).pin_memory()
+    torch.cuda.synchronize()
+    e2e_runs = max(1, min(args.steps, 3))
+    t0 = time.perf_counter()
+    for _ in range(e2e_runs):
+        prompts_dev.copy_(host_prompt, non_blocking=True)
+        prefill()
+        decode()
+        host_out.copy_(out_dev[: decode_steps + 1], non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_s = (time.perf_counter() - t0) / e2e_runs
+    line["e2e"] = {"value": world * tokens_per_step / e2e_s, "unit": "tokens/s",
+                   "h2d_bytes_per_step": int(host_prompt.numel() * 4),
+                   "d2h_bytes_per_step": int((decode_steps + 1) * B * 4)}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_pre, t_step = oracle_sample(wl, weights, n_steps=2)
+        per_seq = (t_pre if with_prefill else 0.0) + decode_steps * t_step
+        cpu_value = tokens_per_step / (per_seq * B)
+        line["cpu_baseline"] = {
+            "value": cpu_value, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"float64 NumPy oracle, one sequence: {T}-token prefill ({t_pre:.1f} s) + 2 decode steps "
+                      f"(median {t_step:.2f} s); extrapolated to {decode_steps} steps and {B} sequences"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    eng.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,239 @@
+/*
+ * wpk.h - C ABI of the persistent decode/prefill library for one B200 (sm_100a).
+ *
+ * The library runs one recurring decoder update - a Llama-style decode step,
+ * and the prompt prefill that yields the first token - as a persistent GPU
+ * program instead of a sequence of kernel launches.  Resident workers (one or
+ * more CTAs per SM) pull tiles from a device-side ticket queue; a host-built
+ * tile graph with per-tile dependency counters replaces the barriers between
+ * ops ("One Megakernel is Not Enough", Table I: cross-kernel readiness); each
+ * tile's weight load is issued into its worker's staging slot before its
+ * predecessors finish (Table I: weight prefetch); tensors consumed inside one
+ * tile are not stored and reloaded (Table I: on-chip forwarding).  The same
+ * tiles can also run as 1-4 region launches or as per-op launches captured in
+ * a CUDA Graph, so compositions can be compared ("One Megakernel is Not
+ * Enough", abstract and Fig. 3; "Persistent threads and megakernels", §7).
+ *
+ * Conventions for every entry point:
+ *   - Return value: WPK_OK (0) or a negative WPK_ERR_* code.  Nothing aborts,
+ *     traps or exits the process.  wpk_last_error() gives a message.
+ *   - Pointers named *_dev are CUDA device pointers; everything else is host.
+ *   - `stream` arguments are cudaStream_t values passed as void* (NULL = the
+ *     legacy default stream).
+ *   - A handle is not thread-safe: use it from one host thread at a time.
+ *   - Ownership: the caller allocates and owns the three large device buffers
+ *     sized by wpk_workspace_size (weights, KV pages, scratch) and keeps them
+ *     alive until wpk_destroy.  The library owns the handle, its host tables
+ *     and small device tables (tiles, counters, queue heads, trace, error word).
+ *   - After WPK_ERR_TIMEOUT the handle is poisoned: every call but
+ *     wpk_last_error / wpk_get_error_info / wpk_get_trace / wpk_destroy returns
+ *     WPK_ERR_POISONED.
+ */
+#ifndef WPK_H_
+#define WPK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ codes */
+enum {
+  WPK_OK = 0,
+  WPK_ERR_INVALID_ARG = -1,  /* bad pointer, size or enum value            */
+  WPK_ERR_CUDA = -2,         /* a CUDA runtime call failed                  */
+  WPK_ERR_TIMEOUT = -3,      /* a device or host wait gave up (stall)       */
+  WPK_ERR_NOT_LOADED = -4,   /* weights / prefill missing                   */
+  WPK_ERR_SHAPE = -5,        /* shape outside what the plan was built for   */
+  WPK_ERR_UNSUPPORTED = -6,  /* valid request this build does not implement */
+  WPK_ERR_POISONED = -7      /* handle unusable after a timeout             */
+};
+
+enum { WPK_MEGAKERNEL = 0, WPK_PER_OP_GRAPH = 1 };
+
+/* --------------------------------------------------------------- configs */
+/* Decoder shape.  Weights are bf16, matmul weights stored [out][in]. */
+typedef struct wpk_model_cfg {
+  int n_layers, hidden, n_heads, n_kv_heads, head_dim, ffn, vocab;
+  float rms_eps, rope_theta;
+  int tied_embedding;   /* 1: the LM head is the token embedding */
+} wpk_model_cfg;
+
+/* Execution plan: the operating point the program is compiled for ("Why
+ * real-time inference wants a megakernel", section "The cohort is known":
+ * a model, a device, a session capacity and a context limit).  Zero fields
+ * take the defaults noted. */
+typedef struct wpk_plan_cfg {
+  int max_batch;        /* sequences per step (session capacity)               */
+  int max_context;      /* tokens per sequence, prompt included                */
+  int page_tokens;      /* KV page size in tokens (0 = 64)                     */
+  int n_workers;        /* resident worker CTAs (0 = #SMs x workers_per_sm)    */
+  int workers_per_sm;   /* 0 = 2                                               */
+  int mode;             /* WPK_MEGAKERNEL or WPK_PER_OP_GRAPH                  */
+  int resident;         /* megakernel only: 1 = the grid stays alive across
+                           steps and is driven by a host doorbell              */
+  int n_regions;        /* megakernel only: 1..4 launches per step (0 = 1)     */
+  int region_cut[4];    /* first layer of each region; region_cut[0] = 0; a cut
+                           equal to n_layers puts the LM head in its own region */
+  int trace;            /* 1 = record the per-tile device trace                */
+  uint64_t wait_timeout_ns; /* bound on every device wait (0 = 2 s)            */
+  int slot_bytes;       /* staging slot per worker (0 = 65536)                 */
+  int tile_bytes;       /* target weight bytes per tile (0 = 32768)            */
+  int split_pages;      /* KV pages per attention split (0 = 1)                */
+} wpk_plan_cfg;
+
+/* Host weights: bf16 bit patterns, row-major [out][in]. */
+typedef struct wpk_layer_weights {
+  const uint16_t *attn_norm;   /* [hidden]                     */
+  const uint16_t *wq;          /* [n_heads*head_dim][hidden]   */
+  const uint16_t *wk;          /* [n_kv_heads*head_dim][hidden]*/
+  const uint16_t *wv;          /* [n_kv_heads*head_dim][hidden]*/
+  const uint16_t *wo;          /* [hidden][n_heads*head_dim]   */
+  const uint16_t *ffn_norm;    /* [hidden]                     */
+  const uint16_t *w_gate;      /* [ffn][hidden]                */
+  const uint16_t *w_up;        /* [ffn][hidden]                */
+  const uint16_t *w_down;      /* [hidden][ffn]                */
+} wpk_layer_weights;
+
+typedef struct wpk_weights {
+  const uint16_t *embed;             /* [vocab][hidden]                      */
+  const uint16_t *final_norm;        /* [hidden]                             */
+  const uint16_t *lm_head;           /* [vocab][hidden]; NULL when tied      */
+  const wpk_layer_weights *layers;   /* [n_layers]                           */
+} wpk_weights;
+
+typedef struct wpk_handle wpk_handle;
+
+/* Counts describing a compiled graph (for tests and reports). */
+typedef struct wpk_graph_stats {
+  int64_t n_tiles;          /* tiles per decode step (one epoch)              */
+  int64_t n_counters;       /* dependency counters after dedup                */
+  int64_t n_edges;          /* tile-to-tile edges before counter dedup        */
+  int64_t n_signals;        /* counter increments per step                    */
+  int64_t n_ops;            /* op groups (= launches per step in per-op mode) */
+  int64_t n_workers;        /* worker CTAs of the persistent grid             */
+  int64_t weight_bytes;     /* algorithmic weight bytes read per step         */
+  int64_t region_begin[5];  /* ticket boundaries of the regions               */
+  int64_t n_regions;
+} wpk_graph_stats;
+
+/* One trace record per tile of the last traced step (wpk_plan_cfg.trace). */
+typedef struct wpk_trace_rec {
+  uint32_t tile;        /* tile index (= ticket within the step)               */
+  uint16_t worker;      /* worker CTA that ran it                              */
+  uint16_t op;          /* op code                                             */
+  uint32_t ev_issue;    /* event clock when its staging load was issued        */
+  uint32_t ev_start;    /* event clock after its dependency wait succeeded     */
+  uint32_t ev_done;     /* event clock after its body, before it signalled     */
+  uint32_t epoch;       /* step epoch it belongs to                            */
+  uint64_t t_start_ns;  /* %globaltimer after the wait                         */
+  uint64_t t_end_ns;    /* %globaltimer after the body                         */
+} wpk_trace_rec;
+
+/* The first device error recorded by the program. */
+typedef struct wpk_error_info {
+  int32_t code;         /* WPK_ERR_* or 0                                      */
+  uint32_t tile;        /* tile that failed                                    */
+  uint32_t counter;     /* counter it waited on (0xFFFFFFFF if none)           */
+  uint32_t epoch;
+  uint32_t observed;    /* counter value seen when it gave up                  */
+  uint32_t target;      /* value it waited for                                 */
+} wpk_error_info;
+
+/* ----------------------------------------------------------- entry points */
+
+/* Compile the tile graph for a model and plan (host only; also allocates the
+ * library's small device tables on the current device).  Splits every op into
+ * tiles sized to the staging slot, derives tile-to-tile tensor edges, dedups
+ * counters by predecessor set, emits the ticket order and region cuts
+ * ("Why real-time inference wants a megakernel", "A concrete design": the
+ * compiled program is worker assignment, ordering, synchronization and the
+ * memory plan).  *out receives the handle.  Errors: INVALID_ARG, SHAPE,
+ * UNSUPPORTED, CUDA. */
+int wpk_build_graph(const wpk_model_cfg *model, const wpk_plan_cfg *plan, wpk_handle **out);
+
+/* Bytes the caller must allocate (device memory, 256-byte aligned) for the
+ * arranged weights, the paged KV cache and the activation scratch. */
+int wpk_workspace_size(const wpk_handle *h, size_t *weight_bytes, size_t *kv_bytes,
+                       size_t *scratch_bytes);
+
+/* Arrange the host bf16 weights into tile-contiguous blocks (each tile's
+ * weights become one contiguous bulk copy) and copy them to dev_weights; bind
+ * the KV and scratch buffers.  Synchronous with respect to the host buffers
+ * (they may be freed on return); the device copy is ordered on `stream`. */
+int wpk_load_weights(wpk_handle *h, const wpk_weights *w, void *dev_weights, void *dev_kv,
+                     void *dev_scratch, void *stream);
+
+/* Replace the KV block table (host array [max_batch][max_blocks] of page ids,
+ * each < max_batch*max_blocks and distinct).  Results do not depend on it. */
+int wpk_set_block_table(wpk_handle *h, const int32_t *table);
+
+/* Prompt prefill: tokens_dev [batch][prompt_len] (int32, row-major) fills the
+ * KV cache from position 0, resets the step epoch, and writes the first
+ * greedy token per sequence to first_tok_dev [batch] and, if logits_dev is
+ * not NULL, the fp32 logits at the last prompt position to logits_dev
+ * [batch][vocab].  Stream-ordered on `stream`.  batch <= max_batch,
+ * prompt_len + decode steps <= max_context. */
+int wpk_prefill(wpk_handle *h, const int32_t *tokens_dev, int batch, int prompt_len,
+                int32_t *first_tok_dev, float *logits_dev, void *stream);
+
+/* One decode step for the active batch: consumes in_tok_dev [batch] (NULL =
+ * feed back the last greedy tokens), writes the greedy tokens to out_tok_dev
+ * [batch] (may be NULL) and the fp32 logits to logits_dev [batch][vocab] (may
+ * be NULL).  Stream-ordered in launch modes; in resident mode it rings the
+ * grid's doorbell and returns when the device publishes completion (or
+ * WPK_ERR_TIMEOUT). */
+int wpk_step(wpk_handle *h, const int32_t *in_tok_dev, int32_t *out_tok_dev, float *logits_dev,
+             void *stream);
+
+/* Graph facts; *st is filled. */
+int wpk_graph_stats_get(const wpk_handle *h, wpk_graph_stats *st);
+
+/* Tile-to-tile edges of one step as (producer, consumer) pairs: writes up to
+ * max_pairs pairs into pairs[2*i], pairs[2*i+1]; *n_pairs gets the total. */
+int wpk_get_edges(const wpk_handle *h, int32_t *pairs, int64_t max_pairs, int64_t *n_pairs);
+
+/* Op code of every tile in ticket order (int32 [n_tiles]). */
+int wpk_get_tile_ops(const wpk_handle *h, int32_t *ops, int64_t n);
+
+/* Check the compiled graph on the host: the ticket order is topological,
+ * every read-after-write, write-after-read and write-after-write pair of
+ * accesses to the same tensor range is ordered by a path of edges (commuting
+ * accumulations excepted), and every counter's target equals its signal count.
+ * Returns WPK_OK or WPK_ERR_SHAPE with the first violation in
+ * wpk_last_error.  Cost is quadratic in tiles: meant for small configs. */
+int wpk_verify_graph(const wpk_handle *h);
+
+/* Run the compiled ticket queue on `n_threads` host threads standing in for
+ * workers (same atomic ticket claim, counter targets and signals, random
+ * delays from `seed`) for `n_epochs` steps.  Writes the order in which tiles
+ * finished (int32 [n_epochs*n_tiles]) to done_order if not NULL.  A thread
+ * whose wait exceeds wait_ms returns WPK_ERR_TIMEOUT.  `stuck_tile` >= 0 makes
+ * that tile never signal (fault injection on the host). */
+int wpk_simulate(const wpk_handle *h, int n_threads, int n_epochs, uint64_t seed, int wait_ms,
+                 int stuck_tile, int32_t *done_order);
+
+/* Copy the last traced step's records (n_tiles wpk_trace_rec) to host_buf.
+ * Synchronizes the device. */
+int wpk_get_trace(wpk_handle *h, void *host_buf, size_t bytes);
+
+/* First device error (code 0 if none).  Synchronizes the device. */
+int wpk_get_error_info(wpk_handle *h, wpk_error_info *info);
+
+/* Human-readable message for the last failing call on this handle. */
+const char *wpk_last_error(const wpk_handle *h);
+
+/* Stop the resident grid (if any), release library-owned tables, free h. */
+int wpk_destroy(wpk_handle *h);
+
+/* Test hook: make counter `counter` need one more signal than it can ever get
+ * (an unsatisfiable dependency), so the next step's device wait must time out
+ * and return WPK_ERR_TIMEOUT.  Host-side fault injection; no GPU fault. */
+int wpk_debug_break_counter(wpk_handle *h, int counter);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WPK_H_ */

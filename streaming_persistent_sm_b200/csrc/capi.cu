@@ -1,0 +1,543 @@
+// C ABI of the persistent decode library (declared in include/wpk.h).
+//
+// Host side of the runtime: device tables, launches per step (cooperative
+// persistent grid per region, or per-op launches captured once into a CUDA
+// Graph and replayed), prompt prefill, error word and trace access.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "graph.h"
+
+namespace wpk {
+size_t worker_smem_bytes(int slot_bytes);
+const void* persistent_kernel_ptr();
+const void* per_op_kernel_ptr();
+}  // namespace wpk
+
+using namespace wpk;
+
+struct GraphEntry {
+  int32_t* out_tok;
+  float* logits;
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+};
+
+struct wpk_handle {
+  CompiledGraph g;
+  int device = 0, n_sms = 0, n_workers = 0;
+  size_t smem = 0;
+  // library-owned device tables (one allocation)
+  uint8_t* d_base = nullptr;
+  Tile* d_tiles = nullptr;
+  uint32_t* d_sig = nullptr;
+  uint32_t* d_ctr = nullptr;
+  uint32_t* d_head = nullptr;
+  ErrWord* d_err = nullptr;
+  TraceRec* d_trace = nullptr;
+  uint32_t* d_evclock = nullptr;
+  LayerDev* d_layers = nullptr;
+  float2* d_rope = nullptr;
+  int32_t* d_block_table = nullptr;
+  uint32_t* d_arrive = nullptr;
+  unsigned long long* d_best = nullptr;
+  int32_t* d_seqlen = nullptr;
+  int32_t* d_tok_fb = nullptr;
+  int32_t* d_active = nullptr;
+  int32_t* h_err_code = nullptr;  // pinned mirror of d_err->code
+  // caller-owned buffers
+  uint8_t* weights = nullptr;
+  uint16_t* kv = nullptr;
+  uint8_t* scratch = nullptr;
+  size_t kv_bytes = 0, scratch_bytes = 0;
+  size_t off_xa = 0, off_xb = 0, off_q = 0, off_attn = 0, off_h = 0, off_part = 0;
+  int64_t n_blocks = 0;
+  bool loaded = false, prefilled = false, poisoned = false, has_device = false;
+  int batch = 0, ctx = 0;
+  std::vector<GraphEntry> graphs;
+  cudaStream_t capture_stream = nullptr;
+  std::string err;
+};
+
+namespace {
+
+int fail(wpk_handle* h, int code, const std::string& msg) {
+  if (h) h->err = msg;
+  return code;
+}
+
+#define CUDA_TRY(h, call)                                                                  \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return fail(h, WPK_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+size_t a256(size_t x) { return (x + 255) / 256 * 256; }
+
+int check_live(wpk_handle* h) {
+  if (!h) return WPK_ERR_INVALID_ARG;
+  if (!h->has_device) {
+    h->err = "no CUDA device: host-only handle";
+    return WPK_ERR_CUDA;
+  }
+  if (!h->poisoned && h->h_err_code && *(volatile int32_t*)h->h_err_code != 0) {
+    h->poisoned = true;
+    h->err = "device program reported an error (see wpk_get_error_info)";
+  }
+  if (h->poisoned) return WPK_ERR_POISONED;
+  return WPK_OK;
+}
+
+KParams make_params(const wpk_handle* h) {
+  const CompiledGraph& g = h->g;
+  const wpk_model_cfg& m = g.m;
+  KParams P{};
+  P.n_layers = m.n_layers;
+  P.hidden = m.hidden;
+  P.n_heads = m.n_heads;
+  P.n_kv = m.n_kv_heads;
+  P.head_dim = m.head_dim;
+  P.ffn = m.ffn;
+  P.vocab = m.vocab;
+  P.group = m.n_heads / m.n_kv_heads;
+  P.q_rows = m.n_heads * m.head_dim;
+  P.kv_rows = m.n_kv_heads * m.head_dim;
+  P.qkv_rows = P.q_rows + 2 * P.kv_rows;
+  P.down_kc = g.lay.down_kc;
+  P.n_down_chunks = g.lay.n_down_chunks;
+  P.eps = m.rms_eps;
+  P.max_batch = g.plan.max_batch;
+  P.max_context = g.plan.max_context;
+  P.page_tokens = g.plan.page_tokens;
+  P.max_blocks = g.max_blocks;
+  P.split_tokens = g.split_tokens;
+  P.n_splits = g.n_splits;
+  P.slot_bytes = g.plan.slot_bytes;
+  P.chunk_bytes = g.plan.chunk_bytes;
+  P.timeout_ns = g.plan.wait_timeout_ns;
+  P.trace = g.plan.trace;
+  P.weights = h->weights;
+  P.layers = h->d_layers;
+  P.final_norm_off = g.lay.final_norm;
+  P.embed_off = g.lay.embed;
+  P.lm_head_off = g.lay.lm_head;
+  P.kv = h->kv;
+  P.n_blocks = h->n_blocks;
+  P.block_table = h->d_block_table;
+  P.rope = h->d_rope;
+  P.xa = reinterpret_cast<float*>(h->scratch + h->off_xa);
+  P.xb = reinterpret_cast<float*>(h->scratch + h->off_xb);
+  P.qbuf = reinterpret_cast<float*>(h->scratch + h->off_q);
+  P.attn = reinterpret_cast<float*>(h->scratch + h->off_attn);
+  P.hbuf = reinterpret_cast<float*>(h->scratch + h->off_h);
+  P.part = reinterpret_cast<float*>(h->scratch + h->off_part);
+  P.arrive = h->d_arrive;
+  P.best = h->d_best;
+  P.seqlen = h->d_seqlen;
+  P.tok_fb = h->d_tok_fb;
+  P.active_batch = h->d_active;
+  P.tiles = h->d_tiles;
+  P.sig = h->d_sig;
+  P.ctr = h->d_ctr;
+  P.head = h->d_head;
+  P.err = h->d_err;
+  P.trace_buf = h->d_trace;
+  P.evclock = h->d_evclock;
+  P.in_tok_stride = 1;
+  P.epoch = 1;
+  return P;
+}
+
+void scratch_layout(wpk_handle* h) {
+  const CompiledGraph& g = h->g;
+  const wpk_model_cfg& m = g.m;
+  const size_t B = g.plan.max_batch, q_rows = (size_t)m.n_heads * m.head_dim;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = a256(off + bytes); return o; };
+  h->off_xa = take(B * m.hidden * 4);
+  h->off_xb = take(B * m.hidden * 4);
+  h->off_q = take(B * q_rows * 4);
+  h->off_attn = take(B * q_rows * 4);
+  h->off_h = take(B * m.ffn * 4);
+  h->off_part = take(B * m.n_kv_heads * g.n_splits * (m.n_heads / m.n_kv_heads) * (2 + m.head_dim) * 4);
+  h->scratch_bytes = off;
+  h->n_blocks = (int64_t)B * g.max_blocks;
+  h->kv_bytes = (size_t)m.n_layers * h->n_blocks * 2 * m.n_kv_heads * g.plan.page_tokens * m.head_dim * 2;
+}
+
+int launch_megakernel(wpk_handle* h, const KParams& base, cudaStream_t s) {
+  const CompiledGraph& g = h->g;
+  CUDA_TRY(h, cudaMemsetAsync(h->d_ctr, 0, std::max<size_t>(1, g.ctr_need.size()) * 4, s));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_head, 0, 4 * 4, s));
+  for (int r = 0; r + 1 < (int)g.region_begin.size(); ++r) {
+    KParams P = base;
+    P.t_begin = g.region_begin[r];
+    P.t_end = g.region_begin[r + 1];
+    P.region = r;
+    void* args[] = {&P};
+    CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kThreads), args,
+                                            h->smem, s));
+  }
+  return WPK_OK;
+}
+
+int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* out) {
+  const CompiledGraph& g = h->g;
+  if (!h->capture_stream) CUDA_TRY(h, cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking));
+  KParams base = make_params(h);
+  base.in_tok = nullptr;
+  base.out_tok = out_tok;
+  base.logits = logits;
+  CUDA_TRY(h, cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal));
+  for (const OpGroup& og : g.groups) {
+    KParams P = base;
+    P.t_begin = og.begin;
+    P.t_end = og.end;
+    void* args[] = {&P};
+    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kThreads), args, h->smem,
+                                     h->capture_stream);
+    if (e != cudaSuccess) {
+      cudaGraph_t junk = nullptr;
+      cudaStreamEndCapture(h->capture_stream, &junk);
+      if (junk) cudaGraphDestroy(junk);
+      return fail(h, WPK_ERR_CUDA, std::string("per-op capture: ") + cudaGetErrorString(e));
+    }
+  }
+  out->out_tok = out_tok;
+  out->logits = logits;
+  CUDA_TRY(h, cudaStreamEndCapture(h->capture_stream, &out->graph));
+  CUDA_TRY(h, cudaGraphInstantiate(&out->exec, out->graph, 0));
+  return WPK_OK;
+}
+
+int step_impl(wpk_handle* h, const int32_t* in_tok, int stride, int32_t* out_tok, float* logits, cudaStream_t s) {
+  if (h->g.plan.mode == WPK_MEGAKERNEL) {
+    KParams P = make_params(h);
+    P.in_tok = in_tok;
+    P.in_tok_stride = stride;
+    P.out_tok = out_tok;
+    P.logits = logits;
+    int rc = launch_megakernel(h, P, s);
+    if (rc) return rc;
+  } else {
+    if (in_tok)
+      CUDA_TRY(h, cudaMemcpy2DAsync(h->d_tok_fb, 4, in_tok, (size_t)stride * 4, 4, h->batch,
+                                    cudaMemcpyDeviceToDevice, s));
+    GraphEntry* ge = nullptr;
+    for (auto& e : h->graphs)
+      if (e.out_tok == out_tok && e.logits == logits) ge = &e;
+    if (!ge) {
+      GraphEntry e{};
+      int rc = capture_per_op(h, out_tok, logits, &e);
+      if (rc) return rc;
+      h->graphs.push_back(e);
+      ge = &h->graphs.back();
+    }
+    CUDA_TRY(h, cudaGraphLaunch(ge->exec, s));
+  }
+  CUDA_TRY(h, cudaMemcpyAsync(h->h_err_code, &h->d_err->code, 4, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(h, cudaGetLastError());
+  h->ctx += 1;
+  return WPK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+static int setup_device(wpk_handle* h) {
+  CompiledGraph& g = h->g;
+  const Plan& p = g.plan;
+  const wpk_model_cfg* model = &g.m;
+  CUDA_TRY(h, cudaGetDevice(&h->device));
+  CUDA_TRY(h, cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, h->device));
+  h->smem = worker_smem_bytes(p.slot_bytes);
+  CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)h->smem));
+  CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h->smem));
+  int per_sm = 0;
+  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kThreads, h->smem));
+  h->n_workers = p.n_workers ? p.n_workers : h->n_sms * p.workers_per_sm;
+  if (per_sm < 1 || h->n_workers > per_sm * h->n_sms)
+    return fail(h, WPK_ERR_UNSUPPORTED, "the worker grid cannot be co-resident with this slot size");
+
+  // one allocation for the small tables
+  const size_t n_tiles = g.tiles.size(), n_ctr = std::max<size_t>(1, g.ctr_need.size());
+  const size_t B = p.max_batch, hd2 = model->head_dim / 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = a256(off + bytes); return o; };
+  const size_t o_tiles = take(n_tiles * sizeof(Tile)), o_sig = take(std::max<size_t>(1, g.sig.size()) * 4),
+               o_ctr = take(n_ctr * 4), o_head = take(4 * 4), o_err = take(sizeof(ErrWord)),
+               o_trace = take(n_tiles * sizeof(TraceRec)), o_ev = take(4),
+               o_layers = take(g.lay.layers.size() * sizeof(LayerDev)),
+               o_rope = take((size_t)p.max_context * hd2 * sizeof(float2)),
+               o_bt = take(B * g.max_blocks * 4), o_arr = take(B * model->n_kv_heads * 4), o_best = take(B * 8),
+               o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4);
+  CUDA_TRY(h, cudaMalloc(&h->d_base, off));
+  CUDA_TRY(h, cudaMemset(h->d_base, 0, off));
+  h->d_tiles = reinterpret_cast<Tile*>(h->d_base + o_tiles);
+  h->d_sig = reinterpret_cast<uint32_t*>(h->d_base + o_sig);
+  h->d_ctr = reinterpret_cast<uint32_t*>(h->d_base + o_ctr);
+  h->d_head = reinterpret_cast<uint32_t*>(h->d_base + o_head);
+  h->d_err = reinterpret_cast<ErrWord*>(h->d_base + o_err);
+  h->d_trace = reinterpret_cast<TraceRec*>(h->d_base + o_trace);
+  h->d_evclock = reinterpret_cast<uint32_t*>(h->d_base + o_ev);
+  h->d_layers = reinterpret_cast<LayerDev*>(h->d_base + o_layers);
+  h->d_rope = reinterpret_cast<float2*>(h->d_base + o_rope);
+  h->d_block_table = reinterpret_cast<int32_t*>(h->d_base + o_bt);
+  h->d_arrive = reinterpret_cast<uint32_t*>(h->d_base + o_arr);
+  h->d_best = reinterpret_cast<unsigned long long*>(h->d_base + o_best);
+  h->d_seqlen = reinterpret_cast<int32_t*>(h->d_base + o_seq);
+  h->d_tok_fb = reinterpret_cast<int32_t*>(h->d_base + o_fb);
+  h->d_active = reinterpret_cast<int32_t*>(h->d_base + o_act);
+  CUDA_TRY(h, cudaMemcpy(h->d_tiles, g.tiles.data(), n_tiles * sizeof(Tile), cudaMemcpyHostToDevice));
+  if (!g.sig.empty()) CUDA_TRY(h, cudaMemcpy(h->d_sig, g.sig.data(), g.sig.size() * 4, cudaMemcpyHostToDevice));
+  CUDA_TRY(h, cudaMemcpy(h->d_layers, g.lay.layers.data(), g.lay.layers.size() * sizeof(LayerDev),
+                         cudaMemcpyHostToDevice));
+  // RoPE (cos, sin) table: angle = pos * theta^(-2i/d), evaluated in double
+  std::vector<float2> rope((size_t)p.max_context * hd2);
+  for (int pos = 0; pos < p.max_context; ++pos)
+    for (size_t i = 0; i < hd2; ++i) {
+      const double inv = std::pow((double)model->rope_theta, -2.0 * (double)i / (double)model->head_dim);
+      const double a = (double)pos * inv;
+      rope[(size_t)pos * hd2 + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+    }
+  CUDA_TRY(h, cudaMemcpy(h->d_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice));
+  std::vector<int32_t> bt(B * g.max_blocks);
+  for (size_t i = 0; i < bt.size(); ++i) bt[i] = (int32_t)i;
+  CUDA_TRY(h, cudaMemcpy(h->d_block_table, bt.data(), bt.size() * 4, cudaMemcpyHostToDevice));
+  CUDA_TRY(h, cudaHostAlloc(&h->h_err_code, 4, cudaHostAllocDefault));
+  *h->h_err_code = 0;
+  h->has_device = true;
+  return WPK_OK;
+}
+
+int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out) {
+  if (!model || !plan || !out) return WPK_ERR_INVALID_ARG;
+  *out = nullptr;
+  auto* h = new wpk_handle();
+  int code = 0;
+  Plan p;
+  std::string msg = normalize_plan(*model, *plan, &p, &code);
+  if (msg.empty()) msg = compile_graph(*model, p, &h->g, &code);
+  if (!msg.empty()) {
+    delete h;
+    return code;
+  }
+  scratch_layout(h);
+  // Without a CUDA device the handle is host-only: the compiled tables can be
+  // inspected, verified and simulated; device calls return WPK_ERR_CUDA.
+  int n_dev = 0;
+  if (cudaGetDeviceCount(&n_dev) != cudaSuccess || n_dev == 0) {
+    cudaGetLastError();
+    h->n_workers = p.n_workers;
+    h->err = "no CUDA device: host-only handle";
+    *out = h;
+    return WPK_OK;
+  }
+  int rc = setup_device(h);
+  if (rc) {
+    if (h->d_base) cudaFree(h->d_base);
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return WPK_OK;
+}
+
+int wpk_workspace_size(const wpk_handle* h, size_t* weight_bytes, size_t* kv_bytes, size_t* scratch_bytes) {
+  if (!h) return WPK_ERR_INVALID_ARG;
+  if (weight_bytes) *weight_bytes = h->g.lay.total;
+  if (kv_bytes) *kv_bytes = h->kv_bytes;
+  if (scratch_bytes) *scratch_bytes = h->scratch_bytes;
+  return WPK_OK;
+}
+
+int wpk_load_weights(wpk_handle* h, const wpk_weights* w, void* dev_weights, void* dev_kv, void* dev_scratch,
+                     void* stream) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (!w || !dev_weights || !dev_kv || !dev_scratch)
+    return fail(h, WPK_ERR_INVALID_ARG, "null weights or device buffer");
+  if (((uintptr_t)dev_weights | (uintptr_t)dev_kv | (uintptr_t)dev_scratch) & 255)
+    return fail(h, WPK_ERR_INVALID_ARG, "device buffers must be 256-byte aligned");
+  std::vector<uint8_t> img(h->g.lay.total, 0);
+  std::string msg = arrange_weights(h->g, *w, img.data());
+  if (!msg.empty()) return fail(h, WPK_ERR_INVALID_ARG, msg);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(h, cudaMemcpyAsync(dev_weights, img.data(), img.size(), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaStreamSynchronize(s));
+  h->weights = static_cast<uint8_t*>(dev_weights);
+  h->kv = static_cast<uint16_t*>(dev_kv);
+  h->scratch = static_cast<uint8_t*>(dev_scratch);
+  h->loaded = true;
+  h->prefilled = false;
+  h->graphs.clear();  // captured pointers may have changed
+  return WPK_OK;
+}
+
+int wpk_set_block_table(wpk_handle* h, const int32_t* table) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (!table) return fail(h, WPK_ERR_INVALID_ARG, "null table");
+  const size_t n = (size_t)h->g.plan.max_batch * h->g.max_blocks;
+  std::vector<char> seen(n, 0);
+  for (size_t i = 0; i < n; ++i) {
+    if (table[i] < 0 || (size_t)table[i] >= n || seen[table[i]])
+      return fail(h, WPK_ERR_INVALID_ARG, "block table must be a permutation of page ids");
+    seen[table[i]] = 1;
+  }
+  CUDA_TRY(h, cudaMemcpy(h->d_block_table, table, n * 4, cudaMemcpyHostToDevice));
+  return WPK_OK;
+}
+
+int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len, int32_t* first_tok_dev,
+                float* logits_dev, void* stream) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (!h->loaded) return fail(h, WPK_ERR_NOT_LOADED, "weights not loaded");
+  if (!tokens_dev || batch <= 0 || prompt_len <= 0) return fail(h, WPK_ERR_INVALID_ARG, "bad prefill arguments");
+  if (batch > h->g.plan.max_batch || prompt_len > h->g.plan.max_context)
+    return fail(h, WPK_ERR_SHAPE, "batch or prompt exceeds the plan");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t B = h->g.plan.max_batch;
+  CUDA_TRY(h, cudaMemsetAsync(h->d_seqlen, 0, B * 4, s));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_best, 0, B * 8, s));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_arrive, 0, B * h->g.m.n_kv_heads * 4, s));
+  CUDA_TRY(h, cudaMemcpyAsync(h->d_active, &batch, 4, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaStreamSynchronize(s));  // `batch` lives on this stack frame
+  h->batch = batch;
+  h->ctx = 0;
+  // The prompt runs through the decode program one position at a time.
+  for (int t = 0; t < prompt_len; ++t) {
+    const bool last = (t + 1 == prompt_len);
+    rc = step_impl(h, tokens_dev + t, prompt_len, last ? first_tok_dev : nullptr, last ? logits_dev : nullptr, s);
+    if (rc) return rc;
+  }
+  h->prefilled = true;
+  return WPK_OK;
+}
+
+int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev, void* stream) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");
+  if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  return step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, static_cast<cudaStream_t>(stream));
+}
+
+int wpk_graph_stats_get(const wpk_handle* h, wpk_graph_stats* st) {
+  if (!h || !st) return WPK_ERR_INVALID_ARG;
+  memset(st, 0, sizeof *st);
+  const CompiledGraph& g = h->g;
+  st->n_tiles = (int64_t)g.tiles.size();
+  st->n_counters = (int64_t)g.ctr_need.size();
+  st->n_edges = g.n_edges;
+  st->n_signals = (int64_t)g.sig.size();
+  st->n_ops = (int64_t)g.groups.size();
+  st->n_workers = h->n_workers;
+  st->weight_bytes = g.algo_weight_bytes;
+  st->n_regions = (int64_t)g.region_begin.size() - 1;
+  for (size_t i = 0; i < g.region_begin.size() && i < 5; ++i) st->region_begin[i] = g.region_begin[i];
+  return WPK_OK;
+}
+
+int wpk_get_edges(const wpk_handle* h, int32_t* pairs, int64_t max_pairs, int64_t* n_pairs) {
+  if (!h || !n_pairs) return WPK_ERR_INVALID_ARG;
+  int64_t k = 0;
+  for (size_t v = 0; v < h->g.preds.size(); ++v)
+    for (int u : h->g.preds[v]) {
+      if (pairs && k < max_pairs) {
+        pairs[2 * k] = u;
+        pairs[2 * k + 1] = (int32_t)v;
+      }
+      ++k;
+    }
+  *n_pairs = k;
+  return WPK_OK;
+}
+
+int wpk_get_tile_ops(const wpk_handle* h, int32_t* ops, int64_t n) {
+  if (!h || !ops || n < (int64_t)h->g.tiles.size()) return WPK_ERR_INVALID_ARG;
+  for (size_t i = 0; i < h->g.tiles.size(); ++i) ops[i] = h->g.tiles[i].op;
+  return WPK_OK;
+}
+
+int wpk_verify_graph(const wpk_handle* h) {
+  if (!h) return WPK_ERR_INVALID_ARG;
+  std::string msg = verify_graph(h->g);
+  if (!msg.empty()) {
+    const_cast<wpk_handle*>(h)->err = msg;
+    return WPK_ERR_SHAPE;
+  }
+  return WPK_OK;
+}
+
+int wpk_simulate(const wpk_handle* h, int n_threads, int n_epochs, uint64_t seed, int wait_ms, int stuck_tile,
+                 int32_t* done_order) {
+  if (!h || n_threads <= 0 || n_epochs <= 0 || wait_ms <= 0) return WPK_ERR_INVALID_ARG;
+  std::string msg;
+  int rc = simulate_graph(h->g, n_threads, n_epochs, seed, wait_ms, stuck_tile, done_order, &msg);
+  if (rc) const_cast<wpk_handle*>(h)->err = msg;
+  return rc;
+}
+
+int wpk_get_trace(wpk_handle* h, void* host_buf, size_t bytes) {
+  if (!h || !host_buf) return WPK_ERR_INVALID_ARG;
+  if (!h->has_device) return fail(h, WPK_ERR_CUDA, "no CUDA device");
+  const size_t need = h->g.tiles.size() * sizeof(TraceRec);
+  if (bytes < need) return fail(h, WPK_ERR_INVALID_ARG, "trace buffer too small");
+  if (!h->g.plan.trace) return fail(h, WPK_ERR_UNSUPPORTED, "plan was built without trace");
+  CUDA_TRY(h, cudaDeviceSynchronize());
+  CUDA_TRY(h, cudaMemcpy(host_buf, h->d_trace, need, cudaMemcpyDeviceToHost));
+  return WPK_OK;
+}
+
+int wpk_get_error_info(wpk_handle* h, wpk_error_info* info) {
+  if (!h || !info) return WPK_ERR_INVALID_ARG;
+  if (!h->has_device) return fail(h, WPK_ERR_CUDA, "no CUDA device");
+  CUDA_TRY(h, cudaDeviceSynchronize());
+  ErrWord e{};
+  CUDA_TRY(h, cudaMemcpy(&e, h->d_err, sizeof e, cudaMemcpyDeviceToHost));
+  info->code = e.code;
+  info->tile = e.tile;
+  info->counter = e.counter;
+  info->epoch = e.epoch;
+  info->observed = e.observed;
+  info->target = e.target;
+  if (e.code) h->poisoned = true;
+  return WPK_OK;
+}
+
+const char* wpk_last_error(const wpk_handle* h) { return h ? h->err.c_str() : "null handle"; }
+
+int wpk_destroy(wpk_handle* h) {
+  if (!h) return WPK_ERR_INVALID_ARG;
+  if (h->has_device) cudaDeviceSynchronize();
+  for (auto& e : h->graphs) {
+    if (e.exec) cudaGraphExecDestroy(e.exec);
+    if (e.graph) cudaGraphDestroy(e.graph);
+  }
+  if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
+  if (h->d_base) cudaFree(h->d_base);
+  if (h->h_err_code) cudaFreeHost(h->h_err_code);
+  delete h;
+  return WPK_OK;
+}
+
+int wpk_debug_break_counter(wpk_handle* h, int counter) {
+  if (!h || counter < 0 || counter >= (int)h->g.ctr_need.size()) return WPK_ERR_INVALID_ARG;
+  for (auto& t : h->g.tiles)
+    if (t.wait_ctr == (uint32_t)counter) t.need += 1;
+  if (!h->has_device) return WPK_OK;
+  CUDA_TRY(h, cudaMemcpy(h->d_tiles, h->g.tiles.data(), h->g.tiles.size() * sizeof(Tile), cudaMemcpyHostToDevice));
+  return WPK_OK;
+}
+
+}  // extern "C"

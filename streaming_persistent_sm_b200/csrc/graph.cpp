@@ -1,0 +1,590 @@
+// Host graph compiler for the persistent decode program.
+//
+// The compiler follows the pages' split of responsibilities: it starts from a
+// fixed op list of the decoder (the tensor-level graph of "Why real-time
+// inference wants a megakernel", "A concrete design"), splits every op into
+// tiles sized to one worker's staging slot, derives tile-to-tile tensor
+// edges (dropping the barrier edges between consecutive kernels and keeping
+// the tile-to-tile tensor edges: "One Megakernel is Not Enough", Table I,
+// cross-kernel readiness), dedups dependency counters by identical
+// predecessor set, and emits the ticket order the device queue hands out.
+// Dependency counters that let a consumer start once its own input chunk is
+// ready follow "Persistent threads and megakernels", §6 (Hazy's Llama-1B
+// megakernel); the down projection's K-chunks are that finer edge here.
+#include "graph.h"
+
+#include <algorithm>
+#include <atomic>
+#include <chrono>
+#include <cstring>
+#include <map>
+#include <random>
+#include <thread>
+#include <unordered_map>
+
+namespace wpk {
+
+namespace {
+
+uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+std::string fmt(const char* f, long long a = 0, long long b = 0, long long c = 0) {
+  char buf[512];
+  snprintf(buf, sizeof buf, f, a, b, c);
+  return buf;
+}
+
+}  // namespace
+
+std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan* p, int* code) {
+  *code = WPK_ERR_INVALID_ARG;
+  if (m.n_layers <= 0 || m.hidden <= 0 || m.n_heads <= 0 || m.n_kv_heads <= 0 || m.head_dim <= 0 ||
+      m.ffn <= 0 || m.vocab <= 0)
+    return "model dimensions must be positive";
+  if (m.n_heads % m.n_kv_heads) return "n_heads must be a multiple of n_kv_heads";
+  if (m.n_heads / m.n_kv_heads > kMaxGroup) return "more than 8 query heads per kv head";
+  if (m.head_dim != 64) { *code = WPK_ERR_UNSUPPORTED; return "head_dim must be 64"; }
+  if (m.hidden % 8 || m.ffn % 8) { *code = WPK_ERR_SHAPE; return "hidden and ffn must be multiples of 8"; }
+  if (m.hidden > 2048 * 4) { *code = WPK_ERR_UNSUPPORTED; return "hidden > 8192"; }
+  if (!(m.rms_eps >= 0.f) || !(m.rope_theta > 0.f)) return "bad rms_eps / rope_theta";
+  if (in.max_batch <= 0 || in.max_context <= 0) return "max_batch and max_context must be positive";
+  p->max_batch = in.max_batch;
+  p->max_context = in.max_context;
+  p->page_tokens = in.page_tokens ? in.page_tokens : 64;
+  if (p->page_tokens % 8 || p->page_tokens > 256) return "page_tokens must be a multiple of 8, <= 256";
+  p->workers_per_sm = in.workers_per_sm ? in.workers_per_sm : 2;
+  p->n_workers = in.n_workers;
+  if (p->n_workers < 0 || p->workers_per_sm < 0 || p->workers_per_sm > 4) return "bad worker count";
+  p->mode = in.mode;
+  if (p->mode != WPK_MEGAKERNEL && p->mode != WPK_PER_OP_GRAPH) return "bad mode";
+  p->resident = in.resident;
+  if (p->resident && p->mode != WPK_MEGAKERNEL) return "resident needs WPK_MEGAKERNEL";
+  p->n_regions = in.n_regions ? in.n_regions : 1;
+  if (p->n_regions < 1 || p->n_regions > 4) return "n_regions must be 1..4";
+  if (p->resident && p->n_regions != 1) return "resident mode runs one region";
+  for (int r = 0; r < 4; ++r) p->region_cut[r] = in.region_cut[r];
+  if (p->n_regions > 1) {
+    if (p->region_cut[0] != 0) return "region_cut[0] must be 0";
+    for (int r = 1; r < p->n_regions; ++r)
+      if (p->region_cut[r] <= p->region_cut[r - 1] || p->region_cut[r] > m.n_layers)
+        return "region cuts must increase and be <= n_layers";
+  }
+  p->trace = in.trace;
+  p->wait_timeout_ns = in.wait_timeout_ns ? in.wait_timeout_ns : 2000000000ull;
+  p->slot_bytes = in.slot_bytes ? in.slot_bytes : 65536;
+  if (p->slot_bytes % 1024 || p->slot_bytes < 16384 || p->slot_bytes > 160 * 1024)
+    return "slot_bytes must be a multiple of 1024 in [16K, 160K]";
+  p->tile_bytes = in.tile_bytes ? in.tile_bytes : 32768;
+  if (p->tile_bytes > p->slot_bytes || p->tile_bytes < 1024) return "tile_bytes must be in [1K, slot_bytes]";
+  p->split_pages = in.split_pages ? in.split_pages : 1;
+  if (p->split_pages < 1) return "split_pages must be >= 1";
+  if ((int64_t)p->split_pages * p->page_tokens * m.head_dim * 2 * 2 > p->slot_bytes)
+    return "an attention split's K/V pages do not fit the slot";
+  if (p->split_pages * p->page_tokens * (m.n_heads / m.n_kv_heads) > 8 * kThreads)
+    return "attention split too long for one tile";
+  p->chunk_bytes = p->slot_bytes / kMaxChunks;
+  *code = WPK_OK;
+  return "";
+}
+
+// ---------------------------------------------------------------------------
+// Dataflow edges: for each buffer keep, per element range, the last plain
+// writer and the accumulators since then.  A read depends on the frontier
+// (the accumulators if any, else the last writer); an accumulate depends on
+// the last plain writer.  Write-after-read and write-after-write order is not
+// added as edges; verify_graph proves every such pair is ordered by a path.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct Seg {
+  int lo, hi;
+  int wgroup;                // group id of the current writers (-1 = single)
+  std::vector<int> writers;  // last plain write (one tile, or one write group)
+  std::vector<int> accs;     // accumulators since then
+};
+
+struct BufState {
+  std::vector<Seg> segs;  // sorted, disjoint, covering [0, size)
+  explicit BufState(int size = 1) { segs.push_back({0, size, -1, {}, {}}); }
+  // split so that x is a segment boundary
+  void cut(int x) {
+    for (size_t i = 0; i < segs.size(); ++i) {
+      if (segs[i].lo < x && x < segs[i].hi) {
+        Seg b = segs[i];
+        b.lo = x;
+        segs[i].hi = x;
+        segs.insert(segs.begin() + i + 1, b);
+        return;
+      }
+    }
+  }
+};
+
+struct DataflowBuilder {
+  std::vector<BufState> bufs;
+  const std::vector<std::vector<int32_t>>* preds_of = nullptr;
+  // memo of a read's frontier: (buf, lo, hi) -> preds, dropped when buf changes
+  std::map<std::tuple<int, int, int>, std::vector<int>> memo;
+
+  std::vector<int> frontier(int b, int lo, int hi) {
+    auto key = std::make_tuple(b, lo, hi);
+    auto it = memo.find(key);
+    if (it != memo.end()) return it->second;
+    std::vector<int> out;
+    for (auto& s : bufs[b].segs) {
+      if (s.hi <= lo || s.lo >= hi) continue;
+      const auto& src = s.accs.empty() ? s.writers : s.accs;
+      out.insert(out.end(), src.begin(), src.end());
+    }
+    std::sort(out.begin(), out.end());
+    out.erase(std::unique(out.begin(), out.end()), out.end());
+    memo[key] = out;
+    return out;
+  }
+  void invalidate(int b) {
+    for (auto it = memo.begin(); it != memo.end();) {
+      if (std::get<0>(it->first) == b)
+        it = memo.erase(it);
+      else
+        ++it;
+    }
+  }
+  bool is_pred(int u, int w) const {
+    const auto& P = (*preds_of)[w];
+    return std::binary_search(P.begin(), P.end(), u);
+  }
+  void apply(int t, const std::vector<Access>& acc, std::vector<int>* preds) {
+    std::vector<int> acc_deps;
+    for (auto& a : acc) {
+      if (a.kind == 0) {
+        auto f = frontier(a.buf, a.lo, a.hi);
+        preds->insert(preds->end(), f.begin(), f.end());
+      } else if (a.kind == 2) {
+        for (auto& s : bufs[a.buf].segs)
+          if (!(s.hi <= a.lo || s.lo >= a.hi)) acc_deps.insert(acc_deps.end(), s.writers.begin(), s.writers.end());
+      }
+    }
+    std::sort(preds->begin(), preds->end());
+    preds->erase(std::unique(preds->begin(), preds->end()), preds->end());
+    // An accumulate must follow the write that initialised its range; skip the
+    // edge when one of the tile's read predecessors already depends on it.
+    for (int u : acc_deps) {
+      bool implied = std::binary_search(preds->begin(), preds->end(), u);
+      for (size_t i = 0; !implied && i < preds->size() && i < 4; ++i) implied = is_pred(u, (*preds)[i]);
+      if (!implied) preds->push_back(u);
+    }
+    for (auto& a : acc) {
+      if (a.kind == 0) continue;
+      BufState& B = bufs[a.buf];
+      B.cut(a.lo);
+      B.cut(a.hi);
+      for (auto& s : B.segs) {
+        if (s.hi <= a.lo || s.lo >= a.hi) continue;
+        if (a.kind == 1) {
+          if (a.group >= 0 && s.wgroup == a.group && s.accs.empty()) {
+            s.writers.push_back(t);
+          } else {
+            s.writers.assign(1, t);
+            s.wgroup = a.group;
+            s.accs.clear();
+          }
+        } else {
+          s.accs.push_back(t);
+        }
+      }
+      invalidate(a.buf);
+    }
+    std::sort(preds->begin(), preds->end());
+    preds->erase(std::unique(preds->begin(), preds->end()), preds->end());
+    preds->erase(std::remove(preds->begin(), preds->end(), t), preds->end());
+  }
+};
+
+struct VecHash {
+  size_t operator()(const std::vector<int>& v) const {
+    size_t h = v.size() * 0x9E3779B97F4A7C15ull;
+    for (int x : v) h ^= (size_t)x + 0x9E3779B97F4A7C15ull + (h << 6) + (h >> 2);
+    return h;
+  }
+};
+
+int rows_per_tile(int row_bytes, const Plan& p) {
+  int r = p.tile_bytes / row_bytes;
+  r = r / 8 * 8;
+  if (r < 8) r = 8;
+  while (r > 8 && r * row_bytes > p.slot_bytes) r -= 8;
+  return std::min(r, 256);
+}
+
+}  // namespace
+
+std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code) {
+  *code = WPK_ERR_SHAPE;
+  g->m = m;
+  g->plan = p;
+  const int h = m.hidden, hd = m.head_dim, grp = m.n_heads / m.n_kv_heads;
+  const int q_rows = m.n_heads * hd, kv_rows = m.n_kv_heads * hd, qkv_rows = q_rows + 2 * kv_rows;
+  // down projection K chunks: at most 2048 columns each, multiple of 8
+  int nch = (m.ffn + 2047) / 2048;
+  while (m.ffn % nch || (m.ffn / nch) % 8) ++nch;
+  const int kc = m.ffn / nch;
+  if ((int64_t)h * 4 * 1 > kActBytes * 4) return "hidden too large for activation staging";
+  if (8LL * h * 2 > p.slot_bytes || 8LL * q_rows * 2 > p.slot_bytes || 8LL * kc * 2 > p.slot_bytes)
+    return "a row block of 8 rows does not fit the staging slot";
+  if (q_rows > 8192) return "q_rows > 8192";
+
+  // ---- weight image layout ----
+  Layout& L = g->lay;
+  uint64_t off = 0;
+  auto take = [&](uint64_t bytes) {
+    uint64_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.layers.resize(m.n_layers);
+  for (int l = 0; l < m.n_layers; ++l) {
+    LayerDev& d = L.layers[l];
+    d.attn_norm = take((uint64_t)h * 4);
+    d.ffn_norm = take((uint64_t)h * 4);
+    d.qkv = take((uint64_t)qkv_rows * h * 2);
+    d.wo = take((uint64_t)h * q_rows * 2);
+    d.gu = take((uint64_t)2 * m.ffn * h * 2);
+    d.down = take((uint64_t)h * m.ffn * 2);
+  }
+  L.final_norm = take((uint64_t)h * 4);
+  L.embed = take((uint64_t)m.vocab * h * 2);
+  L.lm_head = m.tied_embedding ? L.embed : take((uint64_t)m.vocab * h * 2);
+  L.total = off;
+  L.down_kc = kc;
+  L.n_down_chunks = nch;
+
+  // ---- attention splits ----
+  g->split_tokens = p.split_pages * p.page_tokens;
+  g->n_splits = (p.max_context + g->split_tokens - 1) / g->split_tokens;
+  g->max_blocks = (p.max_context + p.page_tokens - 1) / p.page_tokens;
+
+  // ---- tiles in ticket order ----
+  std::vector<Tile>& T = g->tiles;
+  std::vector<std::vector<Access>>& A = g->access;
+  T.clear();
+  A.clear();
+  g->groups.clear();
+  int64_t wbytes = 0;
+  auto add = [&](uint16_t op, int layer, uint64_t w_off, uint32_t w_bytes, int a0, int a1, int a2, int a3,
+                 std::vector<Access> acc) {
+    Tile t{};
+    t.op = op;
+    t.layer = (uint16_t)layer;
+    t.wait_ctr = kNoCounter;
+    t.w_off = w_off;
+    t.w_bytes = w_bytes;
+    t.a0 = a0; t.a1 = a1; t.a2 = a2; t.a3 = a3;
+    wbytes += w_bytes;
+    if (g->groups.empty() || g->groups.back().op != op || g->groups.back().layer != layer)
+      g->groups.push_back({op, layer, (uint32_t)T.size(), (uint32_t)T.size()});
+    T.push_back(t);
+    A.push_back(std::move(acc));
+    g->groups.back().end = (uint32_t)T.size();
+  };
+  std::vector<uint32_t> layer_begin(m.n_layers + 1, 0);
+
+  add(OP_EMBED, 0, 0, 0, 0, 0, 0, 0, {{BUF_XA, 0, h, 1}, {BUF_TOK, 0, 1, 0}});
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerDev& d = L.layers[l];
+    layer_begin[l] = (uint32_t)T.size();
+    const int attn_group = 1000 + l;
+    // fused RMSNorm + QKV + RoPE + KV write; tiles never straddle q/k/v sections
+    {
+      int R = rows_per_tile(h * 2, p);
+      int sec_lo[3] = {0, q_rows, q_rows + kv_rows}, sec_hi[3] = {q_rows, q_rows + kv_rows, qkv_rows};
+      for (int s = 0; s < 3; ++s)
+        for (int r0 = sec_lo[s]; r0 < sec_hi[s]; r0 += R) {
+          int n = std::min(R, sec_hi[s] - r0);
+          add(OP_QKV, l, d.qkv + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n, 0, h,
+              {{BUF_XA, 0, h, 0}, {BUF_QKV, r0, r0 + n, 1}});
+        }
+    }
+    // split-KV attention per (sequence, kv head, split)
+    for (int b = 0; b < p.max_batch; ++b)
+      for (int gi = 0; gi < m.n_kv_heads; ++gi)
+        for (int j = 0; j < g->n_splits; ++j)
+          add(OP_ATTN, l, 0, 0, b, gi, j, 0,
+              {{BUF_QKV, gi * grp * hd, (gi + 1) * grp * hd, 0},
+               {BUF_QKV, q_rows + gi * hd, q_rows + (gi + 1) * hd, 0},
+               {BUF_QKV, q_rows + kv_rows + gi * hd, q_rows + kv_rows + (gi + 1) * hd, 0},
+               {BUF_ATTN, gi * grp * hd, (gi + 1) * grp * hd, 1, attn_group}});
+    // O projection + residual
+    {
+      int R = rows_per_tile(q_rows * 2, p);
+      for (int r0 = 0; r0 < h; r0 += R) {
+        int n = std::min(R, h - r0);
+        add(OP_O, l, d.wo + (uint64_t)r0 * q_rows * 2, (uint32_t)n * q_rows * 2, r0, n, 0, q_rows,
+            {{BUF_ATTN, 0, q_rows, 0}, {BUF_XB, r0, r0 + n, 1}, {BUF_XA, r0, r0 + n, 1}});
+      }
+    }
+    // fused RMSNorm + gate/up + SwiGLU (physical rows: gate j at 2j, up j at 2j+1)
+    {
+      int R = rows_per_tile(h * 2, p);
+      for (int r0 = 0; r0 < 2 * m.ffn; r0 += R) {
+        int n = std::min(R, 2 * m.ffn - r0);
+        add(OP_GU, l, d.gu + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n, 0, h,
+            {{BUF_XB, 0, h, 0}, {BUF_H, r0 / 2, (r0 + n) / 2, 1}});
+      }
+    }
+    // down projection, split along K into chunks (finer edges), accumulated into x
+    {
+      int R = rows_per_tile(kc * 2, p);
+      for (int c = 0; c < nch; ++c)
+        for (int r0 = 0; r0 < h; r0 += R) {
+          int n = std::min(R, h - r0);
+          add(OP_DOWN, l, d.down + ((uint64_t)c * h + r0) * kc * 2, (uint32_t)n * kc * 2, r0, n, c * kc, kc,
+              {{BUF_H, c * kc, (c + 1) * kc, 0}, {BUF_XA, r0, r0 + n, 2}});
+        }
+    }
+  }
+  layer_begin[m.n_layers] = (uint32_t)T.size();
+  {
+    int R = rows_per_tile(h * 2, p);
+    for (int r0 = 0; r0 < m.vocab; r0 += R) {
+      int n = std::min(R, m.vocab - r0);
+      add(OP_LMHEAD, m.n_layers, L.lm_head + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n, 0, h,
+          {{BUF_XA, 0, h, 0}, {BUF_LOGITS, r0, r0 + n, 1}, {BUF_BEST, 0, 1, 2}});
+    }
+  }
+  add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0}, {BUF_TOK, 0, 1, 1}});
+  g->algo_weight_bytes = wbytes;
+  if (T.size() >= (1u << 31)) return "too many tiles";
+
+  // ---- edges from dataflow ----
+  DataflowBuilder df;
+  int sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1};
+  for (int b = 0; b < BUF_COUNT; ++b) df.bufs.emplace_back(sizes[b]);
+  g->preds.assign(T.size(), {});
+  df.preds_of = &g->preds;
+  g->n_edges = 0;
+  for (size_t t = 0; t < T.size(); ++t) {
+    df.apply((int)t, A[t], &g->preds[t]);
+    g->n_edges += (int64_t)g->preds[t].size();
+  }
+
+  // ---- counters: one per distinct predecessor set ----
+  std::unordered_map<std::vector<int>, uint32_t, VecHash> ctr_of;
+  std::vector<std::vector<uint32_t>> sig_of(T.size());
+  g->ctr_need.clear();
+  for (size_t t = 0; t < T.size(); ++t) {
+    const auto& P = g->preds[t];
+    if (P.empty()) continue;
+    auto it = ctr_of.find(P);
+    uint32_t c;
+    if (it == ctr_of.end()) {
+      c = (uint32_t)g->ctr_need.size();
+      ctr_of.emplace(P, c);
+      g->ctr_need.push_back((uint32_t)P.size());
+      for (int u : P) sig_of[u].push_back(c);
+    } else {
+      c = it->second;
+    }
+    T[t].wait_ctr = c;
+    T[t].need = g->ctr_need[c];
+  }
+  g->sig.clear();
+  for (size_t t = 0; t < T.size(); ++t) {
+    T[t].sig_off = (uint32_t)g->sig.size();
+    T[t].sig_cnt = (uint32_t)sig_of[t].size();
+    g->sig.insert(g->sig.end(), sig_of[t].begin(), sig_of[t].end());
+  }
+
+  // ---- regions: contiguous ticket ranges starting at layer cuts ----
+  g->region_begin.assign(1, 0);
+  for (int r = 1; r < p.n_regions; ++r) g->region_begin.push_back(layer_begin[p.region_cut[r]]);
+  g->region_begin.push_back((uint32_t)T.size());
+  *code = WPK_OK;
+  return "";
+}
+
+// ---------------------------------------------------------------------------
+std::string verify_graph(const CompiledGraph& g) {
+  const size_t n = g.tiles.size();
+  if (n > 20000) return "graph too large for the quadratic verifier";
+  // topological ticket order and counter consistency
+  std::vector<std::vector<int>> signalers(g.ctr_need.size());
+  for (size_t t = 0; t < n; ++t) {
+    for (int u : g.preds[t])
+      if (u >= (int)t) return fmt("edge %lld -> %lld goes backwards in ticket order", u, (long long)t);
+    const Tile& T = g.tiles[t];
+    for (uint32_t i = 0; i < T.sig_cnt; ++i) signalers[g.sig[T.sig_off + i]].push_back((int)t);
+  }
+  for (size_t t = 0; t < n; ++t) {
+    const Tile& T = g.tiles[t];
+    if (g.preds[t].empty()) {
+      if (T.wait_ctr != kNoCounter) return fmt("tile %lld waits without predecessors", (long long)t);
+      continue;
+    }
+    if (T.wait_ctr == kNoCounter) return fmt("tile %lld has predecessors but no counter", (long long)t);
+    const auto& S = signalers[T.wait_ctr];
+    if (S != g.preds[t]) return fmt("counter %lld of tile %lld: signalers != predecessors", T.wait_ctr, (long long)t);
+    if (T.need != S.size()) return fmt("tile %lld need %lld != signal count", (long long)t, T.need);
+  }
+  // reachability bitsets
+  const size_t W = (n + 63) / 64;
+  std::vector<uint64_t> anc(n * W, 0);
+  for (size_t t = 0; t < n; ++t) {
+    uint64_t* a = &anc[t * W];
+    for (int u : g.preds[t]) {
+      const uint64_t* b = &anc[(size_t)u * W];
+      for (size_t i = 0; i < W; ++i) a[i] |= b[i];
+      a[u / 64] |= 1ull << (u % 64);
+    }
+  }
+  auto reach = [&](int u, int v) { return (anc[(size_t)v * W + u / 64] >> (u % 64)) & 1; };
+  // every conflicting access pair must be ordered by a path
+  struct Acc { int t, lo, hi, kind, group; };
+  std::vector<std::vector<Acc>> per(BUF_COUNT);
+  for (size_t t = 0; t < n; ++t)
+    for (auto& a : g.access[t]) per[a.buf].push_back({(int)t, a.lo, a.hi, a.kind, a.group});
+  for (int b = 0; b < BUF_COUNT; ++b) {
+    const auto& v = per[b];
+    for (size_t i = 0; i < v.size(); ++i)
+      for (size_t j = i + 1; j < v.size(); ++j) {
+        const Acc &x = v[i], &y = v[j];
+        if (x.t == y.t) continue;
+        if (x.hi <= y.lo || y.hi <= x.lo) continue;
+        if (x.kind == 0 && y.kind == 0) continue;
+        if (x.kind == 2 && y.kind == 2) continue;
+        if (x.kind == 1 && y.kind == 1 && x.group >= 0 && x.group == y.group) continue;
+        if (!reach(x.t, y.t))
+          return fmt("unordered conflicting accesses: tile %lld and tile %lld (buffer %lld)", x.t, y.t, b);
+      }
+  }
+  return "";
+}
+
+// ---------------------------------------------------------------------------
+// Host threads standing in for workers: the same ticket queue, counter targets
+// (need x epoch, counters never reset) and signals, with random delays.
+int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t seed, int wait_ms,
+                   int stuck_tile, int32_t* done_order, std::string* msg) {
+  const uint64_t T = g.tiles.size();
+  const uint64_t total = T * (uint64_t)n_epochs;
+  std::vector<std::atomic<uint32_t>> ctr(g.ctr_need.size());
+  for (auto& c : ctr) c.store(0);
+  std::atomic<uint64_t> head{0}, done_idx{0};
+  std::atomic<uint32_t> epochs_done{0};  // the doorbell: step e starts after step e-1 completed
+  std::atomic<int> failed{0};
+  std::atomic<uint64_t> fail_tile{0};
+  auto worker = [&](int wid) {
+    std::mt19937_64 rng(seed * 1000003ull + wid);
+    for (;;) {
+      if (failed.load()) return;
+      uint64_t t = head.fetch_add(1);
+      if (t >= total) return;
+      uint32_t e = (uint32_t)(t / T) + 1;
+      const Tile& tile = g.tiles[t % T];
+      {
+        auto t0 = std::chrono::steady_clock::now();
+        while (epochs_done.load(std::memory_order_acquire) + 1 < e) {
+          if (failed.load()) return;
+          std::this_thread::yield();
+          if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(wait_ms)) {
+            failed.store(1);
+            fail_tile.store(t % T);
+            return;
+          }
+        }
+      }
+      if (tile.wait_ctr != kNoCounter) {
+        uint64_t target = (uint64_t)tile.need * e;
+        auto t0 = std::chrono::steady_clock::now();
+        while (ctr[tile.wait_ctr].load(std::memory_order_acquire) < target) {
+          if (failed.load()) return;
+          std::this_thread::yield();
+          if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(wait_ms)) {
+            failed.store(1);
+            fail_tile.store(t % T);
+            return;
+          }
+        }
+      }
+      if (rng() % 8 == 0) std::this_thread::sleep_for(std::chrono::microseconds(rng() % 50));
+      uint64_t d = done_idx.fetch_add(1);
+      if (done_order && d < total) done_order[d] = (int32_t)(t % T);
+      if ((int64_t)(t % T) == stuck_tile) continue;
+      for (uint32_t i = 0; i < tile.sig_cnt; ++i)
+        ctr[g.sig[tile.sig_off + i]].fetch_add(1, std::memory_order_release);
+      if (t % T == T - 1) epochs_done.fetch_add(1, std::memory_order_release);
+    }
+  };
+  std::vector<std::thread> th;
+  for (int i = 0; i < n_threads; ++i) th.emplace_back(worker, i);
+  for (auto& x : th) x.join();
+  if (failed.load()) {
+    *msg = fmt("simulated worker timed out waiting before tile %lld", (long long)fail_tile.load());
+    return WPK_ERR_TIMEOUT;
+  }
+  return WPK_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Weight image: fp32 norm gains; QKV rows permuted so that RoPE pair rows
+// (i, i + d/2) of every q/k head sit next to each other; gate/up rows
+// interleaved (gate j, up j); down projection stored K-chunk-major.
+std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_t* img) {
+  const wpk_model_cfg& m = g.m;
+  const int h = m.hidden, hd = m.head_dim;
+  const int q_rows = m.n_heads * hd, kv_rows = m.n_kv_heads * hd;
+  if (!w.embed || !w.final_norm || !w.layers || (!m.tied_embedding && !w.lm_head))
+    return "missing weight pointer";
+  auto gain = [&](const uint16_t* src, uint64_t off) {
+    float* dst = reinterpret_cast<float*>(img + off);
+    for (int i = 0; i < h; ++i) {
+      uint32_t u = (uint32_t)src[i] << 16;
+      memcpy(&dst[i], &u, 4);
+    }
+  };
+  auto row = [&](const uint16_t* src, uint64_t dst_off, int64_t dst_row, int64_t src_row, int cols) {
+    memcpy(img + dst_off + (uint64_t)dst_row * cols * 2, src + (uint64_t)src_row * cols, (size_t)cols * 2);
+  };
+  auto rope_phys = [&](int logical) {  // within a head
+    int i = logical % hd, head = logical / hd, half = hd / 2;
+    return head * hd + (i < half ? 2 * i : 2 * (i - half) + 1);
+  };
+  std::vector<std::thread> th;
+  std::string err;
+  for (int l = 0; l < m.n_layers; ++l) {
+    const wpk_layer_weights& W = w.layers[l];
+    if (!W.attn_norm || !W.wq || !W.wk || !W.wv || !W.wo || !W.ffn_norm || !W.w_gate || !W.w_up || !W.w_down)
+      return fmt("missing weight pointer in layer %lld", l);
+  }
+  auto do_layer = [&](int l) {
+    const wpk_layer_weights& W = w.layers[l];
+    const LayerDev& d = g.lay.layers[l];
+    gain(W.attn_norm, d.attn_norm);
+    gain(W.ffn_norm, d.ffn_norm);
+    for (int r = 0; r < q_rows; ++r) row(W.wq, d.qkv, rope_phys(r), r, h);
+    for (int r = 0; r < kv_rows; ++r) row(W.wk, d.qkv, q_rows + rope_phys(r), r, h);
+    for (int r = 0; r < kv_rows; ++r) row(W.wv, d.qkv, q_rows + kv_rows + r, r, h);
+    memcpy(img + d.wo, W.wo, (size_t)h * q_rows * 2);
+    for (int j = 0; j < m.ffn; ++j) {
+      row(W.w_gate, d.gu, 2 * j, j, h);
+      row(W.w_up, d.gu, 2 * j + 1, j, h);
+    }
+    const int kc = g.lay.down_kc;
+    uint16_t* dd = reinterpret_cast<uint16_t*>(img + d.down);
+    for (int c = 0; c < g.lay.n_down_chunks; ++c)
+      for (int r = 0; r < h; ++r)
+        memcpy(dd + ((uint64_t)c * h + r) * kc, W.w_down + (uint64_t)r * m.ffn + (uint64_t)c * kc, (size_t)kc * 2);
+  };
+  unsigned nt = std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
+  std::atomic<int> next{0};
+  for (unsigned i = 0; i < nt; ++i)
+    th.emplace_back([&] {
+      for (int l; (l = next.fetch_add(1)) < m.n_layers;) do_layer(l);
+    });
+  gain(w.final_norm, g.lay.final_norm);
+  memcpy(img + g.lay.embed, w.embed, (size_t)m.vocab * h * 2);
+  if (!m.tied_embedding) memcpy(img + g.lay.lm_head, w.lm_head, (size_t)m.vocab * h * 2);
+  for (auto& x : th) x.join();
+  return "";
+}
+
+}  // namespace wpk

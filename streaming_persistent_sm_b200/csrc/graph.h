@@ -1,0 +1,52 @@
+// Host graph compiler: turns a decoder shape + plan into the step program
+// (tiles in ticket order, dependency counters, signal lists, regions) and the
+// layout of the arranged weight image.
+#pragma once
+#include <string>
+#include <vector>
+
+#include "wpk_internal.h"
+
+namespace wpk {
+
+struct Plan {
+  int max_batch, max_context, page_tokens, n_workers, workers_per_sm, mode, resident, n_regions;
+  int region_cut[4];
+  int trace;
+  uint64_t wait_timeout_ns;
+  int slot_bytes, tile_bytes, split_pages, chunk_bytes;
+};
+
+struct Layout {
+  std::vector<LayerDev> layers;
+  uint64_t final_norm = 0, embed = 0, lm_head = 0;
+  uint64_t total = 0;
+  int down_kc = 0, n_down_chunks = 0;
+};
+
+struct CompiledGraph {
+  wpk_model_cfg m{};
+  Plan plan{};
+  Layout lay;
+  std::vector<Tile> tiles;                    // ticket order
+  std::vector<std::vector<Access>> access;    // per tile (for the verifier)
+  std::vector<std::vector<int32_t>> preds;    // expanded tile edges
+  std::vector<uint32_t> sig;                  // concatenated signal lists
+  std::vector<uint32_t> ctr_need;             // per counter
+  std::vector<OpGroup> groups;                // op groups in ticket order
+  std::vector<uint32_t> region_begin;         // n_regions + 1 ticket boundaries
+  int64_t n_edges = 0;
+  int64_t algo_weight_bytes = 0;              // weight bytes a step reads
+  int n_splits = 0, split_tokens = 0, max_blocks = 0;
+};
+
+// Returns "" on success, else an error message; *code receives the WPK code.
+std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan* out, int* code);
+std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code);
+std::string verify_graph(const CompiledGraph& g);
+int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t seed, int wait_ms,
+                   int stuck_tile, int32_t* done_order, std::string* msg);
+// Arrange host bf16 weights into the image (host buffer of lay.total bytes).
+std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_t* image);
+
+}  // namespace wpk

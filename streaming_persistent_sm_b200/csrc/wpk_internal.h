@@ -1,0 +1,136 @@
+// Internal tables shared by the host graph compiler (graph.cpp), the C ABI
+// (capi.cu) and the persistent kernel (runtime.cu).
+#pragma once
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/wpk.h"
+
+namespace wpk {
+
+constexpr uint32_t kNoCounter = 0xFFFFFFFFu;
+constexpr int kThreads = 256;          // threads per worker CTA
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxChunks = 8;          // mbarriers per staging slot
+constexpr int kActBytes = 32768;       // activation staging (fp32) per worker
+constexpr int kMaxGroup = 8;           // q heads per kv head handled by one attention tile
+
+// Op codes of the tiles.  One "op group" = the tiles of one op of one layer.
+enum Op : uint16_t {
+  OP_EMBED = 0,    // x = E[tok]
+  OP_QKV = 1,      // fused RMSNorm + [q;k;v] = W a + RoPE + KV-cache write
+  OP_ATTN = 2,     // split-KV GQA decode attention + last-arriver combine
+  OP_O = 3,        // x_mid = x + Wo attn  (also re-initialises x for down)
+  OP_GU = 4,       // fused RMSNorm + gate/up + SwiGLU
+  OP_DOWN = 5,     // x += Wd h  (split-K, accumulated)
+  OP_LMHEAD = 6,   // fused final RMSNorm + logits + packed argmax
+  OP_FINAL = 7,    // publish tokens, reset argmax, advance positions
+  OP_COUNT = 8
+};
+
+// One tile of the step program, in ticket order.  48 bytes.
+struct alignas(16) Tile {
+  uint16_t op;
+  uint16_t layer;
+  uint32_t wait_ctr;   // counter to wait on, or kNoCounter
+  uint32_t need;       // signals that counter receives per step
+  uint32_t sig_off;    // first entry of this tile's signal list
+  uint32_t sig_cnt;    // counters it increments when done
+  uint32_t w_bytes;    // bytes staged into the worker's slot before the wait
+  uint64_t w_off;      // byte offset of those bytes in the weight image
+  int32_t a0, a1, a2, a3;  // op arguments (see runtime.cu)
+};
+static_assert(sizeof(Tile) == 48, "Tile layout");
+
+// Device-side offsets of one layer's tensors in the weight image (bytes).
+struct LayerDev {
+  uint64_t attn_norm;   // fp32 [hidden]
+  uint64_t ffn_norm;    // fp32 [hidden]
+  uint64_t qkv;         // bf16 [qkv_rows][hidden], RoPE pairs adjacent
+  uint64_t wo;          // bf16 [hidden][q_rows]
+  uint64_t gu;          // bf16 [2*ffn][hidden], gate/up rows interleaved
+  uint64_t down;        // bf16 [n_kchunks][hidden][kc]
+};
+
+struct TraceRec {
+  uint32_t tile;
+  uint16_t worker;
+  uint16_t op;
+  uint32_t ev_issue, ev_start, ev_done, epoch;
+  uint64_t t_start_ns, t_end_ns;
+};
+static_assert(sizeof(TraceRec) == sizeof(wpk_trace_rec), "trace layout");
+
+struct ErrWord {
+  int32_t code;
+  uint32_t tile, counter, epoch, observed, target;
+};
+
+// Everything a kernel launch needs.  Passed by value.
+struct KParams {
+  // model shape
+  int n_layers, hidden, n_heads, n_kv, head_dim, ffn, vocab, group;
+  int q_rows, kv_rows, qkv_rows, down_kc, n_down_chunks;
+  float eps;
+  // plan
+  int max_batch, max_context, page_tokens, max_blocks, split_tokens, n_splits;
+  int slot_bytes, chunk_bytes;
+  uint64_t timeout_ns;
+  int trace;
+  // device buffers (weights image and KV are caller-owned)
+  const uint8_t* weights;
+  const LayerDev* layers;
+  uint64_t final_norm_off;   // fp32 [hidden]
+  uint64_t embed_off;        // bf16 [vocab][hidden]
+  uint64_t lm_head_off;      // bf16 [vocab][hidden]
+  uint16_t* kv;              // bf16 [n_layers][n_blocks][2][n_kv][page][head_dim]
+  int64_t n_blocks;
+  const int32_t* block_table;  // [max_batch][max_blocks]
+  const float2* rope;          // (cos, sin) [max_context][head_dim/2]
+  // scratch (caller-owned)
+  float* xa;       // [max_batch][hidden]   residual stream
+  float* xb;       // [max_batch][hidden]   residual after attention (read by FFN)
+  float* qbuf;     // [max_batch][q_rows]   roped queries
+  float* attn;     // [max_batch][q_rows]   attention output
+  float* hbuf;     // [max_batch][ffn]      SwiGLU output
+  float* part;     // [max_batch][n_kv][n_splits][group][2 + head_dim] partials
+  // library-owned state
+  uint32_t* arrive;          // [max_batch][n_kv] split arrivals
+  unsigned long long* best;  // [max_batch] packed argmax keys
+  int32_t* seqlen;           // [max_batch] tokens already in the cache
+  int32_t* tok_fb;           // [max_batch] last greedy tokens
+  int32_t* active_batch;     // [1]
+  const Tile* tiles;
+  const uint32_t* sig;
+  uint32_t* ctr;
+  uint32_t* head;            // queue heads, one per region
+  ErrWord* err;
+  TraceRec* trace_buf;
+  uint32_t* evclock;
+  // per-step I/O
+  const int32_t* in_tok;     // NULL = tok_fb
+  int in_tok_stride;
+  int32_t* out_tok;          // may be NULL
+  float* logits;             // may be NULL
+  // launch
+  uint32_t t_begin, t_end;   // ticket range of this launch
+  uint32_t epoch;            // counter target multiplier (>= 1)
+  int region;
+};
+
+// Host-side compiled graph.
+struct Access {
+  int buf;
+  int lo, hi;
+  int kind;        // 0 = read, 1 = write, 2 = accumulate (commutes with itself)
+  int group = -1;  // writes with the same group id (>= 0) form one logical write
+};
+
+enum Buf { BUF_XA = 0, BUF_XB, BUF_QKV, BUF_ATTN, BUF_H, BUF_LOGITS, BUF_BEST, BUF_TOK, BUF_COUNT };
+
+struct OpGroup {
+  int op, layer;
+  uint32_t begin, end;  // ticket range
+};
+
+}  // namespace wpk

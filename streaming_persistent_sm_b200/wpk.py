@@ -1,0 +1,317 @@
+"""ctypes binding of ``libwpk.so`` with the same entry-point names as ``include/wpk.h``.
+
+Argument marshalling only: every step of the decode/prefill path runs in the
+library's CUDA kernels.  Loading fails loudly when the library is missing;
+there is no fallback.  ``Engine`` adds torch-owned device buffers around a
+handle (PyTorch is used for device memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwpk.so")
+
+WPK_OK = 0
+WPK_ERR_INVALID_ARG = -1
+WPK_ERR_CUDA = -2
+WPK_ERR_TIMEOUT = -3
+WPK_ERR_NOT_LOADED = -4
+WPK_ERR_SHAPE = -5
+WPK_ERR_UNSUPPORTED = -6
+WPK_ERR_POISONED = -7
+WPK_MEGAKERNEL = 0
+WPK_PER_OP_GRAPH = 1
+
+OP_NAMES = ["embed", "qkv", "attn", "o", "gate_up", "down", "lm_head", "final"]
+
+_ERR_NAMES = {0: "OK", -1: "INVALID_ARG", -2: "CUDA", -3: "TIMEOUT", -4: "NOT_LOADED", -5: "SHAPE",
+              -6: "UNSUPPORTED", -7: "POISONED"}
+
+
+class WpkError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"wpk error {code} ({_ERR_NAMES.get(code, '?')}): {msg}")
+        self.code = code
+
+
+class wpk_model_cfg(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("hidden", C.c_int), ("n_heads", C.c_int), ("n_kv_heads", C.c_int),
+                ("head_dim", C.c_int), ("ffn", C.c_int), ("vocab", C.c_int), ("rms_eps", C.c_float),
+                ("rope_theta", C.c_float), ("tied_embedding", C.c_int)]
+
+
+class wpk_plan_cfg(C.Structure):
+    _fields_ = [("max_batch", C.c_int), ("max_context", C.c_int), ("page_tokens", C.c_int),
+                ("n_workers", C.c_int), ("workers_per_sm", C.c_int), ("mode", C.c_int), ("resident", C.c_int),
+                ("n_regions", C.c_int), ("region_cut", C.c_int * 4), ("trace", C.c_int),
+                ("wait_timeout_ns", C.c_uint64), ("slot_bytes", C.c_int), ("tile_bytes", C.c_int),
+                ("split_pages", C.c_int)]
+
+
+_P16 = C.POINTER(C.c_uint16)
+
+
+class wpk_layer_weights(C.Structure):
+    _fields_ = [(n, _P16) for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down")]
+
+
+class wpk_weights(C.Structure):
+    _fields_ = [("embed", _P16), ("final_norm", _P16), ("lm_head", _P16), ("layers", C.POINTER(wpk_layer_weights))]
+
+
+class wpk_graph_stats(C.Structure):
+    _fields_ = [("n_tiles", C.c_int64), ("n_counters", C.c_int64), ("n_edges", C.c_int64),
+                ("n_signals", C.c_int64), ("n_ops", C.c_int64), ("n_workers", C.c_int64),
+                ("weight_bytes", C.c_int64), ("region_begin", C.c_int64 * 5), ("n_regions", C.c_int64)]
+
+
+class wpk_error_info(C.Structure):
+    _fields_ = [("code", C.c_int32), ("tile", C.c_uint32), ("counter", C.c_uint32), ("epoch", C.c_uint32),
+                ("observed", C.c_uint32), ("target", C.c_uint32)]
+
+
+TRACE_DTYPE = np.dtype([("tile", "<u4"), ("worker", "<u2"), ("op", "<u2"), ("ev_issue", "<u4"),
+                        ("ev_start", "<u4"), ("ev_done", "<u4"), ("epoch", "<u4"), ("t_start_ns", "<u8"),
+                        ("t_end_ns", "<u8")])
+assert TRACE_DTYPE.itemsize == 40
+
+# Every symbol include/wpk.h declares, with its ctypes signature.
+_H = C.c_void_p
+_SIGS = {
+    "wpk_build_graph": (C.c_int, [C.POINTER(wpk_model_cfg), C.POINTER(wpk_plan_cfg), C.POINTER(_H)]),
+    "wpk_workspace_size": (C.c_int, [_H, C.POINTER(C.c_size_t), C.POINTER(C.c_size_t), C.POINTER(C.c_size_t)]),
+    "wpk_load_weights": (C.c_int, [_H, C.POINTER(wpk_weights), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "wpk_set_block_table": (C.c_int, [_H, C.POINTER(C.c_int32)]),
+    "wpk_prefill": (C.c_int, [_H, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "wpk_step": (C.c_int, [_H, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "wpk_graph_stats_get": (C.c_int, [_H, C.POINTER(wpk_graph_stats)]),
+    "wpk_get_edges": (C.c_int, [_H, C.POINTER(C.c_int32), C.c_int64, C.POINTER(C.c_int64)]),
+    "wpk_get_tile_ops": (C.c_int, [_H, C.POINTER(C.c_int32), C.c_int64]),
+    "wpk_verify_graph": (C.c_int, [_H]),
+    "wpk_simulate": (C.c_int, [_H, C.c_int, C.c_int, C.c_uint64, C.c_int, C.c_int, C.POINTER(C.c_int32)]),
+    "wpk_get_trace": (C.c_int, [_H, C.c_void_p, C.c_size_t]),
+    "wpk_get_error_info": (C.c_int, [_H, C.POINTER(wpk_error_info)]),
+    "wpk_last_error": (C.c_char_p, [_H]),
+    "wpk_destroy": (C.c_int, [_H]),
+    "wpk_debug_break_counter": (C.c_int, [_H, C.c_int]),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> C.CDLL:
+    """Load libwpk.so (raises if it was not built; there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m streaming_persistent_sm_b200.build`")
+    lib = C.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(rc: int, h=None):
+    if rc != WPK_OK:
+        msg = load_library().wpk_last_error(h).decode() if h else ""
+        raise WpkError(rc, msg)
+
+
+def model_cfg(shape) -> wpk_model_cfg:
+    return wpk_model_cfg(shape.n_layers, shape.hidden, shape.n_heads, shape.n_kv_heads, shape.head_dim, shape.ffn,
+                         shape.vocab, shape.rms_eps, shape.rope_theta, 1 if shape.tied_embedding else 0)
+
+
+def plan_cfg(max_batch: int, max_context: int, mode: int = WPK_MEGAKERNEL, n_regions: int = 1,
+             region_cut: Sequence[int] = (0, 0, 0, 0), trace: int = 0, wait_timeout_ns: int = 0,
+             page_tokens: int = 0, n_workers: int = 0, workers_per_sm: int = 0, resident: int = 0,
+             slot_bytes: int = 0, tile_bytes: int = 0, split_pages: int = 0) -> wpk_plan_cfg:
+    cut = (C.c_int * 4)(*list(region_cut) + [0] * (4 - len(region_cut)))
+    return wpk_plan_cfg(max_batch, max_context, page_tokens, n_workers, workers_per_sm, mode, resident, n_regions,
+                        cut, trace, wait_timeout_ns, slot_bytes, tile_bytes, split_pages)
+
+
+# ----------------------------------------------------------- thin wrappers --
+def wpk_build_graph(model: wpk_model_cfg, plan: wpk_plan_cfg) -> C.c_void_p:
+    h = C.c_void_p()
+    _check(load_library().wpk_build_graph(C.byref(model), C.byref(plan), C.byref(h)))
+    return h
+
+
+def wpk_workspace_size(h):
+    w, k, s = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    _check(load_library().wpk_workspace_size(h, C.byref(w), C.byref(k), C.byref(s)), h)
+    return w.value, k.value, s.value
+
+
+def wpk_load_weights(h, weights: wpk_weights, dev_weights: int, dev_kv: int, dev_scratch: int, stream: int = 0):
+    _check(load_library().wpk_load_weights(h, C.byref(weights), dev_weights, dev_kv, dev_scratch, stream), h)
+
+
+def wpk_set_block_table(h, table: np.ndarray):
+    t = np.ascontiguousarray(table, dtype=np.int32)
+    _check(load_library().wpk_set_block_table(h, t.ctypes.data_as(C.POINTER(C.c_int32))), h)
+
+
+def wpk_prefill(h, tokens_dev: int, batch: int, prompt_len: int, first_tok_dev: int, logits_dev: int = 0,
+                stream: int = 0):
+    _check(load_library().wpk_prefill(h, tokens_dev, batch, prompt_len, first_tok_dev, logits_dev or None,
+                                      stream or None), h)
+
+
+def wpk_step(h, in_tok_dev: int = 0, out_tok_dev: int = 0, logits_dev: int = 0, stream: int = 0):
+    _check(load_library().wpk_step(h, in_tok_dev or None, out_tok_dev or None, logits_dev or None, stream or None), h)
+
+
+def wpk_graph_stats_get(h) -> dict:
+    st = wpk_graph_stats()
+    _check(load_library().wpk_graph_stats_get(h, C.byref(st)), h)
+    d = {n: getattr(st, n) for n, _ in wpk_graph_stats._fields_ if n != "region_begin"}
+    d["region_begin"] = list(st.region_begin)[: st.n_regions + 1]
+    return d
+
+
+def wpk_get_edges(h) -> np.ndarray:
+    n = C.c_int64()
+    _check(load_library().wpk_get_edges(h, None, 0, C.byref(n)), h)
+    buf = np.zeros((n.value, 2), dtype=np.int32)
+    _check(load_library().wpk_get_edges(h, buf.ctypes.data_as(C.POINTER(C.c_int32)), n.value, C.byref(n)), h)
+    return buf
+
+
+def wpk_get_tile_ops(h, n_tiles: int) -> np.ndarray:
+    ops = np.zeros(n_tiles, dtype=np.int32)
+    _check(load_library().wpk_get_tile_ops(h, ops.ctypes.data_as(C.POINTER(C.c_int32)), n_tiles), h)
+    return ops
+
+
+def wpk_verify_graph(h):
+    _check(load_library().wpk_verify_graph(h), h)
+
+
+def wpk_simulate(h, n_threads: int, n_epochs: int, seed: int, wait_ms: int = 5000, stuck_tile: int = -1,
+                 n_tiles: int = 0):
+    order = np.full(max(1, n_tiles * n_epochs), -1, dtype=np.int32)
+    rc = load_library().wpk_simulate(h, n_threads, n_epochs, seed, wait_ms, stuck_tile,
+                                     order.ctypes.data_as(C.POINTER(C.c_int32)) if n_tiles else None)
+    return rc, order
+
+
+def wpk_get_trace(h, n_tiles: int) -> np.ndarray:
+    buf = np.zeros(n_tiles, dtype=TRACE_DTYPE)
+    _check(load_library().wpk_get_trace(h, buf.ctypes.data, buf.nbytes), h)
+    return buf
+
+
+def wpk_get_error_info(h) -> dict:
+    e = wpk_error_info()
+    _check(load_library().wpk_get_error_info(h, C.byref(e)), h)
+    return {n: getattr(e, n) for n, _ in wpk_error_info._fields_}
+
+
+def wpk_last_error(h) -> str:
+    return load_library().wpk_last_error(h).decode()
+
+
+def wpk_destroy(h):
+    _check(load_library().wpk_destroy(h))
+
+
+def wpk_debug_break_counter(h, counter: int):
+    _check(load_library().wpk_debug_break_counter(h, counter), h)
+
+
+# ------------------------------------------------------------------ Engine --
+class _HostWeights:
+    """Keeps the numpy arrays alive while their pointers are in a wpk_weights."""
+
+    def __init__(self, shape, weights: Dict[str, np.ndarray], prefix: str = ""):
+        self.arrays = []
+
+        def ptr(name):
+            a = np.ascontiguousarray(weights[prefix + name], dtype=np.uint16)
+            self.arrays.append(a)
+            return a.ctypes.data_as(_P16)
+
+        self.layers = (wpk_layer_weights * shape.n_layers)()
+        for l in range(shape.n_layers):
+            p = f"layers.{l}."
+            for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down"):
+                setattr(self.layers[l], n, ptr(p + n))
+        self.struct = wpk_weights(ptr("embed"), ptr("final_norm"),
+                                  ptr("lm_head") if not shape.tied_embedding else None, self.layers)
+
+
+class Engine:
+    """A handle plus torch-owned device buffers (weights image, KV pages, scratch)."""
+
+    def __init__(self, shape, weights: Dict[str, np.ndarray], max_batch: int, max_context: int, **plan_kw):
+        import torch
+
+        self.torch = torch
+        self.shape = shape
+        self.plan = plan_cfg(max_batch, max_context, **plan_kw)
+        self.h = wpk_build_graph(model_cfg(shape), self.plan)
+        self.stats = wpk_graph_stats_get(self.h)
+        wb, kb, sb = wpk_workspace_size(self.h)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.dev_weights = torch.empty(max(wb, 256), dtype=torch.uint8, device=dev)
+        self.dev_kv = torch.empty(max(kb, 256), dtype=torch.uint8, device=dev)
+        self.dev_scratch = torch.empty(max(sb, 256), dtype=torch.uint8, device=dev)
+        hw = _HostWeights(shape, weights)
+        wpk_load_weights(self.h, hw.struct, self.dev_weights.data_ptr(), self.dev_kv.data_ptr(),
+                         self.dev_scratch.data_ptr(), self._stream())
+        self.max_batch = max_batch
+        self.batch = 0
+
+    def _stream(self) -> int:
+        return self.torch.cuda.current_stream().cuda_stream
+
+    def prefill(self, tokens, want_logits: bool = False):
+        torch = self.torch
+        tok = torch.as_tensor(np.ascontiguousarray(tokens, dtype=np.int32)).cuda()
+        B, T = tok.shape
+        self.batch = B
+        first = torch.empty(B, dtype=torch.int32, device=tok.device)
+        logits = torch.empty((B, self.shape.vocab), dtype=torch.float32, device=tok.device) if want_logits else None
+        wpk_prefill(self.h, tok.data_ptr(), B, T, first.data_ptr(), logits.data_ptr() if want_logits else 0,
+                    self._stream())
+        self._keep = tok
+        return first, logits
+
+    def step(self, in_tok=None, want_logits: bool = False, out_tok=None, logits=None):
+        torch = self.torch
+        B = self.batch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        itp = 0
+        if in_tok is not None:
+            it = in_tok if isinstance(in_tok, torch.Tensor) else torch.as_tensor(
+                np.ascontiguousarray(in_tok, dtype=np.int32), device=dev)
+            self._keep_in = it
+            itp = it.data_ptr()
+        if out_tok is None:
+            out_tok = torch.empty(B, dtype=torch.int32, device=dev)
+        if want_logits and logits is None:
+            logits = torch.empty((B, self.shape.vocab), dtype=torch.float32, device=dev)
+        wpk_step(self.h, itp, out_tok.data_ptr(), logits.data_ptr() if logits is not None else 0, self._stream())
+        return out_tok, logits
+
+    def close(self):
+        if self.h:
+            wpk_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

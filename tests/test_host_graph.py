@@ -1,0 +1,156 @@
+"""Host-side checks of the C ABI and the graph compiler (no GPU needed)."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from streaming_persistent_sm_b200 import wpk as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(W.LIB_PATH):
+        from streaming_persistent_sm_b200 import build
+
+        build.build()
+    return W.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    header = open(os.path.join(ROOT, "include", "wpk.h")).read()
+    declared = set(re.findall(r"^\s*(?:const\s+char\s*\*|int)\s*(wpk_\w+)\s*\(", header, re.M))
+    assert len(declared) >= 16
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    assert declared == set(W._SIGS), declared ^ set(W._SIGS)
+
+
+def _graph(shape=synth.TINY, **kw):
+    B = kw.pop("max_batch", 1)
+    ctx = kw.pop("max_context", 64)
+    return W.wpk_build_graph(W.model_cfg(shape), W.plan_cfg(B, ctx, **kw))
+
+
+def test_tiny_graph_verifies_and_counters_dedup(lib):
+    h = _graph()
+    try:
+        st = W.wpk_graph_stats_get(h)
+        W.wpk_verify_graph(h)
+        ops = W.wpk_get_tile_ops(h, st["n_tiles"])
+        assert ops[0] == 0 and ops[-1] == 7  # embed first, final last
+        # per layer: 1 QKV + one per kv head + O + gate/up + one per down K-chunk
+        assert st["n_counters"] == synth.TINY.n_layers * (4 + synth.TINY.n_kv_heads) + 2
+        # every tile but the last signals exactly one counter
+        assert st["n_signals"] == st["n_tiles"] - 1
+        assert st["weight_bytes"] == sum(np.prod(s) * 2 for n, s, k in synth.tensor_specs(synth.TINY) if k == "normal")
+        edges = W.wpk_get_edges(h)
+        assert np.all(edges[:, 0] < edges[:, 1])  # ticket order is topological
+    finally:
+        W.wpk_destroy(h)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(max_batch=3, max_context=200, split_pages=2),
+    dict(max_batch=2, max_context=130, page_tokens=32, tile_bytes=4096, slot_bytes=16384),
+    dict(max_batch=1, max_context=64, n_regions=3, region_cut=(0, 1, 2, 0)),
+])
+def test_graph_variants_verify(lib, kw):
+    h = _graph(**kw)
+    try:
+        W.wpk_verify_graph(h)
+        st = W.wpk_graph_stats_get(h)
+        rb = st["region_begin"]
+        assert rb[0] == 0 and rb[-1] == st["n_tiles"] and all(a < b for a, b in zip(rb, rb[1:]))
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_down_projection_uses_chunk_edges(lib):
+    # the 1B shape splits the down projection in 4 K-chunks; each chunk's tiles
+    # wait only for the gate/up tiles producing that chunk (finer edges)
+    s = synth.ModelShape(n_layers=1, hidden=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=8192, vocab=512)
+    h = _graph(s)
+    try:
+        W.wpk_verify_graph(h)
+        st = W.wpk_graph_stats_get(h)
+        ops = W.wpk_get_tile_ops(h, st["n_tiles"])
+        e = W.wpk_get_edges(h)
+        gu = np.flatnonzero(ops == 4)
+        down = np.flatnonzero(ops == 5)
+        preds_of_down = {v: set(e[e[:, 1] == v, 0]) for v in down}
+        sizes = {len(p) for p in preds_of_down.values()}
+        assert sizes == {len(gu) // 4}
+        assert len({frozenset(p) for p in preds_of_down.values()}) == 4
+    finally:
+        W.wpk_destroy(h)
+
+
+@pytest.mark.parametrize("threads", [1, 3, 17])
+def test_cpu_schedule_simulator_is_deadlock_free(lib, threads):
+    h = _graph(max_batch=2, max_context=128)
+    try:
+        st = W.wpk_graph_stats_get(h)
+        T = st["n_tiles"]
+        rc, order = W.wpk_simulate(h, threads, 3, 42 + threads, 10000, -1, T)
+        assert rc == 0, W.wpk_last_error(h)
+        e = W.wpk_get_edges(h)
+        for ep in range(3):
+            pos = np.empty(T, dtype=np.int64)
+            seg = order[ep * T:(ep + 1) * T]
+            # a step starts only after the previous one completed (the doorbell),
+            # so epoch ep's tiles are the ep-th block of completions
+            pos[seg] = np.arange(T)
+            assert sorted(seg.tolist()) == list(range(T))
+            assert np.all(pos[e[:, 0]] < pos[e[:, 1]])
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_simulator_reports_stuck_producer_as_timeout(lib):
+    h = _graph()
+    try:
+        rc, _ = W.wpk_simulate(h, 4, 1, 1, 200, 5, 0)
+        assert rc == W.WPK_ERR_TIMEOUT
+        assert "timed out" in W.wpk_last_error(h)
+    finally:
+        W.wpk_destroy(h)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(max_batch=0), dict(n_regions=5), dict(mode=7), dict(slot_bytes=1000),
+    dict(n_regions=2, region_cut=(0, 9, 0, 0)), dict(split_pages=8),
+])
+def test_invalid_plans_are_rejected(lib, bad):
+    with pytest.raises(W.WpkError):
+        _graph(**bad)
+
+
+def test_host_only_handle_refuses_device_calls(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("host-only behaviour")
+    h = _graph()
+    try:
+        with pytest.raises(W.WpkError) as ei:
+            W.wpk_step(h)
+        assert ei.value.code == W.WPK_ERR_CUDA
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_llama1b_graph_shape(lib):
+    h = _graph(synth.LLAMA_1B, max_batch=1, max_context=624)
+    try:
+        st = W.wpk_graph_stats_get(h)
+        # 16 layers x (QKV + 8 kv heads + O + gate/up + 4 down chunks) + LM head + final
+        assert st["n_counters"] == 16 * 15 + 2
+        bf16_bytes = sum(np.prod(s) * 2 for n, s, k in synth.tensor_specs(synth.LLAMA_1B) if k == "normal")
+        # matmul weights and the tied embedding, read once per step (norm gains excluded)
+        assert st["weight_bytes"] == bf16_bytes == 2_471_493_632
+    finally:
+        W.wpk_destroy(h)
