@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--regions", default="", help="comma-separated region cuts, e.g. 0,8")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=None)
+    ap.add_argument("--prompt-len", type=int, default=None, help="override the prompt length (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tile-bytes", type=int, default=0)
     ap.add_argument("--slot-bytes", type=int, default=0)
@@ -207,7 +208,7 @@ def main():
 
     wl = synth.WORKLOADS[args.workload]
     s = wl.model
-    B, T = wl.batch, wl.prompt_len
+    B, T = wl.batch, (wl.prompt_len if args.prompt_len is None else args.prompt_len)
     decode_steps = wl.steps if args.decode_steps is None else args.decode_steps
     tokens_per_step, with_prefill = job_tokens(wl, decode_steps)
     ctx = T + max(decode_steps, 1)

@@ -126,7 +126,9 @@ def test_stalled_dependency_times_out_and_poisons_handle(weights):
         eng.step()
         info = W.wpk_get_error_info(eng.h)
         assert info["code"] == W.WPK_ERR_TIMEOUT
-        assert info["counter"] == 3 and info["observed"] < info["target"]
+        # the first waiter to give up records itself: the broken counter or a
+        # counter downstream of it, in either case one that was never satisfied
+        assert info["counter"] >= 3 and info["observed"] < info["target"]
         with pytest.raises(W.WpkError) as ei:
             eng.step()
         assert ei.value.code == W.WPK_ERR_POISONED
