@@ -70,7 +70,7 @@ typedef struct wpk_plan_cfg {
   int max_context;      /* tokens per sequence, prompt included                */
   int page_tokens;      /* KV page size in tokens (0 = 64)                     */
   int n_workers;        /* resident worker CTAs (0 = #SMs x workers_per_sm)    */
-  int workers_per_sm;   /* 0 = 2                                               */
+  int workers_per_sm;   /* 0 = 1                                               */
   int mode;             /* WPK_MEGAKERNEL or WPK_PER_OP_GRAPH                  */
   int resident;         /* megakernel only: 1 = the grid stays alive across
                            steps and is driven by a host doorbell              */
@@ -79,9 +79,13 @@ typedef struct wpk_plan_cfg {
                            equal to n_layers puts the LM head in its own region */
   int trace;            /* 1 = record the per-tile device trace                */
   uint64_t wait_timeout_ns; /* bound on every device wait (0 = 2 s)            */
-  int slot_bytes;       /* staging slot per worker (0 = 65536)                 */
-  int tile_bytes;       /* target weight bytes per tile (0 = 32768)            */
+  int slot_bytes;       /* staging slot per worker, used as a ring of 16 KB
+                           chunk stages (0 = as large as shared memory allows) */
+  int tile_bytes;       /* target weight bytes per tile (0 = 65536)            */
   int split_pages;      /* KV pages per attention split (0 = 1)                */
+  int lookahead;        /* tiles a worker may claim and stage ahead of the one
+                           it computes (0 = 4); 1 = a tile's weights are staged
+                           only after the previous tile of that worker is done */
 } wpk_plan_cfg;
 
 /* Host weights: bf16 bit patterns, row-major [out][in]. */

@@ -14,7 +14,7 @@
 #include "graph.h"
 
 namespace wpk {
-size_t worker_smem_bytes(int slot_bytes);
+size_t worker_smem_bytes(int n_stages, int act_bytes);
 const void* persistent_kernel_ptr();
 const void* per_op_kernel_ptr();
 }  // namespace wpk
@@ -31,7 +31,7 @@ struct GraphEntry {
 struct wpk_handle {
   CompiledGraph g;
   int device = 0, n_sms = 0, n_workers = 0;
-  size_t smem = 0;
+  size_t smem = 0, smem_per_op = 0;
   // library-owned device tables (one allocation)
   uint8_t* d_base = nullptr;
   Tile* d_tiles = nullptr;
@@ -118,8 +118,9 @@ KParams make_params(const wpk_handle* h) {
   P.max_blocks = g.max_blocks;
   P.split_tokens = g.split_tokens;
   P.n_splits = g.n_splits;
-  P.slot_bytes = g.plan.slot_bytes;
-  P.chunk_bytes = g.plan.chunk_bytes;
+  P.n_stages = g.plan.slot_bytes / kStageBytes;
+  P.lookahead = g.plan.lookahead;
+  P.act_bytes = g.plan.act_bytes;
   P.timeout_ns = g.plan.wait_timeout_ns;
   P.trace = g.plan.trace;
   P.weights = h->weights;
@@ -181,7 +182,7 @@ int launch_megakernel(wpk_handle* h, const KParams& base, cudaStream_t s) {
     P.t_end = g.region_begin[r + 1];
     P.region = r;
     void* args[] = {&P};
-    CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kThreads), args,
+    CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
                                             h->smem, s));
   }
   return WPK_OK;
@@ -199,9 +200,11 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
     KParams P = base;
     P.t_begin = og.begin;
     P.t_end = og.end;
+    P.per_op = 1;
+    P.n_stages = g.plan.per_op_slot / kStageBytes;
     void* args[] = {&P};
-    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kThreads), args, h->smem,
-                                     h->capture_stream);
+    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
+                                     h->smem_per_op, h->capture_stream);
     if (e != cudaSuccess) {
       cudaGraph_t junk = nullptr;
       cudaStreamEndCapture(h->capture_stream, &junk);
@@ -257,12 +260,16 @@ static int setup_device(wpk_handle* h) {
   const wpk_model_cfg* model = &g.m;
   CUDA_TRY(h, cudaGetDevice(&h->device));
   CUDA_TRY(h, cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, h->device));
-  h->smem = worker_smem_bytes(p.slot_bytes);
+  h->smem = worker_smem_bytes(p.slot_bytes / kStageBytes, p.act_bytes);
+  h->smem_per_op = worker_smem_bytes(p.per_op_slot / kStageBytes, p.act_bytes);
+  if (h->smem > (size_t)kMaxSmem || h->smem_per_op > (size_t)kMaxSmem)
+    return fail(h, WPK_ERR_UNSUPPORTED, "staging slot and activations exceed shared memory");
   CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)h->smem));
-  CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)h->smem));
+  CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)h->smem_per_op));
   int per_sm = 0;
-  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kThreads, h->smem));
+  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kCtaThreads, h->smem));
   h->n_workers = p.n_workers ? p.n_workers : h->n_sms * p.workers_per_sm;
   if (per_sm < 1 || h->n_workers > per_sm * h->n_sms)
     return fail(h, WPK_ERR_UNSUPPORTED, "the worker grid cannot be co-resident with this slot size");

@@ -52,7 +52,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   p->max_context = in.max_context;
   p->page_tokens = in.page_tokens ? in.page_tokens : 64;
   if (p->page_tokens % 8 || p->page_tokens > 256) return "page_tokens must be a multiple of 8, <= 256";
-  p->workers_per_sm = in.workers_per_sm ? in.workers_per_sm : 2;
+  p->workers_per_sm = in.workers_per_sm ? in.workers_per_sm : 1;
   p->n_workers = in.n_workers;
   if (p->n_workers < 0 || p->workers_per_sm < 0 || p->workers_per_sm > 4) return "bad worker count";
   p->mode = in.mode;
@@ -71,18 +71,32 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   }
   p->trace = in.trace;
   p->wait_timeout_ns = in.wait_timeout_ns ? in.wait_timeout_ns : 2000000000ull;
-  p->slot_bytes = in.slot_bytes ? in.slot_bytes : 65536;
-  if (p->slot_bytes % 1024 || p->slot_bytes < 16384 || p->slot_bytes > 160 * 1024)
-    return "slot_bytes must be a multiple of 1024 in [16K, 160K]";
-  p->tile_bytes = in.tile_bytes ? in.tile_bytes : 32768;
-  if (p->tile_bytes > p->slot_bytes || p->tile_bytes < 1024) return "tile_bytes must be in [1K, slot_bytes]";
+  p->lookahead = in.lookahead ? in.lookahead : 4;
+  if (p->lookahead < 1 || p->lookahead > kMaxQueue) return "lookahead must be 1..8";
+  // activation staging: up to kMaxGemvBatch rows of the longest GEMV K (<= 2048)
+  const int q_rows = m.n_heads * m.head_dim;
+  const int kmax = std::max(std::max(m.hidden, q_rows), std::min(m.ffn, 2048));
+  if (kmax > 2048) { *code = WPK_ERR_UNSUPPORTED; return "hidden and n_heads*head_dim must be <= 2048"; }
+  p->act_bytes = std::max(16384, std::min(in.max_batch, kMaxGemvBatch) * kmax * 4);
+  p->act_bytes = (p->act_bytes + 1023) / 1024 * 1024;
+  const int fixed = 4096 + 1024;  // partial outputs, tile queue, barriers
+  const int budget = std::min(kMaxSmem, 233472 / p->workers_per_sm - 1024) - p->act_bytes - fixed;
+  if (in.slot_bytes) {
+    if (in.slot_bytes % kStageBytes || in.slot_bytes < kStageBytes || in.slot_bytes > kMaxStages * kStageBytes)
+      return "slot_bytes must be a multiple of 16384, at most 13 stages";
+    if (in.slot_bytes > budget) return "slot_bytes does not fit shared memory with this many workers per SM";
+    p->slot_bytes = in.slot_bytes;
+  } else {
+    p->slot_bytes = std::min(kMaxStages, budget / kStageBytes) * kStageBytes;
+    if (p->slot_bytes < kStageBytes) return "no room for a staging slot";
+  }
+  p->tile_bytes = in.tile_bytes ? in.tile_bytes : 65536;
+  if (p->tile_bytes < 1024 || p->tile_bytes > 1 << 20) return "tile_bytes must be in [1K, 1M]";
   p->split_pages = in.split_pages ? in.split_pages : 1;
   if (p->split_pages < 1) return "split_pages must be >= 1";
-  if ((int64_t)p->split_pages * p->page_tokens * m.head_dim * 2 * 2 > p->slot_bytes)
-    return "an attention split's K/V pages do not fit the slot";
-  if (p->split_pages * p->page_tokens * (m.n_heads / m.n_kv_heads) > 8 * kThreads)
-    return "attention split too long for one tile";
-  p->chunk_bytes = p->slot_bytes / kMaxChunks;
+  if ((int64_t)p->split_pages * p->page_tokens * m.head_dim * 2 * 2 > kStageBytes)
+    return "an attention split's K/V pages do not fit one 16 KB stage";
+  p->per_op_slot = 0;  // set by compile_graph
   *code = WPK_OK;
   return "";
 }
@@ -212,8 +226,7 @@ int rows_per_tile(int row_bytes, const Plan& p) {
   int r = p.tile_bytes / row_bytes;
   r = r / 8 * 8;
   if (r < 8) r = 8;
-  while (r > 8 && r * row_bytes > p.slot_bytes) r -= 8;
-  return std::min(r, 256);
+  return std::min(r, kMaxTileRows);
 }
 
 }  // namespace
@@ -228,10 +241,8 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   int nch = (m.ffn + 2047) / 2048;
   while (m.ffn % nch || (m.ffn / nch) % 8) ++nch;
   const int kc = m.ffn / nch;
-  if ((int64_t)h * 4 * 1 > kActBytes * 4) return "hidden too large for activation staging";
-  if (8LL * h * 2 > p.slot_bytes || 8LL * q_rows * 2 > p.slot_bytes || 8LL * kc * 2 > p.slot_bytes)
-    return "a row block of 8 rows does not fit the staging slot";
-  if (q_rows > 8192) return "q_rows > 8192";
+  if (h * 2 > kStageBytes || q_rows * 2 > kStageBytes || kc * 2 > kStageBytes)
+    return "a weight row does not fit one 16 KB stage";
 
   // ---- weight image layout ----
   Layout& L = g->lay;
@@ -353,6 +364,15 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   }
   add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0}, {BUF_TOK, 0, 1, 1}});
   g->algo_weight_bytes = wbytes;
+  // a per-op CTA holds one whole tile in its ring
+  int max_chunks = 1;
+  for (const Tile& t : T)
+    if (t.op != OP_ATTN && t.w_bytes) {
+      const int rpc = std::max(2, (kStageBytes / (t.a3 * 2)) & ~1);
+      max_chunks = std::max(max_chunks, (t.a1 + rpc - 1) / rpc);
+    }
+  // larger tiles stream through the ring
+  g->plan.per_op_slot = std::min(max_chunks, kMaxStages) * kStageBytes;
   if (T.size() >= (1u << 31)) return "too many tiles";
 
   // ---- edges from dataflow ----

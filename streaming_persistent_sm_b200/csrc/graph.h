@@ -14,7 +14,9 @@ struct Plan {
   int region_cut[4];
   int trace;
   uint64_t wait_timeout_ns;
-  int slot_bytes, tile_bytes, split_pages, chunk_bytes;
+  int slot_bytes, tile_bytes, split_pages, lookahead;
+  int act_bytes;        // activation staging per worker (fp32)
+  int per_op_slot;      // ring bytes of a per-op CTA (holds one whole tile)
 };
 
 struct Layout {

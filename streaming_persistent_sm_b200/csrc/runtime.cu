@@ -1,27 +1,33 @@
-// Persistent decode program for sm_100a: the worker loop and the tile bodies.
+// Persistent decode program for sm_100a: the worker and the tile bodies.
 //
-// Worker loop ("Why real-time inference wants a megakernel", "What the
-// megakernel changes": wait for dependencies, run, signal consumers):
-//   1. take the next ticket from the device queue (one atomic per tile; the
-//      ticket after it is claimed while the current tile runs),
-//   2. issue the tile's staging copy (weights, or the KV pages of an attention
-//      split) into the worker's one staging slot - before waiting, so the load
-//      overlaps the predecessors ("One Megakernel is Not Enough", Table I,
-//      weight prefetch: one staging slot per worker, the load is queued while
-//      predecessors run, compute still waits for them),
-//   3. wait (acquire, bounded by %globaltimer) until the tile's counter holds
-//      need x epoch,
-//   4. run the body; tensors consumed inside the body (normalised activations,
-//      pre-RoPE q/k, gate/up) are never stored (Table I, on-chip forwarding),
-//   5. release-increment the counters of its consumers.
-// Tickets are handed out in a topological order and every resident worker
-// holds at most two, so the smallest unfinished ticket can always run: the
-// program cannot deadlock while all workers are co-resident (cooperative
-// launch guarantees that).
+// A worker is one CTA: a producer warp and eight consumer (compute) warps.
+//   producer: takes tickets from the device queue (one atomic per tile), and
+//     for each tile streams its staging data - weight rows, or the KV pages of
+//     an attention split - into the worker's staging slot, a ring of 16 KB
+//     chunk stages, with bulk copies.  It does this before the tile's
+//     predecessors are done ("One Megakernel is Not Enough", Table I, weight
+//     prefetch: a staged tile's weight load is queued while its predecessors
+//     still run; its compute still waits for them).  It may hold up to
+//     `lookahead` tiles; lookahead 1 stages a tile only once the worker's
+//     previous tile has finished.
+//   consumers: take the worker's tiles in ticket order, wait (acquire,
+//     bounded by %globaltimer) until the tile's counter holds need x epoch,
+//     compute each chunk as it lands, release the stage, and after the
+//     epilogue release-increment the counters of the tile's consumers ("Why
+//     real-time inference wants a megakernel", "What the megakernel changes":
+//     wait for dependencies, run, signal consumers).
+// Tensors consumed inside a tile (normalised activations, pre-RoPE q/k,
+// gate/up) are never stored ("One Megakernel is Not Enough", Table I, on-chip
+// forwarding); the normalised activation a worker staged for one tile is kept
+// for its next tile of the same op.
 //
-// Every wait is bounded: on timeout the worker records {code, tile, counter,
-// epoch, observed, target} in the error word, waits (bounded) for its own
-// copies in flight and returns; other workers see the error word and stop.
+// Deadlock freedom: tickets follow a topological order, each worker computes
+// its tiles in ticket order and streams their data in that order, so the
+// worker holding the smallest unfinished ticket can always run it; the grid
+// is co-resident (cooperative launch).  Every wait is bounded: on timeout a
+// worker records {code, tile, counter, epoch, observed, target} in the error
+// word, the other workers see it and stop, and each waits (bounded) for its
+// own copies in flight before returning.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -32,22 +38,63 @@ namespace wpk {
 
 namespace {
 
-constexpr int kOutFloats = 1024;  // GEMV partial outputs [row][4]
+constexpr int kOutFloats = kMaxTileRows * kMaxGemvBatch;  // GEMV partial outputs [row][8]
+constexpr int kNoAct = -1;
 
-struct Ctx {
-  uint8_t* slot;
-  float* act;
-  float* out;
-  uint64_t* bars;
+struct TQEntry {  // producer -> consumers, one per tile held by the worker
+  Tile tile;
+  uint32_t ticket;
+  int32_t valid;
+  int32_t n_chunks;
+  int32_t rows_per_chunk;
+  uint32_t ev_issue;  // event clock when its first copy was issued (trace)
 };
 
-__device__ __forceinline__ Ctx carve(uint8_t* base, int slot_bytes) {
-  Ctx c;
-  c.slot = base;
-  c.act = reinterpret_cast<float*>(base + slot_bytes);
-  c.out = c.act + kActBytes / 4;
-  c.bars = reinterpret_cast<uint64_t*>(c.out + kOutFloats);
-  return c;
+struct Shared {
+  uint8_t* ring;
+  float* act;
+  float* out;
+  TQEntry* tq;
+  uint64_t* full;    // [n_stages]
+  uint64_t* empty;   // [n_stages]
+  uint64_t* tq_full;   // [kMaxQueue]
+  uint64_t* tq_empty;  // [kMaxQueue]
+};
+
+__device__ __forceinline__ Shared carve(uint8_t* base, const KParams& P) {
+  Shared s;
+  s.ring = base;
+  uint8_t* p = base + (size_t)P.n_stages * kStageBytes;
+  s.act = reinterpret_cast<float*>(p);
+  p += P.act_bytes;
+  s.out = reinterpret_cast<float*>(p);
+  p += kOutFloats * 4;
+  s.tq = reinterpret_cast<TQEntry*>(p);
+  p += kMaxQueue * sizeof(TQEntry);
+  s.full = reinterpret_cast<uint64_t*>(p);
+  s.empty = s.full + kMaxStages;
+  s.tq_full = s.empty + kMaxStages;
+  s.tq_empty = s.tq_full + kMaxQueue;
+  return s;
+}
+
+// Consumer-only barrier (named barrier 1, the eight compute warps).
+__device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool cbar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -92,15 +139,19 @@ __device__ void record_error(const KParams& P, int code, uint32_t tile, uint32_t
   }
 }
 
-// Bounded wait for a staging barrier; every thread calls it.
-__device__ bool wait_bar(const KParams& P, uint64_t* bar, uint32_t parity, uint32_t tile) {
+// Bounded wait on an mbarrier phase.  `abort` (shared) ends the wait early.
+__device__ bool wait_phase(const KParams& P, uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t tile) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31) == 0 && globaltimer() - t0 > P.timeout_ns) {
-      record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, 0, 0);
-      return false;
+    if ((it & 31) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > P.timeout_ns) {
+        record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, 0, 0);
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
@@ -112,9 +163,6 @@ __device__ __forceinline__ size_t kv_index(const KParams& P, int layer, int bloc
 
 __device__ __forceinline__ int active_batch(const KParams& P) { return *P.active_batch; }
 
-// ---------------------------------------------------------------------------
-// Staging: which barriers a tile arms, and the copies (thread 0 only).
-// ---------------------------------------------------------------------------
 struct AttnSpan {
   int b, g, j, pos, t0, t1;  // tokens [t0, t1) of sequence b, current position pos
 };
@@ -130,81 +178,77 @@ __device__ __forceinline__ AttnSpan attn_span(const KParams& P, const Tile& T) {
   return s;
 }
 
-__device__ __forceinline__ int gemv_rows_per_chunk(const KParams& P, int K) {
-  int r = P.chunk_bytes / (K * 2);
-  return r < 1 ? 1 : r;
-}
-
-// Mask of chunk barriers this tile uses (identical on every thread).
-__device__ __forceinline__ uint32_t staging_mask(const KParams& P, const Tile& T) {
-  if (T.op == OP_ATTN) {
-    if (T.a0 >= active_batch(P)) return 0;
-    AttnSpan s = attn_span(P, T);
-    return s.t1 > s.t0 ? 1u : 0u;
-  }
-  if (T.w_bytes == 0) return 0;
-  const int rpc = gemv_rows_per_chunk(P, T.a3);
-  const int n = (T.a1 + rpc - 1) / rpc;
-  return (n >= 32) ? 0xFFFFFFFFu : ((1u << n) - 1u);
-}
-
-__device__ void issue_staging(const KParams& P, const Tile& T, const Ctx& c) {
+// ---------------------------------------------------------------------------
+// Producer side: how a tile's staging data is cut into chunks, and the copies.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int* n_chunks, int* rpc) {
+  *rpc = 0;
+  *n_chunks = 0;
   if (T.op == OP_ATTN) {
     if (T.a0 >= active_batch(P)) return;
-    AttnSpan s = attn_span(P, T);
-    if (s.t1 <= s.t0) return;
+    const AttnSpan s = attn_span(P, T);
+    *n_chunks = s.t1 > s.t0 ? 1 : 0;
+    return;
+  }
+  if (T.w_bytes == 0) return;
+  int r = kStageBytes / (T.a3 * 2);
+  r &= ~1;  // even: RoPE and gate/up row pairs never straddle a chunk
+  *rpc = r < 2 ? 2 : r;
+  *n_chunks = (T.a1 + *rpc - 1) / *rpc;
+}
+
+// Copies of chunk `k` of tile T into `dst`; arms `bar` with their bytes.
+__device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uint8_t* dst, uint64_t* bar) {
+  if (T.op == OP_ATTN) {
+    const AttnSpan s = attn_span(P, T);
     const int page = P.page_tokens, hd = P.head_dim;
     const int p0 = s.t0 / page, p1 = (s.t1 - 1) / page;
     uint32_t total = 0;
-    for (int p = p0; p <= p1; ++p) total += 2u * (uint32_t)(min(page, s.t1 - p * page)) * hd * 2;
-    mbar_arrive_expect_tx(&c.bars[0], total);
+    for (int p = p0; p <= p1; ++p) total += 2u * (uint32_t)min(page, s.t1 - p * page) * hd * 2;
+    mbar_arrive_expect_tx(bar, total);
     const uint32_t vbase = (uint32_t)P.split_tokens * hd * 2;
     for (int p = p0; p <= p1; ++p) {
       const int rows = min(page, s.t1 - p * page);
       const int blk = P.block_table[s.b * P.max_blocks + p];
       const uint32_t bytes = (uint32_t)rows * hd * 2;
-      const uint32_t dst = (uint32_t)(p - p0) * page * hd * 2;
-      bulk_g2s(c.slot + dst, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, &c.bars[0]);
-      bulk_g2s(c.slot + vbase + dst, P.kv + kv_index(P, T.layer, blk, 1, s.g, 0), bytes, &c.bars[0]);
+      const uint32_t off = (uint32_t)(p - p0) * page * hd * 2;
+      bulk_g2s(dst + off, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, bar);
+      bulk_g2s(dst + vbase + off, P.kv + kv_index(P, T.layer, blk, 1, s.g, 0), bytes, bar);
     }
     return;
   }
-  if (T.w_bytes == 0) return;
-  const int row_bytes = T.a3 * 2;
-  const int rpc = gemv_rows_per_chunk(P, T.a3);
-  const uint8_t* src = P.weights + T.w_off;
-  for (int r0 = 0, ci = 0; r0 < T.a1; r0 += rpc, ++ci) {
-    const uint32_t bytes = (uint32_t)min(rpc, T.a1 - r0) * row_bytes;
-    mbar_arrive_expect_tx(&c.bars[ci], bytes);
-    bulk_g2s(c.slot + (size_t)r0 * row_bytes, src + (size_t)r0 * row_bytes, bytes, &c.bars[ci]);
-  }
+  const size_t row_bytes = (size_t)T.a3 * 2;
+  const int r0 = k * rpc;
+  const uint32_t bytes = (uint32_t)(min(rpc, T.a1 - r0) * row_bytes);
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_g2s(dst, P.weights + T.w_off + r0 * row_bytes, bytes, bar);
 }
 
 // ---------------------------------------------------------------------------
-// GEMV bodies (CUDA cores).  Weights: the tile's rows, row-major, in the slot.
-// Activations: fp32 [bg][K] staged in shared memory (RMSNorm fused when the
-// op consumes a normalised residual).  Work item = (row, 256-column segment);
-// lanes read 16 contiguous bytes each, so a warp reads 512 contiguous bytes.
+// GEMV (CUDA cores).  Work item = (row, 256-column segment): each lane reads
+// 16 contiguous bytes of the row (a warp reads 512 contiguous bytes) and the
+// matching activations from shared memory.
 // ---------------------------------------------------------------------------
 template <int BG>
-__device__ __forceinline__ void gemv_items(const uint8_t* slot, int K, int row_lo, int row_hi, const float* act,
-                                           float* out) {
+__device__ __forceinline__ void gemv_items(const uint8_t* chunk, int K, int rows, int row_base, const float* act,
+                                           float* out, int bg) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int segs = (K + 255) >> 8;
-  const int n_items = (row_hi - row_lo) * segs;
+  const int n_items = rows * segs;
   const size_t row_bytes = (size_t)K * 2;
   for (int it = warp; it < n_items; it += kWarps) {
-    const int row = row_lo + it / segs;
+    const int row = it / segs;
     const int k = (it % segs) * 256 + lane * 8;
     float acc[BG];
 #pragma unroll
     for (int b = 0; b < BG; ++b) acc[b] = 0.f;
     if (k < K) {
-      const uint4 w = *reinterpret_cast<const uint4*>(slot + row * row_bytes + (size_t)k * 2);
+      const uint4 w = *reinterpret_cast<const uint4*>(chunk + row * row_bytes + (size_t)k * 2);
       float wf[8];
       unpack8(w, wf);
 #pragma unroll
       for (int b = 0; b < BG; ++b) {
+        if (BG > 4 && b >= bg) break;
         const float4 a0 = *reinterpret_cast<const float4*>(act + b * K + k);
         const float4 a1 = *reinterpret_cast<const float4*>(act + b * K + k + 4);
         float s = wf[0] * a0.x;
@@ -222,60 +266,64 @@ __device__ __forceinline__ void gemv_items(const uint8_t* slot, int K, int row_l
     for (int b = 0; b < BG; ++b) acc[b] = warp_sum(acc[b]);
     if (lane == 0) {
 #pragma unroll
-      for (int b = 0; b < BG; ++b) atomicAdd(&out[row * 4 + b], acc[b]);
+      for (int b = 0; b < BG; ++b) atomicAdd(&out[(row_base + row) * kMaxGemvBatch + b], acc[b]);
     }
   }
 }
 
-// Copy bg rows of K floats (stride `stride`) into act; optionally RMS-normalise
-// each row and multiply by `gain` (which must cover the whole row: K = hidden).
+// Copy bg rows of K floats (row stride `stride`) into act; optionally
+// RMS-normalise each row and multiply by `gain` (then K is the whole row).
 __device__ void stage_act(const float* src, int stride, int K, int bg, const float* gain, float eps, float* act) {
-  __shared__ float red[kWarps][4];
-  float ss[4] = {0.f, 0.f, 0.f, 0.f};
+  __shared__ float red[kWarps][kMaxGemvBatch];
+  __shared__ float scale_s[kMaxGemvBatch];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int b = 0; b < bg; ++b) {
+    float ss = 0.f;
     for (int k = threadIdx.x * 4; k < K; k += kThreads * 4) {
       const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * stride + k));
       *reinterpret_cast<float4*>(act + b * K + k) = v;
-      ss[b] += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    if (gain) {
+      ss = warp_sum(ss);
+      if (lane == 0) red[warp][b] = ss;
     }
   }
   if (gain) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int b = 0; b < bg; ++b) {
-      float v = warp_sum(ss[b]);
-      if (lane == 0) red[warp][b] = v;
-    }
-    __syncthreads();
-    float scale[4];
-    for (int b = 0; b < bg; ++b) {
+    cbar();
+    if (threadIdx.x < bg) {
       float tot = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) tot += red[w][b];
-      scale[b] = 1.0f / sqrtf(tot / (float)K + eps);
+      for (int w = 0; w < kWarps; ++w) tot += red[w][threadIdx.x];
+      scale_s[threadIdx.x] = 1.0f / sqrtf(tot / (float)K + eps);
     }
-    for (int b = 0; b < bg; ++b)
+    cbar();
+    for (int b = 0; b < bg; ++b) {
+      const float sc = scale_s[b];
       for (int k = threadIdx.x * 4; k < K; k += kThreads * 4) {
         float4* a = reinterpret_cast<float4*>(act + b * K + k);
         const float4 gg = __ldg(reinterpret_cast<const float4*>(gain + k));
         float4 v = *a;
-        v.x *= scale[b] * gg.x;
-        v.y *= scale[b] * gg.y;
-        v.z *= scale[b] * gg.z;
-        v.w *= scale[b] * gg.w;
+        v.x *= sc * gg.x;
+        v.y *= sc * gg.y;
+        v.z *= sc * gg.z;
+        v.w *= sc * gg.w;
         *a = v;
       }
+    }
   }
-  __syncthreads();
+  cbar();
 }
 
 __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int b0, int bg) {
   const int r0 = T.a0, R = T.a1, hd = P.head_dim, half = hd / 2;
+  constexpr int S = kMaxGemvBatch;
   switch (T.op) {
     case OP_QKV: {
       for (int idx = threadIdx.x; idx < (R / 2) * bg; idx += kThreads) {
         const int pr = idx % (R / 2), b = idx / (R / 2), bi = b0 + b;
         const int r = r0 + 2 * pr;
-        const float y0 = out[(2 * pr) * 4 + b], y1 = out[(2 * pr + 1) * 4 + b];
+        const float y0 = out[(2 * pr) * S + b], y1 = out[(2 * pr + 1) * S + b];
         const int pos = P.seqlen[bi];
         if (r < P.q_rows + P.kv_rows) {
           const bool is_q = r < P.q_rows;
@@ -309,7 +357,7 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
       for (int idx = threadIdx.x; idx < R * bg; idx += kThreads) {
         const int rr = idx % R, b = idx / R, bi = b0 + b;
         const size_t o = (size_t)bi * P.hidden + r0 + rr;
-        const float x = __ldcg(P.xa + o) + out[rr * 4 + b];
+        const float x = __ldcg(P.xa + o) + out[rr * S + b];
         P.xb[o] = x;
         P.xa[o] = x;
       }
@@ -318,7 +366,7 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
     case OP_GU: {
       for (int idx = threadIdx.x; idx < (R / 2) * bg; idx += kThreads) {
         const int pr = idx % (R / 2), b = idx / (R / 2), bi = b0 + b;
-        const float g = out[(2 * pr) * 4 + b], u = out[(2 * pr + 1) * 4 + b];
+        const float g = out[(2 * pr) * S + b], u = out[(2 * pr + 1) * S + b];
         P.hbuf[(size_t)bi * P.ffn + r0 / 2 + pr] = g / (1.0f + expf(-g)) * u;
       }
       break;
@@ -326,7 +374,7 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
     case OP_DOWN: {
       for (int idx = threadIdx.x; idx < R * bg; idx += kThreads) {
         const int rr = idx % R, b = idx / R, bi = b0 + b;
-        atomicAdd(P.xa + (size_t)bi * P.hidden + r0 + rr, out[rr * 4 + b]);
+        atomicAdd(P.xa + (size_t)bi * P.hidden + r0 + rr, out[rr * S + b]);
       }
       break;
     }
@@ -334,14 +382,14 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
       if (P.logits)
         for (int idx = threadIdx.x; idx < R * bg; idx += kThreads) {
           const int rr = idx % R, b = idx / R, bi = b0 + b;
-          P.logits[(size_t)bi * P.vocab + r0 + rr] = out[rr * 4 + b];
+          P.logits[(size_t)bi * P.vocab + r0 + rr] = out[rr * S + b];
         }
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
       if (warp < bg) {
         float bv = -INFINITY;
         int bidx = 0x7FFFFFFF;
         for (int rr = lane; rr < R; rr += 32) {
-          const float v = out[rr * 4 + warp];
+          const float v = out[rr * S + warp];
           if (v > bv) { bv = v; bidx = r0 + rr; }
         }
 #pragma unroll
@@ -364,26 +412,23 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
   }
 }
 
-template <int BG>
-__device__ void gemv_group(const KParams& P, const Tile& T, const Ctx& c, int b0, bool first, uint32_t phase,
-                           bool* ok) {
-  const int K = T.a3, R = T.a1;
-  const int rpc = gemv_rows_per_chunk(P, K);
-  for (int i = threadIdx.x; i < R * 4; i += kThreads) c.out[i] = 0.f;
-  __syncthreads();
-  for (int r0 = 0, ci = 0; r0 < R; r0 += rpc, ++ci) {
-    if (first && !wait_bar(P, &c.bars[ci], (phase >> ci) & 1u, T.a0)) *ok = false;
-    if (!__syncthreads_and(*ok)) {
-      *ok = false;
-      return;
-    }
-    gemv_items<BG>(c.slot, K, r0, min(R, r0 + rpc), c.act, c.out);
-  }
-  __syncthreads();
-}
+// Consumer-side chunk cursor: chunk c lives in stage c % n_stages and is the
+// (c / n_stages)-th use of that stage.
+struct Cursor {
+  uint32_t c;
+};
 
-__device__ bool body_gemv(const KParams& P, const Tile& T, const Ctx& c, uint32_t phase) {
-  const int K = T.a3;
+struct ConsumerState {
+  int act_key;      // (op, layer, k0) of the staged activation, or kNoAct
+  uint32_t last_ctr;  // counter known satisfied in this launch
+};
+
+__device__ __forceinline__ int act_key_of(const Tile& T) { return (int)T.op | ((int)T.layer << 4) | (T.a2 << 12); }
+
+// GEMV tile body.  Returns false on a wait failure.
+__device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks, int rpc,
+                          ConsumerState& cs, volatile int* abort) {
+  const int K = T.a3, R = T.a1;
   const int nb = active_batch(P);
   const LayerDev* L = P.layers + (T.op == OP_LMHEAD ? 0 : T.layer);
   const float* gain = nullptr;
@@ -396,41 +441,73 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Ctx& c, uint32_
     case OP_DOWN: src = P.hbuf + T.a2; stride = P.ffn; break;
     case OP_LMHEAD: gain = reinterpret_cast<const float*>(P.weights + P.final_norm_off); src = P.xa; stride = P.hidden; break;
   }
-  int bgmax = kActBytes / (K * 4);
-  if (bgmax > 4) bgmax = 4;
-  bool ok = true;
-  for (int b0 = 0; b0 < nb; b0 += bgmax) {
-    const int bg = min(bgmax, nb - b0);
-    stage_act(src + (size_t)b0 * stride, stride, K, bg, gain, P.eps, c.act);
-    const bool first = (b0 == 0);
-    switch (bg) {
-      case 1: gemv_group<1>(P, T, c, b0, first, phase, &ok); break;
-      case 2: gemv_group<2>(P, T, c, b0, first, phase, &ok); break;
-      case 3: gemv_group<3>(P, T, c, b0, first, phase, &ok); break;
-      default: gemv_group<4>(P, T, c, b0, first, phase, &ok); break;
+  int bgmax = P.act_bytes / (K * 4);
+  if (bgmax > kMaxGemvBatch) bgmax = kMaxGemvBatch;
+  const bool one_group = nb <= bgmax;
+  if (one_group) {
+    const int key = act_key_of(T);
+    if (cs.act_key != key) {
+      stage_act(src, stride, K, nb, gain, P.eps, S.act);
+      cs.act_key = key;
     }
-    if (!ok) return false;
-    epilogue(P, T, c.out, b0, bg);
-    __syncthreads();
+  } else {
+    cs.act_key = kNoAct;
   }
-  if (nb == 0) {  // nothing to compute, but the staged chunks must still land
-    const int rpc = gemv_rows_per_chunk(P, K);
-    for (int r0 = 0, ci = 0; r0 < T.a1; r0 += rpc, ++ci)
-      if (!wait_bar(P, &c.bars[ci], (phase >> ci) & 1u, T.a0)) ok = false;
-    ok = __syncthreads_and(ok);
+  for (int i = threadIdx.x; i < R * kMaxGemvBatch; i += kThreads) S.out[i] = 0.f;
+  cbar();
+  bool ok = true;
+  for (int k = 0; k < n_chunks; ++k, ++cur.c) {
+    const int s = cur.c % P.n_stages;
+    const uint32_t par = (cur.c / P.n_stages) & 1u;
+    if (!wait_phase(P, &S.full[s], par, abort, T.a0)) ok = false;
+    if (!cbar_and(ok)) return false;
+    const uint8_t* chunk = S.ring + (size_t)s * kStageBytes;
+    const int r0 = k * rpc, rows = min(rpc, R - r0);
+    for (int b0 = 0; b0 < nb; b0 += bgmax) {
+      const int bg = min(bgmax, nb - b0);
+      if (!one_group) stage_act(src + (size_t)b0 * stride, stride, K, bg, gain, P.eps, S.act);
+      float* out = S.out + (one_group ? 0 : 0);
+      // outputs of token b0+b accumulate at column b (one group) or are
+      // flushed per group below
+      switch (bg) {
+        case 1: gemv_items<1>(chunk, K, rows, r0, S.act, out, bg); break;
+        case 2: gemv_items<2>(chunk, K, rows, r0, S.act, out, bg); break;
+        case 3: gemv_items<3>(chunk, K, rows, r0, S.act, out, bg); break;
+        case 4: gemv_items<4>(chunk, K, rows, r0, S.act, out, bg); break;
+        default: gemv_items<8>(chunk, K, rows, r0, S.act, out, bg); break;
+      }
+      if (!one_group) {
+        cbar();
+        // epilogue of these rows for this token group, then clear them
+        Tile Tc = T;
+        Tc.a0 = T.a0 + r0;
+        Tc.a1 = rows;
+        epilogue(P, Tc, out + r0 * kMaxGemvBatch, b0, bg);
+        cbar();
+        for (int i = threadIdx.x; i < rows * kMaxGemvBatch; i += kThreads) out[r0 * kMaxGemvBatch + i] = 0.f;
+        cbar();
+      }
+    }
+    cbar();
+    if (threadIdx.x == 0) mbar_arrive(&S.empty[s]);
   }
+  if (one_group) {
+    epilogue(P, T, S.out, 0, nb);
+  }
+  cbar();
   return ok;
 }
 
 // ---------------------------------------------------------------------------
-// Split-KV GQA decode attention.  The tile (b, g, j) handles the `group` query
-// heads of kv head g over tokens [j*S, (j+1)*S) of sequence b, writes an
-// online-softmax partial (m, l, o), and the last split to arrive combines all
-// partials of (b, g) ("Persistent threads and megakernels", §6: split long
-// histories into chunks, then combine partial attention with a reduction
-// signalled through global memory).
+// Split-KV GQA decode attention.  The tile (b, g, j) handles the `group`
+// query heads of kv head g over tokens [j*S, (j+1)*S) of sequence b, writes
+// an online-softmax partial (m, l, o), and the last split to arrive combines
+// all partials of (b, g) ("Persistent threads and megakernels", §6: split long
+// histories into chunks, combine partial attention in a reduction signalled
+// through global memory).
 // ---------------------------------------------------------------------------
-__device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_t phase) {
+__device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cursor& cur, int n_chunks,
+                          volatile int* abort) {
   if (T.a0 >= active_batch(P)) return true;
   __shared__ int s_last;
   __shared__ float s_m[kMaxGroup], s_l[kMaxGroup];
@@ -438,29 +515,32 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_
   const int hd = P.head_dim, grp = P.group, S = P.split_tokens;
   const int n = s.t1 - s.t0;
   float* part = P.part + ((((size_t)s.b * P.n_kv + s.g) * P.n_splits + s.j) * grp) * (2 + hd);
-  const uint16_t* Ks = reinterpret_cast<const uint16_t*>(c.slot);
-  const uint16_t* Vs = reinterpret_cast<const uint16_t*>(c.slot + (size_t)S * hd * 2);
-  float* q_s = c.act;                 // [grp][hd]
-  float* p_s = c.act + kMaxGroup * hd;  // [grp][S]
-  if (n > 0) {
-    bool ok = wait_bar(P, &c.bars[0], phase & 1u, 0xFFFFFFFFu);
-    if (!__syncthreads_and(ok)) return false;
+  float* q_s = Sh.act;                    // [grp][hd]
+  float* p_s = Sh.act + kMaxGroup * hd;   // [grp][S]
+  if (n_chunks > 0) {
+    const int st = cur.c % P.n_stages;
+    const uint32_t par = (cur.c / P.n_stages) & 1u;
+    bool ok = wait_phase(P, &Sh.full[st], par, abort, 0xFFFFFFFFu);
+    if (!cbar_and(ok)) return false;
+    uint8_t* stage = Sh.ring + (size_t)st * kStageBytes;
+    const uint16_t* Ks = reinterpret_cast<const uint16_t*>(stage);
+    const uint16_t* Vs = reinterpret_cast<const uint16_t*>(stage + (size_t)S * hd * 2);
     // the current token's row was written this step, after the copy was issued
     if (s.pos >= s.t0 && s.pos < s.t1) {
       const int blk = P.block_table[s.b * P.max_blocks + s.pos / P.page_tokens];
       const int row = s.pos - s.t0;
-      const int lanes = hd * 2 / 16;  // 16-byte pieces per row
+      const int lanes = hd * 2 / 16;
       if (threadIdx.x < 2 * lanes) {
         const int sel = threadIdx.x / lanes, piece = threadIdx.x % lanes;
         const uint4* src = reinterpret_cast<const uint4*>(
             P.kv + kv_index(P, T.layer, blk, sel, s.g, s.pos % P.page_tokens));
-        uint8_t* dst = c.slot + (size_t)sel * S * hd * 2 + (size_t)row * hd * 2;
+        uint8_t* dst = stage + (size_t)sel * S * hd * 2 + (size_t)row * hd * 2;
         reinterpret_cast<uint4*>(dst)[piece] = __ldcg(src + piece);
       }
     }
     for (int i = threadIdx.x; i < grp * hd; i += kThreads)
       q_s[i] = __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * grp * hd + i);
-    __syncthreads();
+    cbar();
     const float scale = 1.0f / sqrtf((float)hd);
     const int words = hd / 2;
     for (int idx = threadIdx.x; idx < grp * n; idx += kThreads) {
@@ -476,7 +556,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_
       }
       p_s[hh * S + t] = acc * scale;
     }
-    __syncthreads();
+    cbar();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < grp) {
       float m = -INFINITY;
@@ -491,7 +571,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_
       l = warp_sum(l);
       if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
     }
-    __syncthreads();
+    cbar();
     for (int idx = threadIdx.x; idx < grp * hd; idx += kThreads) {
       const int hh = idx / hd, d = idx % hd;
       float o = 0.f;
@@ -500,13 +580,16 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_
       pr[2 + d] = o;
       if (d == 0) { pr[0] = s_m[hh]; pr[1] = s_l[hh]; }
     }
+    cbar();
+    if (threadIdx.x == 0) mbar_arrive(&Sh.empty[st]);
+    ++cur.c;
   } else {
     for (int idx = threadIdx.x; idx < grp * (2 + hd); idx += kThreads) {
       const int k = idx % (2 + hd);
       part[idx] = (k == 0) ? -INFINITY : 0.f;
     }
   }
-  __syncthreads();
+  cbar();
   uint32_t* arr = P.arrive + (size_t)s.b * P.n_kv + s.g;
   if (threadIdx.x == 0) {
     __threadfence();
@@ -514,7 +597,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_
     s_last = (old == (uint32_t)P.n_splits - 1u);
     __threadfence();
   }
-  __syncthreads();
+  cbar();
   if (s_last) {
     const float* base = P.part + (((size_t)s.b * P.n_kv + s.g) * P.n_splits) * grp * (2 + hd);
     for (int idx = threadIdx.x; idx < grp * hd; idx += kThreads) {
@@ -535,7 +618,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Ctx& c, uint32_
   return true;
 }
 
-__device__ bool body_embed(const KParams& P, const Tile& T) {
+__device__ bool body_embed(const KParams& P) {
   const int nb = active_batch(P);
   const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
   for (int b = 0; b < nb; ++b) {
@@ -569,27 +652,9 @@ __device__ bool body_final(const KParams& P) {
   return true;
 }
 
-__device__ __forceinline__ bool run_body(const KParams& P, const Tile& T, const Ctx& c, uint32_t phase) {
-  switch (T.op) {
-    case OP_EMBED: return body_embed(P, T);
-    case OP_ATTN: return body_attn(P, T, c, phase);
-    case OP_FINAL: return body_final(P);
-    default: return body_gemv(P, T, c, phase);
-  }
-}
-
-__device__ void drain(const KParams& P, const Ctx& c, uint32_t used, uint32_t phase) {
-  if (threadIdx.x != 0) return;
-  for (int i = 0; i < kMaxChunks; ++i)
-    if ((used >> i) & 1u) {
-      const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&c.bars[i], (phase >> i) & 1u))
-        if (globaltimer() - t0 > P.timeout_ns) break;
-    }
-}
-
-// Thread 0: bounded acquire-wait until the tile's counter reaches need x epoch.
-__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile) {
+// Thread 0 of the consumers: bounded acquire-wait until the tile's counter
+// reaches need x epoch.
+__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, volatile int* abort) {
   if (ld_volatile_s32(&P.err->code) != 0) return false;
   if (T.wait_ctr == kNoCounter) return true;
   const uint32_t target = T.need * P.epoch;
@@ -601,7 +666,7 @@ __device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile) {
     v = ld_acquire_u32(ctr);
     if ((int32_t)(v - target) >= 0) return true;
     if ((it & 15) == 0) {
-      if (ld_volatile_s32(&P.err->code) != 0) return false;
+      if (*abort || ld_volatile_s32(&P.err->code) != 0) return false;
       if (globaltimer() - t0 > P.timeout_ns) {
         record_error(P, WPK_ERR_TIMEOUT, tile, T.wait_ctr, v, target);
         return false;
@@ -610,97 +675,174 @@ __device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// The worker: producer warp (warp 8) + consumer warps (0..7).
+// ---------------------------------------------------------------------------
+__device__ void worker(const KParams& P, uint8_t* smem_raw) {
+  const Shared S = carve(smem_raw, P);
+  __shared__ volatile int s_abort;
+  __shared__ uint32_t s_prod_chunks;  // chunks the producer issued
+  __shared__ uint32_t s_cons_chunks;  // chunks the consumers finished
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < P.n_stages; ++i) {
+      mbar_init(&S.full[i], 1);
+      mbar_init(&S.empty[i], 1);
+    }
+    for (int i = 0; i < kMaxQueue; ++i) {
+      mbar_init(&S.tq_full[i], 1);
+      mbar_init(&S.tq_empty[i], 1);
+    }
+    fence_mbar_init();
+    s_abort = 0;
+    s_prod_chunks = 0;
+    s_cons_chunks = 0;
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // ------------------------------------------------------------ producer
+    if ((threadIdx.x & 31) == 0) {
+      uint32_t c = 0;  // chunks issued
+      const int Q = P.per_op ? 1 : P.lookahead;
+      for (uint32_t i = 0;; ++i) {
+        const int slot = i % Q;
+        if (i >= (uint32_t)Q && !wait_phase(P, &S.tq_empty[slot], ((i / Q) - 1) & 1u, &s_abort, 0xFFFFFFFFu)) break;
+        uint32_t t;
+        if (P.per_op)
+          t = (i == 0) ? P.t_begin + blockIdx.x : P.t_end;
+        else
+          t = P.t_begin + atomicAdd(&P.head[P.region], 1u);
+        TQEntry& e = S.tq[slot];
+        if (t >= P.t_end) {
+          e.valid = 0;
+          mbar_arrive(&S.tq_full[slot]);
+          break;
+        }
+        e.tile = P.tiles[t];
+        e.ticket = t;
+        e.valid = 1;
+        int nch, rpc;
+        tile_chunks(P, e.tile, &nch, &rpc);
+        e.n_chunks = nch;
+        e.rows_per_chunk = rpc;
+        e.ev_issue = P.trace ? atomicAdd(P.evclock, 1u) : 0u;
+        const Tile T = e.tile;
+        mbar_arrive(&S.tq_full[slot]);
+        bool stop = false;
+        for (int k = 0; k < nch; ++k, ++c) {
+          const int s = c % P.n_stages;
+          const uint32_t use = c / P.n_stages;
+          if (use >= 1 && !wait_phase(P, &S.empty[s], (use - 1) & 1u, &s_abort, t)) {
+            stop = true;
+            break;
+          }
+          fence_proxy_async_smem();
+          issue_chunk(P, T, k, rpc, S.ring + (size_t)s * kStageBytes, &S.full[s]);
+        }
+        s_prod_chunks = c;
+        if (stop) break;
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- consumers
+    Cursor cur{0};
+    ConsumerState cs{kNoAct, kNoCounter};
+    const int Q = P.per_op ? 1 : P.lookahead;
+    __shared__ int s_fail;
+    for (uint32_t i = 0;; ++i) {
+      const int slot = i % Q;
+      if (!wait_phase(P, &S.tq_full[slot], (i / Q) & 1u, &s_abort, 0xFFFFFFFFu)) break;
+      const TQEntry& e = S.tq[slot];
+      if (!e.valid) break;
+      const Tile T = e.tile;
+      const uint32_t t = e.ticket;
+      const int n_chunks = e.n_chunks, rpc = e.rows_per_chunk;
+      uint32_t ev_start = 0;
+      uint64_t t_start = 0;
+      if (threadIdx.x == 0) {
+        bool ok = true;
+        if (!P.per_op && T.wait_ctr != cs.last_ctr) {
+          ok = wait_counter(P, T, t, &s_abort);
+          if (ok) cs.last_ctr = T.wait_ctr;
+        } else if (ld_volatile_s32(&P.err->code) != 0) {
+          ok = false;
+        }
+        s_fail = ok ? 0 : 1;
+        if (P.trace) {
+          t_start = globaltimer();
+          if (ok) ev_start = atomicAdd(P.evclock, 1u);
+        }
+      }
+      cbar();
+      bool ok = !s_fail;
+      if (ok) {
+        switch (T.op) {
+          case OP_EMBED: ok = body_embed(P); break;
+          case OP_ATTN: ok = body_attn(P, T, S, cur, n_chunks, &s_abort); break;
+          case OP_FINAL: ok = body_final(P); break;
+          default: ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort); break;
+        }
+        // attention tiles use the activation buffer as scratch
+        if (T.op == OP_ATTN) cs.act_key = kNoAct;
+      }
+      ok = cbar_and(ok);
+      if (!ok) {
+        if (threadIdx.x == 0) s_abort = 1;
+        break;
+      }
+      if (threadIdx.x == 0) {
+        if (P.trace && !P.per_op) {
+          TraceRec r;
+          r.tile = t;
+          r.worker = (uint16_t)blockIdx.x;
+          r.op = T.op;
+          r.ev_issue = e.ev_issue;
+          r.ev_start = ev_start;
+          r.ev_done = atomicAdd(P.evclock, 1u);
+          r.epoch = P.epoch;
+          r.t_start_ns = t_start;
+          r.t_end_ns = globaltimer();
+          P.trace_buf[t] = r;
+        }
+        if (!P.per_op)
+          for (uint32_t k = 0; k < T.sig_cnt; ++k) red_release_add_u32(P.ctr + P.sig[T.sig_off + k], 1u);
+        mbar_arrive(&S.tq_empty[slot]);
+      }
+    }
+    if (threadIdx.x == 0) s_cons_chunks = cur.c;
+  }
+  __syncthreads();
+  // Drain: wait (bounded) for chunks issued but never consumed.
+  if (threadIdx.x == 0) {
+    for (uint32_t c = s_cons_chunks; c < s_prod_chunks; ++c) {
+      const int s = c % P.n_stages;
+      const uint32_t par = (c / P.n_stages) & 1u;
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&S.full[s], par))
+        if (globaltimer() - t0 > P.timeout_ns) break;
+    }
+  }
+}
+
 }  // namespace
 
-// ---------------------------------------------------------------------------
-// The persistent worker grid (one launch per region per step).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 2) wpk_persistent_kernel(const KParams P) {
+// The persistent worker grid (one cooperative launch per region per step).
+__global__ void __launch_bounds__(kCtaThreads, 1) wpk_persistent_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const Ctx c = carve(smem_raw, P.slot_bytes);
-  __shared__ uint32_t s_tk[2];
-  __shared__ int s_fail;
-  __shared__ uint32_t s_ev_issue;
-  __shared__ uint64_t s_t_start;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxChunks; ++i) mbar_init(&c.bars[i], 1);
-    fence_mbar_init();
-    s_tk[0] = P.t_begin + atomicAdd(&P.head[P.region], 1u);
-  }
-  __syncthreads();
-  uint32_t phase = 0;
-  for (;;) {
-    const uint32_t t = s_tk[0];
-    if (t >= P.t_end) break;
-    const Tile T = P.tiles[t];
-    const uint32_t used = staging_mask(P, T);
-    if (threadIdx.x == 0) {
-      fence_proxy_async_smem();
-      issue_staging(P, T, c);
-      if (P.trace) s_ev_issue = atomicAdd(P.evclock, 1u);
-      s_tk[1] = P.t_begin + atomicAdd(&P.head[P.region], 1u);  // claim the next ticket early
-      s_fail = wait_counter(P, T, t) ? 0 : 1;
-      if (P.trace) s_t_start = globaltimer();
-    }
-    __syncthreads();
-    uint32_t ev_start = 0;
-    if (P.trace && threadIdx.x == 0 && !s_fail) ev_start = atomicAdd(P.evclock, 1u);
-    bool ok = !s_fail;
-    if (ok) ok = run_body(P, T, c, phase);
-    ok = __syncthreads_and(ok);
-    if (!ok) {
-      drain(P, c, used, phase);
-      break;
-    }
-    phase ^= used;
-    if (threadIdx.x == 0) {
-      if (P.trace) {
-        TraceRec r;
-        r.tile = t;
-        r.worker = (uint16_t)blockIdx.x;
-        r.op = T.op;
-        r.ev_issue = s_ev_issue;
-        r.ev_start = ev_start;
-        r.ev_done = atomicAdd(P.evclock, 1u);
-        r.epoch = P.epoch;
-        r.t_start_ns = s_t_start;
-        r.t_end_ns = globaltimer();
-        P.trace_buf[t] = r;
-      }
-      __threadfence();
-      for (uint32_t i = 0; i < T.sig_cnt; ++i) red_release_add_u32(P.ctr + P.sig[T.sig_off + i], 1u);
-      s_tk[0] = s_tk[1];
-    }
-    __syncthreads();
-  }
+  worker(P, smem_raw);
 }
 
-// ---------------------------------------------------------------------------
 // Per-op launch: one CTA per tile of one op group; stream order replaces the
 // counters.  Used for the CUDA-Graph comparator.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 2) wpk_per_op_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const Ctx c = carve(smem_raw, P.slot_bytes);
-  const uint32_t t = P.t_begin + blockIdx.x;
-  if (t >= P.t_end) return;
-  const Tile T = P.tiles[t];
-  const uint32_t used = staging_mask(P, T);
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxChunks; ++i) mbar_init(&c.bars[i], 1);
-    fence_mbar_init();
-    issue_staging(P, T, c);
-  }
-  __syncthreads();
-  bool ok = ld_volatile_s32(&P.err->code) == 0;
-  ok = __syncthreads_and(ok);
-  if (ok) ok = run_body(P, T, c, 0u);
-  ok = __syncthreads_and(ok);
-  if (!ok) drain(P, c, used, 0u);
+  worker(P, smem_raw);
 }
 
-size_t worker_smem_bytes(int slot_bytes) {
-  return (size_t)slot_bytes + kActBytes + kOutFloats * 4 + kMaxChunks * 8;
+size_t worker_smem_bytes(int n_stages, int act_bytes) {
+  return (size_t)n_stages * kStageBytes + act_bytes + kOutFloats * 4 + kMaxQueue * sizeof(TQEntry) +
+         (2 * kMaxStages + 2 * kMaxQueue) * 8;
 }
 
 const void* persistent_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_persistent_kernel); }

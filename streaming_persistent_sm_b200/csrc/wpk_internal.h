@@ -9,11 +9,16 @@
 namespace wpk {
 
 constexpr uint32_t kNoCounter = 0xFFFFFFFFu;
-constexpr int kThreads = 256;          // threads per worker CTA
+constexpr int kThreads = 256;          // consumer (compute) threads per worker CTA
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxChunks = 8;          // mbarriers per staging slot
-constexpr int kActBytes = 32768;       // activation staging (fp32) per worker
+constexpr int kCtaThreads = kThreads + 32;  // + one producer warp
+constexpr int kStageBytes = 16384;     // one chunk stage of the staging ring
+constexpr int kMaxStages = 13;         // ring stages per worker
+constexpr int kMaxQueue = 8;           // tiles a worker may hold (lookahead)
+constexpr int kMaxGemvBatch = 8;       // token rows per GEMV pass
+constexpr int kMaxTileRows = 128;      // rows per GEMV tile (partial-output buffer)
 constexpr int kMaxGroup = 8;           // q heads per kv head handled by one attention tile
+constexpr int kMaxSmem = 232448;       // dynamic shared memory per CTA on sm_100
 
 // Op codes of the tiles.  One "op group" = the tiles of one op of one layer.
 enum Op : uint16_t {
@@ -74,7 +79,7 @@ struct KParams {
   float eps;
   // plan
   int max_batch, max_context, page_tokens, max_blocks, split_tokens, n_splits;
-  int slot_bytes, chunk_bytes;
+  int n_stages, lookahead, act_bytes;
   uint64_t timeout_ns;
   int trace;
   // device buffers (weights image and KV are caller-owned)
@@ -116,6 +121,7 @@ struct KParams {
   uint32_t t_begin, t_end;   // ticket range of this launch
   uint32_t epoch;            // counter target multiplier (>= 1)
   int region;
+  int per_op;                // 1: one tile per CTA, no queue, no counters
 };
 
 // Host-side compiled graph.

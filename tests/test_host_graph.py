@@ -44,8 +44,9 @@ def test_tiny_graph_verifies_and_counters_dedup(lib):
         assert ops[0] == 0 and ops[-1] == 7  # embed first, final last
         # per layer: 1 QKV + one per kv head + O + gate/up + one per down K-chunk
         assert st["n_counters"] == synth.TINY.n_layers * (4 + synth.TINY.n_kv_heads) + 2
-        # every tile but the last signals exactly one counter
-        assert st["n_signals"] == st["n_tiles"] - 1
+        # every tile but the last signals at least one counter (a k/v tile that
+        # covers several kv heads signals each head's attention counter)
+        assert st["n_signals"] >= st["n_tiles"] - 1
         assert st["weight_bytes"] == sum(np.prod(s) * 2 for n, s, k in synth.tensor_specs(synth.TINY) if k == "normal")
         edges = W.wpk_get_edges(h)
         assert np.all(edges[:, 0] < edges[:, 1])  # ticket order is topological
@@ -54,8 +55,8 @@ def test_tiny_graph_verifies_and_counters_dedup(lib):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(max_batch=3, max_context=200, split_pages=2),
-    dict(max_batch=2, max_context=130, page_tokens=32, tile_bytes=4096, slot_bytes=16384),
+    dict(max_batch=3, max_context=200, split_pages=2, page_tokens=32),
+    dict(max_batch=2, max_context=130, page_tokens=32, tile_bytes=4096, slot_bytes=16384, lookahead=1),
     dict(max_batch=1, max_context=64, n_regions=3, region_cut=(0, 1, 2, 0)),
 ])
 def test_graph_variants_verify(lib, kw):

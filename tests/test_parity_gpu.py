@@ -32,10 +32,11 @@ def _prompts(B, T, seed=synth.WORKLOADS["tiny"].prompt_seed):
 
 PLANS = {
     "megakernel": dict(),
-    "megakernel_1wps": dict(workers_per_sm=1),
+    "fewer_workers": dict(n_workers=37),
     "regions3": dict(n_regions=3, region_cut=(0, 1, 2, 0)),
     "per_op_graph": dict(mode=W.WPK_PER_OP_GRAPH),
-    "small_tiles": dict(tile_bytes=4096, slot_bytes=16384),
+    "small_tiles_one_slot": dict(tile_bytes=4096, slot_bytes=16384, lookahead=1),
+    "two_stage_ring": dict(slot_bytes=32768, lookahead=2),
     "split2_page32": dict(page_tokens=32, split_pages=2),
 }
 
