@@ -232,6 +232,28 @@ const char *wpk_last_error(const wpk_handle *h);
 /* Stop the resident grid (if any), release library-owned tables, free h. */
 int wpk_destroy(wpk_handle *h);
 
+/* One decode step like wpk_step (megakernel mode only), for callers that
+ * cannot allocate device memory when they step the model: a host application
+ * that owns the whole device pool and gives plugins no allocator, or a
+ * real-time loop that must never enter an allocator.  It allocates nothing
+ * (no cudaMalloc/cudaFree, no allocating library call): the activation
+ * scratch comes from a static 8 MiB device array inside the library instead
+ * of the buffer bound by wpk_load_weights.  The paper has no counterpart;
+ * this entry point exists for those callers only.
+ *   - Every GPU that loads the library holds the 8 MiB until process exit.
+ *   - Plans needing more scratch than 8 MiB (wpk_workspace_size) get
+ *     WPK_ERR_SHAPE; the per-op graph mode gets WPK_ERR_UNSUPPORTED.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     no part of it needs to start at zero (each step writes every scratch
+ *     value before reading it).  Calls that overlap on the GPU, from any
+ *     handle or stream, race on it.
+ * Inputs, outputs and errors are those of wpk_step. */
+int wpk_step_noalloc(wpk_handle *h, const int32_t *in_tok_dev, int32_t *out_tok_dev, float *logits_dev,
+                     void *stream);
+
 /* Test hook: make counter `counter` need one more signal than it can ever get
  * (an unsatisfiable dependency), so the next step's device wait must time out
  * and return WPK_ERR_TIMEOUT.  Host-side fault injection; no GPU fault. */

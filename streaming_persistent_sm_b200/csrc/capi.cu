@@ -538,6 +538,32 @@ int wpk_destroy(wpk_handle* h) {
   return WPK_OK;
 }
 
+// Step with a different scratch buffer (used by wpk_step_noalloc).  The
+// megakernel reads the scratch address at every launch, so swapping it for one
+// call changes nothing else; the per-op mode bakes addresses into a captured
+// graph (and instantiating one may allocate), so it is not offered there.
+int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes, const int32_t* in_tok_dev,
+                              int32_t* out_tok_dev, float* logits_dev, void* stream) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (h->g.plan.mode != WPK_MEGAKERNEL)
+    return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the megakernel mode");
+  if (h->scratch_bytes > scratch_bytes)
+    return fail(h, WPK_ERR_SHAPE, "the plan needs " + std::to_string(h->scratch_bytes) +
+                                      " scratch bytes, more than the " + std::to_string(scratch_bytes) +
+                                      " bytes of the static scratch array");
+  if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");
+  int dev = -1;
+  CUDA_TRY(h, cudaGetDevice(&dev));
+  if (dev != h->device) return fail(h, WPK_ERR_INVALID_ARG, "current device is not the handle's device");
+  if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  uint8_t* saved = h->scratch;
+  h->scratch = static_cast<uint8_t*>(scratch);
+  rc = step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, static_cast<cudaStream_t>(stream));
+  h->scratch = saved;
+  return rc;
+}
+
 int wpk_debug_break_counter(wpk_handle* h, int counter) {
   if (!h || counter < 0 || counter >= (int)h->g.ctr_need.size()) return WPK_ERR_INVALID_ARG;
   for (auto& t : h->g.tiles)

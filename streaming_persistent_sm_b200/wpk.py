@@ -99,6 +99,7 @@ _SIGS = {
     "wpk_last_error": (C.c_char_p, [_H]),
     "wpk_destroy": (C.c_int, [_H]),
     "wpk_debug_break_counter": (C.c_int, [_H, C.c_int]),
+    "wpk_step_noalloc": (C.c_int, [_H, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
 }
 
 _lib = None
@@ -170,6 +171,12 @@ def wpk_prefill(h, tokens_dev: int, batch: int, prompt_len: int, first_tok_dev: 
 
 def wpk_step(h, in_tok_dev: int = 0, out_tok_dev: int = 0, logits_dev: int = 0, stream: int = 0):
     _check(load_library().wpk_step(h, in_tok_dev or None, out_tok_dev or None, logits_dev or None, stream or None), h)
+
+
+def wpk_step_noalloc(h, in_tok_dev: int = 0, out_tok_dev: int = 0, logits_dev: int = 0, stream: int = 0):
+    """wpk_step with the activation scratch in the library's static device array."""
+    _check(load_library().wpk_step_noalloc(h, in_tok_dev or None, out_tok_dev or None, logits_dev or None,
+                                           stream or None), h)
 
 
 def wpk_graph_stats_get(h) -> dict:
