@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--slot-bytes", type=int, default=0)
     ap.add_argument("--workers-per-sm", type=int, default=0)
     ap.add_argument("--lookahead", type=int, default=0)
+    ap.add_argument("--schedule", default="queue", choices=["queue", "static"])
     return ap.parse_args()
 
 
@@ -216,7 +217,8 @@ def main():
     weights = synth.cached_weights(s, seed=0)
     mode = W.WPK_MEGAKERNEL if args.mode == "megakernel" else W.WPK_PER_OP_GRAPH
     plan = dict(mode=mode, tile_bytes=args.tile_bytes, slot_bytes=args.slot_bytes,
-                workers_per_sm=args.workers_per_sm, lookahead=args.lookahead)
+                workers_per_sm=args.workers_per_sm, lookahead=args.lookahead,
+                schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE)
     if args.regions:
         cuts = [int(x) for x in args.regions.split(",")]
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))

@@ -52,6 +52,8 @@ enum {
 };
 
 enum { WPK_MEGAKERNEL = 0, WPK_PER_OP_GRAPH = 1 };
+enum { WPK_SCHED_QUEUE = 0, WPK_SCHED_STATIC = 1 };
+enum { WPK_PREFILL_AUTO = 0, WPK_PREFILL_MMA = 1, WPK_PREFILL_TOKENWISE = 2 };
 
 /* --------------------------------------------------------------- configs */
 /* Decoder shape.  Weights are bf16, matmul weights stored [out][in]. */
@@ -80,12 +82,20 @@ typedef struct wpk_plan_cfg {
   int trace;            /* 1 = record the per-tile device trace                */
   uint64_t wait_timeout_ns; /* bound on every device wait (0 = 2 s)            */
   int slot_bytes;       /* staging slot per worker, used as a ring of 16 KB
-                           chunk stages (0 = as large as shared memory allows) */
+                           chunk stages (0 = 8 stages, 128 KB)                 */
   int tile_bytes;       /* target weight bytes per tile (0 = 65536)            */
   int split_pages;      /* KV pages per attention split (0 = 1)                */
   int lookahead;        /* tiles a worker may claim and stage ahead of the one
                            it computes (0 = 4); 1 = a tile's weights are staged
                            only after the previous tile of that worker is done */
+  int schedule;         /* WPK_SCHED_QUEUE (0): tickets from one atomic device
+                           queue; WPK_SCHED_STATIC: worker w takes tickets
+                           w, w + W, w + 2W, ... (W workers), no atomics       */
+  int prefill;          /* WPK_PREFILL_AUTO (0): the tensor-core prefill program
+                           when the shapes allow, else token by token;
+                           WPK_PREFILL_MMA; WPK_PREFILL_TOKENWISE (the prompt
+                           runs through the decode program one position at a
+                           time)                                                */
 } wpk_plan_cfg;
 
 /* Host weights: bf16 bit patterns, row-major [out][in]. */
@@ -123,17 +133,22 @@ typedef struct wpk_graph_stats {
   int64_t n_regions;
 } wpk_graph_stats;
 
-/* One trace record per tile of the last traced step (wpk_plan_cfg.trace). */
+/* One trace record per tile of the last traced step (wpk_plan_cfg.trace).
+ * Times are %globaltimer nanoseconds; event-clock values come from one global
+ * counter, so they order events across workers exactly. */
 typedef struct wpk_trace_rec {
-  uint32_t tile;        /* tile index (= ticket within the step)               */
-  uint16_t worker;      /* worker CTA that ran it                              */
-  uint16_t op;          /* op code                                             */
-  uint32_t ev_issue;    /* event clock when its staging load was issued        */
-  uint32_t ev_start;    /* event clock after its dependency wait succeeded     */
-  uint32_t ev_done;     /* event clock after its body, before it signalled     */
-  uint32_t epoch;       /* step epoch it belongs to                            */
-  uint64_t t_start_ns;  /* %globaltimer after the wait                         */
-  uint64_t t_end_ns;    /* %globaltimer after the body                         */
+  uint32_t tile;         /* tile index (= ticket within the step)              */
+  uint16_t worker;       /* worker CTA that ran it                             */
+  uint16_t op;           /* op code                                            */
+  uint32_t ev_issue;     /* event clock when its staging copies were issued    */
+  uint32_t ev_start;     /* event clock after its dependency wait succeeded    */
+  uint32_t ev_done;      /* event clock after its body, before it signalled    */
+  uint32_t epoch;        /* step epoch it belongs to                           */
+  uint64_t t_claim_ns;   /* producer took the ticket                           */
+  uint64_t t_issued_ns;  /* producer had issued all its staging copies         */
+  uint64_t t_start_ns;   /* compute warps passed the dependency wait           */
+  uint64_t t_data_ns;    /* the last staged chunk had landed and been consumed */
+  uint64_t t_end_ns;     /* body and epilogue done                             */
 } wpk_trace_rec;
 
 /* The first device error recorded by the program. */
@@ -191,6 +206,13 @@ int wpk_prefill(wpk_handle *h, const int32_t *tokens_dev, int batch, int prompt_
  * WPK_ERR_TIMEOUT). */
 int wpk_step(wpk_handle *h, const int32_t *in_tok_dev, int32_t *out_tok_dev, float *logits_dev,
              void *stream);
+
+/* Choose the program the inspection calls below (stats, edges, tile ops,
+ * verifier, simulator, trace) refer to: batch 0 selects the decode program;
+ * otherwise the prefill program for `batch` prompts of `prompt_len` tokens,
+ * compiled on first use (host work only).  WPK_ERR_UNSUPPORTED when the plan
+ * prefills token by token. */
+int wpk_select_program(wpk_handle *h, int batch, int prompt_len);
 
 /* Graph facts; *st is filled. */
 int wpk_graph_stats_get(const wpk_handle *h, wpk_graph_stats *st);
@@ -253,6 +275,18 @@ int wpk_destroy(wpk_handle *h);
  * Inputs, outputs and errors are those of wpk_step. */
 int wpk_step_noalloc(wpk_handle *h, const int32_t *in_tok_dev, int32_t *out_tok_dev, float *logits_dev,
                      void *stream);
+
+/* Check of the tensor-core tile (tests): D[128][N] = A . (B1 + B2)^T with fp32
+ * accumulation, computed by one CTA through the same path as the program's
+ * tensor-core tiles.  Operands are device "images" of 16-bit values (bf16 if
+ * `bf16`, else fp16): for each 64-column K chunk c, A's 128 rows x 128 bytes
+ * and B's N rows x 128 bytes, each row's eight 16-byte units stored at unit
+ * index (u XOR row % 8) (the 128-byte swizzle).  b2_img_dev may be NULL.
+ * d_dev receives fp32 [128][N] row-major.  N is a multiple of 16 in
+ * [16, 256].  Synchronous on `stream`; WPK_ERR_TIMEOUT if a bounded wait gave
+ * up. */
+int wpk_debug_gemm(const void *a_img_dev, const void *b1_img_dev, const void *b2_img_dev, float *d_dev,
+                   int n_chunks, int N, int bf16, void *stream);
 
 /* Test hook: make counter `counter` need one more signal than it can ever get
  * (an unsatisfiable dependency), so the next step's device wait must time out

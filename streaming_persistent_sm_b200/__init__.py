@@ -24,6 +24,7 @@ from .wpk import (  # noqa: F401
     wpk_last_error,
     wpk_load_weights,
     wpk_prefill,
+    wpk_select_program,
     wpk_set_block_table,
     wpk_simulate,
     wpk_step,

@@ -8,13 +8,14 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <memory>
 #include <string>
 #include <vector>
 
 #include "graph.h"
 
 namespace wpk {
-size_t worker_smem_bytes(int n_stages, int act_bytes);
+size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes);
 const void* persistent_kernel_ptr();
 const void* per_op_kernel_ptr();
 }  // namespace wpk
@@ -22,10 +23,22 @@ const void* per_op_kernel_ptr();
 using namespace wpk;
 
 struct GraphEntry {
-  int32_t* out_tok;
-  float* logits;
+  const void* key0;  // decode: out_tok; prefill: tokens
+  const void* key1;  // decode: logits;  prefill: first_tok
+  const void* key2;  // prefill: logits
   cudaGraph_t graph;
   cudaGraphExec_t exec;
+};
+
+// A prefill program compiled for (B, T), with its own device tables.
+struct PrefillProgram {
+  CompiledGraph g;
+  uint8_t* d_base = nullptr;
+  Tile* d_tiles = nullptr;
+  uint32_t* d_sig = nullptr;
+  uint32_t* d_ctr = nullptr;
+  TraceRec* d_trace = nullptr;
+  std::vector<GraphEntry> graphs;
 };
 
 struct wpk_handle {
@@ -62,6 +75,14 @@ struct wpk_handle {
   std::vector<GraphEntry> graphs;
   cudaStream_t capture_stream = nullptr;
   std::string err;
+  // prefill programs and their scratch (offsets in the caller's scratch)
+  std::vector<std::unique_ptr<PrefillProgram>> prefills;
+  size_t off_px = 0, off_pq = 0, off_xn[2] = {0, 0}, off_att[2] = {0, 0}, off_hi[2] = {0, 0};
+  int64_t prefill_max_tokens = 0;
+  int prefill_stages = 0;
+  size_t smem_prefill = 0;
+  // program the inspection calls refer to (nullptr = the decode program)
+  PrefillProgram* selected = nullptr;
 };
 
 namespace {
@@ -119,6 +140,7 @@ KParams make_params(const wpk_handle* h) {
   P.split_tokens = g.split_tokens;
   P.n_splits = g.n_splits;
   P.n_stages = g.plan.slot_bytes / kStageBytes;
+  P.stage_bytes = kStageBytes;
   P.lookahead = g.plan.lookahead;
   P.act_bytes = g.plan.act_bytes;
   P.timeout_ns = g.plan.wait_timeout_ns;
@@ -152,6 +174,7 @@ KParams make_params(const wpk_handle* h) {
   P.evclock = h->d_evclock;
   P.in_tok_stride = 1;
   P.epoch = 1;
+  P.static_sched = g.plan.schedule == WPK_SCHED_STATIC;
   return P;
 }
 
@@ -167,6 +190,17 @@ void scratch_layout(wpk_handle* h) {
   h->off_attn = take(B * q_rows * 4);
   h->off_h = take(B * m.ffn * 4);
   h->off_part = take(B * m.n_kv_heads * g.n_splits * (m.n_heads / m.n_kv_heads) * (2 + m.head_dim) * 4);
+  if (g.plan.prefill_mode == WPK_PREFILL_MMA) {
+    // prefill of up to max_batch prompts of max_context tokens, in blocks of 128
+    const size_t M = (size_t)g.plan.max_batch * g.plan.max_context;
+    const size_t n_tb = (M + kTokBlock - 1) / kTokBlock;
+    h->prefill_max_tokens = (int64_t)M;
+    h->off_px = take(M * m.hidden * 4);
+    h->off_pq = take(M * q_rows * 4);
+    for (int i = 0; i < 2; ++i) h->off_xn[i] = take(n_tb * (m.hidden / 64) * kMmaChunkBytes);
+    for (int i = 0; i < 2; ++i) h->off_att[i] = take(n_tb * (q_rows / 64) * kMmaChunkBytes);
+    for (int i = 0; i < 2; ++i) h->off_hi[i] = take(n_tb * (m.ffn / 64) * kMmaChunkBytes);
+  }
   h->scratch_bytes = off;
   h->n_blocks = (int64_t)B * g.max_blocks;
   h->kv_bytes = (size_t)m.n_layers * h->n_blocks * 2 * m.n_kv_heads * g.plan.page_tokens * m.head_dim * 2;
@@ -212,8 +246,9 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
       return fail(h, WPK_ERR_CUDA, std::string("per-op capture: ") + cudaGetErrorString(e));
     }
   }
-  out->out_tok = out_tok;
-  out->logits = logits;
+  out->key0 = out_tok;
+  out->key1 = logits;
+  out->key2 = nullptr;
   CUDA_TRY(h, cudaStreamEndCapture(h->capture_stream, &out->graph));
   CUDA_TRY(h, cudaGraphInstantiate(&out->exec, out->graph, 0));
   return WPK_OK;
@@ -234,7 +269,7 @@ int step_impl(wpk_handle* h, const int32_t* in_tok, int stride, int32_t* out_tok
                                     cudaMemcpyDeviceToDevice, s));
     GraphEntry* ge = nullptr;
     for (auto& e : h->graphs)
-      if (e.out_tok == out_tok && e.logits == logits) ge = &e;
+      if (e.key0 == out_tok && e.key1 == logits) ge = &e;
     if (!ge) {
       GraphEntry e{};
       int rc = capture_per_op(h, out_tok, logits, &e);
@@ -250,6 +285,118 @@ int step_impl(wpk_handle* h, const int32_t* in_tok, int stride, int32_t* out_tok
   return WPK_OK;
 }
 
+
+// ------------------------------------------------------------ prefill program
+int get_prefill_program(wpk_handle* h, int B, int T, PrefillProgram** out) {
+  for (auto& p : h->prefills)
+    if (p->g.B == B && p->g.T == T) {
+      *out = p.get();
+      return WPK_OK;
+    }
+  auto prog = std::make_unique<PrefillProgram>();
+  std::string msg = compile_prefill_graph(h->g, B, T, &prog->g);
+  if (!msg.empty()) return fail(h, WPK_ERR_UNSUPPORTED, msg);
+  if (h->has_device) {
+    const CompiledGraph& g = prog->g;
+    const size_t n_tiles = g.tiles.size(), n_ctr = std::max<size_t>(1, g.ctr_need.size());
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = a256(off + bytes); return o; };
+    const size_t o_tiles = take(n_tiles * sizeof(Tile)), o_sig = take(std::max<size_t>(1, g.sig.size()) * 4),
+                 o_ctr = take(n_ctr * 4), o_trace = take(n_tiles * sizeof(TraceRec));
+    CUDA_TRY(h, cudaMalloc(&prog->d_base, off));
+    CUDA_TRY(h, cudaMemset(prog->d_base, 0, off));
+    prog->d_tiles = reinterpret_cast<Tile*>(prog->d_base + o_tiles);
+    prog->d_sig = reinterpret_cast<uint32_t*>(prog->d_base + o_sig);
+    prog->d_ctr = reinterpret_cast<uint32_t*>(prog->d_base + o_ctr);
+    prog->d_trace = reinterpret_cast<TraceRec*>(prog->d_base + o_trace);
+    CUDA_TRY(h, cudaMemcpy(prog->d_tiles, g.tiles.data(), n_tiles * sizeof(Tile), cudaMemcpyHostToDevice));
+    if (!g.sig.empty())
+      CUDA_TRY(h, cudaMemcpy(prog->d_sig, g.sig.data(), g.sig.size() * 4, cudaMemcpyHostToDevice));
+  }
+  *out = prog.get();
+  h->prefills.push_back(std::move(prog));
+  return WPK_OK;
+}
+
+KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const int32_t* tokens, int32_t* first_tok,
+                       float* logits) {
+  KParams P = make_params(h);
+  const CompiledGraph& g = prog->g;
+  P.tiles = prog->d_tiles;
+  P.sig = prog->d_sig;
+  P.ctr = prog->d_ctr;
+  P.trace_buf = prog->d_trace;
+  P.stage_bytes = 3 * kMmaChunkBytes;
+  P.n_stages = h->prefill_stages;
+  P.uses_tmem = 1;
+  P.M = g.M;
+  P.T = g.T;
+  P.n_tb = g.n_tb;
+  P.ptok = tokens;
+  P.px = reinterpret_cast<float*>(h->scratch + h->off_px);
+  P.pq = reinterpret_cast<float*>(h->scratch + h->off_pq);
+  for (int i = 0; i < 2; ++i) {
+    P.xn_img[i] = h->scratch + h->off_xn[i];
+    P.att_img[i] = h->scratch + h->off_att[i];
+    P.h_img[i] = h->scratch + h->off_hi[i];
+  }
+  P.in_tok = nullptr;
+  P.out_tok = first_tok;
+  P.logits = logits;
+  return P;
+}
+
+int launch_prefill(wpk_handle* h, PrefillProgram* prog, const int32_t* tokens, int32_t* first_tok, float* logits,
+                   cudaStream_t s) {
+  const CompiledGraph& g = prog->g;
+  const KParams base = prefill_params(h, prog, tokens, first_tok, logits);
+  if (g.plan.mode == WPK_MEGAKERNEL) {
+    CUDA_TRY(h, cudaMemsetAsync(prog->d_ctr, 0, std::max<size_t>(1, g.ctr_need.size()) * 4, s));
+    CUDA_TRY(h, cudaMemsetAsync(h->d_head, 0, 4 * 4, s));
+    for (int r = 0; r + 1 < (int)g.region_begin.size(); ++r) {
+      KParams P = base;
+      P.t_begin = g.region_begin[r];
+      P.t_end = g.region_begin[r + 1];
+      P.region = r;
+      void* args[] = {&P};
+      CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
+                                              h->smem_prefill, s));
+    }
+    return WPK_OK;
+  }
+  GraphEntry* ge = nullptr;
+  for (auto& e : prog->graphs)
+    if (e.key0 == tokens && e.key1 == first_tok && e.key2 == logits) ge = &e;
+  if (!ge) {
+    if (!h->capture_stream) CUDA_TRY(h, cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking));
+    GraphEntry e{tokens, first_tok, logits, nullptr, nullptr};
+    CUDA_TRY(h, cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal));
+    for (const OpGroup& og : g.groups) {
+      KParams P = base;
+      P.t_begin = og.begin;
+      P.t_end = og.end;
+      P.per_op = 1;
+      void* args[] = {&P};
+      cudaError_t err = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
+                                         h->smem_prefill, h->capture_stream);
+      if (err != cudaSuccess) {
+        cudaGraph_t junk = nullptr;
+        cudaStreamEndCapture(h->capture_stream, &junk);
+        if (junk) cudaGraphDestroy(junk);
+        return fail(h, WPK_ERR_CUDA, std::string("per-op prefill capture: ") + cudaGetErrorString(err));
+      }
+    }
+    CUDA_TRY(h, cudaStreamEndCapture(h->capture_stream, &e.graph));
+    CUDA_TRY(h, cudaGraphInstantiate(&e.exec, e.graph, 0));
+    prog->graphs.push_back(e);
+    ge = &prog->graphs.back();
+  }
+  CUDA_TRY(h, cudaGraphLaunch(ge->exec, s));
+  return WPK_OK;
+}
+
+const CompiledGraph& selected_graph(const wpk_handle* h) { return h->selected ? h->selected->g : h->g; }
+
 }  // namespace
 
 extern "C" {
@@ -260,16 +407,23 @@ static int setup_device(wpk_handle* h) {
   const wpk_model_cfg* model = &g.m;
   CUDA_TRY(h, cudaGetDevice(&h->device));
   CUDA_TRY(h, cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, h->device));
-  h->smem = worker_smem_bytes(p.slot_bytes / kStageBytes, p.act_bytes);
-  h->smem_per_op = worker_smem_bytes(p.per_op_slot / kStageBytes, p.act_bytes);
+  h->smem = worker_smem_bytes(p.slot_bytes / kStageBytes, kStageBytes, p.act_bytes);
+  h->smem_per_op = worker_smem_bytes(p.per_op_slot / kStageBytes, kStageBytes, p.act_bytes);
   if (h->smem > (size_t)kMaxSmem || h->smem_per_op > (size_t)kMaxSmem)
     return fail(h, WPK_ERR_UNSUPPORTED, "staging slot and activations exceed shared memory");
+  if (p.prefill_mode == WPK_PREFILL_MMA) {
+    const size_t fixed = worker_smem_bytes(0, 0, p.act_bytes);
+    h->prefill_stages = (int)std::min<size_t>(kMaxStages, ((size_t)kMaxSmem - fixed) / (3 * kMmaChunkBytes));
+    if (h->prefill_stages < 2) return fail(h, WPK_ERR_UNSUPPORTED, "no room for the prefill staging ring");
+    h->smem_prefill = worker_smem_bytes(h->prefill_stages, 3 * kMmaChunkBytes, p.act_bytes);
+  }
+  const size_t smem_max = std::max(h->smem, h->smem_prefill);
   CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)h->smem));
+                                   (int)smem_max));
   CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)h->smem_per_op));
+                                   (int)std::max(h->smem_per_op, h->smem_prefill)));
   int per_sm = 0;
-  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kCtaThreads, h->smem));
+  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kCtaThreads, smem_max));
   h->n_workers = p.n_workers ? p.n_workers : h->n_sms * p.workers_per_sm;
   if (per_sm < 1 || h->n_workers > per_sm * h->n_sms)
     return fail(h, WPK_ERR_UNSUPPORTED, "the worker grid cannot be co-resident with this slot size");
@@ -421,6 +575,24 @@ int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_
   CUDA_TRY(h, cudaStreamSynchronize(s));  // `batch` lives on this stack frame
   h->batch = batch;
   h->ctx = 0;
+  if (h->g.plan.prefill_mode == WPK_PREFILL_MMA) {
+    if ((int64_t)batch * prompt_len > h->prefill_max_tokens)
+      return fail(h, WPK_ERR_SHAPE, "prompt tokens exceed the prefill scratch");
+    PrefillProgram* prog = nullptr;
+    rc = get_prefill_program(h, batch, prompt_len, &prog);
+    if (rc) return rc;
+    // positions count up from 0; the final tile advances them to prompt_len
+    std::vector<int32_t> pos(h->g.plan.max_batch, prompt_len - 1);
+    CUDA_TRY(h, cudaMemcpyAsync(h->d_seqlen, pos.data(), pos.size() * 4, cudaMemcpyHostToDevice, s));
+    CUDA_TRY(h, cudaStreamSynchronize(s));  // `pos` lives on this stack frame
+    rc = launch_prefill(h, prog, tokens_dev, first_tok_dev, logits_dev, s);
+    if (rc) return rc;
+    CUDA_TRY(h, cudaMemcpyAsync(h->h_err_code, &h->d_err->code, 4, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(h, cudaGetLastError());
+    h->ctx = prompt_len;
+    h->prefilled = true;
+    return WPK_OK;
+  }
   // The prompt runs through the decode program one position at a time.
   for (int t = 0; t < prompt_len; ++t) {
     const bool last = (t + 1 == prompt_len);
@@ -442,7 +614,7 @@ int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, flo
 int wpk_graph_stats_get(const wpk_handle* h, wpk_graph_stats* st) {
   if (!h || !st) return WPK_ERR_INVALID_ARG;
   memset(st, 0, sizeof *st);
-  const CompiledGraph& g = h->g;
+  const CompiledGraph& g = selected_graph(h);
   st->n_tiles = (int64_t)g.tiles.size();
   st->n_counters = (int64_t)g.ctr_need.size();
   st->n_edges = g.n_edges;
@@ -458,8 +630,9 @@ int wpk_graph_stats_get(const wpk_handle* h, wpk_graph_stats* st) {
 int wpk_get_edges(const wpk_handle* h, int32_t* pairs, int64_t max_pairs, int64_t* n_pairs) {
   if (!h || !n_pairs) return WPK_ERR_INVALID_ARG;
   int64_t k = 0;
-  for (size_t v = 0; v < h->g.preds.size(); ++v)
-    for (int u : h->g.preds[v]) {
+  const CompiledGraph& g = selected_graph(h);
+  for (size_t v = 0; v < g.preds.size(); ++v)
+    for (int u : g.preds[v]) {
       if (pairs && k < max_pairs) {
         pairs[2 * k] = u;
         pairs[2 * k + 1] = (int32_t)v;
@@ -471,14 +644,33 @@ int wpk_get_edges(const wpk_handle* h, int32_t* pairs, int64_t max_pairs, int64_
 }
 
 int wpk_get_tile_ops(const wpk_handle* h, int32_t* ops, int64_t n) {
-  if (!h || !ops || n < (int64_t)h->g.tiles.size()) return WPK_ERR_INVALID_ARG;
-  for (size_t i = 0; i < h->g.tiles.size(); ++i) ops[i] = h->g.tiles[i].op;
+  if (!h || !ops) return WPK_ERR_INVALID_ARG;
+  const CompiledGraph& g = selected_graph(h);
+  if (n < (int64_t)g.tiles.size()) return WPK_ERR_INVALID_ARG;
+  for (size_t i = 0; i < g.tiles.size(); ++i) ops[i] = g.tiles[i].op;
+  return WPK_OK;
+}
+
+int wpk_select_program(wpk_handle* h, int batch, int prompt_len) {
+  if (!h) return WPK_ERR_INVALID_ARG;
+  if (batch == 0) {
+    h->selected = nullptr;
+    return WPK_OK;
+  }
+  if (h->g.plan.prefill_mode != WPK_PREFILL_MMA)
+    return fail(h, WPK_ERR_UNSUPPORTED, "the plan prefills token by token through the decode program");
+  if (batch < 0 || prompt_len <= 0 || batch > h->g.plan.max_batch || prompt_len > h->g.plan.max_context)
+    return fail(h, WPK_ERR_SHAPE, "batch or prompt exceeds the plan");
+  PrefillProgram* prog = nullptr;
+  int rc = get_prefill_program(h, batch, prompt_len, &prog);
+  if (rc) return rc;
+  h->selected = prog;
   return WPK_OK;
 }
 
 int wpk_verify_graph(const wpk_handle* h) {
   if (!h) return WPK_ERR_INVALID_ARG;
-  std::string msg = verify_graph(h->g);
+  std::string msg = verify_graph(selected_graph(h));
   if (!msg.empty()) {
     const_cast<wpk_handle*>(h)->err = msg;
     return WPK_ERR_SHAPE;
@@ -490,7 +682,7 @@ int wpk_simulate(const wpk_handle* h, int n_threads, int n_epochs, uint64_t seed
                  int32_t* done_order) {
   if (!h || n_threads <= 0 || n_epochs <= 0 || wait_ms <= 0) return WPK_ERR_INVALID_ARG;
   std::string msg;
-  int rc = simulate_graph(h->g, n_threads, n_epochs, seed, wait_ms, stuck_tile, done_order, &msg);
+  int rc = simulate_graph(selected_graph(h), n_threads, n_epochs, seed, wait_ms, stuck_tile, done_order, &msg);
   if (rc) const_cast<wpk_handle*>(h)->err = msg;
   return rc;
 }
@@ -498,11 +690,12 @@ int wpk_simulate(const wpk_handle* h, int n_threads, int n_epochs, uint64_t seed
 int wpk_get_trace(wpk_handle* h, void* host_buf, size_t bytes) {
   if (!h || !host_buf) return WPK_ERR_INVALID_ARG;
   if (!h->has_device) return fail(h, WPK_ERR_CUDA, "no CUDA device");
-  const size_t need = h->g.tiles.size() * sizeof(TraceRec);
+  const CompiledGraph& g = selected_graph(h);
+  const size_t need = g.tiles.size() * sizeof(TraceRec);
   if (bytes < need) return fail(h, WPK_ERR_INVALID_ARG, "trace buffer too small");
   if (!h->g.plan.trace) return fail(h, WPK_ERR_UNSUPPORTED, "plan was built without trace");
   CUDA_TRY(h, cudaDeviceSynchronize());
-  CUDA_TRY(h, cudaMemcpy(host_buf, h->d_trace, need, cudaMemcpyDeviceToHost));
+  CUDA_TRY(h, cudaMemcpy(host_buf, h->selected ? h->selected->d_trace : h->d_trace, need, cudaMemcpyDeviceToHost));
   return WPK_OK;
 }
 
@@ -530,6 +723,13 @@ int wpk_destroy(wpk_handle* h) {
   for (auto& e : h->graphs) {
     if (e.exec) cudaGraphExecDestroy(e.exec);
     if (e.graph) cudaGraphDestroy(e.graph);
+  }
+  for (auto& p : h->prefills) {
+    for (auto& e : p->graphs) {
+      if (e.exec) cudaGraphExecDestroy(e.exec);
+      if (e.graph) cudaGraphDestroy(e.graph);
+    }
+    if (p->d_base) cudaFree(p->d_base);
   }
   if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
   if (h->d_base) cudaFree(h->d_base);

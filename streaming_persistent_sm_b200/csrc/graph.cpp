@@ -72,12 +72,15 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   p->trace = in.trace;
   p->wait_timeout_ns = in.wait_timeout_ns ? in.wait_timeout_ns : 2000000000ull;
   p->lookahead = in.lookahead ? in.lookahead : 4;
+  p->schedule = in.schedule;
+  if (p->schedule != WPK_SCHED_QUEUE && p->schedule != WPK_SCHED_STATIC) return "bad schedule";
   if (p->lookahead < 1 || p->lookahead > kMaxQueue) return "lookahead must be 1..8";
   // activation staging: up to kMaxGemvBatch rows of the longest GEMV K (<= 2048)
   const int q_rows = m.n_heads * m.head_dim;
   const int kmax = std::max(std::max(m.hidden, q_rows), std::min(m.ffn, 2048));
   if (kmax > 2048) { *code = WPK_ERR_UNSUPPORTED; return "hidden and n_heads*head_dim must be <= 2048"; }
-  p->act_bytes = std::max(16384, std::min(in.max_batch, kMaxGemvBatch) * kmax * 4);
+  const int kmax_pad = (kmax + 255) / 256 * 256;  // staged rows are padded to whole 256-column segments
+  p->act_bytes = std::max(16384, std::min(in.max_batch, kMaxGemvBatch) * kmax_pad * 4);
   p->act_bytes = (p->act_bytes + 1023) / 1024 * 1024;
   const int fixed = 4096 + 1024;  // partial outputs, tile queue, barriers
   const int budget = std::min(kMaxSmem, 233472 / p->workers_per_sm - 1024) - p->act_bytes - fixed;
@@ -87,7 +90,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
     if (in.slot_bytes > budget) return "slot_bytes does not fit shared memory with this many workers per SM";
     p->slot_bytes = in.slot_bytes;
   } else {
-    p->slot_bytes = std::min(kMaxStages, budget / kStageBytes) * kStageBytes;
+    p->slot_bytes = std::min(8, budget / kStageBytes) * kStageBytes;
     if (p->slot_bytes < kStageBytes) return "no room for a staging slot";
   }
   p->tile_bytes = in.tile_bytes ? in.tile_bytes : 65536;
@@ -97,6 +100,20 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   if ((int64_t)p->split_pages * p->page_tokens * m.head_dim * 2 * 2 > kStageBytes)
     return "an attention split's K/V pages do not fit one 16 KB stage";
   p->per_op_slot = 0;  // set by compile_graph
+  {
+    const int qr = m.n_heads * m.head_dim, kvr = m.n_kv_heads * m.head_dim;
+    const bool mma_ok = (qr + 2 * kvr) % 128 == 0 && m.hidden % 128 == 0 && (2 * m.ffn) % 128 == 0 &&
+                        m.hidden % 64 == 0 && qr % 128 == 0 && m.ffn % 64 == 0 && kvr % 128 == 0;
+    if (in.prefill == WPK_PREFILL_AUTO)
+      p->prefill_mode = mma_ok ? WPK_PREFILL_MMA : WPK_PREFILL_TOKENWISE;
+    else if (in.prefill == WPK_PREFILL_MMA) {
+      if (!mma_ok) { *code = WPK_ERR_UNSUPPORTED; return "shapes do not fit the tensor-core prefill tiles"; }
+      p->prefill_mode = WPK_PREFILL_MMA;
+    } else if (in.prefill == WPK_PREFILL_TOKENWISE)
+      p->prefill_mode = WPK_PREFILL_TOKENWISE;
+    else
+      return "bad prefill mode";
+  }
   *code = WPK_OK;
   return "";
 }
@@ -111,26 +128,29 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
 namespace {
 
 struct Seg {
-  int lo, hi;
   int wgroup;                // group id of the current writers (-1 = single)
   std::vector<int> writers;  // last plain write (one tile, or one write group)
   std::vector<int> accs;     // accumulators since then
 };
 
+// Disjoint segments covering [0, size), keyed by their low end.
 struct BufState {
-  std::vector<Seg> segs;  // sorted, disjoint, covering [0, size)
-  explicit BufState(int size = 1) { segs.push_back({0, size, -1, {}, {}}); }
-  // split so that x is a segment boundary
-  void cut(int x) {
-    for (size_t i = 0; i < segs.size(); ++i) {
-      if (segs[i].lo < x && x < segs[i].hi) {
-        Seg b = segs[i];
-        b.lo = x;
-        segs[i].hi = x;
-        segs.insert(segs.begin() + i + 1, b);
-        return;
-      }
-    }
+  std::map<int64_t, Seg> segs;
+  int64_t hi_;
+  explicit BufState(int64_t size = 1) : hi_(size) { segs.emplace(0, Seg{-1, {}, {}}); }
+  // make x a segment boundary
+  void cut(int64_t x) {
+    if (x <= 0 || x >= hi_) return;
+    auto it = segs.upper_bound(x);
+    --it;
+    if (it->first == x) return;
+    segs.emplace(x, it->second);
+  }
+  // first segment overlapping [lo, ...)
+  std::map<int64_t, Seg>::iterator first(int64_t lo) {
+    auto it = segs.upper_bound(lo);
+    --it;
+    return it;
   }
 };
 
@@ -138,16 +158,16 @@ struct DataflowBuilder {
   std::vector<BufState> bufs;
   const std::vector<std::vector<int32_t>>* preds_of = nullptr;
   // memo of a read's frontier: (buf, lo, hi) -> preds, dropped when buf changes
-  std::map<std::tuple<int, int, int>, std::vector<int>> memo;
+  std::map<std::tuple<int, int64_t, int64_t>, std::vector<int>> memo;
 
-  std::vector<int> frontier(int b, int lo, int hi) {
+  std::vector<int> frontier(int b, int64_t lo, int64_t hi) {
     auto key = std::make_tuple(b, lo, hi);
-    auto it = memo.find(key);
-    if (it != memo.end()) return it->second;
+    auto mit = memo.find(key);
+    if (mit != memo.end()) return mit->second;
     std::vector<int> out;
-    for (auto& s : bufs[b].segs) {
-      if (s.hi <= lo || s.lo >= hi) continue;
-      const auto& src = s.accs.empty() ? s.writers : s.accs;
+    BufState& B = bufs[b];
+    for (auto it = B.first(lo); it != B.segs.end() && it->first < hi; ++it) {
+      const auto& src = it->second.accs.empty() ? it->second.writers : it->second.accs;
       out.insert(out.end(), src.begin(), src.end());
     }
     std::sort(out.begin(), out.end());
@@ -174,14 +194,17 @@ struct DataflowBuilder {
         auto f = frontier(a.buf, a.lo, a.hi);
         preds->insert(preds->end(), f.begin(), f.end());
       } else if (a.kind == 2) {
-        for (auto& s : bufs[a.buf].segs)
-          if (!(s.hi <= a.lo || s.lo >= a.hi)) acc_deps.insert(acc_deps.end(), s.writers.begin(), s.writers.end());
+        BufState& B = bufs[a.buf];
+        for (auto it = B.first(a.lo); it != B.segs.end() && it->first < a.hi; ++it)
+          acc_deps.insert(acc_deps.end(), it->second.writers.begin(), it->second.writers.end());
       }
     }
     std::sort(preds->begin(), preds->end());
     preds->erase(std::unique(preds->begin(), preds->end()), preds->end());
     // An accumulate must follow the write that initialised its range; skip the
     // edge when one of the tile's read predecessors already depends on it.
+    std::sort(acc_deps.begin(), acc_deps.end());
+    acc_deps.erase(std::unique(acc_deps.begin(), acc_deps.end()), acc_deps.end());
     for (int u : acc_deps) {
       bool implied = std::binary_search(preds->begin(), preds->end(), u);
       for (size_t i = 0; !implied && i < preds->size() && i < 4; ++i) implied = is_pred(u, (*preds)[i]);
@@ -192,8 +215,8 @@ struct DataflowBuilder {
       BufState& B = bufs[a.buf];
       B.cut(a.lo);
       B.cut(a.hi);
-      for (auto& s : B.segs) {
-        if (s.hi <= a.lo || s.lo >= a.hi) continue;
+      for (auto it = B.first(a.lo); it != B.segs.end() && it->first < a.hi; ++it) {
+        Seg& s = it->second;
         if (a.kind == 1) {
           if (a.group >= 0 && s.wgroup == a.group && s.accs.empty()) {
             s.writers.push_back(t);
@@ -222,10 +245,16 @@ struct VecHash {
   }
 };
 
+// Rows per GEMV tile: about tile_bytes, a multiple of 8, and no more chunk
+// stages than half the staging ring (a GEMV tile releases its stages when it
+// completes, so the ring must hold two tiles for the loads to keep flowing).
 int rows_per_tile(int row_bytes, const Plan& p) {
-  int r = p.tile_bytes / row_bytes;
-  r = r / 8 * 8;
-  if (r < 8) r = 8;
+  int rpc = (kStageBytes / row_bytes) & ~1;
+  if (rpc < 2) rpc = 2;
+  const int half_ring = std::max(1, p.slot_bytes / kStageBytes / 2);
+  int r = std::min(p.tile_bytes / row_bytes, half_ring * rpc);
+  r &= ~1;  // RoPE and gate/up row pairs stay in one tile
+  if (r < 2) r = 2;
   return std::min(r, kMaxTileRows);
 }
 
@@ -265,6 +294,16 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   L.final_norm = take((uint64_t)h * 4);
   L.embed = take((uint64_t)m.vocab * h * 2);
   L.lm_head = m.tied_embedding ? L.embed : take((uint64_t)m.vocab * h * 2);
+  L.mma = p.prefill_mode == WPK_PREFILL_MMA;
+  for (int l = 0; l < m.n_layers; ++l) {
+    LayerDev& d = L.layers[l];
+    d.mma_qkv = d.mma_wo = d.mma_gu = d.mma_down = 0;
+    if (!L.mma) continue;
+    d.mma_qkv = take((uint64_t)qkv_rows * h * 2);
+    d.mma_wo = take((uint64_t)h * q_rows * 2);
+    d.mma_gu = take((uint64_t)2 * m.ffn * h * 2);
+    d.mma_down = take((uint64_t)h * m.ffn * 2);
+  }
   L.total = off;
   L.down_kc = kc;
   L.n_down_chunks = nch;
@@ -423,6 +462,187 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
 }
 
 // ---------------------------------------------------------------------------
+// Prefill program.  Token rows m = b*T + t (M = B*T) are processed in blocks of
+// kTokBlock rows.  Per layer: RMSNorm of each block into a bf16 hi/lo image,
+// tensor-core QKV tiles (RoPE, q to Q, k/v to the KV cache), causal attention
+// tiles of kPrefillQB queries (the GQA group of one kv head), tensor-core O
+// tiles (X += .), RMSNorm again, tensor-core gate/up tiles (SwiGLU into the h
+// image) and down tiles (X += .).  Then the last position of every sequence is
+// gathered and the decode program's LM head + argmax tiles produce the first
+// token.  Buffers are modelled per token block so that edges follow blocks.
+// ---------------------------------------------------------------------------
+std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, CompiledGraph* g) {
+  const wpk_model_cfg& m = dec.m;
+  const Plan& p = dec.plan;
+  if (!dec.lay.mma) return "the weight image has no tensor-core layout";
+  g->m = m;
+  g->plan = p;
+  g->lay = dec.lay;
+  g->split_tokens = dec.split_tokens;
+  g->n_splits = dec.n_splits;
+  g->max_blocks = dec.max_blocks;
+  g->B = B;
+  g->T = T;
+  g->M = B * T;
+  g->n_tb = (g->M + kTokBlock - 1) / kTokBlock;
+  const int h = m.hidden, hd = m.head_dim, grp = m.n_heads / m.n_kv_heads;
+  const int q_rows = m.n_heads * hd, kv_rows = m.n_kv_heads * hd, qkv_rows = q_rows + 2 * kv_rows;
+  const int nq = g->n_tb;
+  const int64_t TB = kTokBlock;
+  std::vector<Tile>& Tl = g->tiles;
+  std::vector<std::vector<Access>>& A = g->access;
+  Tl.clear();
+  A.clear();
+  g->groups.clear();
+  int64_t wbytes = 0;
+  auto add = [&](uint16_t op, int layer, uint64_t w_off, uint32_t w_bytes, int a0, int a1, int a2, int a3,
+                 std::vector<Access> acc) {
+    Tile t{};
+    t.op = op;
+    t.layer = (uint16_t)layer;
+    t.wait_ctr = kNoCounter;
+    t.w_off = w_off;
+    t.w_bytes = w_bytes;
+    t.a0 = a0; t.a1 = a1; t.a2 = a2; t.a3 = a3;
+    wbytes += w_bytes;
+    if (g->groups.empty() || g->groups.back().op != op || g->groups.back().layer != layer)
+      g->groups.push_back({op, layer, (uint32_t)Tl.size(), (uint32_t)Tl.size()});
+    Tl.push_back(t);
+    A.push_back(std::move(acc));
+    g->groups.back().end = (uint32_t)Tl.size();
+  };
+  // modelled intervals: block tb of a buffer with `width` features
+  auto blk = [&](int buf, int width, int tb, int f0, int f1, int kind, int group = -1) {
+    Access a;
+    a.buf = buf;
+    a.lo = (int64_t)tb * width * TB + (int64_t)f0 * TB;
+    a.hi = (int64_t)tb * width * TB + (int64_t)f1 * TB;
+    a.kind = kind;
+    a.group = group;
+    return a;
+  };
+  auto kvblk = [&](int layer, int tb, int f0, int f1, int kind) {  // per-layer KV, features [0, 2*kv_rows)
+    Access a;
+    a.buf = BUF_PKV;
+    a.lo = ((int64_t)layer * nq + tb) * (2 * kv_rows) * TB + (int64_t)f0 * TB;
+    a.hi = ((int64_t)layer * nq + tb) * (2 * kv_rows) * TB + (int64_t)f1 * TB;
+    a.kind = kind;
+    a.group = -1;
+    return a;
+  };
+  std::vector<uint32_t> layer_begin(m.n_layers + 1, 0);
+  for (int tb = 0; tb < nq; ++tb) add(OP_PEMBED, 0, 0, 0, tb, 0, 0, 0, {blk(BUF_PX, h, tb, 0, h, 1)});
+  const uint32_t chunk = kMmaChunkBytes;
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerDev& d = dec.lay.layers[l];
+    layer_begin[l] = (uint32_t)Tl.size();
+    for (int tb = 0; tb < nq; ++tb)
+      add(OP_NORM, l, 0, 0, tb, 0, 0, h, {blk(BUF_PX, h, tb, 0, h, 0), blk(BUF_PXN, h, tb, 0, h, 1)});
+    // QKV: feature blocks of 128 rows; never straddle q/k/v (all multiples of 128)
+    for (int tb = 0; tb < nq; ++tb)
+      for (int fb = 0; fb < qkv_rows / 128; ++fb) {
+        const int f0 = fb * 128;
+        std::vector<Access> acc{blk(BUF_PXN, h, tb, 0, h, 0)};
+        if (f0 < q_rows)
+          acc.push_back(blk(BUF_PQ, q_rows, tb, f0, f0 + 128, 1));
+        else
+          acc.push_back(kvblk(l, tb, f0 - q_rows, f0 - q_rows + 128, 1));
+        add(OP_MQKV, l, d.mma_qkv + (uint64_t)fb * (h / 64) * chunk, (uint32_t)(h / 64) * chunk, fb, tb, 0, h, acc);
+      }
+    // causal attention: (sequence, kv head, query block)
+    const int attn_group = 2000 + l;
+    for (int b = 0; b < B; ++b)
+      for (int gi = 0; gi < m.n_kv_heads; ++gi)
+        for (int qb = 0; qb * kPrefillQB < T; ++qb) {
+          const int t0 = qb * kPrefillQB, t1 = std::min(T, t0 + kPrefillQB);
+          const int m0 = b * T + t0, m1 = b * T + t1;  // query rows
+          std::vector<Access> acc;
+          for (int tb = m0 / kTokBlock; tb <= (m1 - 1) / kTokBlock; ++tb) {
+            acc.push_back(blk(BUF_PQ, q_rows, tb, gi * grp * hd, (gi + 1) * grp * hd, 0));
+            acc.push_back(blk(BUF_PATT, q_rows, tb, gi * grp * hd, (gi + 1) * grp * hd, 1, attn_group));
+          }
+          for (int tb = (b * T) / kTokBlock; tb <= (m1 - 1) / kTokBlock; ++tb) {
+            acc.push_back(kvblk(l, tb, gi * hd, (gi + 1) * hd, 0));                      // k of head gi
+            acc.push_back(kvblk(l, tb, kv_rows + gi * hd, kv_rows + (gi + 1) * hd, 0));  // v of head gi
+          }
+          add(OP_PATTN, l, 0, 0, b, gi, qb, 0, acc);
+        }
+    for (int tb = 0; tb < nq; ++tb)
+      for (int fb = 0; fb < h / 128; ++fb)
+        add(OP_MO, l, d.mma_wo + (uint64_t)fb * (q_rows / 64) * chunk, (uint32_t)(q_rows / 64) * chunk, fb, tb, 0,
+            q_rows, {blk(BUF_PATT, q_rows, tb, 0, q_rows, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
+    for (int tb = 0; tb < nq; ++tb)
+      add(OP_NORM, l, 0, 0, tb, 1, 0, h, {blk(BUF_PX, h, tb, 0, h, 0), blk(BUF_PXN, h, tb, 0, h, 1)});
+    for (int tb = 0; tb < nq; ++tb)
+      for (int fb = 0; fb < 2 * m.ffn / 128; ++fb)
+        add(OP_MGU, l, d.mma_gu + (uint64_t)fb * (h / 64) * chunk, (uint32_t)(h / 64) * chunk, fb, tb, 0, h,
+            {blk(BUF_PXN, h, tb, 0, h, 0), blk(BUF_PH, m.ffn, tb, fb * 64, fb * 64 + 64, 1)});
+    for (int tb = 0; tb < nq; ++tb)
+      for (int fb = 0; fb < h / 128; ++fb)
+        add(OP_MDOWN, l, d.mma_down + (uint64_t)fb * (m.ffn / 64) * chunk, (uint32_t)(m.ffn / 64) * chunk, fb, tb,
+            0, m.ffn, {blk(BUF_PH, m.ffn, tb, 0, m.ffn, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
+  }
+  layer_begin[m.n_layers] = (uint32_t)Tl.size();
+  {
+    std::vector<Access> acc{{BUF_XA, 0, h, 1, -1}};
+    for (int b = 0; b < B; ++b) acc.push_back(blk(BUF_PX, h, (b * T + T - 1) / kTokBlock, 0, h, 0));
+    add(OP_GATHER, m.n_layers, 0, 0, 0, 0, 0, 0, acc);
+  }
+  // LM head + argmax + publish: the decode program's tiles
+  for (const Tile& t : dec.tiles)
+    if (t.op == OP_LMHEAD)
+      add(OP_LMHEAD, m.n_layers, t.w_off, t.w_bytes, t.a0, t.a1, t.a2, t.a3,
+          {{BUF_XA, 0, h, 0, -1}, {BUF_LOGITS, t.a0, t.a0 + t.a1, 1, -1}, {BUF_BEST, 0, 1, 2, -1}});
+  add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0, -1}, {BUF_TOK, 0, 1, 1, -1}});
+  g->algo_weight_bytes = wbytes;
+  if (Tl.size() >= (1u << 31)) return "too many tiles";
+
+  DataflowBuilder df;
+  const int64_t sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1,
+                                    (int64_t)nq * h * TB, (int64_t)nq * h * TB, (int64_t)nq * q_rows * TB,
+                                    (int64_t)m.n_layers * nq * 2 * kv_rows * TB, (int64_t)nq * q_rows * TB,
+                                    (int64_t)nq * m.ffn * TB};
+  for (int b = 0; b < BUF_COUNT; ++b) df.bufs.emplace_back(sizes[b]);
+  g->preds.assign(Tl.size(), {});
+  df.preds_of = &g->preds;
+  g->n_edges = 0;
+  for (size_t t = 0; t < Tl.size(); ++t) {
+    df.apply((int)t, A[t], &g->preds[t]);
+    g->n_edges += (int64_t)g->preds[t].size();
+  }
+  std::unordered_map<std::vector<int>, uint32_t, VecHash> ctr_of;
+  std::vector<std::vector<uint32_t>> sig_of(Tl.size());
+  g->ctr_need.clear();
+  for (size_t t = 0; t < Tl.size(); ++t) {
+    const auto& P = g->preds[t];
+    if (P.empty()) continue;
+    auto it = ctr_of.find(P);
+    uint32_t c;
+    if (it == ctr_of.end()) {
+      c = (uint32_t)g->ctr_need.size();
+      ctr_of.emplace(P, c);
+      g->ctr_need.push_back((uint32_t)P.size());
+      for (int u : P) sig_of[u].push_back(c);
+    } else {
+      c = it->second;
+    }
+    Tl[t].wait_ctr = c;
+    Tl[t].need = g->ctr_need[c];
+  }
+  g->sig.clear();
+  for (size_t t = 0; t < Tl.size(); ++t) {
+    Tl[t].sig_off = (uint32_t)g->sig.size();
+    Tl[t].sig_cnt = (uint32_t)sig_of[t].size();
+    g->sig.insert(g->sig.end(), sig_of[t].begin(), sig_of[t].end());
+  }
+  g->region_begin.assign(1, 0);
+  for (int r = 1; r < p.n_regions; ++r) g->region_begin.push_back(layer_begin[p.region_cut[r]]);
+  g->region_begin.push_back((uint32_t)Tl.size());
+  g->plan.per_op_slot = dec.plan.per_op_slot;
+  return "";
+}
+
+// ---------------------------------------------------------------------------
 std::string verify_graph(const CompiledGraph& g) {
   const size_t n = g.tiles.size();
   if (n > 20000) return "graph too large for the quadratic verifier";
@@ -458,7 +678,7 @@ std::string verify_graph(const CompiledGraph& g) {
   }
   auto reach = [&](int u, int v) { return (anc[(size_t)v * W + u / 64] >> (u % 64)) & 1; };
   // every conflicting access pair must be ordered by a path
-  struct Acc { int t, lo, hi, kind, group; };
+  struct Acc { int t; int64_t lo, hi; int kind, group; };
   std::vector<std::vector<Acc>> per(BUF_COUNT);
   for (size_t t = 0; t < n; ++t)
     for (auto& a : g.access[t]) per[a.buf].push_back({(int)t, a.lo, a.hi, a.kind, a.group});
@@ -492,11 +712,12 @@ int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t
   std::atomic<uint32_t> epochs_done{0};  // the doorbell: step e starts after step e-1 completed
   std::atomic<int> failed{0};
   std::atomic<uint64_t> fail_tile{0};
+  const bool static_sched = g.plan.schedule == WPK_SCHED_STATIC;
   auto worker = [&](int wid) {
     std::mt19937_64 rng(seed * 1000003ull + wid);
-    for (;;) {
+    for (uint64_t i = 0;; ++i) {
       if (failed.load()) return;
-      uint64_t t = head.fetch_add(1);
+      uint64_t t = static_sched ? wid + i * (uint64_t)n_threads : head.fetch_add(1);
       if (t >= total) return;
       uint32_t e = (uint32_t)(t / T) + 1;
       const Tile& tile = g.tiles[t % T];
@@ -575,9 +796,30 @@ std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_
     if (!W.attn_norm || !W.wq || !W.wk || !W.wv || !W.wo || !W.ffn_norm || !W.w_gate || !W.w_up || !W.w_down)
       return fmt("missing weight pointer in layer %lld", l);
   }
+  // tensor-core image: block (r / 128, c / 64) of 128 rows x 64 columns, the
+  // 16-byte unit u of row r stored at unit index u XOR (r % 8)
+  auto mma_row = [&](uint64_t base, int K, int r, const uint16_t* src_row) {
+    const int nkc = K / 64;
+    uint8_t* blk0 = img + base + (uint64_t)(r / 128) * nkc * kMmaChunkBytes;
+    const int rr = r % 128;
+    for (int c = 0; c < nkc; ++c)
+      for (int u = 0; u < 8; ++u)
+        memcpy(blk0 + (uint64_t)c * kMmaChunkBytes + rr * 128 + ((u ^ (rr & 7)) * 16), src_row + c * 64 + u * 8, 16);
+  };
   auto do_layer = [&](int l) {
     const wpk_layer_weights& W = w.layers[l];
     const LayerDev& d = g.lay.layers[l];
+    if (g.lay.mma) {
+      for (int r = 0; r < q_rows; ++r) mma_row(d.mma_qkv, h, rope_phys(r), W.wq + (uint64_t)r * h);
+      for (int r = 0; r < kv_rows; ++r) mma_row(d.mma_qkv, h, q_rows + rope_phys(r), W.wk + (uint64_t)r * h);
+      for (int r = 0; r < kv_rows; ++r) mma_row(d.mma_qkv, h, q_rows + kv_rows + r, W.wv + (uint64_t)r * h);
+      for (int r = 0; r < h; ++r) mma_row(d.mma_wo, q_rows, r, W.wo + (uint64_t)r * q_rows);
+      for (int j = 0; j < m.ffn; ++j) {
+        mma_row(d.mma_gu, h, 2 * j, W.w_gate + (uint64_t)j * h);
+        mma_row(d.mma_gu, h, 2 * j + 1, W.w_up + (uint64_t)j * h);
+      }
+      for (int r = 0; r < h; ++r) mma_row(d.mma_down, m.ffn, r, W.w_down + (uint64_t)r * m.ffn);
+    }
     gain(W.attn_norm, d.attn_norm);
     gain(W.ffn_norm, d.ffn_norm);
     for (int r = 0; r < q_rows; ++r) row(W.wq, d.qkv, rope_phys(r), r, h);

@@ -14,8 +14,9 @@ struct Plan {
   int region_cut[4];
   int trace;
   uint64_t wait_timeout_ns;
-  int slot_bytes, tile_bytes, split_pages, lookahead;
+  int slot_bytes, tile_bytes, split_pages, lookahead, schedule;
   int act_bytes;        // activation staging per worker (fp32)
+  int prefill_mode;     // 1 = tensor-core prefill program, 2 = token by token
   int per_op_slot;      // ring bytes of a per-op CTA (holds one whole tile)
 };
 
@@ -24,6 +25,7 @@ struct Layout {
   uint64_t final_norm = 0, embed = 0, lm_head = 0;
   uint64_t total = 0;
   int down_kc = 0, n_down_chunks = 0;
+  bool mma = false;     // tensor-core image present
 };
 
 struct CompiledGraph {
@@ -40,11 +42,15 @@ struct CompiledGraph {
   int64_t n_edges = 0;
   int64_t algo_weight_bytes = 0;              // weight bytes a step reads
   int n_splits = 0, split_tokens = 0, max_blocks = 0;
+  int B = 0, T = 0, M = 0, n_tb = 0;  // prefill programs
 };
 
 // Returns "" on success, else an error message; *code receives the WPK code.
 std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan* out, int* code);
 std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code);
+// Prefill program for B sequences of T prompt tokens, over the decode graph's
+// weight layout (which must include the tensor-core image).
+std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, CompiledGraph* g);
 std::string verify_graph(const CompiledGraph& g);
 int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t seed, int wait_ms,
                    int stuck_tile, int32_t* done_order, std::string* msg);

@@ -14,7 +14,7 @@ namespace wpk {
 
 constexpr int kMmaChunkK = 64;                 // K elements per chunk (one 128-byte row)
 constexpr int kMmaABytes = 128 * 128;          // A bytes per chunk
-constexpr int kMaxStages = 6;
+
 
 struct MmaRing {
   uint8_t* base;      // stage s at base + s * stage_bytes (1024-aligned)

@@ -156,3 +156,11 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t
 }
 
 }  // namespace wpk
+
+namespace wpk {
+// Order generic-proxy global writes this thread has observed (through an
+// acquire) before its later async-proxy (bulk copy) reads of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+}  // namespace wpk

@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "mma.cuh"
 #include "ptx.cuh"
 #include "wpk_internal.h"
 
@@ -48,6 +49,7 @@ struct TQEntry {  // producer -> consumers, one per tile held by the worker
   int32_t n_chunks;
   int32_t rows_per_chunk;
   uint32_t ev_issue;  // event clock when its first copy was issued (trace)
+  uint64_t t_claim, t_issued;  // trace timestamps
 };
 
 struct Shared {
@@ -59,12 +61,13 @@ struct Shared {
   uint64_t* empty;   // [n_stages]
   uint64_t* tq_full;   // [kMaxQueue]
   uint64_t* tq_empty;  // [kMaxQueue]
+  uint64_t* acc;       // tensor-core accumulator ready
 };
 
 __device__ __forceinline__ Shared carve(uint8_t* base, const KParams& P) {
   Shared s;
   s.ring = base;
-  uint8_t* p = base + (size_t)P.n_stages * kStageBytes;
+  uint8_t* p = base + (size_t)P.n_stages * P.stage_bytes;
   s.act = reinterpret_cast<float*>(p);
   p += P.act_bytes;
   s.out = reinterpret_cast<float*>(p);
@@ -75,6 +78,7 @@ __device__ __forceinline__ Shared carve(uint8_t* base, const KParams& P) {
   s.empty = s.full + kMaxStages;
   s.tq_full = s.empty + kMaxStages;
   s.tq_empty = s.tq_full + kMaxQueue;
+  s.acc = s.tq_empty + kMaxQueue;
   return s;
 }
 
@@ -181,9 +185,28 @@ __device__ __forceinline__ AttnSpan attn_span(const KParams& P, const Tile& T) {
 // ---------------------------------------------------------------------------
 // Producer side: how a tile's staging data is cut into chunks, and the copies.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ bool is_mma_op(int op) { return op >= OP_MQKV && op <= OP_MDOWN; }
+
+// Prefill attention: queries [t0, t1) of sequence b read keys [0, t1).
+__device__ __forceinline__ void pattn_span(const KParams& P, const Tile& T, int* t0, int* t1) {
+  const int qb_tokens = kTokBlock / P.group;
+  *t0 = T.a2 * qb_tokens;
+  *t1 = min(P.T, *t0 + qb_tokens);
+}
+
 __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int* n_chunks, int* rpc) {
   *rpc = 0;
   *n_chunks = 0;
+  if (is_mma_op(T.op)) {
+    *n_chunks = T.a3 / 64;
+    return;
+  }
+  if (T.op == OP_PATTN) {
+    int t0, t1;
+    pattn_span(P, T, &t0, &t1);
+    *n_chunks = (t1 - 1) / P.page_tokens + 1;
+    return;
+  }
   if (T.op == OP_ATTN) {
     if (T.a0 >= active_batch(P)) return;
     const AttnSpan s = attn_span(P, T);
@@ -191,14 +214,43 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
     return;
   }
   if (T.w_bytes == 0) return;
-  int r = kStageBytes / (T.a3 * 2);
+  int r = P.stage_bytes / (T.a3 * 2);
   r &= ~1;  // even: RoPE and gate/up row pairs never straddle a chunk
   *rpc = r < 2 ? 2 : r;
   *n_chunks = (T.a1 + *rpc - 1) / *rpc;
 }
 
+// Source image (hi; lo follows) of a tensor-core tile's activations.
+__device__ __forceinline__ const uint8_t* mma_act_src(const KParams& P, const Tile& T, int part) {
+  const uint8_t* const* img = (T.op == OP_MO) ? P.att_img : (T.op == OP_MDOWN) ? P.h_img : P.xn_img;
+  return img[part] + ((size_t)T.a1 * (T.a3 / 64)) * kMmaChunkBytes;
+}
+
+// Tensor-core tile chunk k: arm the barrier with all its bytes and copy the
+// weight block (the activation blocks follow in issue_mma_act).
+__device__ void issue_mma_w(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
+  mbar_arrive_expect_tx(bar, 3u * kMmaChunkBytes);
+  bulk_g2s(dst, P.weights + T.w_off + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
+}
+__device__ void issue_mma_act(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
+  bulk_g2s(dst + kMmaChunkBytes, mma_act_src(P, T, 0) + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
+  bulk_g2s(dst + 2 * kMmaChunkBytes, mma_act_src(P, T, 1) + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
+}
+
 // Copies of chunk `k` of tile T into `dst`; arms `bar` with their bytes.
 __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uint8_t* dst, uint64_t* bar) {
+  if (T.op == OP_PATTN) {  // one KV page (K rows then V rows) of sequence T.a0, kv head T.a1
+    int t0, t1;
+    pattn_span(P, T, &t0, &t1);
+    const int page = P.page_tokens, hd = P.head_dim;
+    const int rows = min(page, t1 - k * page);
+    const uint32_t bytes = (uint32_t)rows * hd * 2;
+    const int blk = P.block_table[T.a0 * P.max_blocks + k];
+    mbar_arrive_expect_tx(bar, 2 * bytes);
+    bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, T.a1, 0), bytes, bar);
+    bulk_g2s(dst + (size_t)page * hd * 2, P.kv + kv_index(P, T.layer, blk, 1, T.a1, 0), bytes, bar);
+    return;
+  }
   if (T.op == OP_ATTN) {
     const AttnSpan s = attn_span(P, T);
     const int page = P.page_tokens, hd = P.head_dim;
@@ -225,63 +277,34 @@ __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uin
 }
 
 // ---------------------------------------------------------------------------
-// GEMV (CUDA cores).  Work item = (row, 256-column segment): each lane reads
-// 16 contiguous bytes of the row (a warp reads 512 contiguous bytes) and the
-// matching activations from shared memory.
+// GEMV (CUDA cores).  A work item is one row (or one part of a row's 256-column
+// segments when a chunk has fewer rows than warps): each lane reads 16
+// contiguous weight bytes per segment (a warp reads 512 contiguous bytes),
+// accumulates across its segments in registers and reduces once.
+// Activations are staged lane-permuted - element k = 256*seg + 8*lane + 4*h + e
+// lives at 256*seg + 128*h + 4*lane + e - so each float4 read of a warp is 512
+// contiguous bytes (no bank conflicts).  Per token the staged row is padded to
+// whole segments (act_stride floats).
 // ---------------------------------------------------------------------------
-template <int BG>
-__device__ __forceinline__ void gemv_items(const uint8_t* chunk, int K, int rows, int row_base, const float* act,
-                                           float* out, int bg) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int segs = (K + 255) >> 8;
-  const int n_items = rows * segs;
-  const size_t row_bytes = (size_t)K * 2;
-  for (int it = warp; it < n_items; it += kWarps) {
-    const int row = it / segs;
-    const int k = (it % segs) * 256 + lane * 8;
-    float acc[BG];
-#pragma unroll
-    for (int b = 0; b < BG; ++b) acc[b] = 0.f;
-    if (k < K) {
-      const uint4 w = *reinterpret_cast<const uint4*>(chunk + row * row_bytes + (size_t)k * 2);
-      float wf[8];
-      unpack8(w, wf);
-#pragma unroll
-      for (int b = 0; b < BG; ++b) {
-        if (BG > 4 && b >= bg) break;
-        const float4 a0 = *reinterpret_cast<const float4*>(act + b * K + k);
-        const float4 a1 = *reinterpret_cast<const float4*>(act + b * K + k + 4);
-        float s = wf[0] * a0.x;
-        s = fmaf(wf[1], a0.y, s);
-        s = fmaf(wf[2], a0.z, s);
-        s = fmaf(wf[3], a0.w, s);
-        s = fmaf(wf[4], a1.x, s);
-        s = fmaf(wf[5], a1.y, s);
-        s = fmaf(wf[6], a1.z, s);
-        s = fmaf(wf[7], a1.w, s);
-        acc[b] = s;
-      }
-    }
-#pragma unroll
-    for (int b = 0; b < BG; ++b) acc[b] = warp_sum(acc[b]);
-    if (lane == 0) {
-#pragma unroll
-      for (int b = 0; b < BG; ++b) atomicAdd(&out[(row_base + row) * kMaxGemvBatch + b], acc[b]);
-    }
-  }
+__device__ __forceinline__ int act_stride(int K) { return (K + 255) & ~255; }
+
+__device__ __forceinline__ int act_pos(int k) {
+  return (k & ~255) | (((k >> 2) & 1) << 7) | (((k >> 3) & 31) << 2) | (k & 3);
 }
 
-// Copy bg rows of K floats (row stride `stride`) into act; optionally
-// RMS-normalise each row and multiply by `gain` (then K is the whole row).
+// Stage bg rows of K floats (row stride `stride`) into act, lane-permuted;
+// optionally RMS-normalise each row and multiply by `gain` (then K is the whole
+// row).
 __device__ void stage_act(const float* src, int stride, int K, int bg, const float* gain, float eps, float* act) {
   __shared__ float red[kWarps][kMaxGemvBatch];
   __shared__ float scale_s[kMaxGemvBatch];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Kp = act_stride(K);
   for (int b = 0; b < bg; ++b) {
     float ss = 0.f;
     for (int k = threadIdx.x * 4; k < K; k += kThreads * 4) {
       const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)b * stride + k));
-      *reinterpret_cast<float4*>(act + b * K + k) = v;
+      *reinterpret_cast<float4*>(act + b * Kp + act_pos(k)) = v;
       ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
     }
     if (gain) {
@@ -301,7 +324,7 @@ __device__ void stage_act(const float* src, int stride, int K, int bg, const flo
     for (int b = 0; b < bg; ++b) {
       const float sc = scale_s[b];
       for (int k = threadIdx.x * 4; k < K; k += kThreads * 4) {
-        float4* a = reinterpret_cast<float4*>(act + b * K + k);
+        float4* a = reinterpret_cast<float4*>(act + b * Kp + act_pos(k));
         const float4 gg = __ldg(reinterpret_cast<const float4*>(gain + k));
         float4 v = *a;
         v.x *= sc * gg.x;
@@ -412,6 +435,8 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
   }
 }
 
+__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, volatile int* abort);
+
 // Consumer-side chunk cursor: chunk c lives in stage c % n_stages and is the
 // (c / n_stages)-th use of that stage.
 struct Cursor {
@@ -421,11 +446,74 @@ struct Cursor {
 struct ConsumerState {
   int act_key;      // (op, layer, k0) of the staged activation, or kNoAct
   uint32_t last_ctr;  // counter known satisfied in this launch
+  uint32_t acc_phase;  // parity of the accumulator barrier
 };
+
+__shared__ uint32_t s_tmem;  // TMEM base address (tensor-core programs)
+__shared__ int s_mma_ok;
+
+__shared__ uint64_t s_t_data;  // trace: when the tile's last chunk had landed
 
 __device__ __forceinline__ int act_key_of(const Tile& T) { return (int)T.op | ((int)T.layer << 4) | (T.a2 << 12); }
 
-// GEMV tile body.  Returns false on a wait failure.
+// Rows [r_lo, r_hi) of a GEMV tile, computed by one warp: two rows at a time
+// share each activation load; the row's dot product stays in the warp (one
+// shuffle reduction per row, no shared-memory atomics).
+template <int BG>
+__device__ __forceinline__ void gemv_rows(const KParams& P, const Shared& S, uint32_t c0, int rpc, int K, int r_lo,
+                                          int r_hi, const float* act, float* out, int bg) {
+  const int lane = threadIdx.x & 31;
+  const int segs = (K + 255) >> 8;
+  const int Kp = act_stride(K);
+  const size_t row_bytes = (size_t)K * 2;
+  auto row_ptr = [&](int r) {
+    const int k = r / rpc;
+    const uint32_t c = c0 + k;
+    return S.ring + (size_t)(c % P.n_stages) * P.stage_bytes + (size_t)(r - k * rpc) * row_bytes;
+  };
+  for (int r = r_lo; r < r_hi; r += 2) {
+    const bool two = r + 1 < r_hi;
+    const uint8_t* w0 = row_ptr(r);
+    const uint8_t* w1 = two ? row_ptr(r + 1) : w0;
+    float acc0[BG], acc1[BG];
+#pragma unroll
+    for (int b = 0; b < BG; ++b) acc0[b] = acc1[b] = 0.f;
+    for (int seg = 0; seg < segs; ++seg) {
+      const int k = seg * 256 + lane * 8;
+      if (k >= K) continue;
+      float f0[8], f1[8];
+      unpack8(*reinterpret_cast<const uint4*>(w0 + (size_t)k * 2), f0);
+      unpack8(*reinterpret_cast<const uint4*>(w1 + (size_t)k * 2), f1);
+      const float* ap = act + seg * 256 + lane * 4;
+#pragma unroll
+      for (int b = 0; b < BG; ++b) {
+        if (BG > 4 && b >= bg) break;
+        const float4 a0 = *reinterpret_cast<const float4*>(ap + b * Kp);
+        const float4 a1 = *reinterpret_cast<const float4*>(ap + b * Kp + 128);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc0[b] = fmaf(f0[e], av[e], acc0[b]);
+          acc1[b] = fmaf(f1[e], av[e], acc1[b]);
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < BG; ++b) {
+      if (BG > 4 && b >= bg) break;
+      const float s0 = warp_sum(acc0[b]);
+      const float s1 = warp_sum(acc1[b]);
+      if (lane == 0) {
+        out[r * kMaxGemvBatch + b] = s0;
+        if (two) out[(r + 1) * kMaxGemvBatch + b] = s1;
+      }
+    }
+  }
+}
+
+// GEMV tile body.  Each warp owns a contiguous range of the tile's rows and
+// waits only for the stages that hold them; the stages are released together
+// once every warp is done.  Returns false on a wait failure.
 __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks, int rpc,
                           ConsumerState& cs, volatile int* abort) {
   const int K = T.a3, R = T.a1;
@@ -441,7 +529,7 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
     case OP_DOWN: src = P.hbuf + T.a2; stride = P.ffn; break;
     case OP_LMHEAD: gain = reinterpret_cast<const float*>(P.weights + P.final_norm_off); src = P.xa; stride = P.hidden; break;
   }
-  int bgmax = P.act_bytes / (K * 4);
+  int bgmax = P.act_bytes / (act_stride(K) * 4);
   if (bgmax > kMaxGemvBatch) bgmax = kMaxGemvBatch;
   const bool one_group = nb <= bgmax;
   if (one_group) {
@@ -453,49 +541,35 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
   } else {
     cs.act_key = kNoAct;
   }
-  for (int i = threadIdx.x; i < R * kMaxGemvBatch; i += kThreads) S.out[i] = 0.f;
-  cbar();
+  const int warp = threadIdx.x >> 5;
+  const int per = (R + kWarps - 1) / kWarps;
+  const int r_lo = min(R, warp * per), r_hi = min(R, r_lo + per);
   bool ok = true;
-  for (int k = 0; k < n_chunks; ++k, ++cur.c) {
-    const int s = cur.c % P.n_stages;
-    const uint32_t par = (cur.c / P.n_stages) & 1u;
-    if (!wait_phase(P, &S.full[s], par, abort, T.a0)) ok = false;
-    if (!cbar_and(ok)) return false;
-    const uint8_t* chunk = S.ring + (size_t)s * kStageBytes;
-    const int r0 = k * rpc, rows = min(rpc, R - r0);
-    for (int b0 = 0; b0 < nb; b0 += bgmax) {
-      const int bg = min(bgmax, nb - b0);
-      if (!one_group) stage_act(src + (size_t)b0 * stride, stride, K, bg, gain, P.eps, S.act);
-      float* out = S.out + (one_group ? 0 : 0);
-      // outputs of token b0+b accumulate at column b (one group) or are
-      // flushed per group below
-      switch (bg) {
-        case 1: gemv_items<1>(chunk, K, rows, r0, S.act, out, bg); break;
-        case 2: gemv_items<2>(chunk, K, rows, r0, S.act, out, bg); break;
-        case 3: gemv_items<3>(chunk, K, rows, r0, S.act, out, bg); break;
-        case 4: gemv_items<4>(chunk, K, rows, r0, S.act, out, bg); break;
-        default: gemv_items<8>(chunk, K, rows, r0, S.act, out, bg); break;
-      }
-      if (!one_group) {
-        cbar();
-        // epilogue of these rows for this token group, then clear them
-        Tile Tc = T;
-        Tc.a0 = T.a0 + r0;
-        Tc.a1 = rows;
-        epilogue(P, Tc, out + r0 * kMaxGemvBatch, b0, bg);
-        cbar();
-        for (int i = threadIdx.x; i < rows * kMaxGemvBatch; i += kThreads) out[r0 * kMaxGemvBatch + i] = 0.f;
-        cbar();
-      }
+  if (r_lo < r_hi)
+    for (int k = r_lo / rpc; k <= (r_hi - 1) / rpc && ok; ++k) {
+      const uint32_t c = cur.c + k;
+      if (!wait_phase(P, &S.full[c % P.n_stages], (c / P.n_stages) & 1u, abort, T.a0)) ok = false;
+    }
+  if (!cbar_and(ok)) return false;
+  if (P.trace && threadIdx.x == 0) s_t_data = globaltimer();
+  for (int b0 = 0; b0 < nb; b0 += bgmax) {
+    const int bg = min(bgmax, nb - b0);
+    if (!one_group) stage_act(src + (size_t)b0 * stride, stride, K, bg, gain, P.eps, S.act);
+    switch (bg) {
+      case 1: gemv_rows<1>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
+      case 2: gemv_rows<2>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
+      case 3: gemv_rows<3>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
+      case 4: gemv_rows<4>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
+      default: gemv_rows<8>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
     }
     cbar();
-    if (threadIdx.x == 0) mbar_arrive(&S.empty[s]);
+    epilogue(P, T, S.out, b0, bg);
+    cbar();
   }
-  if (one_group) {
-    epilogue(P, T, S.out, 0, nb);
-  }
-  cbar();
-  return ok;
+  if (threadIdx.x == 0)
+    for (int k = 0; k < n_chunks; ++k) mbar_arrive(&S.empty[(cur.c + k) % P.n_stages]);
+  cur.c += n_chunks;
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -522,7 +596,8 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
     const uint32_t par = (cur.c / P.n_stages) & 1u;
     bool ok = wait_phase(P, &Sh.full[st], par, abort, 0xFFFFFFFFu);
     if (!cbar_and(ok)) return false;
-    uint8_t* stage = Sh.ring + (size_t)st * kStageBytes;
+    if (P.trace && threadIdx.x == 0) s_t_data = globaltimer();
+    uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
     const uint16_t* Ks = reinterpret_cast<const uint16_t*>(stage);
     const uint16_t* Vs = reinterpret_cast<const uint16_t*>(stage + (size_t)S * hd * 2);
     // the current token's row was written this step, after the copy was issued
@@ -618,6 +693,332 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   return true;
 }
 
+
+// ---------------------------------------------------------------------------
+// Prefill bodies.  Token row m = b*T + t; block tb holds rows [128 tb, 128 tb + 128).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo_elem, float hi_elem) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ bool body_pembed(const KParams& P, const Tile& T) {
+  const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = P.hidden / 8;
+  for (int n = warp; n < kTokBlock; n += kWarps) {
+    const int m = T.a0 * kTokBlock + n;
+    if (m >= P.M) break;
+    int tok = P.ptok[m];
+    if (tok < 0 || tok >= P.vocab) {
+      if (lane == 0) record_error(P, WPK_ERR_INVALID_ARG, (uint32_t)m, kNoCounter, (uint32_t)tok, (uint32_t)P.vocab);
+      tok = 0;
+    }
+    const uint4* row = reinterpret_cast<const uint4*>(E + (size_t)tok * P.hidden);
+    float4* x = reinterpret_cast<float4*>(P.px + (size_t)m * P.hidden);
+    for (int u = lane; u < units; u += 32) {
+      float f[8];
+      unpack8(__ldg(row + u), f);
+      x[2 * u] = make_float4(f[0], f[1], f[2], f[3]);
+      x[2 * u + 1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+  }
+  return true;
+}
+
+__device__ bool body_gather(const KParams& P) {
+  const int nb = active_batch(P);
+  for (int b = 0; b < nb; ++b) {
+    const float4* src = reinterpret_cast<const float4*>(P.px + ((size_t)b * P.T + P.T - 1) * P.hidden);
+    float4* dst = reinterpret_cast<float4*>(P.xa + (size_t)b * P.hidden);
+    for (int k = threadIdx.x; k < P.hidden / 4; k += kThreads) dst[k] = __ldcg(src + k);
+  }
+  return true;
+}
+
+// RMSNorm of a token block into the hi/lo bf16 image (rows past M become zero).
+__device__ bool body_norm(const KParams& P, const Tile& T) {
+  const LayerDev* L = P.layers + T.layer;
+  const float* gain = reinterpret_cast<const float*>(P.weights + (T.a1 == 0 ? L->attn_norm : L->ffn_norm));
+  const int h = P.hidden, units = h / 8, nkc = h / 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tb = T.a0;
+  uint8_t* hi = P.xn_img[0] + (size_t)tb * nkc * kMmaChunkBytes;
+  uint8_t* lo = P.xn_img[1] + (size_t)tb * nkc * kMmaChunkBytes;
+  constexpr int kMaxUnits = 2048 / 8 / 32;
+  for (int n = warp; n < kTokBlock; n += kWarps) {
+    const int m = tb * kTokBlock + n;
+    const bool valid = m < P.M;
+    float xr[kMaxUnits][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxUnits; ++i) {
+      const int u = lane + 32 * i;
+      if (u < units && valid) {
+        const float4* xs = reinterpret_cast<const float4*>(P.px + (size_t)m * h + 8 * u);
+        const float4 a = __ldcg(xs), b = __ldcg(xs + 1);
+        xr[i][0] = a.x; xr[i][1] = a.y; xr[i][2] = a.z; xr[i][3] = a.w;
+        xr[i][4] = b.x; xr[i][5] = b.y; xr[i][6] = b.z; xr[i][7] = b.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[i][e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += xr[i][e] * xr[i][e];
+    }
+    ss = warp_sum(ss);
+    const float rs = valid ? 1.0f / sqrtf(ss / (float)h + P.eps) : 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxUnits; ++i) {
+      const int u = lane + 32 * i;
+      if (u >= units) continue;
+      const int k = 8 * u;
+      const float4 g0 = __ldg(reinterpret_cast<const float4*>(gain + k));
+      const float4 g1 = __ldg(reinterpret_cast<const float4*>(gain + k + 4));
+      const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float a0 = xr[i][e] * rs * gg[e], a1 = xr[i][e + 1] * rs * gg[e + 1];
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+        const float r0 = a0 - __bfloat162float(hv.x), r1 = a1 - __bfloat162float(hv.y);
+        ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+        pl[e / 2] = pack_bf16x2(r0, r1);
+      }
+      const size_t off = (size_t)(k / 64) * kMmaChunkBytes + sw128_offset(n, k % 64);
+      *reinterpret_cast<uint4*>(hi + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(lo + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    }
+  }
+  return true;
+}
+
+// Tensor-core tile epilogue for 16 token columns n0..n0+15 of feature row fl.
+__device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, const float* v) {
+  const int f = T.a0 * 128 + fl;
+  const int tb = T.a1;
+  const int lane = threadIdx.x & 31;
+  const int hd = P.head_dim, half = hd / 2;
+  switch (T.op) {
+    case OP_MQKV: {
+      const bool is_v = f >= P.q_rows + P.kv_rows;
+      const bool is_q = f < P.q_rows;
+      const int sec = is_q ? f : (is_v ? f - P.q_rows - P.kv_rows : f - P.q_rows);
+      const int head = sec / hd, within = sec % hd;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
+        const int m = tb * kTokBlock + n0 + i;
+        if (m >= P.M) continue;
+        const int b = m / P.T, t = m % P.T;
+        if (is_v) {
+          const int blk = P.block_table[b * P.max_blocks + t / P.page_tokens];
+          P.kv[kv_index(P, T.layer, blk, 1, head, t % P.page_tokens) + within] = f2bf(v[i]);
+          continue;
+        }
+        const int pi = within / 2;
+        const float2 cs = P.rope[(size_t)t * half + pi];
+        const bool even = (lane & 1) == 0;
+        const float y0 = even ? v[i] : partner, y1 = even ? partner : v[i];
+        const float o = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
+        const int dim = even ? pi : pi + half;
+        if (is_q) {
+          P.pq[(size_t)m * P.q_rows + head * hd + dim] = o;
+        } else {
+          const int blk = P.block_table[b * P.max_blocks + t / P.page_tokens];
+          P.kv[kv_index(P, T.layer, blk, 0, head, t % P.page_tokens) + dim] = f2bf(o);
+        }
+      }
+      break;
+    }
+    case OP_MO:
+    case OP_MDOWN: {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int m = tb * kTokBlock + n0 + i;
+        if (m < P.M) P.px[(size_t)m * P.hidden + f] += v[i];
+      }
+      break;
+    }
+    case OP_MGU: {
+      const int j = f / 2, c = j / 64, col = j % 64, nkc = P.ffn / 64;
+      uint8_t* hi = P.h_img[0] + ((size_t)tb * nkc + c) * kMmaChunkBytes;
+      uint8_t* lo = P.h_img[1] + ((size_t)tb * nkc + c) * kMmaChunkBytes;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float up = __shfl_xor_sync(0xffffffffu, v[i], 1);
+        if (lane & 1) continue;
+        const int n = n0 + i;
+        const int m = tb * kTokBlock + n;
+        const float g = v[i];
+        const float hv = (m < P.M) ? g / (1.0f + expf(-g)) * up : 0.f;
+        const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+        const __nv_bfloat16 lb = __float2bfloat16_rn(hv - __bfloat162float(hb));
+        const uint32_t off = sw128_offset(n, col);
+        *reinterpret_cast<__nv_bfloat16*>(hi + off) = hb;
+        *reinterpret_cast<__nv_bfloat16*>(lo + off) = lb;
+      }
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+// Tensor-core tile: D[128 features][128 tokens] = W . (a_hi + a_lo)^T over the
+// tile's K chunks.  Thread 0 issues the MMAs as chunks land and commits each
+// stage back to the producer; all compute warps then read TMEM.
+__device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
+                         ConsumerState& cs, volatile int* abort, uint32_t tile) {
+  const uint32_t tmem = s_tmem;
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    uint32_t cc = cur.c;
+    const uint32_t idesc = idesc_f16(128, kTokBlock, true);
+    for (int k = 0; k < n_chunks; ++k, ++cc) {
+      const int st = cc % P.n_stages;
+      if (!wait_phase(P, &S.full[st], (cc / P.n_stages) & 1u, abort, tile)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t base = smem_u32(S.ring + (size_t)st * P.stage_bytes);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = sdesc_k_sw128(base + kk * 32);
+        umma_f16(tmem, ad, sdesc_k_sw128(base + kMmaChunkBytes + kk * 32), idesc, (k | kk) != 0);
+        umma_f16(tmem, ad, sdesc_k_sw128(base + 2 * kMmaChunkBytes + kk * 32), idesc, 1);
+      }
+      umma_commit(&S.empty[st]);
+    }
+    umma_commit(S.acc);
+    s_mma_ok = ok;
+  }
+  cbar();
+  bool ok = s_mma_ok;
+  if (!wait_phase(P, S.acc, cs.acc_phase, abort, tile)) ok = false;
+  cs.acc_phase ^= 1u;
+  cur.c += n_chunks;
+  if (!cbar_and(ok)) return false;
+  tc_fence_after();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, half = warp >> 2;
+  const int fl = 32 * q + lane;
+  for (int c0 = 0; c0 < kTokBlock / 2; c0 += 16) {
+    float v[16];
+    const int n0 = half * (kTokBlock / 2) + c0;
+    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)n0, v);
+    mma_epilogue(P, T, fl, n0, v);
+  }
+  tc_fence_before();
+  cbar();
+  return true;
+}
+
+// Causal GQA attention for the queries [t0, t1) of sequence b and the query
+// heads of kv head g (online softmax over the staged KV pages, CUDA cores).
+// Thread pair (2r, 2r+1) owns query row r = (query, head) and splits its 64
+// dims in halves; the result goes to the hi/lo attention image.
+__device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
+                           volatile int* abort, uint32_t tile) {
+  const int b = T.a0, g = T.a1, grp = P.group, hd = P.head_dim;
+  int t0, t1;
+  pattn_span(P, T, &t0, &t1);
+  const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
+  const int qi = r / grp, hh = r % grp;
+  const int t = t0 + qi;
+  const bool valid = t < t1;
+  const int m = b * P.T + (valid ? t : t0);
+  const int head = g * grp + hh;
+  const float scale = 1.0f / sqrtf((float)hd);
+  float q[32], o[32];
+  {
+    const float4* qs = reinterpret_cast<const float4*>(P.pq + (size_t)m * P.q_rows + head * hd + 32 * part);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 a = __ldcg(qs + i);
+      q[4 * i] = a.x * scale; q[4 * i + 1] = a.y * scale; q[4 * i + 2] = a.z * scale; q[4 * i + 3] = a.w * scale;
+    }
+  }
+#pragma unroll
+  for (int d = 0; d < 32; ++d) o[d] = 0.f;
+  float mrun = -INFINITY, lrun = 0.f;
+  bool ok = true;
+  for (int k = 0; k < n_chunks; ++k) {
+    const int st = cur.c % P.n_stages;
+    if (!wait_phase(P, &S.full[st], (cur.c / P.n_stages) & 1u, abort, tile)) ok = false;
+    if (!cbar_and(ok)) return false;
+    const uint8_t* stage = S.ring + (size_t)st * P.stage_bytes;
+    const uint32_t* Kw = reinterpret_cast<const uint32_t*>(stage) + 16 * part;
+    const uint32_t* Vw = reinterpret_cast<const uint32_t*>(stage + (size_t)P.page_tokens * hd * 2) + 16 * part;
+    const int rows = min(P.page_tokens, t1 - k * P.page_tokens);
+    for (int j0 = 0; j0 < rows; j0 += 16) {  // 16 keys at a time keeps the scores in registers
+      float sc[16];
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = j0 + jj;
+        float acc = 0.f;
+        if (j < rows) {
+          const uint32_t* kr = Kw + j * (hd / 2);
+#pragma unroll
+          for (int w = 0; w < 16; ++w) {
+            const uint32_t kk = kr[w];
+            acc = fmaf(q[2 * w], __uint_as_float(kk << 16), acc);
+            acc = fmaf(q[2 * w + 1], __uint_as_float(kk & 0xFFFF0000u), acc);
+          }
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        const int key = k * P.page_tokens + j;
+        sc[jj] = (j < rows && key <= t) ? acc : -INFINITY;
+        mloc = fmaxf(mloc, sc[jj]);
+      }
+      const float mnew = fmaxf(mrun, mloc);
+      if (mnew == -INFINITY) continue;
+      const float corr = (mrun > -INFINITY) ? expf(mrun - mnew) : 0.f;
+      lrun *= corr;
+#pragma unroll
+      for (int d = 0; d < 32; ++d) o[d] *= corr;
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) {
+        const float p = (sc[jj] == -INFINITY) ? 0.f : expf(sc[jj] - mnew);
+        lrun += p;
+        const uint32_t* vr = Vw + min(j0 + jj, rows - 1) * (hd / 2);
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          const uint32_t vv = vr[w];
+          o[2 * w] = fmaf(p, __uint_as_float(vv << 16), o[2 * w]);
+          o[2 * w + 1] = fmaf(p, __uint_as_float(vv & 0xFFFF0000u), o[2 * w + 1]);
+        }
+      }
+      mrun = mnew;
+    }
+    cbar();
+    if (threadIdx.x == 0) mbar_arrive(&S.empty[st]);
+    ++cur.c;
+  }
+  if (valid) {
+    const float inv = 1.0f / lrun;
+    const int tb = m / kTokBlock, n = m % kTokBlock, nkc = P.q_rows / 64;
+    const size_t blk = ((size_t)tb * nkc + head) * kMmaChunkBytes;  // 64-column chunk == one head
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float a0 = o[8 * u + e] * inv, a1 = o[8 * u + e + 1] * inv;
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+        ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+        pl[e / 2] = pack_bf16x2(a0 - __bfloat162float(hv.x), a1 - __bfloat162float(hv.y));
+      }
+      const uint32_t off = sw128_offset(n, 32 * part + 8 * u);
+      *reinterpret_cast<uint4*>(P.att_img[0] + blk + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(P.att_img[1] + blk + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    }
+  }
+  return true;
+}
+
 __device__ bool body_embed(const KParams& P) {
   const int nb = active_batch(P);
   const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
@@ -693,12 +1094,19 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       mbar_init(&S.tq_full[i], 1);
       mbar_init(&S.tq_empty[i], 1);
     }
+    mbar_init(S.acc, 1);
     fence_mbar_init();
     s_abort = 0;
     s_prod_chunks = 0;
     s_cons_chunks = 0;
   }
+  if (P.uses_tmem && warp == 0) {
+    tmem_alloc(&s_tmem, kTokBlock);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
 
   if (warp == kWarps) {
     // ------------------------------------------------------------ producer
@@ -711,8 +1119,11 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         uint32_t t;
         if (P.per_op)
           t = (i == 0) ? P.t_begin + blockIdx.x : P.t_end;
+        else if (P.static_sched)
+          t = P.t_begin + blockIdx.x + i * gridDim.x;  // worker w: tickets w, w + W, ...
         else
           t = P.t_begin + atomicAdd(&P.head[P.region], 1u);
+        const uint64_t t_claim = P.trace ? globaltimer() : 0;
         TQEntry& e = S.tq[slot];
         if (t >= P.t_end) {
           e.valid = 0;
@@ -727,19 +1138,52 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         e.n_chunks = nch;
         e.rows_per_chunk = rpc;
         e.ev_issue = P.trace ? atomicAdd(P.evclock, 1u) : 0u;
+        e.t_claim = t_claim;
+        e.t_issued = 0;
         const Tile T = e.tile;
         mbar_arrive(&S.tq_full[slot]);
         bool stop = false;
-        for (int k = 0; k < nch; ++k, ++c) {
-          const int s = c % P.n_stages;
-          const uint32_t use = c / P.n_stages;
-          if (use >= 1 && !wait_phase(P, &S.empty[s], (use - 1) & 1u, &s_abort, t)) {
-            stop = true;
-            break;
-          }
+        auto stage_ptr = [&](uint32_t cc) { return S.ring + (size_t)(cc % P.n_stages) * P.stage_bytes; };
+        auto free_stage = [&](uint32_t cc) {
+          const uint32_t use = cc / P.n_stages;
+          if (use >= 1 && !wait_phase(P, &S.empty[cc % P.n_stages], (use - 1) & 1u, &s_abort, t)) return false;
           fence_proxy_async_smem();
-          issue_chunk(P, T, k, rpc, S.ring + (size_t)s * kStageBytes, &S.full[s]);
+          return true;
+        };
+        if (is_mma_op(T.op)) {
+          // Weights of the first stages are staged before the dependency wait;
+          // the activations are produced inside this program, so they are
+          // copied only after the tile's counter is satisfied.
+          const int pre = min(nch, P.n_stages);
+          const uint32_t c0 = c;
+          for (int k = 0; k < pre && !stop; ++k, ++c) {
+            if (!free_stage(c)) { stop = true; break; }
+            issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
+          }
+          // (per-op launches get their order from the stream; no counters run)
+          if (!stop && !P.per_op && !wait_counter(P, T, t, &s_abort)) stop = true;
+          if (!stop) {
+            fence_proxy_async_global();
+            for (int k = 0; k < pre; ++k) issue_mma_act(P, T, k, stage_ptr(c0 + k), &S.full[(c0 + k) % P.n_stages]);
+          }
+          for (int k = pre; k < nch && !stop; ++k, ++c) {
+            if (!free_stage(c)) { stop = true; break; }
+            issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
+            issue_mma_act(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
+          }
+        } else {
+          if (T.op == OP_PATTN) {  // its KV pages are written inside this program
+            if (!P.per_op && !wait_counter(P, T, t, &s_abort)) stop = true;
+            else fence_proxy_async_global();
+          }
+          for (int k = 0; k < nch && !stop; ++k, ++c) {
+            if (!free_stage(c)) { stop = true; break; }
+            issue_chunk(P, T, k, rpc, stage_ptr(c), &S.full[c % P.n_stages]);
+          }
         }
+        // the entry is still owned by the consumers until they release it;
+        // this plain store is only read for the trace record
+        if (P.trace) *(volatile uint64_t*)&e.t_issued = globaltimer();
         s_prod_chunks = c;
         if (stop) break;
       }
@@ -747,7 +1191,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
   } else {
     // ----------------------------------------------------------- consumers
     Cursor cur{0};
-    ConsumerState cs{kNoAct, kNoCounter};
+    ConsumerState cs{kNoAct, kNoCounter, 0u};
     const int Q = P.per_op ? 1 : P.lookahead;
     __shared__ int s_fail;
     for (uint32_t i = 0;; ++i) {
@@ -761,6 +1205,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       uint32_t ev_start = 0;
       uint64_t t_start = 0;
       if (threadIdx.x == 0) {
+        s_t_data = 0;
         bool ok = true;
         if (!P.per_op && T.wait_ctr != cs.last_ctr) {
           ok = wait_counter(P, T, t, &s_abort);
@@ -781,10 +1226,19 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           case OP_EMBED: ok = body_embed(P); break;
           case OP_ATTN: ok = body_attn(P, T, S, cur, n_chunks, &s_abort); break;
           case OP_FINAL: ok = body_final(P); break;
+          case OP_PEMBED: ok = body_pembed(P, T); break;
+          case OP_GATHER: ok = body_gather(P); break;
+          case OP_NORM: ok = body_norm(P, T); break;
+          case OP_PATTN: ok = body_pattn(P, T, S, cur, n_chunks, &s_abort, t); break;
+          case OP_MQKV:
+          case OP_MO:
+          case OP_MGU:
+          case OP_MDOWN: ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t); break;
           default: ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort); break;
         }
-        // attention tiles use the activation buffer as scratch
-        if (T.op == OP_ATTN) cs.act_key = kNoAct;
+        // attention tiles use the activation buffer as scratch; the gather
+        // rewrites the LM head's input
+        if (T.op == OP_ATTN || T.op == OP_GATHER) cs.act_key = kNoAct;
       }
       ok = cbar_and(ok);
       if (!ok) {
@@ -801,7 +1255,10 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           r.ev_start = ev_start;
           r.ev_done = atomicAdd(P.evclock, 1u);
           r.epoch = P.epoch;
+          r.t_claim_ns = e.t_claim;
+          r.t_issued_ns = *(volatile uint64_t*)&e.t_issued;
           r.t_start_ns = t_start;
+          r.t_data_ns = s_t_data ? s_t_data : t_start;
           r.t_end_ns = globaltimer();
           P.trace_buf[t] = r;
         }
@@ -823,6 +1280,12 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         if (globaltimer() - t0 > P.timeout_ns) break;
     }
   }
+  if (P.uses_tmem) {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(s_tmem, kTokBlock);
+  }
 }
 
 }  // namespace
@@ -840,9 +1303,9 @@ __global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_kernel(const KParam
   worker(P, smem_raw);
 }
 
-size_t worker_smem_bytes(int n_stages, int act_bytes) {
-  return (size_t)n_stages * kStageBytes + act_bytes + kOutFloats * 4 + kMaxQueue * sizeof(TQEntry) +
-         (2 * kMaxStages + 2 * kMaxQueue) * 8;
+size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes) {
+  return (size_t)n_stages * stage_bytes + act_bytes + kOutFloats * 4 + kMaxQueue * sizeof(TQEntry) +
+         (2 * kMaxStages + 2 * kMaxQueue + 1) * 8;
 }
 
 const void* persistent_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_persistent_kernel); }

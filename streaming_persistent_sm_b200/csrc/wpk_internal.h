@@ -30,8 +30,21 @@ enum Op : uint16_t {
   OP_DOWN = 5,     // x += Wd h  (split-K, accumulated)
   OP_LMHEAD = 6,   // fused final RMSNorm + logits + packed argmax
   OP_FINAL = 7,    // publish tokens, reset argmax, advance positions
-  OP_COUNT = 8
+  // prefill program (token blocks of kTokBlock rows; tensor-core tiles)
+  OP_PEMBED = 8,   // X[block] = E[prompt tokens]
+  OP_NORM = 9,     // RMSNorm of X[block] -> bf16 hi/lo activation image
+  OP_MQKV = 10,    // [q;k;v] = W . a on tensor cores, RoPE, q -> Q, k/v -> KV cache
+  OP_MO = 11,      // X += Wo . attn on tensor cores
+  OP_MGU = 12,     // gate/up on tensor cores, SwiGLU -> hi/lo image of h
+  OP_MDOWN = 13,   // X += Wd . h on tensor cores
+  OP_PATTN = 14,   // causal GQA attention of one query block (CUDA cores)
+  OP_GATHER = 15,  // xa[b] = X[last prompt position of b]
+  OP_COUNT = 16
 };
+
+constexpr int kTokBlock = 128;   // tokens per tensor-core tile (the MMA N)
+constexpr int kPrefillQB = 32;   // queries per prefill attention tile
+constexpr int kMmaChunkBytes = 128 * 128;  // 128 rows x 64 bf16, one K chunk
 
 // One tile of the step program, in ticket order.  48 bytes.
 struct alignas(16) Tile {
@@ -55,6 +68,9 @@ struct LayerDev {
   uint64_t wo;          // bf16 [hidden][q_rows]
   uint64_t gu;          // bf16 [2*ffn][hidden], gate/up rows interleaved
   uint64_t down;        // bf16 [n_kchunks][hidden][kc]
+  // tensor-core image: [rows/128][K/64] blocks of 128 rows x 64 columns, each
+  // 16 KB block stored with the 128-byte swizzle (0 when not built)
+  uint64_t mma_qkv, mma_wo, mma_gu, mma_down;
 };
 
 struct TraceRec {
@@ -62,7 +78,7 @@ struct TraceRec {
   uint16_t worker;
   uint16_t op;
   uint32_t ev_issue, ev_start, ev_done, epoch;
-  uint64_t t_start_ns, t_end_ns;
+  uint64_t t_claim_ns, t_issued_ns, t_start_ns, t_data_ns, t_end_ns;
 };
 static_assert(sizeof(TraceRec) == sizeof(wpk_trace_rec), "trace layout");
 
@@ -122,17 +138,33 @@ struct KParams {
   uint32_t epoch;            // counter target multiplier (>= 1)
   int region;
   int per_op;                // 1: one tile per CTA, no queue, no counters
+  int static_sched;          // 1: worker w takes tickets w, w + W, ... (no queue)
+  int stage_bytes;           // bytes per staging-ring stage
+  int uses_tmem;             // the program has tensor-core tiles
+  // prefill program (token rows m = b * T + t, M = B * T, blocks of 128)
+  int M, T, n_tb;
+  const int32_t* ptok;       // prompt tokens [M]
+  float* px;                 // [M][hidden] residual stream
+  float* pq;                 // [M][q_rows] roped queries
+  uint8_t* xn_img[2];        // hi/lo image of the normalised activations [n_tb][hidden/64][16 KB]
+  uint8_t* att_img[2];       // hi/lo image of the attention output     [n_tb][q_rows/64][16 KB]
+  uint8_t* h_img[2];         // hi/lo image of the SwiGLU output        [n_tb][ffn/64][16 KB]
 };
 
 // Host-side compiled graph.
 struct Access {
   int buf;
-  int lo, hi;
+  int64_t lo, hi;
   int kind;        // 0 = read, 1 = write, 2 = accumulate (commutes with itself)
   int group = -1;  // writes with the same group id (>= 0) form one logical write
 };
 
-enum Buf { BUF_XA = 0, BUF_XB, BUF_QKV, BUF_ATTN, BUF_H, BUF_LOGITS, BUF_BEST, BUF_TOK, BUF_COUNT };
+enum Buf {
+  BUF_XA = 0, BUF_XB, BUF_QKV, BUF_ATTN, BUF_H, BUF_LOGITS, BUF_BEST, BUF_TOK,
+  // prefill buffers, modelled per token block (index = block * width * 128 + feature * 128 + row)
+  BUF_PX, BUF_PXN, BUF_PQ, BUF_PKV, BUF_PATT, BUF_PH,
+  BUF_COUNT
+};
 
 struct OpGroup {
   int op, layer;

@@ -26,8 +26,14 @@ WPK_ERR_UNSUPPORTED = -6
 WPK_ERR_POISONED = -7
 WPK_MEGAKERNEL = 0
 WPK_PER_OP_GRAPH = 1
+WPK_SCHED_QUEUE = 0
+WPK_SCHED_STATIC = 1
+WPK_PREFILL_AUTO = 0
+WPK_PREFILL_MMA = 1
+WPK_PREFILL_TOKENWISE = 2
 
-OP_NAMES = ["embed", "qkv", "attn", "o", "gate_up", "down", "lm_head", "final"]
+OP_NAMES = ["embed", "qkv", "attn", "o", "gate_up", "down", "lm_head", "final",
+            "p_embed", "norm", "mma_qkv", "mma_o", "mma_gate_up", "mma_down", "p_attn", "gather"]
 
 _ERR_NAMES = {0: "OK", -1: "INVALID_ARG", -2: "CUDA", -3: "TIMEOUT", -4: "NOT_LOADED", -5: "SHAPE",
               -6: "UNSUPPORTED", -7: "POISONED"}
@@ -50,7 +56,7 @@ class wpk_plan_cfg(C.Structure):
                 ("n_workers", C.c_int), ("workers_per_sm", C.c_int), ("mode", C.c_int), ("resident", C.c_int),
                 ("n_regions", C.c_int), ("region_cut", C.c_int * 4), ("trace", C.c_int),
                 ("wait_timeout_ns", C.c_uint64), ("slot_bytes", C.c_int), ("tile_bytes", C.c_int),
-                ("split_pages", C.c_int), ("lookahead", C.c_int)]
+                ("split_pages", C.c_int), ("lookahead", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int)]
 
 
 _P16 = C.POINTER(C.c_uint16)
@@ -76,9 +82,9 @@ class wpk_error_info(C.Structure):
 
 
 TRACE_DTYPE = np.dtype([("tile", "<u4"), ("worker", "<u2"), ("op", "<u2"), ("ev_issue", "<u4"),
-                        ("ev_start", "<u4"), ("ev_done", "<u4"), ("epoch", "<u4"), ("t_start_ns", "<u8"),
-                        ("t_end_ns", "<u8")])
-assert TRACE_DTYPE.itemsize == 40
+                        ("ev_start", "<u4"), ("ev_done", "<u4"), ("epoch", "<u4"), ("t_claim_ns", "<u8"),
+                        ("t_issued_ns", "<u8"), ("t_start_ns", "<u8"), ("t_data_ns", "<u8"), ("t_end_ns", "<u8")])
+assert TRACE_DTYPE.itemsize == 64
 
 # Every symbol include/wpk.h declares, with its ctypes signature.
 _H = C.c_void_p
@@ -90,6 +96,7 @@ _SIGS = {
     "wpk_prefill": (C.c_int, [_H, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     "wpk_step": (C.c_int, [_H, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "wpk_graph_stats_get": (C.c_int, [_H, C.POINTER(wpk_graph_stats)]),
+    "wpk_select_program": (C.c_int, [_H, C.c_int, C.c_int]),
     "wpk_get_edges": (C.c_int, [_H, C.POINTER(C.c_int32), C.c_int64, C.POINTER(C.c_int64)]),
     "wpk_get_tile_ops": (C.c_int, [_H, C.POINTER(C.c_int32), C.c_int64]),
     "wpk_verify_graph": (C.c_int, [_H]),
@@ -100,6 +107,8 @@ _SIGS = {
     "wpk_destroy": (C.c_int, [_H]),
     "wpk_debug_break_counter": (C.c_int, [_H, C.c_int]),
     "wpk_step_noalloc": (C.c_int, [_H, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "wpk_debug_gemm": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int,
+                                 C.c_void_p]),
 }
 
 _lib = None
@@ -135,10 +144,12 @@ def model_cfg(shape) -> wpk_model_cfg:
 def plan_cfg(max_batch: int, max_context: int, mode: int = WPK_MEGAKERNEL, n_regions: int = 1,
              region_cut: Sequence[int] = (0, 0, 0, 0), trace: int = 0, wait_timeout_ns: int = 0,
              page_tokens: int = 0, n_workers: int = 0, workers_per_sm: int = 0, resident: int = 0,
-             slot_bytes: int = 0, tile_bytes: int = 0, split_pages: int = 0, lookahead: int = 0) -> wpk_plan_cfg:
+             slot_bytes: int = 0, tile_bytes: int = 0, split_pages: int = 0, lookahead: int = 0,
+             schedule: int = 0, prefill: int = 0) -> wpk_plan_cfg:
     cut = (C.c_int * 4)(*list(region_cut) + [0] * (4 - len(region_cut)))
     return wpk_plan_cfg(max_batch, max_context, page_tokens, n_workers, workers_per_sm, mode, resident, n_regions,
-                        cut, trace, wait_timeout_ns, slot_bytes, tile_bytes, split_pages, lookahead)
+                        cut, trace, wait_timeout_ns, slot_bytes, tile_bytes, split_pages, lookahead, schedule,
+                        prefill)
 
 
 # ----------------------------------------------------------- thin wrappers --
@@ -177,6 +188,16 @@ def wpk_step_noalloc(h, in_tok_dev: int = 0, out_tok_dev: int = 0, logits_dev: i
     """wpk_step with the activation scratch in the library's static device array."""
     _check(load_library().wpk_step_noalloc(h, in_tok_dev or None, out_tok_dev or None, logits_dev or None,
                                            stream or None), h)
+
+
+def wpk_debug_gemm(a_img_dev: int, b1_img_dev: int, b2_img_dev: int, d_dev: int, n_chunks: int, N: int,
+                   bf16: bool = True, stream: int = 0):
+    _check(load_library().wpk_debug_gemm(a_img_dev, b1_img_dev, b2_img_dev or None, d_dev, n_chunks, N,
+                                         1 if bf16 else 0, stream or None))
+
+
+def wpk_select_program(h, batch: int = 0, prompt_len: int = 0):
+    _check(load_library().wpk_select_program(h, batch, prompt_len), h)
 
 
 def wpk_graph_stats_get(h) -> dict:

@@ -90,9 +90,9 @@ def test_down_projection_uses_chunk_edges(lib):
         W.wpk_destroy(h)
 
 
-@pytest.mark.parametrize("threads", [1, 3, 17])
-def test_cpu_schedule_simulator_is_deadlock_free(lib, threads):
-    h = _graph(max_batch=2, max_context=128)
+@pytest.mark.parametrize("threads,schedule", [(1, 0), (3, 0), (17, 0), (1, 1), (5, 1), (23, 1)])
+def test_cpu_schedule_simulator_is_deadlock_free(lib, threads, schedule):
+    h = _graph(max_batch=2, max_context=128, schedule=schedule)
     try:
         st = W.wpk_graph_stats_get(h)
         T = st["n_tiles"]
@@ -153,5 +153,38 @@ def test_llama1b_graph_shape(lib):
         bf16_bytes = sum(np.prod(s) * 2 for n, s, k in synth.tensor_specs(synth.LLAMA_1B) if k == "normal")
         # matmul weights and the tied embedding, read once per step (norm gains excluded)
         assert st["weight_bytes"] == bf16_bytes == 2_471_493_632
+    finally:
+        W.wpk_destroy(h)
+
+
+@pytest.mark.parametrize("B,T", [(1, 20), (2, 40), (3, 130)])
+def test_prefill_program_verifies_and_simulates(lib, B, T):
+    h = _graph(max_batch=3, max_context=160)
+    try:
+        W.wpk_select_program(h, B, T)
+        st = W.wpk_graph_stats_get(h)
+        ops = W.wpk_get_tile_ops(h, st["n_tiles"])
+        names = [W.OP_NAMES[o] for o in ops]
+        assert names[0] == "p_embed" and names[-1] == "final" and "mma_qkv" in names and "p_attn" in names
+        W.wpk_verify_graph(h)
+        rc, order = W.wpk_simulate(h, 7, 2, 3, 10000, -1, st["n_tiles"])
+        assert rc == 0, W.wpk_last_error(h)
+        e = W.wpk_get_edges(h)
+        assert np.all(e[:, 0] < e[:, 1])
+        # attention of a later query block waits for the K/V tiles of every earlier token block
+        n_tb = -(-(B * T) // 128)
+        assert ops.tolist().count(W.OP_NAMES.index("norm")) == 2 * synth.TINY.n_layers * n_tb
+        W.wpk_select_program(h, 0, 0)
+        assert W.wpk_graph_stats_get(h)["n_tiles"] != st["n_tiles"]
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_tokenwise_prefill_plan_has_no_prefill_program(lib):
+    h = _graph(prefill=W.WPK_PREFILL_TOKENWISE)
+    try:
+        with pytest.raises(W.WpkError) as ei:
+            W.wpk_select_program(h, 1, 8)
+        assert ei.value.code == W.WPK_ERR_UNSUPPORTED
     finally:
         W.wpk_destroy(h)

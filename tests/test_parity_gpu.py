@@ -38,6 +38,8 @@ PLANS = {
     "small_tiles_one_slot": dict(tile_bytes=4096, slot_bytes=16384, lookahead=1),
     "two_stage_ring": dict(slot_bytes=32768, lookahead=2),
     "split2_page32": dict(page_tokens=32, split_pages=2),
+    "tokenwise_prefill": dict(prefill=W.WPK_PREFILL_TOKENWISE),
+    "static_schedule": dict(schedule=W.WPK_SCHED_STATIC),
 }
 
 
