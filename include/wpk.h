@@ -83,7 +83,8 @@ typedef struct wpk_plan_cfg {
   uint64_t wait_timeout_ns; /* bound on every device wait (0 = 2 s)            */
   int slot_bytes;       /* staging slot per worker, used as a ring of 16 KB
                            chunk stages (0 = 8 stages, 128 KB)                 */
-  int tile_bytes;       /* target weight bytes per tile (0 = 65536)            */
+  int tile_bytes;       /* minimum weight bytes per tile; tiles are sized to give
+                           each worker about one tile per op (0 = 32768)       */
   int split_pages;      /* KV pages per attention split (0 = 1)                */
   int lookahead;        /* tiles a worker may claim and stage ahead of the one
                            it computes (0 = 4); 1 = a tile's weights are staged
@@ -248,7 +249,8 @@ int wpk_get_trace(wpk_handle *h, void *host_buf, size_t bytes);
 /* First device error (code 0 if none).  Synchronizes the device. */
 int wpk_get_error_info(wpk_handle *h, wpk_error_info *info);
 
-/* Human-readable message for the last failing call on this handle. */
+/* Human-readable message for the last failing call on this handle; with
+ * h == NULL, the message of this thread's last failed wpk_build_graph. */
 const char *wpk_last_error(const wpk_handle *h);
 
 /* Stop the resident grid (if any), release library-owned tables, free h. */

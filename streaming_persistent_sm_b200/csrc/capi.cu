@@ -18,6 +18,8 @@ namespace wpk {
 size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes);
 const void* persistent_kernel_ptr();
 const void* per_op_kernel_ptr();
+const void* prefill_kernel_ptr();
+const void* prefill_op_kernel_ptr();
 }  // namespace wpk
 
 using namespace wpk;
@@ -86,6 +88,8 @@ struct wpk_handle {
 };
 
 namespace {
+
+thread_local std::string g_build_error;  // message of the last failed wpk_build_graph
 
 int fail(wpk_handle* h, int code, const std::string& msg) {
   if (h) h->err = msg;
@@ -359,7 +363,7 @@ int launch_prefill(wpk_handle* h, PrefillProgram* prog, const int32_t* tokens, i
       P.t_end = g.region_begin[r + 1];
       P.region = r;
       void* args[] = {&P};
-      CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
+      CUDA_TRY(h, cudaLaunchCooperativeKernel(prefill_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
                                               h->smem_prefill, s));
     }
     return WPK_OK;
@@ -377,7 +381,7 @@ int launch_prefill(wpk_handle* h, PrefillProgram* prog, const int32_t* tokens, i
       P.t_end = og.end;
       P.per_op = 1;
       void* args[] = {&P};
-      cudaError_t err = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
+      cudaError_t err = cudaLaunchKernel(prefill_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
                                          h->smem_prefill, h->capture_stream);
       if (err != cudaSuccess) {
         cudaGraph_t junk = nullptr;
@@ -417,11 +421,21 @@ static int setup_device(wpk_handle* h) {
     if (h->prefill_stages < 2) return fail(h, WPK_ERR_UNSUPPORTED, "no room for the prefill staging ring");
     h->smem_prefill = worker_smem_bytes(h->prefill_stages, 3 * kMmaChunkBytes, p.act_bytes);
   }
-  const size_t smem_max = std::max(h->smem, h->smem_prefill);
+  const size_t smem_max = h->smem;
   CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)smem_max));
   CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)std::max(h->smem_per_op, h->smem_prefill)));
+                                   (int)h->smem_per_op));
+  if (h->smem_prefill) {
+    CUDA_TRY(h, cudaFuncSetAttribute(prefill_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)h->smem_prefill));
+    CUDA_TRY(h, cudaFuncSetAttribute(prefill_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)h->smem_prefill));
+    int per_sm_p = 0;
+    CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreads,
+                                                              h->smem_prefill));
+    if (per_sm_p < 1) return fail(h, WPK_ERR_UNSUPPORTED, "the prefill worker does not fit an SM");
+  }
   int per_sm = 0;
   CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kCtaThreads, smem_max));
   h->n_workers = p.n_workers ? p.n_workers : h->n_sms * p.workers_per_sm;
@@ -486,8 +500,17 @@ int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_ha
   int code = 0;
   Plan p;
   std::string msg = normalize_plan(*model, *plan, &p, &code);
-  if (msg.empty()) msg = compile_graph(*model, p, &h->g, &code);
+  // worker count the tiles are sized for: the plan's, else #SMs x workers per SM
+  int n_dev_w = 0, sms = 148;
+  if (cudaGetDeviceCount(&n_dev_w) == cudaSuccess && n_dev_w > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  cudaGetLastError();
+  const int W = p.n_workers ? p.n_workers : sms * p.workers_per_sm;
+  if (msg.empty()) msg = compile_graph(*model, p, &h->g, &code, W);
   if (!msg.empty()) {
+    g_build_error = msg;
     delete h;
     return code;
   }
@@ -504,6 +527,7 @@ int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_ha
   }
   int rc = setup_device(h);
   if (rc) {
+    g_build_error = h->err;
     if (h->d_base) cudaFree(h->d_base);
     delete h;
     return rc;
@@ -715,7 +739,7 @@ int wpk_get_error_info(wpk_handle* h, wpk_error_info* info) {
   return WPK_OK;
 }
 
-const char* wpk_last_error(const wpk_handle* h) { return h ? h->err.c_str() : "null handle"; }
+const char* wpk_last_error(const wpk_handle* h) { return h ? h->err.c_str() : g_build_error.c_str(); }
 
 int wpk_destroy(wpk_handle* h) {
   if (!h) return WPK_ERR_INVALID_ARG;

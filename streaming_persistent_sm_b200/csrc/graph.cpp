@@ -93,7 +93,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
     p->slot_bytes = std::min(8, budget / kStageBytes) * kStageBytes;
     if (p->slot_bytes < kStageBytes) return "no room for a staging slot";
   }
-  p->tile_bytes = in.tile_bytes ? in.tile_bytes : 65536;
+  p->tile_bytes = in.tile_bytes ? in.tile_bytes : 32768;
   if (p->tile_bytes < 1024 || p->tile_bytes > 1 << 20) return "tile_bytes must be in [1K, 1M]";
   p->split_pages = in.split_pages ? in.split_pages : 1;
   if (p->split_pages < 1) return "split_pages must be >= 1";
@@ -245,22 +245,25 @@ struct VecHash {
   }
 };
 
-// Rows per GEMV tile: about tile_bytes, a multiple of 8, and no more chunk
-// stages than half the staging ring (a GEMV tile releases its stages when it
-// completes, so the ring must hold two tiles for the loads to keep flowing).
-int rows_per_tile(int row_bytes, const Plan& p) {
+// Rows per GEMV tile for an op with `op_rows` rows of `row_bytes`: about
+// 1/W of the op (W workers) so that every worker gets about one tile per op,
+// at least tile_bytes, at most kMaxTileRows, a multiple of the rows per chunk
+// stage.  Chunks stream through the staging ring; only when more than 8
+// sequences force several passes over a tile's chunks must a tile fit the
+// ring.
+int rows_per_tile(int row_bytes, int op_rows, const Plan& p, int W) {
   int rpc = (kStageBytes / row_bytes) & ~1;
   if (rpc < 2) rpc = 2;
-  const int half_ring = std::max(1, p.slot_bytes / kStageBytes / 2);
-  int r = std::min(p.tile_bytes / row_bytes, half_ring * rpc);
-  r &= ~1;  // RoPE and gate/up row pairs stay in one tile
-  if (r < 2) r = 2;
-  return std::min(r, kMaxTileRows);
+  int r = std::max(p.tile_bytes / row_bytes, (op_rows + W - 1) / std::max(1, W));
+  r = (r + rpc - 1) / rpc * rpc;
+  if (p.max_batch > kMaxGemvBatch) r = std::min(r, (p.slot_bytes / kStageBytes) * rpc);
+  r = std::min(r, kMaxTileRows / rpc * rpc);
+  return std::max(r, 2);
 }
 
 }  // namespace
 
-std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code) {
+std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code, int W) {
   *code = WPK_ERR_SHAPE;
   g->m = m;
   g->plan = p;
@@ -345,7 +348,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
     const int attn_group = 1000 + l;
     // fused RMSNorm + QKV + RoPE + KV write; tiles never straddle q/k/v sections
     {
-      int R = rows_per_tile(h * 2, p);
+      int R = rows_per_tile(h * 2, qkv_rows, p, W);
       int sec_lo[3] = {0, q_rows, q_rows + kv_rows}, sec_hi[3] = {q_rows, q_rows + kv_rows, qkv_rows};
       for (int s = 0; s < 3; ++s)
         for (int r0 = sec_lo[s]; r0 < sec_hi[s]; r0 += R) {
@@ -365,7 +368,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
                {BUF_ATTN, gi * grp * hd, (gi + 1) * grp * hd, 1, attn_group}});
     // O projection + residual
     {
-      int R = rows_per_tile(q_rows * 2, p);
+      int R = rows_per_tile(q_rows * 2, h, p, W);
       for (int r0 = 0; r0 < h; r0 += R) {
         int n = std::min(R, h - r0);
         add(OP_O, l, d.wo + (uint64_t)r0 * q_rows * 2, (uint32_t)n * q_rows * 2, r0, n, 0, q_rows,
@@ -374,7 +377,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
     }
     // fused RMSNorm + gate/up + SwiGLU (physical rows: gate j at 2j, up j at 2j+1)
     {
-      int R = rows_per_tile(h * 2, p);
+      int R = rows_per_tile(h * 2, 2 * m.ffn, p, W);
       for (int r0 = 0; r0 < 2 * m.ffn; r0 += R) {
         int n = std::min(R, 2 * m.ffn - r0);
         add(OP_GU, l, d.gu + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n, 0, h,
@@ -383,7 +386,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
     }
     // down projection, split along K into chunks (finer edges), accumulated into x
     {
-      int R = rows_per_tile(kc * 2, p);
+      int R = rows_per_tile(kc * 2, h * nch, p, W);
       for (int c = 0; c < nch; ++c)
         for (int r0 = 0; r0 < h; r0 += R) {
           int n = std::min(R, h - r0);
@@ -394,7 +397,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   }
   layer_begin[m.n_layers] = (uint32_t)T.size();
   {
-    int R = rows_per_tile(h * 2, p);
+    int R = rows_per_tile(h * 2, m.vocab, p, W);
     for (int r0 = 0; r0 < m.vocab; r0 += R) {
       int n = std::min(R, m.vocab - r0);
       add(OP_LMHEAD, m.n_layers, L.lm_head + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n, 0, h,
@@ -410,8 +413,8 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
       const int rpc = std::max(2, (kStageBytes / (t.a3 * 2)) & ~1);
       max_chunks = std::max(max_chunks, (t.a1 + rpc - 1) / rpc);
     }
-  // larger tiles stream through the ring
-  g->plan.per_op_slot = std::min(max_chunks, kMaxStages) * kStageBytes;
+  // a per-op CTA streams its tile through a ring no larger than a worker's
+  g->plan.per_op_slot = std::min(max_chunks * kStageBytes, p.slot_bytes);
   if (T.size() >= (1u << 31)) return "too many tiles";
 
   // ---- edges from dataflow ----

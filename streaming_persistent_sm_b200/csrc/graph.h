@@ -47,7 +47,9 @@ struct CompiledGraph {
 
 // Returns "" on success, else an error message; *code receives the WPK code.
 std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan* out, int* code);
-std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code);
+// W: number of worker CTAs the program will run on (tiles are sized so each
+// worker gets about one tile per op).
+std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code, int W);
 // Prefill program for B sequences of T prompt tokens, over the decode graph's
 // weight layout (which must include the tensor-core image).
 std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, CompiledGraph* g);

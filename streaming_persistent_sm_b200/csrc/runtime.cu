@@ -40,6 +40,8 @@ namespace wpk {
 namespace {
 
 constexpr int kOutFloats = kMaxTileRows * kMaxGemvBatch;  // GEMV partial outputs [row][8]
+constexpr int kSigQueue = 8;                               // finished tiles awaiting their signals
+constexpr uint32_t kSigStop = 0xFFFFFFFFu;
 constexpr int kNoAct = -1;
 
 struct TQEntry {  // producer -> consumers, one per tile held by the worker
@@ -62,6 +64,9 @@ struct Shared {
   uint64_t* tq_full;   // [kMaxQueue]
   uint64_t* tq_empty;  // [kMaxQueue]
   uint64_t* acc;       // tensor-core accumulator ready
+  uint64_t* sig_full;  // [kSigQueue] consumers -> signaller
+  uint64_t* sig_empty; // [kSigQueue] signaller -> consumers
+  uint2* sig_req;      // [kSigQueue] (sig_off, sig_cnt) of a finished tile
 };
 
 __device__ __forceinline__ Shared carve(uint8_t* base, const KParams& P) {
@@ -79,6 +84,9 @@ __device__ __forceinline__ Shared carve(uint8_t* base, const KParams& P) {
   s.tq_full = s.empty + kMaxStages;
   s.tq_empty = s.tq_full + kMaxQueue;
   s.acc = s.tq_empty + kMaxQueue;
+  s.sig_full = s.acc + 1;
+  s.sig_empty = s.sig_full + kSigQueue;
+  s.sig_req = reinterpret_cast<uint2*>(s.sig_empty + kSigQueue);
   return s;
 }
 
@@ -144,14 +152,18 @@ __device__ void record_error(const KParams& P, int code, uint32_t tile, uint32_t
 }
 
 // Bounded wait on an mbarrier phase.  `abort` (shared) ends the wait early.
-__device__ bool wait_phase(const KParams& P, uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t tile) {
+// `slack` multiplies the bound: the producer's and signaller's waits only
+// idle behind the compute warps, so they give up later than any wait of the
+// compute warps and the error word names the wait that actually stalled.
+__device__ bool wait_phase(const KParams& P, uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t tile,
+                           uint32_t slack = 1) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > P.timeout_ns) {
+      if (globaltimer() - t0 > P.timeout_ns * slack) {
         record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, 0, 0);
         *abort = 1;
         return false;
@@ -456,34 +468,32 @@ __shared__ uint64_t s_t_data;  // trace: when the tile's last chunk had landed
 
 __device__ __forceinline__ int act_key_of(const Tile& T) { return (int)T.op | ((int)T.layer << 4) | (T.a2 << 12); }
 
-// Rows [r_lo, r_hi) of a GEMV tile, computed by one warp: two rows at a time
-// share each activation load; the row's dot product stays in the warp (one
-// shuffle reduction per row, no shared-memory atomics).
+// One staged chunk of a GEMV tile (rows [0, rows) of the chunk, rows <= 4 at
+// a time share each activation load), computed by one warp.  The row's dot
+// product stays in the warp: one shuffle reduction per row, plain stores.
 template <int BG>
-__device__ __forceinline__ void gemv_rows(const KParams& P, const Shared& S, uint32_t c0, int rpc, int K, int r_lo,
-                                          int r_hi, const float* act, float* out, int bg) {
+__device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int K, int rows, int row_base, const float* act,
+                                           float* out, int bg) {
   const int lane = threadIdx.x & 31;
   const int segs = (K + 255) >> 8;
   const int Kp = act_stride(K);
   const size_t row_bytes = (size_t)K * 2;
-  auto row_ptr = [&](int r) {
-    const int k = r / rpc;
-    const uint32_t c = c0 + k;
-    return S.ring + (size_t)(c % P.n_stages) * P.stage_bytes + (size_t)(r - k * rpc) * row_bytes;
-  };
-  for (int r = r_lo; r < r_hi; r += 2) {
-    const bool two = r + 1 < r_hi;
-    const uint8_t* w0 = row_ptr(r);
-    const uint8_t* w1 = two ? row_ptr(r + 1) : w0;
-    float acc0[BG], acc1[BG];
+  constexpr int RG = (BG <= 2) ? 4 : 2;  // rows per pass
+  for (int r0 = 0; r0 < rows; r0 += RG) {
+    const int nr = min(RG, rows - r0);
+    float acc[RG][BG];
 #pragma unroll
-    for (int b = 0; b < BG; ++b) acc0[b] = acc1[b] = 0.f;
+    for (int i = 0; i < RG; ++i)
+#pragma unroll
+      for (int b = 0; b < BG; ++b) acc[i][b] = 0.f;
     for (int seg = 0; seg < segs; ++seg) {
       const int k = seg * 256 + lane * 8;
       if (k >= K) continue;
-      float f0[8], f1[8];
-      unpack8(*reinterpret_cast<const uint4*>(w0 + (size_t)k * 2), f0);
-      unpack8(*reinterpret_cast<const uint4*>(w1 + (size_t)k * 2), f1);
+      float f[RG][8];
+#pragma unroll
+      for (int i = 0; i < RG; ++i)
+        unpack8(*reinterpret_cast<const uint4*>(chunk + (size_t)(r0 + min(i, nr - 1)) * row_bytes + (size_t)k * 2),
+                f[i]);
       const float* ap = act + seg * 256 + lane * 4;
 #pragma unroll
       for (int b = 0; b < BG; ++b) {
@@ -492,28 +502,26 @@ __device__ __forceinline__ void gemv_rows(const KParams& P, const Shared& S, uin
         const float4 a1 = *reinterpret_cast<const float4*>(ap + b * Kp + 128);
         const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          acc0[b] = fmaf(f0[e], av[e], acc0[b]);
-          acc1[b] = fmaf(f1[e], av[e], acc1[b]);
-        }
+        for (int i = 0; i < RG; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[i][b] = fmaf(f[i][e], av[e], acc[i][b]);
       }
     }
 #pragma unroll
-    for (int b = 0; b < BG; ++b) {
-      if (BG > 4 && b >= bg) break;
-      const float s0 = warp_sum(acc0[b]);
-      const float s1 = warp_sum(acc1[b]);
-      if (lane == 0) {
-        out[r * kMaxGemvBatch + b] = s0;
-        if (two) out[(r + 1) * kMaxGemvBatch + b] = s1;
+    for (int i = 0; i < RG; ++i)
+#pragma unroll
+      for (int b = 0; b < BG; ++b) {
+        if (BG > 4 && b >= bg) break;
+        const float v = warp_sum(acc[i][b]);
+        if (lane == 0 && i < nr) out[(row_base + r0 + i) * kMaxGemvBatch + b] = v;
       }
-    }
   }
 }
 
-// GEMV tile body.  Each warp owns a contiguous range of the tile's rows and
-// waits only for the stages that hold them; the stages are released together
-// once every warp is done.  Returns false on a wait failure.
+// GEMV tile body.  Chunk k of the tile belongs to warp k % 8: the warp waits
+// for that stage only, computes its rows and hands the stage back at once, so
+// a tile of any size streams through the ring and no block barrier is taken
+// per chunk.  Returns false on a wait failure.
 __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks, int rpc,
                           ConsumerState& cs, volatile int* abort) {
   const int K = T.a3, R = T.a1;
@@ -531,43 +539,47 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
   }
   int bgmax = P.act_bytes / (act_stride(K) * 4);
   if (bgmax > kMaxGemvBatch) bgmax = kMaxGemvBatch;
-  const bool one_group = nb <= bgmax;
-  if (one_group) {
-    const int key = act_key_of(T);
-    if (cs.act_key != key) {
-      stage_act(src, stride, K, nb, gain, P.eps, S.act);
-      cs.act_key = key;
-    }
-  } else {
-    cs.act_key = kNoAct;
-  }
-  const int warp = threadIdx.x >> 5;
-  const int per = (R + kWarps - 1) / kWarps;
-  const int r_lo = min(R, warp * per), r_hi = min(R, r_lo + per);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   bool ok = true;
-  if (r_lo < r_hi)
-    for (int k = r_lo / rpc; k <= (r_hi - 1) / rpc && ok; ++k) {
+  for (int b0 = 0; b0 < nb || (nb == 0 && b0 == 0); b0 += bgmax) {
+    const int bg = max(0, min(bgmax, nb - b0));
+    const bool last_group = b0 + bgmax >= nb;
+    if (bg > 0) {
+      const int key = (b0 == 0 && last_group) ? act_key_of(T) : kNoAct;
+      if (key == kNoAct || cs.act_key != key) {
+        stage_act(src + (size_t)b0 * stride, stride, K, bg, gain, P.eps, S.act);
+        cs.act_key = key;
+      }
+    }
+    for (int k = warp; k < n_chunks; k += kWarps) {
       const uint32_t c = cur.c + k;
-      if (!wait_phase(P, &S.full[c % P.n_stages], (c / P.n_stages) & 1u, abort, T.a0)) ok = false;
+      const int st = c % P.n_stages;
+      // the stage is waited for on the first token group only
+      if (b0 == 0 && !wait_phase(P, &S.full[st], (c / P.n_stages) & 1u, abort, T.a0)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* chunk = S.ring + (size_t)st * P.stage_bytes;
+      const int r0 = k * rpc, rows = min(rpc, R - r0);
+      switch (bg) {
+        case 0: break;
+        case 1: gemv_chunk<1>(chunk, K, rows, r0, S.act, S.out, bg); break;
+        case 2: gemv_chunk<2>(chunk, K, rows, r0, S.act, S.out, bg); break;
+        case 3: gemv_chunk<3>(chunk, K, rows, r0, S.act, S.out, bg); break;
+        case 4: gemv_chunk<4>(chunk, K, rows, r0, S.act, S.out, bg); break;
+        default: gemv_chunk<8>(chunk, K, rows, r0, S.act, S.out, bg); break;
+      }
+      if (last_group) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[st]);
+      }
     }
-  if (!cbar_and(ok)) return false;
-  if (P.trace && threadIdx.x == 0) s_t_data = globaltimer();
-  for (int b0 = 0; b0 < nb; b0 += bgmax) {
-    const int bg = min(bgmax, nb - b0);
-    if (!one_group) stage_act(src + (size_t)b0 * stride, stride, K, bg, gain, P.eps, S.act);
-    switch (bg) {
-      case 1: gemv_rows<1>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
-      case 2: gemv_rows<2>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
-      case 3: gemv_rows<3>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
-      case 4: gemv_rows<4>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
-      default: gemv_rows<8>(P, S, cur.c, rpc, K, r_lo, r_hi, S.act, S.out, bg); break;
-    }
+    if (!cbar_and(ok)) return false;
+    if (P.trace && threadIdx.x == 0 && b0 == 0) s_t_data = globaltimer();
+    if (bg > 0) epilogue(P, T, S.out, b0, bg);
     cbar();
-    epilogue(P, T, S.out, b0, bg);
-    cbar();
+    if (nb == 0) break;
   }
-  if (threadIdx.x == 0)
-    for (int k = 0; k < n_chunks; ++k) mbar_arrive(&S.empty[(cur.c + k) % P.n_stages]);
   cur.c += n_chunks;
   return true;
 }
@@ -1056,7 +1068,6 @@ __device__ bool body_final(const KParams& P) {
 // Thread 0 of the consumers: bounded acquire-wait until the tile's counter
 // reaches need x epoch.
 __device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, volatile int* abort) {
-  if (ld_volatile_s32(&P.err->code) != 0) return false;
   if (T.wait_ctr == kNoCounter) return true;
   const uint32_t target = T.need * P.epoch;
   const uint32_t* ctr = P.ctr + T.wait_ctr;
@@ -1095,6 +1106,10 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       mbar_init(&S.tq_empty[i], 1);
     }
     mbar_init(S.acc, 1);
+    for (int i = 0; i < kSigQueue; ++i) {
+      mbar_init(&S.sig_full[i], 1);
+      mbar_init(&S.sig_empty[i], 1);
+    }
     fence_mbar_init();
     s_abort = 0;
     s_prod_chunks = 0;
@@ -1108,14 +1123,30 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
   __syncthreads();
   tc_fence_after();
 
-  if (warp == kWarps) {
+  if (warp == kWarps && (threadIdx.x & 31) == 1) {
+    // ----------------------------------------------------------- signaller
+    // Release-increments the counters of finished tiles, so that no compute
+    // warp stalls on the release fence.  The compute warps' writes reach it
+    // through the CTA barrier and the mbarrier hand-off (release/acquire at
+    // CTA scope); its gpu-scope release covers them.
+    if (!P.per_op)
+      for (uint32_t j = 0;; ++j) {
+        const int slot = j % kSigQueue;
+        if (!wait_phase(P, &S.sig_full[slot], (j / kSigQueue) & 1u, &s_abort, 0xFFFFFFFFu, 4)) break;
+        const uint2 req = S.sig_req[slot];
+        if (req.y == kSigStop) break;
+        for (uint32_t k = 0; k < req.y; ++k) red_release_add_u32(P.ctr + P.sig[req.x + k], 1u);
+        mbar_arrive(&S.sig_empty[slot]);
+      }
+  } else if (warp == kWarps) {
     // ------------------------------------------------------------ producer
     if ((threadIdx.x & 31) == 0) {
       uint32_t c = 0;  // chunks issued
       const int Q = P.per_op ? 1 : P.lookahead;
       for (uint32_t i = 0;; ++i) {
         const int slot = i % Q;
-        if (i >= (uint32_t)Q && !wait_phase(P, &S.tq_empty[slot], ((i / Q) - 1) & 1u, &s_abort, 0xFFFFFFFFu)) break;
+        if (i >= (uint32_t)Q && !wait_phase(P, &S.tq_empty[slot], ((i / Q) - 1) & 1u, &s_abort, 0xFFFFFFFFu, 4))
+          break;
         uint32_t t;
         if (P.per_op)
           t = (i == 0) ? P.t_begin + blockIdx.x : P.t_end;
@@ -1146,7 +1177,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         auto stage_ptr = [&](uint32_t cc) { return S.ring + (size_t)(cc % P.n_stages) * P.stage_bytes; };
         auto free_stage = [&](uint32_t cc) {
           const uint32_t use = cc / P.n_stages;
-          if (use >= 1 && !wait_phase(P, &S.empty[cc % P.n_stages], (use - 1) & 1u, &s_abort, t)) return false;
+          if (use >= 1 && !wait_phase(P, &S.empty[cc % P.n_stages], (use - 1) & 1u, &s_abort, t, 4)) return false;
           fence_proxy_async_smem();
           return true;
         };
@@ -1192,11 +1223,12 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
     // ----------------------------------------------------------- consumers
     Cursor cur{0};
     ConsumerState cs{kNoAct, kNoCounter, 0u};
+    uint32_t n_sig = 0;  // requests pushed to the signaller (thread 0)
     const int Q = P.per_op ? 1 : P.lookahead;
     __shared__ int s_fail;
     for (uint32_t i = 0;; ++i) {
       const int slot = i % Q;
-      if (!wait_phase(P, &S.tq_full[slot], (i / Q) & 1u, &s_abort, 0xFFFFFFFFu)) break;
+      if (!wait_phase(P, &S.tq_full[slot], (i / Q) & 1u, &s_abort, 0xFFFFFFFFu, 2)) break;
       const TQEntry& e = S.tq[slot];
       if (!e.valid) break;
       const Tile T = e.tile;
@@ -1210,7 +1242,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         if (!P.per_op && T.wait_ctr != cs.last_ctr) {
           ok = wait_counter(P, T, t, &s_abort);
           if (ok) cs.last_ctr = T.wait_ctr;
-        } else if (ld_volatile_s32(&P.err->code) != 0) {
+        } else if (s_abort) {
           ok = false;
         }
         s_fail = ok ? 0 : 1;
@@ -1262,12 +1294,31 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           r.t_end_ns = globaltimer();
           P.trace_buf[t] = r;
         }
-        if (!P.per_op)
-          for (uint32_t k = 0; k < T.sig_cnt; ++k) red_release_add_u32(P.ctr + P.sig[T.sig_off + k], 1u);
+        if (!P.per_op && T.sig_cnt) {
+          const int ss = n_sig % kSigQueue;
+          if (n_sig >= (uint32_t)kSigQueue &&
+              !wait_phase(P, &S.sig_empty[ss], ((n_sig / kSigQueue) - 1) & 1u, &s_abort, t)) {
+            s_fail = 1;
+          } else {
+            S.sig_req[ss] = make_uint2(T.sig_off, T.sig_cnt);
+            mbar_arrive(&S.sig_full[ss]);
+            ++n_sig;
+          }
+        }
         mbar_arrive(&S.tq_empty[slot]);
       }
     }
-    if (threadIdx.x == 0) s_cons_chunks = cur.c;
+    if (threadIdx.x == 0) {
+      s_cons_chunks = cur.c;
+      if (!P.per_op) {  // stop the signaller after the requests already queued
+        const int ss = n_sig % kSigQueue;
+        if (n_sig < (uint32_t)kSigQueue ||
+            wait_phase(P, &S.sig_empty[ss], ((n_sig / kSigQueue) - 1) & 1u, &s_abort, 0xFFFFFFFFu)) {
+          S.sig_req[ss] = make_uint2(0u, kSigStop);
+          mbar_arrive(&S.sig_full[ss]);
+        }
+      }
+    }
   }
   __syncthreads();
   // Drain: wait (bounded) for chunks issued but never consumed.
@@ -1303,12 +1354,25 @@ __global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_kernel(const KParam
   worker(P, smem_raw);
 }
 
+// The prefill program runs the same worker under its own names, so launch
+// lists and profiles separate it from the decode program.
+__global__ void __launch_bounds__(kCtaThreads, 1) wpk_prefill_kernel(const KParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  worker(P, smem_raw);
+}
+__global__ void __launch_bounds__(kCtaThreads, 1) wpk_prefill_op_kernel(const KParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  worker(P, smem_raw);
+}
+
 size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes) {
   return (size_t)n_stages * stage_bytes + act_bytes + kOutFloats * 4 + kMaxQueue * sizeof(TQEntry) +
-         (2 * kMaxStages + 2 * kMaxQueue + 1) * 8;
+         (2 * kMaxStages + 2 * kMaxQueue + 1 + 2 * kSigQueue) * 8 + kSigQueue * sizeof(uint2);
 }
 
 const void* persistent_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_persistent_kernel); }
 const void* per_op_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_per_op_kernel); }
+const void* prefill_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_prefill_kernel); }
+const void* prefill_op_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_prefill_op_kernel); }
 
 }  // namespace wpk

@@ -155,7 +155,9 @@ def plan_cfg(max_batch: int, max_context: int, mode: int = WPK_MEGAKERNEL, n_reg
 # ----------------------------------------------------------- thin wrappers --
 def wpk_build_graph(model: wpk_model_cfg, plan: wpk_plan_cfg) -> C.c_void_p:
     h = C.c_void_p()
-    _check(load_library().wpk_build_graph(C.byref(model), C.byref(plan), C.byref(h)))
+    rc = load_library().wpk_build_graph(C.byref(model), C.byref(plan), C.byref(h))
+    if rc != WPK_OK:
+        raise WpkError(rc, load_library().wpk_last_error(None).decode())
     return h
 
 
