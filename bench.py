@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--workers-per-sm", type=int, default=0)
     ap.add_argument("--lookahead", type=int, default=0)
     ap.add_argument("--schedule", default="queue", choices=["queue", "static"])
+    ap.add_argument("--prefill", default="auto", choices=["auto", "mma", "tokenwise"])
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     return ap.parse_args()
 
 
@@ -210,6 +212,10 @@ def main():
 
     wl = synth.WORKLOADS[args.workload]
     s = wl.model
+    if args.layers:
+        import dataclasses
+
+        s = dataclasses.replace(s, n_layers=args.layers)
     B, T = wl.batch, (wl.prompt_len if args.prompt_len is None else args.prompt_len)
     decode_steps = wl.steps if args.decode_steps is None else args.decode_steps
     tokens_per_step, with_prefill = job_tokens(wl, decode_steps)
@@ -218,7 +224,9 @@ def main():
     mode = W.WPK_MEGAKERNEL if args.mode == "megakernel" else W.WPK_PER_OP_GRAPH
     plan = dict(mode=mode, tile_bytes=args.tile_bytes, slot_bytes=args.slot_bytes,
                 workers_per_sm=args.workers_per_sm, lookahead=args.lookahead,
-                schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE)
+                schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE,
+                prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
+                         "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill])
     if args.regions:
         cuts = [int(x) for x in args.regions.split(",")]
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))
@@ -322,7 +330,8 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "accum_dtype": "fp32", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": B, "prompt_len": T, "decode_steps": decode_steps,
+        "config": {"workload": wl.name + (f" ({s.n_layers} layers)" if args.layers else ""), "batch": B,
+                   "prompt_len": T, "decode_steps": decode_steps, "schedule": args.schedule,
                    "timed": "prefill + decode steps" if with_prefill else "decode steps (prompt prefilled untimed)",
                    "mode": args.mode, "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
                    "prefill": "tensor-core prefill program" if prefill_tensor_cores else "token by token",

@@ -82,7 +82,7 @@ typedef struct wpk_plan_cfg {
   int trace;            /* 1 = record the per-tile device trace                */
   uint64_t wait_timeout_ns; /* bound on every device wait (0 = 2 s)            */
   int slot_bytes;       /* staging slot per worker, used as a ring of 16 KB
-                           chunk stages (0 = 8 stages, 128 KB)                 */
+                           chunk stages (0 = 12 stages, 192 KB, or what fits) */
   int tile_bytes;       /* minimum weight bytes per tile; tiles are sized to give
                            each worker about one tile per op (0 = 32768)       */
   int split_pages;      /* KV pages per attention split (0 = 1)                */

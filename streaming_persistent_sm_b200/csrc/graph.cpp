@@ -90,7 +90,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
     if (in.slot_bytes > budget) return "slot_bytes does not fit shared memory with this many workers per SM";
     p->slot_bytes = in.slot_bytes;
   } else {
-    p->slot_bytes = std::min(8, budget / kStageBytes) * kStageBytes;
+    p->slot_bytes = std::min(12, budget / kStageBytes) * kStageBytes;
     if (p->slot_bytes < kStageBytes) return "no room for a staging slot";
   }
   p->tile_bytes = in.tile_bytes ? in.tile_bytes : 32768;

@@ -687,16 +687,24 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   cbar();
   if (s_last) {
     const float* base = P.part + (((size_t)s.b * P.n_kv + s.g) * P.n_splits) * grp * (2 + hd);
+    // (m, l) of every split and head into shared memory in one parallel step
+    float* ml = Sh.act;  // [n_splits][grp][2]
+    for (int i = threadIdx.x; i < P.n_splits * grp; i += kThreads) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(base + (size_t)i * (2 + hd)));
+      ml[2 * i] = v.x;
+      ml[2 * i + 1] = v.y;
+    }
+    cbar();
     for (int idx = threadIdx.x; idx < grp * hd; idx += kThreads) {
       const int hh = idx / hd, d = idx % hd;
       float M = -INFINITY;
-      for (int j = 0; j < P.n_splits; ++j) M = fmaxf(M, __ldcg(base + ((size_t)j * grp + hh) * (2 + hd)));
+      for (int j = 0; j < P.n_splits; ++j) M = fmaxf(M, ml[2 * (j * grp + hh)]);
       float L = 0.f, O = 0.f;
+#pragma unroll 8
       for (int j = 0; j < P.n_splits; ++j) {
-        const float* pr = base + ((size_t)j * grp + hh) * (2 + hd);
-        const float w = expf(__ldcg(pr) - M);
-        L = fmaf(__ldcg(pr + 1), w, L);
-        O = fmaf(__ldcg(pr + 2 + d), w, O);
+        const float w = expf(ml[2 * (j * grp + hh)] - M);
+        L = fmaf(ml[2 * (j * grp + hh) + 1], w, L);
+        O = fmaf(__ldcg(base + ((size_t)j * grp + hh) * (2 + hd) + 2 + d), w, O);
       }
       P.attn[(size_t)s.b * P.q_rows + ((size_t)s.g * grp + hh) * hd + d] = O / L;
     }
