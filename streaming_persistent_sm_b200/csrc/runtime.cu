@@ -465,6 +465,8 @@ __shared__ uint32_t s_tmem;  // TMEM base address (tensor-core programs)
 __shared__ int s_mma_ok;
 
 __shared__ uint64_t s_t_data;  // trace: when the tile's last chunk had landed
+// GEMV: per stage, 1 + the global index of the last chunk a warp saw land there
+__shared__ volatile uint32_t s_seen[kMaxStages];
 
 __device__ __forceinline__ int act_key_of(const Tile& T) { return (int)T.op | ((int)T.layer << 4) | (T.a2 << 12); }
 
@@ -518,6 +520,23 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int K, int rows
   }
 }
 
+// Bounded wait (one warp) until the GEMV warp that owns stage st's previous
+// use has seen that use land: s_seen[st] >= target.
+__device__ bool wait_seen(const KParams& P, int st, uint32_t target, volatile int* abort, uint32_t tile) {
+  if (s_seen[st] >= target) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (s_seen[st] >= target) return true;
+    if ((it & 15) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > P.timeout_ns) {
+        if ((threadIdx.x & 31) == 0) record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, s_seen[st], target);
+        return false;
+      }
+    }
+  }
+}
+
 // GEMV tile body.  Chunk k of the tile belongs to warp k % 8: the warp waits
 // for that stage only, computes its rows and hands the stage back at once, so
 // a tile of any size streams through the ring and no block barrier is taken
@@ -555,9 +574,22 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
       const uint32_t c = cur.c + k;
       const int st = c % P.n_stages;
       // the stage is waited for on the first token group only
-      if (b0 == 0 && !wait_phase(P, &S.full[st], (c / P.n_stages) & 1u, abort, T.a0)) {
-        ok = false;
-        break;
+      if (b0 == 0) {
+        // A parity wait only tells the current phase from the one before it.
+        // When the stage's previous use (chunk c - n_stages) is this tile's
+        // too, another warp owns it and may not have seen it land yet: wait
+        // for that first, so that the parity wait below cannot be satisfied
+        // by the phase before the previous one.
+        if (k >= P.n_stages && !wait_seen(P, st, c - P.n_stages + 1, abort, T.a0)) {
+          ok = false;
+          break;
+        }
+        if (!wait_phase(P, &S.full[st], (c / P.n_stages) & 1u, abort, T.a0)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        if (lane == 0) s_seen[st] = c + 1;
       }
       const uint8_t* chunk = S.ring + (size_t)st * P.stage_bytes;
       const int r0 = k * rpc, rows = min(rpc, R - r0);
@@ -1119,6 +1151,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       mbar_init(&S.sig_empty[i], 1);
     }
     fence_mbar_init();
+    for (int i = 0; i < kMaxStages; ++i) s_seen[i] = 0;
     s_abort = 0;
     s_prod_chunks = 0;
     s_cons_chunks = 0;
