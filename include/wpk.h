@@ -54,6 +54,7 @@ enum {
 enum { WPK_MEGAKERNEL = 0, WPK_PER_OP_GRAPH = 1 };
 enum { WPK_SCHED_QUEUE = 0, WPK_SCHED_STATIC = 1 };
 enum { WPK_PREFILL_AUTO = 0, WPK_PREFILL_MMA = 1, WPK_PREFILL_TOKENWISE = 2 };
+enum { WPK_DECODE_AUTO = 0, WPK_DECODE_GEMV = 1, WPK_DECODE_MMA = 2 };
 
 /* --------------------------------------------------------------- configs */
 /* Decoder shape.  Weights are bf16, matmul weights stored [out][in]. */
@@ -85,7 +86,8 @@ typedef struct wpk_plan_cfg {
                            chunk stages (0 = 12 stages, 192 KB, or what fits) */
   int tile_bytes;       /* minimum weight bytes per tile; tiles are sized to give
                            each worker about one tile per op (0 = 32768)       */
-  int split_pages;      /* KV pages per attention split (0 = 1)                */
+  int split_pages;      /* KV pages per attention tile (split); 0 = chosen so that
+                           a step has about two attention tiles per worker     */
   int lookahead;        /* tiles a worker may claim and stage ahead of the one
                            it computes (0 = 4); 1 = a tile's weights are staged
                            only after the previous tile of that worker is done */
@@ -97,6 +99,11 @@ typedef struct wpk_plan_cfg {
                            WPK_PREFILL_MMA; WPK_PREFILL_TOKENWISE (the prompt
                            runs through the decode program one position at a
                            time)                                                */
+  int decode;           /* WPK_DECODE_AUTO (0): tensor-core decode tiles when
+                           max_batch > 8 and the shapes allow, else CUDA-core
+                           GEMV tiles; WPK_DECODE_GEMV; WPK_DECODE_MMA (the
+                           step's sequences are the MMA N dimension, so
+                           max_batch <= 128)                                    */
 } wpk_plan_cfg;
 
 /* Host weights: bf16 bit patterns, row-major [out][in]. */

@@ -60,6 +60,7 @@ struct wpk_handle {
   float2* d_rope = nullptr;
   int32_t* d_block_table = nullptr;
   uint32_t* d_arrive = nullptr;
+  uint32_t* d_rb_arrive = nullptr;  // batched decode: split arrivals per O / down row block
   unsigned long long* d_best = nullptr;
   int32_t* d_seqlen = nullptr;
   int32_t* d_tok_fb = nullptr;
@@ -71,6 +72,9 @@ struct wpk_handle {
   uint8_t* scratch = nullptr;
   size_t kv_bytes = 0, scratch_bytes = 0;
   size_t off_xa = 0, off_xb = 0, off_q = 0, off_attn = 0, off_h = 0, off_part = 0;
+  // batched decode program: residual (feature-major), q/k/v sums, x^2 sums,
+  // hi/lo images of x*g_attn, x*g_ffn, the attention output and h
+  size_t off_xt = 0, off_acc = 0, off_ss = 0, off_dimg[4][2] = {};
   int64_t n_blocks = 0;
   bool loaded = false, prefilled = false, poisoned = false, has_device = false;
   int batch = 0, ctx = 0;
@@ -179,6 +183,30 @@ KParams make_params(const wpk_handle* h) {
   P.in_tok_stride = 1;
   P.epoch = 1;
   P.static_sched = g.plan.schedule == WPK_SCHED_STATIC;
+  P.mma_n = kTokBlock;
+  P.act_chunk = kMmaChunkBytes;
+  if (g.plan.decode_mode == WPK_DECODE_MMA) {
+    P.dec_mma = 1;
+    P.uses_tmem = 1;
+    P.mma_n = g.plan.dec_n;
+    P.act_chunk = g.plan.dec_n * 128;
+    P.stage_bytes = g.plan.dec_stage_bytes;
+    P.n_stages = g.plan.dec_stages;
+    P.act_bytes = g.plan.dec_act_bytes;
+    P.o_splits = g.o_splits;
+    P.down_splits = g.down_splits;
+    P.xt = reinterpret_cast<float*>(h->scratch + h->off_xt);
+    P.acc = reinterpret_cast<float*>(h->scratch + h->off_acc);
+    P.ss = reinterpret_cast<float*>(h->scratch + h->off_ss);
+    for (int i = 0; i < 2; ++i) {
+      P.xn_img[i] = h->scratch + h->off_dimg[0][i];
+      P.xf_img[i] = h->scratch + h->off_dimg[1][i];
+      P.att_img[i] = h->scratch + h->off_dimg[2][i];
+      P.h_img[i] = h->scratch + h->off_dimg[3][i];
+    }
+    P.rb_arrive = h->d_rb_arrive;
+    P.lm_mma_off = g.lay.lm_mma;
+  }
   return P;
 }
 
@@ -204,6 +232,16 @@ void scratch_layout(wpk_handle* h) {
     for (int i = 0; i < 2; ++i) h->off_xn[i] = take(n_tb * (m.hidden / 64) * kMmaChunkBytes);
     for (int i = 0; i < 2; ++i) h->off_att[i] = take(n_tb * (q_rows / 64) * kMmaChunkBytes);
     for (int i = 0; i < 2; ++i) h->off_hi[i] = take(n_tb * (m.ffn / 64) * kMmaChunkBytes);
+  }
+  if (g.plan.decode_mode == WPK_DECODE_MMA) {
+    const size_t N = g.plan.dec_n, chunk = N * 128;
+    const size_t qkv_rows = q_rows + 2 * (size_t)m.n_kv_heads * m.head_dim;
+    h->off_xt = take((size_t)m.hidden * N * 4);
+    h->off_acc = take(qkv_rows * N * 4);
+    h->off_ss = take((2 * (size_t)m.n_layers + 1) * N * 4);
+    const size_t widths[4] = {(size_t)m.hidden, (size_t)m.hidden, q_rows, (size_t)m.ffn};
+    for (int t = 0; t < 4; ++t)
+      for (int i = 0; i < 2; ++i) h->off_dimg[t][i] = take(widths[t] / 64 * chunk);
   }
   h->scratch_bytes = off;
   h->n_blocks = (int64_t)B * g.max_blocks;
@@ -239,7 +277,7 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
     P.t_begin = og.begin;
     P.t_end = og.end;
     P.per_op = 1;
-    P.n_stages = g.plan.per_op_slot / kStageBytes;
+    if (!P.dec_mma) P.n_stages = g.plan.per_op_slot / kStageBytes;
     void* args[] = {&P};
     cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
                                      h->smem_per_op, h->capture_stream);
@@ -333,6 +371,11 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.stage_bytes = 3 * kMmaChunkBytes;
   P.n_stages = h->prefill_stages;
   P.uses_tmem = 1;
+  // the prefill program's own geometry (its LM head tiles are GEMV tiles)
+  P.dec_mma = 0;
+  P.act_bytes = g.plan.act_bytes;
+  P.mma_n = kTokBlock;
+  P.act_chunk = kMmaChunkBytes;
   P.M = g.M;
   P.T = g.T;
   P.n_tb = g.n_tb;
@@ -411,8 +454,13 @@ static int setup_device(wpk_handle* h) {
   const wpk_model_cfg* model = &g.m;
   CUDA_TRY(h, cudaGetDevice(&h->device));
   CUDA_TRY(h, cudaDeviceGetAttribute(&h->n_sms, cudaDevAttrMultiProcessorCount, h->device));
-  h->smem = worker_smem_bytes(p.slot_bytes / kStageBytes, kStageBytes, p.act_bytes);
-  h->smem_per_op = worker_smem_bytes(p.per_op_slot / kStageBytes, kStageBytes, p.act_bytes);
+  if (p.decode_mode == WPK_DECODE_MMA) {
+    h->smem = worker_smem_bytes(p.dec_stages, p.dec_stage_bytes, p.dec_act_bytes);
+    h->smem_per_op = h->smem;
+  } else {
+    h->smem = worker_smem_bytes(p.slot_bytes / kStageBytes, kStageBytes, p.act_bytes);
+    h->smem_per_op = worker_smem_bytes(p.per_op_slot / kStageBytes, kStageBytes, p.act_bytes);
+  }
   if (h->smem > (size_t)kMaxSmem || h->smem_per_op > (size_t)kMaxSmem)
     return fail(h, WPK_ERR_UNSUPPORTED, "staging slot and activations exceed shared memory");
   if (p.prefill_mode == WPK_PREFILL_MMA) {
@@ -453,7 +501,8 @@ static int setup_device(wpk_handle* h) {
                o_layers = take(g.lay.layers.size() * sizeof(LayerDev)),
                o_rope = take((size_t)p.max_context * hd2 * sizeof(float2)),
                o_bt = take(B * g.max_blocks * 4), o_arr = take(B * model->n_kv_heads * 4), o_best = take(B * 8),
-               o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4);
+               o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4),
+               o_rb = take((size_t)model->n_layers * 2 * (model->hidden / 128 + 1) * 4);
   CUDA_TRY(h, cudaMalloc(&h->d_base, off));
   CUDA_TRY(h, cudaMemset(h->d_base, 0, off));
   h->d_tiles = reinterpret_cast<Tile*>(h->d_base + o_tiles);
@@ -471,6 +520,7 @@ static int setup_device(wpk_handle* h) {
   h->d_seqlen = reinterpret_cast<int32_t*>(h->d_base + o_seq);
   h->d_tok_fb = reinterpret_cast<int32_t*>(h->d_base + o_fb);
   h->d_active = reinterpret_cast<int32_t*>(h->d_base + o_act);
+  h->d_rb_arrive = reinterpret_cast<uint32_t*>(h->d_base + o_rb);
   CUDA_TRY(h, cudaMemcpy(h->d_tiles, g.tiles.data(), n_tiles * sizeof(Tile), cudaMemcpyHostToDevice));
   if (!g.sig.empty()) CUDA_TRY(h, cudaMemcpy(h->d_sig, g.sig.data(), g.sig.size() * 4, cudaMemcpyHostToDevice));
   CUDA_TRY(h, cudaMemcpy(h->d_layers, g.lay.layers.data(), g.lay.layers.size() * sizeof(LayerDev),
@@ -595,6 +645,15 @@ int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_
   CUDA_TRY(h, cudaMemsetAsync(h->d_seqlen, 0, B * 4, s));
   CUDA_TRY(h, cudaMemsetAsync(h->d_best, 0, B * 8, s));
   CUDA_TRY(h, cudaMemsetAsync(h->d_arrive, 0, B * h->g.m.n_kv_heads * 4, s));
+  if (h->g.plan.decode_mode == WPK_DECODE_MMA) {
+    // the batched decode program keeps these at zero between steps itself
+    const wpk_model_cfg& m = h->g.m;
+    const size_t N = h->g.plan.dec_n;
+    const size_t qkv_rows = (size_t)(m.n_heads + 2 * m.n_kv_heads) * m.head_dim;
+    CUDA_TRY(h, cudaMemsetAsync(h->scratch + h->off_acc, 0, qkv_rows * N * 4, s));
+    CUDA_TRY(h, cudaMemsetAsync(h->scratch + h->off_ss, 0, (2 * (size_t)m.n_layers + 1) * N * 4, s));
+    CUDA_TRY(h, cudaMemsetAsync(h->d_rb_arrive, 0, (size_t)m.n_layers * 2 * (m.hidden / 128 + 1) * 4, s));
+  }
   CUDA_TRY(h, cudaMemcpyAsync(h->d_active, &batch, 4, cudaMemcpyHostToDevice, s));
   CUDA_TRY(h, cudaStreamSynchronize(s));  // `batch` lives on this stack frame
   h->batch = batch;
@@ -772,6 +831,9 @@ int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes
   if (rc) return rc;
   if (h->g.plan.mode != WPK_MEGAKERNEL)
     return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the megakernel mode");
+  if (h->g.plan.decode_mode == WPK_DECODE_MMA)
+    return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the GEMV decode program (the tensor-core "
+                                        "decode program keeps sums in its scratch between steps)");
   if (h->scratch_bytes > scratch_bytes)
     return fail(h, WPK_ERR_SHAPE, "the plan needs " + std::to_string(h->scratch_bytes) +
                                       " scratch bytes, more than the " + std::to_string(scratch_bytes) +

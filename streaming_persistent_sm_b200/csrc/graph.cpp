@@ -95,15 +95,41 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   }
   p->tile_bytes = in.tile_bytes ? in.tile_bytes : 32768;
   if (p->tile_bytes < 1024 || p->tile_bytes > 1 << 20) return "tile_bytes must be in [1K, 1M]";
-  p->split_pages = in.split_pages ? in.split_pages : 1;
-  if (p->split_pages < 1) return "split_pages must be >= 1";
-  if ((int64_t)p->split_pages * p->page_tokens * m.head_dim * 2 * 2 > kStageBytes)
-    return "an attention split's K/V pages do not fit one 16 KB stage";
+  p->split_pages = in.split_pages;  // 0: chosen by compile_graph
+  if (p->split_pages < 0) return "split_pages must be >= 0";
+  if ((int64_t)p->page_tokens * m.head_dim * 2 * 2 > kStageBytes)
+    return "a KV page (K and V rows) does not fit one 16 KB stage";
   p->per_op_slot = 0;  // set by compile_graph
   {
     const int qr = m.n_heads * m.head_dim, kvr = m.n_kv_heads * m.head_dim;
     const bool mma_ok = (qr + 2 * kvr) % 128 == 0 && m.hidden % 128 == 0 && (2 * m.ffn) % 128 == 0 &&
                         m.hidden % 64 == 0 && qr % 128 == 0 && m.ffn % 64 == 0 && kvr % 128 == 0;
+    if (in.decode == WPK_DECODE_AUTO)
+      p->decode_mode = (in.max_batch > kMaxGemvBatch && in.max_batch <= kMaxMmaBatch && mma_ok) ? WPK_DECODE_MMA
+                                                                                                : WPK_DECODE_GEMV;
+    else if (in.decode == WPK_DECODE_MMA) {
+      if (!mma_ok) { *code = WPK_ERR_UNSUPPORTED; return "shapes do not fit the tensor-core decode tiles"; }
+      if (in.max_batch > kMaxMmaBatch) { *code = WPK_ERR_SHAPE; return "tensor-core decode takes at most 128 sequences"; }
+      p->decode_mode = WPK_DECODE_MMA;
+    } else if (in.decode == WPK_DECODE_GEMV)
+      p->decode_mode = WPK_DECODE_GEMV;
+    else
+      return "bad decode mode";
+    p->dec_n = p->dec_stage_bytes = p->dec_stages = p->dec_act_bytes = 0;
+    if (p->decode_mode == WPK_DECODE_MMA) {
+      // one ring stage = a 16 KB weight chunk + the hi/lo activation chunks of
+      // N tokens (N rows of 128 bytes each)
+      p->dec_n = (in.max_batch + 15) / 16 * 16;
+      p->dec_stage_bytes = kMmaChunkBytes + 2 * p->dec_n * 128;
+      // attention scratch: queries, one page of scores, the combine's (m, l) pairs
+      const int max_pages = (in.max_context + p->page_tokens - 1) / p->page_tokens;
+      const int need = std::max(kMaxGroup * (m.head_dim + p->page_tokens) * 4, max_pages * kMaxGroup * 2 * 4);
+      p->dec_act_bytes = std::max(16384, (need + 1023) / 1024 * 1024);
+      const int room = kMaxSmem - fixed - 4096 - p->dec_act_bytes;  // 4 KB: the kernel's static shared memory
+      int want = in.slot_bytes ? in.slot_bytes / kStageBytes : 12;
+      p->dec_stages = std::min(std::min(want, kMaxStages), room / p->dec_stage_bytes);
+      if (p->dec_stages < 2) { *code = WPK_ERR_UNSUPPORTED; return "no room for the tensor-core decode ring"; }
+    }
     if (in.prefill == WPK_PREFILL_AUTO)
       p->prefill_mode = mma_ok ? WPK_PREFILL_MMA : WPK_PREFILL_TOKENWISE;
     else if (in.prefill == WPK_PREFILL_MMA) {
@@ -187,6 +213,38 @@ struct DataflowBuilder {
     const auto& P = (*preds_of)[w];
     return std::binary_search(P.begin(), P.end(), u);
   }
+  // Exact "is u an ancestor of one of `preds`" for the few writers that
+  // accumulations need ordering after: per watched writer, a descendant flag
+  // per tile, extended as tiles are finished.
+  std::unordered_map<int, std::vector<char>> desc;
+  int n_done = 0;
+  bool descends(int u, const std::vector<int>& preds) {
+    auto it = desc.find(u);
+    if (it == desc.end()) {
+      std::vector<char> d(preds_of->size(), 0);
+      for (int t = u + 1; t < n_done; ++t)
+        for (int x : (*preds_of)[t])
+          if (x == u || d[x]) {
+            d[t] = 1;
+            break;
+          }
+      it = desc.emplace(u, std::move(d)).first;
+    }
+    for (int x : preds)
+      if (x == u || it->second[x]) return true;
+    return false;
+  }
+  void finish(int t) {
+    for (auto& kv : desc) {
+      if (t <= kv.first) continue;
+      for (int x : (*preds_of)[t])
+        if (x == kv.first || kv.second[x]) {
+          kv.second[t] = 1;
+          break;
+        }
+    }
+    n_done = t + 1;
+  }
   void apply(int t, const std::vector<Access>& acc, std::vector<int>* preds) {
     std::vector<int> acc_deps;
     for (auto& a : acc) {
@@ -208,6 +266,7 @@ struct DataflowBuilder {
     for (int u : acc_deps) {
       bool implied = std::binary_search(preds->begin(), preds->end(), u);
       for (size_t i = 0; !implied && i < preds->size() && i < 4; ++i) implied = is_pred(u, (*preds)[i]);
+      if (!implied && !preds->empty()) implied = descends(u, *preds);
       if (!implied) preds->push_back(u);
     }
     for (auto& a : acc) {
@@ -234,6 +293,7 @@ struct DataflowBuilder {
     std::sort(preds->begin(), preds->end());
     preds->erase(std::unique(preds->begin(), preds->end()), preds->end());
     preds->erase(std::remove(preds->begin(), preds->end(), t), preds->end());
+    finish(t);
   }
 };
 
@@ -259,6 +319,109 @@ int rows_per_tile(int row_bytes, int op_rows, const Plan& p, int W) {
   if (p.max_batch > kMaxGemvBatch) r = std::min(r, (p.slot_bytes / kStageBytes) * rpc);
   r = std::min(r, kMaxTileRows / rpc * rpc);
   return std::max(r, 2);
+}
+
+// GEMV LM head tiles (fused final RMSNorm + logits + argmax): row ranges of
+// the LM head in the weight image.
+struct LmTile {
+  uint64_t w_off;
+  uint32_t w_bytes;
+  int r0, n;
+};
+std::vector<LmTile> gemv_lm_tiles(const wpk_model_cfg& m, const Plan& p, int W, const Layout& L) {
+  std::vector<LmTile> out;
+  const int h = m.hidden;
+  const int R = rows_per_tile(h * 2, m.vocab, p, W);
+  for (int r0 = 0; r0 < m.vocab; r0 += R) {
+    const int n = std::min(R, m.vocab - r0);
+    out.push_back({L.lm_head + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n});
+  }
+  return out;
+}
+
+// K splits of a tensor-core op with `rb` blocks of 128 rows and `nkc` 64-column
+// chunks: enough tiles for every worker, none smaller than tile_bytes.
+int mma_splits(int rb, int nkc, const Plan& p, int W) {
+  const int want = (W + rb - 1) / rb;
+  const int most = std::max(1, nkc * kMmaChunkBytes / std::max(p.tile_bytes, kMmaChunkBytes));
+  return std::max(1, std::min(std::min(want, most), nkc));
+}
+
+// Batched decode program: every projection is a tensor-core tile of 128
+// weight rows x (K range) x (the step's N tokens), swap-AB (the weights are
+// the MMA's M operand, the tokens its N).  Projections followed by a
+// nonlinearity (gate/up, LM head) take the whole K; the others are split
+// along K so that every worker has a tile and sum into fp32 buffers.  The
+// last split of each O / down row block turns its finished residual rows into
+// the next RMSNorm's input image (x * g) and adds their x^2 to the per-token
+// sums; consumers apply 1/rms per token column in their epilogue.
+template <class Add>
+void build_mma_decode_tiles(const wpk_model_cfg& m, const Plan& p, int W, CompiledGraph& g, Add& add,
+                            std::vector<uint32_t>* layer_begin) {
+  const int h = m.hidden, hd = m.head_dim, grp = m.n_heads / m.n_kv_heads;
+  const int q_rows = m.n_heads * hd, kv_rows = m.n_kv_heads * hd, qkv_rows = q_rows + 2 * kv_rows;
+  const uint32_t chunk = kMmaChunkBytes;
+  const int nkc_h = h / 64, nkc_q = q_rows / 64, nkc_f = m.ffn / 64;
+  const int s_qkv = mma_splits(qkv_rows / 128, nkc_h, p, W);
+  g.o_splits = mma_splits(h / 128, nkc_q, p, W);
+  g.down_splits = mma_splits(h / 128, nkc_f, p, W);
+  auto krange = [](int nkc, int s, int i, int* c0, int* c1) {
+    *c0 = (int)((int64_t)nkc * i / s);
+    *c1 = (int)((int64_t)nkc * (i + 1) / s);
+  };
+  const Layout& L = g.lay;
+  // x = E[tok] per 128-feature block, with the first RMSNorm's input image
+  for (int fb = 0; fb < h / 128; ++fb)
+    add(OP_EMBED, 0, 0, 0, fb, 0, 0, 0,
+        {{BUF_XA, fb * 128, fb * 128 + 128, 1}, {BUF_DXN, fb * 128, fb * 128 + 128, 1}, {BUF_TOK, 0, 1, 0}});
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerDev& d = L.layers[l];
+    (*layer_begin)[l] = (uint32_t)g.tiles.size();
+    for (int fb = 0; fb < qkv_rows / 128; ++fb)
+      for (int i = 0; i < s_qkv; ++i) {
+        int c0, c1;
+        krange(nkc_h, s_qkv, i, &c0, &c1);
+        add(OP_BQKV, l, d.mma_qkv + ((uint64_t)fb * nkc_h + c0) * chunk, (uint32_t)(c1 - c0) * chunk, fb, 0, c0 * 64,
+            (c1 - c0) * 64, {{BUF_DXN, 0, h, 0}, {BUF_QKV, fb * 128, fb * 128 + 128, 2}});
+      }
+    const int attn_group = 1000 + l;
+    for (int b = 0; b < p.max_batch; ++b)
+      for (int gi = 0; gi < m.n_kv_heads; ++gi)
+        for (int j = 0; j < g.n_splits; ++j)
+          add(OP_ATTN, l, 0, 0, b, gi, j, 0,
+              {{BUF_QKV, gi * grp * hd, (gi + 1) * grp * hd, 0},
+               {BUF_QKV, q_rows + gi * hd, q_rows + (gi + 1) * hd, 0},
+               {BUF_QKV, q_rows + kv_rows + gi * hd, q_rows + kv_rows + (gi + 1) * hd, 0},
+               {BUF_ATTN, gi * grp * hd, (gi + 1) * grp * hd, 1, attn_group}});
+    for (int fb = 0; fb < h / 128; ++fb)
+      for (int i = 0; i < g.o_splits; ++i) {
+        int c0, c1;
+        krange(nkc_q, g.o_splits, i, &c0, &c1);
+        add(OP_BO, l, d.mma_wo + ((uint64_t)fb * nkc_q + c0) * chunk, (uint32_t)(c1 - c0) * chunk, fb, 0, c0 * 64,
+            (c1 - c0) * 64,
+            {{BUF_ATTN, c0 * 64, c1 * 64, 0}, {BUF_XA, fb * 128, fb * 128 + 128, 2},
+             {BUF_DXF, fb * 128, fb * 128 + 128, 1, 3000 + l}});
+      }
+    for (int fb = 0; fb < 2 * m.ffn / 128; ++fb)
+      add(OP_BGU, l, d.mma_gu + (uint64_t)fb * nkc_h * chunk, (uint32_t)nkc_h * chunk, fb, 0, 0, h,
+          {{BUF_DXF, 0, h, 0}, {BUF_H, fb * 64, fb * 64 + 64, 1}});
+    for (int fb = 0; fb < h / 128; ++fb)
+      for (int i = 0; i < g.down_splits; ++i) {
+        int c0, c1;
+        krange(nkc_f, g.down_splits, i, &c0, &c1);
+        add(OP_BDOWN, l, d.mma_down + ((uint64_t)fb * nkc_f + c0) * chunk, (uint32_t)(c1 - c0) * chunk, fb, 0,
+            c0 * 64, (c1 - c0) * 64,
+            {{BUF_H, c0 * 64, c1 * 64, 0}, {BUF_XA, fb * 128, fb * 128 + 128, 2},
+             {BUF_DXN, fb * 128, fb * 128 + 128, 1, 4000 + l}});
+      }
+  }
+  (*layer_begin)[m.n_layers] = (uint32_t)g.tiles.size();
+  for (int vb = 0; vb < L.vocab_blocks; ++vb) {
+    const int r0 = vb * 128, n = std::min(128, m.vocab - r0);
+    add(OP_BLM, m.n_layers, L.lm_mma + (uint64_t)vb * nkc_h * chunk, (uint32_t)nkc_h * chunk, vb, 0, 0, h,
+        {{BUF_DXN, 0, h, 0}, {BUF_LOGITS, r0, r0 + n, 1}, {BUF_BEST, 0, 1, 2}});
+  }
+  add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0}, {BUF_TOK, 0, 1, 1}});
 }
 
 }  // namespace
@@ -297,7 +460,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   L.final_norm = take((uint64_t)h * 4);
   L.embed = take((uint64_t)m.vocab * h * 2);
   L.lm_head = m.tied_embedding ? L.embed : take((uint64_t)m.vocab * h * 2);
-  L.mma = p.prefill_mode == WPK_PREFILL_MMA;
+  L.mma = p.prefill_mode == WPK_PREFILL_MMA || p.decode_mode == WPK_DECODE_MMA;
   for (int l = 0; l < m.n_layers; ++l) {
     LayerDev& d = L.layers[l];
     d.mma_qkv = d.mma_wo = d.mma_gu = d.mma_down = 0;
@@ -307,14 +470,31 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
     d.mma_gu = take((uint64_t)2 * m.ffn * h * 2);
     d.mma_down = take((uint64_t)h * m.ffn * 2);
   }
+  L.lm_mma = 0;
+  L.vocab_blocks = 0;
+  if (p.decode_mode == WPK_DECODE_MMA) {
+    L.vocab_blocks = (m.vocab + 127) / 128;
+    L.lm_mma = take((uint64_t)L.vocab_blocks * (h / 64) * kMmaChunkBytes);
+  }
   L.total = off;
   L.down_kc = kc;
   L.n_down_chunks = nch;
 
-  // ---- attention splits ----
-  g->split_tokens = p.split_pages * p.page_tokens;
-  g->n_splits = (p.max_context + g->split_tokens - 1) / g->split_tokens;
+  // ---- attention splits: KV pages per tile; by default about two attention
+  // tiles per worker over the batch and kv heads ----
+  g->W = W;
   g->max_blocks = (p.max_context + p.page_tokens - 1) / p.page_tokens;
+  {
+    int sp = p.split_pages;
+    if (sp == 0) {
+      const int pairs = p.max_batch * m.n_kv_heads;
+      const int ns = std::max(1, std::min(g->max_blocks, (2 * W + pairs / 2) / pairs));
+      sp = (g->max_blocks + ns - 1) / ns;
+    }
+    g->plan.split_pages = sp;
+    g->split_tokens = sp * p.page_tokens;
+  }
+  g->n_splits = (p.max_context + g->split_tokens - 1) / g->split_tokens;
 
   // ---- tiles in ticket order ----
   std::vector<Tile>& T = g->tiles;
@@ -341,6 +521,9 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   };
   std::vector<uint32_t> layer_begin(m.n_layers + 1, 0);
 
+  if (p.decode_mode == WPK_DECODE_MMA) {
+    build_mma_decode_tiles(m, p, W, *g, add, &layer_begin);
+  } else {
   add(OP_EMBED, 0, 0, 0, 0, 0, 0, 0, {{BUF_XA, 0, h, 1}, {BUF_TOK, 0, 1, 0}});
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerDev& d = L.layers[l];
@@ -396,20 +579,16 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
     }
   }
   layer_begin[m.n_layers] = (uint32_t)T.size();
-  {
-    int R = rows_per_tile(h * 2, m.vocab, p, W);
-    for (int r0 = 0; r0 < m.vocab; r0 += R) {
-      int n = std::min(R, m.vocab - r0);
-      add(OP_LMHEAD, m.n_layers, L.lm_head + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n, 0, h,
-          {{BUF_XA, 0, h, 0}, {BUF_LOGITS, r0, r0 + n, 1}, {BUF_BEST, 0, 1, 2}});
-    }
-  }
+  for (const LmTile& t : gemv_lm_tiles(m, p, W, L))
+    add(OP_LMHEAD, m.n_layers, t.w_off, t.w_bytes, t.r0, t.n, 0, h,
+        {{BUF_XA, 0, h, 0}, {BUF_LOGITS, t.r0, t.r0 + t.n, 1}, {BUF_BEST, 0, 1, 2}});
   add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0}, {BUF_TOK, 0, 1, 1}});
+  }
   g->algo_weight_bytes = wbytes;
   // a per-op CTA holds one whole tile in its ring
   int max_chunks = 1;
   for (const Tile& t : T)
-    if (t.op != OP_ATTN && t.w_bytes) {
+    if (t.op != OP_ATTN && t.w_bytes && t.op < OP_BQKV) {
       const int rpc = std::max(2, (kStageBytes / (t.a3 * 2)) & ~1);
       max_chunks = std::max(max_chunks, (t.a1 + rpc - 1) / rpc);
     }
@@ -419,7 +598,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
 
   // ---- edges from dataflow ----
   DataflowBuilder df;
-  int sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1};
+  int sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1, 1, 1, 1, 1, 1, 1, h, h};
   for (int b = 0; b < BUF_COUNT; ++b) df.bufs.emplace_back(sizes[b]);
   g->preds.assign(T.size(), {});
   df.preds_of = &g->preds;
@@ -488,6 +667,7 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
   g->T = T;
   g->M = B * T;
   g->n_tb = (g->M + kTokBlock - 1) / kTokBlock;
+  g->W = dec.W;
   const int h = m.hidden, hd = m.head_dim, grp = m.n_heads / m.n_kv_heads;
   const int q_rows = m.n_heads * hd, kv_rows = m.n_kv_heads * hd, qkv_rows = q_rows + 2 * kv_rows;
   const int nq = g->n_tb;
@@ -534,6 +714,12 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
     return a;
   };
   std::vector<uint32_t> layer_begin(m.n_layers + 1, 0);
+  const int s_o = mma_splits(nq * (h / 128), q_rows / 64, p, dec.W);
+  const int s_dn = mma_splits(nq * (h / 128), m.ffn / 64, p, dec.W);
+  auto krange = [](int nkc, int s, int i, int* c0, int* c1) {
+    *c0 = (int)((int64_t)nkc * i / s);
+    *c1 = (int)((int64_t)nkc * (i + 1) / s);
+  };
   for (int tb = 0; tb < nq; ++tb) add(OP_PEMBED, 0, 0, 0, tb, 0, 0, 0, {blk(BUF_PX, h, tb, 0, h, 1)});
   const uint32_t chunk = kMmaChunkBytes;
   for (int l = 0; l < m.n_layers; ++l) {
@@ -570,10 +756,17 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
           }
           add(OP_PATTN, l, 0, 0, b, gi, qb, 0, acc);
         }
+    // O and down: split along K when the token blocks alone give too few tiles
+    // for the workers; the splits add into X
     for (int tb = 0; tb < nq; ++tb)
       for (int fb = 0; fb < h / 128; ++fb)
-        add(OP_MO, l, d.mma_wo + (uint64_t)fb * (q_rows / 64) * chunk, (uint32_t)(q_rows / 64) * chunk, fb, tb, 0,
-            q_rows, {blk(BUF_PATT, q_rows, tb, 0, q_rows, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
+        for (int i = 0; i < s_o; ++i) {
+          int c0, c1;
+          krange(q_rows / 64, s_o, i, &c0, &c1);
+          add(OP_MO, l, d.mma_wo + ((uint64_t)fb * (q_rows / 64) + c0) * chunk, (uint32_t)(c1 - c0) * chunk, fb, tb,
+              c0 * 64, (c1 - c0) * 64,
+              {blk(BUF_PATT, q_rows, tb, c0 * 64, c1 * 64, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
+        }
     for (int tb = 0; tb < nq; ++tb)
       add(OP_NORM, l, 0, 0, tb, 1, 0, h, {blk(BUF_PX, h, tb, 0, h, 0), blk(BUF_PXN, h, tb, 0, h, 1)});
     for (int tb = 0; tb < nq; ++tb)
@@ -582,8 +775,13 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
             {blk(BUF_PXN, h, tb, 0, h, 0), blk(BUF_PH, m.ffn, tb, fb * 64, fb * 64 + 64, 1)});
     for (int tb = 0; tb < nq; ++tb)
       for (int fb = 0; fb < h / 128; ++fb)
-        add(OP_MDOWN, l, d.mma_down + (uint64_t)fb * (m.ffn / 64) * chunk, (uint32_t)(m.ffn / 64) * chunk, fb, tb,
-            0, m.ffn, {blk(BUF_PH, m.ffn, tb, 0, m.ffn, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
+        for (int i = 0; i < s_dn; ++i) {
+          int c0, c1;
+          krange(m.ffn / 64, s_dn, i, &c0, &c1);
+          add(OP_MDOWN, l, d.mma_down + ((uint64_t)fb * (m.ffn / 64) + c0) * chunk, (uint32_t)(c1 - c0) * chunk, fb,
+              tb, c0 * 64, (c1 - c0) * 64,
+              {blk(BUF_PH, m.ffn, tb, c0 * 64, c1 * 64, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
+        }
   }
   layer_begin[m.n_layers] = (uint32_t)Tl.size();
   {
@@ -591,11 +789,10 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
     for (int b = 0; b < B; ++b) acc.push_back(blk(BUF_PX, h, (b * T + T - 1) / kTokBlock, 0, h, 0));
     add(OP_GATHER, m.n_layers, 0, 0, 0, 0, 0, 0, acc);
   }
-  // LM head + argmax + publish: the decode program's tiles
-  for (const Tile& t : dec.tiles)
-    if (t.op == OP_LMHEAD)
-      add(OP_LMHEAD, m.n_layers, t.w_off, t.w_bytes, t.a0, t.a1, t.a2, t.a3,
-          {{BUF_XA, 0, h, 0, -1}, {BUF_LOGITS, t.a0, t.a0 + t.a1, 1, -1}, {BUF_BEST, 0, 1, 2, -1}});
+  // LM head + argmax + publish: GEMV tiles over the gathered last positions
+  for (const LmTile& t : gemv_lm_tiles(m, p, dec.W, dec.lay))
+    add(OP_LMHEAD, m.n_layers, t.w_off, t.w_bytes, t.r0, t.n, 0, h,
+        {{BUF_XA, 0, h, 0, -1}, {BUF_LOGITS, t.r0, t.r0 + t.n, 1, -1}, {BUF_BEST, 0, 1, 2, -1}});
   add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0, -1}, {BUF_TOK, 0, 1, 1, -1}});
   g->algo_weight_bytes = wbytes;
   if (Tl.size() >= (1u << 31)) return "too many tiles";
@@ -604,7 +801,7 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
   const int64_t sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1,
                                     (int64_t)nq * h * TB, (int64_t)nq * h * TB, (int64_t)nq * q_rows * TB,
                                     (int64_t)m.n_layers * nq * 2 * kv_rows * TB, (int64_t)nq * q_rows * TB,
-                                    (int64_t)nq * m.ffn * TB};
+                                    (int64_t)nq * m.ffn * TB, h, h};
   for (int b = 0; b < BUF_COUNT; ++b) df.bufs.emplace_back(sizes[b]);
   g->preds.assign(Tl.size(), {});
   df.preds_of = &g->preds;
@@ -839,11 +1036,23 @@ std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_
       for (int r = 0; r < h; ++r)
         memcpy(dd + ((uint64_t)c * h + r) * kc, W.w_down + (uint64_t)r * m.ffn + (uint64_t)c * kc, (size_t)kc * 2);
   };
+  // the LM head's tensor-core image (batched decode), in 16 row slices per task
+  const uint16_t* lm_src = m.tied_embedding ? w.embed : w.lm_head;
+  const int lm_tasks = g.lay.lm_mma ? 16 : 0;
+  auto do_lm = [&](int i) {
+    const int r0 = (int)((int64_t)m.vocab * i / lm_tasks), r1 = (int)((int64_t)m.vocab * (i + 1) / lm_tasks);
+    for (int r = r0; r < r1; ++r) mma_row(g.lay.lm_mma, h, r, lm_src + (uint64_t)r * h);
+  };
   unsigned nt = std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
   std::atomic<int> next{0};
   for (unsigned i = 0; i < nt; ++i)
     th.emplace_back([&] {
-      for (int l; (l = next.fetch_add(1)) < m.n_layers;) do_layer(l);
+      for (int l; (l = next.fetch_add(1)) < m.n_layers + lm_tasks;) {
+        if (l < m.n_layers)
+          do_layer(l);
+        else
+          do_lm(l - m.n_layers);
+      }
     });
   gain(w.final_norm, g.lay.final_norm);
   memcpy(img + g.lay.embed, w.embed, (size_t)m.vocab * h * 2);

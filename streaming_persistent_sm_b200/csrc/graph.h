@@ -18,6 +18,10 @@ struct Plan {
   int act_bytes;        // activation staging per worker (fp32)
   int prefill_mode;     // 1 = tensor-core prefill program, 2 = token by token
   int per_op_slot;      // ring bytes of a per-op CTA (holds one whole tile)
+  int decode_mode;      // WPK_DECODE_GEMV or WPK_DECODE_MMA (resolved)
+  // batched decode program: MMA N (max_batch rounded up to 16), its ring
+  // stage (16 KB of weights + hi/lo activation chunks), stages, scratch bytes
+  int dec_n, dec_stage_bytes, dec_stages, dec_act_bytes;
 };
 
 struct Layout {
@@ -26,6 +30,8 @@ struct Layout {
   uint64_t total = 0;
   int down_kc = 0, n_down_chunks = 0;
   bool mma = false;     // tensor-core image present
+  uint64_t lm_mma = 0;  // tensor-core image of the LM head (batched decode only)
+  int vocab_blocks = 0; // 128-row blocks of that image (last one zero-padded)
 };
 
 struct CompiledGraph {
@@ -43,6 +49,8 @@ struct CompiledGraph {
   int64_t algo_weight_bytes = 0;              // weight bytes a step reads
   int n_splits = 0, split_tokens = 0, max_blocks = 0;
   int B = 0, T = 0, M = 0, n_tb = 0;  // prefill programs
+  int W = 0;                          // workers the tiles were sized for
+  int o_splits = 0, down_splits = 0;  // batched decode: K splits of O and down
 };
 
 // Returns "" on success, else an error message; *code receives the WPK code.

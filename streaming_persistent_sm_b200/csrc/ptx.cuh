@@ -150,6 +150,12 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16) {
 
 // Byte offset of element (row, col) inside a [rows][64] 16-bit tile stored
 // with the 128-byte swizzle: the 16-byte unit index is XORed with row % 8.
+// Relaxed add of four floats to a 16-byte aligned global address (one vector
+// reduction instead of four scalar ones).
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
   const uint32_t unit = (col >> 3) ^ (row & 7u);
   return row * 128u + unit * 16u + (col & 7u) * 2u;

@@ -197,7 +197,9 @@ __device__ __forceinline__ AttnSpan attn_span(const KParams& P, const Tile& T) {
 // ---------------------------------------------------------------------------
 // Producer side: how a tile's staging data is cut into chunks, and the copies.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool is_mma_op(int op) { return op >= OP_MQKV && op <= OP_MDOWN; }
+__device__ __forceinline__ bool is_mma_op(int op) {
+  return (op >= OP_MQKV && op <= OP_MDOWN) || (op >= OP_BQKV && op <= OP_BLM);
+}
 
 // Prefill attention: queries [t0, t1) of sequence b read keys [0, t1).
 __device__ __forceinline__ void pattn_span(const KParams& P, const Tile& T, int* t0, int* t1) {
@@ -219,10 +221,10 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
     *n_chunks = (t1 - 1) / P.page_tokens + 1;
     return;
   }
-  if (T.op == OP_ATTN) {
+  if (T.op == OP_ATTN) {  // one KV page per chunk
     if (T.a0 >= active_batch(P)) return;
     const AttnSpan s = attn_span(P, T);
-    *n_chunks = s.t1 > s.t0 ? 1 : 0;
+    *n_chunks = s.t1 > s.t0 ? (s.t1 - 1) / P.page_tokens - s.t0 / P.page_tokens + 1 : 0;
     return;
   }
   if (T.w_bytes == 0) return;
@@ -232,21 +234,32 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
   *n_chunks = (T.a1 + *rpc - 1) / *rpc;
 }
 
-// Source image (hi; lo follows) of a tensor-core tile's activations.
+// Source image (hi or lo) of a tensor-core tile's activations: the tile covers
+// the K range [a2, a2 + a3) of token block a1 (the batched decode program has
+// one token block); a token block's image holds the op's whole K.
 __device__ __forceinline__ const uint8_t* mma_act_src(const KParams& P, const Tile& T, int part) {
-  const uint8_t* const* img = (T.op == OP_MO) ? P.att_img : (T.op == OP_MDOWN) ? P.h_img : P.xn_img;
-  return img[part] + ((size_t)T.a1 * (T.a3 / 64)) * kMmaChunkBytes;
+  const uint8_t* const* img;
+  int k_full;  // the op's whole K: a token block's image holds k_full / 64 chunks
+  switch (T.op) {
+    case OP_MO: case OP_BO: img = P.att_img; k_full = P.q_rows; break;
+    case OP_MDOWN: case OP_BDOWN: img = P.h_img; k_full = P.ffn; break;
+    case OP_BGU: img = P.xf_img; k_full = P.hidden; break;
+    default: img = P.xn_img; k_full = P.hidden; break;
+  }
+  return img[part] + ((size_t)T.a1 * (k_full / 64) + T.a2 / 64) * P.act_chunk;
 }
 
 // Tensor-core tile chunk k: arm the barrier with all its bytes and copy the
-// weight block (the activation blocks follow in issue_mma_act).
+// weight block (the activation blocks follow in issue_mma_act).  A stage holds
+// the 16 KB weight block, then the hi and the lo activation chunk.
 __device__ void issue_mma_w(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
-  mbar_arrive_expect_tx(bar, 3u * kMmaChunkBytes);
+  mbar_arrive_expect_tx(bar, (uint32_t)kMmaChunkBytes + 2u * (uint32_t)P.act_chunk);
   bulk_g2s(dst, P.weights + T.w_off + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
 }
 __device__ void issue_mma_act(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
-  bulk_g2s(dst + kMmaChunkBytes, mma_act_src(P, T, 0) + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
-  bulk_g2s(dst + 2 * kMmaChunkBytes, mma_act_src(P, T, 1) + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
+  const uint32_t a = (uint32_t)P.act_chunk;
+  bulk_g2s(dst + kMmaChunkBytes, mma_act_src(P, T, 0) + (size_t)k * a, a, bar);
+  bulk_g2s(dst + kMmaChunkBytes + a, mma_act_src(P, T, 1) + (size_t)k * a, a, bar);
 }
 
 // Copies of chunk `k` of tile T into `dst`; arms `bar` with their bytes.
@@ -263,22 +276,16 @@ __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uin
     bulk_g2s(dst + (size_t)page * hd * 2, P.kv + kv_index(P, T.layer, blk, 1, T.a1, 0), bytes, bar);
     return;
   }
-  if (T.op == OP_ATTN) {
+  if (T.op == OP_ATTN) {  // page k of the split: K rows, then V rows at page * head_dim
     const AttnSpan s = attn_span(P, T);
     const int page = P.page_tokens, hd = P.head_dim;
-    const int p0 = s.t0 / page, p1 = (s.t1 - 1) / page;
-    uint32_t total = 0;
-    for (int p = p0; p <= p1; ++p) total += 2u * (uint32_t)min(page, s.t1 - p * page) * hd * 2;
-    mbar_arrive_expect_tx(bar, total);
-    const uint32_t vbase = (uint32_t)P.split_tokens * hd * 2;
-    for (int p = p0; p <= p1; ++p) {
-      const int rows = min(page, s.t1 - p * page);
-      const int blk = P.block_table[s.b * P.max_blocks + p];
-      const uint32_t bytes = (uint32_t)rows * hd * 2;
-      const uint32_t off = (uint32_t)(p - p0) * page * hd * 2;
-      bulk_g2s(dst + off, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, bar);
-      bulk_g2s(dst + vbase + off, P.kv + kv_index(P, T.layer, blk, 1, s.g, 0), bytes, bar);
-    }
+    const int p = s.t0 / page + k;
+    const int rows = min(page, s.t1 - p * page);
+    const int blk = P.block_table[s.b * P.max_blocks + p];
+    const uint32_t bytes = (uint32_t)rows * hd * 2;
+    mbar_arrive_expect_tx(bar, 2 * bytes);
+    bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, bar);
+    bulk_g2s(dst + (size_t)page * hd * 2, P.kv + kv_index(P, T.layer, blk, 1, s.g, 0), bytes, bar);
     return;
   }
   const size_t row_bytes = (size_t)T.a3 * 2;
@@ -618,49 +625,90 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
 
 // ---------------------------------------------------------------------------
 // Split-KV GQA decode attention.  The tile (b, g, j) handles the `group`
-// query heads of kv head g over tokens [j*S, (j+1)*S) of sequence b, writes
-// an online-softmax partial (m, l, o), and the last split to arrive combines
-// all partials of (b, g) ("Persistent threads and megakernels", §6: split long
-// histories into chunks, combine partial attention in a reduction signalled
-// through global memory).
+// query heads of kv head g over the tokens of split j of sequence b, one KV
+// page per staged chunk with an online softmax across the pages; it writes a
+// partial (m, l, o) and the last split to arrive combines all partials of
+// (b, g) ("Persistent threads and megakernels", §6: split long histories into
+// chunks, combine partial attention in a reduction signalled through global
+// memory).  A single split writes its result directly.
+//
+// Batched decode program: the current token's q, k and v are still fp32 sums
+// (acc, feature-major); the tile whose split holds the current position rounds
+// k and v to bf16, writes them to the KV cache and clears their sums, and the
+// tile that writes the result clears the q sums.  The result goes to the hi/lo
+// attention image that the O projection's tensor-core tiles read.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void attn_result(const KParams& P, int b, int f, float v) {
+  if (P.dec_mma) {
+    const size_t off = (size_t)(f >> 6) * P.act_chunk + sw128_offset(b, f & 63);
+    const __nv_bfloat16 hb = __float2bfloat16_rn(v);
+    *reinterpret_cast<__nv_bfloat16*>(P.att_img[0] + off) = hb;
+    *reinterpret_cast<__nv_bfloat16*>(P.att_img[1] + off) = __float2bfloat16_rn(v - __bfloat162float(hb));
+    P.acc[(size_t)f * P.mma_n + b] = 0.f;  // q sums start from zero next step
+  } else {
+    P.attn[(size_t)b * P.q_rows + f] = v;
+  }
+}
+
 __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cursor& cur, int n_chunks,
                           volatile int* abort) {
   if (T.a0 >= active_batch(P)) return true;
   __shared__ int s_last;
-  __shared__ float s_m[kMaxGroup], s_l[kMaxGroup];
+  __shared__ float s_m[kMaxGroup], s_l[kMaxGroup], s_sc[kMaxGroup];
   const AttnSpan s = attn_span(P, T);
-  const int hd = P.head_dim, grp = P.group, S = P.split_tokens;
-  const int n = s.t1 - s.t0;
+  const int hd = P.head_dim, grp = P.group, page = P.page_tokens;
+  const int nq = grp * hd;  // (head, dim) pairs: thread i owns pairs i and i + 256
   float* part = P.part + ((((size_t)s.b * P.n_kv + s.g) * P.n_splits + s.j) * grp) * (2 + hd);
   float* q_s = Sh.act;                    // [grp][hd]
-  float* p_s = Sh.act + kMaxGroup * hd;   // [grp][S]
-  if (n_chunks > 0) {
-    const int st = cur.c % P.n_stages;
-    const uint32_t par = (cur.c / P.n_stages) & 1u;
-    bool ok = wait_phase(P, &Sh.full[st], par, abort, 0xFFFFFFFFu);
+  float* p_s = Sh.act + kMaxGroup * hd;   // [grp][page]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float scale = 1.0f / sqrtf((float)hd);
+  float o[2] = {0.f, 0.f};
+  if (threadIdx.x < kMaxGroup) {
+    s_m[threadIdx.x] = -INFINITY;
+    s_l[threadIdx.x] = 0.f;
+  }
+  cbar();
+  for (int k = 0; k < n_chunks; ++k) {
+    const uint32_t c = cur.c;
+    const int st = c % P.n_stages;
+    const bool ok = wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu);
     if (!cbar_and(ok)) return false;
-    if (P.trace && threadIdx.x == 0) s_t_data = globaltimer();
+    if (P.trace && threadIdx.x == 0 && k + 1 == n_chunks) s_t_data = globaltimer();
     uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
-    const uint16_t* Ks = reinterpret_cast<const uint16_t*>(stage);
-    const uint16_t* Vs = reinterpret_cast<const uint16_t*>(stage + (size_t)S * hd * 2);
+    uint16_t* Ks = reinterpret_cast<uint16_t*>(stage);
+    uint16_t* Vs = reinterpret_cast<uint16_t*>(stage + (size_t)page * hd * 2);
+    const int p0 = (s.t0 / page + k) * page;  // first token of the staged page
+    const int n = min(page, s.t1 - p0);
     // the current token's row was written this step, after the copy was issued
-    if (s.pos >= s.t0 && s.pos < s.t1) {
-      const int blk = P.block_table[s.b * P.max_blocks + s.pos / P.page_tokens];
-      const int row = s.pos - s.t0;
-      const int lanes = hd * 2 / 16;
-      if (threadIdx.x < 2 * lanes) {
-        const int sel = threadIdx.x / lanes, piece = threadIdx.x % lanes;
-        const uint4* src = reinterpret_cast<const uint4*>(
-            P.kv + kv_index(P, T.layer, blk, sel, s.g, s.pos % P.page_tokens));
-        uint8_t* dst = stage + (size_t)sel * S * hd * 2 + (size_t)row * hd * 2;
-        reinterpret_cast<uint4*>(dst)[piece] = __ldcg(src + piece);
+    if (s.pos >= p0 && s.pos < p0 + n) {
+      const int row = s.pos - p0;
+      const int blk = P.block_table[s.b * P.max_blocks + s.pos / page];
+      if (P.dec_mma) {
+        for (int i = threadIdx.x; i < 2 * hd; i += kThreads) {
+          const int sel = i / hd, d = i % hd;
+          float* a = P.acc + (size_t)(P.q_rows + sel * P.kv_rows + s.g * hd + d) * P.mma_n + s.b;
+          const uint16_t v = f2bf(__ldcg(a));
+          *a = 0.f;
+          P.kv[kv_index(P, T.layer, blk, sel, s.g, s.pos % page) + d] = v;
+          (sel ? Vs : Ks)[(size_t)row * hd + d] = v;
+        }
+      } else {
+        const int lanes = hd * 2 / 16;
+        if (threadIdx.x < 2 * lanes) {
+          const int sel = threadIdx.x / lanes, piece = threadIdx.x % lanes;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              P.kv + kv_index(P, T.layer, blk, sel, s.g, s.pos % page));
+          uint8_t* dst = reinterpret_cast<uint8_t*>(sel ? Vs : Ks) + (size_t)row * hd * 2;
+          reinterpret_cast<uint4*>(dst)[piece] = __ldcg(src + piece);
+        }
       }
     }
-    for (int i = threadIdx.x; i < grp * hd; i += kThreads)
-      q_s[i] = __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * grp * hd + i);
+    if (k == 0)
+      for (int i = threadIdx.x; i < nq; i += kThreads)
+        q_s[i] = P.dec_mma ? __ldcg(P.acc + (size_t)(s.g * nq + i) * P.mma_n + s.b)
+                           : __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * nq + i);
     cbar();
-    const float scale = 1.0f / sqrtf((float)hd);
     const int words = hd / 2;
     for (int idx = threadIdx.x; idx < grp * n; idx += kThreads) {
       const int hh = idx / n, t = idx % n;
@@ -673,39 +721,62 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
         acc = fmaf(qr[2 * ww], __uint_as_float(kk << 16), acc);
         acc = fmaf(qr[2 * ww + 1], __uint_as_float(kk & 0xFFFF0000u), acc);
       }
-      p_s[hh * S + t] = acc * scale;
+      p_s[hh * page + t] = acc * scale;
     }
     cbar();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp < grp) {
-      float m = -INFINITY;
-      for (int t = lane; t < n; t += 32) m = fmaxf(m, p_s[warp * S + t]);
-      m = warp_max(m);
+    if (warp < grp) {  // running max and sum of head `warp`
+      float mx = -INFINITY;
+      for (int t = lane; t < n; t += 32) mx = fmaxf(mx, p_s[warp * page + t]);
+      mx = warp_max(mx);
+      const float m_old = s_m[warp], m_new = fmaxf(m_old, mx);
       float l = 0.f;
       for (int t = lane; t < n; t += 32) {
-        const float e = expf(p_s[warp * S + t] - m);
-        p_s[warp * S + t] = e;
+        const float e = expf(p_s[warp * page + t] - m_new);
+        p_s[warp * page + t] = e;
         l += e;
       }
       l = warp_sum(l);
-      if (lane == 0) { s_m[warp] = m; s_l[warp] = l; }
+      if (lane == 0) {
+        const float sc = expf(m_old - m_new);
+        s_sc[warp] = sc;
+        s_l[warp] = s_l[warp] * sc + l;
+        s_m[warp] = m_new;
+      }
     }
     cbar();
-    for (int idx = threadIdx.x; idx < grp * hd; idx += kThreads) {
-      const int hh = idx / hd, d = idx % hd;
-      float o = 0.f;
-      for (int t = 0; t < n; ++t) o = fmaf(p_s[hh * S + t], bf2f(Vs[(size_t)t * hd + d]), o);
-      float* pr = part + (size_t)hh * (2 + hd);
-      pr[2 + d] = o;
-      if (d == 0) { pr[0] = s_m[hh]; pr[1] = s_l[hh]; }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = threadIdx.x + r * kThreads;
+      if (i < nq) {
+        const int hh = i / hd, d = i % hd;
+        float a = 0.f;
+        for (int t = 0; t < n; ++t) a = fmaf(p_s[hh * page + t], bf2f(Vs[(size_t)t * hd + d]), a);
+        o[r] = o[r] * s_sc[hh] + a;
+      }
     }
     cbar();
     if (threadIdx.x == 0) mbar_arrive(&Sh.empty[st]);
     ++cur.c;
-  } else {
-    for (int idx = threadIdx.x; idx < grp * (2 + hd); idx += kThreads) {
-      const int k = idx % (2 + hd);
-      part[idx] = (k == 0) ? -INFINITY : 0.f;
+  }
+  if (P.n_splits == 1) {  // the only split: the result directly
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int i = threadIdx.x + r * kThreads;
+      if (i < nq) attn_result(P, s.b, s.g * nq + i, o[r] / s_l[i / hd]);
+    }
+    return true;
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int i = threadIdx.x + r * kThreads;
+    if (i < nq) {
+      const int hh = i / hd, d = i % hd;
+      float* pr = part + (size_t)hh * (2 + hd);
+      pr[2 + d] = o[r];
+      if (d == 0) {
+        pr[0] = s_m[hh];  // -inf with l = 0 for a split past the current position
+        pr[1] = s_l[hh];
+      }
     }
   }
   cbar();
@@ -727,7 +798,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
       ml[2 * i + 1] = v.y;
     }
     cbar();
-    for (int idx = threadIdx.x; idx < grp * hd; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < nq; idx += kThreads) {
       const int hh = idx / hd, d = idx % hd;
       float M = -INFINITY;
       for (int j = 0; j < P.n_splits; ++j) M = fmaxf(M, ml[2 * (j * grp + hh)]);
@@ -738,13 +809,12 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
         L = fmaf(ml[2 * (j * grp + hh) + 1], w, L);
         O = fmaf(__ldcg(base + ((size_t)j * grp + hh) * (2 + hd) + 2 + d), w, O);
       }
-      P.attn[(size_t)s.b * P.q_rows + ((size_t)s.g * grp + hh) * hd + d] = O / L;
+      attn_result(P, s.b, s.g * nq + idx, O / L);
     }
     if (threadIdx.x == 0) *arr = 0u;
   }
   return true;
 }
-
 
 // ---------------------------------------------------------------------------
 // Prefill bodies.  Token row m = b*T + t; block tb holds rows [128 tb, 128 tb + 128).
@@ -845,6 +915,32 @@ __device__ bool body_norm(const KParams& P, const Tile& T) {
   return true;
 }
 
+// Batched decode: 1/rms of each token column for the RMSNorm a tile consumes,
+// and the tile's best (value, index) key per token of the LM head.
+__shared__ float s_rn[kMaxMmaBatch];
+__shared__ unsigned long long s_best[kMaxMmaBatch];
+
+// Adds the 16 token columns n0..n0+15 (those below nb) of one feature row to a
+// feature-major fp32 buffer row `dst` (16-byte aligned at column n0).
+__device__ __forceinline__ void red_add_cols(float* dst, const float* o, int n0, int nb) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 4) {
+    if (n0 + j + 4 <= nb) {
+      red_add_v4_f32(dst + j, o[j], o[j + 1], o[j + 2], o[j + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (n0 + j + e < nb) atomicAdd(dst + j + e, o[j + e]);
+    }
+  }
+}
+
+__device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
+  const uint32_t fb = __float_as_uint(v);
+  const uint32_t ord = (fb & 0x80000000u) ? ~fb : (fb | 0x80000000u);
+  return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)idx);
+}
+
 // Tensor-core tile epilogue for 16 token columns n0..n0+15 of feature row fl.
 __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, const float* v) {
   const int f = T.a0 * 128 + fl;
@@ -852,6 +948,74 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
   const int lane = threadIdx.x & 31;
   const int hd = P.head_dim, half = hd / 2;
   switch (T.op) {
+    case OP_BQKV: {
+      // 128-row blocks never straddle q / k / v; q and k rows hold RoPE pairs
+      // (i, i + hd/2) next to each other (even lane: i, odd lane: i + hd/2)
+      const int nb = active_batch(P);
+      const bool is_q = f < P.q_rows, is_v = f >= P.q_rows + P.kv_rows;
+      const int sec0 = is_q ? 0 : (is_v ? P.q_rows + P.kv_rows : P.q_rows);
+      const int head = (f - sec0) / hd, within = (f - sec0) % hd;
+      const bool even = (lane & 1) == 0;
+      const int pi = within / 2;
+      const int dim = is_v ? within : (even ? pi : pi + half);
+      float o[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float y = v[i] * s_rn[n0 + i];
+        const float partner = __shfl_xor_sync(0xffffffffu, y, 1);
+        if (is_v) {
+          o[i] = y;
+        } else {
+          const int n = n0 + i;
+          const float2 cs = P.rope[(size_t)(n < nb ? P.seqlen[n] : 0) * half + pi];
+          const float y0 = even ? y : partner, y1 = even ? partner : y;
+          o[i] = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
+        }
+      }
+      red_add_cols(P.acc + (size_t)(sec0 + head * hd + dim) * P.mma_n + n0, o, n0, nb);
+      break;
+    }
+    case OP_BO:
+    case OP_BDOWN:
+      red_add_cols(P.xt + (size_t)f * P.mma_n + n0, v, n0, active_batch(P));
+      break;
+    case OP_BGU: {
+      const int nb = active_batch(P);
+      const int col = fl / 2;  // h feature 64 * a0 + col
+      uint8_t* hi = P.h_img[0] + (size_t)T.a0 * P.act_chunk;
+      uint8_t* lo = P.h_img[1] + (size_t)T.a0 * P.act_chunk;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float g = v[i] * s_rn[n0 + i];
+        const float up = __shfl_xor_sync(0xffffffffu, g, 1);
+        if (lane & 1) continue;
+        const int n = n0 + i;
+        const float hv = (n < nb) ? g / (1.0f + expf(-g)) * up : 0.f;
+        const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+        const uint32_t off = sw128_offset(n, col);
+        *reinterpret_cast<__nv_bfloat16*>(hi + off) = hb;
+        *reinterpret_cast<__nv_bfloat16*>(lo + off) = __float2bfloat16_rn(hv - __bfloat162float(hb));
+      }
+      break;
+    }
+    case OP_BLM: {
+      const int nb = active_batch(P);
+      const bool valid = f < P.vocab;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int n = n0 + i;
+        const float val = v[i] * s_rn[n];
+        if (P.logits && valid && n < nb) P.logits[(size_t)n * P.vocab + f] = val;
+        unsigned long long key = valid ? argmax_key(val, f) : 0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+          key = other > key ? other : key;
+        }
+        if (lane == 0 && n < nb) atomicMax(&s_best[n], key);
+      }
+      break;
+    }
     case OP_MQKV: {
       const bool is_v = f >= P.q_rows + P.kv_rows;
       const bool is_q = f < P.q_rows;
@@ -884,11 +1048,11 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       break;
     }
     case OP_MO:
-    case OP_MDOWN: {
+    case OP_MDOWN: {  // K splits of one row block add into X
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int m = tb * kTokBlock + n0 + i;
-        if (m < P.M) P.px[(size_t)m * P.hidden + f] += v[i];
+        if (m < P.M) atomicAdd(P.px + (size_t)m * P.hidden + f, v[i]);
       }
       break;
     }
@@ -917,16 +1081,78 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
   }
 }
 
+// Batched decode, after an O or down tile: the last of the K splits of its
+// 128-row block to finish holds the block's final residual rows.  It writes
+// them, times the gain of the RMSNorm that reads them next (this layer's FFN
+// norm after O; the next layer's attention norm, or the final norm, after
+// down), into that norm's hi/lo input image and adds their squares to the
+// per-token sums of x^2 (the consumers scale by 1/rms per token).  Splits
+// arrive on a counter per row block (release/acquire through fences, as the
+// attention combine).  Columns past the active batch get zeros.
+__device__ void rowblock_done(const KParams& P, const Tile& T) {
+  __shared__ int s_last_rb;
+  __shared__ float s_sq[kMaxMmaBatch];
+  const bool down = T.op == OP_BDOWN;
+  const int splits = down ? P.down_splits : P.o_splits;
+  const int N = P.mma_n, nb = active_batch(P);
+  if (threadIdx.x < N) s_sq[threadIdx.x] = 0.f;
+  if (threadIdx.x == 0) {
+    uint32_t* a = P.rb_arrive + ((size_t)T.layer * 2 + (down ? 1 : 0)) * (P.hidden / 128) + T.a0;
+    __threadfence();
+    const uint32_t old = atomicAdd(a, 1u);
+    s_last_rb = old == (uint32_t)splits - 1u;
+    if (s_last_rb) *a = 0u;
+    __threadfence();
+  }
+  cbar();
+  if (!s_last_rb) return;
+  const int nidx = down ? 2 * T.layer + 2 : 2 * T.layer + 1;
+  const uint64_t goff = !down ? P.layers[T.layer].ffn_norm
+                              : (T.layer + 1 < P.n_layers ? P.layers[T.layer + 1].attn_norm : P.final_norm_off);
+  const float* gain = reinterpret_cast<const float*>(P.weights + goff);
+  uint8_t* const* img = down ? P.xn_img : P.xf_img;
+  for (int u = threadIdx.x; u < 16 * N; u += kThreads) {  // (8 features, token n) per step
+    const int j = u / N, n = u % N;
+    const int f0 = T.a0 * 128 + 8 * j;
+    float x[8];
+    float sq = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      x[e] = n < nb ? __ldcg(P.xt + (size_t)(f0 + e) * N + n) : 0.f;
+      sq = fmaf(x[e], x[e], sq);
+    }
+    const float4 g0 = __ldg(reinterpret_cast<const float4*>(gain + f0));
+    const float4 g1 = __ldg(reinterpret_cast<const float4*>(gain + f0 + 4));
+    const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    uint32_t ph[4], pl[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float a0 = x[e] * gg[e], a1 = x[e + 1] * gg[e + 1];
+      const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+      ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+      pl[e / 2] = pack_bf16x2(a0 - __bfloat162float(hv.x), a1 - __bfloat162float(hv.y));
+    }
+    const size_t off = (size_t)(f0 / 64) * P.act_chunk + sw128_offset(n, f0 % 64);
+    *reinterpret_cast<uint4*>(img[0] + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+    *reinterpret_cast<uint4*>(img[1] + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+    if (n < nb) atomicAdd(&s_sq[n], sq);
+  }
+  cbar();
+  if (threadIdx.x < nb) atomicAdd(P.ss + (size_t)nidx * N + threadIdx.x, s_sq[threadIdx.x]);
+}
+
 // Tensor-core tile: D[128 features][128 tokens] = W . (a_hi + a_lo)^T over the
 // tile's K chunks.  Thread 0 issues the MMAs as chunks land and commits each
 // stage back to the producer; all compute warps then read TMEM.
 __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
                          ConsumerState& cs, volatile int* abort, uint32_t tile) {
   const uint32_t tmem = s_tmem;
+  const int N = P.mma_n;
   if (threadIdx.x == 0) {
     bool ok = true;
     uint32_t cc = cur.c;
-    const uint32_t idesc = idesc_f16(128, kTokBlock, true);
+    const uint32_t idesc = idesc_f16(128, N, true);
+    const uint32_t a_off = (uint32_t)P.act_chunk;
     for (int k = 0; k < n_chunks; ++k, ++cc) {
       const int st = cc % P.n_stages;
       if (!wait_phase(P, &S.full[st], (cc / P.n_stages) & 1u, abort, tile)) {
@@ -939,12 +1165,20 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = sdesc_k_sw128(base + kk * 32);
         umma_f16(tmem, ad, sdesc_k_sw128(base + kMmaChunkBytes + kk * 32), idesc, (k | kk) != 0);
-        umma_f16(tmem, ad, sdesc_k_sw128(base + 2 * kMmaChunkBytes + kk * 32), idesc, 1);
+        umma_f16(tmem, ad, sdesc_k_sw128(base + kMmaChunkBytes + a_off + kk * 32), idesc, 1);
       }
       umma_commit(&S.empty[st]);
     }
     umma_commit(S.acc);
     s_mma_ok = ok;
+  }
+  // batched decode: 1/rms per token column of the RMSNorm this tile consumes
+  // (its x^2 sums are complete: the tile's counter covers every contribution)
+  if (T.op == OP_BQKV || T.op == OP_BGU || T.op == OP_BLM) {
+    const int idx = T.op == OP_BQKV ? 2 * T.layer : (T.op == OP_BGU ? 2 * T.layer + 1 : 2 * P.n_layers);
+    if (threadIdx.x < N)
+      s_rn[threadIdx.x] = 1.0f / sqrtf(__ldcg(P.ss + (size_t)idx * N + threadIdx.x) / (float)P.hidden + P.eps);
+    if (threadIdx.x < N) s_best[threadIdx.x] = 0ull;
   }
   cbar();
   bool ok = s_mma_ok;
@@ -956,14 +1190,19 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, half = warp >> 2;
   const int fl = 32 * q + lane;
-  for (int c0 = 0; c0 < kTokBlock / 2; c0 += 16) {
+  for (int cg = half; cg < N / 16; cg += 2) {  // 16-column groups alternate between the two warp halves
     float v[16];
-    const int n0 = half * (kTokBlock / 2) + c0;
-    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)n0, v);
-    mma_epilogue(P, T, fl, n0, v);
+    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(16 * cg), v);
+    mma_epilogue(P, T, fl, 16 * cg, v);
   }
   tc_fence_before();
   cbar();
+  if (T.op == OP_BO || T.op == OP_BDOWN) {
+    rowblock_done(P, T);
+  } else if (T.op == OP_BLM) {
+    const int nb = active_batch(P);
+    if (threadIdx.x < nb && s_best[threadIdx.x]) atomicMax(P.best + threadIdx.x, s_best[threadIdx.x]);
+  }
   return true;
 }
 
@@ -1092,8 +1331,60 @@ __device__ bool body_embed(const KParams& P) {
   return true;
 }
 
+// Batched decode: x = E[tok] for the 128 features of block a0, feature-major,
+// with the first RMSNorm's input image (x * g) and the x^2 sums.
+__device__ bool body_embed_mma(const KParams& P, const Tile& T) {
+  __shared__ int s_tok[kMaxMmaBatch];
+  __shared__ float s_sq2[kMaxMmaBatch];
+  const int N = P.mma_n, nb = active_batch(P);
+  if (threadIdx.x < N) {
+    int tok = 0;
+    if (threadIdx.x < nb) {
+      tok = P.in_tok ? P.in_tok[(size_t)threadIdx.x * P.in_tok_stride] : P.tok_fb[threadIdx.x];
+      if (tok < 0 || tok >= P.vocab) {
+        record_error(P, WPK_ERR_INVALID_ARG, 0, kNoCounter, (uint32_t)tok, (uint32_t)P.vocab);
+        tok = 0;
+      }
+    }
+    s_tok[threadIdx.x] = tok;
+    s_sq2[threadIdx.x] = 0.f;
+  }
+  cbar();
+  const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
+  const float* gain = reinterpret_cast<const float*>(P.weights + P.layers[0].attn_norm);
+  for (int u = threadIdx.x; u < 16 * N; u += kThreads) {
+    const int j = u / N, n = u % N;
+    const int f0 = T.a0 * 128 + 8 * j;
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (n < nb) unpack8(__ldg(reinterpret_cast<const uint4*>(E + (size_t)s_tok[n] * P.hidden + f0)), x);
+    float sq = 0.f;
+    uint32_t ph[4], pl[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      sq = fmaf(x[e], x[e], fmaf(x[e + 1], x[e + 1], sq));
+      const float a0 = x[e] * gain[f0 + e], a1 = x[e + 1] * gain[f0 + e + 1];
+      const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+      ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+      pl[e / 2] = pack_bf16x2(a0 - __bfloat162float(hv.x), a1 - __bfloat162float(hv.y));
+    }
+    if (n < nb) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) P.xt[(size_t)(f0 + e) * N + n] = x[e];
+      atomicAdd(&s_sq2[n], sq);
+    }
+    const size_t off = (size_t)(f0 / 64) * P.act_chunk + sw128_offset(n, f0 % 64);
+    *reinterpret_cast<uint4*>(P.xn_img[0] + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+    *reinterpret_cast<uint4*>(P.xn_img[1] + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+  }
+  cbar();
+  if (threadIdx.x < nb) atomicAdd(P.ss + threadIdx.x, s_sq2[threadIdx.x]);
+  return true;
+}
+
 __device__ bool body_final(const KParams& P) {
   const int nb = active_batch(P);
+  if (P.dec_mma)  // the x^2 sums start from zero next step
+    for (int i = threadIdx.x; i < (2 * P.n_layers + 1) * P.mma_n; i += kThreads) P.ss[i] = 0.f;
   for (int b = threadIdx.x; b < nb; b += kThreads) {
     const unsigned long long key = P.best[b];
     const int32_t idx = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
@@ -1131,6 +1422,11 @@ __device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, vol
 // The worker: producer warp (warp 8) + consumer warps (0..7).
 // ---------------------------------------------------------------------------
 __device__ void worker(const KParams& P, uint8_t* smem_raw) {
+  // the 128-byte-swizzled tensor-core operands need 1024-byte aligned stages
+  if (P.uses_tmem && (smem_u32(smem_raw) & 1023u)) {
+    if (threadIdx.x == 0) record_error(P, WPK_ERR_UNSUPPORTED, 0xFFFFFFFFu, kNoCounter, smem_u32(smem_raw), 1024u);
+    return;
+  }
   const Shared S = carve(smem_raw, P);
   __shared__ volatile int s_abort;
   __shared__ uint32_t s_prod_chunks;  // chunks the producer issued
@@ -1296,7 +1592,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       bool ok = !s_fail;
       if (ok) {
         switch (T.op) {
-          case OP_EMBED: ok = body_embed(P); break;
+          case OP_EMBED: ok = P.dec_mma ? body_embed_mma(P, T) : body_embed(P); break;
           case OP_ATTN: ok = body_attn(P, T, S, cur, n_chunks, &s_abort); break;
           case OP_FINAL: ok = body_final(P); break;
           case OP_PEMBED: ok = body_pembed(P, T); break;
@@ -1306,7 +1602,12 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           case OP_MQKV:
           case OP_MO:
           case OP_MGU:
-          case OP_MDOWN: ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t); break;
+          case OP_MDOWN:
+          case OP_BQKV:
+          case OP_BO:
+          case OP_BGU:
+          case OP_BDOWN:
+          case OP_BLM: ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t); break;
           default: ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort); break;
         }
         // attention tiles use the activation buffer as scratch; the gather

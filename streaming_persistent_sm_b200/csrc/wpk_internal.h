@@ -39,11 +39,18 @@ enum Op : uint16_t {
   OP_MDOWN = 13,   // X += Wd . h on tensor cores
   OP_PATTN = 14,   // causal GQA attention of one query block (CUDA cores)
   OP_GATHER = 15,  // xa[b] = X[last prompt position of b]
-  OP_COUNT = 16
+  // batched decode program (the step's tokens are the MMA N dimension)
+  OP_BQKV = 16,    // [q;k;v] partial over a K range on tensor cores, RoPE, summed into acc
+  OP_BO = 17,      // x += Wo . attn over a K range; last split -> RMSNorm input image
+  OP_BGU = 18,     // gate/up on tensor cores, SwiGLU -> hi/lo image of h
+  OP_BDOWN = 19,   // x += Wd . h over a K range; last split -> RMSNorm input image
+  OP_BLM = 20,     // logits on tensor cores + packed argmax
+  OP_COUNT = 21
 };
 
 constexpr int kTokBlock = 128;   // tokens per tensor-core tile (the MMA N)
 constexpr int kPrefillQB = 32;   // queries per prefill attention tile
+constexpr int kMaxMmaBatch = 128;  // sequences of a batched decode step (MMA N <= 128)
 constexpr int kMmaChunkBytes = 128 * 128;  // 128 rows x 64 bf16, one K chunk
 
 // One tile of the step program, in ticket order.  48 bytes.
@@ -149,6 +156,19 @@ struct KParams {
   uint8_t* xn_img[2];        // hi/lo image of the normalised activations [n_tb][hidden/64][16 KB]
   uint8_t* att_img[2];       // hi/lo image of the attention output     [n_tb][q_rows/64][16 KB]
   uint8_t* h_img[2];         // hi/lo image of the SwiGLU output        [n_tb][ffn/64][16 KB]
+  // tensor-core operand geometry: the MMA N (tokens per tile) and the bytes of
+  // one 64-column activation chunk (N rows of 128 bytes, 128-byte swizzle)
+  int mma_n, act_chunk;
+  // batched decode program (dec_mma = 1).  Token n of the step is MMA column n;
+  // columns >= the active batch hold zeros.  Images are [K/64][act_chunk].
+  int dec_mma;
+  int o_splits, down_splits;  // K splits of the O and down projections
+  float* xt;                  // [hidden][mma_n] residual stream, feature-major
+  float* acc;                 // [qkv_rows][mma_n] q/k/v sums (zero between uses)
+  float* ss;                  // [2 n_layers + 1][mma_n] sums of x^2 per RMSNorm
+  uint8_t* xf_img[2];         // hi/lo image of x * g_ffn (xn_img holds x * g_attn / g_final)
+  uint32_t* rb_arrive;        // [n_layers][2][hidden/128] split-K arrivals per row block
+  uint64_t lm_mma_off;        // tensor-core image of the LM head [vocab/128][hidden/64][16 KB]
 };
 
 // Host-side compiled graph.
@@ -163,6 +183,8 @@ enum Buf {
   BUF_XA = 0, BUF_XB, BUF_QKV, BUF_ATTN, BUF_H, BUF_LOGITS, BUF_BEST, BUF_TOK,
   // prefill buffers, modelled per token block (index = block * width * 128 + feature * 128 + row)
   BUF_PX, BUF_PXN, BUF_PQ, BUF_PKV, BUF_PATT, BUF_PH,
+  // batched decode: the RMSNorm input images (x * g_attn or g_final; x * g_ffn)
+  BUF_DXN, BUF_DXF,
   BUF_COUNT
 };
 

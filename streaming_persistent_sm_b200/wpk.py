@@ -31,9 +31,13 @@ WPK_SCHED_STATIC = 1
 WPK_PREFILL_AUTO = 0
 WPK_PREFILL_MMA = 1
 WPK_PREFILL_TOKENWISE = 2
+WPK_DECODE_AUTO = 0
+WPK_DECODE_GEMV = 1
+WPK_DECODE_MMA = 2
 
 OP_NAMES = ["embed", "qkv", "attn", "o", "gate_up", "down", "lm_head", "final",
-            "p_embed", "norm", "mma_qkv", "mma_o", "mma_gate_up", "mma_down", "p_attn", "gather"]
+            "p_embed", "norm", "mma_qkv", "mma_o", "mma_gate_up", "mma_down", "p_attn", "gather",
+            "b_qkv", "b_o", "b_gate_up", "b_down", "b_lm_head"]
 
 _ERR_NAMES = {0: "OK", -1: "INVALID_ARG", -2: "CUDA", -3: "TIMEOUT", -4: "NOT_LOADED", -5: "SHAPE",
               -6: "UNSUPPORTED", -7: "POISONED"}
@@ -56,7 +60,8 @@ class wpk_plan_cfg(C.Structure):
                 ("n_workers", C.c_int), ("workers_per_sm", C.c_int), ("mode", C.c_int), ("resident", C.c_int),
                 ("n_regions", C.c_int), ("region_cut", C.c_int * 4), ("trace", C.c_int),
                 ("wait_timeout_ns", C.c_uint64), ("slot_bytes", C.c_int), ("tile_bytes", C.c_int),
-                ("split_pages", C.c_int), ("lookahead", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int)]
+                ("split_pages", C.c_int), ("lookahead", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int),
+                ("decode", C.c_int)]
 
 
 _P16 = C.POINTER(C.c_uint16)
@@ -145,11 +150,11 @@ def plan_cfg(max_batch: int, max_context: int, mode: int = WPK_MEGAKERNEL, n_reg
              region_cut: Sequence[int] = (0, 0, 0, 0), trace: int = 0, wait_timeout_ns: int = 0,
              page_tokens: int = 0, n_workers: int = 0, workers_per_sm: int = 0, resident: int = 0,
              slot_bytes: int = 0, tile_bytes: int = 0, split_pages: int = 0, lookahead: int = 0,
-             schedule: int = 0, prefill: int = 0) -> wpk_plan_cfg:
+             schedule: int = 0, prefill: int = 0, decode: int = 0) -> wpk_plan_cfg:
     cut = (C.c_int * 4)(*list(region_cut) + [0] * (4 - len(region_cut)))
     return wpk_plan_cfg(max_batch, max_context, page_tokens, n_workers, workers_per_sm, mode, resident, n_regions,
                         cut, trace, wait_timeout_ns, slot_bytes, tile_bytes, split_pages, lookahead, schedule,
-                        prefill)
+                        prefill, decode)
 
 
 # ----------------------------------------------------------- thin wrappers --

@@ -123,7 +123,8 @@ def test_simulator_reports_stuck_producer_as_timeout(lib):
 
 @pytest.mark.parametrize("bad", [
     dict(max_batch=0), dict(n_regions=5), dict(mode=7), dict(slot_bytes=1000),
-    dict(n_regions=2, region_cut=(0, 9, 0, 0)), dict(split_pages=8),
+    dict(n_regions=2, region_cut=(0, 9, 0, 0)), dict(split_pages=-1), dict(page_tokens=128), dict(decode=7),
+    dict(decode=W.WPK_DECODE_MMA, max_batch=129),
 ])
 def test_invalid_plans_are_rejected(lib, bad):
     with pytest.raises(W.WpkError):
@@ -186,5 +187,125 @@ def test_tokenwise_prefill_plan_has_no_prefill_program(lib):
         with pytest.raises(W.WpkError) as ei:
             W.wpk_select_program(h, 1, 8)
         assert ei.value.code == W.WPK_ERR_UNSUPPORTED
+    finally:
+        W.wpk_destroy(h)
+
+
+# ------------------------------------------------------- batched decode program
+def _ops(h):
+    st = W.wpk_graph_stats_get(h)
+    return st, np.array([W.OP_NAMES[o] for o in W.wpk_get_tile_ops(h, st["n_tiles"])])
+
+
+@pytest.mark.parametrize("B", [16, 12, 9])
+def test_batched_decode_program_verifies_and_simulates(lib, B):
+    # more than 8 sequences: the step runs on tensor-core tiles (AUTO)
+    h = _graph(max_batch=B, max_context=160)
+    try:
+        st, names = _ops(h)
+        for op in ("b_qkv", "b_o", "b_gate_up", "b_down", "b_lm_head"):
+            assert op in names, op
+        assert not {"qkv", "o", "gate_up", "down", "lm_head"} & set(names)
+        assert names[0] == "embed" and names[-1] == "final"
+        W.wpk_verify_graph(h)
+        # same weight bytes as the GEMV program: every matrix once, LM head tied
+        assert st["weight_bytes"] == sum(np.prod(s) * 2 for n, s, k in synth.tensor_specs(synth.TINY)
+                                         if k == "normal")
+        rc, order = W.wpk_simulate(h, 11, 2, 5, 10000, -1, st["n_tiles"])
+        assert rc == 0, W.wpk_last_error(h)
+        e = W.wpk_get_edges(h)
+        T = st["n_tiles"]
+        pos = np.empty(T, dtype=np.int64)
+        pos[order[:T]] = np.arange(T)
+        assert np.all(pos[e[:, 0]] < pos[e[:, 1]])
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_batched_decode_k_split_edges(lib):
+    # each down tile waits only for the gate/up tiles of its K range (one gate/up
+    # tile = 64 h features = one 64-column chunk), each O tile only for the
+    # attention tiles of the heads in its K range
+    s = synth.ModelShape(n_layers=1, hidden=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=2048, vocab=512)
+    h = _graph(s, max_batch=16, max_context=64, n_workers=64)
+    try:
+        W.wpk_verify_graph(h)
+        st, names = _ops(h)
+        e = W.wpk_get_edges(h)
+        gu = set(np.flatnonzero(names == "b_gate_up"))
+        down = np.flatnonzero(names == "b_down")
+        attn = set(np.flatnonzero(names == "attn"))
+        o = np.flatnonzero(names == "b_o")
+        assert len(down) > 2 and len(o) > 2  # both projections are split along K
+        pred_sets = []
+        for v in down:
+            p = set(e[e[:, 1] == v, 0])
+            assert p <= gu and 0 < len(p) < len(gu)
+            pred_sets.append(frozenset(p))
+        assert len(set(pred_sets)) > 1
+        for v in o:
+            p = set(e[e[:, 1] == v, 0]) - set(np.flatnonzero(names == "embed"))
+            assert p <= attn and 0 < len(p) <= len(attn)
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_decode_mode_selection(lib):
+    for B, want in ((8, "lm_head"), (9, "b_lm_head"), (48, "b_lm_head")):
+        h = _graph(max_batch=B, max_context=64)
+        try:
+            _, names = _ops(h)
+            assert want in names and names[-2] == want
+        finally:
+            W.wpk_destroy(h)
+    h = _graph(max_batch=32, max_context=64, decode=W.WPK_DECODE_GEMV)
+    try:
+        _, names = _ops(h)
+        assert "lm_head" in names and "b_qkv" not in names
+    finally:
+        W.wpk_destroy(h)
+    # shapes that are not multiples of the 128-row tensor-core tiles
+    odd = synth.ModelShape(n_layers=1, hidden=192, n_heads=3, n_kv_heads=1, head_dim=64, ffn=320, vocab=300)
+    with pytest.raises(W.WpkError) as ei:
+        _graph(odd, max_batch=16, decode=W.WPK_DECODE_MMA)
+    assert ei.value.code == W.WPK_ERR_UNSUPPORTED
+    h = _graph(odd, max_batch=16)  # AUTO falls back to GEMV tiles
+    try:
+        _, names = _ops(h)
+        assert "lm_head" in names
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_llama1b_batched_decode_graph_shape(lib):
+    h = _graph(synth.LLAMA_1B, max_batch=48, max_context=624, n_workers=148)
+    try:
+        st, names = _ops(h)
+        # the LM head's 128-row blocks: 128256 = 1002 x 128
+        assert (names == "b_lm_head").sum() == 1002
+        assert st["weight_bytes"] == 2_471_493_632
+        # one attention tile per (sequence, kv head): 48 x 8 per layer
+        assert (names == "attn").sum() == 16 * 48 * 8
+        for op in ("b_qkv", "b_o", "b_down"):
+            assert (names == op).sum() >= 16 * 128, op  # split along K: about one tile per worker
+    finally:
+        W.wpk_destroy(h)
+
+
+def test_prefill_splits_o_and_down_along_k(lib):
+    # one 128-token block gives only hidden/128 = 16 O and down row blocks:
+    # both are split along K so every worker gets a tile, and each split waits
+    # only for the producers of its K range
+    h = _graph(synth.LLAMA_1B, max_batch=1, max_context=256, n_workers=148)
+    try:
+        W.wpk_select_program(h, 1, 128)
+        st, names = _ops(h)
+        n_o, n_down = (names == "mma_o").sum(), (names == "mma_down").sum()
+        assert n_o >= 16 * 128 and n_down >= 16 * 128, (n_o, n_down)
+        e = W.wpk_get_edges(h)
+        gu = set(np.flatnonzero(names == "mma_gate_up"))
+        for v in np.flatnonzero(names == "mma_down")[:64]:
+            p = set(e[e[:, 1] == v, 0])
+            assert p <= gu and len(p) < 128
     finally:
         W.wpk_destroy(h)

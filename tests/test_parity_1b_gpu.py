@@ -50,11 +50,11 @@ def test_llama1b_b1_per_op_graph(weights, dec):
         eng.close()
 
 
-def test_llama1b_b16_sampled_rows(weights, dec):
-    wl = synth.WORKLOADS["llama1b_decode_b16"]
-    B = 16
+@pytest.mark.parametrize("B,decode", [(16, W.WPK_DECODE_MMA), (16, W.WPK_DECODE_GEMV), (48, W.WPK_DECODE_MMA)])
+def test_llama1b_batched_sampled_rows(weights, dec, B, decode):
+    wl = synth.WORKLOADS[f"llama1b_decode_b{B}"]
     ctx = wl.prompt_len + wl.steps
-    eng = W.Engine(S, weights, B, ctx)
+    eng = W.Engine(S, weights, B, ctx, decode=decode)
     try:
         prompts = synth.make_prompts(S.vocab, B, wl.prompt_len, wl.prompt_seed)
         run_teacher_forced(eng, dec, prompts, steps=3, max_context=ctx, rows=[0, B // 2, B - 1])
