@@ -53,9 +53,10 @@ def parse():
     ap.add_argument("--slot-bytes", type=int, default=0)
     ap.add_argument("--workers-per-sm", type=int, default=0)
     ap.add_argument("--lookahead", type=int, default=0)
-    ap.add_argument("--schedule", default="queue", choices=["queue", "static"])
+    ap.add_argument("--schedule", default="static", choices=["queue", "static"])
     ap.add_argument("--prefill", default="auto", choices=["auto", "mma", "tokenwise"])
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--resident", action="store_true", help="one resident grid serves every decode step")
     return ap.parse_args()
 
 
@@ -183,6 +184,16 @@ def run_reference(args):
 
 
 # -------------------------------------------------------------------- ours --
+def prefill_flops(s, batch, prompt_len):
+    """Algorithmic FLOPs of prefilling `batch` prompts of `prompt_len` tokens:
+    every projection once per token, causal attention (QK^T and PV over the
+    tokens at or before each query), the LM head at the last position."""
+    q, kv = s.n_heads * s.head_dim, s.n_kv_heads * s.head_dim
+    per_token = s.n_layers * (s.hidden * (q + 2 * kv) + q * s.hidden + 3 * s.ffn * s.hidden)
+    attn = s.n_layers * 4 * s.n_heads * s.head_dim * prompt_len * (prompt_len + 1) // 2
+    return 2 * per_token * batch * prompt_len + batch * attn + 2 * s.vocab * s.hidden * batch
+
+
 def algorithmic_bytes_per_step(shape, weight_bytes, batch, ctx_len):
     """Weights once + KV read over ctx_len tokens + KV written for 1 token, per sequence."""
     kv = KV_BYTES_PER_TOKEN(shape)
@@ -226,7 +237,8 @@ def main():
                 workers_per_sm=args.workers_per_sm, lookahead=args.lookahead,
                 schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE,
                 prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
-                         "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill])
+                         "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill],
+                resident=1 if args.resident else 0)
     if args.regions:
         cuts = [int(x) for x in args.regions.split(",")]
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))
@@ -317,14 +329,32 @@ def main():
     # launch over the launch durations measured above
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     kvb = KV_BYTES_PER_TOKEN(s)
-    dec_ctx = [T + i for i in range(decode_steps)]  # tokens already cached at each decode step
-    algo_dec = [algorithmic_bytes_per_step(s, stats["weight_bytes"], B, c) for c in dec_ctx]
-    # the dominant kernel is the decode program (one launch per step): its
-    # algorithmic bytes per launch over the launch times measured above
-    launch_bytes = sum(algo_dec)
-    launch_ms = sum(dec_us) / 1e3 / args.steps
-    achieved_gbs = launch_bytes / (launch_ms / 1e3) / 1e9
-    dec_gbs = statistics.mean(algo_dec) / (statistics.median(dec_us) / 1e6) / 1e9
+    kernel_name = "wpk_persistent_kernel" if mode == W.WPK_MEGAKERNEL else "wpk_per_op_kernel"
+    decode_summary = None
+    if decode_steps > 0:
+        dec_ctx = [T + i for i in range(decode_steps)]  # tokens already cached at each decode step
+        algo_dec = [algorithmic_bytes_per_step(s, stats["weight_bytes"], B, c) for c in dec_ctx]
+        # the dominant kernel is the decode program (one launch per step): its
+        # algorithmic bytes per launch over the launch times measured above
+        launch_bytes = sum(algo_dec)
+        launch_ms = sum(dec_us) / 1e3 / args.steps
+        achieved_gbs = launch_bytes / (launch_ms / 1e3) / 1e9
+        dec_gbs = statistics.mean(algo_dec) / (statistics.median(dec_us) / 1e6) / 1e9
+        decode_summary = {"median": statistics.median(dec_us), "p95": float(np.percentile(dec_us, 95)),
+                          "achieved_gbs": dec_gbs, "frac_of_8tbs": dec_gbs / 8000.0}
+        roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved_gbs / hbm_peak, "traffic": None,
+                    "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel_name}
+    else:
+        # prefill only: the prefill program dominates and is a dense contraction;
+        # algorithmic FLOPs (one bf16 product per weight and token) over its time
+        flops = prefill_flops(s, B, T)
+        achieved_tf = flops / (statistics.median(pre_ms) / 1e3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": achieved_tf / tc_peak, "traffic": None,
+                    "peak_source": f"{peak_kind} cuBLAS bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
+                    "kernel": "wpk_prefill_kernel" if mode == W.WPK_MEGAKERNEL else "wpk_prefill_op_kernel",
+                    "flops_per_launch": flops}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -333,17 +363,14 @@ def main():
         "config": {"workload": wl.name + (f" ({s.n_layers} layers)" if args.layers else ""), "batch": B,
                    "prompt_len": T, "decode_steps": decode_steps, "schedule": args.schedule,
                    "timed": "prefill + decode steps" if with_prefill else "decode steps (prompt prefilled untimed)",
-                   "mode": args.mode, "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
+                   "mode": args.mode + (" (resident grid)" if args.resident else ""),
+                   "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
                    "prefill": "tensor-core prefill program" if prefill_tensor_cores else "token by token",
                    "workers": stats["n_workers"],
                    "l2": "inputs larger than L2: %.2f GB of weights streamed per step" % (stats["weight_bytes"] / 1e9)},
-        "decode_step_us": {"median": statistics.median(dec_us), "p95": float(np.percentile(dec_us, 95)),
-                           "achieved_gbs": dec_gbs, "frac_of_8tbs": dec_gbs / 8000.0},
+        "decode_step_us": decode_summary,
         "ttft_ms": statistics.median(pre_ms) if pre_ms else None,
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm_peak, "traffic": None,
-                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                     "kernel": "wpk_persistent_kernel" if mode == W.WPK_MEGAKERNEL else "wpk_per_op_kernel"},
+        "roofline": roofline,
         "gpu_launches": args.steps * ((launches_per_prefill if with_prefill else 0) + launches_per_decode * decode_steps),
         "clocks": clk.summary(),
     }

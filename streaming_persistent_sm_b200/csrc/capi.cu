@@ -6,7 +6,10 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
+#include <thread>
 #include <cstring>
 #include <memory>
 #include <string>
@@ -61,6 +64,7 @@ struct wpk_handle {
   int32_t* d_block_table = nullptr;
   uint32_t* d_arrive = nullptr;
   uint32_t* d_rb_arrive = nullptr;  // batched decode: split arrivals per O / down row block
+  ResDev* d_res = nullptr;          // resident grid: device copy of the doorbell
   unsigned long long* d_best = nullptr;
   int32_t* d_seqlen = nullptr;
   int32_t* d_tok_fb = nullptr;
@@ -89,6 +93,13 @@ struct wpk_handle {
   size_t smem_prefill = 0;
   // program the inspection calls refer to (nullptr = the decode program)
   PrefillProgram* selected = nullptr;
+  // resident grid: control block in mapped host memory, its own stream
+  ResCtl* res_ctl = nullptr;      // host view
+  ResCtl* res_ctl_dev = nullptr;  // device view
+  cudaStream_t res_stream = nullptr;
+  bool res_live = false;
+  uint32_t res_epoch = 0;         // last step rung on the live grid
+  std::chrono::steady_clock::time_point res_last;
 };
 
 namespace {
@@ -121,6 +132,16 @@ int check_live(wpk_handle* h) {
   }
   if (h->poisoned) return WPK_ERR_POISONED;
   return WPK_OK;
+}
+
+// Tensor-core accumulators: up to 4 of 2N columns each within the 512 TMEM
+// columns of an SM (one worker CTA per SM when a tile uses tensor cores).
+void set_mma_geometry(KParams* P) {
+  const int w = 2 * P->mma_n;
+  P->mma_acc = std::max(1, std::min(4, 512 / w));
+  int cols = 32;
+  while (cols < w * P->mma_acc) cols <<= 1;
+  P->tmem_cols = cols;
 }
 
 KParams make_params(const wpk_handle* h) {
@@ -182,6 +203,7 @@ KParams make_params(const wpk_handle* h) {
   P.evclock = h->d_evclock;
   P.in_tok_stride = 1;
   P.epoch = 1;
+  P.idle_ns = std::max<uint64_t>(200000000ull, 20 * g.plan.wait_timeout_ns);
   P.static_sched = g.plan.schedule == WPK_SCHED_STATIC;
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
@@ -207,6 +229,7 @@ KParams make_params(const wpk_handle* h) {
     P.rb_arrive = h->d_rb_arrive;
     P.lm_mma_off = g.lay.lm_mma;
   }
+  set_mma_geometry(&P);
   return P;
 }
 
@@ -296,7 +319,102 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
   return WPK_OK;
 }
 
+// ------------------------------------------------------------- resident grid
+// Stops a live resident grid (doorbell = shutdown) and waits for it to return.
+int res_shutdown(wpk_handle* h) {
+  if (!h->res_live) return WPK_OK;
+  h->res_ctl->db = kResShutdown;
+  std::atomic_thread_fence(std::memory_order_seq_cst);
+  h->res_live = false;
+  CUDA_TRY(h, cudaStreamSynchronize(h->res_stream));
+  if (h->res_ctl->err && h->h_err_code) *h->h_err_code = h->res_ctl->err;
+  return WPK_OK;
+}
+
+int res_launch(wpk_handle* h) {
+  const CompiledGraph& g = h->g;
+  CUDA_TRY(h, cudaMemsetAsync(h->d_ctr, 0, std::max<size_t>(1, g.ctr_need.size()) * 4, h->res_stream));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_head, 0, 4 * 4, h->res_stream));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_res, 0, sizeof(ResDev), h->res_stream));
+  ResCtl* c = h->res_ctl;
+  c->db = 0;
+  c->ack = 0;
+  c->err = 0;
+  c->t_done_ns = 0;
+  std::atomic_thread_fence(std::memory_order_seq_cst);
+  KParams P = make_params(h);
+  P.resident = 1;
+  P.ctl = h->res_ctl_dev;
+  P.rdev = h->d_res;
+  P.t_begin = 0;
+  P.t_end = (uint32_t)g.tiles.size();
+  P.region = 0;
+  void* args[] = {&P};
+  CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
+                                          h->smem, h->res_stream));
+  h->res_live = true;
+  h->res_epoch = 0;
+  h->res_last = std::chrono::steady_clock::now();
+  return WPK_OK;
+}
+
+// One step on the resident grid: the step's inputs must be complete on stream
+// `s`; returns once the grid has acknowledged the step.
+int res_step(wpk_handle* h, const int32_t* in_tok, int stride, int32_t* out_tok, float* logits, cudaStream_t s) {
+  const uint64_t idle_ns = std::max<uint64_t>(200000000ull, 20 * h->g.plan.wait_timeout_ns);
+  const auto now = std::chrono::steady_clock::now();
+  // never ring a grid that may be about to leave on its idle limit, and start
+  // a fresh grid before 32-bit tickets could wrap
+  const uint32_t max_steps = (uint32_t)((1u << 31) / std::max<size_t>(1, h->g.tiles.size()));
+  if (h->res_live && (cudaStreamQuery(h->res_stream) != cudaErrorNotReady || h->res_epoch >= max_steps ||
+                      (uint64_t)std::chrono::duration_cast<std::chrono::nanoseconds>(now - h->res_last).count() >
+                          idle_ns / 2)) {
+    int rc = res_shutdown(h);
+    if (rc) return rc;
+  }
+  cudaGetLastError();
+  CUDA_TRY(h, cudaStreamSynchronize(s));  // the step's inputs
+  if (!h->res_live) {
+    int rc = res_launch(h);
+    if (rc) return rc;
+  }
+  ResCtl* c = h->res_ctl;
+  c->in_tok = (uint64_t)(uintptr_t)in_tok;
+  c->in_stride = stride;
+  c->out_tok = (uint64_t)(uintptr_t)out_tok;
+  c->logits = (uint64_t)(uintptr_t)logits;
+  std::atomic_thread_fence(std::memory_order_seq_cst);
+  const uint32_t e = ++h->res_epoch;
+  c->db = e;
+  const auto t0 = std::chrono::steady_clock::now();
+  const uint64_t limit = 2 * h->g.plan.wait_timeout_ns + 1000000000ull;
+  for (uint64_t it = 0; c->ack < e; ++it) {
+    if (c->err) {
+      *h->h_err_code = c->err;
+      h->poisoned = true;
+      res_shutdown(h);
+      return fail(h, WPK_ERR_POISONED, "device program reported an error (see wpk_get_error_info)");
+    }
+    if ((it & 1023) == 1023) {
+      const uint64_t el =
+          std::chrono::duration_cast<std::chrono::nanoseconds>(std::chrono::steady_clock::now() - t0).count();
+      if (el > limit || cudaStreamQuery(h->res_stream) != cudaErrorNotReady) {
+        if (c->ack >= e) break;
+        h->poisoned = true;
+        res_shutdown(h);
+        return fail(h, WPK_ERR_TIMEOUT, "resident grid did not acknowledge the step");
+      }
+      std::this_thread::yield();
+    }
+  }
+  std::atomic_thread_fence(std::memory_order_seq_cst);
+  h->res_last = std::chrono::steady_clock::now();
+  h->ctx += 1;
+  return WPK_OK;
+}
+
 int step_impl(wpk_handle* h, const int32_t* in_tok, int stride, int32_t* out_tok, float* logits, cudaStream_t s) {
+  if (h->g.plan.resident) return res_step(h, in_tok, stride, out_tok, logits, s);
   if (h->g.plan.mode == WPK_MEGAKERNEL) {
     KParams P = make_params(h);
     P.in_tok = in_tok;
@@ -376,6 +494,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.act_bytes = g.plan.act_bytes;
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
+  set_mma_geometry(&P);
   P.M = g.M;
   P.T = g.T;
   P.n_tb = g.n_tb;
@@ -486,6 +605,25 @@ static int setup_device(wpk_handle* h) {
   }
   int per_sm = 0;
   CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kCtaThreads, smem_max));
+  {
+    // tcgen05.alloc waits until the SM has free TMEM columns: workers that
+    // share an SM must fit its 512 columns together
+    KParams probe{};
+    probe.mma_n = p.decode_mode == WPK_DECODE_MMA ? p.dec_n : kTokBlock;
+    set_mma_geometry(&probe);
+    if (p.decode_mode == WPK_DECODE_MMA && per_sm * probe.tmem_cols > 512)
+      return fail(h, WPK_ERR_UNSUPPORTED, "co-resident decode workers would not fit the SM's tensor memory");
+    if (h->smem_prefill) {
+      KParams pp{};
+      pp.mma_n = kTokBlock;
+      set_mma_geometry(&pp);
+      int per_sm_p = 0;
+      CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreads,
+                                                                h->smem_prefill));
+      if (per_sm_p * pp.tmem_cols > 512)
+        return fail(h, WPK_ERR_UNSUPPORTED, "co-resident prefill workers would not fit the SM's tensor memory");
+    }
+  }
   h->n_workers = p.n_workers ? p.n_workers : h->n_sms * p.workers_per_sm;
   if (per_sm < 1 || h->n_workers > per_sm * h->n_sms)
     return fail(h, WPK_ERR_UNSUPPORTED, "the worker grid cannot be co-resident with this slot size");
@@ -502,7 +640,8 @@ static int setup_device(wpk_handle* h) {
                o_rope = take((size_t)p.max_context * hd2 * sizeof(float2)),
                o_bt = take(B * g.max_blocks * 4), o_arr = take(B * model->n_kv_heads * 4), o_best = take(B * 8),
                o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4),
-               o_rb = take((size_t)model->n_layers * 2 * (model->hidden / 128 + 1) * 4);
+               o_rb = take((size_t)model->n_layers * 2 * (model->hidden / 128 + 1) * 4),
+               o_res = take(sizeof(ResDev));
   CUDA_TRY(h, cudaMalloc(&h->d_base, off));
   CUDA_TRY(h, cudaMemset(h->d_base, 0, off));
   h->d_tiles = reinterpret_cast<Tile*>(h->d_base + o_tiles);
@@ -521,6 +660,7 @@ static int setup_device(wpk_handle* h) {
   h->d_tok_fb = reinterpret_cast<int32_t*>(h->d_base + o_fb);
   h->d_active = reinterpret_cast<int32_t*>(h->d_base + o_act);
   h->d_rb_arrive = reinterpret_cast<uint32_t*>(h->d_base + o_rb);
+  h->d_res = reinterpret_cast<ResDev*>(h->d_base + o_res);
   CUDA_TRY(h, cudaMemcpy(h->d_tiles, g.tiles.data(), n_tiles * sizeof(Tile), cudaMemcpyHostToDevice));
   if (!g.sig.empty()) CUDA_TRY(h, cudaMemcpy(h->d_sig, g.sig.data(), g.sig.size() * 4, cudaMemcpyHostToDevice));
   CUDA_TRY(h, cudaMemcpy(h->d_layers, g.lay.layers.data(), g.lay.layers.size() * sizeof(LayerDev),
@@ -539,6 +679,12 @@ static int setup_device(wpk_handle* h) {
   CUDA_TRY(h, cudaMemcpy(h->d_block_table, bt.data(), bt.size() * 4, cudaMemcpyHostToDevice));
   CUDA_TRY(h, cudaHostAlloc(&h->h_err_code, 4, cudaHostAllocDefault));
   *h->h_err_code = 0;
+  if (p.resident) {
+    CUDA_TRY(h, cudaHostAlloc(&h->res_ctl, sizeof(ResCtl), cudaHostAllocMapped));
+    memset((void*)h->res_ctl, 0, sizeof(ResCtl));
+    CUDA_TRY(h, cudaHostGetDevicePointer((void**)&h->res_ctl_dev, (void*)h->res_ctl, 0));
+    CUDA_TRY(h, cudaStreamCreateWithFlags(&h->res_stream, cudaStreamNonBlocking));
+  }
   h->has_device = true;
   return WPK_OK;
 }
@@ -598,6 +744,8 @@ int wpk_load_weights(wpk_handle* h, const wpk_weights* w, void* dev_weights, voi
                      void* stream) {
   int rc = check_live(h);
   if (rc) return rc;
+  rc = res_shutdown(h);
+  if (rc) return rc;
   if (!w || !dev_weights || !dev_kv || !dev_scratch)
     return fail(h, WPK_ERR_INVALID_ARG, "null weights or device buffer");
   if (((uintptr_t)dev_weights | (uintptr_t)dev_kv | (uintptr_t)dev_scratch) & 255)
@@ -635,6 +783,8 @@ int wpk_set_block_table(wpk_handle* h, const int32_t* table) {
 int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len, int32_t* first_tok_dev,
                 float* logits_dev, void* stream) {
   int rc = check_live(h);
+  if (rc) return rc;
+  rc = res_shutdown(h);
   if (rc) return rc;
   if (!h->loaded) return fail(h, WPK_ERR_NOT_LOADED, "weights not loaded");
   if (!tokens_dev || batch <= 0 || prompt_len <= 0) return fail(h, WPK_ERR_INVALID_ARG, "bad prefill arguments");
@@ -773,6 +923,8 @@ int wpk_simulate(const wpk_handle* h, int n_threads, int n_epochs, uint64_t seed
 int wpk_get_trace(wpk_handle* h, void* host_buf, size_t bytes) {
   if (!h || !host_buf) return WPK_ERR_INVALID_ARG;
   if (!h->has_device) return fail(h, WPK_ERR_CUDA, "no CUDA device");
+  int rc = res_shutdown(h);
+  if (rc) return rc;
   const CompiledGraph& g = selected_graph(h);
   const size_t need = g.tiles.size() * sizeof(TraceRec);
   if (bytes < need) return fail(h, WPK_ERR_INVALID_ARG, "trace buffer too small");
@@ -785,6 +937,8 @@ int wpk_get_trace(wpk_handle* h, void* host_buf, size_t bytes) {
 int wpk_get_error_info(wpk_handle* h, wpk_error_info* info) {
   if (!h || !info) return WPK_ERR_INVALID_ARG;
   if (!h->has_device) return fail(h, WPK_ERR_CUDA, "no CUDA device");
+  int rc = res_shutdown(h);
+  if (rc) return rc;
   CUDA_TRY(h, cudaDeviceSynchronize());
   ErrWord e{};
   CUDA_TRY(h, cudaMemcpy(&e, h->d_err, sizeof e, cudaMemcpyDeviceToHost));
@@ -802,7 +956,12 @@ const char* wpk_last_error(const wpk_handle* h) { return h ? h->err.c_str() : g_
 
 int wpk_destroy(wpk_handle* h) {
   if (!h) return WPK_ERR_INVALID_ARG;
-  if (h->has_device) cudaDeviceSynchronize();
+  if (h->has_device) {
+    res_shutdown(h);
+    cudaDeviceSynchronize();
+  }
+  if (h->res_stream) cudaStreamDestroy(h->res_stream);
+  if (h->res_ctl) cudaFreeHost((void*)h->res_ctl);
   for (auto& e : h->graphs) {
     if (e.exec) cudaGraphExecDestroy(e.exec);
     if (e.graph) cudaGraphDestroy(e.graph);
@@ -831,6 +990,9 @@ int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes
   if (rc) return rc;
   if (h->g.plan.mode != WPK_MEGAKERNEL)
     return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the megakernel mode");
+  if (h->g.plan.resident)
+    return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs a launch per step (the resident grid keeps its "
+                                        "scratch pointer for its lifetime)");
   if (h->g.plan.decode_mode == WPK_DECODE_MMA)
     return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the GEMV decode program (the tensor-core "
                                         "decode program keeps sums in its scratch between steps)");
@@ -852,6 +1014,7 @@ int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes
 
 int wpk_debug_break_counter(wpk_handle* h, int counter) {
   if (!h || counter < 0 || counter >= (int)h->g.ctr_need.size()) return WPK_ERR_INVALID_ARG;
+  if (h->has_device && res_shutdown(h)) return WPK_ERR_CUDA;
   for (auto& t : h->g.tiles)
     if (t.wait_ctr == (uint32_t)counter) t.need += 1;
   if (!h->has_device) return WPK_OK;

@@ -69,6 +69,10 @@ __device__ __forceinline__ int32_t ld_volatile_s32(const int32_t* p) {
   return v;
 }
 
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void red_release_add_u32(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -127,6 +131,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Adds 16 consecutive 32-bit columns at two TMEM addresses of the thread's lane
+// into v (both loads in flight before one wait).
+__device__ __forceinline__ void tmem_add16x2(uint32_t ta, uint32_t tb, float* v) {
+  uint32_t a[16], b[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+        "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15])
+      : "r"(ta)
+      : "memory");
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+        "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(tb)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes (64 16-bit elements), 8-row groups 1024 bytes apart.  The tile
 // base must be 1024-byte aligned; a K-step of 16 elements inside the 128-byte
@@ -148,14 +173,14 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// Byte offset of element (row, col) inside a [rows][64] 16-bit tile stored
-// with the 128-byte swizzle: the 16-byte unit index is XORed with row % 8.
 // Relaxed add of four floats to a 16-byte aligned global address (one vector
 // reduction instead of four scalar ones).
 __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
+// Byte offset of element (row, col) inside a [rows][64] 16-bit tile stored
+// with the 128-byte swizzle: the 16-byte unit index is XORed with row % 8.
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
   const uint32_t unit = (col >> 3) ^ (row & 7u);
   return row * 128u + unit * 16u + (col & 7u) * 2u;

@@ -44,6 +44,14 @@ constexpr int kSigQueue = 8;                               // finished tiles awa
 constexpr uint32_t kSigStop = 0xFFFFFFFFu;
 constexpr int kNoAct = -1;
 
+// the current step's I/O pointers (from the launch, or per step from the
+// resident control block), set by compute thread 0 before each tile
+__shared__ const int32_t* s_in_tok;
+__shared__ int s_in_stride;
+__shared__ int32_t* s_out_tok;
+__shared__ float* s_logits;
+__shared__ uint32_t s_io_epoch;
+
 struct TQEntry {  // producer -> consumers, one per tile held by the worker
   Tile tile;
   uint32_t ticket;
@@ -51,6 +59,7 @@ struct TQEntry {  // producer -> consumers, one per tile held by the worker
   int32_t n_chunks;
   int32_t rows_per_chunk;
   uint32_t ev_issue;  // event clock when its first copy was issued (trace)
+  uint32_t epoch;     // step the tile belongs to (counter targets are need x epoch)
   uint64_t t_claim, t_issued;  // trace timestamps
 };
 
@@ -148,6 +157,10 @@ __device__ void record_error(const KParams& P, int code, uint32_t tile, uint32_t
     P.err->observed = obs;
     P.err->target = target;
     __threadfence();
+    if (P.resident) {
+      P.ctl->err = code;
+      __threadfence_system();
+    }
   }
 }
 
@@ -159,11 +172,14 @@ __device__ bool wait_phase(const KParams& P, uint64_t* bar, uint32_t parity, vol
                            uint32_t slack = 1) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
+  // waits that only idle behind other warps (slack > 1) also idle while a
+  // resident grid waits for its next step
+  const uint64_t bound = (P.resident && slack > 1) ? max(P.timeout_ns * slack, 2 * P.idle_ns) : P.timeout_ns * slack;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > P.timeout_ns * slack) {
+      if (globaltimer() - t0 > bound) {
         record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, 0, 0);
         *abort = 1;
         return false;
@@ -421,10 +437,10 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
       break;
     }
     case OP_LMHEAD: {
-      if (P.logits)
+      if (s_logits)
         for (int idx = threadIdx.x; idx < R * bg; idx += kThreads) {
           const int rr = idx % R, b = idx / R, bi = b0 + b;
-          P.logits[(size_t)bi * P.vocab + r0 + rr] = out[rr * S + b];
+          s_logits[(size_t)bi * P.vocab + r0 + rr] = out[rr * S + b];
         }
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
       if (warp < bg) {
@@ -454,7 +470,56 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
   }
 }
 
-__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, volatile int* abort);
+__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, uint32_t epoch, volatile int* abort);
+
+// Resident grid: bounded wait until the host has rung the doorbell for step
+// `epoch`.  False ends the worker: shutdown, an error elsewhere, or no step for
+// idle_ns (an idle grid exits; the host launches a new one for the next step).
+// Worker 0 polls the mapped control block and publishes each step (its I/O
+// pointers, then the step number with release semantics) in device memory;
+// the other workers poll that copy.  `seen` caches the last step observed.
+__device__ bool wait_doorbell(const KParams& P, uint32_t epoch, volatile int* abort, uint32_t* seen) {
+  if (epoch <= *seen) return true;
+  const uint64_t t0 = globaltimer();
+  if (blockIdx.x == 0) {
+    // worker 0 publishes every step it sees, also steps it holds no ticket of
+    for (;;) {
+      const uint32_t db = P.ctl->db;
+      const bool quit = db == kResShutdown || *abort || ld_volatile_s32(&P.err->code) != 0 ||
+                        globaltimer() - t0 > P.idle_ns;
+      if (quit) {
+        __threadfence();
+        st_release_u32(&P.rdev->db, kResShutdown);
+        return false;
+      }
+      if (db > *seen) {
+        __threadfence_system();  // the host wrote the pointers before the step number
+        P.rdev->in_tok = P.ctl->in_tok;
+        P.rdev->in_stride = P.ctl->in_stride;
+        P.rdev->out_tok = P.ctl->out_tok;
+        P.rdev->logits = P.ctl->logits;
+        __threadfence();
+        st_release_u32(&P.rdev->db, db);
+        *seen = db;
+      }
+      if (db >= epoch) return true;
+      __nanosleep(256);
+    }
+  }
+  for (uint32_t it = 1;; ++it) {
+    const uint32_t db = ld_acquire_u32(&P.rdev->db);
+    if (db == kResShutdown) return false;
+    if (db >= epoch) {
+      *seen = db;
+      return true;
+    }
+    if ((it & 15) == 0) {
+      if (*abort || ld_volatile_s32(&P.err->code) != 0) return false;
+      if (globaltimer() - t0 > 2 * P.idle_ns + P.timeout_ns) return false;
+    }
+    __nanosleep(128);
+  }
+}
 
 // Consumer-side chunk cursor: chunk c lives in stage c % n_stages and is the
 // (c / n_stages)-th use of that stage.
@@ -464,8 +529,10 @@ struct Cursor {
 
 struct ConsumerState {
   int act_key;      // (op, layer, k0) of the staged activation, or kNoAct
-  uint32_t last_ctr;  // counter known satisfied in this launch
+  uint32_t last_ctr;    // counter known satisfied in this launch ...
+  uint32_t last_epoch;  // ... for this step
   uint32_t acc_phase;  // parity of the accumulator barrier
+  uint32_t act_epoch;  // step the staged activation belongs to
 };
 
 __shared__ uint32_t s_tmem;  // TMEM base address (tensor-core programs)
@@ -660,7 +727,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   const int nq = grp * hd;  // (head, dim) pairs: thread i owns pairs i and i + 256
   float* part = P.part + ((((size_t)s.b * P.n_kv + s.g) * P.n_splits + s.j) * grp) * (2 + hd);
   float* q_s = Sh.act;                    // [grp][hd]
-  float* p_s = Sh.act + kMaxGroup * hd;   // [grp][page]
+  float* p_s = Sh.act + kMaxGroup * hd;   // [grp][kAttnPages * page]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float scale = 1.0f / sqrtf((float)hd);
   float o[2] = {0.f, 0.f};
@@ -669,20 +736,27 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
     s_l[threadIdx.x] = 0.f;
   }
   cbar();
-  for (int k = 0; k < n_chunks; ++k) {
-    const uint32_t c = cur.c;
-    const int st = c % P.n_stages;
-    const bool ok = wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu);
+  // up to G pages (one ring stage each) are computed per round
+  const int G = min(kAttnPages, P.n_stages);
+  const int span = G * page;
+  auto stage_of = [&](int j) { return Sh.ring + (size_t)((cur.c + j) % P.n_stages) * P.stage_bytes; };
+  for (int k0 = 0; k0 < n_chunks; k0 += G) {
+    const int gn = min(G, n_chunks - k0);
+    bool ok = true;
+    for (int j = 0; j < gn && ok; ++j) {
+      const uint32_t c = cur.c + j;
+      ok = wait_phase(P, &Sh.full[c % P.n_stages], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu);
+    }
     if (!cbar_and(ok)) return false;
-    if (P.trace && threadIdx.x == 0 && k + 1 == n_chunks) s_t_data = globaltimer();
-    uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
-    uint16_t* Ks = reinterpret_cast<uint16_t*>(stage);
-    uint16_t* Vs = reinterpret_cast<uint16_t*>(stage + (size_t)page * hd * 2);
-    const int p0 = (s.t0 / page + k) * page;  // first token of the staged page
-    const int n = min(page, s.t1 - p0);
+    if (P.trace && threadIdx.x == 0 && k0 + gn == n_chunks) s_t_data = globaltimer();
+    const int p0 = (s.t0 / page + k0) * page;  // first token of the round
+    const int n = min(gn * page, s.t1 - p0);   // tokens of the round
     // the current token's row was written this step, after the copy was issued
     if (s.pos >= p0 && s.pos < p0 + n) {
-      const int row = s.pos - p0;
+      uint8_t* stage = stage_of((s.pos - p0) / page);
+      uint16_t* Ks = reinterpret_cast<uint16_t*>(stage);
+      uint16_t* Vs = reinterpret_cast<uint16_t*>(stage + (size_t)page * hd * 2);
+      const int row = (s.pos - p0) % page;
       const int blk = P.block_table[s.b * P.max_blocks + s.pos / page];
       if (P.dec_mma) {
         for (int i = threadIdx.x; i < 2 * hd; i += kThreads) {
@@ -704,35 +778,68 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
         }
       }
     }
-    if (k == 0)
+    if (k0 == 0)
       for (int i = threadIdx.x; i < nq; i += kThreads)
         q_s[i] = P.dec_mma ? __ldcg(P.acc + (size_t)(s.g * nq + i) * P.mma_n + s.b)
                            : __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * nq + i);
     cbar();
-    const int words = hd / 2;
-    for (int idx = threadIdx.x; idx < grp * n; idx += kThreads) {
-      const int hh = idx / n, t = idx % n;
-      const uint32_t* kr = reinterpret_cast<const uint32_t*>(Ks + (size_t)t * hd);
-      const float* qr = q_s + hh * hd;
-      float acc = 0.f;
-      for (int w = 0; w < words; ++w) {
-        const int ww = (w + t) & (words - 1);
-        const uint32_t kk = kr[ww];
-        acc = fmaf(qr[2 * ww], __uint_as_float(kk << 16), acc);
-        acc = fmaf(qr[2 * ww + 1], __uint_as_float(kk & 0xFFFF0000u), acc);
+    // scores.  Few tokens: one (head, token) pair per thread.  Otherwise one
+    // token per thread against every head of the group (one read of the K
+    // row).  Either way the row's units are visited in a rotated order so that
+    // neighbouring threads hit different banks.
+    if (grp * n <= kThreads) {
+      if (threadIdx.x < grp * n) {
+        const int hh = threadIdx.x / n, tt = threadIdx.x % n, t = tt % page;
+        const uint4* kr = reinterpret_cast<const uint4*>(stage_of(tt / page) + (size_t)t * hd * 2);
+        const float* qr = q_s + hh * kHeadDim;
+        float acc = 0.f;
+#pragma unroll
+        for (int u = 0; u < kHeadDim / 8; ++u) {
+          const int uu = (u + t) & (kHeadDim / 8 - 1);
+          float kf[8];
+          unpack8(kr[uu], kf);
+          const float4 qa = *reinterpret_cast<const float4*>(qr + 8 * uu);
+          const float4 qb = *reinterpret_cast<const float4*>(qr + 8 * uu + 4);
+          acc = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], acc))));
+          acc = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], acc))));
+        }
+        p_s[hh * span + tt] = acc * scale;
       }
-      p_s[hh * page + t] = acc * scale;
+    } else
+    for (int tt = threadIdx.x; tt < n; tt += kThreads) {
+      const int t = tt % page;
+      const uint4* kr = reinterpret_cast<const uint4*>(stage_of(tt / page) + (size_t)t * hd * 2);
+      float acc[kMaxGroup];
+#pragma unroll
+      for (int hh = 0; hh < kMaxGroup; ++hh) acc[hh] = 0.f;
+#pragma unroll
+      for (int u = 0; u < kHeadDim / 8; ++u) {
+        const int uu = (u + t) & (kHeadDim / 8 - 1);
+        float kf[8];
+        unpack8(kr[uu], kf);
+#pragma unroll
+        for (int hh = 0; hh < kMaxGroup; ++hh) {
+          if (hh >= grp) break;
+          const float4 qa = *reinterpret_cast<const float4*>(q_s + hh * kHeadDim + 8 * uu);
+          const float4 qb = *reinterpret_cast<const float4*>(q_s + hh * kHeadDim + 8 * uu + 4);
+          acc[hh] = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], acc[hh]))));
+          acc[hh] = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], acc[hh]))));
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < kMaxGroup; ++hh)
+        if (hh < grp) p_s[hh * span + tt] = acc[hh] * scale;
     }
     cbar();
     if (warp < grp) {  // running max and sum of head `warp`
       float mx = -INFINITY;
-      for (int t = lane; t < n; t += 32) mx = fmaxf(mx, p_s[warp * page + t]);
+      for (int tt = lane; tt < n; tt += 32) mx = fmaxf(mx, p_s[warp * span + tt]);
       mx = warp_max(mx);
       const float m_old = s_m[warp], m_new = fmaxf(m_old, mx);
       float l = 0.f;
-      for (int t = lane; t < n; t += 32) {
-        const float e = expf(p_s[warp * page + t] - m_new);
-        p_s[warp * page + t] = e;
+      for (int tt = lane; tt < n; tt += 32) {
+        const float e = expf(p_s[warp * span + tt] - m_new);
+        p_s[warp * span + tt] = e;
         l += e;
       }
       l = warp_sum(l);
@@ -750,13 +857,19 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
       if (i < nq) {
         const int hh = i / hd, d = i % hd;
         float a = 0.f;
-        for (int t = 0; t < n; ++t) a = fmaf(p_s[hh * page + t], bf2f(Vs[(size_t)t * hd + d]), a);
+        for (int j = 0; j < gn; ++j) {
+          const int tn = min(page, n - j * page);
+          const uint16_t* Vs = reinterpret_cast<const uint16_t*>(stage_of(j) + (size_t)page * hd * 2);
+          const float* pr = p_s + hh * span + j * page;
+          for (int t = 0; t < tn; ++t) a = fmaf(pr[t], bf2f(Vs[(size_t)t * hd + d]), a);
+        }
         o[r] = o[r] * s_sc[hh] + a;
       }
     }
     cbar();
-    if (threadIdx.x == 0) mbar_arrive(&Sh.empty[st]);
-    ++cur.c;
+    if (threadIdx.x == 0)
+      for (int j = 0; j < gn; ++j) mbar_arrive(&Sh.empty[(cur.c + j) % P.n_stages]);
+    cur.c += gn;
   }
   if (P.n_splits == 1) {  // the only split: the result directly
 #pragma unroll
@@ -1005,7 +1118,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       for (int i = 0; i < 16; ++i) {
         const int n = n0 + i;
         const float val = v[i] * s_rn[n];
-        if (P.logits && valid && n < nb) P.logits[(size_t)n * P.vocab + f] = val;
+        if (s_logits && valid && n < nb) s_logits[(size_t)n * P.vocab + f] = val;
         unsigned long long key = valid ? argmax_key(val, f) : 0ull;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -1147,12 +1260,15 @@ __device__ void rowblock_done(const KParams& P, const Tile& T) {
 __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
                          ConsumerState& cs, volatile int* abort, uint32_t tile) {
   const uint32_t tmem = s_tmem;
-  const int N = P.mma_n;
+  const int N = P.mma_n, NA = P.mma_acc;
   if (threadIdx.x == 0) {
+    // The hi and lo activation rows sit back to back in the stage, so one MMA
+    // with N' = 2N covers both: columns [0, N) get W . hi, [N, 2N) W . lo.
+    // Successive K-steps rotate over NA accumulators (2N columns each), so the
+    // MMAs of a chunk do not wait on one another.
     bool ok = true;
     uint32_t cc = cur.c;
-    const uint32_t idesc = idesc_f16(128, N, true);
-    const uint32_t a_off = (uint32_t)P.act_chunk;
+    const uint32_t idesc = idesc_f16(128, 2 * N, true);
     for (int k = 0; k < n_chunks; ++k, ++cc) {
       const int st = cc % P.n_stages;
       if (!wait_phase(P, &S.full[st], (cc / P.n_stages) & 1u, abort, tile)) {
@@ -1163,9 +1279,9 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
       const uint32_t base = smem_u32(S.ring + (size_t)st * P.stage_bytes);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = sdesc_k_sw128(base + kk * 32);
-        umma_f16(tmem, ad, sdesc_k_sw128(base + kMmaChunkBytes + kk * 32), idesc, (k | kk) != 0);
-        umma_f16(tmem, ad, sdesc_k_sw128(base + kMmaChunkBytes + a_off + kk * 32), idesc, 1);
+        const int a = kk % NA;
+        umma_f16(tmem + (uint32_t)(a * 2 * N), sdesc_k_sw128(base + kk * 32),
+                 sdesc_k_sw128(base + kMmaChunkBytes + kk * 32), idesc, (k > 0 || kk >= NA) ? 1u : 0u);
       }
       umma_commit(&S.empty[st]);
     }
@@ -1192,7 +1308,11 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
   const int fl = 32 * q + lane;
   for (int cg = half; cg < N / 16; cg += 2) {  // 16-column groups alternate between the two warp halves
     float v[16];
-    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(16 * cg), v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(16 * cg);
+    for (int a = 0; a < NA; ++a)  // hi and lo parts of every accumulator
+      tmem_add16x2(lane_base + (uint32_t)(a * 2 * N), lane_base + (uint32_t)(a * 2 * N + N), v);
     mma_epilogue(P, T, fl, 16 * cg, v);
   }
   tc_fence_before();
@@ -1314,7 +1434,7 @@ __device__ bool body_embed(const KParams& P) {
   const int nb = active_batch(P);
   const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
   for (int b = 0; b < nb; ++b) {
-    int tok = P.in_tok ? P.in_tok[(size_t)b * P.in_tok_stride] : P.tok_fb[b];
+    int tok = s_in_tok ? s_in_tok[(size_t)b * s_in_stride] : P.tok_fb[b];
     if (tok < 0 || tok >= P.vocab) {
       if (threadIdx.x == 0) record_error(P, WPK_ERR_INVALID_ARG, 0, kNoCounter, (uint32_t)tok, (uint32_t)P.vocab);
       tok = 0;
@@ -1340,7 +1460,7 @@ __device__ bool body_embed_mma(const KParams& P, const Tile& T) {
   if (threadIdx.x < N) {
     int tok = 0;
     if (threadIdx.x < nb) {
-      tok = P.in_tok ? P.in_tok[(size_t)threadIdx.x * P.in_tok_stride] : P.tok_fb[threadIdx.x];
+      tok = s_in_tok ? s_in_tok[(size_t)threadIdx.x * s_in_stride] : P.tok_fb[threadIdx.x];
       if (tok < 0 || tok >= P.vocab) {
         record_error(P, WPK_ERR_INVALID_ARG, 0, kNoCounter, (uint32_t)tok, (uint32_t)P.vocab);
         tok = 0;
@@ -1381,26 +1501,35 @@ __device__ bool body_embed_mma(const KParams& P, const Tile& T) {
   return true;
 }
 
-__device__ bool body_final(const KParams& P) {
+__device__ bool body_final(const KParams& P, uint32_t epoch) {
   const int nb = active_batch(P);
   if (P.dec_mma)  // the x^2 sums start from zero next step
     for (int i = threadIdx.x; i < (2 * P.n_layers + 1) * P.mma_n; i += kThreads) P.ss[i] = 0.f;
   for (int b = threadIdx.x; b < nb; b += kThreads) {
     const unsigned long long key = P.best[b];
     const int32_t idx = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
-    if (P.out_tok) P.out_tok[b] = idx;
+    if (s_out_tok) s_out_tok[b] = idx;
     P.tok_fb[b] = idx;
     P.best[b] = 0ull;
     P.seqlen[b] += 1;
+  }
+  if (P.resident) {  // the step is complete: tell the host
+    cbar();
+    if (threadIdx.x == 0) {
+      __threadfence_system();
+      P.ctl->t_done_ns = globaltimer();
+      __threadfence_system();
+      P.ctl->ack = epoch;
+    }
   }
   return true;
 }
 
 // Thread 0 of the consumers: bounded acquire-wait until the tile's counter
 // reaches need x epoch.
-__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, volatile int* abort) {
+__device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, uint32_t epoch, volatile int* abort) {
   if (T.wait_ctr == kNoCounter) return true;
-  const uint32_t target = T.need * P.epoch;
+  const uint32_t target = T.need * epoch;
   const uint32_t* ctr = P.ctr + T.wait_ctr;
   uint32_t v = ld_acquire_u32(ctr);
   if ((int32_t)(v - target) >= 0) return true;
@@ -1448,12 +1577,13 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
     }
     fence_mbar_init();
     for (int i = 0; i < kMaxStages; ++i) s_seen[i] = 0;
+    s_io_epoch = 0;
     s_abort = 0;
     s_prod_chunks = 0;
     s_cons_chunks = 0;
   }
   if (P.uses_tmem && warp == 0) {
-    tmem_alloc(&s_tmem, kTokBlock);
+    tmem_alloc(&s_tmem, (uint32_t)P.tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1479,6 +1609,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
     // ------------------------------------------------------------ producer
     if ((threadIdx.x & 31) == 0) {
       uint32_t c = 0;  // chunks issued
+      uint32_t db_seen = 0;  // resident: last step the doorbell showed
       const int Q = P.per_op ? 1 : P.lookahead;
       for (uint32_t i = 0;; ++i) {
         const int slot = i % Q;
@@ -1493,13 +1624,27 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           t = P.t_begin + atomicAdd(&P.head[P.region], 1u);
         const uint64_t t_claim = P.trace ? globaltimer() : 0;
         TQEntry& e = S.tq[slot];
-        if (t >= P.t_end) {
+        uint32_t epoch = P.epoch;
+        if (P.resident) {
+          // tickets run on across steps; nothing of a step is copied before
+          // the host has asked for it (the previous step is then complete)
+          const uint32_t n_tiles = P.t_end - P.t_begin;
+          epoch = t / n_tiles + 1;
+          t = P.t_begin + t % n_tiles;
+          if (!wait_doorbell(P, epoch, &s_abort, &db_seen)) {
+            e.valid = 0;
+            mbar_arrive(&S.tq_full[slot]);
+            break;
+          }
+          fence_proxy_async_global();
+        } else if (t >= P.t_end) {
           e.valid = 0;
           mbar_arrive(&S.tq_full[slot]);
           break;
         }
         e.tile = P.tiles[t];
         e.ticket = t;
+        e.epoch = epoch;
         e.valid = 1;
         int nch, rpc;
         tile_chunks(P, e.tile, &nch, &rpc);
@@ -1529,7 +1674,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
             issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
           }
           // (per-op launches get their order from the stream; no counters run)
-          if (!stop && !P.per_op && !wait_counter(P, T, t, &s_abort)) stop = true;
+          if (!stop && !P.per_op && !wait_counter(P, T, t, e.epoch, &s_abort)) stop = true;
           if (!stop) {
             fence_proxy_async_global();
             for (int k = 0; k < pre; ++k) issue_mma_act(P, T, k, stage_ptr(c0 + k), &S.full[(c0 + k) % P.n_stages]);
@@ -1541,7 +1686,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           }
         } else {
           if (T.op == OP_PATTN) {  // its KV pages are written inside this program
-            if (!P.per_op && !wait_counter(P, T, t, &s_abort)) stop = true;
+            if (!P.per_op && !wait_counter(P, T, t, e.epoch, &s_abort)) stop = true;
             else fence_proxy_async_global();
           }
           for (int k = 0; k < nch && !stop; ++k, ++c) {
@@ -1559,7 +1704,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
   } else {
     // ----------------------------------------------------------- consumers
     Cursor cur{0};
-    ConsumerState cs{kNoAct, kNoCounter, 0u};
+    ConsumerState cs{kNoAct, kNoCounter, 0u, 0u, 0u};
     uint32_t n_sig = 0;  // requests pushed to the signaller (thread 0)
     const int Q = P.per_op ? 1 : P.lookahead;
     __shared__ int s_fail;
@@ -1571,14 +1716,35 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       const Tile T = e.tile;
       const uint32_t t = e.ticket;
       const int n_chunks = e.n_chunks, rpc = e.rows_per_chunk;
+      if (e.epoch != cs.act_epoch) {  // a staged activation never outlives its step
+        cs.act_key = kNoAct;
+        cs.act_epoch = e.epoch;
+      }
       uint32_t ev_start = 0;
       uint64_t t_start = 0;
       if (threadIdx.x == 0) {
         s_t_data = 0;
+        if (e.epoch != s_io_epoch) {  // this step's I/O pointers
+          if (P.resident) {  // published by worker 0 before the step number
+            s_in_tok = reinterpret_cast<const int32_t*>(__ldcg(&P.rdev->in_tok));
+            s_in_stride = __ldcg(&P.rdev->in_stride);
+            s_out_tok = reinterpret_cast<int32_t*>(__ldcg(&P.rdev->out_tok));
+            s_logits = reinterpret_cast<float*>(__ldcg(&P.rdev->logits));
+          } else {
+            s_in_tok = P.in_tok;
+            s_in_stride = P.in_tok_stride;
+            s_out_tok = P.out_tok;
+            s_logits = P.logits;
+          }
+          s_io_epoch = e.epoch;
+        }
         bool ok = true;
-        if (!P.per_op && T.wait_ctr != cs.last_ctr) {
-          ok = wait_counter(P, T, t, &s_abort);
-          if (ok) cs.last_ctr = T.wait_ctr;
+        if (!P.per_op && (T.wait_ctr != cs.last_ctr || e.epoch != cs.last_epoch)) {
+          ok = wait_counter(P, T, t, e.epoch, &s_abort);
+          if (ok) {
+            cs.last_ctr = T.wait_ctr;
+            cs.last_epoch = e.epoch;
+          }
         } else if (s_abort) {
           ok = false;
         }
@@ -1594,7 +1760,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         switch (T.op) {
           case OP_EMBED: ok = P.dec_mma ? body_embed_mma(P, T) : body_embed(P); break;
           case OP_ATTN: ok = body_attn(P, T, S, cur, n_chunks, &s_abort); break;
-          case OP_FINAL: ok = body_final(P); break;
+          case OP_FINAL: ok = body_final(P, e.epoch); break;
           case OP_PEMBED: ok = body_pembed(P, T); break;
           case OP_GATHER: ok = body_gather(P); break;
           case OP_NORM: ok = body_norm(P, T); break;
@@ -1628,7 +1794,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           r.ev_issue = e.ev_issue;
           r.ev_start = ev_start;
           r.ev_done = atomicAdd(P.evclock, 1u);
-          r.epoch = P.epoch;
+          r.epoch = e.epoch;
           r.t_claim_ns = e.t_claim;
           r.t_issued_ns = *(volatile uint64_t*)&e.t_issued;
           r.t_start_ns = t_start;
@@ -1677,7 +1843,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(s_tmem, kTokBlock);
+    if (warp == 0) tmem_dealloc(s_tmem, (uint32_t)P.tmem_cols);
   }
 }
 

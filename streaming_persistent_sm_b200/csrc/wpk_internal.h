@@ -18,6 +18,8 @@ constexpr int kMaxQueue = 8;           // tiles a worker may hold (lookahead)
 constexpr int kMaxGemvBatch = 8;       // token rows per GEMV pass
 constexpr int kMaxTileRows = 128;      // rows per GEMV tile (partial-output buffer)
 constexpr int kMaxGroup = 8;           // q heads per kv head handled by one attention tile
+constexpr int kHeadDim = 64;           // the head dimension the attention tiles are written for
+constexpr int kAttnPages = 4;          // KV pages an attention tile computes per round
 constexpr int kMaxSmem = 232448;       // dynamic shared memory per CTA on sm_100
 
 // Op codes of the tiles.  One "op group" = the tiles of one op of one layer.
@@ -89,6 +91,29 @@ struct TraceRec {
 };
 static_assert(sizeof(TraceRec) == sizeof(wpk_trace_rec), "trace layout");
 
+// Resident grid control block in mapped (pinned) host memory: the host rings
+// the doorbell with the step number (steps count from 1 per grid launch) after
+// writing the step's I/O pointers; the last tile of a step stores its number
+// in `ack` after a system-scope fence.
+constexpr uint32_t kResShutdown = 0xFFFFFFFFu;
+struct ResCtl {
+  volatile uint32_t db;        // host: last step requested, or kResShutdown
+  volatile uint32_t ack;       // device: last step completed
+  volatile int32_t err;        // device: copy of the error word's code
+  volatile int32_t in_stride;  // step input: token stride
+  volatile uint64_t in_tok, out_tok, logits;  // step I/O device pointers (0 = none)
+  volatile uint64_t t_done_ns; // device %globaltimer when the last step completed
+};
+
+// Device-memory copy of the doorbell and step I/O: worker 0 alone polls the
+// mapped control block and publishes each step here (release), so the other
+// workers poll L2 instead of host memory.
+struct ResDev {
+  uint32_t db;
+  int32_t in_stride;
+  uint64_t in_tok, out_tok, logits;
+};
+
 struct ErrWord {
   int32_t code;
   uint32_t tile, counter, epoch, observed, target;
@@ -146,6 +171,10 @@ struct KParams {
   int region;
   int per_op;                // 1: one tile per CTA, no queue, no counters
   int static_sched;          // 1: worker w takes tickets w, w + W, ... (no queue)
+  int resident;              // 1: tickets run on across steps (epoch = ticket / tiles + 1)
+  uint64_t idle_ns;          // resident: how long a worker waits for the next step
+  ResCtl* ctl;               // resident: control block (device view of mapped memory)
+  ResDev* rdev;              // resident: its device-memory copy
   int stage_bytes;           // bytes per staging-ring stage
   int uses_tmem;             // the program has tensor-core tiles
   // prefill program (token rows m = b * T + t, M = B * T, blocks of 128)
@@ -159,6 +188,9 @@ struct KParams {
   // tensor-core operand geometry: the MMA N (tokens per tile) and the bytes of
   // one 64-column activation chunk (N rows of 128 bytes, 128-byte swizzle)
   int mma_n, act_chunk;
+  // accumulators a tile rotates its K-steps over (2 mma_n TMEM columns each)
+  // and the TMEM columns a worker allocates (a power of two >= 2 mma_n mma_acc)
+  int mma_acc, tmem_cols;
   // batched decode program (dec_mma = 1).  Token n of the step is MMA column n;
   // columns >= the active batch hold zeros.  Images are [K/64][act_chunk].
   int dec_mma;
