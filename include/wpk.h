@@ -57,11 +57,29 @@ enum { WPK_PREFILL_AUTO = 0, WPK_PREFILL_MMA = 1, WPK_PREFILL_TOKENWISE = 2 };
 enum { WPK_DECODE_AUTO = 0, WPK_DECODE_GEMV = 1, WPK_DECODE_MMA = 2 };
 
 /* --------------------------------------------------------------- configs */
-/* Decoder shape.  Weights are bf16, matmul weights stored [out][in]. */
+/* Decoder shape.  Weights are bf16, matmul weights stored [out][in].
+ *
+ * Two-stage streaming model ("Why real-time inference wants a megakernel":
+ * a backbone step followed by a short sequence of dependent head steps per
+ * frame; "One Megakernel is Not Enough", Table I, the two-stage TTS rows):
+ * set n_codebooks > 0 and `head` to the head decoder's shape.  The decoder
+ * described by the other fields is then the backbone; per frame and sequence
+ *   p = W_proj . RMSNorm(backbone state)          (the backbone's output head)
+ *   head step k (0..n_codebooks-1) reads p (k = 0) or head_embed_k[c_(k-1)],
+ *   c_k = argmax(out_head_k . RMSNorm(head state)), the head's cache restarting
+ *   every frame; the next backbone input is sum_k frame_embed_k[c_k].
+ * wpk_prefill / wpk_step then produce codes [B][n_codebooks] per frame (and
+ * logits [B][n_codebooks][codebook_vocab] when asked); the step's input is
+ * the previous frame's codes.  Two-stage handles run in WPK_MEGAKERNEL mode,
+ * without a resident grid. */
 typedef struct wpk_model_cfg {
   int n_layers, hidden, n_heads, n_kv_heads, head_dim, ffn, vocab;
   float rms_eps, rope_theta;
   int tied_embedding;   /* 1: the LM head is the token embedding */
+  int n_codebooks;      /* two-stage model: codebooks per frame (<= 16), else 0      */
+  int codebook_vocab;   /* two-stage model: codes per codebook                      */
+  const struct wpk_model_cfg *head;  /* two-stage model: the head decoder (its vocab,
+                                        n_codebooks and head fields are ignored) */
 } wpk_model_cfg;
 
 /* Execution plan: the operating point the program is compiled for ("Why
@@ -124,6 +142,13 @@ typedef struct wpk_weights {
   const uint16_t *final_norm;        /* [hidden]                             */
   const uint16_t *lm_head;           /* [vocab][hidden]; NULL when tied      */
   const wpk_layer_weights *layers;   /* [n_layers]                           */
+  /* two-stage model only (NULL otherwise); K = n_codebooks, V = codebook_vocab */
+  const uint16_t *proj;                   /* [head.hidden][hidden]                 */
+  const uint16_t *const *frame_embed;     /* K tables [V][hidden]                  */
+  const uint16_t *const *head_embed;      /* K tables [V][head.hidden]; entry 0 unused */
+  const uint16_t *const *out_head;        /* K tables [V][head.hidden]             */
+  const wpk_layer_weights *head_layers;   /* [head.n_layers]                       */
+  const uint16_t *head_final_norm;        /* [head.hidden]                         */
 } wpk_weights;
 
 typedef struct wpk_handle wpk_handle;

@@ -100,6 +100,20 @@ struct wpk_handle {
   bool res_live = false;
   uint32_t res_epoch = 0;         // last step rung on the live grid
   std::chrono::steady_clock::time_point res_last;
+  // per-launch step I/O overrides (the two-stage composition)
+  struct IO {
+    bool set = false;
+    int n_in = 1, in_rows = 0, logits_stride = 0, out_stride = 1;
+    uint64_t in_off[kMaxInTables] = {};
+    const float* in_vec = nullptr;
+    uint64_t lm_head_off = 0, lm_mma_off = 0;
+  } io;
+  // two-stage model: the head decoder and the tables outside both decoders
+  wpk_handle* head = nullptr;
+  int n_cb = 0, cb_vocab = 0;
+  uint64_t head_base = 0, weights_total = 0;  // head image offset; whole image
+  std::vector<uint64_t> frame_embed_off, head_embed_off, out_head_off, out_head_mma_off;
+  size_t off_p = 0, off_codes = 0;  // scratch: projection output [B][head hidden], last codes [B][K]
 };
 
 namespace {
@@ -126,7 +140,8 @@ int check_live(wpk_handle* h) {
     h->err = "no CUDA device: host-only handle";
     return WPK_ERR_CUDA;
   }
-  if (!h->poisoned && h->h_err_code && *(volatile int32_t*)h->h_err_code != 0) {
+  const bool head_err = h->head && h->head->h_err_code && *(volatile int32_t*)h->head->h_err_code != 0;
+  if (!h->poisoned && ((h->h_err_code && *(volatile int32_t*)h->h_err_code != 0) || head_err)) {
     h->poisoned = true;
     h->err = "device program reported an error (see wpk_get_error_info)";
   }
@@ -179,6 +194,13 @@ KParams make_params(const wpk_handle* h) {
   P.final_norm_off = g.lay.final_norm;
   P.embed_off = g.lay.embed;
   P.lm_head_off = g.lay.lm_head;
+  P.lm_rows = g.plan.lm_rows;
+  P.logits_stride = g.plan.lm_rows;
+  P.out_stride = 1;
+  P.n_in = 1;
+  P.in_rows = m.vocab;
+  P.in_table_off[0] = g.lay.embed;
+  P.in_vec = nullptr;
   P.kv = h->kv;
   P.n_blocks = h->n_blocks;
   P.block_table = h->d_block_table;
@@ -230,6 +252,16 @@ KParams make_params(const wpk_handle* h) {
     P.lm_mma_off = g.lay.lm_mma;
   }
   set_mma_geometry(&P);
+  if (h->io.set) {
+    P.n_in = h->io.n_in;
+    P.in_rows = h->io.in_rows;
+    for (int k = 0; k < kMaxInTables; ++k) P.in_table_off[k] = h->io.in_off[k];
+    P.in_vec = h->io.in_vec;
+    P.lm_head_off = h->io.lm_head_off;
+    if (P.dec_mma) P.lm_mma_off = h->io.lm_mma_off;
+    P.logits_stride = h->io.logits_stride;
+    P.out_stride = h->io.out_stride;
+  }
   return P;
 }
 
@@ -689,13 +721,16 @@ static int setup_device(wpk_handle* h) {
   return WPK_OK;
 }
 
-int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out) {
-  if (!model || !plan || !out) return WPK_ERR_INVALID_ARG;
+static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out);
+
+// One decoder; lm_rows > 0 replaces its output head's row count.
+static int build_decoder(const wpk_model_cfg* model, const wpk_plan_cfg* plan, int lm_rows, wpk_handle** out) {
   *out = nullptr;
   auto* h = new wpk_handle();
   int code = 0;
   Plan p;
   std::string msg = normalize_plan(*model, *plan, &p, &code);
+  if (lm_rows > 0) p.lm_rows = lm_rows;
   // worker count the tiles are sized for: the plan's, else #SMs x workers per SM
   int n_dev_w = 0, sms = 148;
   if (cudaGetDeviceCount(&n_dev_w) == cudaSuccess && n_dev_w > 0) {
@@ -732,11 +767,145 @@ int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_ha
   return WPK_OK;
 }
 
+int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out) {
+  if (!model || !plan || !out) return WPK_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (model->n_codebooks < 0) {
+    g_build_error = "n_codebooks must be >= 0";
+    return WPK_ERR_INVALID_ARG;
+  }
+  if (model->n_codebooks > 0) return build_two_stage(model, plan, out);
+  return build_decoder(model, plan, 0, out);
+}
+
+// Two-stage model: a backbone decoder whose output head is the projection into
+// the head's width, and a head decoder (its own handle, tables and program)
+// whose input and output tables change from one head step to the next.  Both
+// images, the frame / head-input / output tables and the tensor-core images of
+// the output tables share one weight buffer; KV and scratch likewise.
+static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out) {
+  const int K = model->n_codebooks, V = model->codebook_vocab;
+  if (!model->head || K > kMaxInTables || V <= 0) {
+    g_build_error = "two-stage model: needs a head shape, n_codebooks <= 16 and codebook_vocab > 0";
+    return WPK_ERR_INVALID_ARG;
+  }
+  if (plan->mode != WPK_MEGAKERNEL || plan->resident) {
+    g_build_error = "two-stage model: runs in WPK_MEGAKERNEL mode without a resident grid";
+    return WPK_ERR_UNSUPPORTED;
+  }
+  wpk_model_cfg mb = *model;  // backbone: output head = projection (untied)
+  mb.n_codebooks = 0;
+  mb.codebook_vocab = 0;
+  mb.head = nullptr;
+  mb.tied_embedding = 0;
+  wpk_model_cfg mh = *model->head;  // head: input and output tables have V rows
+  mh.vocab = V;
+  mh.tied_embedding = 0;
+  mh.n_codebooks = 0;
+  mh.codebook_vocab = 0;
+  mh.head = nullptr;
+  wpk_plan_cfg ph = *plan;  // the head's cache holds one frame
+  ph.max_context = K;
+  ph.page_tokens = (K + 7) / 8 * 8;
+  ph.n_regions = 1;
+  ph.prefill = WPK_PREFILL_TOKENWISE;
+  wpk_handle* h = nullptr;
+  int rc = build_decoder(&mb, plan, mh.hidden, &h);
+  if (rc) return rc;
+  wpk_handle* hh = nullptr;
+  rc = build_decoder(&mh, &ph, 0, &hh);
+  if (rc) {
+    wpk_destroy(h);
+    return rc;
+  }
+  h->head = hh;
+  h->n_cb = K;
+  h->cb_vocab = V;
+  // combined weight image: backbone, head, then the per-codebook tables
+  uint64_t off = a256(h->g.lay.total);
+  h->head_base = off;
+  off = a256(off + hh->g.lay.total);
+  auto take = [&](uint64_t bytes) { uint64_t o = off; off = a256(off + bytes); return o; };
+  const uint64_t vb = (uint64_t)(V + 127) / 128;
+  for (int k = 0; k < K; ++k) h->frame_embed_off.push_back(take((uint64_t)V * mb.hidden * 2));
+  for (int k = 0; k < K; ++k) h->head_embed_off.push_back(k ? take((uint64_t)V * mh.hidden * 2) : 0);
+  for (int k = 0; k < K; ++k) h->out_head_off.push_back(take((uint64_t)V * mh.hidden * 2));
+  for (int k = 0; k < K; ++k)
+    h->out_head_mma_off.push_back(hh->g.plan.decode_mode == WPK_DECODE_MMA
+                                      ? take(vb * (mh.hidden / 64) * kMmaChunkBytes)
+                                      : 0);
+  h->weights_total = off;
+  // scratch: the projection output and the last frame's codes, then the head's
+  const size_t B = plan->max_batch;
+  size_t so = h->scratch_bytes;
+  h->off_p = so;
+  so = a256(so + B * mh.hidden * 4);
+  h->off_codes = so;
+  so = a256(so + B * K * 4);
+  h->scratch_bytes = so;
+  *out = h;
+  return WPK_OK;
+}
+
 int wpk_workspace_size(const wpk_handle* h, size_t* weight_bytes, size_t* kv_bytes, size_t* scratch_bytes) {
   if (!h) return WPK_ERR_INVALID_ARG;
+  if (h->head) {
+    if (weight_bytes) *weight_bytes = h->weights_total;
+    if (kv_bytes) *kv_bytes = h->kv_bytes + h->head->kv_bytes;
+    if (scratch_bytes) *scratch_bytes = h->scratch_bytes + h->head->scratch_bytes;
+    return WPK_OK;
+  }
   if (weight_bytes) *weight_bytes = h->g.lay.total;
   if (kv_bytes) *kv_bytes = h->kv_bytes;
   if (scratch_bytes) *scratch_bytes = h->scratch_bytes;
+  return WPK_OK;
+}
+
+// Two-stage weights: the backbone (output head = projection), the head, and
+// the per-codebook tables, arranged into one image.
+static int load_two_stage(wpk_handle* h, const wpk_weights* w, void* dev_weights, void* dev_kv, void* dev_scratch,
+                          void* stream) {
+  wpk_handle* hh = h->head;
+  const int K = h->n_cb, V = h->cb_vocab;
+  if (!w->proj || !w->frame_embed || !w->head_embed || !w->out_head || !w->head_layers || !w->head_final_norm)
+    return fail(h, WPK_ERR_INVALID_ARG, "two-stage model: missing table pointers");
+  for (int k = 0; k < K; ++k)
+    if (!w->frame_embed[k] || !w->out_head[k] || (k > 0 && !w->head_embed[k]))
+      return fail(h, WPK_ERR_INVALID_ARG, "two-stage model: missing per-codebook table");
+  std::vector<uint8_t> img(h->weights_total, 0);
+  wpk_weights wb{};
+  wb.embed = w->embed;
+  wb.final_norm = w->final_norm;
+  wb.lm_head = w->proj;
+  wb.layers = w->layers;
+  if (!wb.embed) return fail(h, WPK_ERR_INVALID_ARG, "missing token embedding");
+  std::string msg = arrange_weights(h->g, wb, img.data());
+  if (!msg.empty()) return fail(h, WPK_ERR_INVALID_ARG, msg);
+  wpk_weights wh{};
+  wh.final_norm = w->head_final_norm;
+  wh.layers = w->head_layers;
+  msg = arrange_weights(hh->g, wh, img.data() + h->head_base);
+  if (!msg.empty()) return fail(h, WPK_ERR_INVALID_ARG, msg);
+  const int hb = h->g.m.hidden, hd = hh->g.m.hidden;
+  for (int k = 0; k < K; ++k) {
+    memcpy(img.data() + h->frame_embed_off[k], w->frame_embed[k], (size_t)V * hb * 2);
+    if (k) memcpy(img.data() + h->head_embed_off[k], w->head_embed[k], (size_t)V * hd * 2);
+    memcpy(img.data() + h->out_head_off[k], w->out_head[k], (size_t)V * hd * 2);
+    if (h->out_head_mma_off[k]) arrange_mma_image(img.data() + h->out_head_mma_off[k], hd, V, w->out_head[k]);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUDA_TRY(h, cudaMemcpyAsync(dev_weights, img.data(), img.size(), cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaStreamSynchronize(s));
+  h->weights = static_cast<uint8_t*>(dev_weights);
+  h->kv = static_cast<uint16_t*>(dev_kv);
+  h->scratch = static_cast<uint8_t*>(dev_scratch);
+  hh->weights = h->weights + h->head_base;
+  hh->kv = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(dev_kv) + h->kv_bytes);
+  hh->scratch = h->scratch + h->scratch_bytes;
+  h->loaded = hh->loaded = true;
+  h->prefilled = hh->prefilled = false;
+  h->graphs.clear();
+  hh->graphs.clear();
   return WPK_OK;
 }
 
@@ -750,6 +919,7 @@ int wpk_load_weights(wpk_handle* h, const wpk_weights* w, void* dev_weights, voi
     return fail(h, WPK_ERR_INVALID_ARG, "null weights or device buffer");
   if (((uintptr_t)dev_weights | (uintptr_t)dev_kv | (uintptr_t)dev_scratch) & 255)
     return fail(h, WPK_ERR_INVALID_ARG, "device buffers must be 256-byte aligned");
+  if (h->head) return load_two_stage(h, w, dev_weights, dev_kv, dev_scratch, stream);
   std::vector<uint8_t> img(h->g.lay.total, 0);
   std::string msg = arrange_weights(h->g, *w, img.data());
   if (!msg.empty()) return fail(h, WPK_ERR_INVALID_ARG, msg);
@@ -780,8 +950,55 @@ int wpk_set_block_table(wpk_handle* h, const int32_t* table) {
   return WPK_OK;
 }
 
+static int prefill_impl(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len, int32_t* first_tok_dev,
+                        float* logits_dev, void* stream);
+
+// State the step programs keep between steps, cleared for a new batch of
+// sequences: argmax keys, split arrivals and (tensor-core decode) the fp32
+// sums and per-token x^2 sums, which the program itself returns to zero.
+static int reset_step_state(wpk_handle* h, cudaStream_t s) {
+  const size_t B = h->g.plan.max_batch;
+  CUDA_TRY(h, cudaMemsetAsync(h->d_seqlen, 0, B * 4, s));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_best, 0, B * 8, s));
+  CUDA_TRY(h, cudaMemsetAsync(h->d_arrive, 0, B * h->g.m.n_kv_heads * 4, s));
+  if (h->g.plan.decode_mode == WPK_DECODE_MMA) {
+    const wpk_model_cfg& m = h->g.m;
+    const size_t N = h->g.plan.dec_n;
+    const size_t qkv_rows = (size_t)(m.n_heads + 2 * m.n_kv_heads) * m.head_dim;
+    CUDA_TRY(h, cudaMemsetAsync(h->scratch + h->off_acc, 0, qkv_rows * N * 4, s));
+    CUDA_TRY(h, cudaMemsetAsync(h->scratch + h->off_ss, 0, (2 * (size_t)m.n_layers + 1) * N * 4, s));
+    CUDA_TRY(h, cudaMemsetAsync(h->d_rb_arrive, 0, (size_t)m.n_layers * 2 * (m.hidden / 128 + 1) * 4, s));
+  }
+  return WPK_OK;
+}
+static int head_frame(wpk_handle* h, int32_t* codes_out, float* logits, cudaStream_t s);
+
 int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len, int32_t* first_tok_dev,
                 float* logits_dev, void* stream) {
+  if (!h || !h->head) return prefill_impl(h, tokens_dev, batch, prompt_len, first_tok_dev, logits_dev, stream);
+  // two-stage: the prompt through the backbone, whose output head yields the
+  // projection p at the last position; then the head's first frame
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* codes = reinterpret_cast<int32_t*>(h->scratch + h->off_codes);
+  float* p = reinterpret_cast<float*>(h->scratch + h->off_p);
+  int rc = prefill_impl(h, tokens_dev, batch, prompt_len, codes, p, stream);
+  if (rc) return rc;
+  wpk_handle* hh = h->head;
+  rc = reset_step_state(hh, s);
+  if (rc) return rc;
+  CUDA_TRY(h, cudaMemcpyAsync(hh->d_active, &batch, 4, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaStreamSynchronize(s));  // `batch` lives on this stack frame
+  hh->batch = batch;
+  hh->prefilled = true;
+  rc = head_frame(h, first_tok_dev ? first_tok_dev : codes, logits_dev, s);
+  if (rc) return rc;
+  if (first_tok_dev)
+    CUDA_TRY(h, cudaMemcpyAsync(codes, first_tok_dev, (size_t)batch * h->n_cb * 4, cudaMemcpyDeviceToDevice, s));
+  return WPK_OK;
+}
+
+static int prefill_impl(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len, int32_t* first_tok_dev,
+                        float* logits_dev, void* stream) {
   int rc = check_live(h);
   if (rc) return rc;
   rc = res_shutdown(h);
@@ -791,19 +1008,8 @@ int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_
   if (batch > h->g.plan.max_batch || prompt_len > h->g.plan.max_context)
     return fail(h, WPK_ERR_SHAPE, "batch or prompt exceeds the plan");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t B = h->g.plan.max_batch;
-  CUDA_TRY(h, cudaMemsetAsync(h->d_seqlen, 0, B * 4, s));
-  CUDA_TRY(h, cudaMemsetAsync(h->d_best, 0, B * 8, s));
-  CUDA_TRY(h, cudaMemsetAsync(h->d_arrive, 0, B * h->g.m.n_kv_heads * 4, s));
-  if (h->g.plan.decode_mode == WPK_DECODE_MMA) {
-    // the batched decode program keeps these at zero between steps itself
-    const wpk_model_cfg& m = h->g.m;
-    const size_t N = h->g.plan.dec_n;
-    const size_t qkv_rows = (size_t)(m.n_heads + 2 * m.n_kv_heads) * m.head_dim;
-    CUDA_TRY(h, cudaMemsetAsync(h->scratch + h->off_acc, 0, qkv_rows * N * 4, s));
-    CUDA_TRY(h, cudaMemsetAsync(h->scratch + h->off_ss, 0, (2 * (size_t)m.n_layers + 1) * N * 4, s));
-    CUDA_TRY(h, cudaMemsetAsync(h->d_rb_arrive, 0, (size_t)m.n_layers * 2 * (m.hidden / 128 + 1) * 4, s));
-  }
+  rc = reset_step_state(h, s);
+  if (rc) return rc;
   CUDA_TRY(h, cudaMemcpyAsync(h->d_active, &batch, 4, cudaMemcpyHostToDevice, s));
   CUDA_TRY(h, cudaStreamSynchronize(s));  // `batch` lives on this stack frame
   h->batch = batch;
@@ -841,7 +1047,65 @@ int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, flo
   if (rc) return rc;
   if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");
   if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
-  return step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, static_cast<cudaStream_t>(stream));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!h->head) return step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, s);
+  // two-stage frame: backbone step on sum_k frame_embed_k[c_k] -> p, then the head
+  int32_t* codes = reinterpret_cast<int32_t*>(h->scratch + h->off_codes);
+  const int K = h->n_cb;
+  h->io = wpk_handle::IO{};
+  h->io.set = true;
+  h->io.n_in = K;
+  h->io.in_rows = h->cb_vocab;
+  for (int k = 0; k < K; ++k) h->io.in_off[k] = h->frame_embed_off[k];
+  h->io.lm_head_off = h->g.lay.lm_head;
+  h->io.lm_mma_off = h->g.lay.lm_mma;
+  h->io.logits_stride = h->g.plan.lm_rows;
+  h->io.out_stride = 1;
+  rc = step_impl(h, in_tok_dev ? in_tok_dev : codes, K, nullptr,
+                 reinterpret_cast<float*>(h->scratch + h->off_p), s);
+  h->io.set = false;
+  if (rc) return rc;
+  rc = head_frame(h, out_tok_dev ? out_tok_dev : codes, logits_dev, s);
+  if (rc) return rc;
+  if (out_tok_dev)
+    CUDA_TRY(h, cudaMemcpyAsync(codes, out_tok_dev, (size_t)h->batch * K * 4, cudaMemcpyDeviceToDevice, s));
+  return WPK_OK;
+}
+
+// The head's K steps of one frame: step k reads p (k = 0) or head_embed_k of
+// code k-1, writes code k (and its logits) through output table k; the head's
+// positions restart at 0.
+static int head_frame(wpk_handle* h, int32_t* codes_out, float* logits, cudaStream_t s) {
+  wpk_handle* hh = h->head;
+  const int K = h->n_cb, V = h->cb_vocab;
+  CUDA_TRY(h, cudaMemsetAsync(hh->d_seqlen, 0, (size_t)hh->g.plan.max_batch * 4, s));
+  hh->ctx = 0;
+  int rc = WPK_OK;
+  for (int k = 0; k < K && !rc; ++k) {
+    hh->io = wpk_handle::IO{};
+    hh->io.set = true;
+    if (k == 0) {
+      hh->io.n_in = 0;
+      hh->io.in_vec = reinterpret_cast<const float*>(h->scratch + h->off_p);
+    } else {
+      hh->io.n_in = 1;
+      hh->io.in_off[0] = h->head_embed_off[k] - h->head_base;
+    }
+    hh->io.in_rows = V;
+    hh->io.lm_head_off = h->out_head_off[k] - h->head_base;
+    hh->io.lm_mma_off = h->out_head_mma_off[k] ? h->out_head_mma_off[k] - h->head_base : 0;
+    hh->io.logits_stride = K * V;
+    hh->io.out_stride = K;
+    rc = step_impl(hh, k ? codes_out + (k - 1) : nullptr, K, codes_out + k, logits ? logits + (size_t)k * V : nullptr,
+                   s);
+  }
+  hh->io.set = false;
+  if (rc) {
+    h->err = "head: " + hh->err;
+    return rc;
+  }
+  if (*hh->h_err_code && !*h->h_err_code) *h->h_err_code = *hh->h_err_code;
+  return WPK_OK;
 }
 
 int wpk_graph_stats_get(const wpk_handle* h, wpk_graph_stats* st) {
@@ -956,6 +1220,10 @@ const char* wpk_last_error(const wpk_handle* h) { return h ? h->err.c_str() : g_
 
 int wpk_destroy(wpk_handle* h) {
   if (!h) return WPK_ERR_INVALID_ARG;
+  if (h->head) {
+    wpk_destroy(h->head);
+    h->head = nullptr;
+  }
   if (h->has_device) {
     res_shutdown(h);
     cudaDeviceSynchronize();

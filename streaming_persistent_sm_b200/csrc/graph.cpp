@@ -100,6 +100,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   if ((int64_t)p->page_tokens * m.head_dim * 2 * 2 > kStageBytes)
     return "a KV page (K and V rows) does not fit one 16 KB stage";
   p->per_op_slot = 0;  // set by compile_graph
+  p->lm_rows = m.vocab;  // a two-stage backbone overrides it with its projection width
   {
     const int qr = m.n_heads * m.head_dim, kvr = m.n_kv_heads * m.head_dim;
     const bool mma_ok = (qr + 2 * kvr) % 128 == 0 && m.hidden % 128 == 0 && (2 * m.ffn) % 128 == 0 &&
@@ -329,13 +330,15 @@ struct LmTile {
   uint32_t w_bytes;
   int r0, n;
 };
+// Offsets are relative to the LM head's base (the launch's lm_head_off).
 std::vector<LmTile> gemv_lm_tiles(const wpk_model_cfg& m, const Plan& p, int W, const Layout& L) {
+  (void)L;
   std::vector<LmTile> out;
-  const int h = m.hidden;
-  const int R = rows_per_tile(h * 2, m.vocab, p, W);
-  for (int r0 = 0; r0 < m.vocab; r0 += R) {
-    const int n = std::min(R, m.vocab - r0);
-    out.push_back({L.lm_head + (uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n});
+  const int h = m.hidden, rows = p.lm_rows;
+  const int R = rows_per_tile(h * 2, rows, p, W);
+  for (int r0 = 0; r0 < rows; r0 += R) {
+    const int n = std::min(R, rows - r0);
+    out.push_back({(uint64_t)r0 * h * 2, (uint32_t)n * h * 2, r0, n});
   }
   return out;
 }
@@ -417,9 +420,9 @@ void build_mma_decode_tiles(const wpk_model_cfg& m, const Plan& p, int W, Compil
       }
   }
   (*layer_begin)[m.n_layers] = (uint32_t)g.tiles.size();
-  for (int vb = 0; vb < L.vocab_blocks; ++vb) {
-    const int r0 = vb * 128, n = std::min(128, m.vocab - r0);
-    add(OP_BLM, m.n_layers, L.lm_mma + (uint64_t)vb * nkc_h * chunk, (uint32_t)nkc_h * chunk, vb, 0, 0, h,
+  for (int vb = 0; vb < L.vocab_blocks; ++vb) {  // offsets relative to the launch's lm_mma_off
+    const int r0 = vb * 128, n = std::min(128, p.lm_rows - r0);
+    add(OP_BLM, m.n_layers, (uint64_t)vb * nkc_h * chunk, (uint32_t)nkc_h * chunk, vb, 0, 0, h,
         {{BUF_DXN, 0, h, 0}, {BUF_LOGITS, r0, r0 + n, 1}, {BUF_BEST, 0, 1, 2}});
   }
   add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0}, {BUF_TOK, 0, 1, 1}});
@@ -460,7 +463,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   }
   L.final_norm = take((uint64_t)h * 4);
   L.embed = take((uint64_t)m.vocab * h * 2);
-  L.lm_head = m.tied_embedding ? L.embed : take((uint64_t)m.vocab * h * 2);
+  L.lm_head = m.tied_embedding ? L.embed : take((uint64_t)p.lm_rows * h * 2);
   L.mma = p.prefill_mode == WPK_PREFILL_MMA || p.decode_mode == WPK_DECODE_MMA;
   for (int l = 0; l < m.n_layers; ++l) {
     LayerDev& d = L.layers[l];
@@ -474,7 +477,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   L.lm_mma = 0;
   L.vocab_blocks = 0;
   if (p.decode_mode == WPK_DECODE_MMA) {
-    L.vocab_blocks = (m.vocab + 127) / 128;
+    L.vocab_blocks = (p.lm_rows + 127) / 128;
     L.lm_mma = take((uint64_t)L.vocab_blocks * (h / 64) * kMmaChunkBytes);
   }
   L.total = off;
@@ -599,7 +602,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
 
   // ---- edges from dataflow ----
   DataflowBuilder df;
-  int sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1, 1, 1, 1, 1, 1, 1, h, h};
+  int sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, p.lm_rows, 1, 1, 1, 1, 1, 1, 1, 1, h, h};
   for (int b = 0; b < BUF_COUNT; ++b) df.bufs.emplace_back(sizes[b]);
   g->preds.assign(T.size(), {});
   df.preds_of = &g->preds;
@@ -799,7 +802,7 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
   if (Tl.size() >= (1u << 31)) return "too many tiles";
 
   DataflowBuilder df;
-  const int64_t sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, m.vocab, 1, 1,
+  const int64_t sizes[BUF_COUNT] = {h, h, qkv_rows, q_rows, m.ffn, p.lm_rows, 1, 1,
                                     (int64_t)nq * h * TB, (int64_t)nq * h * TB, (int64_t)nq * q_rows * TB,
                                     (int64_t)m.n_layers * nq * 2 * kv_rows * TB, (int64_t)nq * q_rows * TB,
                                     (int64_t)nq * m.ffn * TB, h, h};
@@ -966,6 +969,22 @@ int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t
   return WPK_OK;
 }
 
+// Tensor-core image of a [rows][K] bf16 matrix: blocks of 128 rows x 64
+// columns (16 KB), block (r / 128, c / 64) at ((r / 128) * K / 64 + c / 64) *
+// 16 KB, the 16-byte unit u of row r stored at unit u XOR (r % 8); rows past
+// `rows` in the last block stay as the caller initialised them.
+void arrange_mma_image(uint8_t* base, int K, int rows, const uint16_t* src) {
+  const int nkc = K / 64;
+  for (int r = 0; r < rows; ++r) {
+    uint8_t* blk0 = base + (uint64_t)(r / 128) * nkc * kMmaChunkBytes;
+    const int rr = r % 128;
+    for (int c = 0; c < nkc; ++c)
+      for (int u = 0; u < 8; ++u)
+        memcpy(blk0 + (uint64_t)c * kMmaChunkBytes + rr * 128 + ((u ^ (rr & 7)) * 16),
+               src + (uint64_t)r * K + c * 64 + u * 8, 16);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Weight image: fp32 norm gains; QKV rows permuted so that RoPE pair rows
 // (i, i + d/2) of every q/k head sit next to each other; gate/up rows
@@ -974,8 +993,9 @@ std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_
   const wpk_model_cfg& m = g.m;
   const int h = m.hidden, hd = m.head_dim;
   const int q_rows = m.n_heads * hd, kv_rows = m.n_kv_heads * hd;
-  if (!w.embed || !w.final_norm || !w.layers || (!m.tied_embedding && !w.lm_head))
-    return "missing weight pointer";
+  // (a two-stage head has no token embedding, and its output heads live
+  // outside this decoder's image: both pointers may then be NULL)
+  if (!w.final_norm || !w.layers || (m.tied_embedding && !w.embed)) return "missing weight pointer";
   auto gain = [&](const uint16_t* src, uint64_t off) {
     float* dst = reinterpret_cast<float*>(img + off);
     for (int i = 0; i < h; ++i) {
@@ -1039,9 +1059,10 @@ std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_
   };
   // the LM head's tensor-core image (batched decode), in 16 row slices per task
   const uint16_t* lm_src = m.tied_embedding ? w.embed : w.lm_head;
-  const int lm_tasks = g.lay.lm_mma ? 16 : 0;
+  const int lm_tasks = (g.lay.lm_mma && lm_src) ? 16 : 0;
   auto do_lm = [&](int i) {
-    const int r0 = (int)((int64_t)m.vocab * i / lm_tasks), r1 = (int)((int64_t)m.vocab * (i + 1) / lm_tasks);
+    const int rows = g.plan.lm_rows;
+    const int r0 = (int)((int64_t)rows * i / lm_tasks), r1 = (int)((int64_t)rows * (i + 1) / lm_tasks);
     for (int r = r0; r < r1; ++r) mma_row(g.lay.lm_mma, h, r, lm_src + (uint64_t)r * h);
   };
   unsigned nt = std::max(1u, std::min(16u, std::thread::hardware_concurrency()));
@@ -1056,8 +1077,8 @@ std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_
       }
     });
   gain(w.final_norm, g.lay.final_norm);
-  memcpy(img + g.lay.embed, w.embed, (size_t)m.vocab * h * 2);
-  if (!m.tied_embedding) memcpy(img + g.lay.lm_head, w.lm_head, (size_t)m.vocab * h * 2);
+  if (w.embed) memcpy(img + g.lay.embed, w.embed, (size_t)m.vocab * h * 2);
+  if (!m.tied_embedding && w.lm_head) memcpy(img + g.lay.lm_head, w.lm_head, (size_t)g.plan.lm_rows * h * 2);
   for (auto& x : th) x.join();
   return "";
 }

@@ -22,6 +22,7 @@ struct Plan {
   // batched decode program: MMA N (max_batch rounded up to 16), its ring
   // stage (16 KB of weights + hi/lo activation chunks), stages, scratch bytes
   int dec_n, dec_stage_bytes, dec_stages, dec_act_bytes;
+  int lm_rows;          // rows of the output head (0 = vocab; the two-stage backbone's is its projection)
 };
 
 struct Layout {
@@ -66,5 +67,7 @@ int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t
                    int stuck_tile, int32_t* done_order, std::string* msg);
 // Arrange host bf16 weights into the image (host buffer of lay.total bytes).
 std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_t* image);
+// Tensor-core image of one [rows][K] bf16 matrix (see graph.cpp).
+void arrange_mma_image(uint8_t* base, int K, int rows, const uint16_t* src);
 
 }  // namespace wpk

@@ -270,7 +270,8 @@ __device__ __forceinline__ const uint8_t* mma_act_src(const KParams& P, const Ti
 // the 16 KB weight block, then the hi and the lo activation chunk.
 __device__ void issue_mma_w(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
   mbar_arrive_expect_tx(bar, (uint32_t)kMmaChunkBytes + 2u * (uint32_t)P.act_chunk);
-  bulk_g2s(dst, P.weights + T.w_off + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
+  const uint64_t base = (T.op == OP_BLM) ? P.lm_mma_off : 0;  // LM tiles are relative to the launch's head
+  bulk_g2s(dst, P.weights + base + T.w_off + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
 }
 __device__ void issue_mma_act(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
   const uint32_t a = (uint32_t)P.act_chunk;
@@ -307,8 +308,9 @@ __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uin
   const size_t row_bytes = (size_t)T.a3 * 2;
   const int r0 = k * rpc;
   const uint32_t bytes = (uint32_t)(min(rpc, T.a1 - r0) * row_bytes);
+  const uint64_t base = (T.op == OP_LMHEAD) ? P.lm_head_off : 0;  // LM tiles are relative to the launch's head
   mbar_arrive_expect_tx(bar, bytes);
-  bulk_g2s(dst, P.weights + T.w_off + r0 * row_bytes, bytes, bar);
+  bulk_g2s(dst, P.weights + base + T.w_off + r0 * row_bytes, bytes, bar);
 }
 
 // ---------------------------------------------------------------------------
@@ -440,7 +442,7 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
       if (s_logits)
         for (int idx = threadIdx.x; idx < R * bg; idx += kThreads) {
           const int rr = idx % R, b = idx / R, bi = b0 + b;
-          s_logits[(size_t)bi * P.vocab + r0 + rr] = out[rr * S + b];
+          s_logits[(size_t)bi * P.logits_stride + r0 + rr] = out[rr * S + b];
         }
       const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
       if (warp < bg) {
@@ -1113,12 +1115,12 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
     }
     case OP_BLM: {
       const int nb = active_batch(P);
-      const bool valid = f < P.vocab;
+      const bool valid = f < P.lm_rows;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int n = n0 + i;
         const float val = v[i] * s_rn[n];
-        if (s_logits && valid && n < nb) s_logits[(size_t)n * P.vocab + f] = val;
+        if (s_logits && valid && n < nb) s_logits[(size_t)n * P.logits_stride + f] = val;
         unsigned long long key = valid ? argmax_key(val, f) : 0ull;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -1430,53 +1432,88 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
   return true;
 }
 
-__device__ bool body_embed(const KParams& P) {
-  const int nb = active_batch(P);
-  const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
-  for (int b = 0; b < nb; ++b) {
-    int tok = s_in_tok ? s_in_tok[(size_t)b * s_in_stride] : P.tok_fb[b];
-    if (tok < 0 || tok >= P.vocab) {
-      if (threadIdx.x == 0) record_error(P, WPK_ERR_INVALID_ARG, 0, kNoCounter, (uint32_t)tok, (uint32_t)P.vocab);
+// x[b] = the step's input of sequence b: the sum over n_in tables of
+// table_k[code_k] (code_k at input row b, column k; the last greedy token when
+// no input is given), or the vector in_vec[b] when n_in == 0.
+__device__ bool step_codes(const KParams& P, int b, int* codes) {
+  if (threadIdx.x < P.n_in) {
+    int tok = s_in_tok ? s_in_tok[(size_t)b * s_in_stride + threadIdx.x] : P.tok_fb[b];
+    if (tok < 0 || tok >= P.in_rows) {
+      record_error(P, WPK_ERR_INVALID_ARG, (uint32_t)b, kNoCounter, (uint32_t)tok, (uint32_t)P.in_rows);
       tok = 0;
     }
-    const uint4* row = reinterpret_cast<const uint4*>(E + (size_t)tok * P.hidden);
+    codes[threadIdx.x] = tok;
+  }
+  return true;
+}
+
+__device__ bool body_embed(const KParams& P) {
+  __shared__ int s_code[kMaxInTables];
+  const int nb = active_batch(P);
+  for (int b = 0; b < nb; ++b) {
+    step_codes(P, b, s_code);
+    cbar();
     float* x = P.xa + (size_t)b * P.hidden;
     for (int k = threadIdx.x; k < P.hidden / 8; k += kThreads) {
-      float f[8];
-      unpack8(__ldg(row + k), f);
+      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (P.n_in == 0) {
+        const float4* v = reinterpret_cast<const float4*>(P.in_vec + (size_t)b * P.hidden) + 2 * k;
+        const float4 a = __ldcg(v), c = __ldcg(v + 1);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = c.x; f[5] = c.y; f[6] = c.z; f[7] = c.w;
+      }
+      for (int t = 0; t < P.n_in; ++t) {
+        const uint4* row = reinterpret_cast<const uint4*>(P.weights + P.in_table_off[t]) + (size_t)s_code[t] * (P.hidden / 8);
+        float e[8];
+        unpack8(__ldg(row + k), e);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] += e[q];
+      }
       reinterpret_cast<float4*>(x)[2 * k] = make_float4(f[0], f[1], f[2], f[3]);
       reinterpret_cast<float4*>(x)[2 * k + 1] = make_float4(f[4], f[5], f[6], f[7]);
     }
+    cbar();
   }
   return true;
 }
 
 // Batched decode: x = E[tok] for the 128 features of block a0, feature-major,
 // with the first RMSNorm's input image (x * g) and the x^2 sums.
-__device__ bool body_embed_mma(const KParams& P, const Tile& T) {
-  __shared__ int s_tok[kMaxMmaBatch];
+__device__ bool body_embed_mma(const KParams& P, const Tile& T, int* codes /* [mma_n][n_in], shared */) {
   __shared__ float s_sq2[kMaxMmaBatch];
   const int N = P.mma_n, nb = active_batch(P);
-  if (threadIdx.x < N) {
+  for (int i = threadIdx.x; i < N * P.n_in; i += kThreads) {
+    const int n = i / P.n_in, t = i % P.n_in;
     int tok = 0;
-    if (threadIdx.x < nb) {
-      tok = s_in_tok ? s_in_tok[(size_t)threadIdx.x * s_in_stride] : P.tok_fb[threadIdx.x];
-      if (tok < 0 || tok >= P.vocab) {
-        record_error(P, WPK_ERR_INVALID_ARG, 0, kNoCounter, (uint32_t)tok, (uint32_t)P.vocab);
+    if (n < nb) {
+      tok = s_in_tok ? s_in_tok[(size_t)n * s_in_stride + t] : P.tok_fb[n];
+      if (tok < 0 || tok >= P.in_rows) {
+        record_error(P, WPK_ERR_INVALID_ARG, (uint32_t)n, kNoCounter, (uint32_t)tok, (uint32_t)P.in_rows);
         tok = 0;
       }
     }
-    s_tok[threadIdx.x] = tok;
-    s_sq2[threadIdx.x] = 0.f;
+    codes[i] = tok;
   }
+  if (threadIdx.x < N) s_sq2[threadIdx.x] = 0.f;
   cbar();
-  const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.embed_off);
   const float* gain = reinterpret_cast<const float*>(P.weights + P.layers[0].attn_norm);
   for (int u = threadIdx.x; u < 16 * N; u += kThreads) {
     const int j = u / N, n = u % N;
     const int f0 = T.a0 * 128 + 8 * j;
     float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (n < nb) unpack8(__ldg(reinterpret_cast<const uint4*>(E + (size_t)s_tok[n] * P.hidden + f0)), x);
+    if (n < nb) {
+      if (P.n_in == 0) {
+        const float4* v = reinterpret_cast<const float4*>(P.in_vec + (size_t)n * P.hidden + f0);
+        const float4 a = __ldcg(v), c = __ldcg(v + 1);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+      }
+      for (int t = 0; t < P.n_in; ++t) {
+        const uint16_t* E = reinterpret_cast<const uint16_t*>(P.weights + P.in_table_off[t]);
+        float e[8];
+        unpack8(__ldg(reinterpret_cast<const uint4*>(E + (size_t)codes[n * P.n_in + t] * P.hidden + f0)), e);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) x[q] += e[q];
+      }
+    }
     float sq = 0.f;
     uint32_t ph[4], pl[4];
 #pragma unroll
@@ -1508,7 +1545,7 @@ __device__ bool body_final(const KParams& P, uint32_t epoch) {
   for (int b = threadIdx.x; b < nb; b += kThreads) {
     const unsigned long long key = P.best[b];
     const int32_t idx = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
-    if (s_out_tok) s_out_tok[b] = idx;
+    if (s_out_tok) s_out_tok[(size_t)b * P.out_stride] = idx;
     P.tok_fb[b] = idx;
     P.best[b] = 0ull;
     P.seqlen[b] += 1;
@@ -1758,7 +1795,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       bool ok = !s_fail;
       if (ok) {
         switch (T.op) {
-          case OP_EMBED: ok = P.dec_mma ? body_embed_mma(P, T) : body_embed(P); break;
+          case OP_EMBED: ok = P.dec_mma ? body_embed_mma(P, T, reinterpret_cast<int*>(S.act)) : body_embed(P); break;
           case OP_ATTN: ok = body_attn(P, T, S, cur, n_chunks, &s_abort); break;
           case OP_FINAL: ok = body_final(P, e.epoch); break;
           case OP_PEMBED: ok = body_pembed(P, T); break;

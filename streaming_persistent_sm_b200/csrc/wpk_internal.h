@@ -53,6 +53,7 @@ enum Op : uint16_t {
 constexpr int kTokBlock = 128;   // tokens per tensor-core tile (the MMA N)
 constexpr int kPrefillQB = 32;   // queries per prefill attention tile
 constexpr int kMaxMmaBatch = 128;  // sequences of a batched decode step (MMA N <= 128)
+constexpr int kMaxInTables = 16;   // input tables a step's input may sum over
 constexpr int kMmaChunkBytes = 128 * 128;  // 128 rows x 64 bf16, one K chunk
 
 // One tile of the step program, in ticket order.  48 bytes.
@@ -200,7 +201,18 @@ struct KParams {
   float* ss;                  // [2 n_layers + 1][mma_n] sums of x^2 per RMSNorm
   uint8_t* xf_img[2];         // hi/lo image of x * g_ffn (xn_img holds x * g_attn / g_final)
   uint32_t* rb_arrive;        // [n_layers][2][hidden/128] split-K arrivals per row block
-  uint64_t lm_mma_off;        // tensor-core image of the LM head [vocab/128][hidden/64][16 KB]
+  uint64_t lm_mma_off;        // tensor-core image of the LM head [lm_rows/128][hidden/64][16 KB]
+  // output head and step I/O layout: LM head tiles hold offsets relative to
+  // lm_head_off / lm_mma_off, so one program can switch output tables per launch
+  int lm_rows;                // rows of the output head (= vocab for a plain decoder)
+  int logits_stride;          // floats between two sequences' logits
+  int out_stride;             // int32s between two sequences' output tokens
+  // step input: x = sum over n_in tables of table_k[code_k] (codes at
+  // in_tok[b * stride + k], below in_rows), or the vector in_vec[b][hidden]
+  // when n_in == 0
+  int n_in, in_rows;
+  uint64_t in_table_off[kMaxInTables];
+  const float* in_vec;
 };
 
 // Host-side compiled graph.

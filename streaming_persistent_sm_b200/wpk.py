@@ -50,9 +50,13 @@ class WpkError(RuntimeError):
 
 
 class wpk_model_cfg(C.Structure):
-    _fields_ = [("n_layers", C.c_int), ("hidden", C.c_int), ("n_heads", C.c_int), ("n_kv_heads", C.c_int),
-                ("head_dim", C.c_int), ("ffn", C.c_int), ("vocab", C.c_int), ("rms_eps", C.c_float),
-                ("rope_theta", C.c_float), ("tied_embedding", C.c_int)]
+    pass
+
+
+wpk_model_cfg._fields_ = [("n_layers", C.c_int), ("hidden", C.c_int), ("n_heads", C.c_int), ("n_kv_heads", C.c_int),
+                          ("head_dim", C.c_int), ("ffn", C.c_int), ("vocab", C.c_int), ("rms_eps", C.c_float),
+                          ("rope_theta", C.c_float), ("tied_embedding", C.c_int), ("n_codebooks", C.c_int),
+                          ("codebook_vocab", C.c_int), ("head", C.POINTER(wpk_model_cfg))]
 
 
 class wpk_plan_cfg(C.Structure):
@@ -72,7 +76,10 @@ class wpk_layer_weights(C.Structure):
 
 
 class wpk_weights(C.Structure):
-    _fields_ = [("embed", _P16), ("final_norm", _P16), ("lm_head", _P16), ("layers", C.POINTER(wpk_layer_weights))]
+    _fields_ = [("embed", _P16), ("final_norm", _P16), ("lm_head", _P16), ("layers", C.POINTER(wpk_layer_weights)),
+                ("proj", _P16), ("frame_embed", C.POINTER(_P16)), ("head_embed", C.POINTER(_P16)),
+                ("out_head", C.POINTER(_P16)), ("head_layers", C.POINTER(wpk_layer_weights)),
+                ("head_final_norm", _P16)]
 
 
 class wpk_graph_stats(C.Structure):
@@ -142,8 +149,17 @@ def _check(rc: int, h=None):
 
 
 def model_cfg(shape) -> wpk_model_cfg:
+    """A decoder shape, or a two-stage shape (backbone + codebook head)."""
+    if hasattr(shape, "backbone"):
+        head = model_cfg(shape.head)
+        m = model_cfg(shape.backbone)
+        m.n_codebooks = shape.n_codebooks
+        m.codebook_vocab = shape.codebook_vocab
+        m._head = head  # keep the head struct alive
+        m.head = C.pointer(head)
+        return m
     return wpk_model_cfg(shape.n_layers, shape.hidden, shape.n_heads, shape.n_kv_heads, shape.head_dim, shape.ffn,
-                         shape.vocab, shape.rms_eps, shape.rope_theta, 1 if shape.tied_embedding else 0)
+                         shape.vocab, shape.rms_eps, shape.rope_theta, 1 if shape.tied_embedding else 0, 0, 0, None)
 
 
 def plan_cfg(max_batch: int, max_context: int, mode: int = WPK_MEGAKERNEL, n_regions: int = 1,
@@ -273,17 +289,32 @@ class _HostWeights:
         self.arrays = []
 
         def ptr(name):
-            a = np.ascontiguousarray(weights[prefix + name], dtype=np.uint16)
+            a = np.ascontiguousarray(weights[name], dtype=np.uint16)
             self.arrays.append(a)
             return a.ctypes.data_as(_P16)
 
-        self.layers = (wpk_layer_weights * shape.n_layers)()
-        for l in range(shape.n_layers):
-            p = f"layers.{l}."
-            for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down"):
-                setattr(self.layers[l], n, ptr(p + n))
-        self.struct = wpk_weights(ptr("embed"), ptr("final_norm"),
-                                  ptr("lm_head") if not shape.tied_embedding else None, self.layers)
+        def layers(s, pre):
+            arr = (wpk_layer_weights * s.n_layers)()
+            for l in range(s.n_layers):
+                p = f"{pre}layers.{l}."
+                for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate", "w_up", "w_down"):
+                    setattr(arr[l], n, ptr(p + n))
+            return arr
+
+        if hasattr(shape, "backbone"):  # two-stage model
+            bb, K = shape.backbone, shape.n_codebooks
+            self.layers = layers(bb, "backbone.")
+            self.head_layers = layers(shape.head, "head.")
+            tables = lambda name, first: (_P16 * K)(*([None] * first + [ptr(f"{name}.{k}") for k in range(first, K)]))
+            self.frame_embed, self.head_embed, self.out_head = (tables("frame_embed", 0), tables("head_embed", 1),
+                                                                tables("out_head", 0))
+            self.struct = wpk_weights(ptr("backbone.embed"), ptr("backbone.final_norm"), None, self.layers,
+                                      ptr("proj"), self.frame_embed, self.head_embed, self.out_head,
+                                      self.head_layers, ptr("head.final_norm"))
+            return
+        self.layers = layers(shape, prefix)
+        self.struct = wpk_weights(ptr(prefix + "embed"), ptr(prefix + "final_norm"),
+                                  ptr(prefix + "lm_head") if not shape.tied_embedding else None, self.layers)
 
 
 class Engine:
@@ -307,6 +338,12 @@ class Engine:
                          self.dev_scratch.data_ptr(), self._stream())
         self.max_batch = max_batch
         self.batch = 0
+        # outputs per sequence: a token and its logits, or (two-stage) the
+        # frame's codes and their logits per codebook
+        if hasattr(shape, "backbone"):
+            self._tok_shape, self._logit_shape = (shape.n_codebooks,), (shape.n_codebooks, shape.codebook_vocab)
+        else:
+            self._tok_shape, self._logit_shape = (), (shape.vocab,)
 
     def _stream(self) -> int:
         return self.torch.cuda.current_stream().cuda_stream
@@ -316,8 +353,9 @@ class Engine:
         tok = torch.as_tensor(np.ascontiguousarray(tokens, dtype=np.int32)).cuda()
         B, T = tok.shape
         self.batch = B
-        first = torch.empty(B, dtype=torch.int32, device=tok.device)
-        logits = torch.empty((B, self.shape.vocab), dtype=torch.float32, device=tok.device) if want_logits else None
+        first = torch.empty((B,) + self._tok_shape, dtype=torch.int32, device=tok.device)
+        logits = (torch.empty((B,) + self._logit_shape, dtype=torch.float32, device=tok.device)
+                  if want_logits else None)
         wpk_prefill(self.h, tok.data_ptr(), B, T, first.data_ptr(), logits.data_ptr() if want_logits else 0,
                     self._stream())
         self._keep = tok
@@ -334,9 +372,9 @@ class Engine:
             self._keep_in = it
             itp = it.data_ptr()
         if out_tok is None:
-            out_tok = torch.empty(B, dtype=torch.int32, device=dev)
+            out_tok = torch.empty((B,) + self._tok_shape, dtype=torch.int32, device=dev)
         if want_logits and logits is None:
-            logits = torch.empty((B, self.shape.vocab), dtype=torch.float32, device=dev)
+            logits = torch.empty((B,) + self._logit_shape, dtype=torch.float32, device=dev)
         wpk_step(self.h, itp, out_tok.data_ptr(), logits.data_ptr() if logits is not None else 0, self._stream())
         return out_tok, logits
 

@@ -71,6 +71,10 @@ CODEBOOK_HEAD = ModelShape(n_layers=4, hidden=1024, n_heads=16, n_kv_heads=4, he
                            ffn=4096, vocab=2048, rms_eps=1e-5, rope_theta=500000.0,
                            tied_embedding=False)
 TWO_STAGE = TwoStageShape(backbone=LLAMA_1B, head=CODEBOOK_HEAD)
+# a small two-stage model for parity tests: the tiny backbone, a 2-layer head
+TINY_HEAD = ModelShape(n_layers=2, hidden=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=512, vocab=256,
+                       rms_eps=1e-5, rope_theta=10000.0, tied_embedding=False)
+TINY_TWO_STAGE = TwoStageShape(backbone=TINY, head=TINY_HEAD, n_codebooks=4, codebook_vocab=256)
 
 
 @dataclass(frozen=True)

@@ -309,3 +309,27 @@ def test_prefill_splits_o_and_down_along_k(lib):
             assert p <= gu and len(p) < 128
     finally:
         W.wpk_destroy(h)
+
+
+def test_two_stage_handle_host_side(lib):
+    s = synth.TINY_TWO_STAGE
+    h = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(16, 64))
+    try:
+        W.wpk_verify_graph(h)  # the backbone program
+        st, names = _ops(h)
+        # the backbone's output head is the projection into the head's width
+        bb = s.backbone
+        matrices = sum(np.prod(x) * 2 for n, x, k in synth.tensor_specs(bb) if k == "normal" and n != "embed")
+        assert st["weight_bytes"] == matrices + s.head.hidden * bb.hidden * 2
+        wb, kb, sb = W.wpk_workspace_size(h)
+        # every table is in the image: frame inputs, head inputs (K-1), output heads
+        K, V = s.n_codebooks, s.codebook_vocab
+        assert wb > (K * bb.hidden + (2 * K - 1) * s.head.hidden) * V * 2
+    finally:
+        W.wpk_destroy(h)
+    bad = W.model_cfg(s)
+    bad.n_codebooks = 17
+    with pytest.raises(W.WpkError):
+        W.wpk_build_graph(bad, W.plan_cfg(1, 64))
+    with pytest.raises(W.WpkError):
+        W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(1, 64, resident=1))
