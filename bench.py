@@ -60,6 +60,28 @@ def parse():
     return ap.parse_args()
 
 
+def profiled_traffic(B, mean_ctx):
+    """DRAM bytes per launch of the decode program from the committed ncu
+    summary, scaled by the KV bytes to this run's batch and context - or None
+    when the kernel sources changed since the capture."""
+    import hashlib
+    import re
+
+    p = os.path.join(ROOT, "profiles", "wpk_persistent_kernel_llama1b_b1.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    src = os.path.join(ROOT, "streaming_persistent_sm_b200", "csrc")
+    sha = hashlib.sha1(b"".join(open(os.path.join(src, f), "rb").read()
+                                for f in ("runtime.cu", "ptx.cuh", "wpk_internal.h"))).hexdigest()
+    m = {k: v for k, v in re.findall(r"^(\w+)(?:\([^)]*\))?: (\S+)$", txt, re.M)}
+    if m.get("source_sha1") != sha:
+        return None
+    kv = float(m["kv_bytes_per_token"])
+    base = float(m["traffic_bytes_per_launch"]) - float(m["traffic_batch"]) * float(m["traffic_context"]) * kv
+    return base + B * mean_ctx * kv
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -112,32 +134,53 @@ class ClockSampler:
 # ---------------------------------------------------------- CPU reference --
 def oracle_sample(wl, weights, n_steps: int = 2):
     """Time the float64 oracle on host cores: the workload's prefill and a few
-    decode steps for one sequence; tokens/s extrapolated to the whole job."""
-    import oracle
+    steps for one sequence; tokens/s extrapolated to the whole job."""
+    return oracle_job_sample(wl, weights, n_steps)
 
-    s = wl.model
-    dec = oracle.Decoder(s, weights)
-    prompts = synth.make_prompts(s.vocab, 1, wl.prompt_len, wl.prompt_seed)
-    cache = dec.new_cache(1, wl.prompt_len + n_steps + 1)
-    t0 = time.perf_counter()
-    lg = dec.prefill(cache, prompts)
-    t_prefill = time.perf_counter() - t0
-    tok = oracle.argmax_lowest(lg)
-    ts = []
-    for _ in range(n_steps):
-        t0 = time.perf_counter()
-        lg = dec.step(cache, tok)
-        ts.append(time.perf_counter() - t0)
-        tok = oracle.argmax_lowest(lg)
-    t_step = statistics.median(ts)
-    return t_prefill, t_step
+
+def codes_per_step(model):
+    """Tokens one sequence emits per step: one, or a frame of codebook codes."""
+    return model.n_codebooks if hasattr(model, "backbone") else 1
 
 
 def job_tokens(wl, decode_steps):
     """Tokens one bench step generates, and whether the prefill is part of it
     (decode-only workloads start from an already-prefilled prompt)."""
     with_prefill = not wl.name.startswith("llama1b_decode")
-    return wl.batch * ((1 if with_prefill else 0) + decode_steps), with_prefill
+    return wl.batch * codes_per_step(wl.model) * ((1 if with_prefill else 0) + decode_steps), with_prefill
+
+
+def oracle_job_sample(wl, weights, n_steps: int):
+    """One sequence through the float64 oracle: (prefill seconds, median step
+    seconds) - a decode step, or a two-stage frame."""
+    import oracle
+
+    s = wl.model
+    if hasattr(s, "backbone"):
+        ts = oracle.TwoStage(s, weights)
+        prompts = synth.make_prompts(s.backbone.vocab, 1, wl.prompt_len, wl.prompt_seed)
+        cache = ts.backbone.new_cache(1, wl.prompt_len + n_steps + 1)
+        t0 = time.perf_counter()
+        codes, _ = ts.prefill(cache, prompts)
+        t_prefill = time.perf_counter() - t0
+        times = []
+        for _ in range(n_steps):
+            t0 = time.perf_counter()
+            codes, _ = ts.frame(cache, codes)
+            times.append(time.perf_counter() - t0)
+        return t_prefill, statistics.median(times)
+    dec = oracle.Decoder(s, weights)
+    prompts = synth.make_prompts(s.vocab, 1, wl.prompt_len, wl.prompt_seed)
+    cache = dec.new_cache(1, wl.prompt_len + n_steps + 1)
+    t0 = time.perf_counter()
+    tok = oracle.argmax_lowest(dec.prefill(cache, prompts))
+    t_prefill = time.perf_counter() - t0
+    times = []
+    for _ in range(n_steps):
+        t0 = time.perf_counter()
+        tok = oracle.argmax_lowest(dec.step(cache, tok))
+        times.append(time.perf_counter() - t0)
+    return t_prefill, statistics.median(times)
 
 
 def run_reference(args):
@@ -148,23 +191,8 @@ def run_reference(args):
     decode_steps = wl.steps if args.decode_steps is None else args.decode_steps
     weights = synth.cached_weights(wl.model, seed=0)
     cores = os.cpu_count()
-    # warm-up + timed samples: one decode step each, prefill measured once
-    import oracle
-
-    s = wl.model
-    dec = oracle.Decoder(s, weights)
-    prompts = synth.make_prompts(s.vocab, 1, wl.prompt_len, wl.prompt_seed)
-    cache = dec.new_cache(1, wl.prompt_len + args.warmup + args.steps + 1)
-    t0 = time.perf_counter()
-    tok = oracle.argmax_lowest(dec.prefill(cache, prompts))
-    t_prefill = time.perf_counter() - t0
-    times = []
-    for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        tok = oracle.argmax_lowest(dec.step(cache, tok))
-        if i >= args.warmup:
-            times.append(time.perf_counter() - t0)
-    t_step = statistics.median(times)
+    # one prefill, then warm-up + timed steps (decode steps or frames)
+    t_prefill, t_step = oracle_job_sample(wl, weights, args.warmup + args.steps)
     tokens, with_prefill = job_tokens(wl, decode_steps)
     per_seq = (t_prefill if with_prefill else 0.0) + decode_steps * t_step
     value = tokens / (per_seq * wl.batch)  # the oracle runs the sequences one after another
@@ -230,6 +258,8 @@ def main():
     B, T = wl.batch, (wl.prompt_len if args.prompt_len is None else args.prompt_len)
     decode_steps = wl.steps if args.decode_steps is None else args.decode_steps
     tokens_per_step, with_prefill = job_tokens(wl, decode_steps)
+    two = hasattr(s, "backbone")
+    K = codes_per_step(s)
     ctx = T + max(decode_steps, 1)
     weights = synth.cached_weights(s, seed=0)
     mode = W.WPK_MEGAKERNEL if args.mode == "megakernel" else W.WPK_PER_OP_GRAPH
@@ -244,12 +274,14 @@ def main():
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))
     eng = W.Engine(s, weights, B, ctx, **plan)
     stats = eng.stats
-    prompts = synth.make_prompts(s.vocab, B, T, wl.prompt_seed + 17 * rank)
+    prompts = synth.make_prompts(s.backbone.vocab if two else s.vocab, B, T, wl.prompt_seed + 17 * rank)
     prompts_dev = torch.as_tensor(prompts, device=dev)
-    out_dev = torch.empty((max(decode_steps, 1) + 1, B), dtype=torch.int32, device=dev)
+    out_dev = torch.empty((max(decode_steps, 1) + 1, B) + ((K,) if two else ()), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
     launches_per_decode = stats["n_regions"] if mode == W.WPK_MEGAKERNEL else stats["n_ops"]
+    if two:
+        launches_per_decode += K  # a frame: the backbone step, then K head steps
     prefill_tensor_cores = True
     try:
         W.wpk_select_program(eng.h, B, T)
@@ -328,12 +360,20 @@ def main():
     # roofline of the dominant kernel (the persistent decode program): bytes per
     # launch over the launch durations measured above
     hbm_peak, tc_peak, peak_kind = measured_peaks()
-    kvb = KV_BYTES_PER_TOKEN(s)
     kernel_name = "wpk_persistent_kernel" if mode == W.WPK_MEGAKERNEL else "wpk_per_op_kernel"
     decode_summary = None
     if decode_steps > 0:
         dec_ctx = [T + i for i in range(decode_steps)]  # tokens already cached at each decode step
-        algo_dec = [algorithmic_bytes_per_step(s, stats["weight_bytes"], B, c) for c in dec_ctx]
+        if two:  # a frame: backbone step + K head steps (head weights, output head k, head KV)
+            hs = s.head
+            head_w = 2 * hs.n_layers * (hs.hidden * (hs.n_heads + 2 * hs.n_kv_heads) * hs.head_dim
+                                        + hs.n_heads * hs.head_dim * hs.hidden + 3 * hs.ffn * hs.hidden)
+            head_bytes = sum(head_w + 2 * s.codebook_vocab * hs.hidden + B * (k + 1) * KV_BYTES_PER_TOKEN(hs)
+                             for k in range(K))
+            algo_dec = [algorithmic_bytes_per_step(s.backbone, stats["weight_bytes"], B, c) + head_bytes
+                        for c in dec_ctx]
+        else:
+            algo_dec = [algorithmic_bytes_per_step(s, stats["weight_bytes"], B, c) for c in dec_ctx]
         # the dominant kernel is the decode program (one launch per step): its
         # algorithmic bytes per launch over the launch times measured above
         launch_bytes = sum(algo_dec)
@@ -342,8 +382,12 @@ def main():
         dec_gbs = statistics.mean(algo_dec) / (statistics.median(dec_us) / 1e6) / 1e9
         decode_summary = {"median": statistics.median(dec_us), "p95": float(np.percentile(dec_us, 95)),
                           "achieved_gbs": dec_gbs, "frac_of_8tbs": dec_gbs / 8000.0}
+        # DRAM traffic per launch from the committed capture (plain decoder, one
+        # launch per step; None for other programs or after a kernel change)
+        traffic = (profiled_traffic(B, statistics.mean(dec_ctx)) if not two and mode == W.WPK_MEGAKERNEL
+                   and stats["n_regions"] == 1 and not args.layers else None)
         roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved_gbs / hbm_peak, "traffic": None,
+                    "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel_name}
     else:
         # prefill only: the prefill program dominates and is a dense contraction;
@@ -367,7 +411,9 @@ def main():
                    "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
                    "prefill": "tensor-core prefill program" if prefill_tensor_cores else "token by token",
                    "workers": stats["n_workers"],
-                   "l2": "inputs larger than L2: %.2f GB of weights streamed per step" % (stats["weight_bytes"] / 1e9)},
+                   "l2": "inputs larger than L2: %.2f GB of weights streamed per step" % (stats["weight_bytes"] / 1e9),
+                   **({"codes_per_frame": K, "tokens": "codebook codes (a frame per sequence per step)"}
+                      if two else {})},
         "decode_step_us": decode_summary,
         "ttft_ms": statistics.median(pre_ms) if pre_ms else None,
         "roofline": roofline,
@@ -378,7 +424,7 @@ def main():
     # end to end through the C ABI with host buffers: pinned prompt -> device,
     # prefill + decode, tokens -> pinned host, all inside the timed region
     host_prompt = torch.from_numpy(prompts).pin_memory()
-    host_out = torch.empty((decode_steps + 1, B), dtype=torch.int32).pin_memory()
+    host_out = torch.empty(tuple(out_dev[: decode_steps + 1].shape), dtype=torch.int32).pin_memory()
     torch.cuda.synchronize()
     e2e_runs = max(1, min(args.steps, 3))
     t0 = time.perf_counter()
@@ -391,16 +437,17 @@ def main():
     e2e_s = (time.perf_counter() - t0) / e2e_runs
     line["e2e"] = {"value": world * tokens_per_step / e2e_s, "unit": "tokens/s",
                    "h2d_bytes_per_step": int(host_prompt.numel() * 4),
-                   "d2h_bytes_per_step": int((decode_steps + 1) * B * 4)}
+                   "d2h_bytes_per_step": int(host_out.numel() * 4)}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_pre, t_step = oracle_sample(wl, weights, n_steps=2)
         per_seq = (t_pre if with_prefill else 0.0) + decode_steps * t_step
         cpu_value = tokens_per_step / (per_seq * B)
+        what = "frames" if two else "decode steps"
         line["cpu_baseline"] = {
             "value": cpu_value, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"float64 NumPy oracle, one sequence: {T}-token prefill ({t_pre:.1f} s) + 2 decode steps "
-                      f"(median {t_step:.2f} s); extrapolated to {decode_steps} steps and {B} sequences"}
+            "sample": f"float64 NumPy oracle, one sequence: {T}-token prefill ({t_pre:.1f} s) + 2 {what} "
+                      f"(median {t_step:.2f} s); extrapolated to {decode_steps} {what} and {B} sequences"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     eng.close()
