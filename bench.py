@@ -57,6 +57,7 @@ def parse():
     ap.add_argument("--prefill", default="auto", choices=["auto", "mma", "tokenwise"])
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--resident", action="store_true", help="one resident grid serves every decode step")
+    ap.add_argument("--split-pages", type=int, default=0)
     return ap.parse_args()
 
 
@@ -268,7 +269,8 @@ def main():
                 schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE,
                 prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
                          "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill],
-                resident=1 if args.resident else 0)
+                resident=1 if args.resident else 0,
+                split_pages=args.split_pages)
     if args.regions:
         cuts = [int(x) for x in args.regions.split(",")]
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))

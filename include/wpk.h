@@ -103,7 +103,8 @@ typedef struct wpk_plan_cfg {
   int slot_bytes;       /* staging slot per worker, used as a ring of 16 KB
                            chunk stages (0 = 12 stages, 192 KB, or what fits) */
   int tile_bytes;       /* minimum weight bytes per tile; tiles are sized to give
-                           each worker about one tile per op (0 = 32768)       */
+                           each worker about one tile per op (0 = 32768, or
+                           65536 for tensor-core decode tiles)                 */
   int split_pages;      /* KV pages per attention tile (split); 0 = chosen so that
                            a step has about two attention tiles per worker     */
   int lookahead;        /* tiles a worker may claim and stage ahead of the one

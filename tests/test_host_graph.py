@@ -227,7 +227,7 @@ def test_batched_decode_k_split_edges(lib):
     # tile = 64 h features = one 64-column chunk), each O tile only for the
     # attention tiles of the heads in its K range
     s = synth.ModelShape(n_layers=1, hidden=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=2048, vocab=512)
-    h = _graph(s, max_batch=16, max_context=64, n_workers=64)
+    h = _graph(s, max_batch=16, max_context=64, n_workers=64, tile_bytes=16384)
     try:
         W.wpk_verify_graph(h)
         st, names = _ops(h)
