@@ -362,7 +362,9 @@ def main():
     # roofline of the dominant kernel (the persistent decode program): bytes per
     # launch over the launch durations measured above
     hbm_peak, tc_peak, peak_kind = measured_peaks()
-    kernel_name = "wpk_persistent_kernel" if mode == W.WPK_MEGAKERNEL else "wpk_per_op_kernel"
+    # the decode program's kernel: tensor-core decode tiles (op codes from 16 on) run in their own kernel
+    mma_decode = bool((W.wpk_get_tile_ops(eng.h, stats["n_tiles"]) >= W.OP_NAMES.index("b_qkv")).any())
+    kernel_name = ("wpk_persistent" if mode == W.WPK_MEGAKERNEL else "wpk_per_op") + ("_mma" if mma_decode else "") + "_kernel"
     decode_summary = None
     if decode_steps > 0:
         dec_ctx = [T + i for i in range(decode_steps)]  # tokens already cached at each decode step

@@ -19,8 +19,8 @@
 
 namespace wpk {
 size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes);
-const void* persistent_kernel_ptr();
-const void* per_op_kernel_ptr();
+const void* persistent_kernel_ptr(bool mma);  // decode on tensor cores (mma) or CUDA cores
+const void* per_op_kernel_ptr(bool mma);
 const void* prefill_kernel_ptr();
 const void* prefill_op_kernel_ptr();
 }  // namespace wpk
@@ -313,7 +313,7 @@ int launch_megakernel(wpk_handle* h, const KParams& base, cudaStream_t s) {
     P.t_end = g.region_begin[r + 1];
     P.region = r;
     void* args[] = {&P};
-    CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
+    CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(h->n_workers), dim3(kCtaThreads), args,
                                             h->smem, s));
   }
   return WPK_OK;
@@ -334,7 +334,7 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
     P.per_op = 1;
     if (!P.dec_mma) P.n_stages = g.plan.per_op_slot / kStageBytes;
     void* args[] = {&P};
-    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
+    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(og.end - og.begin), dim3(kCtaThreads), args,
                                      h->smem_per_op, h->capture_stream);
     if (e != cudaSuccess) {
       cudaGraph_t junk = nullptr;
@@ -382,7 +382,7 @@ int res_launch(wpk_handle* h) {
   P.t_end = (uint32_t)g.tiles.size();
   P.region = 0;
   void* args[] = {&P};
-  CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
+  CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(h->n_workers), dim3(kCtaThreads), args,
                                           h->smem, h->res_stream));
   h->res_live = true;
   h->res_epoch = 0;
@@ -621,9 +621,9 @@ static int setup_device(wpk_handle* h) {
     h->smem_prefill = worker_smem_bytes(h->prefill_stages, 3 * kMmaChunkBytes, p.act_bytes);
   }
   const size_t smem_max = h->smem;
-  CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)smem_max));
-  CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+  CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)h->smem_per_op));
   if (h->smem_prefill) {
     CUDA_TRY(h, cudaFuncSetAttribute(prefill_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -636,7 +636,7 @@ static int setup_device(wpk_handle* h) {
     if (per_sm_p < 1) return fail(h, WPK_ERR_UNSUPPORTED, "the prefill worker does not fit an SM");
   }
   int per_sm = 0;
-  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(), kCtaThreads, smem_max));
+  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), kCtaThreads, smem_max));
   {
     // tcgen05.alloc waits until the SM has free TMEM columns: workers that
     // share an SM must fit its 512 columns together

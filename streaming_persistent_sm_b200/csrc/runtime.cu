@@ -1587,6 +1587,13 @@ __device__ bool wait_counter(const KParams& P, const Tile& T, uint32_t tile, uin
 // ---------------------------------------------------------------------------
 // The worker: producer warp (warp 8) + consumer warps (0..7).
 // ---------------------------------------------------------------------------
+// Program kinds: each kernel carries only the tile bodies its program uses, so
+// that the compiler sizes registers for that program alone.
+constexpr int kProgGemv = 0;     // decode on CUDA cores (GEMV tiles)
+constexpr int kProgMma = 1;      // batched decode on tensor cores
+constexpr int kProgPrefill = 2;  // prefill (tensor-core tiles, causal attention, GEMV LM head)
+
+template <int kProg>
 __device__ void worker(const KParams& P, uint8_t* smem_raw) {
   // the 128-byte-swizzled tensor-core operands need 1024-byte aligned stages
   if (P.uses_tmem && (smem_u32(smem_raw) & 1023u)) {
@@ -1794,24 +1801,53 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
       cbar();
       bool ok = !s_fail;
       if (ok) {
+        bool known = true;  // the op belongs to this kernel's program
         switch (T.op) {
-          case OP_EMBED: ok = P.dec_mma ? body_embed_mma(P, T, reinterpret_cast<int*>(S.act)) : body_embed(P); break;
-          case OP_ATTN: ok = body_attn(P, T, S, cur, n_chunks, &s_abort); break;
+          case OP_EMBED:
+            if constexpr (kProg == kProgMma)
+              ok = body_embed_mma(P, T, reinterpret_cast<int*>(S.act));
+            else
+              ok = body_embed(P);
+            break;
+          case OP_ATTN:
+            if constexpr (kProg != kProgPrefill) ok = body_attn(P, T, S, cur, n_chunks, &s_abort);
+            else known = false;
+            break;
           case OP_FINAL: ok = body_final(P, e.epoch); break;
-          case OP_PEMBED: ok = body_pembed(P, T); break;
-          case OP_GATHER: ok = body_gather(P); break;
-          case OP_NORM: ok = body_norm(P, T); break;
-          case OP_PATTN: ok = body_pattn(P, T, S, cur, n_chunks, &s_abort, t); break;
+          case OP_PEMBED:
+          case OP_GATHER:
+          case OP_NORM:
+          case OP_PATTN:
           case OP_MQKV:
           case OP_MO:
           case OP_MGU:
           case OP_MDOWN:
+            if constexpr (kProg == kProgPrefill) {
+              if (T.op == OP_PEMBED) ok = body_pembed(P, T);
+              else if (T.op == OP_GATHER) ok = body_gather(P);
+              else if (T.op == OP_NORM) ok = body_norm(P, T);
+              else if (T.op == OP_PATTN) ok = body_pattn(P, T, S, cur, n_chunks, &s_abort, t);
+              else ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t);
+            } else {
+              known = false;
+            }
+            break;
           case OP_BQKV:
           case OP_BO:
           case OP_BGU:
           case OP_BDOWN:
-          case OP_BLM: ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t); break;
-          default: ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort); break;
+          case OP_BLM:
+            if constexpr (kProg == kProgMma) ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t);
+            else known = false;
+            break;
+          default:  // GEMV tiles (decode ops, and the prefill's LM head)
+            if constexpr (kProg != kProgMma) ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort);
+            else known = false;
+            break;
+        }
+        if (!known) {
+          if (threadIdx.x == 0) record_error(P, WPK_ERR_UNSUPPORTED, t, kNoCounter, T.op, (uint32_t)kProg);
+          ok = false;
         }
         // attention tiles use the activation buffer as scratch; the gather
         // rewrites the LM head's input
@@ -1886,28 +1922,38 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
 
 }  // namespace
 
-// The persistent worker grid (one cooperative launch per region per step).
+// Decode on CUDA cores: the persistent worker grid (one cooperative launch per
+// region per step, or one for many steps when resident).
 __global__ void __launch_bounds__(kCtaThreads, 1) wpk_persistent_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  worker(P, smem_raw);
+  worker<kProgGemv>(P, smem_raw);
 }
 
 // Per-op launch: one CTA per tile of one op group; stream order replaces the
 // counters.  Used for the CUDA-Graph comparator.
 __global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  worker(P, smem_raw);
+  worker<kProgGemv>(P, smem_raw);
 }
 
-// The prefill program runs the same worker under its own names, so launch
-// lists and profiles separate it from the decode program.
+// Batched decode on tensor cores: the same two launch forms.
+__global__ void __launch_bounds__(kCtaThreads, 1) wpk_persistent_mma_kernel(const KParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  worker<kProgMma>(P, smem_raw);
+}
+__global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_mma_kernel(const KParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  worker<kProgMma>(P, smem_raw);
+}
+
+// The prefill program.
 __global__ void __launch_bounds__(kCtaThreads, 1) wpk_prefill_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  worker(P, smem_raw);
+  worker<kProgPrefill>(P, smem_raw);
 }
 __global__ void __launch_bounds__(kCtaThreads, 1) wpk_prefill_op_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  worker(P, smem_raw);
+  worker<kProgPrefill>(P, smem_raw);
 }
 
 size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes) {
@@ -1915,8 +1961,13 @@ size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes) {
          (2 * kMaxStages + 2 * kMaxQueue + 1 + 2 * kSigQueue) * 8 + kSigQueue * sizeof(uint2);
 }
 
-const void* persistent_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_persistent_kernel); }
-const void* per_op_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_per_op_kernel); }
+const void* persistent_kernel_ptr(bool mma) {
+  return mma ? reinterpret_cast<const void*>(&wpk_persistent_mma_kernel)
+             : reinterpret_cast<const void*>(&wpk_persistent_kernel);
+}
+const void* per_op_kernel_ptr(bool mma) {
+  return mma ? reinterpret_cast<const void*>(&wpk_per_op_mma_kernel) : reinterpret_cast<const void*>(&wpk_per_op_kernel);
+}
 const void* prefill_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_prefill_kernel); }
 const void* prefill_op_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_prefill_op_kernel); }
 
