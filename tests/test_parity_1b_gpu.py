@@ -60,3 +60,43 @@ def test_llama1b_batched_sampled_rows(weights, dec, B, decode):
         run_teacher_forced(eng, dec, prompts, steps=3, max_context=ctx, rows=[0, B // 2, B - 1])
     finally:
         eng.close()
+
+
+def test_llama1b_prefill_b32_sampled_rows(weights, dec):
+    # the C4 shape at its largest batch: 32 prompts of 496 tokens (15872 rows)
+    wl = synth.WORKLOADS["llama1b_prefill_b32"]
+    B = wl.batch
+    eng = W.Engine(S, weights, B, wl.prompt_len + 4)
+    try:
+        prompts = synth.make_prompts(S.vocab, B, wl.prompt_len, wl.prompt_seed)
+        run_teacher_forced(eng, dec, prompts, steps=1, max_context=wl.prompt_len + 4, rows=[0, B // 2, B - 1])
+    finally:
+        eng.close()
+
+
+def test_two_stage_1b_shape_b32_sampled_rows():
+    # the C5 shape: the 1B backbone, a 4-layer h1024 head, 16 codebooks of 2048,
+    # batch 32 (tensor-core decode for both), 200-token prompts, two frames
+    from tests.test_two_stage_gpu import _check_frame_shape
+
+    s = synth.TWO_STAGE
+    w = synth.cached_weights(s, seed=0)
+    ora = oracle.TwoStage(s, w)
+    wl = synth.WORKLOADS["two_stage_b32"]
+    B, T, rows = wl.batch, wl.prompt_len, [0, 16, 31]
+    eng = W.Engine(s, w, B, T + 4)
+    try:
+        prompts = synth.make_prompts(s.backbone.vocab, B, T, wl.prompt_seed)
+        codes, lg = eng.prefill(prompts, want_logits=True)
+        codes, lg = codes.cpu().numpy(), lg.cpu().numpy()
+        cache = ora.backbone.new_cache(len(rows), T + 4)
+        _, ref = ora.prefill(cache, prompts[rows], forced=codes[rows])
+        _check_frame_shape(s, codes[rows], lg[rows], ref, "prefill")
+        for f in range(2):
+            prev = codes
+            out, lg = eng.step(want_logits=True)
+            codes, lg = out.cpu().numpy(), lg.cpu().numpy()
+            _, ref = ora.frame(cache, prev[rows], forced=codes[rows])
+            _check_frame_shape(s, codes[rows], lg[rows], ref, f"frame {f}")
+    finally:
+        eng.close()

@@ -28,9 +28,13 @@ def ora(weights):
     return oracle.TwoStage(S, weights)
 
 
-def _check_frame(gpu_codes, gpu_logits, ref_logits, where):
-    for k in range(S.n_codebooks):
+def _check_frame_shape(shape, gpu_codes, gpu_logits, ref_logits, where):
+    for k in range(shape.n_codebooks):
         check_logits(gpu_logits[:, k], ref_logits[:, k], gpu_codes[:, k], f"{where} codebook {k}")
+
+
+def _check_frame(gpu_codes, gpu_logits, ref_logits, where):
+    _check_frame_shape(S, gpu_codes, gpu_logits, ref_logits, where)
 
 
 @pytest.mark.parametrize("B,plan", [(1, {}), (3, {}), (16, {}), (12, dict(schedule=W.WPK_SCHED_STATIC)),
