@@ -130,8 +130,8 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
       p->dec_stage_bytes = kMmaChunkBytes + 2 * p->dec_n * 128;
       // attention scratch: queries, one page of scores, the combine's (m, l) pairs
       const int max_pages = (in.max_context + p->page_tokens - 1) / p->page_tokens;
-      const int need =
-          std::max(kMaxGroup * (m.head_dim + kAttnPages * p->page_tokens) * 4, max_pages * kMaxGroup * 2 * 4);
+      const int need = std::max((kMaxGroup * kHeadDim + 2 * kHeadDim + kWarps * (2 + kHeadDim)) * 4,
+                                max_pages * kMaxGroup * 2 * 4);
       p->dec_act_bytes = std::max(16384, (need + 1023) / 1024 * 1024);
       const int room = kMaxSmem - fixed - 4096 - p->dec_act_bytes;  // 4 KB: the kernel's static shared memory
       int want = in.slot_bytes ? in.slot_bytes / kStageBytes : 12;

@@ -723,177 +723,150 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
                           volatile int* abort) {
   if (T.a0 >= active_batch(P)) return true;
   __shared__ int s_last;
-  __shared__ float s_m[kMaxGroup], s_l[kMaxGroup], s_sc[kMaxGroup];
+  __shared__ uint32_t s_page_rel[kMaxStages];  // warps done with a stage, this tile
   const AttnSpan s = attn_span(P, T);
   const int hd = P.head_dim, grp = P.group, page = P.page_tokens;
-  const int nq = grp * hd;  // (head, dim) pairs: thread i owns pairs i and i + 256
+  const int nq = grp * hd;
   float* part = P.part + ((((size_t)s.b * P.n_kv + s.g) * P.n_splits + s.j) * grp) * (2 + hd);
-  float* q_s = Sh.act;                    // [grp][hd]
-  float* p_s = Sh.act + kMaxGroup * hd;   // [grp][kAttnPages * page]
+  float* q_s = Sh.act;                          // [grp][hd]
+  float* kv_cur = Sh.act + kMaxGroup * hd;      // [2][hd]: the current token's k and v
+  float* st_s = kv_cur + 2 * kHeadDim;          // [kWarps][2 + hd]: each warp's (m, l, o)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp w attends with query head w % grp over every parts-th 32-token block
+  const int parts = kWarps / grp;
+  const int head = warp % grp, prt = warp / grp;
   const float scale = 1.0f / sqrtf((float)hd);
-  float o[2] = {0.f, 0.f};
-  if (threadIdx.x < kMaxGroup) {
-    s_m[threadIdx.x] = -INFINITY;
-    s_l[threadIdx.x] = 0.f;
+  const bool has_cur = s.pos >= s.t0 && s.pos < s.t1;
+  for (int i = threadIdx.x; i < nq; i += kThreads)
+    q_s[i] = P.dec_mma ? __ldcg(P.acc + (size_t)(s.g * nq + i) * P.mma_n + s.b)
+                       : __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * nq + i);
+  // the current token's k and v were produced this step, after its page was
+  // copied: read them directly (tensor-core decode: round the fp32 sums to the
+  // cache's bf16 here, store them and clear the sums)
+  if (has_cur && threadIdx.x < 2 * hd) {
+    const int sel = threadIdx.x / hd, d = threadIdx.x % hd;
+    const int blk = P.block_table[s.b * P.max_blocks + s.pos / page];
+    uint16_t* dst = P.kv + kv_index(P, T.layer, blk, sel, s.g, s.pos % page) + d;
+    uint16_t v;
+    if (P.dec_mma) {
+      float* a = P.acc + (size_t)(P.q_rows + sel * P.kv_rows + s.g * hd + d) * P.mma_n + s.b;
+      v = f2bf(__ldcg(a));
+      *a = 0.f;
+      *dst = v;
+    } else {
+      v = __ldcg(dst);
+    }
+    kv_cur[sel * kHeadDim + d] = bf2f(v);
+  }
+  if (threadIdx.x < kMaxStages) s_page_rel[threadIdx.x] = 0;
+  cbar();
+  const float* qh = q_s + head * hd;
+  float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;  // this warp's state; lane holds dims 2 lane, 2 lane + 1
+  bool ok = true;
+  for (int k = 0; k < n_chunks; ++k) {  // page k of the split, one ring stage each
+    const uint32_t c = cur.c + k;
+    const int st = c % P.n_stages;
+    if (ok && !wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu)) ok = false;
+    if (ok) {
+      if (P.trace && threadIdx.x == 0 && k + 1 == n_chunks) s_t_data = globaltimer();
+      const uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
+      const int p0 = (s.t0 / page + k) * page;
+      const int n = min(page, s.t1 - p0);
+      const int blk0 = (p0 - s.t0) / 32;
+      for (int b = 0; b * 32 < n; ++b) {
+        if ((blk0 + b) % parts != prt) continue;
+        const int t = b * 32 + lane;
+        const bool valid = t < n && p0 + t != s.pos;
+        float sc = -INFINITY;
+        if (valid) {
+          const uint4* kr = reinterpret_cast<const uint4*>(stage + (size_t)t * hd * 2);
+          float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+          for (int u = 0; u < kHeadDim / 8; ++u) {
+            const int uu = (u + lane) & (kHeadDim / 8 - 1);  // rotated: neighbouring lanes, other banks
+            float kf[8];
+            unpack8(kr[uu], kf);
+            const float4 qa = *reinterpret_cast<const float4*>(qh + 8 * uu);
+            const float4 qb = *reinterpret_cast<const float4*>(qh + 8 * uu + 4);
+            a0 = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], a0))));
+            a1 = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], a1))));
+          }
+          sc = (a0 + a1) * scale;
+        }
+        const float m_new = fmaxf(m, warp_max(sc));
+        if (m_new == -INFINITY) continue;  // no valid token yet (warp-uniform)
+        const float corr = expf(m - m_new);
+        const float pp = valid ? expf(sc - m_new) : 0.f;
+        l = l * corr + warp_sum(pp);
+        o0 *= corr;
+        o1 *= corr;
+        const uint32_t* vrow = reinterpret_cast<const uint32_t*>(stage + (size_t)page * hd * 2 + (size_t)b * 32 * hd * 2) + lane;
+        const int cnt = min(32, n - b * 32);
+        // the staged copy of the current token's row is stale (it was copied
+        // before this step wrote it): read zeros there, never its bytes
+        const int stale = s.pos - p0 - b * 32;
+        for (int j = 0; j < cnt; ++j) {
+          const float pj = __shfl_sync(0xffffffffu, pp, j);
+          const uint32_t vv = (j == stale) ? 0u : vrow[(size_t)j * (hd / 2)];
+          o0 = fmaf(pj, __uint_as_float(vv << 16), o0);
+          o1 = fmaf(pj, __uint_as_float(vv & 0xFFFF0000u), o1);
+        }
+        m = m_new;
+      }
+    }
+    // the last warp to finish with the page hands the stage back
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t r = atomicAdd(&s_page_rel[st], 1u) + 1u;
+      if (r == (uint32_t)kWarps * (uint32_t)(k / P.n_stages + 1)) mbar_arrive(&Sh.empty[st]);
+    }
+  }
+  cur.c += n_chunks;
+  if (!cbar_and(ok)) return false;
+  if (has_cur && prt == 0) {  // the current token, once per head
+    float d = qh[2 * lane] * kv_cur[2 * lane] + qh[2 * lane + 1] * kv_cur[2 * lane + 1];
+    const float sc = warp_sum(d) * scale;
+    const float m_new = fmaxf(m, sc);
+    const float corr = expf(m - m_new), pp = expf(sc - m_new);
+    l = l * corr + pp;
+    o0 = o0 * corr + pp * kv_cur[kHeadDim + 2 * lane];
+    o1 = o1 * corr + pp * kv_cur[kHeadDim + 2 * lane + 1];
+    m = m_new;
+  }
+  float* mine = st_s + warp * (2 + kHeadDim);
+  mine[2 + 2 * lane] = o0;
+  mine[3 + 2 * lane] = o1;
+  if (lane == 0) {
+    mine[0] = m;
+    mine[1] = l;
   }
   cbar();
-  // up to G pages (one ring stage each) are computed per round
-  const int G = min(kAttnPages, P.n_stages);
-  const int span = G * page;
-  auto stage_of = [&](int j) { return Sh.ring + (size_t)((cur.c + j) % P.n_stages) * P.stage_bytes; };
-  for (int k0 = 0; k0 < n_chunks; k0 += G) {
-    const int gn = min(G, n_chunks - k0);
-    bool ok = true;
-    for (int j = 0; j < gn && ok; ++j) {
-      const uint32_t c = cur.c + j;
-      ok = wait_phase(P, &Sh.full[c % P.n_stages], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu);
-    }
-    if (!cbar_and(ok)) return false;
-    if (P.trace && threadIdx.x == 0 && k0 + gn == n_chunks) s_t_data = globaltimer();
-    const int p0 = (s.t0 / page + k0) * page;  // first token of the round
-    const int n = min(gn * page, s.t1 - p0);   // tokens of the round
-    // the current token's row was written this step, after the copy was issued
-    if (s.pos >= p0 && s.pos < p0 + n) {
-      uint8_t* stage = stage_of((s.pos - p0) / page);
-      uint16_t* Ks = reinterpret_cast<uint16_t*>(stage);
-      uint16_t* Vs = reinterpret_cast<uint16_t*>(stage + (size_t)page * hd * 2);
-      const int row = (s.pos - p0) % page;
-      const int blk = P.block_table[s.b * P.max_blocks + s.pos / page];
-      if (P.dec_mma) {
-        for (int i = threadIdx.x; i < 2 * hd; i += kThreads) {
-          const int sel = i / hd, d = i % hd;
-          float* a = P.acc + (size_t)(P.q_rows + sel * P.kv_rows + s.g * hd + d) * P.mma_n + s.b;
-          const uint16_t v = f2bf(__ldcg(a));
-          *a = 0.f;
-          P.kv[kv_index(P, T.layer, blk, sel, s.g, s.pos % page) + d] = v;
-          (sel ? Vs : Ks)[(size_t)row * hd + d] = v;
-        }
-      } else {
-        const int lanes = hd * 2 / 16;
-        if (threadIdx.x < 2 * lanes) {
-          const int sel = threadIdx.x / lanes, piece = threadIdx.x % lanes;
-          const uint4* src = reinterpret_cast<const uint4*>(
-              P.kv + kv_index(P, T.layer, blk, sel, s.g, s.pos % page));
-          uint8_t* dst = reinterpret_cast<uint8_t*>(sel ? Vs : Ks) + (size_t)row * hd * 2;
-          reinterpret_cast<uint4*>(dst)[piece] = __ldcg(src + piece);
-        }
+  // merge the parts of each head; one split: the result directly, else the
+  // split's partial (m, l, o) for the combine
+  for (int i = threadIdx.x; i < nq; i += kThreads) {
+    const int hh = i / hd, d = i % hd;
+    float M = -INFINITY;
+    for (int q = 0; q < parts; ++q) M = fmaxf(M, st_s[(q * grp + hh) * (2 + kHeadDim)]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY)
+      for (int q = 0; q < parts; ++q) {
+        const float* w = st_s + (q * grp + hh) * (2 + kHeadDim);
+        const float f = expf(w[0] - M);
+        L = fmaf(w[1], f, L);
+        O = fmaf(w[2 + d], f, O);
       }
-    }
-    if (k0 == 0)
-      for (int i = threadIdx.x; i < nq; i += kThreads)
-        q_s[i] = P.dec_mma ? __ldcg(P.acc + (size_t)(s.g * nq + i) * P.mma_n + s.b)
-                           : __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * nq + i);
-    cbar();
-    // scores.  Few tokens: one (head, token) pair per thread.  Otherwise one
-    // token per thread against every head of the group (one read of the K
-    // row).  Either way the row's units are visited in a rotated order so that
-    // neighbouring threads hit different banks.
-    if (grp * n <= kThreads) {
-      if (threadIdx.x < grp * n) {
-        const int hh = threadIdx.x / n, tt = threadIdx.x % n, t = tt % page;
-        const uint4* kr = reinterpret_cast<const uint4*>(stage_of(tt / page) + (size_t)t * hd * 2);
-        const float* qr = q_s + hh * kHeadDim;
-        float acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < kHeadDim / 8; ++u) {
-          const int uu = (u + t) & (kHeadDim / 8 - 1);
-          float kf[8];
-          unpack8(kr[uu], kf);
-          const float4 qa = *reinterpret_cast<const float4*>(qr + 8 * uu);
-          const float4 qb = *reinterpret_cast<const float4*>(qr + 8 * uu + 4);
-          acc = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], acc))));
-          acc = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], acc))));
-        }
-        p_s[hh * span + tt] = acc * scale;
-      }
-    } else
-    for (int tt = threadIdx.x; tt < n; tt += kThreads) {
-      const int t = tt % page;
-      const uint4* kr = reinterpret_cast<const uint4*>(stage_of(tt / page) + (size_t)t * hd * 2);
-      float acc[kMaxGroup];
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) acc[hh] = 0.f;
-#pragma unroll
-      for (int u = 0; u < kHeadDim / 8; ++u) {
-        const int uu = (u + t) & (kHeadDim / 8 - 1);
-        float kf[8];
-        unpack8(kr[uu], kf);
-#pragma unroll
-        for (int hh = 0; hh < kMaxGroup; ++hh) {
-          if (hh >= grp) break;
-          const float4 qa = *reinterpret_cast<const float4*>(q_s + hh * kHeadDim + 8 * uu);
-          const float4 qb = *reinterpret_cast<const float4*>(q_s + hh * kHeadDim + 8 * uu + 4);
-          acc[hh] = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], acc[hh]))));
-          acc[hh] = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], acc[hh]))));
-        }
-      }
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh)
-        if (hh < grp) p_s[hh * span + tt] = acc[hh] * scale;
-    }
-    cbar();
-    if (warp < grp) {  // running max and sum of head `warp`
-      float mx = -INFINITY;
-      for (int tt = lane; tt < n; tt += 32) mx = fmaxf(mx, p_s[warp * span + tt]);
-      mx = warp_max(mx);
-      const float m_old = s_m[warp], m_new = fmaxf(m_old, mx);
-      float l = 0.f;
-      for (int tt = lane; tt < n; tt += 32) {
-        const float e = expf(p_s[warp * span + tt] - m_new);
-        p_s[warp * span + tt] = e;
-        l += e;
-      }
-      l = warp_sum(l);
-      if (lane == 0) {
-        const float sc = expf(m_old - m_new);
-        s_sc[warp] = sc;
-        s_l[warp] = s_l[warp] * sc + l;
-        s_m[warp] = m_new;
-      }
-    }
-    cbar();
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int i = threadIdx.x + r * kThreads;
-      if (i < nq) {
-        const int hh = i / hd, d = i % hd;
-        float a = 0.f;
-        for (int j = 0; j < gn; ++j) {
-          const int tn = min(page, n - j * page);
-          const uint16_t* Vs = reinterpret_cast<const uint16_t*>(stage_of(j) + (size_t)page * hd * 2);
-          const float* pr = p_s + hh * span + j * page;
-          for (int t = 0; t < tn; ++t) a = fmaf(pr[t], bf2f(Vs[(size_t)t * hd + d]), a);
-        }
-        o[r] = o[r] * s_sc[hh] + a;
-      }
-    }
-    cbar();
-    if (threadIdx.x == 0)
-      for (int j = 0; j < gn; ++j) mbar_arrive(&Sh.empty[(cur.c + j) % P.n_stages]);
-    cur.c += gn;
-  }
-  if (P.n_splits == 1) {  // the only split: the result directly
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int i = threadIdx.x + r * kThreads;
-      if (i < nq) attn_result(P, s.b, s.g * nq + i, o[r] / s_l[i / hd]);
-    }
-    return true;
-  }
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int i = threadIdx.x + r * kThreads;
-    if (i < nq) {
-      const int hh = i / hd, d = i % hd;
+    if (P.n_splits == 1) {
+      attn_result(P, s.b, s.g * nq + i, O / L);
+    } else {
       float* pr = part + (size_t)hh * (2 + hd);
-      pr[2 + d] = o[r];
+      pr[2 + d] = O;
       if (d == 0) {
-        pr[0] = s_m[hh];  // -inf with l = 0 for a split past the current position
-        pr[1] = s_l[hh];
+        pr[0] = M;  // -inf with l = 0 for a split past the current position
+        pr[1] = L;
       }
     }
   }
+  if (P.n_splits == 1) return true;
   cbar();
   uint32_t* arr = P.arrive + (size_t)s.b * P.n_kv + s.g;
   if (threadIdx.x == 0) {

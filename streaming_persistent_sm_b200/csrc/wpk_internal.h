@@ -19,7 +19,6 @@ constexpr int kMaxGemvBatch = 8;       // token rows per GEMV pass
 constexpr int kMaxTileRows = 128;      // rows per GEMV tile (partial-output buffer)
 constexpr int kMaxGroup = 8;           // q heads per kv head handled by one attention tile
 constexpr int kHeadDim = 64;           // the head dimension the attention tiles are written for
-constexpr int kAttnPages = 4;          // KV pages an attention tile computes per round
 constexpr int kMaxSmem = 232448;       // dynamic shared memory per CTA on sm_100
 
 // Op codes of the tiles.  One "op group" = the tiles of one op of one layer.
