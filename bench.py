@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--resident", action="store_true", help="one resident grid serves every decode step")
     ap.add_argument("--split-pages", type=int, default=0)
+    ap.add_argument("--frame-chunks", type=int, default=0,
+                    help="two-stage: split the batch into chunks whose backbone and head launches overlap")
+    ap.add_argument("--head-workers", type=int, default=0, help="two-stage with --frame-chunks: the heads' workers")
     return ap.parse_args()
 
 
@@ -270,7 +273,7 @@ def main():
                 prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
                          "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill],
                 resident=1 if args.resident else 0,
-                split_pages=args.split_pages)
+                split_pages=args.split_pages, frame_chunks=args.frame_chunks, head_workers=args.head_workers)
     if args.regions:
         cuts = [int(x) for x in args.regions.split(",")]
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))
@@ -282,17 +285,24 @@ def main():
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
     launches_per_decode = stats["n_regions"] if mode == W.WPK_MEGAKERNEL else stats["n_ops"]
-    if two:
-        launches_per_decode += K  # a frame: the backbone step, then K head steps
+    # chunked two-stage frame: a backbone + head pair per chunk of ceil(B / C) sequences
+    chunks = args.frame_chunks if two and args.frame_chunks > 1 else 1
+    rows = -(-B // chunks)
+    n_chunks = -(-B // rows)
     prefill_tensor_cores = True
     try:
-        W.wpk_select_program(eng.h, B, T)
+        W.wpk_select_program(eng.h, rows, T)
         pst = W.wpk_graph_stats_get(eng.h)
         W.wpk_select_program(eng.h, 0, 0)
         launches_per_prefill = pst["n_regions"] if mode == W.WPK_MEGAKERNEL else pst["n_ops"]
     except W.WpkError:
         prefill_tensor_cores = False
         launches_per_prefill = T * launches_per_decode
+    if two:  # the backbone, then the head's K steps of the frame
+        launches_per_decode += K
+        launches_per_prefill += K
+    launches_per_decode *= n_chunks
+    launches_per_prefill *= n_chunks
 
     def prefill():
         W.wpk_prefill(eng.h, prompts_dev.data_ptr(), B, T, out_dev[0].data_ptr(), 0, sp)
@@ -417,7 +427,11 @@ def main():
                    "workers": stats["n_workers"],
                    "l2": "inputs larger than L2: %.2f GB of weights streamed per step" % (stats["weight_bytes"] / 1e9),
                    **({"codes_per_frame": K, "tokens": "codebook codes (a frame per sequence per step)"}
-                      if two else {})},
+                      if two else {}),
+                   **({"frame_chunks": n_chunks, "backbone_workers": stats["n_workers"],
+                       "head_workers": args.head_workers or (torch.cuda.get_device_properties(dev).multi_processor_count
+                                                             * max(1, args.workers_per_sm) - stats["n_workers"])}
+                      if chunks > 1 else {})},
         "decode_step_us": decode_summary,
         "ttft_ms": statistics.median(pre_ms) if pre_ms else None,
         "roofline": roofline,

@@ -123,6 +123,24 @@ typedef struct wpk_plan_cfg {
                            GEMV tiles; WPK_DECODE_GEMV; WPK_DECODE_MMA (the
                            step's sequences are the MMA N dimension, so
                            max_batch <= 128)                                    */
+  int frame_chunks;     /* two-stage model only.  0 or 1: a frame is the backbone
+                           step, then the head steps, each on all workers.
+                           C >= 2 (C <= max_batch, C <= 8): the sequences split
+                           into C chunks of ceil(max_batch / C), each with its
+                           own backbone and head programs over one shared weight
+                           image.  Per frame, the backbones run chunk after chunk
+                           on the caller's stream and the heads on a second
+                           stream, as separate persistent launches on disjoint
+                           worker sets; the head of chunk c starts as soon as the
+                           backbone has finished chunk c, overlapping the
+                           backbone of chunk c + 1 ("One Megakernel is Not
+                           Enough", Table I, producer-consumer overlap).  The
+                           call returns with the caller's stream ordered after
+                           the whole frame.  wpk_set_block_table is not
+                           supported then.                                      */
+  int head_workers;     /* frame_chunks >= 2: worker CTAs of the head programs
+                           (0 = half of the workers); the backbones take the
+                           rest of n_workers (0 = #SMs x workers_per_sm)        */
 } wpk_plan_cfg;
 
 /* Host weights: bf16 bit patterns, row-major [out][in]. */

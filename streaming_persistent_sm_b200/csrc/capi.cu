@@ -3,6 +3,8 @@
 // Host side of the runtime: device tables, launches per step (cooperative
 // persistent grid per region, or per-op launches captured once into a CUDA
 // Graph and replayed), prompt prefill, error word and trace access.
+#include <map>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -114,6 +116,17 @@ struct wpk_handle {
   uint64_t head_base = 0, weights_total = 0;  // head image offset; whole image
   std::vector<uint64_t> frame_embed_off, head_embed_off, out_head_off, out_head_mma_off;
   size_t off_p = 0, off_codes = 0;  // scratch: projection output [B][head hidden], last codes [B][K]
+  // chunked two-stage frame: this handle is chunk 0's backbone; `chunks` holds
+  // the (backbone + head) pairs of chunks 1.., all over this handle's weights
+  std::vector<wpk_handle*> chunks;
+  int chunk_rows = 0;                   // sequences per chunk
+  cudaStream_t head_stream = nullptr;   // the heads' stream
+  // a chunk pair's programs run beside another persistent launch: a
+  // cooperative launch may then be refused, so they launch as plain grids
+  // (backbone + head workers fit the SMs together, one CTA per SM)
+  bool plain_launch = false;
+  int per_sm = 0, per_sm_prefill = 0;  // co-resident workers an SM holds (decode, prefill programs)
+  std::vector<cudaEvent_t> chunk_ev;    // [0] fork, [1] join, [2 + c] backbone of chunk c done
 };
 
 namespace {
@@ -140,8 +153,12 @@ int check_live(wpk_handle* h) {
     h->err = "no CUDA device: host-only handle";
     return WPK_ERR_CUDA;
   }
-  const bool head_err = h->head && h->head->h_err_code && *(volatile int32_t*)h->head->h_err_code != 0;
-  if (!h->poisoned && ((h->h_err_code && *(volatile int32_t*)h->h_err_code != 0) || head_err)) {
+  auto dev_err = [](const wpk_handle* x) {
+    return x && x->h_err_code && *(volatile int32_t*)x->h_err_code != 0;
+  };
+  bool any = dev_err(h) || dev_err(h->head);
+  for (const wpk_handle* c : h->chunks) any = any || dev_err(c) || dev_err(c->head);
+  if (!h->poisoned && any) {
     h->poisoned = true;
     h->err = "device program reported an error (see wpk_get_error_info)";
   }
@@ -303,6 +320,13 @@ void scratch_layout(wpk_handle* h) {
   h->kv_bytes = (size_t)m.n_layers * h->n_blocks * 2 * m.n_kv_heads * g.plan.page_tokens * m.head_dim * 2;
 }
 
+// A worker grid: cooperative, so that all its CTAs are co-resident, unless
+// the handle runs beside another persistent grid (plain_launch).
+cudaError_t launch_grid(const wpk_handle* h, const void* fn, void** args, size_t smem, cudaStream_t s) {
+  if (h->plain_launch) return cudaLaunchKernel(fn, dim3(h->n_workers), dim3(kCtaThreads), args, smem, s);
+  return cudaLaunchCooperativeKernel(fn, dim3(h->n_workers), dim3(kCtaThreads), args, smem, s);
+}
+
 int launch_megakernel(wpk_handle* h, const KParams& base, cudaStream_t s) {
   const CompiledGraph& g = h->g;
   CUDA_TRY(h, cudaMemsetAsync(h->d_ctr, 0, std::max<size_t>(1, g.ctr_need.size()) * 4, s));
@@ -313,8 +337,7 @@ int launch_megakernel(wpk_handle* h, const KParams& base, cudaStream_t s) {
     P.t_end = g.region_begin[r + 1];
     P.region = r;
     void* args[] = {&P};
-    CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(h->n_workers), dim3(kCtaThreads), args,
-                                            h->smem, s));
+    CUDA_TRY(h, launch_grid(h, persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), args, h->smem, s));
   }
   return WPK_OK;
 }
@@ -557,8 +580,7 @@ int launch_prefill(wpk_handle* h, PrefillProgram* prog, const int32_t* tokens, i
       P.t_end = g.region_begin[r + 1];
       P.region = r;
       void* args[] = {&P};
-      CUDA_TRY(h, cudaLaunchCooperativeKernel(prefill_kernel_ptr(), dim3(h->n_workers), dim3(kCtaThreads), args,
-                                              h->smem_prefill, s));
+      CUDA_TRY(h, launch_grid(h, prefill_kernel_ptr(), args, h->smem_prefill, s));
     }
     return WPK_OK;
   }
@@ -599,6 +621,23 @@ const CompiledGraph& selected_graph(const wpk_handle* h) { return h->selected ? 
 
 extern "C" {
 
+// The dynamic shared memory limit is an attribute of the kernel function,
+// shared by every handle of the process: it only ever rises, to the largest
+// worker any handle on this device launches.
+static cudaError_t raise_smem_limit(const void* fn, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> limit;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t& cur = limit[{dev, fn}];
+  if (bytes <= cur) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) cur = bytes;
+  return e;
+}
+
 static int setup_device(wpk_handle* h) {
   CompiledGraph& g = h->g;
   const Plan& p = g.plan;
@@ -621,15 +660,11 @@ static int setup_device(wpk_handle* h) {
     h->smem_prefill = worker_smem_bytes(h->prefill_stages, 3 * kMmaChunkBytes, p.act_bytes);
   }
   const size_t smem_max = h->smem;
-  CUDA_TRY(h, cudaFuncSetAttribute(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem_max));
-  CUDA_TRY(h, cudaFuncSetAttribute(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)h->smem_per_op));
+  CUDA_TRY(h, raise_smem_limit(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), smem_max));
+  CUDA_TRY(h, raise_smem_limit(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), h->smem_per_op));
   if (h->smem_prefill) {
-    CUDA_TRY(h, cudaFuncSetAttribute(prefill_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)h->smem_prefill));
-    CUDA_TRY(h, cudaFuncSetAttribute(prefill_op_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)h->smem_prefill));
+    CUDA_TRY(h, raise_smem_limit(prefill_kernel_ptr(), h->smem_prefill));
+    CUDA_TRY(h, raise_smem_limit(prefill_op_kernel_ptr(), h->smem_prefill));
     int per_sm_p = 0;
     CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreads,
                                                               h->smem_prefill));
@@ -637,6 +672,7 @@ static int setup_device(wpk_handle* h) {
   }
   int per_sm = 0;
   CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), kCtaThreads, smem_max));
+  h->per_sm = per_sm;
   {
     // tcgen05.alloc waits until the SM has free TMEM columns: workers that
     // share an SM must fit its 512 columns together
@@ -652,6 +688,7 @@ static int setup_device(wpk_handle* h) {
       int per_sm_p = 0;
       CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreads,
                                                                 h->smem_prefill));
+      h->per_sm_prefill = per_sm_p;
       if (per_sm_p * pp.tmem_cols > 512)
         return fail(h, WPK_ERR_UNSUPPORTED, "co-resident prefill workers would not fit the SM's tensor memory");
     }
@@ -723,6 +760,17 @@ static int setup_device(wpk_handle* h) {
 
 static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out);
 
+// SMs of the current device (148, a B200's count, when there is no device).
+static int device_sms() {
+  int n_dev = 0, sms = 148;
+  if (cudaGetDeviceCount(&n_dev) == cudaSuccess && n_dev > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  cudaGetLastError();
+  return sms;
+}
+
 // One decoder; lm_rows > 0 replaces its output head's row count.
 static int build_decoder(const wpk_model_cfg* model, const wpk_plan_cfg* plan, int lm_rows, wpk_handle** out) {
   *out = nullptr;
@@ -732,13 +780,7 @@ static int build_decoder(const wpk_model_cfg* model, const wpk_plan_cfg* plan, i
   std::string msg = normalize_plan(*model, *plan, &p, &code);
   if (lm_rows > 0) p.lm_rows = lm_rows;
   // worker count the tiles are sized for: the plan's, else #SMs x workers per SM
-  int n_dev_w = 0, sms = 148;
-  if (cudaGetDeviceCount(&n_dev_w) == cudaSuccess && n_dev_w > 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  }
-  cudaGetLastError();
-  const int W = p.n_workers ? p.n_workers : sms * p.workers_per_sm;
+  const int W = p.n_workers ? p.n_workers : device_sms() * p.workers_per_sm;
   if (msg.empty()) msg = compile_graph(*model, p, &h->g, &code, W);
   if (!msg.empty()) {
     g_build_error = msg;
@@ -774,7 +816,15 @@ int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_ha
     g_build_error = "n_codebooks must be >= 0";
     return WPK_ERR_INVALID_ARG;
   }
+  if (plan->frame_chunks < 0 || plan->frame_chunks > 8 || plan->head_workers < 0) {
+    g_build_error = "frame_chunks must be 0..8 and head_workers >= 0";
+    return WPK_ERR_INVALID_ARG;
+  }
   if (model->n_codebooks > 0) return build_two_stage(model, plan, out);
+  if (plan->frame_chunks > 1 || plan->head_workers) {
+    g_build_error = "frame_chunks and head_workers apply to the two-stage model only";
+    return WPK_ERR_INVALID_ARG;
+  }
   return build_decoder(model, plan, 0, out);
 }
 
@@ -783,16 +833,11 @@ int wpk_build_graph(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_ha
 // whose input and output tables change from one head step to the next.  Both
 // images, the frame / head-input / output tables and the tensor-core images of
 // the output tables share one weight buffer; KV and scratch likewise.
-static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out) {
+// One backbone + head pair: the backbone for `plan`, the head for `head_plan`
+// (its batch and worker count; the head's cache holds one frame).
+static int build_pair(const wpk_model_cfg* model, const wpk_plan_cfg* plan, const wpk_plan_cfg* head_plan,
+                      wpk_handle** out) {
   const int K = model->n_codebooks, V = model->codebook_vocab;
-  if (!model->head || K > kMaxInTables || V <= 0) {
-    g_build_error = "two-stage model: needs a head shape, n_codebooks <= 16 and codebook_vocab > 0";
-    return WPK_ERR_INVALID_ARG;
-  }
-  if (plan->mode != WPK_MEGAKERNEL || plan->resident) {
-    g_build_error = "two-stage model: runs in WPK_MEGAKERNEL mode without a resident grid";
-    return WPK_ERR_UNSUPPORTED;
-  }
   wpk_model_cfg mb = *model;  // backbone: output head = projection (untied)
   mb.n_codebooks = 0;
   mb.codebook_vocab = 0;
@@ -804,7 +849,7 @@ static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan,
   mh.n_codebooks = 0;
   mh.codebook_vocab = 0;
   mh.head = nullptr;
-  wpk_plan_cfg ph = *plan;  // the head's cache holds one frame
+  wpk_plan_cfg ph = *head_plan;  // the head's cache holds one frame
   ph.max_context = K;
   ph.page_tokens = (K + 7) / 8 * 8;
   ph.n_regions = 1;
@@ -847,12 +892,82 @@ static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan,
   return WPK_OK;
 }
 
+static int build_two_stage(const wpk_model_cfg* model, const wpk_plan_cfg* plan, wpk_handle** out) {
+  const int K = model->n_codebooks, V = model->codebook_vocab;
+  if (!model->head || K > kMaxInTables || V <= 0) {
+    g_build_error = "two-stage model: needs a head shape, n_codebooks <= 16 and codebook_vocab > 0";
+    return WPK_ERR_INVALID_ARG;
+  }
+  if (plan->mode != WPK_MEGAKERNEL || plan->resident) {
+    g_build_error = "two-stage model: runs in WPK_MEGAKERNEL mode without a resident grid";
+    return WPK_ERR_UNSUPPORTED;
+  }
+  const int C = plan->frame_chunks;
+  if (C <= 1) {
+    if (plan->head_workers) {
+      g_build_error = "head_workers needs frame_chunks >= 2";
+      return WPK_ERR_INVALID_ARG;
+    }
+    return build_pair(model, plan, plan, out);
+  }
+  // chunked frame: C pairs of ceil(B / C) sequences; backbones and heads on
+  // disjoint worker counts that together fill the grid
+  if (C > plan->max_batch) {
+    g_build_error = "frame_chunks exceeds max_batch";
+    return WPK_ERR_INVALID_ARG;
+  }
+  const int W = plan->n_workers ? plan->n_workers : device_sms() * std::max(1, plan->workers_per_sm);
+  const int Wh = plan->head_workers ? plan->head_workers : W / 2;
+  if (Wh < 1 || Wh >= W) {
+    g_build_error = "head_workers must leave the backbones at least one worker";
+    return WPK_ERR_INVALID_ARG;
+  }
+  wpk_plan_cfg pb = *plan;
+  pb.max_batch = (plan->max_batch + C - 1) / C;
+  pb.n_workers = W - Wh;
+  pb.frame_chunks = 0;
+  pb.head_workers = 0;
+  wpk_plan_cfg ph = pb;
+  ph.n_workers = Wh;
+  std::vector<wpk_handle*> pairs;
+  for (int c = 0; c < C; ++c) {
+    wpk_handle* x = nullptr;
+    const int rc = build_pair(model, &pb, &ph, &x);
+    if (rc) {
+      for (wpk_handle* y : pairs) wpk_destroy(y);
+      return rc;
+    }
+    pairs.push_back(x);
+  }
+  // Grids of different programs share SMs only if an SM holds more than one
+  // worker; tensor-memory programs then could wait on each other's columns
+  for (wpk_handle* x : pairs)
+    for (wpk_handle* y : {x, x->head})
+      if (y->has_device && (y->per_sm > 1 || y->per_sm_prefill > 1) && y->g.lay.mma) {
+        for (wpk_handle* z : pairs) wpk_destroy(z);
+        g_build_error = "chunked frames with tensor-core programs need one worker per SM";
+        return WPK_ERR_UNSUPPORTED;
+      }
+  for (wpk_handle* x : pairs) x->plain_launch = x->head->plain_launch = true;
+  wpk_handle* h = pairs[0];
+  h->chunks.assign(pairs.begin() + 1, pairs.end());
+  h->chunk_rows = pb.max_batch;
+  *out = h;
+  return WPK_OK;
+}
+
 int wpk_workspace_size(const wpk_handle* h, size_t* weight_bytes, size_t* kv_bytes, size_t* scratch_bytes) {
   if (!h) return WPK_ERR_INVALID_ARG;
-  if (h->head) {
+  if (h->head) {  // every pair's KV and scratch, one after another
+    size_t kv = 0, sc = 0;
+    for (int c = 0; c <= (int)h->chunks.size(); ++c) {
+      const wpk_handle* x = c ? h->chunks[c - 1] : h;
+      kv += x->kv_bytes + x->head->kv_bytes;
+      sc += x->scratch_bytes + x->head->scratch_bytes;
+    }
     if (weight_bytes) *weight_bytes = h->weights_total;
-    if (kv_bytes) *kv_bytes = h->kv_bytes + h->head->kv_bytes;
-    if (scratch_bytes) *scratch_bytes = h->scratch_bytes + h->head->scratch_bytes;
+    if (kv_bytes) *kv_bytes = kv;
+    if (scratch_bytes) *scratch_bytes = sc;
     return WPK_OK;
   }
   if (weight_bytes) *weight_bytes = h->g.lay.total;
@@ -896,16 +1011,27 @@ static int load_two_stage(wpk_handle* h, const wpk_weights* w, void* dev_weights
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUDA_TRY(h, cudaMemcpyAsync(dev_weights, img.data(), img.size(), cudaMemcpyHostToDevice, s));
   CUDA_TRY(h, cudaStreamSynchronize(s));
-  h->weights = static_cast<uint8_t*>(dev_weights);
-  h->kv = static_cast<uint16_t*>(dev_kv);
-  h->scratch = static_cast<uint8_t*>(dev_scratch);
-  hh->weights = h->weights + h->head_base;
-  hh->kv = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(dev_kv) + h->kv_bytes);
-  hh->scratch = h->scratch + h->scratch_bytes;
-  h->loaded = hh->loaded = true;
-  h->prefilled = hh->prefilled = false;
-  h->graphs.clear();
-  hh->graphs.clear();
+  // every pair reads the one image; KV and scratch are laid out pair by pair
+  uint8_t* kv = static_cast<uint8_t*>(dev_kv);
+  uint8_t* sc = static_cast<uint8_t*>(dev_scratch);
+  for (int c = 0; c <= (int)h->chunks.size(); ++c) {
+    wpk_handle* x = c ? h->chunks[c - 1] : h;
+    wpk_handle* xh = x->head;
+    x->weights = static_cast<uint8_t*>(dev_weights);
+    xh->weights = x->weights + x->head_base;
+    x->kv = reinterpret_cast<uint16_t*>(kv);
+    kv += x->kv_bytes;
+    xh->kv = reinterpret_cast<uint16_t*>(kv);
+    kv += xh->kv_bytes;
+    x->scratch = sc;
+    sc += x->scratch_bytes;
+    xh->scratch = sc;
+    sc += xh->scratch_bytes;
+    x->loaded = xh->loaded = true;
+    x->prefilled = xh->prefilled = false;
+    x->graphs.clear();
+    xh->graphs.clear();
+  }
   return WPK_OK;
 }
 
@@ -939,6 +1065,7 @@ int wpk_set_block_table(wpk_handle* h, const int32_t* table) {
   int rc = check_live(h);
   if (rc) return rc;
   if (!table) return fail(h, WPK_ERR_INVALID_ARG, "null table");
+  if (!h->chunks.empty()) return fail(h, WPK_ERR_UNSUPPORTED, "a chunked two-stage frame keeps its own block tables");
   const size_t n = (size_t)h->g.plan.max_batch * h->g.max_blocks;
   std::vector<char> seen(n, 0);
   for (size_t i = 0; i < n; ++i) {
@@ -973,12 +1100,96 @@ static int reset_step_state(wpk_handle* h, cudaStream_t s) {
 }
 static int head_frame(wpk_handle* h, int32_t* codes_out, float* logits, cudaStream_t s);
 
+// Chunked two-stage frame: the pair of chunk c, and the stream and events
+// that let each head overlap the next chunk's backbone.
+static wpk_handle* pair_of(wpk_handle* h, int c) { return c ? h->chunks[c - 1] : h; }
+
+static int chunk_streams(wpk_handle* h) {
+  if (h->head_stream) return WPK_OK;
+  CUDA_TRY(h, cudaStreamCreateWithFlags(&h->head_stream, cudaStreamNonBlocking));
+  const int n = 2 + 1 + (int)h->chunks.size();
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t e;
+    CUDA_TRY(h, cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    h->chunk_ev.push_back(e);
+  }
+  return WPK_OK;
+}
+
+// The heads' stream starts after what the caller's stream holds so far.
+static int chunk_fork(wpk_handle* h, cudaStream_t s) {
+  CUDA_TRY(h, cudaEventRecord(h->chunk_ev[0], s));
+  CUDA_TRY(h, cudaStreamWaitEvent(h->head_stream, h->chunk_ev[0], 0));
+  return WPK_OK;
+}
+
+// The caller's stream continues after every head; taken on error paths too.
+static int chunk_join(wpk_handle* h, cudaStream_t s, int rc) {
+  const cudaError_t e1 = cudaEventRecord(h->chunk_ev[1], h->head_stream);
+  const cudaError_t e2 = cudaStreamWaitEvent(s, h->chunk_ev[1], 0);
+  if (!rc && (e1 != cudaSuccess || e2 != cudaSuccess)) return fail(h, WPK_ERR_CUDA, "stream join failed");
+  return rc;
+}
+
+// Head c may start once the caller's stream has finished chunk c's backbone.
+static int chunk_handoff(wpk_handle* h, int c, cudaStream_t s) {
+  CUDA_TRY(h, cudaEventRecord(h->chunk_ev[2 + c], s));
+  CUDA_TRY(h, cudaStreamWaitEvent(h->head_stream, h->chunk_ev[2 + c], 0));
+  return WPK_OK;
+}
+
+static int chunked_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len,
+                           int32_t* first_tok_dev, float* logits_dev, cudaStream_t s) {
+  if (!tokens_dev || batch <= 0 || prompt_len <= 0) return fail(h, WPK_ERR_INVALID_ARG, "bad prefill arguments");
+  const int C = 1 + (int)h->chunks.size(), bc = h->chunk_rows, K = h->n_cb, V = h->cb_vocab;
+  if (batch > bc * C) return fail(h, WPK_ERR_SHAPE, "batch or prompt exceeds the plan");
+  int rc = chunk_streams(h);
+  if (rc) return rc;
+  // every head's batch is set before any launch, so nothing below waits on a head
+  std::vector<int32_t> n(C);
+  for (int c = 0; c < C; ++c) {
+    wpk_handle* x = pair_of(h, c);
+    n[c] = std::max(0, std::min(bc, batch - c * bc));
+    x->batch = n[c];
+    x->prefilled = false;
+    if (!n[c]) continue;
+    rc = reset_step_state(x->head, s);
+    if (rc) return rc;
+    CUDA_TRY(h, cudaMemcpyAsync(x->head->d_active, &n[c], 4, cudaMemcpyHostToDevice, s));
+  }
+  CUDA_TRY(h, cudaStreamSynchronize(s));  // `n` lives on this stack frame
+  rc = chunk_fork(h, s);
+  if (rc) return rc;
+  for (int c = 0; c < C && !rc && n[c]; ++c) {
+    wpk_handle* x = pair_of(h, c);
+    const size_t r0 = (size_t)c * bc;
+    int32_t* codes = reinterpret_cast<int32_t*>(x->scratch + x->off_codes);
+    rc = prefill_impl(x, tokens_dev + r0 * prompt_len, n[c], prompt_len, codes,
+                      reinterpret_cast<float*>(x->scratch + x->off_p), s);
+    if (!rc) rc = chunk_handoff(h, c, s);
+    if (rc) break;
+    x->head->batch = n[c];
+    x->head->prefilled = true;
+    int32_t* out = first_tok_dev ? first_tok_dev + r0 * K : codes;
+    rc = head_frame(x, out, logits_dev ? logits_dev + r0 * K * V : nullptr, h->head_stream);
+    if (!rc && first_tok_dev)
+      CUDA_TRY(h, cudaMemcpyAsync(codes, out, (size_t)n[c] * K * 4, cudaMemcpyDeviceToDevice, h->head_stream));
+    if (x != h && rc) h->err = x->err;
+  }
+  return chunk_join(h, s, rc);
+}
+
 int wpk_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, int prompt_len, int32_t* first_tok_dev,
                 float* logits_dev, void* stream) {
   if (!h || !h->head) return prefill_impl(h, tokens_dev, batch, prompt_len, first_tok_dev, logits_dev, stream);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!h->chunks.empty()) {
+    int rc = check_live(h);
+    if (rc) return rc;
+    return chunked_prefill(h, tokens_dev, batch, prompt_len, first_tok_dev, logits_dev, s);
+  }
   // two-stage: the prompt through the backbone, whose output head yields the
   // projection p at the last position; then the head's first frame
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* codes = reinterpret_cast<int32_t*>(h->scratch + h->off_codes);
   float* p = reinterpret_cast<float*>(h->scratch + h->off_p);
   int rc = prefill_impl(h, tokens_dev, batch, prompt_len, codes, p, stream);
@@ -1042,15 +1253,9 @@ static int prefill_impl(wpk_handle* h, const int32_t* tokens_dev, int batch, int
   return WPK_OK;
 }
 
-int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev, void* stream) {
-  int rc = check_live(h);
-  if (rc) return rc;
-  if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");
-  if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!h->head) return step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, s);
-  // two-stage frame: backbone step on sum_k frame_embed_k[c_k] -> p, then the head
-  int32_t* codes = reinterpret_cast<int32_t*>(h->scratch + h->off_codes);
+// The backbone step of a two-stage frame: input sum_k frame_embed_k[c_k] of
+// the codes at in_codes ([batch][K]); output p through the projection.
+static int backbone_step(wpk_handle* h, const int32_t* in_codes, cudaStream_t s) {
   const int K = h->n_cb;
   h->io = wpk_handle::IO{};
   h->io.set = true;
@@ -1061,14 +1266,52 @@ int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, flo
   h->io.lm_mma_off = h->g.lay.lm_mma;
   h->io.logits_stride = h->g.plan.lm_rows;
   h->io.out_stride = 1;
-  rc = step_impl(h, in_tok_dev ? in_tok_dev : codes, K, nullptr,
-                 reinterpret_cast<float*>(h->scratch + h->off_p), s);
+  const int rc = step_impl(h, in_codes, K, nullptr, reinterpret_cast<float*>(h->scratch + h->off_p), s);
   h->io.set = false;
+  return rc;
+}
+
+static int chunked_frame(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev,
+                         cudaStream_t s) {
+  const int C = 1 + (int)h->chunks.size(), bc = h->chunk_rows, K = h->n_cb, V = h->cb_vocab;
+  int rc = chunk_fork(h, s);
+  if (rc) return rc;
+  for (int c = 0; c < C && !rc; ++c) {
+    wpk_handle* x = pair_of(h, c);
+    if (!x->batch) break;
+    const size_t r0 = (size_t)c * bc;
+    int32_t* codes = reinterpret_cast<int32_t*>(x->scratch + x->off_codes);
+    rc = backbone_step(x, in_tok_dev ? in_tok_dev + r0 * K : codes, s);
+    if (!rc) rc = chunk_handoff(h, c, s);
+    if (rc) {
+      if (x != h) h->err = x->err;
+      break;
+    }
+    int32_t* out = out_tok_dev ? out_tok_dev + r0 * K : codes;
+    rc = head_frame(x, out, logits_dev ? logits_dev + r0 * K * V : nullptr, h->head_stream);
+    if (!rc && out_tok_dev)
+      CUDA_TRY(h, cudaMemcpyAsync(codes, out, (size_t)x->batch * K * 4, cudaMemcpyDeviceToDevice, h->head_stream));
+    if (x != h && rc) h->err = x->err;
+  }
+  return chunk_join(h, s, rc);
+}
+
+int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev, void* stream) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");
+  if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!h->head) return step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, s);
+  if (!h->chunks.empty()) return chunked_frame(h, in_tok_dev, out_tok_dev, logits_dev, s);
+  // two-stage frame: backbone step on sum_k frame_embed_k[c_k] -> p, then the head
+  int32_t* codes = reinterpret_cast<int32_t*>(h->scratch + h->off_codes);
+  rc = backbone_step(h, in_tok_dev ? in_tok_dev : codes, s);
   if (rc) return rc;
   rc = head_frame(h, out_tok_dev ? out_tok_dev : codes, logits_dev, s);
   if (rc) return rc;
   if (out_tok_dev)
-    CUDA_TRY(h, cudaMemcpyAsync(codes, out_tok_dev, (size_t)h->batch * K * 4, cudaMemcpyDeviceToDevice, s));
+    CUDA_TRY(h, cudaMemcpyAsync(codes, out_tok_dev, (size_t)h->batch * h->n_cb * 4, cudaMemcpyDeviceToDevice, s));
   return WPK_OK;
 }
 
@@ -1204,8 +1447,18 @@ int wpk_get_error_info(wpk_handle* h, wpk_error_info* info) {
   int rc = res_shutdown(h);
   if (rc) return rc;
   CUDA_TRY(h, cudaDeviceSynchronize());
+  // the first error among this program and (two-stage) the head and chunk pairs
+  std::vector<const wpk_handle*> progs{h, h->head};
+  for (const wpk_handle* c : h->chunks) {
+    progs.push_back(c);
+    progs.push_back(c->head);
+  }
   ErrWord e{};
-  CUDA_TRY(h, cudaMemcpy(&e, h->d_err, sizeof e, cudaMemcpyDeviceToHost));
+  for (const wpk_handle* x : progs) {
+    if (!x || !x->d_err) continue;
+    CUDA_TRY(h, cudaMemcpy(&e, x->d_err, sizeof e, cudaMemcpyDeviceToHost));
+    if (e.code) break;
+  }
   info->code = e.code;
   info->tile = e.tile;
   info->counter = e.counter;
@@ -1224,6 +1477,13 @@ int wpk_destroy(wpk_handle* h) {
     wpk_destroy(h->head);
     h->head = nullptr;
   }
+  for (wpk_handle* c : h->chunks) wpk_destroy(c);
+  h->chunks.clear();
+  if (h->head_stream) {
+    cudaStreamSynchronize(h->head_stream);
+    cudaStreamDestroy(h->head_stream);
+  }
+  for (cudaEvent_t e : h->chunk_ev) cudaEventDestroy(e);
   if (h->has_device) {
     res_shutdown(h);
     cudaDeviceSynchronize();
@@ -1258,6 +1518,8 @@ int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes
   if (rc) return rc;
   if (h->g.plan.mode != WPK_MEGAKERNEL)
     return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the megakernel mode");
+  if (h->head)
+    return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc runs a single decoder, not the two-stage model");
   if (h->g.plan.resident)
     return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs a launch per step (the resident grid keeps its "
                                         "scratch pointer for its lifetime)");

@@ -65,7 +65,7 @@ class wpk_plan_cfg(C.Structure):
                 ("n_regions", C.c_int), ("region_cut", C.c_int * 4), ("trace", C.c_int),
                 ("wait_timeout_ns", C.c_uint64), ("slot_bytes", C.c_int), ("tile_bytes", C.c_int),
                 ("split_pages", C.c_int), ("lookahead", C.c_int), ("schedule", C.c_int), ("prefill", C.c_int),
-                ("decode", C.c_int)]
+                ("decode", C.c_int), ("frame_chunks", C.c_int), ("head_workers", C.c_int)]
 
 
 _P16 = C.POINTER(C.c_uint16)
@@ -166,11 +166,12 @@ def plan_cfg(max_batch: int, max_context: int, mode: int = WPK_MEGAKERNEL, n_reg
              region_cut: Sequence[int] = (0, 0, 0, 0), trace: int = 0, wait_timeout_ns: int = 0,
              page_tokens: int = 0, n_workers: int = 0, workers_per_sm: int = 0, resident: int = 0,
              slot_bytes: int = 0, tile_bytes: int = 0, split_pages: int = 0, lookahead: int = 0,
-             schedule: int = 0, prefill: int = 0, decode: int = 0) -> wpk_plan_cfg:
+             schedule: int = 0, prefill: int = 0, decode: int = 0, frame_chunks: int = 0,
+             head_workers: int = 0) -> wpk_plan_cfg:
     cut = (C.c_int * 4)(*list(region_cut) + [0] * (4 - len(region_cut)))
     return wpk_plan_cfg(max_batch, max_context, page_tokens, n_workers, workers_per_sm, mode, resident, n_regions,
                         cut, trace, wait_timeout_ns, slot_bytes, tile_bytes, split_pages, lookahead, schedule,
-                        prefill, decode)
+                        prefill, decode, frame_chunks, head_workers)
 
 
 # ----------------------------------------------------------- thin wrappers --

@@ -333,3 +333,30 @@ def test_two_stage_handle_host_side(lib):
         W.wpk_build_graph(bad, W.plan_cfg(1, 64))
     with pytest.raises(W.WpkError):
         W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(1, 64, resident=1))
+
+
+def test_two_stage_chunked_frame_host_side(lib):
+    """frame_chunks = C builds C backbone + head pairs of ceil(B / C) sequences
+    over one weight image; KV and scratch are the pairs' sums."""
+    s = synth.TINY_TWO_STAGE
+    one = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16))
+    per3 = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(3, 64, n_workers=12))
+    h = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16, frame_chunks=2, head_workers=4))
+    try:
+        W.wpk_verify_graph(h)
+        st = W.wpk_graph_stats_get(h)
+        assert st["n_workers"] == 12  # the backbones' share of the 16 workers
+        wb1, _, _ = W.wpk_workspace_size(one)
+        wb, kb, sb = W.wpk_workspace_size(h)
+        _, kb3, sb3 = W.wpk_workspace_size(per3)
+        assert wb == wb1  # one shared image
+        assert kb == 2 * kb3 and sb == 2 * sb3  # two pairs of three sequences each
+    finally:
+        for x in (one, per3, h):
+            W.wpk_destroy(x)
+    for bad in (dict(frame_chunks=9), dict(frame_chunks=6), dict(frame_chunks=-1),
+                dict(frame_chunks=2, head_workers=16), dict(head_workers=4)):
+        with pytest.raises(W.WpkError):
+            W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16, **bad))
+    with pytest.raises(W.WpkError):  # a plain decoder has no frame
+        W.wpk_build_graph(W.model_cfg(synth.TINY), W.plan_cfg(4, 64, frame_chunks=2))

@@ -74,9 +74,11 @@ def test_llama1b_prefill_b32_sampled_rows(weights, dec):
         eng.close()
 
 
-def test_two_stage_1b_shape_b32_sampled_rows():
+@pytest.mark.parametrize("plan", [{}, dict(frame_chunks=2)])
+def test_two_stage_1b_shape_b32_sampled_rows(plan):
     # the C5 shape: the 1B backbone, a 4-layer h1024 head, 16 codebooks of 2048,
-    # batch 32 (tensor-core decode for both), 200-token prompts, two frames
+    # batch 32 (tensor-core decode for both), 200-token prompts, two frames;
+    # chunked: two pairs of 16 sequences, row 16 is the second chunk's first
     from tests.test_two_stage_gpu import _check_frame_shape
 
     s = synth.TWO_STAGE
@@ -84,7 +86,7 @@ def test_two_stage_1b_shape_b32_sampled_rows():
     ora = oracle.TwoStage(s, w)
     wl = synth.WORKLOADS["two_stage_b32"]
     B, T, rows = wl.batch, wl.prompt_len, [0, 16, 31]
-    eng = W.Engine(s, w, B, T + 4)
+    eng = W.Engine(s, w, B, T + 4, **plan)
     try:
         prompts = synth.make_prompts(s.backbone.vocab, B, T, wl.prompt_seed)
         codes, lg = eng.prefill(prompts, want_logits=True)

@@ -38,7 +38,10 @@ def _check_frame(gpu_codes, gpu_logits, ref_logits, where):
 
 
 @pytest.mark.parametrize("B,plan", [(1, {}), (3, {}), (16, {}), (12, dict(schedule=W.WPK_SCHED_STATIC)),
-                                    (2, dict(n_regions=2, region_cut=(0, 1, 0, 0)))])
+                                    (2, dict(n_regions=2, region_cut=(0, 1, 0, 0))),
+                                    # chunked frames: backbone and head launches overlap on two streams
+                                    (3, dict(frame_chunks=2)), (5, dict(frame_chunks=3, head_workers=40)),
+                                    (16, dict(frame_chunks=2, schedule=W.WPK_SCHED_STATIC))])
 def test_two_stage_prefill_and_frames(weights, ora, B, plan):
     T, frames, ctx = 17, 6, 32
     eng = W.Engine(S, weights, B, ctx, **plan)
@@ -60,9 +63,10 @@ def test_two_stage_prefill_and_frames(weights, ora, B, plan):
         eng.close()
 
 
-def test_two_stage_explicit_codes_are_the_next_input(weights, ora):
+@pytest.mark.parametrize("plan", [{}, dict(frame_chunks=2)])
+def test_two_stage_explicit_codes_are_the_next_input(weights, ora, plan):
     B, T, ctx = 2, 9, 16
-    eng = W.Engine(S, weights, B, ctx)
+    eng = W.Engine(S, weights, B, ctx, **plan)
     try:
         prompts = synth.make_prompts(S.backbone.vocab, B, T, 7)
         codes, _ = eng.prefill(prompts)
