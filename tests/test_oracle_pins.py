@@ -350,3 +350,27 @@ def test_two_stage_head_position0_reads_projected_state():
     ts.proj = np.zeros_like(ts.proj)
     c_b, l_b = ts.head_frame(h)
     assert not np.allclose(l_a[:, 0], l_b[:, 0])
+
+
+def test_oracle_matches_its_regression_fixture():
+    """The oracle still computes what tests/golden/make_golden.py recorded
+    (a regression guard on the oracle's arithmetic; the outside pins are the
+    tests above)."""
+    import importlib.util
+    import json
+    import os
+
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(here, "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    with open(os.path.join(here, "oracle_regression.json")) as f:
+        want = json.load(f)
+    got = {"decoder": mg.decoder_case(), "two_stage": mg.two_stage_case()}
+    for a, b in zip(want["decoder"]["steps"], got["decoder"]["steps"]):
+        assert a["tokens"] == b["tokens"], a["step"]
+        np.testing.assert_allclose(b["logits_sample"], a["logits_sample"], rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(b["logsumexp"], a["logsumexp"], rtol=1e-9, atol=1e-12)
+    for a, b in zip(want["two_stage"]["frames"], got["two_stage"]["frames"]):
+        assert a["codes"] == b["codes"], a["frame"]
+        np.testing.assert_allclose(b["logits_k0_sample"], a["logits_k0_sample"], rtol=1e-9, atol=1e-12)
