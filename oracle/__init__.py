@@ -22,8 +22,11 @@ Parity status per function (what pins each one, besides the code itself):
   Decoder           - transformers' LlamaForCausalLM (float64) on the tiny
                       shape; prefill == incremental decode; batch rows
                       independent; paged cache == contiguous cache
-  TwoStage          - parity unpinned beyond the primitives above (the
-                      composition is this repository's own definition)
+  TwoStage          - the composition is this repository's own definition;
+                      its implementation is pinned against an independent
+                      build of that definition from transformers' float64
+                      Llama driven by input vectors (three planted slips in
+                      the composition are shown to break the pin)
 """
 from .llama import (  # noqa: F401
     KVCache,

@@ -260,8 +260,9 @@ class TwoStage:
     head_embed_k[c_{k-1}]; c_k = argmax(out_head_k . RMSNorm(y_k; g_head_final)).
     The head's cache restarts every frame.  The next backbone input is
     sum_k frame_embed_k[c_k].  This composition is this repository's reading of
-    a two-stage streaming model (the pages name such models but print none);
-    parity for it is unpinned beyond its primitives.
+    a two-stage streaming model (the pages name such models but print none).
+    The tests check this implementation of it against one assembled from
+    transformers' Llama layers.
     """
 
     def __init__(self, shape, weights: Dict[str, np.ndarray], round_kv: bool = True):

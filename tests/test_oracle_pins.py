@@ -352,6 +352,134 @@ def test_two_stage_head_position0_reads_projected_state():
     assert not np.allclose(l_a[:, 0], l_b[:, 0])
 
 
+
+# ---- the two-stage model against transformers' Llama run on input vectors ----
+def _hf_llama_body(shape, weights, prefix):
+    """transformers' LlamaModel in float64 carrying one decoder's layers and
+    final norm; it is driven through inputs_embeds, so its own embedding
+    table is never read."""
+    import torch
+    from transformers import LlamaConfig, LlamaModel
+
+    cfg = LlamaConfig(vocab_size=8, hidden_size=shape.hidden, intermediate_size=shape.ffn,
+                      num_hidden_layers=shape.n_layers, num_attention_heads=shape.n_heads,
+                      num_key_value_heads=shape.n_kv_heads, head_dim=shape.head_dim, rms_norm_eps=shape.rms_eps,
+                      rope_theta=shape.rope_theta, max_position_embeddings=4096, attention_bias=False,
+                      mlp_bias=False)
+    m = LlamaModel(cfg).double().eval()
+    f = lambda n: torch.from_numpy(oracle.bf16_to_f64(weights[prefix + n]))
+    names = {"norm.weight": "final_norm"}
+    for l in range(shape.n_layers):
+        p, q = f"layers.{l}.", f"layers.{l}."
+        names.update({p + "self_attn.q_proj.weight": q + "wq", p + "self_attn.k_proj.weight": q + "wk",
+                      p + "self_attn.v_proj.weight": q + "wv", p + "self_attn.o_proj.weight": q + "wo",
+                      p + "mlp.gate_proj.weight": q + "w_gate", p + "mlp.up_proj.weight": q + "w_up",
+                      p + "mlp.down_proj.weight": q + "w_down", p + "input_layernorm.weight": q + "attn_norm",
+                      p + "post_attention_layernorm.weight": q + "ffn_norm"})
+    sd = m.state_dict()
+    with torch.no_grad():
+        for hf, ours in names.items():
+            sd[hf].copy_(f(ours))
+    return m
+
+
+def _hf_two_stage_logits(s, weights, prompts, frame_codes):
+    """Per-frame head logits [B][K][V] from two transformers models.
+
+    The backbone runs once over the prompt's embeddings followed by each
+    frame's input sum_k frame_embed_k[c_k] (frame f's state is at position
+    T - 1 + f).  For every frame the head runs from position 0 on
+    [W_proj . state, head_embed_1[c_0], ..., head_embed_(K-1)[c_(K-2)]]."""
+    import torch
+
+    f64 = lambda n: oracle.bf16_to_f64(weights[n])
+    K = s.n_codebooks
+    B, T = prompts.shape
+    seq = [f64("backbone.embed")[prompts]]
+    for codes in frame_codes[:-1]:
+        seq.append(sum(f64(f"frame_embed.{k}")[codes[:, k]] for k in range(K))[:, None, :])
+    bb = _hf_llama_body(s.backbone, weights, "backbone.")
+    hd = _hf_llama_body(s.head, weights, "head.")
+    with torch.no_grad():
+        hid = bb(inputs_embeds=torch.from_numpy(np.concatenate(seq, axis=1))).last_hidden_state.numpy()
+        out = []
+        for f, codes in enumerate(frame_codes):
+            xs = [hid[:, T - 1 + f] @ f64("proj").T]
+            xs += [f64(f"head_embed.{k}")[codes[:, k - 1]] for k in range(1, K)]
+            y = hd(inputs_embeds=torch.from_numpy(np.stack(xs, axis=1))).last_hidden_state.numpy()
+            out.append(np.stack([y[:, k] @ f64(f"out_head.{k}").T for k in range(K)], axis=1))
+    return out
+
+
+def _oracle_two_stage_frames(ts, prompts, n_frames):
+    cache = ts.backbone.new_cache(prompts.shape[0], prompts.shape[1] + n_frames)
+    codes, lg = ts.prefill(cache, prompts)
+    out = [(codes, lg)]
+    for _ in range(n_frames - 1):
+        codes, lg = ts.frame(cache, codes)
+        out.append((codes, lg))
+    return out
+
+
+@pytest.fixture(scope="module")
+def two_stage_case():
+    s = synth.TINY_TWO_STAGE
+    return s, synth.make_weights(s, seed=0), synth.make_prompts(s.backbone.vocab, 2, 6, seed=5)
+
+
+def test_two_stage_matches_transformers_llama_fp64(two_stage_case):
+    """The oracle's two-stage composition (projection, head inputs, per-frame
+    head cache, output heads, next-frame input) against an independent build
+    of the same definition from transformers' float64 Llama."""
+    s, w, prompts = two_stage_case
+    ours = _oracle_two_stage_frames(oracle.TwoStage(s, w, round_kv=False), prompts, 3)
+    ref = _hf_two_stage_logits(s, w, prompts, [c for c, _ in ours])
+    for f, ((codes, lg), r) in enumerate(zip(ours, ref)):
+        np.testing.assert_allclose(lg, r, atol=2e-6, rtol=0, err_msg=f"frame {f}")
+        assert (codes == oracle.argmax_lowest(r.reshape(-1, r.shape[-1])).reshape(codes.shape)).all()
+
+
+class _HeadCacheKept(oracle.TwoStage):
+    """Planted slip: the head's cache runs on across frames."""
+
+    def head_frame(self, h, forced=None):
+        kept = getattr(self, "_kept", None)
+        orig = self.head.new_cache
+        if kept is None:
+            kept = self._kept = orig(h.shape[0], 4 * self.s.n_codebooks, page_tokens=self.s.n_codebooks)
+        self.head.new_cache = lambda *a, **k: kept
+        try:
+            return super().head_frame(h, forced)
+        finally:
+            self.head.new_cache = orig
+
+
+class _HeadTableShifted(oracle.TwoStage):
+    """Planted slip: head step k looks code c_(k-1) up in the table of step
+    k + 1 (the last step wraps to table 1)."""
+
+    def __init__(self, *a, **k):
+        super().__init__(*a, **k)
+        self.head_embed = [None] + self.head_embed[2:] + [self.head_embed[1]]
+
+
+class _FrameInputFirstCode(oracle.TwoStage):
+    """Planted slip: the next frame's input is frame_embed_0[c_0] alone."""
+
+    def frame(self, cache, prev_codes, forced=None):
+        x = self.frame_embed[0][np.asarray(prev_codes[:, 0], dtype=np.int64)]
+        hid = self.backbone.forward_hidden(cache, x[:, None, :])
+        return self.head_frame(hid[:, 0, :], forced)
+
+
+@pytest.mark.parametrize("cls", [_HeadCacheKept, _HeadTableShifted, _FrameInputFirstCode])
+def test_planted_two_stage_slips_are_caught(two_stage_case, cls):
+    s, w, prompts = two_stage_case
+    ours = _oracle_two_stage_frames(cls(s, w, round_kv=False), prompts, 3)
+    ref = _hf_two_stage_logits(s, w, prompts, [c for c, _ in ours])
+    assert max(np.max(np.abs(lg - r)) for (_, lg), r in zip(ours, ref)) > 1e-3
+
+
 def test_oracle_matches_its_regression_fixture():
     """The oracle still computes what tests/golden/make_golden.py recorded
     (a regression guard on the oracle's arithmetic; the outside pins are the
