@@ -2,8 +2,9 @@
 the oracle's TwoStage, teacher-forced with the GPU's codes.
 
 The composition (projection, head inputs, output heads, next-frame input) is
-this repository's reading of a two-stage streaming model; its primitives are
-pinned, the composition itself is not (see the oracle's header).
+this repository's reading of a two-stage streaming model.  The oracle's
+implementation of it is pinned against transformers' Llama layers in
+tests/test_oracle_pins.py.
 """
 import numpy as np
 import pytest
