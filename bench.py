@@ -64,26 +64,26 @@ def parse():
     return ap.parse_args()
 
 
-def profiled_traffic(B, mean_ctx):
-    """DRAM bytes per launch of the decode program from the committed ncu
-    summary, scaled by the KV bytes to this run's batch and context - or None
-    when the kernel sources changed since the capture."""
+def profiled_traffic(kernel, B, mean_ctx):
+    """DRAM bytes per launch of a decode program from the committed ncu summary
+    of that kernel, scaled by the KV bytes to this run's batch and context - or
+    None when no summary covers the kernel or its sources changed since the
+    capture."""
+    import glob
     import hashlib
     import re
 
-    p = os.path.join(ROOT, "profiles", "wpk_persistent_kernel_llama1b_b1.md")
-    if not os.path.exists(p):
-        return None
-    txt = open(p).read()
     src = os.path.join(ROOT, "streaming_persistent_sm_b200", "csrc")
     sha = hashlib.sha1(b"".join(open(os.path.join(src, f), "rb").read()
                                 for f in ("runtime.cu", "ptx.cuh", "wpk_internal.h"))).hexdigest()
-    m = {k: v for k, v in re.findall(r"^(\w+)(?:\([^)]*\))?: (\S+)$", txt, re.M)}
-    if m.get("source_sha1") != sha:
-        return None
-    kv = float(m["kv_bytes_per_token"])
-    base = float(m["traffic_bytes_per_launch"]) - float(m["traffic_batch"]) * float(m["traffic_context"]) * kv
-    return base + B * mean_ctx * kv
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        m = {k: v for k, v in re.findall(r"^(\w+)(?:\([^)]*\))?: (\S+)$", open(p).read(), re.M)}
+        if m.get("traffic_kernel") != kernel or m.get("source_sha1") != sha:
+            continue
+        kv = float(m["kv_bytes_per_token"])
+        base = float(m["traffic_bytes_per_launch"]) - float(m["traffic_batch"]) * float(m["traffic_context"]) * kv
+        return base + B * mean_ctx * kv
+    return None
 
 
 def measured_peaks():
@@ -398,8 +398,8 @@ def main():
                           "achieved_gbs": dec_gbs, "frac_of_8tbs": dec_gbs / 8000.0}
         # DRAM traffic per launch from the committed capture (plain decoder, one
         # launch per step; None for other programs or after a kernel change)
-        traffic = (profiled_traffic(B, statistics.mean(dec_ctx)) if not two and mode == W.WPK_MEGAKERNEL
-                   and stats["n_regions"] == 1 and not args.layers else None)
+        traffic = (profiled_traffic(kernel_name, B, statistics.mean(dec_ctx)) if not two
+                   and mode == W.WPK_MEGAKERNEL and stats["n_regions"] == 1 and not args.layers else None)
         roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                     "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)", "kernel": kernel_name}
