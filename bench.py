@@ -232,6 +232,26 @@ def algorithmic_bytes_per_step(shape, weight_bytes, batch, ctx_len):
     return weight_bytes + batch * (ctx_len * kv + kv)
 
 
+def slowest_rank_ms(total_ms, world, device):
+    """The job's time: the slowest rank's, agreed by every rank (each rank
+    calls this once, after its timed region), then a barrier."""
+    if world == 1:
+        return total_ms
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.barrier()
+    return float(t.item())
+
+
+def job_value(world, tokens_per_step, ms_per_step):
+    """Whole-job throughput: the tokens of all ranks (each runs the same
+    workload on its own sessions) over the slowest rank's time."""
+    return world * tokens_per_step / (ms_per_step / 1e3)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -361,13 +381,9 @@ def main():
                 torch.cuda.synchronize()
                 total_ms += t0.elapsed_time(t1)
                 dec_us += [a.elapsed_time(b) * 1e3 for a, b in evs]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        dist.barrier()
+    total_ms = slowest_rank_ms(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * tokens_per_step / (ms_per_step / 1e3)
+    value = job_value(world, tokens_per_step, ms_per_step)
 
     # roofline of the dominant kernel (the persistent decode program): bytes per
     # launch over the launch durations measured above
@@ -452,8 +468,8 @@ def main():
         decode()
         host_out.copy_(out_dev[: decode_steps + 1], non_blocking=True)
         torch.cuda.synchronize()
-    e2e_s = (time.perf_counter() - t0) / e2e_runs
-    line["e2e"] = {"value": world * tokens_per_step / e2e_s, "unit": "tokens/s",
+    e2e_s = slowest_rank_ms((time.perf_counter() - t0) / e2e_runs * 1e3, world, dev) / 1e3
+    line["e2e"] = {"value": job_value(world, tokens_per_step, e2e_s * 1e3), "unit": "tokens/s",
                    "h2d_bytes_per_step": int(host_prompt.numel() * 4),
                    "d2h_bytes_per_step": int(host_out.numel() * 4)}
 
