@@ -137,7 +137,9 @@ typedef struct wpk_plan_cfg {
                            Enough", Table I, producer-consumer overlap).  The
                            call returns with the caller's stream ordered after
                            the whole frame.  wpk_set_block_table is not
-                           supported then.                                      */
+                           supported then; the inspection calls (stats,
+                           edges, trace, program selection) see chunk 0's
+                           backbone program.                                    */
   int head_workers;     /* frame_chunks >= 2: worker CTAs of the head programs
                            (0 = half of the workers); the backbones take the
                            rest of n_workers (0 = #SMs x workers_per_sm)        */
