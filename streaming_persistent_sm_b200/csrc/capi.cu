@@ -1172,9 +1172,11 @@ static int chunked_prefill(wpk_handle* h, const int32_t* tokens_dev, int batch, 
     x->head->prefilled = true;
     int32_t* out = first_tok_dev ? first_tok_dev + r0 * K : codes;
     rc = head_frame(x, out, logits_dev ? logits_dev + r0 * K * V : nullptr, h->head_stream);
-    if (!rc && first_tok_dev)
-      CUDA_TRY(h, cudaMemcpyAsync(codes, out, (size_t)n[c] * K * 4, cudaMemcpyDeviceToDevice, h->head_stream));
-    if (x != h && rc) h->err = x->err;
+    if (!rc && first_tok_dev &&
+        cudaMemcpyAsync(codes, out, (size_t)n[c] * K * 4, cudaMemcpyDeviceToDevice, h->head_stream) != cudaSuccess)
+      rc = fail(h, WPK_ERR_CUDA, "copying a chunk's codes failed");
+    else if (x != h && rc)
+      h->err = x->err;
   }
   return chunk_join(h, s, rc);
 }
@@ -1289,9 +1291,11 @@ static int chunked_frame(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_
     }
     int32_t* out = out_tok_dev ? out_tok_dev + r0 * K : codes;
     rc = head_frame(x, out, logits_dev ? logits_dev + r0 * K * V : nullptr, h->head_stream);
-    if (!rc && out_tok_dev)
-      CUDA_TRY(h, cudaMemcpyAsync(codes, out, (size_t)x->batch * K * 4, cudaMemcpyDeviceToDevice, h->head_stream));
-    if (x != h && rc) h->err = x->err;
+    if (!rc && out_tok_dev &&
+        cudaMemcpyAsync(codes, out, (size_t)x->batch * K * 4, cudaMemcpyDeviceToDevice, h->head_stream) != cudaSuccess)
+      rc = fail(h, WPK_ERR_CUDA, "copying a chunk's codes failed");
+    else if (x != h && rc)
+      h->err = x->err;
   }
   return chunk_join(h, s, rc);
 }
