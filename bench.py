@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--resident", action="store_true", help="one resident grid serves every decode step")
     ap.add_argument("--split-pages", type=int, default=0)
+    ap.add_argument("--page-tokens", type=int, default=0, help="KV page size in tokens (0 = the plan's default)")
     ap.add_argument("--frame-chunks", type=int, default=0,
                     help="two-stage: split the batch into chunks whose backbone and head launches overlap")
     ap.add_argument("--head-workers", type=int, default=0, help="two-stage with --frame-chunks: the heads' workers")
@@ -293,7 +294,8 @@ def main():
                 prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
                          "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill],
                 resident=1 if args.resident else 0,
-                split_pages=args.split_pages, frame_chunks=args.frame_chunks, head_workers=args.head_workers)
+                split_pages=args.split_pages, page_tokens=args.page_tokens, frame_chunks=args.frame_chunks,
+                head_workers=args.head_workers)
     if args.regions:
         cuts = [int(x) for x in args.regions.split(",")]
         plan.update(n_regions=len(cuts), region_cut=tuple(cuts))
