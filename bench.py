@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--lookahead", type=int, default=0)
     ap.add_argument("--schedule", default="static", choices=["queue", "static"])
     ap.add_argument("--prefill", default="auto", choices=["auto", "mma", "tokenwise"])
+    ap.add_argument("--decode", default="auto", choices=["auto", "gemv", "mma"],
+                    help="decode program: CUDA-core GEMV tiles or tensor-core tiles (auto: by batch)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--resident", action="store_true", help="one resident grid serves every decode step")
     ap.add_argument("--split-pages", type=int, default=0)
@@ -188,6 +190,23 @@ def oracle_job_sample(wl, weights, n_steps: int):
     return t_prefill, statistics.median(times)
 
 
+def model_weight_bytes(model):
+    """bf16 bytes of every tensor of the model (the tied LM head once)."""
+    return 2 * sum(int(np.prod(shp)) for _, shp, _ in synth.tensor_specs(model))
+
+
+def workload_config(wl, prompt_len, decode_steps, layers=0):
+    """The workload a bench line measures - the same keys for both arms."""
+    _, with_prefill = job_tokens(wl, decode_steps)
+    wb = model_weight_bytes(wl.model)
+    l2 = ("inputs larger than L2 (126 MB): %.2f GB of weights streamed from HBM per step" % (wb / 1e9)
+          if wb > 126e6 else "weights fit in L2 (%.1f MB): latency-bound, no HBM claim" % (wb / 1e6))
+    return {"workload": wl.name + (f" ({layers} layers)" if layers else ""), "batch": wl.batch,
+            "prompt_len": prompt_len, "decode_steps": decode_steps,
+            "timed": "prefill + decode steps" if with_prefill else "decode steps (prompt prefilled untimed)",
+            "l2": l2}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -200,16 +219,19 @@ def run_reference(args):
     t_prefill, t_step = oracle_job_sample(wl, weights, args.warmup + args.steps)
     tokens, with_prefill = job_tokens(wl, decode_steps)
     per_seq = (t_prefill if with_prefill else 0.0) + decode_steps * t_step
-    value = tokens / (per_seq * wl.batch)  # the oracle runs the sequences one after another
+    job_s = per_seq * wl.batch  # the oracle runs the sequences one after another
+    value = tokens / job_s
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": job_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "prompt_len": wl.prompt_len, "decode_steps": decode_steps},
+        "config": workload_config(wl, wl.prompt_len, decode_steps),
+        "decode_step_us": {"median": t_step * 1e6},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"float64 NumPy oracle, one sequence: prefill of {wl.prompt_len} tokens "
                                    f"({t_prefill:.2f} s) and {args.steps} timed decode steps (median "
-                                   f"{t_step * 1e3:.0f} ms); job time extrapolated to {decode_steps} steps"},
+                                   f"{t_step * 1e3:.0f} ms); one bench step = the whole job (prefill and "
+                                   f"{decode_steps} steps for each of the {wl.batch} sequences), extrapolated"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -293,6 +315,7 @@ def main():
                 schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE,
                 prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
                          "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill],
+                decode={"auto": W.WPK_DECODE_AUTO, "gemv": W.WPK_DECODE_GEMV, "mma": W.WPK_DECODE_MMA}[args.decode],
                 resident=1 if args.resident else 0,
                 split_pages=args.split_pages, page_tokens=args.page_tokens, frame_chunks=args.frame_chunks,
                 head_workers=args.head_workers)
@@ -436,20 +459,18 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "accum_dtype": "fp32", "data": "synthetic",
-        "config": {"workload": wl.name + (f" ({s.n_layers} layers)" if args.layers else ""), "batch": B,
-                   "prompt_len": T, "decode_steps": decode_steps, "schedule": args.schedule,
-                   "timed": "prefill + decode steps" if with_prefill else "decode steps (prompt prefilled untimed)",
-                   "mode": args.mode + (" (resident grid)" if args.resident else ""),
-                   "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
-                   "prefill": "tensor-core prefill program" if prefill_tensor_cores else "token by token",
-                   "workers": stats["n_workers"],
-                   "l2": "inputs larger than L2: %.2f GB of weights streamed per step" % (stats["weight_bytes"] / 1e9),
-                   **({"codes_per_frame": K, "tokens": "codebook codes (a frame per sequence per step)"}
-                      if two else {}),
-                   **({"frame_chunks": n_chunks, "backbone_workers": stats["n_workers"],
-                       "head_workers": args.head_workers or (torch.cuda.get_device_properties(dev).multi_processor_count
-                                                             * max(1, args.workers_per_sm) - stats["n_workers"])}
-                      if chunks > 1 else {})},
+        "config": workload_config(wl, T, decode_steps, args.layers),
+        "plan": {"schedule": args.schedule,
+                 "mode": args.mode + (" (resident grid)" if args.resident else ""),
+                 "regions": stats["n_regions"], "tiles_per_step": stats["n_tiles"],
+                 "prefill": "tensor-core prefill program" if prefill_tensor_cores else "token by token",
+                 "workers": stats["n_workers"], "lookahead": args.lookahead or "library default (4)",
+                 **({"codes_per_frame": K, "tokens": "codebook codes (a frame per sequence per step)"}
+                    if two else {}),
+                 **({"frame_chunks": n_chunks, "backbone_workers": stats["n_workers"],
+                     "head_workers": args.head_workers or (torch.cuda.get_device_properties(dev).multi_processor_count
+                                                           * max(1, args.workers_per_sm) - stats["n_workers"])}
+                    if chunks > 1 else {})},
         "decode_step_us": decode_summary,
         "ttft_ms": statistics.median(pre_ms) if pre_ms else None,
         "roofline": roofline,

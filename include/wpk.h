@@ -318,11 +318,18 @@ int wpk_destroy(wpk_handle *h);
  * of the buffer bound by wpk_load_weights.  The paper has no counterpart;
  * this entry point exists for those callers only.
  *   - Every GPU that loads the library holds the 8 MiB until process exit.
- *   - Plans needing more scratch than 8 MiB (wpk_workspace_size) get
- *     WPK_ERR_SHAPE; the per-op graph mode gets WPK_ERR_UNSUPPORTED.
+ *   - The limit applies to the decode step's part of the scratch (the GEMV
+ *     decode buffers; about 6.9 MiB for the 1B shape at batch 48 and a
+ *     624-token context); the prefill program keeps using the caller's
+ *     buffer.  A larger decode scratch gets WPK_ERR_SHAPE.
+ *   - WPK_ERR_UNSUPPORTED for: the per-op graph mode (its captured graph
+ *     holds the scratch address), the resident grid (it keeps its scratch
+ *     pointer for its lifetime), the tensor-core decode program (it keeps
+ *     sums in its scratch between steps) and the two-stage model.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is cached per device: do not
+ *     use this entry point across a device reset.
  *   - All calls share the one array and it keeps the last call's contents;
  *     no part of it needs to start at zero (each step writes every scratch
  *     value before reading it).  Calls that overlap on the GPU, from any

@@ -77,6 +77,9 @@ struct wpk_handle {
   uint16_t* kv = nullptr;
   uint8_t* scratch = nullptr;
   size_t kv_bytes = 0, scratch_bytes = 0;
+  // the part of the scratch a GEMV decode step touches (its buffers are laid
+  // out first; prefill and tensor-core regions follow)
+  size_t decode_scratch_bytes = 0;
   size_t off_xa = 0, off_xb = 0, off_q = 0, off_attn = 0, off_h = 0, off_part = 0;
   // batched decode program: residual (feature-major), q/k/v sums, x^2 sums,
   // hi/lo images of x*g_attn, x*g_ffn, the attention output and h
@@ -294,6 +297,7 @@ void scratch_layout(wpk_handle* h) {
   h->off_attn = take(B * q_rows * 4);
   h->off_h = take(B * m.ffn * 4);
   h->off_part = take(B * m.n_kv_heads * g.n_splits * (m.n_heads / m.n_kv_heads) * (2 + m.head_dim) * 4);
+  h->decode_scratch_bytes = off;
   if (g.plan.prefill_mode == WPK_PREFILL_MMA) {
     // prefill of up to max_batch prompts of max_context tokens, in blocks of 128
     const size_t M = (size_t)g.plan.max_batch * g.plan.max_context;
@@ -1530,8 +1534,10 @@ int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes
   if (h->g.plan.decode_mode == WPK_DECODE_MMA)
     return fail(h, WPK_ERR_UNSUPPORTED, "wpk_step_noalloc needs the GEMV decode program (the tensor-core "
                                         "decode program keeps sums in its scratch between steps)");
-  if (h->scratch_bytes > scratch_bytes)
-    return fail(h, WPK_ERR_SHAPE, "the plan needs " + std::to_string(h->scratch_bytes) +
+  // only the decode step's part of the scratch moves into the static array;
+  // the prefill program keeps the caller's buffer
+  if (h->decode_scratch_bytes > scratch_bytes)
+    return fail(h, WPK_ERR_SHAPE, "the decode step needs " + std::to_string(h->decode_scratch_bytes) +
                                       " scratch bytes, more than the " + std::to_string(scratch_bytes) +
                                       " bytes of the static scratch array");
   if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");

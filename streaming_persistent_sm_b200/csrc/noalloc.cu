@@ -13,13 +13,17 @@
 // not this entry point is used.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "wpk_internal.h"
 
 extern "C" int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes,
                                          const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev,
                                          void* stream);
 
-// 8 MiB: the 1B shape at batch 48 with a 624-token context needs ~6.9 MiB.
+// 8 MiB: a GEMV decode step of the 1B shape at batch 48 with a 624-token
+// context needs ~6.9 MiB (only the decode step's scratch moves here; the
+// prefill program's buffers stay in the caller's scratch).
 static constexpr size_t kStaticScratchBytes = 8u << 20;
 static constexpr int kMaxDevices = 64;
 
@@ -28,7 +32,10 @@ static constexpr int kMaxDevices = 64;
 // cudaGetSymbolAddress below and is what the kernels receive.
 static __device__ __align__(256) uint8_t g_step_scratch[kStaticScratchBytes];
 
-static void* g_scratch_addr[kMaxDevices];  // device address of g_step_scratch, per device
+// Device address of g_step_scratch, per device, looked up by the first call
+// on that device.  A device reset (cudaDeviceReset) or a new primary context
+// may move the array: this entry point is not meant to be used across one.
+static std::atomic<void*> g_scratch_addr[kMaxDevices];
 
 extern "C" int wpk_step_noalloc(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev,
                                 void* stream) {
@@ -36,12 +43,12 @@ extern "C" int wpk_step_noalloc(wpk_handle* h, const int32_t* in_tok_dev, int32_
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return WPK_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return WPK_ERR_UNSUPPORTED;
-  if (!g_scratch_addr[dev]) {
-    // One-time set-up on this device (the device must be current).
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_step_scratch) != cudaSuccess || !p) return WPK_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void* addr = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!addr) {
+    // One-time set-up on this device (the device must be current).  Racing
+    // first callers on different host threads look up the same address.
+    if (cudaGetSymbolAddress(&addr, g_step_scratch) != cudaSuccess || !addr) return WPK_ERR_CUDA;
+    g_scratch_addr[dev].store(addr, std::memory_order_release);
   }
-  return wpk_internal_step_scratch(h, g_scratch_addr[dev], kStaticScratchBytes, in_tok_dev, out_tok_dev,
-                                   logits_dev, stream);
+  return wpk_internal_step_scratch(h, addr, kStaticScratchBytes, in_tok_dev, out_tok_dev, logits_dev, stream);
 }

@@ -1875,14 +1875,25 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
     }
   }
   __syncthreads();
-  // Drain: wait (bounded) for chunks issued but never consumed.
+  // Drain: wait (bounded) for chunks issued but never consumed.  Every copy
+  // reads a valid global range, so it lands; the bound is a guard only.  If it
+  // ever runs out, the error word says so (the handle is then poisoned) before
+  // the CTA leaves with that copy still counted as in flight.
   if (threadIdx.x == 0) {
     for (uint32_t c = s_cons_chunks; c < s_prod_chunks; ++c) {
       const int s = c % P.n_stages;
       const uint32_t par = (c / P.n_stages) & 1u;
       const uint64_t t0 = globaltimer();
+      bool landed = true;
       while (!mbar_try_wait(&S.full[s], par))
-        if (globaltimer() - t0 > P.timeout_ns) break;
+        if (globaltimer() - t0 > P.timeout_ns) {
+          landed = false;
+          break;
+        }
+      if (!landed) {
+        record_error(P, WPK_ERR_TIMEOUT, 0xFFFFFFFEu, kNoCounter, c, s_prod_chunks);
+        break;
+      }
     }
   }
   if (P.uses_tmem) {

@@ -28,13 +28,18 @@ def dec(weights):
 
 
 def test_llama1b_b1_prefill_and_steps(weights, dec):
+    # the bench's job in the bench's launch configuration (static schedule):
+    # prefill and all 128 steps, to context 623, so the attention splits past
+    # the 512- and 576-token page boundaries hold data; every 8th step and the
+    # last are compared on all 128256 logits (the oracle runs every step)
     wl = synth.WORKLOADS["llama1b_b1"]
     ctx = wl.prompt_len + wl.steps
-    eng = W.Engine(S, weights, 1, ctx)
+    eng = W.Engine(S, weights, 1, ctx, schedule=W.WPK_SCHED_STATIC)
     try:
         prompts = synth.make_prompts(S.vocab, 1, wl.prompt_len, wl.prompt_seed)
-        worst = run_teacher_forced(eng, dec, prompts, steps=6, max_context=ctx)
-        print("worst per step:", worst)
+        worst = run_teacher_forced(eng, dec, prompts, steps=wl.steps, max_context=ctx, check_every=8)
+        assert len(worst) == 1 + wl.steps // 8 + (1 if (wl.steps - 1) % 8 else 0)
+        print("worst per checked step:", worst)
     finally:
         eng.close()
 
@@ -58,6 +63,21 @@ def test_llama1b_batched_sampled_rows(weights, dec, B, decode):
     try:
         prompts = synth.make_prompts(S.vocab, B, wl.prompt_len, wl.prompt_seed)
         run_teacher_forced(eng, dec, prompts, steps=3, max_context=ctx, rows=[0, B // 2, B - 1])
+    finally:
+        eng.close()
+
+
+def test_llama1b_decode_b32_sampled_rows(weights, dec):
+    # the C3 shape at batch 32 in the bench's configuration (tensor-core
+    # decode, static schedule): 24 steps, rows {0, 16, 31}
+    wl = synth.WORKLOADS["llama1b_decode_b32"]
+    B = wl.batch
+    ctx = wl.prompt_len + wl.steps
+    eng = W.Engine(S, weights, B, ctx, schedule=W.WPK_SCHED_STATIC)
+    try:
+        assert "b_qkv" in [W.OP_NAMES[o] for o in W.wpk_get_tile_ops(eng.h, eng.stats["n_tiles"])]
+        prompts = synth.make_prompts(S.vocab, B, wl.prompt_len, wl.prompt_seed)
+        run_teacher_forced(eng, dec, prompts, steps=24, max_context=ctx, check_every=4, rows=[0, B // 2, B - 1])
     finally:
         eng.close()
 

@@ -65,6 +65,17 @@ def test_batched_decode_ragged(weights, dec, plan_b, active, T):
         eng.close()
 
 
+def test_batched_decode_at_the_maximum_batch(weights, dec):
+    # the largest tensor-core N: a plan of 128 sequences (two 128-row hi/lo
+    # images per stage), 117 of them active, prompts ending inside a page
+    eng = W.Engine(S, weights, 128, CTX, decode=W.WPK_DECODE_MMA)
+    try:
+        assert "b_qkv" in [W.OP_NAMES[o] for o in W.wpk_get_tile_ops(eng.h, eng.stats["n_tiles"])]
+        run_teacher_forced(eng, dec, _prompts(117, 23, seed=117), steps=6, max_context=CTX)
+    finally:
+        eng.close()
+
+
 def test_batched_decode_matches_gemv_program(weights):
     # the tensor-core and the CUDA-core decode programs agree with each other
     # as closely as each agrees with the oracle
