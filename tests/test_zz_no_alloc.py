@@ -47,6 +47,36 @@ def test_noalloc_step_matches_step_on_two_calls_in_a_row():
         eng.close()
 
 
+def test_noalloc_step_on_the_1b_shape_with_the_default_plan():
+    # the default plan prefills on tensor cores, whose scratch is far larger
+    # than the static array; only the decode step's scratch moves there
+    import torch
+
+    s = synth.LLAMA_1B
+    w = synth.cached_weights(s, seed=0)
+    prompts = synth.make_prompts(s.vocab, 1, 64, seed=1001)
+    ref = W.Engine(s, w, 1, 624)
+    eng = W.Engine(s, w, 1, 624)
+    try:
+        _, _, scratch = W.wpk_workspace_size(eng.h)
+        assert scratch > (8 << 20)  # the whole plan would not fit
+        first_ref, _ = ref.prefill(prompts)
+        eng.prefill(prompts)
+        tok = first_ref.clone()
+        stream = torch.cuda.current_stream().cuda_stream
+        for call in range(2):
+            out_ref, lg_ref = ref.step(tok, want_logits=True)
+            out = torch.empty(1, dtype=torch.int32, device="cuda")
+            lg = torch.empty((1, s.vocab), dtype=torch.float32, device="cuda")
+            W.wpk_step_noalloc(eng.h, tok.data_ptr(), out.data_ptr(), lg.data_ptr(), stream)
+            torch.cuda.synchronize()
+            check_logits(lg.cpu().numpy(), lg_ref.cpu().numpy(), out.cpu().numpy(), f"call {call}")
+            tok = out_ref.clone()
+    finally:
+        ref.close()
+        eng.close()
+
+
 def test_noalloc_step_rejects_plans_larger_than_the_static_array():
     # 2048 sequences of the tiny shape need ~16 MiB of scratch (> 8 MiB)
     eng = W.Engine(S, synth.make_weights(S, seed=0), 2048, 64)
