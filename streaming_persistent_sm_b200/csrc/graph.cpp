@@ -43,6 +43,10 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
     return "model dimensions must be positive";
   if (m.n_heads % m.n_kv_heads) return "n_heads must be a multiple of n_kv_heads";
   if (m.n_heads / m.n_kv_heads > kMaxGroup) return "more than 8 query heads per kv head";
+  {  // decode attention serves a kv group's heads in at most two head groups of <= 4
+    const int grp = m.n_heads / m.n_kv_heads;
+    if (grp > 4 && grp % 2) { *code = WPK_ERR_UNSUPPORTED; return "query heads per kv head must be 1-4, 6 or 8"; }
+  }
   if (m.head_dim != 64) { *code = WPK_ERR_UNSUPPORTED; return "head_dim must be 64"; }
   if (m.hidden % 8 || m.ffn % 8) { *code = WPK_ERR_SHAPE; return "hidden and ffn must be multiples of 8"; }
   if (m.hidden > 2048 * 4) { *code = WPK_ERR_UNSUPPORTED; return "hidden > 8192"; }
@@ -80,7 +84,11 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   const int kmax = std::max(std::max(m.hidden, q_rows), std::min(m.ffn, 2048));
   if (kmax > 2048) { *code = WPK_ERR_UNSUPPORTED; return "hidden and n_heads*head_dim must be <= 2048"; }
   const int kmax_pad = (kmax + 255) / 256 * 256;  // staged rows are padded to whole 256-column segments
-  p->act_bytes = std::max(16384, std::min(in.max_batch, kMaxGemvBatch) * kmax_pad * 4);
+  // the decode attention tiles use the same buffer: q, the current k/v, each
+  // warp's per-head (m, l, o) and probabilities
+  const int grp = m.n_heads / m.n_kv_heads;
+  const int attn_need = (kMaxGroup * kHeadDim + 2 * kHeadDim + kWarps * grp * (2 + kHeadDim) + kWarps * 32 * grp) * 4;
+  p->act_bytes = std::max(std::max(16384, attn_need), std::min(in.max_batch, kMaxGemvBatch) * kmax_pad * 4);
   p->act_bytes = (p->act_bytes + 1023) / 1024 * 1024;
   const int fixed = 4096 + 1024;  // partial outputs, tile queue, barriers
   const int budget = std::min(kMaxSmem, 233472 / p->workers_per_sm - 1024) - p->act_bytes - fixed;
@@ -130,8 +138,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
       p->dec_stage_bytes = kMmaChunkBytes + 2 * p->dec_n * 128;
       // attention scratch: queries, one page of scores, the combine's (m, l) pairs
       const int max_pages = (in.max_context + p->page_tokens - 1) / p->page_tokens;
-      const int need = std::max((kMaxGroup * kHeadDim + 2 * kHeadDim + kWarps * (2 + kHeadDim)) * 4,
-                                max_pages * kMaxGroup * 2 * 4);
+      const int need = std::max(attn_need, max_pages * kMaxGroup * 2 * 4);
       p->dec_act_bytes = std::max(16384, (need + 1023) / 1024 * 1024);
       const int room = kMaxSmem - fixed - 4096 - p->dec_act_bytes;  // 4 KB: the kernel's static shared memory
       int want = in.slot_bytes ? in.slot_bytes / kStageBytes : 12;
@@ -350,9 +357,11 @@ std::vector<LmTile> gemv_lm_tiles(const wpk_model_cfg& m, const Plan& p, int W, 
 }
 
 // K splits of a tensor-core op with `rb` blocks of 128 rows and `nkc` 64-column
-// chunks: enough tiles for every worker, none smaller than tile_bytes.
+// chunks: as many tiles as fit the workers in one round (rb x splits <= W, so
+// that no worker runs two tiles of the op while another idles), none smaller
+// than tile_bytes.
 int mma_splits(int rb, int nkc, const Plan& p, int W) {
-  const int want = (W + rb - 1) / rb;
+  const int want = std::max(1, W / rb);
   const int most = std::max(1, nkc * kMmaChunkBytes / std::max(p.tile_bytes, kMmaChunkBytes));
   return std::max(1, std::min(std::min(want, most), nkc));
 }
@@ -735,8 +744,14 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerDev& d = dec.lay.layers[l];
     layer_begin[l] = (uint32_t)Tl.size();
-    for (int tb = 0; tb < nq; ++tb)
-      add(OP_NORM, l, 0, 0, tb, 0, 0, h, {blk(BUF_PX, h, tb, 0, h, 0), blk(BUF_PXN, h, tb, 0, h, 1)});
+    // RMSNorm tiles of kNormRows rows; the tiles of one block form one write
+    auto norms = [&](int which) {
+      for (int tb = 0; tb < nq; ++tb)
+        for (int r0 = 0; r0 < kTokBlock; r0 += kNormRows)
+          add(OP_NORM, l, 0, 0, tb, which, r0, h,
+              {blk(BUF_PX, h, tb, 0, h, 0), blk(BUF_PXN, h, tb, 0, h, 1, 100000 + (2 * l + which) * nq + tb)});
+    };
+    norms(0);
     // QKV: feature blocks of 128 rows; never straddle q/k/v (all multiples of 128)
     for (int tb = 0; tb < nq; ++tb)
       for (int fb = 0; fb < qkv_rows / 128; ++fb) {
@@ -777,8 +792,7 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
               c0 * 64, (c1 - c0) * 64,
               {blk(BUF_PATT, q_rows, tb, c0 * 64, c1 * 64, 0), blk(BUF_PX, h, tb, fb * 128, fb * 128 + 128, 2)});
         }
-    for (int tb = 0; tb < nq; ++tb)
-      add(OP_NORM, l, 0, 0, tb, 1, 0, h, {blk(BUF_PX, h, tb, 0, h, 0), blk(BUF_PXN, h, tb, 0, h, 1)});
+    norms(1);
     for (int tb = 0; tb < nq; ++tb)
       for (int fb = 0; fb < 2 * m.ffn / 128; ++fb)
         add(OP_MGU, l, d.mma_gu + (uint64_t)fb * (h / 64) * chunk, (uint32_t)(h / 64) * chunk, fb, tb, 0, h,

@@ -265,6 +265,17 @@ __device__ __forceinline__ const uint8_t* mma_act_src(const KParams& P, const Ti
   return img[part] + ((size_t)T.a1 * (k_full / 64) + T.a2 / 64) * P.act_chunk;
 }
 
+// Order in which a tensor-core tile walks its K chunks: rotated by the tile's
+// row block, so that tiles running at the same time copy different activation
+// chunks (every tile of an op reads the same activation image; in lockstep
+// they would all hit the same L2 lines at once).  The sum over K is the same;
+// only the fp32 summation order differs between tiles.
+__device__ __forceinline__ int mma_chunk_of(const Tile& T, int k, int nch) {
+  const int rot = nch > 1 ? (int)((uint32_t)T.a0 % (uint32_t)nch) : 0;
+  const int kr = k + rot;
+  return kr >= nch ? kr - nch : kr;
+}
+
 // Tensor-core tile chunk k: arm the barrier with all its bytes and copy the
 // weight block (the activation blocks follow in issue_mma_act).  A stage holds
 // the 16 KB weight block, then the hi and the lo activation chunk.
@@ -719,6 +730,158 @@ __device__ __forceinline__ void attn_result(const KParams& P, int b, int f, floa
   }
 }
 
+// Scores and P.V of one 32-token block of a staged KV page for all GRP query
+// heads of the kv group, by one warp: lane t scores token t against every head
+// (its K row is read once), then lane l accumulates head dims 2l, 2l+1 of every
+// head over the block's tokens (each V row is read once, the probabilities come
+// from a per-warp shared array).  `skip` is the block row holding the stale
+// copy of the current token (its score is left out and its V row is read as
+// zero); `cnt` rows of the block are valid.
+template <int GRP>
+__device__ __forceinline__ void attn_block(const uint8_t* krows, const uint8_t* vrows, int cnt, int skip,
+                                           const float* q_perm, float scale, float* p_w, float (&m)[GRP],
+                                           float (&l)[GRP], float (&o0)[GRP], float (&o1)[GRP]) {
+  const int lane = threadIdx.x & 31;
+  const bool valid = lane < cnt && lane != skip;
+  float sc[GRP];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) sc[h] = 0.f;
+  if (valid) {
+    const uint4* kr = reinterpret_cast<const uint4*>(krows + (size_t)lane * kHeadDim * 2);
+#pragma unroll
+    for (int u = 0; u < kHeadDim / 8; ++u) {
+      const int uu = (u + lane) & (kHeadDim / 8 - 1);  // rotated: neighbouring lanes, other banks
+      float kf[8];
+      unpack8(kr[uu], kf);
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        // q is stored [head][half][unit][4]: the 8 lanes of a phase read 8
+        // consecutive 16-byte units (no bank conflict)
+        const float4 qa = *reinterpret_cast<const float4*>(q_perm + h * kHeadDim + 4 * uu);
+        const float4 qb = *reinterpret_cast<const float4*>(q_perm + h * kHeadDim + 32 + 4 * uu);
+        sc[h] = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], sc[h]))));
+        sc[h] = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], sc[h]))));
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    const float s_h = valid ? sc[h] * scale : -INFINITY;
+    const float m_new = fmaxf(m[h], warp_max(s_h));
+    float pp = 0.f, corr = 1.f;
+    if (m_new != -INFINITY) {  // warp-uniform
+      corr = expf(m[h] - m_new);
+      pp = valid ? expf(s_h - m_new) : 0.f;
+      m[h] = m_new;
+    }
+    l[h] = l[h] * corr + warp_sum(pp);
+    o0[h] *= corr;
+    o1[h] *= corr;
+    p_w[lane * GRP + h] = pp;
+  }
+  __syncwarp();
+  const uint32_t* vrow = reinterpret_cast<const uint32_t*>(vrows) + lane;
+  for (int j = 0; j < cnt; ++j) {
+    const uint32_t vv = (j == skip) ? 0u : vrow[(size_t)j * (kHeadDim / 2)];
+    const float v0 = __uint_as_float(vv << 16), v1 = __uint_as_float(vv & 0xFFFF0000u);
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      const float pj = p_w[j * GRP + h];  // same address in every lane: a broadcast
+      o0[h] = fmaf(pj, v0, o0[h]);
+      o1[h] = fmaf(pj, v1, o1[h]);
+    }
+  }
+  __syncwarp();
+}
+
+// The page loop of a decode attention tile.  The group's query heads are cut
+// into head groups of GRP heads (one head group when the kv group has at most
+// four heads, two otherwise), each served by `wpg` warps: warp w attends with
+// heads [head0, head0 + GRP) over the tile's 32-token blocks wi, wi + wpg, ...
+// (wi = w mod wpg); its per-head state (m, l, o) goes to st_s[w][h] for the
+// merge.
+template <int GRP>
+__device__ bool attn_pages(const KParams& P, const AttnSpan& s, const Shared& Sh, Cursor& cur, int n_chunks,
+                           volatile int* abort, const float* q_perm, const float* kv_cur, float* st_s, float* p_s,
+                           uint32_t* page_rel, bool has_cur, int wpg) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wi = warp % wpg, head0 = (warp / wpg) * GRP;
+  q_perm += head0 * kHeadDim;
+  const int page = P.page_tokens, hd = kHeadDim;
+  const float scale = 1.0f / sqrtf((float)hd);
+  float m[GRP], l[GRP], o0[GRP], o1[GRP];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+    o0[h] = 0.f;
+    o1[h] = 0.f;
+  }
+  float* p_w = p_s + warp * 32 * GRP;
+  bool ok = true;
+  for (int k = 0; k < n_chunks; ++k) {  // page k of the split, one ring stage each
+    const uint32_t c = cur.c + k;
+    const int st = c % P.n_stages;
+    const int p0 = (s.t0 / page + k) * page;
+    const int n = min(page, s.t1 - p0);
+    const int nblk = (n + 31) / 32;
+    // blocks are numbered across the tile's pages so that every warp gets work
+    const int first = (k * ((page + 31) / 32)) % wpg;
+    const int mine = (wi - first + wpg) % wpg;  // this warp's first block in the page
+    // every warp waits for every page, also one without a block for it: a
+    // parity wait only tells a phase from the one before it, so no warp may
+    // run a whole ring ahead of a stage it has not seen land
+    if (ok && !wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu)) ok = false;
+    if (mine < nblk) {
+      if (ok) {
+        const uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
+        for (int b = mine; b < nblk; b += wpg) {
+          const int cnt = min(32, n - b * 32);
+          // the staged copy of the current token's row is stale (it was copied
+          // before this step wrote it): leave it out, read zeros for its V
+          const int rel = s.pos - p0 - b * 32;
+          const int skip = (rel >= 0 && rel < 32) ? rel : -1;
+          attn_block<GRP>(stage + (size_t)b * 32 * hd * 2, stage + (size_t)page * hd * 2 + (size_t)b * 32 * hd * 2,
+                          cnt, skip, q_perm, scale, p_w, m, l, o0, o1);
+        }
+      }
+    }
+    // the last warp to finish with the page hands the stage back
+    __syncwarp();
+    if (lane == 0) {
+      const uint32_t r = atomicAdd(&page_rel[st], 1u) + 1u;
+      if (r == (uint32_t)kWarps * (uint32_t)(k / P.n_stages + 1)) mbar_arrive(&Sh.empty[st]);
+    }
+  }
+  cur.c += n_chunks;
+  if (has_cur && wi == 0) {  // the current token, read from where this step wrote it
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      const int u0 = (2 * lane) >> 3, e0 = (2 * lane) & 7;  // dims 2 lane, 2 lane + 1 in the permuted q
+      const float* qh = q_perm + h * hd;
+      const float qd0 = qh[(e0 >> 2) * 32 + 4 * u0 + (e0 & 3)], qd1 = qh[(e0 >> 2) * 32 + 4 * u0 + (e0 & 3) + 1];
+      const float sc = warp_sum(qd0 * kv_cur[2 * lane] + qd1 * kv_cur[2 * lane + 1]) * scale;
+      const float m_new = fmaxf(m[h], sc);
+      const float corr = expf(m[h] - m_new), pp = expf(sc - m_new);
+      l[h] = l[h] * corr + pp;
+      o0[h] = o0[h] * corr + pp * kv_cur[hd + 2 * lane];
+      o1[h] = o1[h] * corr + pp * kv_cur[hd + 2 * lane + 1];
+      m[h] = m_new;
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    float* mine = st_s + (warp * GRP + h) * (2 + kHeadDim);
+    mine[2 + 2 * lane] = o0[h];
+    mine[3 + 2 * lane] = o1[h];
+    if (lane == 0) {
+      mine[0] = m[h];
+      mine[1] = l[h];
+    }
+  }
+  return ok;
+}
+
 __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cursor& cur, int n_chunks,
                           volatile int* abort) {
   if (T.a0 >= active_batch(P)) return true;
@@ -728,18 +891,21 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   const int hd = P.head_dim, grp = P.group, page = P.page_tokens;
   const int nq = grp * hd;
   float* part = P.part + ((((size_t)s.b * P.n_kv + s.g) * P.n_splits + s.j) * grp) * (2 + hd);
-  float* q_s = Sh.act;                          // [grp][hd]
-  float* kv_cur = Sh.act + kMaxGroup * hd;      // [2][hd]: the current token's k and v
-  float* st_s = kv_cur + 2 * kHeadDim;          // [kWarps][2 + hd]: each warp's (m, l, o)
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // warp w attends with query head w % grp over every parts-th 32-token block
-  const int parts = kWarps / grp;
-  const int head = warp % grp, prt = warp / grp;
-  const float scale = 1.0f / sqrtf((float)hd);
+  // shared scratch (the activation buffer): q permuted per head as
+  // [half][unit][4], the current token's k and v, each warp's per-head
+  // (m, l, o), each warp's probabilities [32][grp]
+  float* q_perm = Sh.act;                          // [grp][hd]
+  float* kv_cur = q_perm + kMaxGroup * hd;         // [2][hd]
+  float* st_s = kv_cur + 2 * kHeadDim;             // [kWarps][grp][2 + hd]
+  float* p_s = st_s + kWarps * grp * (2 + kHeadDim);  // [kWarps][32][grp]
   const bool has_cur = s.pos >= s.t0 && s.pos < s.t1;
-  for (int i = threadIdx.x; i < nq; i += kThreads)
-    q_s[i] = P.dec_mma ? __ldcg(P.acc + (size_t)(s.g * nq + i) * P.mma_n + s.b)
-                       : __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * nq + i);
+  (void)page;
+  for (int i = threadIdx.x; i < nq; i += kThreads) {
+    const float v = P.dec_mma ? __ldcg(P.acc + (size_t)(s.g * nq + i) * P.mma_n + s.b)
+                              : __ldcg(P.qbuf + (size_t)s.b * P.q_rows + (size_t)s.g * nq + i);
+    const int h = i / hd, d = i % hd, u = d >> 3, e = d & 7;
+    q_perm[h * hd + (e >> 2) * 32 + 4 * u + (e & 3)] = v;
+  }
   // the current token's k and v were produced this step, after its page was
   // copied: read them directly (tensor-core decode: round the fp32 sums to the
   // cache's bf16 here, store them and clear the sums)
@@ -760,97 +926,28 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   }
   if (threadIdx.x < kMaxStages) s_page_rel[threadIdx.x] = 0;
   cbar();
-  const float* qh = q_s + head * hd;
-  float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;  // this warp's state; lane holds dims 2 lane, 2 lane + 1
-  bool ok = true;
-  for (int k = 0; k < n_chunks; ++k) {  // page k of the split, one ring stage each
-    const uint32_t c = cur.c + k;
-    const int st = c % P.n_stages;
-    if (ok && !wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu)) ok = false;
-    if (ok) {
-      if (P.trace && threadIdx.x == 0 && k + 1 == n_chunks) s_t_data = globaltimer();
-      const uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
-      const int p0 = (s.t0 / page + k) * page;
-      const int n = min(page, s.t1 - p0);
-      const int blk0 = (p0 - s.t0) / 32;
-      for (int b = 0; b * 32 < n; ++b) {
-        if ((blk0 + b) % parts != prt) continue;
-        const int t = b * 32 + lane;
-        const bool valid = t < n && p0 + t != s.pos;
-        float sc = -INFINITY;
-        if (valid) {
-          const uint4* kr = reinterpret_cast<const uint4*>(stage + (size_t)t * hd * 2);
-          float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-          for (int u = 0; u < kHeadDim / 8; ++u) {
-            const int uu = (u + lane) & (kHeadDim / 8 - 1);  // rotated: neighbouring lanes, other banks
-            float kf[8];
-            unpack8(kr[uu], kf);
-            const float4 qa = *reinterpret_cast<const float4*>(qh + 8 * uu);
-            const float4 qb = *reinterpret_cast<const float4*>(qh + 8 * uu + 4);
-            a0 = fmaf(qa.x, kf[0], fmaf(qa.y, kf[1], fmaf(qa.z, kf[2], fmaf(qa.w, kf[3], a0))));
-            a1 = fmaf(qb.x, kf[4], fmaf(qb.y, kf[5], fmaf(qb.z, kf[6], fmaf(qb.w, kf[7], a1))));
-          }
-          sc = (a0 + a1) * scale;
-        }
-        const float m_new = fmaxf(m, warp_max(sc));
-        if (m_new == -INFINITY) continue;  // no valid token yet (warp-uniform)
-        const float corr = expf(m - m_new);
-        const float pp = valid ? expf(sc - m_new) : 0.f;
-        l = l * corr + warp_sum(pp);
-        o0 *= corr;
-        o1 *= corr;
-        const uint32_t* vrow = reinterpret_cast<const uint32_t*>(stage + (size_t)page * hd * 2 + (size_t)b * 32 * hd * 2) + lane;
-        const int cnt = min(32, n - b * 32);
-        // the staged copy of the current token's row is stale (it was copied
-        // before this step wrote it): read zeros there, never its bytes
-        const int stale = s.pos - p0 - b * 32;
-        for (int j = 0; j < cnt; ++j) {
-          const float pj = __shfl_sync(0xffffffffu, pp, j);
-          const uint32_t vv = (j == stale) ? 0u : vrow[(size_t)j * (hd / 2)];
-          o0 = fmaf(pj, __uint_as_float(vv << 16), o0);
-          o1 = fmaf(pj, __uint_as_float(vv & 0xFFFF0000u), o1);
-        }
-        m = m_new;
-      }
-    }
-    // the last warp to finish with the page hands the stage back
-    __syncwarp();
-    if (lane == 0) {
-      const uint32_t r = atomicAdd(&s_page_rel[st], 1u) + 1u;
-      if (r == (uint32_t)kWarps * (uint32_t)(k / P.n_stages + 1)) mbar_arrive(&Sh.empty[st]);
-    }
+  // head groups: all heads at once up to four, else two halves (6 or 8 heads)
+  const int hg = grp <= 4 ? grp : grp / 2;
+  const int wpg = grp <= 4 ? kWarps : kWarps / 2;
+  bool ok;
+  switch (hg) {
+    case 1: ok = attn_pages<1>(P, s, Sh, cur, n_chunks, abort, q_perm, kv_cur, st_s, p_s, s_page_rel, has_cur, wpg); break;
+    case 2: ok = attn_pages<2>(P, s, Sh, cur, n_chunks, abort, q_perm, kv_cur, st_s, p_s, s_page_rel, has_cur, wpg); break;
+    case 3: ok = attn_pages<3>(P, s, Sh, cur, n_chunks, abort, q_perm, kv_cur, st_s, p_s, s_page_rel, has_cur, wpg); break;
+    default: ok = attn_pages<4>(P, s, Sh, cur, n_chunks, abort, q_perm, kv_cur, st_s, p_s, s_page_rel, has_cur, wpg); break;
   }
-  cur.c += n_chunks;
   if (!cbar_and(ok)) return false;
-  if (has_cur && prt == 0) {  // the current token, once per head
-    float d = qh[2 * lane] * kv_cur[2 * lane] + qh[2 * lane + 1] * kv_cur[2 * lane + 1];
-    const float sc = warp_sum(d) * scale;
-    const float m_new = fmaxf(m, sc);
-    const float corr = expf(m - m_new), pp = expf(sc - m_new);
-    l = l * corr + pp;
-    o0 = o0 * corr + pp * kv_cur[kHeadDim + 2 * lane];
-    o1 = o1 * corr + pp * kv_cur[kHeadDim + 2 * lane + 1];
-    m = m_new;
-  }
-  float* mine = st_s + warp * (2 + kHeadDim);
-  mine[2 + 2 * lane] = o0;
-  mine[3 + 2 * lane] = o1;
-  if (lane == 0) {
-    mine[0] = m;
-    mine[1] = l;
-  }
-  cbar();
-  // merge the parts of each head; one split: the result directly, else the
+  // merge the warps of each head; one split: the result directly, else the
   // split's partial (m, l, o) for the combine
   for (int i = threadIdx.x; i < nq; i += kThreads) {
     const int hh = i / hd, d = i % hd;
+    const int w0 = (hh / hg) * wpg, hl = hh % hg;  // the warps serving head hh, its slot in their state
     float M = -INFINITY;
-    for (int q = 0; q < parts; ++q) M = fmaxf(M, st_s[(q * grp + hh) * (2 + kHeadDim)]);
+    for (int q = w0; q < w0 + wpg; ++q) M = fmaxf(M, st_s[(q * hg + hl) * (2 + kHeadDim)]);
     float L = 0.f, O = 0.f;
     if (M != -INFINITY)
-      for (int q = 0; q < parts; ++q) {
-        const float* w = st_s + (q * grp + hh) * (2 + kHeadDim);
+      for (int q = w0; q < w0 + wpg; ++q) {
+        const float* w = st_s + (q * hg + hl) * (2 + kHeadDim);
         const float f = expf(w[0] - M);
         L = fmaf(w[1], f, L);
         O = fmaf(w[2 + d], f, O);
@@ -956,7 +1053,7 @@ __device__ bool body_norm(const KParams& P, const Tile& T) {
   uint8_t* hi = P.xn_img[0] + (size_t)tb * nkc * kMmaChunkBytes;
   uint8_t* lo = P.xn_img[1] + (size_t)tb * nkc * kMmaChunkBytes;
   constexpr int kMaxUnits = 2048 / 8 / 32;
-  for (int n = warp; n < kTokBlock; n += kWarps) {
+  for (int n = T.a2 + warp; n < T.a2 + kNormRows; n += kWarps) {  // the tile's rows of the block
     const int m = tb * kTokBlock + n;
     const bool valid = m < P.M;
     float xr[kMaxUnits][8];
@@ -1346,12 +1443,19 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
         const int j = j0 + jj;
         float acc = 0.f;
         if (j < rows) {
-          const uint32_t* kr = Kw + j * (hd / 2);
+          // the thread's 32 dims of key j: four 16-byte loads (a broadcast
+          // across the threads of the same half)
+          const uint4* kr = reinterpret_cast<const uint4*>(Kw + j * (hd / 2));
 #pragma unroll
-          for (int w = 0; w < 16; ++w) {
-            const uint32_t kk = kr[w];
-            acc = fmaf(q[2 * w], __uint_as_float(kk << 16), acc);
-            acc = fmaf(q[2 * w + 1], __uint_as_float(kk & 0xFFFF0000u), acc);
+          for (int w4 = 0; w4 < 4; ++w4) {
+            const uint4 k4 = kr[w4];
+            const uint32_t kw[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int w = 4 * w4 + e;
+              acc = fmaf(q[2 * w], __uint_as_float(kw[e] << 16), acc);
+              acc = fmaf(q[2 * w + 1], __uint_as_float(kw[e] & 0xFFFF0000u), acc);
+            }
           }
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
@@ -1369,12 +1473,17 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
       for (int jj = 0; jj < 16; ++jj) {
         const float p = (sc[jj] == -INFINITY) ? 0.f : expf(sc[jj] - mnew);
         lrun += p;
-        const uint32_t* vr = Vw + min(j0 + jj, rows - 1) * (hd / 2);
+        const uint4* vr = reinterpret_cast<const uint4*>(Vw + min(j0 + jj, rows - 1) * (hd / 2));
 #pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          const uint32_t vv = vr[w];
-          o[2 * w] = fmaf(p, __uint_as_float(vv << 16), o[2 * w]);
-          o[2 * w + 1] = fmaf(p, __uint_as_float(vv & 0xFFFF0000u), o[2 * w + 1]);
+        for (int w4 = 0; w4 < 4; ++w4) {
+          const uint4 v4 = vr[w4];
+          const uint32_t vw[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int w = 4 * w4 + e;
+            o[2 * w] = fmaf(p, __uint_as_float(vw[e] << 16), o[2 * w]);
+            o[2 * w + 1] = fmaf(p, __uint_as_float(vw[e] & 0xFFFF0000u), o[2 * w + 1]);
+          }
         }
       }
       mrun = mnew;
@@ -1688,18 +1797,20 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           const uint32_t c0 = c;
           for (int k = 0; k < pre && !stop; ++k, ++c) {
             if (!free_stage(c)) { stop = true; break; }
-            issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
+            issue_mma_w(P, T, mma_chunk_of(T, k, nch), stage_ptr(c), &S.full[c % P.n_stages]);
           }
           // (per-op launches get their order from the stream; no counters run)
           if (!stop && !P.per_op && !wait_counter(P, T, t, e.epoch, &s_abort)) stop = true;
           if (!stop) {
             fence_proxy_async_global();
-            for (int k = 0; k < pre; ++k) issue_mma_act(P, T, k, stage_ptr(c0 + k), &S.full[(c0 + k) % P.n_stages]);
+            for (int k = 0; k < pre; ++k)
+              issue_mma_act(P, T, mma_chunk_of(T, k, nch), stage_ptr(c0 + k), &S.full[(c0 + k) % P.n_stages]);
           }
           for (int k = pre; k < nch && !stop; ++k, ++c) {
             if (!free_stage(c)) { stop = true; break; }
-            issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
-            issue_mma_act(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
+            const int kc = mma_chunk_of(T, k, nch);
+            issue_mma_w(P, T, kc, stage_ptr(c), &S.full[c % P.n_stages]);
+            issue_mma_act(P, T, kc, stage_ptr(c), &S.full[c % P.n_stages]);
           }
         } else {
           if (T.op == OP_PATTN) {  // its KV pages are written inside this program

@@ -51,6 +51,7 @@ enum Op : uint16_t {
 
 constexpr int kTokBlock = 128;   // tokens per tensor-core tile (the MMA N)
 constexpr int kPrefillQB = 32;   // queries per prefill attention tile
+constexpr int kNormRows = 16;    // token rows per prefill RMSNorm tile
 constexpr int kMaxMmaBatch = 128;  // sequences of a batched decode step (MMA N <= 128)
 constexpr int kMaxInTables = 16;   // input tables a step's input may sum over
 constexpr int kMmaChunkBytes = 128 * 128;  // 128 rows x 64 bf16, one K chunk

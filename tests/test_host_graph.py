@@ -174,7 +174,8 @@ def test_prefill_program_verifies_and_simulates(lib, B, T):
         assert np.all(e[:, 0] < e[:, 1])
         # attention of a later query block waits for the K/V tiles of every earlier token block
         n_tb = -(-(B * T) // 128)
-        assert ops.tolist().count(W.OP_NAMES.index("norm")) == 2 * synth.TINY.n_layers * n_tb
+        # two RMSNorms per layer, each as 128 / 16 tiles of 16 rows per token block
+        assert ops.tolist().count(W.OP_NAMES.index("norm")) == 2 * synth.TINY.n_layers * n_tb * (128 // 16)
         W.wpk_select_program(h, 0, 0)
         assert W.wpk_graph_stats_get(h)["n_tiles"] != st["n_tiles"]
     finally:
