@@ -278,6 +278,11 @@ int wpk_get_edges(const wpk_handle *h, int32_t *pairs, int64_t max_pairs, int64_
 /* Op code of every tile in ticket order (int32 [n_tiles]). */
 int wpk_get_tile_ops(const wpk_handle *h, int32_t *ops, int64_t n);
 
+/* Weight bytes each tile stages into its worker's slot before its
+ * dependency wait (int64 [n_tiles], ticket order; 0 for tiles that stage no
+ * weights), for the selected program. */
+int wpk_get_tile_bytes(const wpk_handle *h, int64_t *bytes, int64_t n);
+
 /* Check the compiled graph on the host: the ticket order is topological,
  * every read-after-write, write-after-read and write-after-write pair of
  * accesses to the same tensor range is ordered by a path of edges (commuting
@@ -294,6 +299,35 @@ int wpk_verify_graph(const wpk_handle *h);
  * that tile never signal (fault injection on the host). */
 int wpk_simulate(const wpk_handle *h, int n_threads, int n_epochs, uint64_t seed, int wait_ms,
                  int stuck_tile, int32_t *done_order);
+
+/* A candidate composition for wpk_predict ("One Megakernel is Not Enough",
+ * Table I: the feature rows it models and how). */
+typedef struct wpk_predict_cfg {
+  int mode;              /* WPK_MEGAKERNEL (persistent launches) or
+                            WPK_PER_OP_GRAPH (one conventional launch per op) */
+  int n_regions;         /* megakernel: persistent launches, 1..4 */
+  int region_cut[4];     /* first layer of each region (region_cut[0] = 0) */
+  int n_workers;         /* persistent workers of each launch (the CTA budget) */
+  int n_sms;             /* SMs a conventional launch spreads its CTAs over */
+  int schedule;          /* WPK_SCHED_QUEUE or WPK_SCHED_STATIC */
+  int slots;             /* staging slots per worker: a tile's weight load is
+                            issued when one is free, before its predecessors
+                            are done (1 = one staging slot per worker) */
+  double dispatch_ns;    /* cost of a launch: a dispatch node before each */
+  double sync_ns;        /* added to a tile's ready time when it waits on a
+                            counter inside a persistent launch */
+  double first_chunk_ns; /* from a load's issue to its first bytes landing */
+} wpk_predict_cfg;
+
+/* Predict the time (ns) of one run of the selected program (the decode step,
+ * or the prefill program chosen with wpk_select_program) under composition
+ * `cfg`, by list-scheduling its tile graph (the compiled tile-to-tile edges)
+ * on the composition's workers and launches.  service_ns[t] is tile t's busy
+ * time once its weights are staged and its inputs ready; load_ns[t] the time
+ * to stage its weights (both double [n_tiles], host memory).  Host-only; it
+ * runs nothing on the GPU.  WPK_ERR_INVALID_ARG for a bad configuration. */
+int wpk_predict(const wpk_handle *h, const double *service_ns, const double *load_ns, const wpk_predict_cfg *cfg,
+                double *out_ns);
 
 /* Copy the last traced step's records (n_tiles wpk_trace_rec) to host_buf.
  * Synchronizes the device. */

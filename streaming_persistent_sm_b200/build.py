@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libwpk.so")
-SOURCES = ["graph.cpp", "runtime.cu", "capi.cu", "noalloc.cu", "debug_gemm.cu"]
+SOURCES = ["graph.cpp", "planner.cpp", "runtime.cu", "capi.cu", "noalloc.cu", "debug_gemm.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

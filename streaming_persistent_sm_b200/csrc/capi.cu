@@ -1399,6 +1399,14 @@ int wpk_get_tile_ops(const wpk_handle* h, int32_t* ops, int64_t n) {
   return WPK_OK;
 }
 
+int wpk_get_tile_bytes(const wpk_handle* h, int64_t* bytes, int64_t n) {
+  if (!h || !bytes) return WPK_ERR_INVALID_ARG;
+  const CompiledGraph& g = selected_graph(h);
+  if (n < (int64_t)g.tiles.size()) return WPK_ERR_INVALID_ARG;
+  for (size_t i = 0; i < g.tiles.size(); ++i) bytes[i] = g.tiles[i].w_bytes;
+  return WPK_OK;
+}
+
 int wpk_select_program(wpk_handle* h, int batch, int prompt_len) {
   if (!h) return WPK_ERR_INVALID_ARG;
   if (batch == 0) {
@@ -1433,6 +1441,17 @@ int wpk_simulate(const wpk_handle* h, int n_threads, int n_epochs, uint64_t seed
   int rc = simulate_graph(selected_graph(h), n_threads, n_epochs, seed, wait_ms, stuck_tile, done_order, &msg);
   if (rc) const_cast<wpk_handle*>(h)->err = msg;
   return rc;
+}
+
+int wpk_predict(const wpk_handle* h, const double* service_ns, const double* load_ns, const wpk_predict_cfg* cfg,
+                double* out_ns) {
+  if (!h || !service_ns || !load_ns || !cfg || !out_ns) return WPK_ERR_INVALID_ARG;
+  std::string msg = predict_program(selected_graph(h), service_ns, load_ns, *cfg, out_ns);
+  if (!msg.empty()) {
+    const_cast<wpk_handle*>(h)->err = msg;
+    return WPK_ERR_INVALID_ARG;
+  }
+  return WPK_OK;
 }
 
 int wpk_get_trace(wpk_handle* h, void* host_buf, size_t bytes) {

@@ -65,6 +65,11 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
 std::string verify_graph(const CompiledGraph& g);
 int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t seed, int wait_ms,
                    int stuck_tile, int32_t* done_order, std::string* msg);
+// Composition planner (planner.cpp): predicted time of one run of program g
+// under composition c from per-tile service and load times (ns).
+using PredictCfg = wpk_predict_cfg;
+std::string predict_program(const CompiledGraph& g, const double* service_ns, const double* load_ns,
+                            const PredictCfg& c, double* out_ns);
 // Arrange host bf16 weights into the image (host buffer of lay.total bytes).
 std::string arrange_weights(const CompiledGraph& g, const wpk_weights& w, uint8_t* image);
 // Tensor-core image of one [rows][K] bf16 matrix (see graph.cpp).

@@ -88,6 +88,12 @@ class wpk_graph_stats(C.Structure):
                 ("weight_bytes", C.c_int64), ("region_begin", C.c_int64 * 5), ("n_regions", C.c_int64)]
 
 
+class wpk_predict_cfg(C.Structure):
+    _fields_ = [("mode", C.c_int), ("n_regions", C.c_int), ("region_cut", C.c_int * 4), ("n_workers", C.c_int),
+                ("n_sms", C.c_int), ("schedule", C.c_int), ("slots", C.c_int), ("dispatch_ns", C.c_double),
+                ("sync_ns", C.c_double), ("first_chunk_ns", C.c_double)]
+
+
 class wpk_error_info(C.Structure):
     _fields_ = [("code", C.c_int32), ("tile", C.c_uint32), ("counter", C.c_uint32), ("epoch", C.c_uint32),
                 ("observed", C.c_uint32), ("target", C.c_uint32)]
@@ -113,6 +119,9 @@ _SIGS = {
     "wpk_get_tile_ops": (C.c_int, [_H, C.POINTER(C.c_int32), C.c_int64]),
     "wpk_verify_graph": (C.c_int, [_H]),
     "wpk_simulate": (C.c_int, [_H, C.c_int, C.c_int, C.c_uint64, C.c_int, C.c_int, C.POINTER(C.c_int32)]),
+    "wpk_get_tile_bytes": (C.c_int, [_H, C.POINTER(C.c_int64), C.c_int64]),
+    "wpk_predict": (C.c_int, [_H, C.POINTER(C.c_double), C.POINTER(C.c_double), C.POINTER(wpk_predict_cfg),
+                              C.POINTER(C.c_double)]),
     "wpk_get_trace": (C.c_int, [_H, C.c_void_p, C.c_size_t]),
     "wpk_get_error_info": (C.c_int, [_H, C.POINTER(wpk_error_info)]),
     "wpk_last_error": (C.c_char_p, [_H]),
@@ -256,6 +265,26 @@ def wpk_simulate(h, n_threads: int, n_epochs: int, seed: int, wait_ms: int = 500
     rc = load_library().wpk_simulate(h, n_threads, n_epochs, seed, wait_ms, stuck_tile,
                                      order.ctypes.data_as(C.POINTER(C.c_int32)) if n_tiles else None)
     return rc, order
+
+
+def wpk_get_tile_bytes(h, n_tiles: int) -> np.ndarray:
+    out = np.zeros(n_tiles, dtype=np.int64)
+    _check(load_library().wpk_get_tile_bytes(h, out.ctypes.data_as(C.POINTER(C.c_int64)), n_tiles), h)
+    return out
+
+
+def wpk_predict(h, service_ns, load_ns, mode: int = 0, n_regions: int = 1, region_cut=(0, 0, 0, 0),
+                n_workers: int = 148, n_sms: int = 148, schedule: int = 1, slots: int = 4, dispatch_ns: float = 0.0,
+                sync_ns: float = 0.0, first_chunk_ns: float = 0.0) -> float:
+    """Predicted ns of one run of the selected program under a composition."""
+    sv = np.ascontiguousarray(service_ns, dtype=np.float64)
+    ld = np.ascontiguousarray(load_ns, dtype=np.float64)
+    cfg = wpk_predict_cfg(mode, n_regions, (C.c_int * 4)(*region_cut), n_workers, n_sms, schedule, slots,
+                          dispatch_ns, sync_ns, first_chunk_ns)
+    out = C.c_double()
+    _check(load_library().wpk_predict(h, sv.ctypes.data_as(C.POINTER(C.c_double)),
+                                      ld.ctypes.data_as(C.POINTER(C.c_double)), C.byref(cfg), C.byref(out)), h)
+    return out.value
 
 
 def wpk_get_trace(h, n_tiles: int) -> np.ndarray:
