@@ -83,7 +83,7 @@ struct wpk_handle {
   size_t off_xa = 0, off_xb = 0, off_q = 0, off_attn = 0, off_h = 0, off_part = 0;
   // batched decode program: residual (feature-major), q/k/v sums, x^2 sums,
   // hi/lo images of x*g_attn, x*g_ffn, the attention output and h
-  size_t off_xt = 0, off_acc = 0, off_ss = 0, off_dimg[4][2] = {};
+  size_t off_xt = 0, off_acc = 0, off_ss = 0, off_dimg[4] = {};
   int64_t n_blocks = 0;
   bool loaded = false, prefilled = false, poisoned = false, has_device = false;
   int batch = 0, ctx = 0;
@@ -249,11 +249,15 @@ KParams make_params(const wpk_handle* h) {
   P.static_sched = g.plan.schedule == WPK_SCHED_STATIC;
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
+  P.img_stride = kMmaChunkBytes;
+  P.mma_cps = 1;
   if (g.plan.decode_mode == WPK_DECODE_MMA) {
     P.dec_mma = 1;
     P.uses_tmem = 1;
     P.mma_n = g.plan.dec_n;
     P.act_chunk = g.plan.dec_n * 128;
+    P.img_stride = 2 * P.act_chunk;  // hi and lo rows of a chunk adjacent
+    P.mma_cps = g.plan.dec_cps;
     P.stage_bytes = g.plan.dec_stage_bytes;
     P.n_stages = g.plan.dec_stages;
     P.act_bytes = g.plan.dec_act_bytes;
@@ -262,11 +266,11 @@ KParams make_params(const wpk_handle* h) {
     P.xt = reinterpret_cast<float*>(h->scratch + h->off_xt);
     P.acc = reinterpret_cast<float*>(h->scratch + h->off_acc);
     P.ss = reinterpret_cast<float*>(h->scratch + h->off_ss);
-    for (int i = 0; i < 2; ++i) {
-      P.xn_img[i] = h->scratch + h->off_dimg[0][i];
-      P.xf_img[i] = h->scratch + h->off_dimg[1][i];
-      P.att_img[i] = h->scratch + h->off_dimg[2][i];
-      P.h_img[i] = h->scratch + h->off_dimg[3][i];
+    for (int i = 0; i < 2; ++i) {  // lo rows follow the hi rows of each chunk
+      P.xn_img[i] = h->scratch + h->off_dimg[0] + i * P.act_chunk;
+      P.xf_img[i] = h->scratch + h->off_dimg[1] + i * P.act_chunk;
+      P.att_img[i] = h->scratch + h->off_dimg[2] + i * P.act_chunk;
+      P.h_img[i] = h->scratch + h->off_dimg[3] + i * P.act_chunk;
     }
     P.rb_arrive = h->d_rb_arrive;
     P.lm_mma_off = g.lay.lm_mma;
@@ -316,8 +320,7 @@ void scratch_layout(wpk_handle* h) {
     h->off_acc = take(qkv_rows * N * 4);
     h->off_ss = take((2 * (size_t)m.n_layers + 1) * N * 4);
     const size_t widths[4] = {(size_t)m.hidden, (size_t)m.hidden, q_rows, (size_t)m.ffn};
-    for (int t = 0; t < 4; ++t)
-      for (int i = 0; i < 2; ++i) h->off_dimg[t][i] = take(widths[t] / 64 * chunk);
+    for (int t = 0; t < 4; ++t) h->off_dimg[t] = take(widths[t] / 64 * 2 * chunk);  // [K/64][hi, lo][chunk]
   }
   h->scratch_bytes = off;
   h->n_blocks = (int64_t)B * g.max_blocks;
@@ -553,6 +556,8 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.act_bytes = g.plan.act_bytes;
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
+  P.img_stride = kMmaChunkBytes;
+  P.mma_cps = 1;
   set_mma_geometry(&P);
   P.M = g.M;
   P.T = g.T;

@@ -130,18 +130,22 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
       p->decode_mode = WPK_DECODE_GEMV;
     else
       return "bad decode mode";
-    p->dec_n = p->dec_stage_bytes = p->dec_stages = p->dec_act_bytes = 0;
+    p->dec_n = p->dec_stage_bytes = p->dec_stages = p->dec_act_bytes = p->dec_cps = 0;
     if (p->decode_mode == WPK_DECODE_MMA) {
-      // one ring stage = a 16 KB weight chunk + the hi/lo activation chunks of
-      // N tokens (N rows of 128 bytes each)
+      // one ring stage = cps 16 KB weight chunks + their hi/lo activation
+      // chunks of N tokens (N rows of 128 bytes each), each part one bulk copy
+      // (an SM's copy engine completes only a few copies per microsecond, so
+      // two chunks per stage when three or more stages still fit)
       p->dec_n = (in.max_batch + 15) / 16 * 16;
-      p->dec_stage_bytes = kMmaChunkBytes + 2 * p->dec_n * 128;
       // attention scratch: queries, one page of scores, the combine's (m, l) pairs
       const int max_pages = (in.max_context + p->page_tokens - 1) / p->page_tokens;
       const int need = std::max(attn_need, max_pages * kMaxGroup * 2 * 4);
       p->dec_act_bytes = std::max(16384, (need + 1023) / 1024 * 1024);
       const int room = kMaxSmem - fixed - 4096 - p->dec_act_bytes;  // 4 KB: the kernel's static shared memory
       int want = in.slot_bytes ? in.slot_bytes / kStageBytes : 12;
+      const int one = kMmaChunkBytes + 2 * p->dec_n * 128;
+      p->dec_cps = room / (2 * one) >= 3 ? 2 : 1;
+      p->dec_stage_bytes = p->dec_cps * one;
       p->dec_stages = std::min(std::min(want, kMaxStages), room / p->dec_stage_bytes);
       if (p->dec_stages < 2) { *code = WPK_ERR_UNSUPPORTED; return "no room for the tensor-core decode ring"; }
     }

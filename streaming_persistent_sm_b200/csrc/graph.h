@@ -22,6 +22,7 @@ struct Plan {
   // batched decode program: MMA N (max_batch rounded up to 16), its ring
   // stage (16 KB of weights + hi/lo activation chunks), stages, scratch bytes
   int dec_n, dec_stage_bytes, dec_stages, dec_act_bytes;
+  int dec_cps;          // K chunks per ring stage of the batched decode tiles (1 or 2)
   int lm_rows;          // rows of the output head (0 = vocab; the two-stage backbone's is its projection)
 };
 

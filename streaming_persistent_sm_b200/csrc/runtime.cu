@@ -188,8 +188,11 @@ __device__ bool wait_phase(const KParams& P, uint64_t* bar, uint32_t parity, vol
   }
 }
 
+// KV cache element (layer, block, kv head g, sel = 0 for K / 1 for V, row):
+// the K page and the V page of one (block, head) are adjacent, so a page is
+// staged with one bulk copy.
 __device__ __forceinline__ size_t kv_index(const KParams& P, int layer, int block, int sel, int g, int row) {
-  return ((((size_t)layer * P.n_blocks + block) * 2 + sel) * P.n_kv + g) * P.page_tokens * P.head_dim +
+  return ((((size_t)layer * P.n_blocks + block) * P.n_kv + g) * 2 + sel) * P.page_tokens * P.head_dim +
          (size_t)row * P.head_dim;
 }
 
@@ -227,8 +230,8 @@ __device__ __forceinline__ void pattn_span(const KParams& P, const Tile& T, int*
 __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int* n_chunks, int* rpc) {
   *rpc = 0;
   *n_chunks = 0;
-  if (is_mma_op(T.op)) {
-    *n_chunks = T.a3 / 64;
+  if (is_mma_op(T.op)) {  // ring stages: units of mma_cps K chunks
+    *n_chunks = (T.a3 / 64 + P.mma_cps - 1) / P.mma_cps;
     return;
   }
   if (T.op == OP_PATTN) {
@@ -262,58 +265,69 @@ __device__ __forceinline__ const uint8_t* mma_act_src(const KParams& P, const Ti
     case OP_BGU: img = P.xf_img; k_full = P.hidden; break;
     default: img = P.xn_img; k_full = P.hidden; break;
   }
-  return img[part] + ((size_t)T.a1 * (k_full / 64) + T.a2 / 64) * P.act_chunk;
+  return img[part] + ((size_t)T.a1 * (k_full / 64) + T.a2 / 64) * P.img_stride;
 }
 
-// Order in which a tensor-core tile walks its K chunks: rotated by the tile's
-// row block, so that tiles running at the same time copy different activation
-// chunks (every tile of an op reads the same activation image; in lockstep
-// they would all hit the same L2 lines at once).  The sum over K is the same;
-// only the fp32 summation order differs between tiles.
-__device__ __forceinline__ int mma_chunk_of(const Tile& T, int k, int nch) {
-  const int rot = nch > 1 ? (int)((uint32_t)T.a0 % (uint32_t)nch) : 0;
-  const int kr = k + rot;
-  return kr >= nch ? kr - nch : kr;
+// A tensor-core tile stages its K chunks in units of mma_cps consecutive
+// chunks, one ring stage each: [the units' weight blocks, 16 KB each][their
+// activation chunks, hi then lo rows of each].  Units are walked rotated by
+// the tile's row block, so that tiles running at the same time copy different
+// activation chunks (every tile of an op reads the same activation image).
+// The sum over K is the same; only the fp32 summation order differs.
+struct MmaUnit {
+  int c0, nc;  // first K chunk of the unit, chunks in it
+};
+__device__ __forceinline__ MmaUnit mma_unit(const KParams& P, const Tile& T, int u) {
+  const int nch = T.a3 / 64, cps = P.mma_cps;
+  const int nu = (nch + cps - 1) / cps;
+  const int rot = nu > 1 ? (int)((uint32_t)T.a0 % (uint32_t)nu) : 0;
+  const int ur = u + rot >= nu ? u + rot - nu : u + rot;
+  MmaUnit m;
+  m.c0 = ur * cps;
+  m.nc = min(cps, nch - m.c0);
+  return m;
 }
 
-// Tensor-core tile chunk k: arm the barrier with all its bytes and copy the
-// weight block (the activation blocks follow in issue_mma_act).  A stage holds
-// the 16 KB weight block, then the hi and the lo activation chunk.
-__device__ void issue_mma_w(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
-  mbar_arrive_expect_tx(bar, (uint32_t)kMmaChunkBytes + 2u * (uint32_t)P.act_chunk);
+// Tensor-core unit u: arm the barrier with all its bytes and copy its weight
+// blocks (the activation chunks follow in issue_mma_act).
+__device__ void issue_mma_w(const KParams& P, const Tile& T, int u, uint8_t* dst, uint64_t* bar) {
+  const MmaUnit m = mma_unit(P, T, u);
+  mbar_arrive_expect_tx(bar, (uint32_t)m.nc * ((uint32_t)kMmaChunkBytes + 2u * (uint32_t)P.act_chunk));
   const uint64_t base = (T.op == OP_BLM) ? P.lm_mma_off : 0;  // LM tiles are relative to the launch's head
-  bulk_g2s(dst, P.weights + base + T.w_off + (size_t)k * kMmaChunkBytes, kMmaChunkBytes, bar);
+  bulk_g2s(dst, P.weights + base + T.w_off + (size_t)m.c0 * kMmaChunkBytes, (uint32_t)m.nc * kMmaChunkBytes, bar);
 }
-__device__ void issue_mma_act(const KParams& P, const Tile& T, int k, uint8_t* dst, uint64_t* bar) {
+__device__ void issue_mma_act(const KParams& P, const Tile& T, int u, uint8_t* dst, uint64_t* bar) {
+  const MmaUnit m = mma_unit(P, T, u);
   const uint32_t a = (uint32_t)P.act_chunk;
-  bulk_g2s(dst + kMmaChunkBytes, mma_act_src(P, T, 0) + (size_t)k * a, a, bar);
-  bulk_g2s(dst + kMmaChunkBytes + a, mma_act_src(P, T, 1) + (size_t)k * a, a, bar);
+  uint8_t* act = dst + (size_t)P.mma_cps * kMmaChunkBytes;
+  if (P.img_stride == 2 * P.act_chunk) {  // hi and lo rows adjacent: the unit's chunks in one copy
+    bulk_g2s(act, mma_act_src(P, T, 0) + (size_t)m.c0 * P.img_stride, (uint32_t)m.nc * 2u * a, bar);
+  } else {  // separate hi and lo images (prefill: one chunk per unit)
+    bulk_g2s(act, mma_act_src(P, T, 0) + (size_t)m.c0 * P.img_stride, a, bar);
+    bulk_g2s(act + a, mma_act_src(P, T, 1) + (size_t)m.c0 * P.img_stride, a, bar);
+  }
 }
 
 // Copies of chunk `k` of tile T into `dst`; arms `bar` with their bytes.
 __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uint8_t* dst, uint64_t* bar) {
-  if (T.op == OP_PATTN) {  // one KV page (K rows then V rows) of sequence T.a0, kv head T.a1
-    int t0, t1;
-    pattn_span(P, T, &t0, &t1);
-    const int page = P.page_tokens, hd = P.head_dim;
-    const int rows = min(page, t1 - k * page);
-    const uint32_t bytes = (uint32_t)rows * hd * 2;
-    const int blk = P.block_table[T.a0 * P.max_blocks + k];
-    mbar_arrive_expect_tx(bar, 2 * bytes);
-    bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, T.a1, 0), bytes, bar);
-    bulk_g2s(dst + (size_t)page * hd * 2, P.kv + kv_index(P, T.layer, blk, 1, T.a1, 0), bytes, bar);
-    return;
-  }
-  if (T.op == OP_ATTN) {  // page k of the split: K rows, then V rows at page * head_dim
-    const AttnSpan s = attn_span(P, T);
-    const int page = P.page_tokens, hd = P.head_dim;
-    const int p = s.t0 / page + k;
-    const int rows = min(page, s.t1 - p * page);
-    const int blk = P.block_table[s.b * P.max_blocks + p];
-    const uint32_t bytes = (uint32_t)rows * hd * 2;
-    mbar_arrive_expect_tx(bar, 2 * bytes);
-    bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, bar);
-    bulk_g2s(dst + (size_t)page * hd * 2, P.kv + kv_index(P, T.layer, blk, 1, s.g, 0), bytes, bar);
+  if (T.op == OP_PATTN || T.op == OP_ATTN) {
+    // one whole KV page - its K rows, then its V rows at page * head_dim - in
+    // one copy (rows past the span are never read); prefill attention: page
+    // k of sequence a0, kv head a1; decode: page k of the split
+    int b, g, p;
+    if (T.op == OP_PATTN) {
+      b = T.a0;
+      g = T.a1;
+      p = k;
+    } else {
+      b = T.a0;
+      g = T.a1;
+      p = T.a2 * (P.split_tokens / P.page_tokens) + k;
+    }
+    const uint32_t bytes = 2u * (uint32_t)P.page_tokens * (uint32_t)P.head_dim * 2u;
+    const int blk = P.block_table[b * P.max_blocks + p];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, g, 0), bytes, bar);
     return;
   }
   const size_t row_bytes = (size_t)T.a3 * 2;
@@ -720,7 +734,7 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void attn_result(const KParams& P, int b, int f, float v) {
   if (P.dec_mma) {
-    const size_t off = (size_t)(f >> 6) * P.act_chunk + sw128_offset(b, f & 63);
+    const size_t off = (size_t)(f >> 6) * P.img_stride + sw128_offset(b, f & 63);
     const __nv_bfloat16 hb = __float2bfloat16_rn(v);
     *reinterpret_cast<__nv_bfloat16*>(P.att_img[0] + off) = hb;
     *reinterpret_cast<__nv_bfloat16*>(P.att_img[1] + off) = __float2bfloat16_rn(v - __bfloat162float(hb));
@@ -832,6 +846,7 @@ __device__ bool attn_pages(const KParams& P, const AttnSpan& s, const Shared& Sh
     // parity wait only tells a phase from the one before it, so no warp may
     // run a whole ring ahead of a stage it has not seen land
     if (ok && !wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu)) ok = false;
+    if (P.trace && threadIdx.x == 0 && k + 1 == n_chunks) s_t_data = globaltimer();  // the last page landed
     if (mine < nblk) {
       if (ok) {
         const uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
@@ -926,9 +941,16 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   }
   if (threadIdx.x < kMaxStages) s_page_rel[threadIdx.x] = 0;
   cbar();
-  // head groups: all heads at once up to four, else two halves (6 or 8 heads)
-  const int hg = grp <= 4 ? grp : grp / 2;
-  const int wpg = grp <= 4 ? kWarps : kWarps / 2;
+  // Head groups: the kv group's heads are split into n_hg groups of hg heads
+  // (hg <= 4), each served by wpg = 8 / n_hg warps over the tile's 32-token
+  // blocks.  A long tile reads every K/V row once for all heads (one group);
+  // a tile of few blocks splits the heads so that all eight warps have work.
+  const int nb_tot = n_chunks * ((page + 31) / 32);
+  int n_hg = 8;
+  while (n_hg > 1 && (grp % n_hg || n_hg * nb_tot > kWarps)) n_hg >>= 1;
+  while (grp / n_hg > 4 || grp % n_hg) n_hg <<= 1;  // at most four heads per group
+  const int hg = grp / n_hg;
+  const int wpg = kWarps / n_hg;
   bool ok;
   switch (hg) {
     case 1: ok = attn_pages<1>(P, s, Sh, cur, n_chunks, abort, q_perm, kv_cur, st_s, p_s, s_page_rel, has_cur, wpg); break;
@@ -1167,8 +1189,8 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
     case OP_BGU: {
       const int nb = active_batch(P);
       const int col = fl / 2;  // h feature 64 * a0 + col
-      uint8_t* hi = P.h_img[0] + (size_t)T.a0 * P.act_chunk;
-      uint8_t* lo = P.h_img[1] + (size_t)T.a0 * P.act_chunk;
+      uint8_t* hi = P.h_img[0] + (size_t)T.a0 * P.img_stride;
+      uint8_t* lo = P.h_img[1] + (size_t)T.a0 * P.img_stride;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float g = v[i] * s_rn[n0 + i];
@@ -1317,7 +1339,7 @@ __device__ void rowblock_done(const KParams& P, const Tile& T) {
       ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
       pl[e / 2] = pack_bf16x2(a0 - __bfloat162float(hv.x), a1 - __bfloat162float(hv.y));
     }
-    const size_t off = (size_t)(f0 / 64) * P.act_chunk + sw128_offset(n, f0 % 64);
+    const size_t off = (size_t)(f0 / 64) * P.img_stride + sw128_offset(n, f0 % 64);
     *reinterpret_cast<uint4*>(img[0] + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
     *reinterpret_cast<uint4*>(img[1] + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
     if (n < nb) atomicAdd(&s_sq[n], sq);
@@ -1341,7 +1363,8 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
     bool ok = true;
     uint32_t cc = cur.c;
     const uint32_t idesc = idesc_f16(128, 2 * N, true);
-    for (int k = 0; k < n_chunks; ++k, ++cc) {
+    uint32_t mi = 0;  // MMAs issued for this tile
+    for (int k = 0; k < n_chunks; ++k, ++cc) {  // one unit of K chunks per stage
       const int st = cc % P.n_stages;
       if (!wait_phase(P, &S.full[st], (cc / P.n_stages) & 1u, abort, tile)) {
         ok = false;
@@ -1349,11 +1372,15 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
       }
       tc_fence_after();
       const uint32_t base = smem_u32(S.ring + (size_t)st * P.stage_bytes);
+      const uint32_t act = base + (uint32_t)P.mma_cps * kMmaChunkBytes;
+      const int nc = mma_unit(P, T, k).nc;
+      for (int j = 0; j < nc; ++j) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int a = kk % NA;
-        umma_f16(tmem + (uint32_t)(a * 2 * N), sdesc_k_sw128(base + kk * 32),
-                 sdesc_k_sw128(base + kMmaChunkBytes + kk * 32), idesc, (k > 0 || kk >= NA) ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk, ++mi) {
+          const int a = (int)(mi % (uint32_t)NA);
+          umma_f16(tmem + (uint32_t)(a * 2 * N), sdesc_k_sw128(base + j * kMmaChunkBytes + kk * 32),
+                   sdesc_k_sw128(act + j * 2 * P.act_chunk + kk * 32), idesc, mi >= (uint32_t)NA ? 1u : 0u);
+        }
       }
       umma_commit(&S.empty[st]);
     }
@@ -1611,7 +1638,7 @@ __device__ bool body_embed_mma(const KParams& P, const Tile& T, int* codes /* [m
       for (int e = 0; e < 8; ++e) P.xt[(size_t)(f0 + e) * N + n] = x[e];
       atomicAdd(&s_sq2[n], sq);
     }
-    const size_t off = (size_t)(f0 / 64) * P.act_chunk + sw128_offset(n, f0 % 64);
+    const size_t off = (size_t)(f0 / 64) * P.img_stride + sw128_offset(n, f0 % 64);
     *reinterpret_cast<uint4*>(P.xn_img[0] + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
     *reinterpret_cast<uint4*>(P.xn_img[1] + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
   }
@@ -1797,20 +1824,18 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           const uint32_t c0 = c;
           for (int k = 0; k < pre && !stop; ++k, ++c) {
             if (!free_stage(c)) { stop = true; break; }
-            issue_mma_w(P, T, mma_chunk_of(T, k, nch), stage_ptr(c), &S.full[c % P.n_stages]);
+            issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
           }
           // (per-op launches get their order from the stream; no counters run)
           if (!stop && !P.per_op && !wait_counter(P, T, t, e.epoch, &s_abort)) stop = true;
           if (!stop) {
             fence_proxy_async_global();
-            for (int k = 0; k < pre; ++k)
-              issue_mma_act(P, T, mma_chunk_of(T, k, nch), stage_ptr(c0 + k), &S.full[(c0 + k) % P.n_stages]);
+            for (int k = 0; k < pre; ++k) issue_mma_act(P, T, k, stage_ptr(c0 + k), &S.full[(c0 + k) % P.n_stages]);
           }
           for (int k = pre; k < nch && !stop; ++k, ++c) {
             if (!free_stage(c)) { stop = true; break; }
-            const int kc = mma_chunk_of(T, k, nch);
-            issue_mma_w(P, T, kc, stage_ptr(c), &S.full[c % P.n_stages]);
-            issue_mma_act(P, T, kc, stage_ptr(c), &S.full[c % P.n_stages]);
+            issue_mma_w(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
+            issue_mma_act(P, T, k, stage_ptr(c), &S.full[c % P.n_stages]);
           }
         } else {
           if (T.op == OP_PATTN) {  // its KV pages are written inside this program

@@ -189,6 +189,11 @@ struct KParams {
   // tensor-core operand geometry: the MMA N (tokens per tile) and the bytes of
   // one 64-column activation chunk (N rows of 128 bytes, 128-byte swizzle)
   int mma_n, act_chunk;
+  // bytes between two consecutive 64-column chunks of an activation image
+  // (batched decode: 2 act_chunk, the hi and the lo rows of a chunk adjacent;
+  // prefill: the hi and lo images are separate, one chunk apart), and the K
+  // chunks a tensor-core tile stages per ring stage (1 or 2)
+  int img_stride, mma_cps;
   // accumulators a tile rotates its K-steps over (2 mma_n TMEM columns each)
   // and the TMEM columns a worker allocates (a power of two >= 2 mma_n mma_acc)
   int mma_acc, tmem_cols;
