@@ -64,6 +64,11 @@ def parse():
     ap.add_argument("--frame-chunks", type=int, default=0,
                     help="two-stage: split the batch into chunks whose backbone and head launches overlap")
     ap.add_argument("--head-workers", type=int, default=0, help="two-stage with --frame-chunks: the heads' workers")
+    ap.add_argument("--capacity", action="store_true",
+                    help="also measure the real-time capacity: the largest fixed cohort whose q-quantile step "
+                         "time fits --period-ms")
+    ap.add_argument("--period-ms", type=float, default=80.0, help="update period P of the capacity metric")
+    ap.add_argument("--quantile", type=float, default=0.99, help="quantile q of the capacity metric")
     return ap.parse_args()
 
 
@@ -253,6 +258,47 @@ def algorithmic_bytes_per_step(shape, weight_bytes, batch, ctx_len):
     """Weights once + KV read over ctx_len tokens + KV written for 1 token, per sequence."""
     kv = KV_BYTES_PER_TOKEN(shape)
     return weight_bytes + batch * (ctx_len * kv + kv)
+
+
+def deadline_capacity(step_ms_by_n, period_ms, q):
+    """Real-time capacity ("Why real-time inference wants a megakernel", "Real
+    time changes the objective"): the largest number of live sessions N whose
+    q-quantile update latency is within the period P - updates must keep
+    finishing on time, so a mean or a throughput does not decide it.  Returns
+    (N or 0 if none fits, {N: q-quantile ms})."""
+    qs = {int(n): float(np.quantile(np.asarray(t, dtype=np.float64), q)) for n, t in step_ms_by_n.items() if len(t)}
+    ok = [n for n, v in qs.items() if v <= period_ms]
+    return (max(ok) if ok else 0), dict(sorted(qs.items()))
+
+
+def measure_capacity(W, s, weights, prompt_len, sizes, steps, period_ms, q, seed):
+    """Per-step device times of fixed cohorts of each size in `sizes` (a plan
+    compiled for N sessions, all live, prompts prefilled untimed), and the
+    deadline capacity they give."""
+    import torch
+
+    times = {}
+    for n in sizes:
+        eng = W.Engine(s, weights, n, prompt_len + steps + 1)
+        try:
+            prompts = synth.make_prompts(s.vocab, n, prompt_len, seed)
+            eng.prefill_slots(0, prompts)
+            out = torch.empty((steps, n), dtype=torch.int32, device="cuda")
+            stream = torch.cuda.current_stream()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for i in range(steps):
+                ev[i][0].record(stream)
+                W.wpk_step(eng.h, 0, out[i].data_ptr(), 0, stream.cuda_stream)
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            times[n] = [a.elapsed_time(b) for a, b in ev[1:]]  # the first step warms up
+        finally:
+            eng.close()
+    cap, by_n = deadline_capacity(times, period_ms, q)
+    return {"period_ms": period_ms, "quantile": q, "capacity_sessions": cap, "step_ms_at_quantile": by_n,
+            "sizes": list(sizes), "steps": steps - 1,
+            "note": "largest cohort whose q-quantile step time fits the period; plans are capped at "
+                    "128 sessions (the tensor-core decode's largest N)"}
 
 
 def slowest_rank_ms(total_ms, world, device):
@@ -496,6 +542,9 @@ def main():
                    "h2d_bytes_per_step": int(host_prompt.numel() * 4),
                    "d2h_bytes_per_step": int(host_out.numel() * 4)}
 
+    if args.capacity and not two:
+        line["capacity"] = measure_capacity(W, s, weights, T, (1, 8, 16, 32, 48, 64, 96, 128), 17,
+                                            args.period_ms, args.quantile, wl.prompt_seed)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t_pre, t_step = oracle_sample(wl, weights, n_steps=2)
         per_seq = (t_pre if with_prefill else 0.0) + decode_steps * t_step

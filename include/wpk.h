@@ -343,6 +343,32 @@ const char *wpk_last_error(const wpk_handle *h);
 /* Stop the resident grid (if any), release library-owned tables, free h. */
 int wpk_destroy(wpk_handle *h);
 
+/* Fixed-cohort serving ("Why real-time inference wants a megakernel", "The
+ * cohort is known": compile for a session capacity, keep separate state per
+ * slot, step the live sessions together and mask the idle ones so that
+ * arrivals do not change the execution shape).
+ *
+ * wpk_prefill_slots prefills `batch` new sequences (tokens_dev [batch][T],
+ * device) into slots [slot0, slot0 + batch) of the plan, leaving every other
+ * slot's cache, position and last token as they were; the new slots become
+ * live.  The first call after a plain wpk_prefill (or on a fresh handle)
+ * enters the cohort mode: all slots start empty and idle.  From then on each
+ * wpk_step steps every slot of the plan (max_batch): a live slot as usual, an
+ * idle slot with a neutral input (code 0, RoPE position 0) that writes
+ * nothing to its cache, keeps its position and last token, and outputs -1 in
+ * out_tok_dev.  Slots keep their own context lengths; a step that would take
+ * a live slot past max_context fails with WPK_ERR_SHAPE.  first_tok_dev gets
+ * [batch] tokens and logits_dev (or NULL) [batch][vocab].  Needs the
+ * tensor-core prefill program (WPK_ERR_UNSUPPORTED otherwise) and a single
+ * decoder.  Stream-ordered; synchronizes `stream` once before the launch. */
+int wpk_prefill_slots(wpk_handle *h, const int32_t *tokens_dev, int slot0, int batch, int prompt_len,
+                      int32_t *first_tok_dev, float *logits_dev, void *stream);
+
+/* Cohort mode: set the live mask of slots [0, n) from active[n] (host, nonzero
+ * = live).  A slot that holds no prefilled sequence cannot be made live
+ * (WPK_ERR_INVALID_ARG).  Synchronizes the device (call it between steps). */
+int wpk_set_active_slots(wpk_handle *h, const int32_t *active, int n);
+
 /* One decode step like wpk_step (megakernel mode only), for callers that
  * cannot allocate device memory when they step the model: a host application
  * that owns the whole device pool and gives plugins no allocator, or a

@@ -71,6 +71,15 @@ struct wpk_handle {
   int32_t* d_seqlen = nullptr;
   int32_t* d_tok_fb = nullptr;
   int32_t* d_active = nullptr;
+  int32_t* d_slot_active = nullptr;  // [max_batch] slot mask (nonzero = stepped)
+  // fixed-cohort serving (wpk_prefill_slots): every slot of the plan is
+  // stepped, the mask says which are live; host mirrors of each slot's cached
+  // tokens and mask
+  bool cohort = false;
+  std::vector<int> slot_len;
+  std::vector<char> slot_on;
+  int32_t cohort_batch = 0;          // stable source of an asynchronous copy
+  int prefill_slot0 = 0;             // first slot of the prefill being launched
   int32_t* h_err_code = nullptr;  // pinned mirror of d_err->code
   // caller-owned buffers
   uint8_t* weights = nullptr;
@@ -236,6 +245,8 @@ KParams make_params(const wpk_handle* h) {
   P.seqlen = h->d_seqlen;
   P.tok_fb = h->d_tok_fb;
   P.active_batch = h->d_active;
+  P.slot_active = h->d_slot_active;
+  P.slot0 = 0;
   P.tiles = h->d_tiles;
   P.sig = h->d_sig;
   P.ctr = h->d_ctr;
@@ -573,6 +584,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.in_tok = nullptr;
   P.out_tok = first_tok;
   P.logits = logits;
+  P.slot0 = h->prefill_slot0;
   return P;
 }
 
@@ -717,7 +729,7 @@ static int setup_device(wpk_handle* h) {
                o_layers = take(g.lay.layers.size() * sizeof(LayerDev)),
                o_rope = take((size_t)p.max_context * hd2 * sizeof(float2)),
                o_bt = take(B * g.max_blocks * 4), o_arr = take(B * model->n_kv_heads * 4), o_best = take(B * 8),
-               o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4),
+               o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4), o_slot = take(B * 4),
                o_rb = take((size_t)model->n_layers * 2 * (model->hidden / 128 + 1) * 4),
                o_res = take(sizeof(ResDev));
   CUDA_TRY(h, cudaMalloc(&h->d_base, off));
@@ -737,6 +749,7 @@ static int setup_device(wpk_handle* h) {
   h->d_seqlen = reinterpret_cast<int32_t*>(h->d_base + o_seq);
   h->d_tok_fb = reinterpret_cast<int32_t*>(h->d_base + o_fb);
   h->d_active = reinterpret_cast<int32_t*>(h->d_base + o_act);
+  h->d_slot_active = reinterpret_cast<int32_t*>(h->d_base + o_slot);
   h->d_rb_arrive = reinterpret_cast<uint32_t*>(h->d_base + o_rb);
   h->d_res = reinterpret_cast<ResDev*>(h->d_base + o_res);
   CUDA_TRY(h, cudaMemcpy(h->d_tiles, g.tiles.data(), n_tiles * sizeof(Tile), cudaMemcpyHostToDevice));
@@ -1095,6 +1108,9 @@ static int prefill_impl(wpk_handle* h, const int32_t* tokens_dev, int batch, int
 static int reset_step_state(wpk_handle* h, cudaStream_t s) {
   const size_t B = h->g.plan.max_batch;
   CUDA_TRY(h, cudaMemsetAsync(h->d_seqlen, 0, B * 4, s));
+  // every slot live (bytes 0x01: a nonzero word); a new batch leaves the cohort mode
+  CUDA_TRY(h, cudaMemsetAsync(h->d_slot_active, 1, B * 4, s));
+  h->cohort = false;
   CUDA_TRY(h, cudaMemsetAsync(h->d_best, 0, B * 8, s));
   CUDA_TRY(h, cudaMemsetAsync(h->d_arrive, 0, B * h->g.m.n_kv_heads * 4, s));
   if (h->g.plan.decode_mode == WPK_DECODE_MMA) {
@@ -1309,13 +1325,120 @@ static int chunked_frame(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_
   return chunk_join(h, s, rc);
 }
 
+// Fixed-cohort serving: refuse a step that would take a live slot past the
+// context limit; after a step, the live slots hold one more token.
+static int cohort_check(wpk_handle* h) {
+  if (!h->cohort) return WPK_OK;
+  for (size_t b = 0; b < h->slot_on.size(); ++b)
+    if (h->slot_on[b] && h->slot_len[b] >= h->g.plan.max_context)
+      return fail(h, WPK_ERR_SHAPE, "slot " + std::to_string(b) + " reached the context limit");
+  return WPK_OK;
+}
+static void cohort_advance(wpk_handle* h) {
+  if (!h->cohort) return;
+  int mx = 0;
+  for (size_t b = 0; b < h->slot_on.size(); ++b) {
+    if (h->slot_on[b]) ++h->slot_len[b];
+    if (h->slot_on[b]) mx = std::max(mx, h->slot_len[b]);
+  }
+  h->ctx = mx;
+}
+
+int wpk_set_active_slots(wpk_handle* h, const int32_t* active, int n) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (!active || n <= 0 || n > h->g.plan.max_batch) return fail(h, WPK_ERR_INVALID_ARG, "bad slot mask");
+  if (h->head) return fail(h, WPK_ERR_UNSUPPORTED, "slot masks are for a single decoder");
+  if (!h->cohort) return fail(h, WPK_ERR_NOT_LOADED, "no slot was filled with wpk_prefill_slots");
+  for (int b = 0; b < n; ++b)
+    if (active[b] && h->slot_len[b] == 0)
+      return fail(h, WPK_ERR_INVALID_ARG, "slot " + std::to_string(b) + " holds no prefilled sequence");
+  rc = res_shutdown(h);
+  if (rc) return rc;
+  std::vector<int32_t> m(n);
+  for (int b = 0; b < n; ++b) {
+    m[b] = active[b] ? 1 : 0;
+    h->slot_on[b] = (char)(active[b] != 0);
+  }
+  CUDA_TRY(h, cudaDeviceSynchronize());  // no step of this handle is in flight
+  CUDA_TRY(h, cudaMemcpy(h->d_slot_active, m.data(), (size_t)n * 4, cudaMemcpyHostToDevice));
+  int mx = 0;
+  for (size_t b = 0; b < h->slot_on.size(); ++b)
+    if (h->slot_on[b]) mx = std::max(mx, h->slot_len[b]);
+  h->ctx = mx;
+  return WPK_OK;
+}
+
+int wpk_prefill_slots(wpk_handle* h, const int32_t* tokens_dev, int slot0, int batch, int prompt_len,
+                      int32_t* first_tok_dev, float* logits_dev, void* stream) {
+  int rc = check_live(h);
+  if (rc) return rc;
+  if (h->head) return fail(h, WPK_ERR_UNSUPPORTED, "slot prefill is for a single decoder");
+  if (h->g.plan.prefill_mode != WPK_PREFILL_MMA)
+    return fail(h, WPK_ERR_UNSUPPORTED, "slot prefill needs the tensor-core prefill program");
+  if (!h->loaded) return fail(h, WPK_ERR_NOT_LOADED, "weights not loaded");
+  const int B = h->g.plan.max_batch;
+  if (!tokens_dev || batch <= 0 || prompt_len <= 0 || slot0 < 0)
+    return fail(h, WPK_ERR_INVALID_ARG, "bad slot prefill arguments");
+  if (slot0 + batch > B || prompt_len > h->g.plan.max_context)
+    return fail(h, WPK_ERR_SHAPE, "slots or prompt exceed the plan");
+  if ((int64_t)batch * prompt_len > h->prefill_max_tokens)
+    return fail(h, WPK_ERR_SHAPE, "prompt tokens exceed the prefill scratch");
+  rc = res_shutdown(h);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PrefillProgram* prog = nullptr;
+  rc = get_prefill_program(h, batch, prompt_len, &prog);
+  if (rc) return rc;
+  if (!h->cohort) {  // entering the cohort mode: every slot empty and idle
+    rc = reset_step_state(h, s);
+    if (rc) return rc;
+    CUDA_TRY(h, cudaMemsetAsync(h->d_slot_active, 0, (size_t)B * 4, s));
+    h->cohort = true;
+    h->slot_len.assign(B, 0);
+    h->slot_on.assign(B, 0);
+  }
+  // the new slots: positions count up from 0 (the final tile advances them
+  // to prompt_len), live from now on; the prefill runs `batch` sequences
+  std::vector<int32_t> pos(batch, prompt_len - 1), on(batch, 1);
+  CUDA_TRY(h, cudaMemcpyAsync(h->d_seqlen + slot0, pos.data(), (size_t)batch * 4, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaMemcpyAsync(h->d_slot_active + slot0, on.data(), (size_t)batch * 4, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaMemcpyAsync(h->d_active, &batch, 4, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaStreamSynchronize(s));  // the sources live on this stack frame
+  h->prefill_slot0 = slot0;
+  rc = launch_prefill(h, prog, tokens_dev, first_tok_dev, logits_dev, s);
+  h->prefill_slot0 = 0;
+  if (rc) return rc;
+  // the decode steps run every slot of the cohort
+  h->cohort_batch = B;
+  CUDA_TRY(h, cudaMemcpyAsync(h->d_active, &h->cohort_batch, 4, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(h, cudaMemcpyAsync(h->h_err_code, &h->d_err->code, 4, cudaMemcpyDeviceToHost, s));
+  CUDA_TRY(h, cudaGetLastError());
+  for (int b = 0; b < batch; ++b) {
+    h->slot_len[slot0 + b] = prompt_len;
+    h->slot_on[slot0 + b] = 1;
+  }
+  h->batch = B;
+  h->ctx = 0;
+  for (int b = 0; b < B; ++b)
+    if (h->slot_on[b]) h->ctx = std::max(h->ctx, h->slot_len[b]);
+  h->prefilled = true;
+  return WPK_OK;
+}
+
 int wpk_step(wpk_handle* h, const int32_t* in_tok_dev, int32_t* out_tok_dev, float* logits_dev, void* stream) {
   int rc = check_live(h);
   if (rc) return rc;
   if (!h->loaded || !h->prefilled) return fail(h, WPK_ERR_NOT_LOADED, "weights or prefill missing");
-  if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  if (!h->cohort && h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  rc = cohort_check(h);
+  if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!h->head) return step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, s);
+  if (!h->head) {
+    rc = step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, s);
+    if (!rc) cohort_advance(h);
+    return rc;
+  }
   if (!h->chunks.empty()) return chunked_frame(h, in_tok_dev, out_tok_dev, logits_dev, s);
   // two-stage frame: backbone step on sum_k frame_embed_k[c_k] -> p, then the head
   int32_t* codes = reinterpret_cast<int32_t*>(h->scratch + h->off_codes);
@@ -1568,11 +1691,14 @@ int wpk_internal_step_scratch(wpk_handle* h, void* scratch, size_t scratch_bytes
   int dev = -1;
   CUDA_TRY(h, cudaGetDevice(&dev));
   if (dev != h->device) return fail(h, WPK_ERR_INVALID_ARG, "current device is not the handle's device");
-  if (h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  if (!h->cohort && h->ctx >= h->g.plan.max_context) return fail(h, WPK_ERR_SHAPE, "context limit reached");
+  rc = cohort_check(h);
+  if (rc) return rc;
   uint8_t* saved = h->scratch;
   h->scratch = static_cast<uint8_t*>(scratch);
   rc = step_impl(h, in_tok_dev, 1, out_tok_dev, logits_dev, static_cast<cudaStream_t>(stream));
   h->scratch = saved;
+  if (!rc) cohort_advance(h);
   return rc;
 }
 

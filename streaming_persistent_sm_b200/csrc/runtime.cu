@@ -197,6 +197,7 @@ __device__ __forceinline__ size_t kv_index(const KParams& P, int layer, int bloc
 }
 
 __device__ __forceinline__ int active_batch(const KParams& P) { return *P.active_batch; }
+__device__ __forceinline__ bool slot_on(const KParams& P, int b) { return P.slot_active[b] != 0; }
 
 struct AttnSpan {
   int b, g, j, pos, t0, t1;  // tokens [t0, t1) of sequence b, current position pos
@@ -241,7 +242,7 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
     return;
   }
   if (T.op == OP_ATTN) {  // one KV page per chunk
-    if (T.a0 >= active_batch(P)) return;
+    if (T.a0 >= active_batch(P) || !slot_on(P, T.a0)) return;
     const AttnSpan s = attn_span(P, T);
     *n_chunks = s.t1 > s.t0 ? (s.t1 - 1) / P.page_tokens - s.t0 / P.page_tokens + 1 : 0;
     return;
@@ -316,7 +317,7 @@ __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uin
     // k of sequence a0, kv head a1; decode: page k of the split
     int b, g, p;
     if (T.op == OP_PATTN) {
-      b = T.a0;
+      b = P.slot0 + T.a0;
       g = T.a1;
       p = k;
     } else {
@@ -409,7 +410,8 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
         const int pr = idx % (R / 2), b = idx / (R / 2), bi = b0 + b;
         const int r = r0 + 2 * pr;
         const float y0 = out[(2 * pr) * S + b], y1 = out[(2 * pr + 1) * S + b];
-        const int pos = P.seqlen[bi];
+        const bool on = slot_on(P, bi);
+        const int pos = on ? P.seqlen[bi] : 0;
         if (r < P.q_rows + P.kv_rows) {
           const bool is_q = r < P.q_rows;
           const int rr = is_q ? r : r - P.q_rows;
@@ -421,13 +423,13 @@ __device__ void epilogue(const KParams& P, const Tile& T, const float* out, int 
             float* q = P.qbuf + (size_t)bi * P.q_rows + head * hd;
             q[i] = o0;
             q[i + half] = o1;
-          } else {
+          } else if (on) {
             const int blk = P.block_table[bi * P.max_blocks + pos / P.page_tokens];
             uint16_t* k = P.kv + kv_index(P, T.layer, blk, 0, head, pos % P.page_tokens);
             k[i] = f2bf(o0);
             k[i + half] = f2bf(o1);
           }
-        } else {
+        } else if (on) {
           const int rr = r - P.q_rows - P.kv_rows;
           const int head = rr / hd, d = rr % hd;
           const int blk = P.block_table[bi * P.max_blocks + pos / P.page_tokens];
@@ -900,6 +902,19 @@ __device__ bool attn_pages(const KParams& P, const AttnSpan& s, const Shared& Sh
 __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cursor& cur, int n_chunks,
                           volatile int* abort) {
   if (T.a0 >= active_batch(P)) return true;
+  if (!slot_on(P, T.a0)) {
+    // an inactive slot attends to nothing; the tensor-core decode still
+    // returns its q/k/v sums to zero for the next step (split 0 does it)
+    if (P.dec_mma && T.a2 == 0) {
+      const int nq = P.group * P.head_dim, hd = P.head_dim;
+      for (int i = threadIdx.x; i < nq + 2 * hd; i += kThreads) {
+        const int f = i < nq ? T.a1 * nq + i
+                             : P.q_rows + ((i - nq) / hd) * P.kv_rows + T.a1 * hd + (i - nq) % hd;
+        P.acc[(size_t)f * P.mma_n + T.a0] = 0.f;
+      }
+    }
+    return true;
+  }
   __shared__ int s_last;
   __shared__ uint32_t s_page_rel[kMaxStages];  // warps done with a stage, this tile
   const AttnSpan s = attn_span(P, T);
@@ -1174,7 +1189,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
           o[i] = y;
         } else {
           const int n = n0 + i;
-          const float2 cs = P.rope[(size_t)(n < nb ? P.seqlen[n] : 0) * half + pi];
+          const float2 cs = P.rope[(size_t)(n < nb && slot_on(P, n) ? P.seqlen[n] : 0) * half + pi];
           const float y0 = even ? y : partner, y1 = even ? partner : y;
           o[i] = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
         }
@@ -1233,7 +1248,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
         const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
         const int m = tb * kTokBlock + n0 + i;
         if (m >= P.M) continue;
-        const int b = m / P.T, t = m % P.T;
+        const int b = P.slot0 + m / P.T, t = m % P.T;
         if (is_v) {
           const int blk = P.block_table[b * P.max_blocks + t / P.page_tokens];
           P.kv[kv_index(P, T.layer, blk, 1, head, t % P.page_tokens) + within] = f2bf(v[i]);
@@ -1547,6 +1562,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
 __device__ bool step_codes(const KParams& P, int b, int* codes) {
   if (threadIdx.x < P.n_in) {
     int tok = s_in_tok ? s_in_tok[(size_t)b * s_in_stride + threadIdx.x] : P.tok_fb[b];
+    if (!slot_on(P, b)) tok = 0;  // an inactive slot gets a neutral input
     if (tok < 0 || tok >= P.in_rows) {
       record_error(P, WPK_ERR_INVALID_ARG, (uint32_t)b, kNoCounter, (uint32_t)tok, (uint32_t)P.in_rows);
       tok = 0;
@@ -1595,6 +1611,7 @@ __device__ bool body_embed_mma(const KParams& P, const Tile& T, int* codes /* [m
     int tok = 0;
     if (n < nb) {
       tok = s_in_tok ? s_in_tok[(size_t)n * s_in_stride + t] : P.tok_fb[n];
+      if (!slot_on(P, n)) tok = 0;  // an inactive slot gets a neutral input
       if (tok < 0 || tok >= P.in_rows) {
         record_error(P, WPK_ERR_INVALID_ARG, (uint32_t)n, kNoCounter, (uint32_t)tok, (uint32_t)P.in_rows);
         tok = 0;
@@ -1654,10 +1671,14 @@ __device__ bool body_final(const KParams& P, uint32_t epoch) {
   for (int b = threadIdx.x; b < nb; b += kThreads) {
     const unsigned long long key = P.best[b];
     const int32_t idx = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFull));
-    if (s_out_tok) s_out_tok[(size_t)b * P.out_stride] = idx;
-    P.tok_fb[b] = idx;
+    const int sb = P.slot0 + b;  // the prefill program's sequence b fills slot slot0 + b
+    const bool on = slot_on(P, sb);
+    if (s_out_tok) s_out_tok[(size_t)b * P.out_stride] = on ? idx : -1;
+    if (on) {
+      P.tok_fb[sb] = idx;
+      P.seqlen[sb] += 1;
+    }
     P.best[b] = 0ull;
-    P.seqlen[b] += 1;
   }
   if (P.resident) {  // the step is complete: tell the host
     cbar();

@@ -154,6 +154,13 @@ struct KParams {
   int32_t* seqlen;           // [max_batch] tokens already in the cache
   int32_t* tok_fb;           // [max_batch] last greedy tokens
   int32_t* active_batch;     // [1]
+  // fixed-cohort serving: slot b of the decode programs is stepped only when
+  // slot_active[b] != 0; an inactive slot gets a neutral input (code 0, RoPE
+  // position 0), writes nothing to its KV cache, keeps its position and last
+  // token, and outputs -1.  The prefill program writes sequence b's cache and
+  // state into slot slot0 + b.
+  const int32_t* slot_active;  // [max_batch]
+  int slot0;
   const Tile* tiles;
   const uint32_t* sig;
   uint32_t* ctr;

@@ -120,6 +120,8 @@ _SIGS = {
     "wpk_verify_graph": (C.c_int, [_H]),
     "wpk_simulate": (C.c_int, [_H, C.c_int, C.c_int, C.c_uint64, C.c_int, C.c_int, C.POINTER(C.c_int32)]),
     "wpk_get_tile_bytes": (C.c_int, [_H, C.POINTER(C.c_int64), C.c_int64]),
+    "wpk_prefill_slots": (C.c_int, [_H, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    "wpk_set_active_slots": (C.c_int, [_H, C.POINTER(C.c_int32), C.c_int]),
     "wpk_predict": (C.c_int, [_H, C.POINTER(C.c_double), C.POINTER(C.c_double), C.POINTER(wpk_predict_cfg),
                               C.POINTER(C.c_double)]),
     "wpk_get_trace": (C.c_int, [_H, C.c_void_p, C.c_size_t]),
@@ -267,6 +269,17 @@ def wpk_simulate(h, n_threads: int, n_epochs: int, seed: int, wait_ms: int = 500
     return rc, order
 
 
+def wpk_prefill_slots(h, tokens_dev: int, slot0: int, batch: int, prompt_len: int, first_tok_dev: int,
+                      logits_dev: int = 0, stream: int = 0):
+    _check(load_library().wpk_prefill_slots(h, tokens_dev, slot0, batch, prompt_len, first_tok_dev,
+                                            logits_dev or None, stream or None), h)
+
+
+def wpk_set_active_slots(h, active) -> None:
+    a = np.ascontiguousarray(active, dtype=np.int32)
+    _check(load_library().wpk_set_active_slots(h, a.ctypes.data_as(C.POINTER(C.c_int32)), len(a)), h)
+
+
 def wpk_get_tile_bytes(h, n_tiles: int) -> np.ndarray:
     out = np.zeros(n_tiles, dtype=np.int64)
     _check(load_library().wpk_get_tile_bytes(h, out.ctypes.data_as(C.POINTER(C.c_int64)), n_tiles), h)
@@ -389,6 +402,21 @@ class Engine:
         wpk_prefill(self.h, tok.data_ptr(), B, T, first.data_ptr(), logits.data_ptr() if want_logits else 0,
                     self._stream())
         self._keep = tok
+        return first, logits
+
+    def prefill_slots(self, slot0: int, tokens, want_logits: bool = False):
+        """Prefill len(tokens) new sequences into slots slot0.. of the cohort
+        (every slot of the plan is stepped from now on; see wpk_prefill_slots)."""
+        torch = self.torch
+        tok = torch.as_tensor(np.ascontiguousarray(tokens, dtype=np.int32)).cuda()
+        B, T = tok.shape
+        self.batch = self.max_batch
+        first = torch.empty((B,) + self._tok_shape, dtype=torch.int32, device=tok.device)
+        logits = (torch.empty((B,) + self._logit_shape, dtype=torch.float32, device=tok.device)
+                  if want_logits else None)
+        wpk_prefill_slots(self.h, tok.data_ptr(), slot0, B, T, first.data_ptr(),
+                          logits.data_ptr() if want_logits else 0, self._stream())
+        self.torch.cuda.current_stream().synchronize()
         return first, logits
 
     def step(self, in_tok=None, want_logits: bool = False, out_tok=None, logits=None):

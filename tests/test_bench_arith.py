@@ -85,3 +85,17 @@ def test_weight_bytes_match_the_compiled_decode_program():
     hd, q, kv, f, L, V = 2048, 2048, 512, 8192, 16, 128256
     matrices = 2 * (L * (hd * (q + 2 * kv) + q * hd + 3 * f * hd) + V * hd)
     assert st["weight_bytes"] == W_BYTES == matrices
+
+
+def test_deadline_capacity_is_the_largest_cohort_within_the_period():
+    import bench
+
+    # per-size step times (ms): the q-quantile, not the mean, decides
+    times = {1: [1.0] * 99 + [2.0], 8: [5.0] * 99 + [50.0], 16: [6.0] * 98 + [90.0, 95.0], 32: [70.0] * 100}
+    cap, qs = bench.deadline_capacity(times, period_ms=80.0, q=0.99)
+    assert qs[1] == pytest.approx(1.01) and qs[32] == pytest.approx(70.0)  # linear interpolation
+    assert qs[16] > 80.0  # its mean is 7.7 ms, its 99th percentile misses the period
+    assert cap == 32  # sizes need not be monotone; the largest that fits
+    assert bench.deadline_capacity(times, period_ms=0.5, q=0.5) == (0, {1: 1.0, 8: 5.0, 16: 6.0, 32: 70.0})
+    cap, _ = bench.deadline_capacity(times, period_ms=80.0, q=0.5)
+    assert cap == 32
