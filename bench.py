@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--slot-bytes", type=int, default=0)
     ap.add_argument("--workers-per-sm", type=int, default=0)
     ap.add_argument("--lookahead", type=int, default=0)
-    ap.add_argument("--schedule", default="static", choices=["queue", "static"])
+    ap.add_argument("--schedule", default="static", choices=["queue", "static", "teams"])
     ap.add_argument("--prefill", default="auto", choices=["auto", "mma", "tokenwise"])
     ap.add_argument("--decode", default="auto", choices=["auto", "gemv", "mma"],
                     help="decode program: CUDA-core GEMV tiles or tensor-core tiles (auto: by batch)")
@@ -358,7 +358,8 @@ def main():
     mode = W.WPK_MEGAKERNEL if args.mode == "megakernel" else W.WPK_PER_OP_GRAPH
     plan = dict(mode=mode, tile_bytes=args.tile_bytes, slot_bytes=args.slot_bytes,
                 workers_per_sm=args.workers_per_sm, lookahead=args.lookahead,
-                schedule=W.WPK_SCHED_STATIC if args.schedule == "static" else W.WPK_SCHED_QUEUE,
+                schedule={"static": W.WPK_SCHED_STATIC, "queue": W.WPK_SCHED_QUEUE,
+                          "teams": W.WPK_SCHED_TEAMS}[args.schedule],
                 prefill={"auto": W.WPK_PREFILL_AUTO, "mma": W.WPK_PREFILL_MMA,
                          "tokenwise": W.WPK_PREFILL_TOKENWISE}[args.prefill],
                 decode={"auto": W.WPK_DECODE_AUTO, "gemv": W.WPK_DECODE_GEMV, "mma": W.WPK_DECODE_MMA}[args.decode],

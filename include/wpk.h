@@ -52,7 +52,7 @@ enum {
 };
 
 enum { WPK_MEGAKERNEL = 0, WPK_PER_OP_GRAPH = 1 };
-enum { WPK_SCHED_QUEUE = 0, WPK_SCHED_STATIC = 1 };
+enum { WPK_SCHED_QUEUE = 0, WPK_SCHED_STATIC = 1, WPK_SCHED_TEAMS = 2 };
 enum { WPK_PREFILL_AUTO = 0, WPK_PREFILL_MMA = 1, WPK_PREFILL_TOKENWISE = 2 };
 enum { WPK_DECODE_AUTO = 0, WPK_DECODE_GEMV = 1, WPK_DECODE_MMA = 2 };
 
@@ -112,7 +112,14 @@ typedef struct wpk_plan_cfg {
                            only after the previous tile of that worker is done */
   int schedule;         /* WPK_SCHED_QUEUE (0): tickets from one atomic device
                            queue; WPK_SCHED_STATIC: worker w takes tickets
-                           w, w + W, w + 2W, ... (W workers), no atomics       */
+                           w, w + W, w + 2W, ... (W workers), no atomics;
+                           WPK_SCHED_TEAMS: every op of the step is given a
+                           team of workers (all, a half, a quarter, ... one),
+                           the least loaded one, and each worker walks its own
+                           compiled stream of tiles; an edge between two tiles
+                           of one worker's stream needs no counter (decode
+                           program, one region, launch per step; the prefill
+                           program runs the static streams)                  */
   int prefill;          /* WPK_PREFILL_AUTO (0): the tensor-core prefill program
                            when the shapes allow, else token by token;
                            WPK_PREFILL_MMA; WPK_PREFILL_TOKENWISE (the prompt

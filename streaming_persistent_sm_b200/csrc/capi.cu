@@ -72,6 +72,8 @@ struct wpk_handle {
   int32_t* d_tok_fb = nullptr;
   int32_t* d_active = nullptr;
   int32_t* d_slot_active = nullptr;  // [max_batch] slot mask (nonzero = stepped)
+  uint32_t* d_stream_begin = nullptr;  // team schedule: worker streams
+  uint32_t* d_stream = nullptr;
   // fixed-cohort serving (wpk_prefill_slots): every slot of the plan is
   // stepped, the mask says which are live; host mirrors of each slot's cached
   // tokens and mask
@@ -257,7 +259,12 @@ KParams make_params(const wpk_handle* h) {
   P.in_tok_stride = 1;
   P.epoch = 1;
   P.idle_ns = std::max<uint64_t>(200000000ull, 20 * g.plan.wait_timeout_ns);
-  P.static_sched = g.plan.schedule == WPK_SCHED_STATIC;
+  // the team schedule's streams belong to the decode program; any other
+  // program of the handle (the prefill) runs the static streams
+  P.static_sched = g.plan.schedule == WPK_SCHED_STATIC || g.plan.schedule == WPK_SCHED_TEAMS;
+  P.team_sched = g.plan.schedule == WPK_SCHED_TEAMS;
+  P.stream_begin = h->d_stream_begin;
+  P.stream = h->d_stream;
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
   P.img_stride = kMmaChunkBytes;
@@ -585,6 +592,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.out_tok = first_tok;
   P.logits = logits;
   P.slot0 = h->prefill_slot0;
+  P.team_sched = 0;  // the prefill program runs the static streams
   return P;
 }
 
@@ -730,6 +738,7 @@ static int setup_device(wpk_handle* h) {
                o_rope = take((size_t)p.max_context * hd2 * sizeof(float2)),
                o_bt = take(B * g.max_blocks * 4), o_arr = take(B * model->n_kv_heads * 4), o_best = take(B * 8),
                o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4), o_slot = take(B * 4),
+               o_sb = take((g.stream_begin.size() + 1) * 4), o_st = take((g.stream.size() + 1) * 4),
                o_rb = take((size_t)model->n_layers * 2 * (model->hidden / 128 + 1) * 4),
                o_res = take(sizeof(ResDev));
   CUDA_TRY(h, cudaMalloc(&h->d_base, off));
@@ -750,6 +759,13 @@ static int setup_device(wpk_handle* h) {
   h->d_tok_fb = reinterpret_cast<int32_t*>(h->d_base + o_fb);
   h->d_active = reinterpret_cast<int32_t*>(h->d_base + o_act);
   h->d_slot_active = reinterpret_cast<int32_t*>(h->d_base + o_slot);
+  h->d_stream_begin = reinterpret_cast<uint32_t*>(h->d_base + o_sb);
+  h->d_stream = reinterpret_cast<uint32_t*>(h->d_base + o_st);
+  if (!g.stream.empty()) {
+    CUDA_TRY(h, cudaMemcpy(h->d_stream_begin, g.stream_begin.data(), g.stream_begin.size() * 4,
+                           cudaMemcpyHostToDevice));
+    CUDA_TRY(h, cudaMemcpy(h->d_stream, g.stream.data(), g.stream.size() * 4, cudaMemcpyHostToDevice));
+  }
   h->d_rb_arrive = reinterpret_cast<uint32_t*>(h->d_base + o_rb);
   h->d_res = reinterpret_cast<ResDev*>(h->d_base + o_res);
   CUDA_TRY(h, cudaMemcpy(h->d_tiles, g.tiles.data(), n_tiles * sizeof(Tile), cudaMemcpyHostToDevice));

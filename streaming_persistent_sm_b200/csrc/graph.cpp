@@ -77,7 +77,12 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   p->wait_timeout_ns = in.wait_timeout_ns ? in.wait_timeout_ns : 2000000000ull;
   p->lookahead = in.lookahead ? in.lookahead : 4;
   p->schedule = in.schedule;
-  if (p->schedule != WPK_SCHED_QUEUE && p->schedule != WPK_SCHED_STATIC) return "bad schedule";
+  if (p->schedule != WPK_SCHED_QUEUE && p->schedule != WPK_SCHED_STATIC && p->schedule != WPK_SCHED_TEAMS)
+    return "bad schedule";
+  if (p->schedule == WPK_SCHED_TEAMS && (p->n_regions != 1 || p->resident || p->mode != WPK_MEGAKERNEL)) {
+    *code = WPK_ERR_UNSUPPORTED;
+    return "the team schedule runs one megakernel region launched per step";
+  }
   if (p->lookahead < 1 || p->lookahead > kMaxQueue) return "lookahead must be 1..8";
   // activation staging: up to kMaxGemvBatch rows of the longest GEMV K (<= 2048)
   const int q_rows = m.n_heads * m.head_dim;
@@ -447,6 +452,73 @@ void build_mma_decode_tiles(const wpk_model_cfg& m, const Plan& p, int W, Compil
   add(OP_FINAL, m.n_layers, 0, 0, 0, 0, 0, 0, {{BUF_BEST, 0, 1, 0}, {BUF_TOK, 0, 1, 1}});
 }
 
+// Team schedule ("Why real-time inference wants a megakernel", "A concrete
+// design: one WPK update"): every op group (phase) goes to one team of
+// workers - all W workers, a half, a quarter, ... or one worker (aligned
+// blocks of floor(W / 2^j)) - the smallest team with at least as many workers
+// as the op has tiles, and among those the team whose busiest worker has the
+// least work so far; inside the team each tile goes to the least loaded
+// worker.  Work is estimated as the bytes a tile stages (weights or KV pages)
+// plus a fixed cost per tile.  Each worker's tiles form its stream, in ticket
+// order, so an edge between two tiles of one stream is already kept by that
+// order and is dropped; only edges between streams keep a counter.  Deadlock
+// freedom holds as for the static streams: every remaining edge points to a
+// smaller ticket, and the worker holding the smallest unfinished ticket has
+// finished everything before it in its own stream.
+void assign_teams(CompiledGraph* g, int W) {
+  const size_t n = g->tiles.size();
+  const double kTileCost = 32768.0;  // fixed cost of a tile, in staged-byte equivalents
+  std::vector<double> load(W, 0.0);
+  g->worker_of.assign(n, 0);
+  for (const OpGroup& og : g->groups) {
+    const int tiles = (int)(og.end - og.begin);
+    int size = W;
+    while (size > 1 && size / 2 >= tiles) size /= 2;
+    const int n_teams = W / size;
+    int best_team = 0;
+    double best = 1e300;
+    for (int k = 0; k < n_teams; ++k) {
+      double mx = 0.0;
+      for (int w = k * size; w < (k + 1) * size; ++w) mx = std::max(mx, load[w]);
+      if (mx < best) {
+        best = mx;
+        best_team = k;
+      }
+    }
+    for (uint32_t t = og.begin; t < og.end; ++t) {
+      const Tile& T = g->tiles[t];
+      double cost = kTileCost + (double)T.w_bytes;
+      if (T.op == OP_ATTN) cost += (double)g->split_tokens * g->m.head_dim * 4;  // K and V bf16 rows
+      int w0 = best_team * size, wb = w0;
+      for (int w = w0; w < w0 + size; ++w)
+        if (load[w] < load[wb]) wb = w;
+      g->worker_of[t] = wb;
+      load[wb] += cost;
+    }
+  }
+  // streams in ticket order, and each tile's predecessor in its stream
+  std::vector<std::vector<uint32_t>> per(W);
+  for (size_t t = 0; t < n; ++t) per[g->worker_of[t]].push_back((uint32_t)t);
+  g->stream_begin.assign(W + 1, 0);
+  g->stream.clear();
+  g->stream_prev.assign(n, -1);
+  for (int w = 0; w < W; ++w) {
+    g->stream_begin[w] = (uint32_t)g->stream.size();
+    for (size_t i = 0; i < per[w].size(); ++i) {
+      g->stream.push_back(per[w][i]);
+      if (i) g->stream_prev[per[w][i]] = (int32_t)per[w][i - 1];
+    }
+  }
+  g->stream_begin[W] = (uint32_t)g->stream.size();
+  // drop the edges one stream already orders
+  g->n_edges = 0;
+  for (size_t t = 0; t < n; ++t) {
+    auto& P = g->preds[t];
+    P.erase(std::remove_if(P.begin(), P.end(), [&](int u) { return g->worker_of[u] == g->worker_of[t]; }), P.end());
+    g->n_edges += (int64_t)P.size();
+  }
+}
+
 }  // namespace
 
 std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* g, int* code, int W) {
@@ -630,6 +702,9 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
     df.apply((int)t, A[t], &g->preds[t]);
     g->n_edges += (int64_t)g->preds[t].size();
   }
+
+  // ---- team schedule: teams per op, worker streams, same-stream edges dropped ----
+  if (p.schedule == WPK_SCHED_TEAMS) assign_teams(g, W);
 
   // ---- counters: one per distinct predecessor set ----
   std::unordered_map<std::vector<int>, uint32_t, VecHash> ctr_of;
@@ -898,11 +973,14 @@ std::string verify_graph(const CompiledGraph& g) {
   std::vector<uint64_t> anc(n * W, 0);
   for (size_t t = 0; t < n; ++t) {
     uint64_t* a = &anc[t * W];
-    for (int u : g.preds[t]) {
+    auto add = [&](int u) {
       const uint64_t* b = &anc[(size_t)u * W];
       for (size_t i = 0; i < W; ++i) a[i] |= b[i];
       a[u / 64] |= 1ull << (u % 64);
-    }
+    };
+    for (int u : g.preds[t]) add(u);
+    // team schedule: the tile before t in its worker's stream ran first
+    if (!g.stream_prev.empty() && g.stream_prev[t] >= 0) add(g.stream_prev[t]);
   }
   auto reach = [&](int u, int v) { return (anc[(size_t)v * W + u / 64] >> (u % 64)) & 1; };
   // every conflicting access pair must be ordered by a path
@@ -941,11 +1019,23 @@ int simulate_graph(const CompiledGraph& g, int n_threads, int n_epochs, uint64_t
   std::atomic<int> failed{0};
   std::atomic<uint64_t> fail_tile{0};
   const bool static_sched = g.plan.schedule == WPK_SCHED_STATIC;
+  const bool teams = g.plan.schedule == WPK_SCHED_TEAMS && !g.stream.empty();
+  if (teams && n_threads != (int)g.stream_begin.size() - 1) {
+    *msg = "the team schedule simulates exactly its compiled workers";
+    return WPK_ERR_INVALID_ARG;
+  }
   auto worker = [&](int wid) {
     std::mt19937_64 rng(seed * 1000003ull + wid);
     for (uint64_t i = 0;; ++i) {
       if (failed.load()) return;
-      uint64_t t = static_sched ? wid + i * (uint64_t)n_threads : head.fetch_add(1);
+      uint64_t t;
+      if (teams) {  // the worker's own stream, epoch after epoch
+        const uint64_t len = g.stream_begin[wid + 1] - g.stream_begin[wid];
+        if (len == 0 || i >= len * (uint64_t)n_epochs) return;
+        t = (i / len) * T + g.stream[g.stream_begin[wid] + i % len];
+      } else {
+        t = static_sched ? wid + i * (uint64_t)n_threads : head.fetch_add(1);
+      }
       if (t >= total) return;
       uint32_t e = (uint32_t)(t / T) + 1;
       const Tile& tile = g.tiles[t % T];

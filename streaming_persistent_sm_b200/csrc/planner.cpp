@@ -109,7 +109,9 @@ std::string predict_program(const CompiledGraph& g, const double* service_ns, co
     double end = launch;
     for (uint32_t t = b; t < e; ++t) {
       int w;
-      if (c.schedule == WPK_SCHED_STATIC) {
+      if (c.schedule == WPK_SCHED_TEAMS && !g.worker_of.empty()) {
+        w = g.worker_of[t] % W;  // the compiled team streams
+      } else if (c.schedule == WPK_SCHED_STATIC) {
         w = (int)((t - b) % (uint32_t)W);
       } else {
         w = 0;

@@ -1792,7 +1792,10 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         uint32_t t;
         if (P.per_op)
           t = (i == 0) ? P.t_begin + blockIdx.x : P.t_end;
-        else if (P.static_sched)
+        else if (P.team_sched) {  // the worker's compiled stream
+          const uint32_t b0 = P.stream_begin[blockIdx.x], len = P.stream_begin[blockIdx.x + 1] - b0;
+          t = i < len ? P.stream[b0 + i] : P.t_end;
+        } else if (P.static_sched)
           t = P.t_begin + blockIdx.x + i * gridDim.x;  // worker w: tickets w, w + W, ...
         else
           t = P.t_begin + atomicAdd(&P.head[P.region], 1u);

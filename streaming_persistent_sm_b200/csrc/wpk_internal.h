@@ -179,6 +179,9 @@ struct KParams {
   int region;
   int per_op;                // 1: one tile per CTA, no queue, no counters
   int static_sched;          // 1: worker w takes tickets w, w + W, ... (no queue)
+  int team_sched;            // 1: worker w walks stream[stream_begin[w] .. stream_begin[w + 1])
+  const uint32_t* stream_begin;  // [W + 1]
+  const uint32_t* stream;        // tickets of every worker's stream
   int resident;              // 1: tickets run on across steps (epoch = ticket / tiles + 1)
   uint64_t idle_ns;          // resident: how long a worker waits for the next step
   ResCtl* ctl;               // resident: control block (device view of mapped memory)

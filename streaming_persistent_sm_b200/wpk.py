@@ -28,6 +28,7 @@ WPK_MEGAKERNEL = 0
 WPK_PER_OP_GRAPH = 1
 WPK_SCHED_QUEUE = 0
 WPK_SCHED_STATIC = 1
+WPK_SCHED_TEAMS = 2
 WPK_PREFILL_AUTO = 0
 WPK_PREFILL_MMA = 1
 WPK_PREFILL_TOKENWISE = 2

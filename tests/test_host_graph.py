@@ -361,3 +361,40 @@ def test_two_stage_chunked_frame_host_side(lib):
             W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16, **bad))
     with pytest.raises(W.WpkError):  # a plain decoder has no frame
         W.wpk_build_graph(W.model_cfg(synth.TINY), W.plan_cfg(4, 64, frame_chunks=2))
+
+
+@pytest.mark.parametrize("shape,B", [(synth.TINY, 1), (synth.TINY, 3), (synth.LLAMA_1B, 1)])
+def test_team_schedule_streams_partition_the_step_and_drop_same_stream_edges(lib, shape, B):
+    # "Why real-time inference wants a megakernel", "A concrete design": every op
+    # goes to a team of workers, each worker walks its own stream, and only
+    # dependencies between streams need a counter
+    W_ = 16 if shape is synth.TINY else 148
+    h = _graph(shape, max_batch=B, max_context=640 if shape is synth.LLAMA_1B else 64,
+               schedule=W.WPK_SCHED_TEAMS, n_workers=W_)
+    ref = _graph(shape, max_batch=B, max_context=640 if shape is synth.LLAMA_1B else 64,
+                 schedule=W.WPK_SCHED_STATIC, n_workers=W_)
+    try:
+        st, st_ref = W.wpk_graph_stats_get(h), W.wpk_graph_stats_get(ref)
+        assert st["n_tiles"] == st_ref["n_tiles"]
+        assert st["n_edges"] < st_ref["n_edges"]  # some edges are kept by stream order instead
+        if shape is synth.TINY:
+            W.wpk_verify_graph(h)  # stream order counts as an edge for the hazard check
+            rc, order = W.wpk_simulate(h, W_, 3, 5, 10000, -1, st["n_tiles"])
+            assert rc == 0, W.wpk_last_error(h)
+            for e in range(3):  # every tile once per step
+                assert sorted(order[e * st["n_tiles"]:(e + 1) * st["n_tiles"]].tolist()) == list(range(st["n_tiles"]))
+            # a stuck tile is still caught
+            rc, _ = W.wpk_simulate(h, W_, 1, 5, 300, st["n_tiles"] // 2, 0)
+            assert rc == W.WPK_ERR_TIMEOUT
+        e = W.wpk_get_edges(h)
+        assert np.all(e[:, 0] < e[:, 1])
+    finally:
+        W.wpk_destroy(h)
+        W.wpk_destroy(ref)
+
+
+def test_team_schedule_is_one_region_launched_per_step(lib):
+    for kw in (dict(n_regions=2, region_cut=(0, 1, 0, 0)), dict(resident=1), dict(mode=W.WPK_PER_OP_GRAPH)):
+        with pytest.raises(W.WpkError) as ei:
+            _graph(schedule=W.WPK_SCHED_TEAMS, **kw)
+        assert ei.value.code == W.WPK_ERR_UNSUPPORTED
