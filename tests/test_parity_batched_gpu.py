@@ -41,6 +41,7 @@ PLANS = {
     "fewer_workers": dict(n_workers=29),
     "page32_split1": dict(page_tokens=32, split_pages=1),
     "two_stage_ring": dict(slot_bytes=32768, lookahead=2),
+    "team_schedule": dict(schedule=W.WPK_SCHED_TEAMS),
 }
 
 

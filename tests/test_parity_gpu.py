@@ -40,6 +40,8 @@ PLANS = {
     "split2_page32": dict(page_tokens=32, split_pages=2),
     "tokenwise_prefill": dict(prefill=W.WPK_PREFILL_TOKENWISE),
     "static_schedule": dict(schedule=W.WPK_SCHED_STATIC),
+    "team_schedule": dict(schedule=W.WPK_SCHED_TEAMS),
+    "team_schedule_few_workers": dict(schedule=W.WPK_SCHED_TEAMS, n_workers=5),
 }
 
 
@@ -119,6 +121,37 @@ def test_trace_respects_every_edge_and_prefetches(weights):
         assert len(set(tr["worker"].tolist())) > 1
     finally:
         eng.close()
+
+
+def test_team_schedule_trace_respects_every_dataflow_edge(weights):
+    # the team schedule drops edges between tiles of one worker's stream: every
+    # edge of the full dataflow graph (taken from a static plan of the same
+    # step) must still hold in the traced run
+    eng = W.Engine(S, weights, 2, CTX, trace=1, schedule=W.WPK_SCHED_TEAMS, n_workers=24)
+    full = W.wpk_build_graph(W.model_cfg(S), W.plan_cfg(2, CTX, schedule=W.WPK_SCHED_STATIC, n_workers=24))
+    try:
+        st = eng.stats
+        eng.prefill(_prompts(2, 20), want_logits=False)
+        eng.step()
+        eng.step()
+        import torch
+
+        torch.cuda.synchronize()
+        tr = W.wpk_get_trace(eng.h, st["n_tiles"])
+        assert sorted(tr["tile"].tolist()) == list(range(st["n_tiles"]))
+        e_full, e_team = W.wpk_get_edges(full), W.wpk_get_edges(eng.h)
+        assert len(e_team) < len(e_full)
+        done, start = tr["ev_done"].astype(np.int64), tr["ev_start"].astype(np.int64)
+        idx = np.empty(st["n_tiles"], dtype=np.int64)
+        idx[tr["tile"]] = np.arange(st["n_tiles"])
+        assert np.all(done[idx[e_full[:, 0]]] < start[idx[e_full[:, 1]]])
+        # each worker ran its tiles in ticket order
+        for w in set(tr["worker"].tolist()):
+            mine = np.sort(tr["tile"][tr["worker"] == w])
+            assert np.all(np.diff(start[idx[mine]]) > 0)
+    finally:
+        eng.close()
+        W.wpk_destroy(full)
 
 
 def test_stalled_dependency_times_out_and_poisons_handle(weights):
