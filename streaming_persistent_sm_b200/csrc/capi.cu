@@ -103,7 +103,7 @@ struct wpk_handle {
   std::string err;
   // prefill programs and their scratch (offsets in the caller's scratch)
   std::vector<std::unique_ptr<PrefillProgram>> prefills;
-  size_t off_px = 0, off_pq = 0, off_xn[2] = {0, 0}, off_att[2] = {0, 0}, off_hi[2] = {0, 0};
+  size_t off_px = 0, off_pq = 0, off_xn = 0, off_att = 0, off_hi = 0;
   int64_t prefill_max_tokens = 0;
   int prefill_stages = 0;
   size_t smem_prefill = 0;
@@ -327,9 +327,11 @@ void scratch_layout(wpk_handle* h) {
     h->prefill_max_tokens = (int64_t)M;
     h->off_px = take(M * m.hidden * 4);
     h->off_pq = take(M * q_rows * 4);
-    for (int i = 0; i < 2; ++i) h->off_xn[i] = take(n_tb * (m.hidden / 64) * kMmaChunkBytes);
-    for (int i = 0; i < 2; ++i) h->off_att[i] = take(n_tb * (q_rows / 64) * kMmaChunkBytes);
-    for (int i = 0; i < 2; ++i) h->off_hi[i] = take(n_tb * (m.ffn / 64) * kMmaChunkBytes);
+    // activation images [token block][K / 64][hi, lo][128 rows x 128 B]: the
+    // hi and lo halves of a chunk adjacent, so one bulk copy stages both
+    h->off_xn = take(n_tb * (m.hidden / 64) * 2 * kMmaChunkBytes);
+    h->off_att = take(n_tb * (q_rows / 64) * 2 * kMmaChunkBytes);
+    h->off_hi = take(n_tb * (m.ffn / 64) * 2 * kMmaChunkBytes);
   }
   if (g.plan.decode_mode == WPK_DECODE_MMA) {
     const size_t N = g.plan.dec_n, chunk = N * 128;
@@ -574,7 +576,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.act_bytes = g.plan.act_bytes;
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
-  P.img_stride = kMmaChunkBytes;
+  P.img_stride = 2 * kMmaChunkBytes;  // hi and lo halves of a chunk adjacent
   P.mma_cps = 1;
   set_mma_geometry(&P);
   P.M = g.M;
@@ -584,9 +586,9 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.px = reinterpret_cast<float*>(h->scratch + h->off_px);
   P.pq = reinterpret_cast<float*>(h->scratch + h->off_pq);
   for (int i = 0; i < 2; ++i) {
-    P.xn_img[i] = h->scratch + h->off_xn[i];
-    P.att_img[i] = h->scratch + h->off_att[i];
-    P.h_img[i] = h->scratch + h->off_hi[i];
+    P.xn_img[i] = h->scratch + h->off_xn + i * kMmaChunkBytes;
+    P.att_img[i] = h->scratch + h->off_att + i * kMmaChunkBytes;
+    P.h_img[i] = h->scratch + h->off_hi + i * kMmaChunkBytes;
   }
   P.in_tok = nullptr;
   P.out_tok = first_tok;

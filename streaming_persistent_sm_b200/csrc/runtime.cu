@@ -303,7 +303,7 @@ __device__ void issue_mma_act(const KParams& P, const Tile& T, int u, uint8_t* d
   uint8_t* act = dst + (size_t)P.mma_cps * kMmaChunkBytes;
   if (P.img_stride == 2 * P.act_chunk) {  // hi and lo rows adjacent: the unit's chunks in one copy
     bulk_g2s(act, mma_act_src(P, T, 0) + (size_t)m.c0 * P.img_stride, (uint32_t)m.nc * 2u * a, bar);
-  } else {  // separate hi and lo images (prefill: one chunk per unit)
+  } else {  // separate hi and lo images (one chunk per unit)
     bulk_g2s(act, mma_act_src(P, T, 0) + (size_t)m.c0 * P.img_stride, a, bar);
     bulk_g2s(act + a, mma_act_src(P, T, 1) + (size_t)m.c0 * P.img_stride, a, bar);
   }
@@ -1087,8 +1087,8 @@ __device__ bool body_norm(const KParams& P, const Tile& T) {
   const int h = P.hidden, units = h / 8, nkc = h / 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tb = T.a0;
-  uint8_t* hi = P.xn_img[0] + (size_t)tb * nkc * kMmaChunkBytes;
-  uint8_t* lo = P.xn_img[1] + (size_t)tb * nkc * kMmaChunkBytes;
+  uint8_t* hi = P.xn_img[0] + (size_t)tb * nkc * P.img_stride;
+  uint8_t* lo = P.xn_img[1] + (size_t)tb * nkc * P.img_stride;
   constexpr int kMaxUnits = 2048 / 8 / 32;
   for (int n = T.a2 + warp; n < T.a2 + kNormRows; n += kWarps) {  // the tile's rows of the block
     const int m = tb * kTokBlock + n;
@@ -1129,7 +1129,7 @@ __device__ bool body_norm(const KParams& P, const Tile& T) {
         ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
         pl[e / 2] = pack_bf16x2(r0, r1);
       }
-      const size_t off = (size_t)(k / 64) * kMmaChunkBytes + sw128_offset(n, k % 64);
+      const size_t off = (size_t)(k / 64) * P.img_stride + sw128_offset(n, k % 64);
       *reinterpret_cast<uint4*>(hi + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
       *reinterpret_cast<uint4*>(lo + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
     }
@@ -1280,8 +1280,8 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
     }
     case OP_MGU: {
       const int j = f / 2, c = j / 64, col = j % 64, nkc = P.ffn / 64;
-      uint8_t* hi = P.h_img[0] + ((size_t)tb * nkc + c) * kMmaChunkBytes;
-      uint8_t* lo = P.h_img[1] + ((size_t)tb * nkc + c) * kMmaChunkBytes;
+      uint8_t* hi = P.h_img[0] + ((size_t)tb * nkc + c) * P.img_stride;
+      uint8_t* lo = P.h_img[1] + ((size_t)tb * nkc + c) * P.img_stride;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float up = __shfl_xor_sync(0xffffffffu, v[i], 1);
@@ -1537,7 +1537,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
   if (valid) {
     const float inv = 1.0f / lrun;
     const int tb = m / kTokBlock, n = m % kTokBlock, nkc = P.q_rows / 64;
-    const size_t blk = ((size_t)tb * nkc + head) * kMmaChunkBytes;  // 64-column chunk == one head
+    const size_t blk = ((size_t)tb * nkc + head) * P.img_stride;  // 64-column chunk == one head
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       uint32_t ph[4], pl[4];
