@@ -510,13 +510,46 @@ void assign_teams(CompiledGraph* g, int W) {
     }
   }
   g->stream_begin[W] = (uint32_t)g->stream.size();
-  // drop the edges one stream already orders
-  g->n_edges = 0;
-  for (size_t t = 0; t < n; ++t) {
-    auto& P = g->preds[t];
-    P.erase(std::remove_if(P.begin(), P.end(), [&](int u) { return g->worker_of[u] == g->worker_of[t]; }), P.end());
-    g->n_edges += (int64_t)P.size();
+}
+
+// Team schedule counters: a worker signals once per op group it served, from
+// its last tile of the group (the phase barrier of the pages' design); a tile
+// waits for the workers that hold its predecessors in each predecessor group -
+// itself included, so that every consumer of a group shares one counter -
+// except when all of them are on its own worker, where its stream order
+// already keeps the dependency.  Returns, per tile, the signalling tiles it
+// waits for (sorted).
+std::vector<std::vector<int>> team_waits(const CompiledGraph& g) {
+  const size_t n = g.tiles.size();
+  std::vector<int> group_of(n, 0);
+  for (size_t gi = 0; gi < g.groups.size(); ++gi)
+    for (uint32_t t = g.groups[gi].begin; t < g.groups[gi].end; ++t) group_of[t] = (int)gi;
+  // last tile of (group, worker): scan in ticket order
+  std::unordered_map<uint64_t, int> last;
+  for (size_t t = 0; t < n; ++t) last[((uint64_t)group_of[t] << 32) | (uint32_t)g.worker_of[t]] = (int)t;
+  std::vector<std::vector<int>> waits(n);
+  for (size_t v = 0; v < n; ++v) {
+    std::map<int, std::vector<int>> by_group;  // predecessor group -> workers holding v's predecessors there
+    for (int u : g.preds[v]) by_group[group_of[u]].push_back(g.worker_of[u]);
+    for (auto& kv : by_group) {
+      auto& ws = kv.second;
+      std::sort(ws.begin(), ws.end());
+      ws.erase(std::unique(ws.begin(), ws.end()), ws.end());
+      if (ws.size() == 1 && ws[0] == g.worker_of[v]) continue;  // kept by v's own stream
+      for (int w : ws) {
+        const int x = last[((uint64_t)kv.first << 32) | (uint32_t)w];
+        if (x < (int)v) {
+          waits[v].push_back(x);
+        } else {  // the group reaches past v (an edge inside one op): keep the tile edges
+          for (int u : g.preds[v])
+            if (group_of[u] == kv.first && g.worker_of[u] == w) waits[v].push_back(u);
+        }
+      }
+    }
+    std::sort(waits[v].begin(), waits[v].end());
+    waits[v].erase(std::unique(waits[v].begin(), waits[v].end()), waits[v].end());
   }
+  return waits;
 }
 
 }  // namespace
@@ -706,12 +739,15 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   // ---- team schedule: teams per op, worker streams, same-stream edges dropped ----
   if (p.schedule == WPK_SCHED_TEAMS) assign_teams(g, W);
 
-  // ---- counters: one per distinct predecessor set ----
+  // ---- counters: one per distinct predecessor set (the team schedule: per
+  //      distinct set of signalling tiles, one per worker and group) ----
+  std::vector<std::vector<int>> tw;
+  if (p.schedule == WPK_SCHED_TEAMS) tw = team_waits(*g);
   std::unordered_map<std::vector<int>, uint32_t, VecHash> ctr_of;
   std::vector<std::vector<uint32_t>> sig_of(T.size());
   g->ctr_need.clear();
   for (size_t t = 0; t < T.size(); ++t) {
-    const auto& P = g->preds[t];
+    const auto& P = tw.empty() ? g->preds[t] : tw[t];
     if (P.empty()) continue;
     auto it = ctr_of.find(P);
     uint32_t c;
@@ -957,8 +993,28 @@ std::string verify_graph(const CompiledGraph& g) {
     const Tile& T = g.tiles[t];
     for (uint32_t i = 0; i < T.sig_cnt; ++i) signalers[g.sig[T.sig_off + i]].push_back((int)t);
   }
+  const bool teams = !g.worker_of.empty();
   for (size_t t = 0; t < n; ++t) {
     const Tile& T = g.tiles[t];
+    if (teams) {
+      // every predecessor is on the tile's own worker (stream order) or is
+      // covered by a signaller of its counter: a tile of the predecessor's
+      // worker and op group at or after it in ticket order
+      const std::vector<int> none;
+      const auto& S = T.wait_ctr == kNoCounter ? none : signalers[T.wait_ctr];
+      if (T.wait_ctr != kNoCounter && T.need != S.size())
+        return fmt("tile %lld need %lld != signal count", (long long)t, T.need);
+      for (int u : g.preds[t]) {
+        if (g.worker_of[u] == g.worker_of[t]) continue;
+        bool covered = false;
+        for (int x : S)
+          if (x >= u && x < (int)t && g.worker_of[x] == g.worker_of[u] && g.tiles[x].op == g.tiles[u].op &&
+              g.tiles[x].layer == g.tiles[u].layer)
+            covered = true;
+        if (!covered) return fmt("team schedule: edge %lld -> %lld is not signalled", u, (long long)t);
+      }
+      continue;
+    }
     if (g.preds[t].empty()) {
       if (T.wait_ctr != kNoCounter) return fmt("tile %lld waits without predecessors", (long long)t);
       continue;

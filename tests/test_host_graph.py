@@ -376,15 +376,16 @@ def test_team_schedule_streams_partition_the_step_and_drop_same_stream_edges(lib
     try:
         st, st_ref = W.wpk_graph_stats_get(h), W.wpk_graph_stats_get(ref)
         assert st["n_tiles"] == st_ref["n_tiles"]
-        assert st["n_edges"] < st_ref["n_edges"]  # some edges are kept by stream order instead
+        # a worker signals once per op it served, not once per tile
+        assert st["n_signals"] < st_ref["n_signals"]
         if shape is synth.TINY:
             W.wpk_verify_graph(h)  # stream order counts as an edge for the hazard check
             rc, order = W.wpk_simulate(h, W_, 3, 5, 10000, -1, st["n_tiles"])
             assert rc == 0, W.wpk_last_error(h)
             for e in range(3):  # every tile once per step
                 assert sorted(order[e * st["n_tiles"]:(e + 1) * st["n_tiles"]].tolist()) == list(range(st["n_tiles"]))
-            # a stuck tile is still caught
-            rc, _ = W.wpk_simulate(h, W_, 1, 5, 300, st["n_tiles"] // 2, 0)
+            # a stuck tile is still caught (the embed tile: it signals the first layer)
+            rc, _ = W.wpk_simulate(h, W_, 1, 5, 300, 0, 0)
             assert rc == W.WPK_ERR_TIMEOUT
         e = W.wpk_get_edges(h)
         assert np.all(e[:, 0] < e[:, 1])
