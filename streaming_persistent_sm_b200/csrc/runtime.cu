@@ -1732,7 +1732,6 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
   }
   const Shared S = carve(smem_raw, P);
   __shared__ volatile int s_abort;
-  __shared__ volatile uint32_t s_prod_i;  // tiles the producer has claimed (the KV prefetcher trails it)
   __shared__ uint32_t s_prod_chunks;  // chunks the producer issued
   __shared__ uint32_t s_cons_chunks;  // chunks the consumers finished
   const int warp = threadIdx.x >> 5;
@@ -1754,7 +1753,6 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
     for (int i = 0; i < kMaxStages; ++i) s_seen[i] = 0;
     s_io_epoch = 0;
     s_abort = 0;
-    s_prod_i = 0;
     s_prod_chunks = 0;
     s_cons_chunks = 0;
   }
@@ -1781,47 +1779,6 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         for (uint32_t k = 0; k < req.y; ++k) red_release_add_u32(P.ctr + P.sig[req.x + k], 1u);
         mbar_arrive(&S.sig_empty[slot]);
       }
-  } else if (warp == kWarps && (threadIdx.x & 31) == 2) {
-    // ------------------------------------------------------- KV prefetcher
-    // Walks the worker's own coming tickets (static or team streams; the
-    // tickets of a launch per step are known ahead) up to kPrefetchAhead
-    // tiles past the producer, and asks L2 for the KV pages of every
-    // attention tile among them.  Past tokens' pages do not depend on this
-    // step, so they can be fetched while the step's earlier ops still run;
-    // the producer's copies into the ring then find them in L2.
-    constexpr uint32_t kPrefetchAhead = 6;
-    if (!P.per_op && !P.resident && (P.static_sched || P.team_sched)) {
-      for (uint32_t i = 0;; ++i) {
-        uint32_t t;
-        if (P.team_sched) {
-          const uint32_t b0 = P.stream_begin[blockIdx.x], len = P.stream_begin[blockIdx.x + 1] - b0;
-          if (i >= len) break;
-          t = P.stream[b0 + i];
-        } else {
-          t = P.t_begin + blockIdx.x + i * gridDim.x;
-          if (t >= P.t_end) break;
-        }
-        const uint64_t t0 = globaltimer();
-        bool quit = false;
-        while (i > s_prod_i + kPrefetchAhead) {  // stay within a few tiles of the producer
-          if (s_abort || globaltimer() - t0 > P.timeout_ns) {
-            quit = true;
-            break;
-          }
-          __nanosleep(200);
-        }
-        if (quit) break;
-        const Tile T = P.tiles[t];
-        if (T.op != OP_ATTN || T.a0 >= active_batch(P) || !slot_on(P, T.a0)) continue;
-        const AttnSpan sp = attn_span(P, T);
-        if (sp.t1 <= sp.t0) continue;
-        const uint32_t bytes = 2u * (uint32_t)P.page_tokens * (uint32_t)P.head_dim * 2u;
-        for (int p = sp.t0 / P.page_tokens; p <= (sp.t1 - 1) / P.page_tokens; ++p) {
-          const int blk = P.block_table[sp.b * P.max_blocks + p];
-          bulk_prefetch_l2(P.kv + kv_index(P, T.layer, blk, 0, sp.g, 0), bytes);
-        }
-      }
-    }
   } else if (warp == kWarps) {
     // ------------------------------------------------------------ producer
     if ((threadIdx.x & 31) == 0) {
@@ -1843,7 +1800,6 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         else
           t = P.t_begin + atomicAdd(&P.head[P.region], 1u);
         const uint64_t t_claim = P.trace ? globaltimer() : 0;
-        s_prod_i = i;
         TQEntry& e = S.tq[slot];
         uint32_t epoch = P.epoch;
         if (P.resident) {
