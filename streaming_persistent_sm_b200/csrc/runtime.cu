@@ -203,6 +203,12 @@ struct AttnSpan {
   int b, g, j, pos, t0, t1;  // tokens [t0, t1) of sequence b, current position pos
 };
 
+// KV pages a decode attention tile stages per ring stage (a tensor-core decode
+// stage holds two 64-token pages).
+__device__ __forceinline__ int attn_pps(const KParams& P) {
+  return max(1, P.stage_bytes / (2 * P.page_tokens * P.head_dim * 2));
+}
+
 __device__ __forceinline__ AttnSpan attn_span(const KParams& P, const Tile& T) {
   AttnSpan s;
   s.b = T.a0;
@@ -241,10 +247,11 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
     *n_chunks = (t1 - 1) / P.page_tokens + 1;
     return;
   }
-  if (T.op == OP_ATTN) {  // one KV page per chunk
+  if (T.op == OP_ATTN) {  // attn_pps KV pages per ring stage
     if (T.a0 >= active_batch(P) || !slot_on(P, T.a0)) return;
     const AttnSpan s = attn_span(P, T);
-    *n_chunks = s.t1 > s.t0 ? (s.t1 - 1) / P.page_tokens - s.t0 / P.page_tokens + 1 : 0;
+    const int pages = s.t1 > s.t0 ? (s.t1 - 1) / P.page_tokens - s.t0 / P.page_tokens + 1 : 0;
+    *n_chunks = (pages + attn_pps(P) - 1) / attn_pps(P);
     return;
   }
   if (T.w_bytes == 0) return;
@@ -312,23 +319,25 @@ __device__ void issue_mma_act(const KParams& P, const Tile& T, int u, uint8_t* d
 // Copies of chunk `k` of tile T into `dst`; arms `bar` with their bytes.
 __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uint8_t* dst, uint64_t* bar) {
   if (T.op == OP_PATTN || T.op == OP_ATTN) {
-    // one whole KV page - its K rows, then its V rows at page * head_dim - in
-    // one copy (rows past the span are never read); prefill attention: page
-    // k of sequence a0, kv head a1; decode: page k of the split
-    int b, g, p;
-    if (T.op == OP_PATTN) {
-      b = P.slot0 + T.a0;
-      g = T.a1;
-      p = k;
-    } else {
-      b = T.a0;
-      g = T.a1;
-      p = T.a2 * (P.split_tokens / P.page_tokens) + k;
-    }
+    // whole KV pages - a page's K rows, then its V rows at page * head_dim -
+    // one copy each (rows past the span are never read); prefill attention:
+    // page k of sequence a0, kv head a1; decode: pages k * attn_pps .. of the
+    // split, packed into the stage
     const uint32_t bytes = 2u * (uint32_t)P.page_tokens * (uint32_t)P.head_dim * 2u;
-    const int blk = P.block_table[b * P.max_blocks + p];
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, g, 0), bytes, bar);
+    if (T.op == OP_PATTN) {
+      const int blk = P.block_table[(P.slot0 + T.a0) * P.max_blocks + k];
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, T.a1, 0), bytes, bar);
+      return;
+    }
+    const AttnSpan s = attn_span(P, T);
+    const int first = s.t0 / P.page_tokens + k * attn_pps(P);
+    const int n = min(attn_pps(P), (s.t1 - 1) / P.page_tokens + 1 - first);
+    mbar_arrive_expect_tx(bar, (uint32_t)n * bytes);
+    for (int j = 0; j < n; ++j) {
+      const int blk = P.block_table[s.b * P.max_blocks + first + j];
+      bulk_g2s(dst + (size_t)j * bytes, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, bar);
+    }
     return;
   }
   const size_t row_bytes = (size_t)T.a3 * 2;
@@ -835,32 +844,34 @@ __device__ bool attn_pages(const KParams& P, const AttnSpan& s, const Shared& Sh
   }
   float* p_w = p_s + warp * 32 * GRP;
   bool ok = true;
-  for (int k = 0; k < n_chunks; ++k) {  // page k of the split, one ring stage each
+  const int pps = attn_pps(P);
+  const int page_bytes = 2 * page * hd * 2;
+  for (int k = 0; k < n_chunks; ++k) {  // ring stage k: pages k * pps .. of the split
     const uint32_t c = cur.c + k;
     const int st = c % P.n_stages;
-    const int p0 = (s.t0 / page + k) * page;
-    const int n = min(page, s.t1 - p0);
-    const int nblk = (n + 31) / 32;
-    // blocks are numbered across the tile's pages so that every warp gets work
-    const int first = (k * ((page + 31) / 32)) % wpg;
-    const int mine = (wi - first + wpg) % wpg;  // this warp's first block in the page
-    // every warp waits for every page, also one without a block for it: a
+    // every warp waits for every stage, also one without a block for it: a
     // parity wait only tells a phase from the one before it, so no warp may
     // run a whole ring ahead of a stage it has not seen land
     if (ok && !wait_phase(P, &Sh.full[st], (c / P.n_stages) & 1u, abort, 0xFFFFFFFFu)) ok = false;
     if (P.trace && threadIdx.x == 0 && k + 1 == n_chunks) s_t_data = globaltimer();  // the last page landed
-    if (mine < nblk) {
-      if (ok) {
-        const uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes;
-        for (int b = mine; b < nblk; b += wpg) {
-          const int cnt = min(32, n - b * 32);
-          // the staged copy of the current token's row is stale (it was copied
-          // before this step wrote it): leave it out, read zeros for its V
-          const int rel = s.pos - p0 - b * 32;
-          const int skip = (rel >= 0 && rel < 32) ? rel : -1;
-          attn_block<GRP>(stage + (size_t)b * 32 * hd * 2, stage + (size_t)page * hd * 2 + (size_t)b * 32 * hd * 2,
-                          cnt, skip, q_perm, scale, p_w, m, l, o0, o1);
-        }
+    for (int j = 0; j < pps && ok; ++j) {
+      const int pg = k * pps + j;  // page of the split
+      const int p0 = (s.t0 / page + pg) * page;
+      if (p0 >= s.t1) break;
+      const int n = min(page, s.t1 - p0);
+      const int nblk = (n + 31) / 32;
+      // blocks are numbered across the tile's pages so that every warp gets work
+      const int first = (pg * ((page + 31) / 32)) % wpg;
+      const int mine = (wi - first + wpg) % wpg;  // this warp's first block in the page
+      const uint8_t* stage = Sh.ring + (size_t)st * P.stage_bytes + (size_t)j * page_bytes;
+      for (int b = mine; b < nblk; b += wpg) {
+        const int cnt = min(32, n - b * 32);
+        // the staged copy of the current token's row is stale (it was copied
+        // before this step wrote it): leave it out, read zeros for its V
+        const int rel = s.pos - p0 - b * 32;
+        const int skip = (rel >= 0 && rel < 32) ? rel : -1;
+        attn_block<GRP>(stage + (size_t)b * 32 * hd * 2, stage + (size_t)page * hd * 2 + (size_t)b * 32 * hd * 2,
+                        cnt, skip, q_perm, scale, p_w, m, l, o0, o1);
       }
     }
     // the last warp to finish with the page hands the stage back
@@ -960,7 +971,7 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   // (hg <= 4), each served by wpg = 8 / n_hg warps over the tile's 32-token
   // blocks.  A long tile reads every K/V row once for all heads (one group);
   // a tile of few blocks splits the heads so that all eight warps have work.
-  const int nb_tot = n_chunks * ((page + 31) / 32);
+  const int nb_tot = n_chunks * attn_pps(P) * ((page + 31) / 32);
   int n_hg = 8;
   while (n_hg > 1 && (grp % n_hg || n_hg * nb_tot > kWarps)) n_hg >>= 1;
   while (grp / n_hg > 4 || grp % n_hg) n_hg <<= 1;  // at most four heads per group
