@@ -600,7 +600,8 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int K, int rows
     for (int i = 0; i < RG; ++i)
 #pragma unroll
       for (int b = 0; b < BG; ++b) acc[i][b] = 0.f;
-    for (int seg = 0; seg < segs; ++seg) {
+#pragma unroll 2
+    for (int seg = 0; seg < segs; ++seg) {  // two segments in flight: the stage is held for less time
       const int k = seg * 256 + lane * 8;
       if (k >= K) continue;
       float f[RG][8];
@@ -1424,6 +1425,7 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
   cbar();
   bool ok = s_mma_ok;
   if (!wait_phase(P, S.acc, cs.acc_phase, abort, tile)) ok = false;
+  if (P.trace && threadIdx.x == 0) s_t_data = globaltimer();  // the accumulators are complete
   cs.acc_phase ^= 1u;
   cur.c += n_chunks;
   if (!cbar_and(ok)) return false;
