@@ -1153,6 +1153,14 @@ __device__ bool body_norm(const KParams& P, const Tile& T) {
 // and the tile's best (value, index) key per token of the LM head.
 __shared__ float s_rn[kMaxMmaBatch];
 __shared__ unsigned long long s_best[kMaxMmaBatch];
+// Per token column of a tensor-core QKV tile, filled once per tile: the RoPE
+// position (batched decode: the sequence's position, 0 for an idle or absent
+// column; prefill: the token's position, -1 past the prompt tokens), and
+// (prefill) the element index of the token's row in its KV page for kv head 0's
+// K (the other heads and V follow at fixed offsets).  The prefill table shares
+// its storage with s_best, which only the batched decode's LM head uses.
+__shared__ int s_col_pos[kMaxMmaBatch];
+#define s_col_kv s_best
 
 // Adds the 16 token columns n0..n0+15 (those below nb) of one feature row to a
 // feature-major fp32 buffer row `dst` (16-byte aligned at column n0).
@@ -1201,7 +1209,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
           o[i] = y;
         } else {
           const int n = n0 + i;
-          const float2 cs = P.rope[(size_t)(n < nb && slot_on(P, n) ? P.seqlen[n] : 0) * half + pi];
+          const float2 cs = P.rope[(size_t)s_col_pos[n] * half + pi];
           const float y0 = even ? y : partner, y1 = even ? partner : y;
           o[i] = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
         }
@@ -1251,33 +1259,33 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       break;
     }
     case OP_MQKV: {
+      // per-token position and KV row base come from the tile's table
+      // (s_col_pos / s_col_kv, filled once per tile before the epilogue)
       const bool is_v = f >= P.q_rows + P.kv_rows;
       const bool is_q = f < P.q_rows;
       const int sec = is_q ? f : (is_v ? f - P.q_rows - P.kv_rows : f - P.q_rows);
       const int head = sec / hd, within = sec % hd;
+      const size_t kv_off = (size_t)(head * 2 + (is_v ? 1 : 0)) * P.page_tokens * hd;  // (head, K or V) in a page row
+      const int pi = within / 2;
+      const bool even = (lane & 1) == 0;
+      const int dim = is_v ? within : (even ? pi : pi + half);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
-        const int m = tb * kTokBlock + n0 + i;
-        if (m >= P.M) continue;
-        const int b = P.slot0 + m / P.T, t = m % P.T;
+        const int n = n0 + i;
+        const int t = s_col_pos[n];
+        if (t < 0) continue;  // a row past the prompt tokens
         if (is_v) {
-          const int blk = P.block_table[b * P.max_blocks + t / P.page_tokens];
-          P.kv[kv_index(P, T.layer, blk, 1, head, t % P.page_tokens) + within] = f2bf(v[i]);
+          P.kv[s_col_kv[n] + kv_off + dim] = f2bf(v[i]);
           continue;
         }
-        const int pi = within / 2;
         const float2 cs = P.rope[(size_t)t * half + pi];
-        const bool even = (lane & 1) == 0;
         const float y0 = even ? v[i] : partner, y1 = even ? partner : v[i];
         const float o = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
-        const int dim = even ? pi : pi + half;
-        if (is_q) {
-          P.pq[(size_t)m * P.q_rows + head * hd + dim] = o;
-        } else {
-          const int blk = P.block_table[b * P.max_blocks + t / P.page_tokens];
-          P.kv[kv_index(P, T.layer, blk, 0, head, t % P.page_tokens) + dim] = f2bf(o);
-        }
+        if (is_q)
+          P.pq[(size_t)(tb * kTokBlock + n) * P.q_rows + head * hd + dim] = o;
+        else
+          P.kv[s_col_kv[n] + kv_off + dim] = f2bf(o);
       }
       break;
     }
@@ -1413,6 +1421,26 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
     }
     umma_commit(S.acc);
     s_mma_ok = ok;
+  }
+  // QKV tiles: the per-column position / KV-row table (threads 32.. while
+  // thread 0 issues the MMAs)
+  if (T.op == OP_BQKV || T.op == OP_MQKV) {
+    const int n = (int)threadIdx.x - 32;
+    if (n >= 0 && n < N) {
+      if (T.op == OP_BQKV) {
+        s_col_pos[n] = (n < active_batch(P) && slot_on(P, n)) ? P.seqlen[n] : 0;
+      } else {
+        const int m = T.a1 * kTokBlock + n;
+        if (m < P.M) {
+          const int b = P.slot0 + m / P.T, t = m % P.T;
+          const int blk = P.block_table[b * P.max_blocks + t / P.page_tokens];
+          s_col_pos[n] = t;
+          s_col_kv[n] = kv_index(P, T.layer, blk, 0, 0, t % P.page_tokens);
+        } else {
+          s_col_pos[n] = -1;
+        }
+      }
+    }
   }
   // batched decode: 1/rms per token column of the RMSNorm this tile consumes
   // (its x^2 sums are complete: the tile's counter covers every contribution)
