@@ -152,6 +152,22 @@ __device__ __forceinline__ void tmem_add16x2(uint32_t ta, uint32_t tb, float* v)
   for (int i = 0; i < 16; ++i) v[i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
 }
 
+// The same for 8 consecutive columns.
+__device__ __forceinline__ void tmem_add8x2(uint32_t ta, uint32_t tb, float* v) {
+  uint32_t a[8], b[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7])
+               : "r"(ta)
+               : "memory");
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7])
+               : "r"(tb)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes (64 16-bit elements), 8-row groups 1024 bytes apart.  The tile
 // base must be 1024-byte aligned; a K-step of 16 elements inside the 128-byte

@@ -1164,9 +1164,10 @@ __shared__ int s_col_pos[kMaxMmaBatch];
 
 // Adds the 16 token columns n0..n0+15 (those below nb) of one feature row to a
 // feature-major fp32 buffer row `dst` (16-byte aligned at column n0).
+template <int CW>
 __device__ __forceinline__ void red_add_cols(float* dst, const float* o, int n0, int nb) {
 #pragma unroll
-  for (int j = 0; j < 16; j += 4) {
+  for (int j = 0; j < CW; j += 4) {
     if (n0 + j + 4 <= nb) {
       red_add_v4_f32(dst + j, o[j], o[j + 1], o[j + 2], o[j + 3]);
     } else {
@@ -1183,7 +1184,10 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
   return ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)idx);
 }
 
-// Tensor-core tile epilogue for 16 token columns n0..n0+15 of feature row fl.
+// Tensor-core tile epilogue for CW token columns n0..n0+CW-1 of feature row fl
+// (CW = 8 for the batched decode, whose few columns are split finer so that all
+// eight warps share the work; 16 for the prefill).
+template <int CW>
 __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, const float* v) {
   const int f = T.a0 * 128 + fl;
   const int tb = T.a1;
@@ -1200,9 +1204,9 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       const bool even = (lane & 1) == 0;
       const int pi = within / 2;
       const int dim = is_v ? within : (even ? pi : pi + half);
-      float o[16];
+      float o[CW];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < CW; ++i) {
         const float y = v[i] * s_rn[n0 + i];
         const float partner = __shfl_xor_sync(0xffffffffu, y, 1);
         if (is_v) {
@@ -1214,12 +1218,12 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
           o[i] = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
         }
       }
-      red_add_cols(P.acc + (size_t)(sec0 + head * hd + dim) * P.mma_n + n0, o, n0, nb);
+      red_add_cols<CW>(P.acc + (size_t)(sec0 + head * hd + dim) * P.mma_n + n0, o, n0, nb);
       break;
     }
     case OP_BO:
     case OP_BDOWN:
-      red_add_cols(P.xt + (size_t)f * P.mma_n + n0, v, n0, active_batch(P));
+      red_add_cols<CW>(P.xt + (size_t)f * P.mma_n + n0, v, n0, active_batch(P));
       break;
     case OP_BGU: {
       const int nb = active_batch(P);
@@ -1227,7 +1231,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       uint8_t* hi = P.h_img[0] + (size_t)T.a0 * P.img_stride;
       uint8_t* lo = P.h_img[1] + (size_t)T.a0 * P.img_stride;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < CW; ++i) {
         const float g = v[i] * s_rn[n0 + i];
         const float up = __shfl_xor_sync(0xffffffffu, g, 1);
         if (lane & 1) continue;
@@ -1244,7 +1248,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       const int nb = active_batch(P);
       const bool valid = f < P.lm_rows;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < CW; ++i) {
         const int n = n0 + i;
         const float val = v[i] * s_rn[n];
         if (s_logits && valid && n < nb) s_logits[(size_t)n * P.logits_stride + f] = val;
@@ -1270,7 +1274,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       const bool even = (lane & 1) == 0;
       const int dim = is_v ? within : (even ? pi : pi + half);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < CW; ++i) {
         const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
         const int n = n0 + i;
         const int t = s_col_pos[n];
@@ -1292,7 +1296,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
     case OP_MO:
     case OP_MDOWN: {  // K splits of one row block add into X
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < CW; ++i) {
         const int m = tb * kTokBlock + n0 + i;
         if (m < P.M) atomicAdd(P.px + (size_t)m * P.hidden + f, v[i]);
       }
@@ -1303,7 +1307,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       uint8_t* hi = P.h_img[0] + ((size_t)tb * nkc + c) * P.img_stride;
       uint8_t* lo = P.h_img[1] + ((size_t)tb * nkc + c) * P.img_stride;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < CW; ++i) {
         const float up = __shfl_xor_sync(0xffffffffu, v[i], 1);
         if (lane & 1) continue;
         const int n = n0 + i;
@@ -1461,14 +1465,26 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, half = warp >> 2;
   const int fl = 32 * q + lane;
-  for (int cg = half; cg < N / 16; cg += 2) {  // 16-column groups alternate between the two warp halves
-    float v[16];
+  if (P.dec_mma) {
+    for (int cg = half; cg < N / 8; cg += 2) {  // 8-column groups alternate between the two warp halves
+      float v[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = 0.f;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(16 * cg);
-    for (int a = 0; a < NA; ++a)  // hi and lo parts of every accumulator
-      tmem_add16x2(lane_base + (uint32_t)(a * 2 * N), lane_base + (uint32_t)(a * 2 * N + N), v);
-    mma_epilogue(P, T, fl, 16 * cg, v);
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(8 * cg);
+      for (int a = 0; a < NA; ++a)  // hi and lo parts of every accumulator
+        tmem_add8x2(lane_base + (uint32_t)(a * 2 * N), lane_base + (uint32_t)(a * 2 * N + N), v);
+      mma_epilogue<8>(P, T, fl, 8 * cg, v);
+    }
+  } else {
+    for (int cg = half; cg < N / 16; cg += 2) {  // 16-column groups alternate between the two warp halves
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(16 * cg);
+      for (int a = 0; a < NA; ++a)  // hi and lo parts of every accumulator
+        tmem_add16x2(lane_base + (uint32_t)(a * 2 * N), lane_base + (uint32_t)(a * 2 * N + N), v);
+      mma_epilogue<16>(P, T, fl, 16 * cg, v);
+    }
   }
   tc_fence_before();
   cbar();
