@@ -72,6 +72,7 @@ struct wpk_handle {
   int32_t* d_tok_fb = nullptr;
   int32_t* d_active = nullptr;
   int32_t* d_slot_active = nullptr;  // [max_batch] slot mask (nonzero = stepped)
+  uint32_t* d_pattn_arrive = nullptr;  // prefill key-split attention: arrivals per tile
   uint32_t* d_stream_begin = nullptr;  // team schedule: worker streams
   uint32_t* d_stream = nullptr;
   // fixed-cohort serving (wpk_prefill_slots): every slot of the plan is
@@ -103,7 +104,7 @@ struct wpk_handle {
   std::string err;
   // prefill programs and their scratch (offsets in the caller's scratch)
   std::vector<std::unique_ptr<PrefillProgram>> prefills;
-  size_t off_px = 0, off_pq = 0, off_xn = 0, off_att = 0, off_hi = 0;
+  size_t off_px = 0, off_pq = 0, off_xn = 0, off_att = 0, off_hi = 0, off_ppart = 0;
   int64_t prefill_max_tokens = 0;
   int prefill_stages = 0;
   size_t smem_prefill = 0;
@@ -332,6 +333,10 @@ void scratch_layout(wpk_handle* h) {
     h->off_xn = take(n_tb * (m.hidden / 64) * 2 * kMmaChunkBytes);
     h->off_att = take(n_tb * (q_rows / 64) * 2 * kMmaChunkBytes);
     h->off_hi = take(n_tb * (m.ffn / 64) * 2 * kMmaChunkBytes);
+    // key-split attention partials: fewer (sequence, kv head, query block)
+    // tiles than workers, each with up to kMaxKeySplits splits of 128 rows
+    const int Wk = g.W > 0 ? g.W : 148;
+    h->off_ppart = take((size_t)Wk * kMaxKeySplits * 128 * (2 + kHeadDim) * 4);
   }
   if (g.plan.decode_mode == WPK_DECODE_MMA) {
     const size_t N = g.plan.dec_n, chunk = N * 128;
@@ -582,6 +587,9 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.M = g.M;
   P.T = g.T;
   P.n_tb = g.n_tb;
+  P.pattn_ks = g.pattn_ks;
+  P.ppart = reinterpret_cast<float*>(h->scratch + h->off_ppart);
+  P.pattn_arrive = h->d_pattn_arrive;
   P.ptok = tokens;
   P.px = reinterpret_cast<float*>(h->scratch + h->off_px);
   P.pq = reinterpret_cast<float*>(h->scratch + h->off_pq);
@@ -741,6 +749,7 @@ static int setup_device(wpk_handle* h) {
                o_bt = take(B * g.max_blocks * 4), o_arr = take(B * model->n_kv_heads * 4), o_best = take(B * 8),
                o_seq = take(B * 4), o_fb = take(B * 4), o_act = take(4), o_slot = take(B * 4),
                o_sb = take((g.stream_begin.size() + 1) * 4), o_st = take((g.stream.size() + 1) * 4),
+               o_pa = take((size_t)std::max(1, g.W) * 4),
                o_rb = take((size_t)model->n_layers * 2 * (model->hidden / 128 + 1) * 4),
                o_res = take(sizeof(ResDev));
   CUDA_TRY(h, cudaMalloc(&h->d_base, off));
@@ -761,6 +770,7 @@ static int setup_device(wpk_handle* h) {
   h->d_tok_fb = reinterpret_cast<int32_t*>(h->d_base + o_fb);
   h->d_active = reinterpret_cast<int32_t*>(h->d_base + o_act);
   h->d_slot_active = reinterpret_cast<int32_t*>(h->d_base + o_slot);
+  h->d_pattn_arrive = reinterpret_cast<uint32_t*>(h->d_base + o_pa);
   h->d_stream_begin = reinterpret_cast<uint32_t*>(h->d_base + o_sb);
   h->d_stream = reinterpret_cast<uint32_t*>(h->d_base + o_st);
   if (!g.stream.empty()) {

@@ -781,7 +781,7 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
 // Prefill program.  Token rows m = b*T + t (M = B*T) are processed in blocks of
 // kTokBlock rows.  Per layer: RMSNorm of each block into a bf16 hi/lo image,
 // tensor-core QKV tiles (RoPE, q to Q, k/v to the KV cache), causal attention
-// tiles of kPrefillQB queries (the GQA group of one kv head), tensor-core O
+// tiles of 128 / group queries (the GQA group of one kv head: 128 rows), tensor-core O
 // tiles (X += .), RMSNorm again, tensor-core gate/up tiles (SwiGLU into the h
 // image) and down tiles (X += .).  Then the last position of every sequence is
 // gathered and the decode program's LM head + argmax tiles produce the first
@@ -848,6 +848,16 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
     return a;
   };
   std::vector<uint32_t> layer_begin(m.n_layers + 1, 0);
+  // prefill attention: query blocks of qbt tokens (x group heads = 128 rows);
+  // split along the keys when the tiles would leave workers idle
+  const int qbt = kTokBlock / grp;
+  int KS = 0;
+  if ((int64_t)B * m.n_kv_heads * ((T + qbt - 1) / qbt) < dec.W) {
+    KS = std::max(2 * p.page_tokens, (T + kMaxKeySplits - 1) / kMaxKeySplits);
+    KS = (KS + p.page_tokens - 1) / p.page_tokens * p.page_tokens;
+    if (KS >= T) KS = 0;
+  }
+  g->pattn_ks = KS;
   const int s_o = mma_splits(nq * (h / 128), q_rows / 64, p, dec.W);
   const int s_dn = mma_splits(nq * (h / 128), m.ffn / 64, p, dec.W);
   auto krange = [](int nkc, int s, int i, int* c0, int* c1) {
@@ -878,23 +888,29 @@ std::string compile_prefill_graph(const CompiledGraph& dec, int B, int T, Compil
           acc.push_back(kvblk(l, tb, f0 - q_rows, f0 - q_rows + 128, 1));
         add(OP_MQKV, l, d.mma_qkv + (uint64_t)fb * (h / 64) * chunk, (uint32_t)(h / 64) * chunk, fb, tb, 0, h, acc);
       }
-    // causal attention: (sequence, kv head, query block)
+    // causal attention: (sequence, kv head, query block), split along the
+    // keys into splits of KS keys when those tiles are fewer than the workers
+    // (the last split to finish combines them)
     const int attn_group = 2000 + l;
     for (int b = 0; b < B; ++b)
       for (int gi = 0; gi < m.n_kv_heads; ++gi)
-        for (int qb = 0; qb * kPrefillQB < T; ++qb) {
-          const int t0 = qb * kPrefillQB, t1 = std::min(T, t0 + kPrefillQB);
+        for (int qb = 0; qb * qbt < T; ++qb) {
+          const int t0 = qb * qbt, t1 = std::min(T, t0 + qbt);
           const int m0 = b * T + t0, m1 = b * T + t1;  // query rows
-          std::vector<Access> acc;
-          for (int tb = m0 / kTokBlock; tb <= (m1 - 1) / kTokBlock; ++tb) {
-            acc.push_back(blk(BUF_PQ, q_rows, tb, gi * grp * hd, (gi + 1) * grp * hd, 0));
-            acc.push_back(blk(BUF_PATT, q_rows, tb, gi * grp * hd, (gi + 1) * grp * hd, 1, attn_group));
+          const int n_ks = KS ? (t1 + KS - 1) / KS : 1;
+          for (int ks = 0; ks < n_ks; ++ks) {
+            const int k0 = ks * KS, k1 = KS ? std::min(t1, k0 + KS) : t1;  // keys [k0, k1)
+            std::vector<Access> acc;
+            for (int tb = m0 / kTokBlock; tb <= (m1 - 1) / kTokBlock; ++tb) {
+              acc.push_back(blk(BUF_PQ, q_rows, tb, gi * grp * hd, (gi + 1) * grp * hd, 0));
+              acc.push_back(blk(BUF_PATT, q_rows, tb, gi * grp * hd, (gi + 1) * grp * hd, 1, attn_group));
+            }
+            for (int tb = (b * T + k0) / kTokBlock; tb <= (b * T + k1 - 1) / kTokBlock; ++tb) {
+              acc.push_back(kvblk(l, tb, gi * hd, (gi + 1) * hd, 0));                      // k of head gi
+              acc.push_back(kvblk(l, tb, kv_rows + gi * hd, kv_rows + (gi + 1) * hd, 0));  // v of head gi
+            }
+            add(OP_PATTN, l, 0, 0, b, gi, qb, ks, acc);
           }
-          for (int tb = (b * T) / kTokBlock; tb <= (m1 - 1) / kTokBlock; ++tb) {
-            acc.push_back(kvblk(l, tb, gi * hd, (gi + 1) * hd, 0));                      // k of head gi
-            acc.push_back(kvblk(l, tb, kv_rows + gi * hd, kv_rows + (gi + 1) * hd, 0));  // v of head gi
-          }
-          add(OP_PATTN, l, 0, 0, b, gi, qb, 0, acc);
         }
     // O and down: split along K when the token blocks alone give too few tiles
     // for the workers; the splits add into X

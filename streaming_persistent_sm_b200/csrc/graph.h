@@ -53,6 +53,7 @@ struct CompiledGraph {
   int B = 0, T = 0, M = 0, n_tb = 0;  // prefill programs
   int W = 0;                          // workers the tiles were sized for
   int o_splits = 0, down_splits = 0;  // batched decode: K splits of O and down
+  int pattn_ks = 0;                   // prefill: keys per attention split (0 = none)
   // team schedule: each tile's worker, every worker's stream of tickets
   // (stream_begin[w] .. stream_begin[w + 1] in `stream`), and each tile's
   // predecessor in its worker's stream (-1 for the first), an implicit edge

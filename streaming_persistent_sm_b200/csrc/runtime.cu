@@ -233,6 +233,11 @@ __device__ __forceinline__ void pattn_span(const KParams& P, const Tile& T, int*
   *t0 = T.a2 * qb_tokens;
   *t1 = min(P.T, *t0 + qb_tokens);
 }
+// Its keys [k0, k1): split a3 of pattn_ks keys, or all keys up to t1.
+__device__ __forceinline__ void pattn_keys(const KParams& P, const Tile& T, int t1, int* k0, int* k1) {
+  *k0 = P.pattn_ks ? T.a3 * P.pattn_ks : 0;
+  *k1 = P.pattn_ks ? min(t1, *k0 + P.pattn_ks) : t1;
+}
 
 __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int* n_chunks, int* rpc) {
   *rpc = 0;
@@ -242,9 +247,10 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
     return;
   }
   if (T.op == OP_PATTN) {
-    int t0, t1;
+    int t0, t1, k0, k1;
     pattn_span(P, T, &t0, &t1);
-    *n_chunks = (t1 - 1) / P.page_tokens + 1;
+    pattn_keys(P, T, t1, &k0, &k1);
+    *n_chunks = (k1 - 1) / P.page_tokens - k0 / P.page_tokens + 1;
     return;
   }
   if (T.op == OP_ATTN) {  // attn_pps KV pages per ring stage
@@ -325,7 +331,10 @@ __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uin
     // split, packed into the stage
     const uint32_t bytes = 2u * (uint32_t)P.page_tokens * (uint32_t)P.head_dim * 2u;
     if (T.op == OP_PATTN) {
-      const int blk = P.block_table[(P.slot0 + T.a0) * P.max_blocks + k];
+      int t0, t1, k0, k1;
+      pattn_span(P, T, &t0, &t1);
+      pattn_keys(P, T, t1, &k0, &k1);
+      const int blk = P.block_table[(P.slot0 + T.a0) * P.max_blocks + k0 / P.page_tokens + k];
       mbar_arrive_expect_tx(bar, bytes);
       bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, T.a1, 0), bytes, bar);
       return;
@@ -1504,8 +1513,10 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
 __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
                            volatile int* abort, uint32_t tile) {
   const int b = T.a0, g = T.a1, grp = P.group, hd = P.head_dim;
-  int t0, t1;
+  int t0, t1, k_first, k_end;
   pattn_span(P, T, &t0, &t1);
+  pattn_keys(P, T, t1, &k_first, &k_end);
+  k_first = k_first / P.page_tokens * P.page_tokens;  // splits start on a page
   const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
   const int qi = r / grp, hh = r % grp;
   const int t = t0 + qi;
@@ -1533,7 +1544,8 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     const uint8_t* stage = S.ring + (size_t)st * P.stage_bytes;
     const uint32_t* Kw = reinterpret_cast<const uint32_t*>(stage) + 16 * part;
     const uint32_t* Vw = reinterpret_cast<const uint32_t*>(stage + (size_t)P.page_tokens * hd * 2) + 16 * part;
-    const int rows = min(P.page_tokens, t1 - k * P.page_tokens);
+    const int kp = k_first + k * P.page_tokens;  // first key of this page
+    const int rows = min(P.page_tokens, k_end - kp);
     for (int j0 = 0; j0 < rows; j0 += 16) {  // 16 keys at a time keeps the scores in registers
       float sc[16];
       float mloc = -INFINITY;
@@ -1558,7 +1570,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
           }
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        const int key = k * P.page_tokens + j;
+        const int key = kp + j;
         sc[jj] = (j < rows && key <= t) ? acc : -INFINITY;
         mloc = fmaxf(mloc, sc[jj]);
       }
@@ -1590,6 +1602,44 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     cbar();
     if (threadIdx.x == 0) mbar_arrive(&S.empty[st]);
     ++cur.c;
+  }
+  if (P.pattn_ks) {
+    // a key split: store this split's (m, l, o) of every row; the last split
+    // of the (sequence, kv head, query block) to arrive combines them
+    const int n_ks = (t1 + P.pattn_ks - 1) / P.pattn_ks;
+    const int n_qb = (P.T + kTokBlock / grp - 1) / (kTokBlock / grp);
+    const int idx = (b * P.n_kv + g) * n_qb + T.a2;
+    float* base = P.ppart + (size_t)idx * kMaxKeySplits * 128 * (2 + kHeadDim);
+    float* mine = base + ((size_t)T.a3 * 128 + r) * (2 + kHeadDim);
+#pragma unroll
+    for (int d = 0; d < 32; ++d) mine[2 + 32 * part + d] = o[d];
+    if (part == 0) {
+      mine[0] = mrun;  // -inf with l = 0 when no key of the split is at or before the query
+      mine[1] = lrun;
+    }
+    __shared__ int s_last_split;
+    cbar();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const uint32_t old = atomicAdd(P.pattn_arrive + idx, 1u);
+      s_last_split = old == (uint32_t)n_ks - 1u;
+      if (s_last_split) P.pattn_arrive[idx] = 0u;
+      __threadfence();
+    }
+    cbar();
+    if (!s_last_split) return true;
+    float M = -INFINITY;
+    for (int j = 0; j < n_ks; ++j) M = fmaxf(M, __ldcg(base + ((size_t)j * 128 + r) * (2 + kHeadDim)));
+    lrun = 0.f;
+#pragma unroll
+    for (int d = 0; d < 32; ++d) o[d] = 0.f;
+    for (int j = 0; j < n_ks; ++j) {
+      const float* w = base + ((size_t)j * 128 + r) * (2 + kHeadDim);
+      const float f = M == -INFINITY ? 0.f : expf(__ldcg(w) - M);
+      lrun = fmaf(__ldcg(w + 1), f, lrun);
+#pragma unroll
+      for (int d = 0; d < 32; ++d) o[d] = fmaf(__ldcg(w + 2 + 32 * part + d), f, o[d]);
+    }
   }
   if (valid) {
     const float inv = 1.0f / lrun;

@@ -50,8 +50,8 @@ enum Op : uint16_t {
 };
 
 constexpr int kTokBlock = 128;   // tokens per tensor-core tile (the MMA N)
-constexpr int kPrefillQB = 32;   // queries per prefill attention tile
 constexpr int kNormRows = 16;    // token rows per prefill RMSNorm tile
+constexpr int kMaxKeySplits = 8; // key splits of one prefill attention tile, at most
 constexpr int kMaxMmaBatch = 128;  // sequences of a batched decode step (MMA N <= 128)
 constexpr int kMaxInTables = 16;   // input tables a step's input may sum over
 constexpr int kMmaChunkBytes = 128 * 128;  // 128 rows x 64 bf16, one K chunk
@@ -196,6 +196,13 @@ struct KParams {
   uint8_t* xn_img[2];        // hi/lo image of the normalised activations [n_tb][hidden/64][16 KB]
   uint8_t* att_img[2];       // hi/lo image of the attention output     [n_tb][q_rows/64][16 KB]
   uint8_t* h_img[2];         // hi/lo image of the SwiGLU output        [n_tb][ffn/64][16 KB]
+  // prefill attention split along keys (small batches, where the (sequence,
+  // kv head, query block) tiles are fewer than the workers): keys per split
+  // (0 = no split), the splits' partial (m, l, o) per query row, and an
+  // arrival counter per (sequence, kv head, query block)
+  int pattn_ks;
+  float* ppart;              // [tiles][kMaxKeySplits][128 rows][2 + head_dim]
+  uint32_t* pattn_arrive;    // [workers]
   // tensor-core operand geometry: the MMA N (tokens per tile) and the bytes of
   // one 64-column activation chunk (N rows of 128 bytes, 128-byte swizzle)
   int mma_n, act_chunk;

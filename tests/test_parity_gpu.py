@@ -54,6 +54,17 @@ def test_tiny_prefill_and_16_steps(weights, dec, name):
         eng.close()
 
 
+def test_tiny_prefill_attention_split_along_keys(weights, dec):
+    # 2 x 2 (sequence, kv head) pairs x 3 query blocks of 64 tokens are fewer
+    # tiles than the workers, so the prefill's causal attention is split along
+    # the keys (128 per split) and the last split to finish combines them
+    eng = W.Engine(S, weights, 2, 256)
+    try:
+        run_teacher_forced(eng, dec, _prompts(2, 190, seed=7), steps=3, max_context=256)
+    finally:
+        eng.close()
+
+
 def test_tiny_batch3_ragged_tail(weights, dec):
     # 3 sequences; prompt of 37 tokens ends inside the second 32-token page
     eng = W.Engine(S, weights, 3, 96, page_tokens=32)
