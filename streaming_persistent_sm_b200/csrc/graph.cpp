@@ -615,8 +615,13 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   {
     int sp = p.split_pages;
     if (sp == 0) {
+      // about two attention tiles per worker on CUDA cores; on the tensor-core
+      // decode, whose ring stages also hold the preceding QKV tile's weights,
+      // at most one per worker (a second tile's pages would be staged late:
+      // 1572 against 1767 us per step at batch 16)
       const int pairs = p.max_batch * m.n_kv_heads;
-      const int ns = std::max(1, std::min(g->max_blocks, (2 * W + pairs / 2) / pairs));
+      const int per = p.decode_mode == WPK_DECODE_MMA ? W : 2 * W;
+      const int ns = std::max(1, std::min(g->max_blocks, (per + pairs / 2) / pairs));
       sp = (g->max_blocks + ns - 1) / ns;
     }
     g->plan.split_pages = sp;
