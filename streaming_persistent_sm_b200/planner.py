@@ -59,8 +59,11 @@ def calibrate(trace: np.ndarray, tile_bytes: np.ndarray, edges: np.ndarray, byte
     """Per-tile costs from a trace of the monolith (records in any order).
 
     service = end - start of each tile; load = its staged weight bytes over one
-    worker's share of the load bandwidth; sync = the median, over tiles with
-    predecessors, of start - (latest predecessor end)."""
+    worker's share of the load bandwidth; sync = the median, over tiles that
+    waited for a predecessor (its last predecessor ended after the worker's
+    previous tile did, so the worker was idle), of start - (latest predecessor
+    end).  A tile that waited for its own worker measures the queue, not the
+    hop, and is left out."""
     tr = np.sort(trace, order="tile")
     n = len(tr)
     start = tr["t_start_ns"].astype(np.float64)
@@ -70,9 +73,16 @@ def calibrate(trace: np.ndarray, tile_bytes: np.ndarray, edges: np.ndarray, byte
     last_pred = np.full(n, -np.inf)
     if len(edges):
         np.maximum.at(last_pred, edges[:, 1], end[edges[:, 0]])
-    has = np.isfinite(last_pred)
-    hops = start[has] - last_pred[has]
-    sync = float(np.median(hops[hops >= 0])) if np.any(hops >= 0) else 0.0
+    # end of the previous tile on the same worker (tiles of a worker in start order)
+    prev_end = np.full(n, -np.inf)
+    worker = tr["worker"].astype(np.int64)
+    order = np.lexsort((start, worker))
+    same = worker[order][1:] == worker[order][:-1]
+    prev_end[order[1:][same]] = end[order[:-1][same]]
+    waited = np.isfinite(last_pred) & (last_pred >= prev_end)
+    hops = start[waited] - last_pred[waited]
+    hops = hops[hops >= 0]
+    sync = float(np.median(hops)) if len(hops) else 0.0
     return Calibration(service, load, sync, first_chunk_ns)
 
 

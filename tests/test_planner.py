@@ -116,6 +116,7 @@ def test_calibration_from_a_synthetic_trace(h):
     e = W.wpk_get_edges(h)
     tr = np.zeros(n, dtype=W.TRACE_DTYPE)
     tr["tile"] = np.arange(n)[::-1]  # records in any order
+    tr["worker"] = (tr["tile"] % 7).astype(np.uint16)
     tr["t_start_ns"] = (10_000 * tr["tile"]).astype(np.uint64)
     tr["t_end_ns"] = tr["t_start_ns"] + 4_000
     cal = PL.calibrate(tr, np.full(n, 8192), e, bytes_per_ns_per_worker=4.096)
@@ -124,8 +125,24 @@ def test_calibration_from_a_synthetic_trace(h):
     start = 10_000.0 * np.arange(n)
     last = np.full(n, -np.inf)
     np.maximum.at(last, e[:, 1], start[e[:, 0]] + 4000.0)
-    hop = start[np.isfinite(last)] - last[np.isfinite(last)]
-    assert cal.sync_ns == pytest.approx(np.median(hop))
+    # tile t follows tile t - 7 on its worker; the hop counts only where the
+    # last predecessor ended after that
+    prev = np.where(np.arange(n) >= 7, start - 70_000.0 + 4000.0, -np.inf)
+    ok = np.isfinite(last) & (last >= prev)
+    hop = start[ok] - last[ok]
+    assert cal.sync_ns == pytest.approx(np.median(hop[hop >= 0]))
+
+
+def test_calibration_leaves_out_tiles_that_waited_for_their_worker(h):
+    # one worker runs every tile back to back: no tile waited on a dependency,
+    # so no hop is measured
+    n = W.wpk_graph_stats_get(h)["n_tiles"]
+    e = W.wpk_get_edges(h)
+    tr = np.zeros(n, dtype=W.TRACE_DTYPE)
+    tr["tile"] = np.arange(n)
+    tr["t_start_ns"] = (1000 * np.arange(n)).astype(np.uint64)
+    tr["t_end_ns"] = tr["t_start_ns"] + 1000
+    assert PL.calibrate(tr, np.zeros(n), e, bytes_per_ns_per_worker=1.0).sync_ns == 0.0
 
 
 def test_dispatch_fit_and_ranking(h):
