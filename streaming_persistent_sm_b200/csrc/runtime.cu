@@ -1507,98 +1507,189 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
 }
 
 // Causal GQA attention for the queries [t0, t1) of sequence b and the query
-// heads of kv head g (online softmax over the staged KV pages, CUDA cores).
-// Thread pair (2r, 2r+1) owns query row r = (query, head) and splits its 64
-// dims in halves; the result goes to the hi/lo attention image.
+// heads of kv head g, on the tensor cores.  The tile's 128 rows (query qi and
+// head hh at row qi * group + hh) are the MMA's M and TMEM lanes 0-127; warps
+// 0-3 own one row per thread.  Per staged KV page of 64 keys:
+//   1. all warps build, in the stage, the page's K rows and its V transposed
+//      ([dim][key]) as K-major operands with the 128-byte swizzle;
+//   2. S = (Q_hi + Q_lo) K^T on the tensor cores, Q (scaled by 1/sqrt(d))
+//      split into bf16 hi and lo halves held in TMEM;
+//   3. each row's online softmax over S (causal mask key <= query), the
+//      probabilities split into bf16 hi and lo written to TMEM;
+//   4. O_page = (P_hi + P_lo) V^T on the tensor cores, added into the row's
+//      fp32 output registers.
+// The hi/lo splits keep q and p to about 16 significant bits; K and V are
+// the cache's bf16 values; every product accumulates in fp32.  A key split
+// (pattn_ks) writes its (m, l, o) partial and the last split to finish
+// combines them, as the decode attention does.
+namespace pattn {
+constexpr uint32_t kS = 0, kO = 64, kQh = 128, kQl = 160, kPh = 192, kPl = 224;  // TMEM columns
+constexpr int kKRows = 16384, kVt = 24576;  // stage offsets of the swizzled K rows and V transposed
+}
+
 __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
-                           volatile int* abort, uint32_t tile) {
+                           ConsumerState& cs, volatile int* abort, uint32_t tile) {
   const int b = T.a0, g = T.a1, grp = P.group, hd = P.head_dim;
   int t0, t1, k_first, k_end;
   pattn_span(P, T, &t0, &t1);
   pattn_keys(P, T, t1, &k_first, &k_end);
   k_first = k_first / P.page_tokens * P.page_tokens;  // splits start on a page
-  const int r = threadIdx.x >> 1, part = threadIdx.x & 1;
+  const int warp = threadIdx.x >> 5;
+  const bool row_thread = warp < 4;  // warps 0-3: one tile row (TMEM lane) each
+  const int r = threadIdx.x;         // the row, for row threads
   const int qi = r / grp, hh = r % grp;
   const int t = t0 + qi;
-  const bool valid = t < t1;
+  const bool valid = row_thread && t < t1;
   const int m = b * P.T + (valid ? t : t0);
   const int head = g * grp + hh;
-  const float scale = 1.0f / sqrtf((float)hd);
-  float q[32], o[32];
-  {
-    const float4* qs = reinterpret_cast<const float4*>(P.pq + (size_t)m * P.q_rows + head * hd + 32 * part);
+  const uint32_t tmem = s_tmem;
+  const uint32_t lane_addr = ((uint32_t)(32 * (warp & 3)) << 16);
+  // Q row -> TMEM (hi, lo), scaled by 1/sqrt(64) = 1/8 (exact in bf16)
+  if (row_thread) {
+    const float4* qs = reinterpret_cast<const float4*>(P.pq + (size_t)m * P.q_rows + head * hd);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 a = __ldcg(qs + i);
-      q[4 * i] = a.x * scale; q[4 * i + 1] = a.y * scale; q[4 * i + 2] = a.z * scale; q[4 * i + 3] = a.w * scale;
+    for (int c = 0; c < 4; ++c) {  // 16 dims = 8 columns per store
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 q4 = __ldcg(qs + 4 * c + e);
+        const float qv[4] = {q4.x * 0.125f, q4.y * 0.125f, q4.z * 0.125f, q4.w * 0.125f};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(qv[2 * h2], qv[2 * h2 + 1]);
+          hi[2 * e + h2] = *reinterpret_cast<const uint32_t*>(&hv);
+          lo[2 * e + h2] = pack_bf16x2(qv[2 * h2] - __bfloat162float(hv.x), qv[2 * h2 + 1] - __bfloat162float(hv.y));
+        }
+      }
+      tmem_st8(tmem + lane_addr + pattn::kQh + 8 * c, hi);
+      tmem_st8(tmem + lane_addr + pattn::kQl + 8 * c, lo);
     }
+    tmem_st_wait();
   }
+  float o[64];
 #pragma unroll
-  for (int d = 0; d < 32; ++d) o[d] = 0.f;
+  for (int d = 0; d < 64; ++d) o[d] = 0.f;
   float mrun = -INFINITY, lrun = 0.f;
+  const uint32_t idesc = idesc_f16(128, 64, true);
   bool ok = true;
   for (int k = 0; k < n_chunks; ++k) {
     const int st = cur.c % P.n_stages;
     if (!wait_phase(P, &S.full[st], (cur.c / P.n_stages) & 1u, abort, tile)) ok = false;
     if (!cbar_and(ok)) return false;
-    const uint8_t* stage = S.ring + (size_t)st * P.stage_bytes;
-    const uint32_t* Kw = reinterpret_cast<const uint32_t*>(stage) + 16 * part;
-    const uint32_t* Vw = reinterpret_cast<const uint32_t*>(stage + (size_t)P.page_tokens * hd * 2) + 16 * part;
+    uint8_t* stage = S.ring + (size_t)st * P.stage_bytes;
     const int kp = k_first + k * P.page_tokens;  // first key of this page
     const int rows = min(P.page_tokens, k_end - kp);
-    for (int j0 = 0; j0 < rows; j0 += 16) {  // 16 keys at a time keeps the scores in registers
-      float sc[16];
-      float mloc = -INFINITY;
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const int j = j0 + jj;
-        float acc = 0.f;
-        if (j < rows) {
-          // the thread's 32 dims of key j: four 16-byte loads (a broadcast
-          // across the threads of the same half)
-          const uint4* kr = reinterpret_cast<const uint4*>(Kw + j * (hd / 2));
-#pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) {
-            const uint4 k4 = kr[w4];
-            const uint32_t kw[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int w = 4 * w4 + e;
-              acc = fmaf(q[2 * w], __uint_as_float(kw[e] << 16), acc);
-              acc = fmaf(q[2 * w + 1], __uint_as_float(kw[e] & 0xFFFF0000u), acc);
-            }
-          }
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        const int key = kp + j;
-        sc[jj] = (j < rows && key <= t) ? acc : -INFINITY;
-        mloc = fmaxf(mloc, sc[jj]);
+    // 1. swizzled K rows (unit u of row j at u ^ (j & 7)) and V transposed
+    {
+      const uint4* kr = reinterpret_cast<const uint4*>(stage);
+      for (int i = threadIdx.x; i < 64 * 8; i += kThreads) {
+        const int j = i >> 3, u = i & 7;
+        const uint4 v = j < rows ? kr[i] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(stage + pattn::kKRows + j * 128 + ((u ^ (j & 7)) << 4)) = v;
       }
-      const float mnew = fmaxf(mrun, mloc);
-      if (mnew == -INFINITY) continue;
-      const float corr = (mrun > -INFINITY) ? expf(mrun - mnew) : 0.f;
-      lrun *= corr;
+      const uint16_t* vr = reinterpret_cast<const uint16_t*>(stage + (size_t)P.page_tokens * hd * 2);
+      for (int i = threadIdx.x; i < 64 * 8; i += kThreads) {  // (dim d, keys 8 ku .. 8 ku + 7)
+        const int d = i & 63, ku = i >> 6;  // a warp reads 32 adjacent dims of one key row
+        uint32_t w[4];
 #pragma unroll
-      for (int d = 0; d < 32; ++d) o[d] *= corr;
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const float p = (sc[jj] == -INFINITY) ? 0.f : expf(sc[jj] - mnew);
-        lrun += p;
-        const uint4* vr = reinterpret_cast<const uint4*>(Vw + min(j0 + jj, rows - 1) * (hd / 2));
-#pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) {
-          const uint4 v4 = vr[w4];
-          const uint32_t vw[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int w = 4 * w4 + e;
-            o[2 * w] = fmaf(p, __uint_as_float(vw[e] << 16), o[2 * w]);
-            o[2 * w + 1] = fmaf(p, __uint_as_float(vw[e] & 0xFFFF0000u), o[2 * w + 1]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const int j0 = 8 * ku + 2 * e;
+          const uint32_t x0 = j0 < rows ? vr[j0 * 64 + d] : 0u, x1 = j0 + 1 < rows ? vr[(j0 + 1) * 64 + d] : 0u;
+          w[e] = x0 | (x1 << 16);
         }
+        *reinterpret_cast<uint4*>(stage + pattn::kVt + d * 128 + ((ku ^ (d & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      mrun = mnew;
     }
+    fence_proxy_async_smem();  // the MMAs read these generic-proxy writes
+    tc_fence_before();
+    cbar();
+    tc_fence_after();
+    // 2. S = Q K^T
+    if (threadIdx.x == 0) {
+      const uint32_t kb = smem_u32(stage + pattn::kKRows);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        umma_f16_ta(tmem + pattn::kS, tmem + pattn::kQh + 8 * kk, sdesc_k_sw128(kb + kk * 32), idesc, kk > 0);
+        umma_f16_ta(tmem + pattn::kS, tmem + pattn::kQl + 8 * kk, sdesc_k_sw128(kb + kk * 32), idesc, 1u);
+      }
+      umma_commit(S.acc);
+    }
+    if (!wait_phase(P, S.acc, cs.acc_phase, abort, tile)) ok = false;
+    cs.acc_phase ^= 1u;
+    if (!cbar_and(ok)) return false;
+    tc_fence_after();
+    // 3. online softmax of the row over the page's keys; P (hi, lo) -> TMEM
+    float corr = 1.f;
+    if (row_thread) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float sv[16];
+        tmem_ld16(tmem + lane_addr + pattn::kS + 16 * c, sv);
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int key = kp + 16 * c + jj;
+          if (valid && 16 * c + jj < rows && key <= t) mx = fmaxf(mx, sv[jj]);
+        }
+      }
+      const float mnew = fmaxf(mrun, mx);
+      if (mnew != -INFINITY) {
+        corr = mrun == -INFINITY ? 0.f : expf(mrun - mnew);
+        mrun = mnew;
+      }
+      float psum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float sv[16];
+        tmem_ld16(tmem + lane_addr + pattn::kS + 16 * c, sv);
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int jj = 0; jj < 16; jj += 2) {
+          float pv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = kp + 16 * c + jj + e;
+            pv[e] = (valid && 16 * c + jj + e < rows && key <= t) ? expf(sv[jj + e] - mrun) : 0.f;
+            psum += pv[e];
+          }
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(pv[0], pv[1]);
+          hi[jj / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          lo[jj / 2] = pack_bf16x2(pv[0] - __bfloat162float(hv.x), pv[1] - __bfloat162float(hv.y));
+        }
+        tmem_st8(tmem + lane_addr + pattn::kPh + 8 * c, hi);
+        tmem_st8(tmem + lane_addr + pattn::kPl + 8 * c, lo);
+      }
+      tmem_st_wait();
+      lrun = lrun * corr + psum;
+    }
+    tc_fence_before();
+    cbar();
+    tc_fence_after();
+    // 4. O_page = P V^T
+    if (threadIdx.x == 0) {
+      const uint32_t vb = smem_u32(stage + pattn::kVt);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        umma_f16_ta(tmem + pattn::kO, tmem + pattn::kPh + 8 * kk, sdesc_k_sw128(vb + kk * 32), idesc, kk > 0);
+        umma_f16_ta(tmem + pattn::kO, tmem + pattn::kPl + 8 * kk, sdesc_k_sw128(vb + kk * 32), idesc, 1u);
+      }
+      umma_commit(S.acc);
+    }
+    if (!wait_phase(P, S.acc, cs.acc_phase, abort, tile)) ok = false;
+    cs.acc_phase ^= 1u;
+    if (!cbar_and(ok)) return false;
+    tc_fence_after();
+    if (row_thread) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float ov[16];
+        tmem_ld16(tmem + lane_addr + pattn::kO + 16 * c, ov);
+#pragma unroll
+        for (int d = 0; d < 16; ++d) o[16 * c + d] = fmaf(o[16 * c + d], corr, ov[d]);
+      }
+    }
+    // the stage and the TMEM operands are free again: hand the stage back
+    tc_fence_before();
     cbar();
     if (threadIdx.x == 0) mbar_arrive(&S.empty[st]);
     ++cur.c;
@@ -1610,10 +1701,10 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     const int n_qb = (P.T + kTokBlock / grp - 1) / (kTokBlock / grp);
     const int idx = (b * P.n_kv + g) * n_qb + T.a2;
     float* base = P.ppart + (size_t)idx * kMaxKeySplits * 128 * (2 + kHeadDim);
-    float* mine = base + ((size_t)T.a3 * 128 + r) * (2 + kHeadDim);
+    if (row_thread) {
+      float* mine = base + ((size_t)T.a3 * 128 + r) * (2 + kHeadDim);
 #pragma unroll
-    for (int d = 0; d < 32; ++d) mine[2 + 32 * part + d] = o[d];
-    if (part == 0) {
+      for (int d = 0; d < 64; d += 2) *reinterpret_cast<float2*>(mine + 2 + d) = make_float2(o[d], o[d + 1]);
       mine[0] = mrun;  // -inf with l = 0 when no key of the split is at or before the query
       mine[1] = lrun;
     }
@@ -1628,17 +1719,23 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     }
     cbar();
     if (!s_last_split) return true;
-    float M = -INFINITY;
-    for (int j = 0; j < n_ks; ++j) M = fmaxf(M, __ldcg(base + ((size_t)j * 128 + r) * (2 + kHeadDim)));
-    lrun = 0.f;
+    if (row_thread) {
+      float M = -INFINITY;
+      for (int j = 0; j < n_ks; ++j) M = fmaxf(M, __ldcg(base + ((size_t)j * 128 + r) * (2 + kHeadDim)));
+      lrun = 0.f;
 #pragma unroll
-    for (int d = 0; d < 32; ++d) o[d] = 0.f;
-    for (int j = 0; j < n_ks; ++j) {
-      const float* w = base + ((size_t)j * 128 + r) * (2 + kHeadDim);
-      const float f = M == -INFINITY ? 0.f : expf(__ldcg(w) - M);
-      lrun = fmaf(__ldcg(w + 1), f, lrun);
+      for (int d = 0; d < 64; ++d) o[d] = 0.f;
+      for (int j = 0; j < n_ks; ++j) {
+        const float* w = base + ((size_t)j * 128 + r) * (2 + kHeadDim);
+        const float f = M == -INFINITY ? 0.f : expf(__ldcg(w) - M);
+        lrun = fmaf(__ldcg(w + 1), f, lrun);
 #pragma unroll
-      for (int d = 0; d < 32; ++d) o[d] = fmaf(__ldcg(w + 2 + 32 * part + d), f, o[d]);
+        for (int d = 0; d < 64; d += 2) {  // records are 66 floats: 8-byte aligned
+          const float2 x = __ldcg(reinterpret_cast<const float2*>(w + 2 + d));
+          o[d] = fmaf(x.x, f, o[d]);
+          o[d + 1] = fmaf(x.y, f, o[d + 1]);
+        }
+      }
     }
   }
   if (valid) {
@@ -1646,7 +1743,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     const int tb = m / kTokBlock, n = m % kTokBlock, nkc = P.q_rows / 64;
     const size_t blk = ((size_t)tb * nkc + head) * P.img_stride;  // 64-column chunk == one head
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       uint32_t ph[4], pl[4];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
@@ -1655,7 +1752,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
         ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
         pl[e / 2] = pack_bf16x2(a0 - __bfloat162float(hv.x), a1 - __bfloat162float(hv.y));
       }
-      const uint32_t off = sw128_offset(n, 32 * part + 8 * u);
+      const uint32_t off = sw128_offset(n, 8 * u);
       *reinterpret_cast<uint4*>(P.att_img[0] + blk + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
       *reinterpret_cast<uint4*>(P.att_img[1] + blk + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
     }
@@ -2066,7 +2163,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
               if (T.op == OP_PEMBED) ok = body_pembed(P, T);
               else if (T.op == OP_GATHER) ok = body_gather(P);
               else if (T.op == OP_NORM) ok = body_norm(P, T);
-              else if (T.op == OP_PATTN) ok = body_pattn(P, T, S, cur, n_chunks, &s_abort, t);
+              else if (T.op == OP_PATTN) ok = body_pattn(P, T, S, cur, n_chunks, cs, &s_abort, t);
               else ok = body_mma(P, T, S, cur, n_chunks, cs, &s_abort, t);
             } else {
               known = false;
