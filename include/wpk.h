@@ -126,7 +126,7 @@ typedef struct wpk_plan_cfg {
                            runs through the decode program one position at a
                            time)                                                */
   int decode;           /* WPK_DECODE_AUTO (0): tensor-core decode tiles when
-                           max_batch > 8 and the shapes allow, else CUDA-core
+                           max_batch > 4 and the shapes allow, else CUDA-core
                            GEMV tiles; WPK_DECODE_GEMV; WPK_DECODE_MMA (the
                            step's sequences are the MMA N dimension, so
                            max_batch <= 128)                                    */

@@ -181,13 +181,15 @@ int check_live(wpk_handle* h) {
   return WPK_OK;
 }
 
-// Tensor-core accumulators: up to 4 of 2N columns each within the 512 TMEM
-// columns of an SM (one worker CTA per SM when a tile uses tensor cores).
+// Tensor-core accumulators: a tile's buffer holds up to 4 accumulators of 2N
+// columns; a worker holds two buffers within the 512 TMEM columns of an SM
+// (one worker CTA per SM when its buffers take all 512).
 void set_mma_geometry(KParams* P) {
   const int w = 2 * P->mma_n;
-  P->mma_acc = std::max(1, std::min(4, 512 / w));
+  P->mma_acc = std::max(1, std::min(4, 256 / w));
+  P->mma_buf_cols = w * P->mma_acc;
   int cols = 32;
-  while (cols < w * P->mma_acc) cols <<= 1;
+  while (cols < 2 * P->mma_buf_cols) cols <<= 1;
   P->tmem_cols = cols;
 }
 
@@ -215,8 +217,9 @@ KParams make_params(const wpk_handle* h) {
   P.max_blocks = g.max_blocks;
   P.split_tokens = g.split_tokens;
   P.n_splits = g.n_splits;
-  P.n_stages = g.plan.slot_bytes / kStageBytes;
-  P.stage_bytes = kStageBytes;
+  P.gemv_cps = gemv_chunks_per_stage(g.plan.slot_bytes);
+  P.stage_bytes = P.gemv_cps * kStageBytes;
+  P.n_stages = g.plan.slot_bytes / P.stage_bytes;
   P.lookahead = g.plan.lookahead;
   P.act_bytes = g.plan.act_bytes;
   P.timeout_ns = g.plan.wait_timeout_ns;
@@ -279,6 +282,7 @@ KParams make_params(const wpk_handle* h) {
     P.mma_cps = g.plan.dec_cps;
     P.stage_bytes = g.plan.dec_stage_bytes;
     P.n_stages = g.plan.dec_stages;
+    P.gemv_cps = 1;
     P.act_bytes = g.plan.dec_act_bytes;
     P.o_splits = g.o_splits;
     P.down_splits = g.down_splits;
@@ -387,7 +391,11 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
     P.t_begin = og.begin;
     P.t_end = og.end;
     P.per_op = 1;
-    if (!P.dec_mma) P.n_stages = g.plan.per_op_slot / kStageBytes;
+    if (!P.dec_mma) {
+      P.gemv_cps = gemv_chunks_per_stage(g.plan.per_op_slot);
+      P.stage_bytes = P.gemv_cps * kStageBytes;
+      P.n_stages = g.plan.per_op_slot / P.stage_bytes;
+    }
     void* args[] = {&P};
     cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(og.end - og.begin), dim3(kCtaThreads), args,
                                      h->smem_per_op, h->capture_stream);
@@ -575,6 +583,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.trace_buf = prog->d_trace;
   P.stage_bytes = 3 * kMmaChunkBytes;
   P.n_stages = h->prefill_stages;
+  P.gemv_cps = 1;
   P.uses_tmem = 1;
   // the prefill program's own geometry (its LM head tiles are GEMV tiles)
   P.dec_mma = 0;
@@ -693,7 +702,11 @@ static int setup_device(wpk_handle* h) {
   if (h->smem > (size_t)kMaxSmem || h->smem_per_op > (size_t)kMaxSmem)
     return fail(h, WPK_ERR_UNSUPPORTED, "staging slot and activations exceed shared memory");
   if (p.prefill_mode == WPK_PREFILL_MMA) {
-    const size_t fixed = worker_smem_bytes(0, 0, p.act_bytes);
+    // the kernel's static shared memory counts against the same per-CTA limit
+    cudaFuncAttributes fa{};
+    CUDA_TRY(h, cudaFuncGetAttributes(&fa, prefill_kernel_ptr()));
+    const size_t fixed = worker_smem_bytes(0, 0, p.act_bytes) + fa.sharedSizeBytes;
+    if (fixed >= (size_t)kMaxSmem) return fail(h, WPK_ERR_UNSUPPORTED, "no room for the prefill staging ring");
     h->prefill_stages = (int)std::min<size_t>(kMaxStages, ((size_t)kMaxSmem - fixed) / (3 * kMmaChunkBytes));
     if (h->prefill_stages < 2) return fail(h, WPK_ERR_UNSUPPORTED, "no room for the prefill staging ring");
     h->smem_prefill = worker_smem_bytes(h->prefill_stages, 3 * kMmaChunkBytes, p.act_bytes);

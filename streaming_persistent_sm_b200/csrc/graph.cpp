@@ -110,7 +110,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
   // faster with fewer, larger splits (64 KB measured best at batch 16 and 48)
   p->tile_bytes = in.tile_bytes ? in.tile_bytes
                                 : ((in.decode == WPK_DECODE_MMA ||
-                                    (in.decode == WPK_DECODE_AUTO && in.max_batch > kMaxGemvBatch))
+                                    (in.decode == WPK_DECODE_AUTO && in.max_batch > kAutoGemvBatch))
                                        ? 65536
                                        : 32768);
   if (p->tile_bytes < 1024 || p->tile_bytes > 1 << 20) return "tile_bytes must be in [1K, 1M]";
@@ -125,7 +125,7 @@ std::string normalize_plan(const wpk_model_cfg& m, const wpk_plan_cfg& in, Plan*
     const bool mma_ok = (qr + 2 * kvr) % 128 == 0 && m.hidden % 128 == 0 && (2 * m.ffn) % 128 == 0 &&
                         m.hidden % 64 == 0 && qr % 128 == 0 && m.ffn % 64 == 0 && kvr % 128 == 0;
     if (in.decode == WPK_DECODE_AUTO)
-      p->decode_mode = (in.max_batch > kMaxGemvBatch && in.max_batch <= kMaxMmaBatch && mma_ok) ? WPK_DECODE_MMA
+      p->decode_mode = (in.max_batch > kAutoGemvBatch && in.max_batch <= kMaxMmaBatch && mma_ok) ? WPK_DECODE_MMA
                                                                                                 : WPK_DECODE_GEMV;
     else if (in.decode == WPK_DECODE_MMA) {
       if (!mma_ok) { *code = WPK_ERR_UNSUPPORTED; return "shapes do not fit the tensor-core decode tiles"; }
@@ -340,7 +340,7 @@ int rows_per_tile(int row_bytes, int op_rows, const Plan& p, int W) {
   if (rpc < 2) rpc = 2;
   int r = std::max(p.tile_bytes / row_bytes, (op_rows + W - 1) / std::max(1, W));
   r = (r + rpc - 1) / rpc * rpc;
-  if (p.max_batch > kMaxGemvBatch) r = std::min(r, (p.slot_bytes / kStageBytes) * rpc);
+  if (p.max_batch > kMaxGemvBatch) r = std::min(r, gemv_ring_chunks(p.slot_bytes) * rpc);
   r = std::min(r, kMaxTileRows / rpc * rpc);
   return std::max(r, 2);
 }
@@ -564,8 +564,10 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
   int nch = (m.ffn + 2047) / 2048;
   while (m.ffn % nch || (m.ffn / nch) % 8) ++nch;
   const int kc = m.ffn / nch;
-  if (h * 2 > kStageBytes || q_rows * 2 > kStageBytes || kc * 2 > kStageBytes)
-    return "a weight row does not fit one 16 KB stage";
+  // a GEMV chunk holds an even number of rows (RoPE and gate/up pairs): two
+  // rows of every GEMV op must fit one 16 KB chunk
+  if (h * 4 > kStageBytes || q_rows * 4 > kStageBytes || kc * 4 > kStageBytes)
+    return "two weight rows do not fit one 16 KB chunk";
 
   // ---- weight image layout ----
   Layout& L = g->lay;
@@ -726,7 +728,8 @@ std::string compile_graph(const wpk_model_cfg& m, const Plan& p, CompiledGraph* 
       max_chunks = std::max(max_chunks, (t.a1 + rpc - 1) / rpc);
     }
   // a per-op CTA streams its tile through a ring no larger than a worker's
-  g->plan.per_op_slot = std::min(max_chunks * kStageBytes, p.slot_bytes);
+  // (an even chunk count: GEMV stages take two chunks)
+  g->plan.per_op_slot = std::min((max_chunks + 1) / 2 * 2 * kStageBytes, p.slot_bytes);
   if (T.size() >= (1u << 31)) return "too many tiles";
 
   // ---- edges from dataflow ----

@@ -117,6 +117,9 @@ __device__ __forceinline__ bool cbar_and(bool v) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n) : "memory");
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -181,6 +184,25 @@ __device__ bool wait_phase(const KParams& P, uint64_t* bar, uint32_t parity, vol
       if (*abort) return false;
       if (globaltimer() - t0 > bound) {
         record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, 0, 0);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait until a shared counter written by other warps of this CTA
+// reaches `target`.
+__device__ bool wait_count(const KParams& P, volatile uint32_t* v, uint32_t target, volatile int* abort,
+                           uint32_t tile) {
+  if (*v >= target) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (*v >= target) return true;
+    if ((it & 31) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > 4 * P.timeout_ns) {
+        record_error(P, WPK_ERR_TIMEOUT, tile, kNoCounter, target, *v);
         *abort = 1;
         return false;
       }
@@ -261,10 +283,11 @@ __device__ __forceinline__ void tile_chunks(const KParams& P, const Tile& T, int
     return;
   }
   if (T.w_bytes == 0) return;
-  int r = P.stage_bytes / (T.a3 * 2);
+  int r = P.stage_bytes / P.gemv_cps / (T.a3 * 2);
   r &= ~1;  // even: RoPE and gate/up row pairs never straddle a chunk
   *rpc = r < 2 ? 2 : r;
-  *n_chunks = (T.a1 + *rpc - 1) / *rpc;
+  // ring stages of gemv_cps chunks each
+  *n_chunks = ((T.a1 + *rpc - 1) / *rpc + P.gemv_cps - 1) / P.gemv_cps;
 }
 
 // Source image (hi or lo) of a tensor-core tile's activations: the tile covers
@@ -349,9 +372,10 @@ __device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uin
     }
     return;
   }
+  // GEMV stage k: chunks k gemv_cps .. (consecutive rows), one copy
   const size_t row_bytes = (size_t)T.a3 * 2;
-  const int r0 = k * rpc;
-  const uint32_t bytes = (uint32_t)(min(rpc, T.a1 - r0) * row_bytes);
+  const int r0 = k * P.gemv_cps * rpc;
+  const uint32_t bytes = (uint32_t)(min(P.gemv_cps * rpc, T.a1 - r0) * row_bytes);
   const uint64_t base = (T.op == OP_LMHEAD) ? P.lm_head_off : 0;  // LM tiles are relative to the launch's head
   mbar_arrive_expect_tx(bar, bytes);
   bulk_g2s(dst, P.weights + base + T.w_off + r0 * row_bytes, bytes, bar);
@@ -578,12 +602,18 @@ struct ConsumerState {
   int act_key;      // (op, layer, k0) of the staged activation, or kNoAct
   uint32_t last_ctr;    // counter known satisfied in this launch ...
   uint32_t last_epoch;  // ... for this step
-  uint32_t acc_phase;  // parity of the accumulator barrier
+  uint32_t acc_phase;  // parity of the accumulator barrier (prefill attention)
   uint32_t act_epoch;  // step the staged activation belongs to
+  uint32_t n_mma;      // tensor-core tiles taken (accumulator buffer n_mma % 2)
 };
 
 __shared__ uint32_t s_tmem;  // TMEM base address (tensor-core programs)
-__shared__ int s_mma_ok;
+// Tensor-core tiles: the issuer warp fills accumulator buffer b (s_accf[b]
+// completes when the tile's MMAs have), the consumers empty it after the
+// epilogue (s_acce[b]); s_mma_fin covers every MMA issued before TMEM is freed.
+__shared__ uint64_t s_accf[2], s_acce[2], s_mma_fin;
+// tiles (queue positions) the consumers have finished
+__shared__ volatile uint32_t s_cons_tiles;
 
 __shared__ uint64_t s_t_data;  // trace: when the tile's last chunk had landed
 // GEMV: per stage, 1 + the global index of the last chunk a warp saw land there
@@ -680,6 +710,7 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
   }
   int bgmax = P.act_bytes / (act_stride(K) * 4);
   if (bgmax > kMaxGemvBatch) bgmax = kMaxGemvBatch;
+  const int cps = P.gemv_cps, n_real = (R + rpc - 1) / rpc;  // chunks: gemv_cps per stage
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   bool ok = true;
   for (int b0 = 0; b0 < nb || (nb == 0 && b0 == 0); b0 += bgmax) {
@@ -692,17 +723,18 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
         cs.act_key = key;
       }
     }
-    for (int k = warp; k < n_chunks; k += kWarps) {
-      const uint32_t c = cur.c + k;
+    for (int k = warp; k < n_real; k += kWarps) {
+      const int u = k / cps;  // the tile's stage holding chunk k
+      const uint32_t c = cur.c + u;
       const int st = c % P.n_stages;
       // the stage is waited for on the first token group only
       if (b0 == 0) {
         // A parity wait only tells the current phase from the one before it.
-        // When the stage's previous use (chunk c - n_stages) is this tile's
-        // too, another warp owns it and may not have seen it land yet: wait
-        // for that first, so that the parity wait below cannot be satisfied
-        // by the phase before the previous one.
-        if (k >= P.n_stages && !wait_seen(P, st, c - P.n_stages + 1, abort, T.a0)) {
+        // When the stage's previous use (c - n_stages) is this tile's too,
+        // another warp owns it and may not have seen it land yet: wait for
+        // that first, so that the parity wait below cannot be satisfied by
+        // the phase before the previous one.
+        if (u >= P.n_stages && !wait_seen(P, st, c - P.n_stages + 1, abort, T.a0)) {
           ok = false;
           break;
         }
@@ -713,7 +745,7 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
         __syncwarp();
         if (lane == 0) s_seen[st] = c + 1;
       }
-      const uint8_t* chunk = S.ring + (size_t)st * P.stage_bytes;
+      const uint8_t* chunk = S.ring + (size_t)st * P.stage_bytes + (size_t)(k % cps) * rpc * K * 2;
       const int r0 = k * rpc, rows = min(rpc, R - r0);
       switch (bg) {
         case 0: break;
@@ -724,8 +756,11 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
         default: gemv_chunk<8>(chunk, K, rows, r0, S.act, S.out, bg); break;
       }
       if (last_group) {
+        // the stage takes gemv_cps arrivals: the last chunk of a short stage
+        // arrives for the chunks it lacks
+        const int in_stage = min(cps, n_real - u * cps);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[st]);
+        if (lane == 0) mbar_arrive_n(&S.empty[st], (k % cps == in_stage - 1) ? (uint32_t)(cps - in_stage + 1) : 1u);
       }
     }
     if (!cbar_and(ok)) return false;
@@ -888,7 +923,7 @@ __device__ bool attn_pages(const KParams& P, const AttnSpan& s, const Shared& Sh
     __syncwarp();
     if (lane == 0) {
       const uint32_t r = atomicAdd(&page_rel[st], 1u) + 1u;
-      if (r == (uint32_t)kWarps * (uint32_t)(k / P.n_stages + 1)) mbar_arrive(&Sh.empty[st]);
+      if (r == (uint32_t)kWarps * (uint32_t)(k / P.n_stages + 1)) mbar_arrive_n(&Sh.empty[st], (uint32_t)P.gemv_cps);
     }
   }
   cur.c += n_chunks;
@@ -981,7 +1016,8 @@ __device__ bool body_attn(const KParams& P, const Tile& T, const Shared& Sh, Cur
   // (hg <= 4), each served by wpg = 8 / n_hg warps over the tile's 32-token
   // blocks.  A long tile reads every K/V row once for all heads (one group);
   // a tile of few blocks splits the heads so that all eight warps have work.
-  const int nb_tot = n_chunks * attn_pps(P) * ((page + 31) / 32);
+  const int pages = s.t1 > s.t0 ? (s.t1 - 1) / page - s.t0 / page + 1 : 0;  // the split's pages
+  const int nb_tot = pages * ((page + 31) / 32);
   int n_hg = 8;
   while (n_hg > 1 && (grp % n_hg || n_hg * nb_tot > kWarps)) n_hg >>= 1;
   while (grp / n_hg > 4 || grp % n_hg) n_hg <<= 1;  // at most four heads per group
@@ -1214,6 +1250,10 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       const int pi = within / 2;
       const int dim = is_v ? within : (even ? pi : pi + half);
       float o[CW];
+      float2 rp[CW];  // the columns' RoPE factors, loaded before any store
+#pragma unroll
+      for (int i = 0; i < CW; ++i)
+        rp[i] = is_v ? make_float2(1.f, 0.f) : __ldg(P.rope + (size_t)s_col_pos[n0 + i] * half + pi);
 #pragma unroll
       for (int i = 0; i < CW; ++i) {
         const float y = v[i] * s_rn[n0 + i];
@@ -1221,8 +1261,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
         if (is_v) {
           o[i] = y;
         } else {
-          const int n = n0 + i;
-          const float2 cs = P.rope[(size_t)s_col_pos[n] * half + pi];
+          const float2 cs = rp[i];
           const float y0 = even ? y : partner, y1 = even ? partner : y;
           o[i] = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
         }
@@ -1282,6 +1321,15 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       const int pi = within / 2;
       const bool even = (lane & 1) == 0;
       const int dim = is_v ? within : (even ? pi : pi + half);
+      // every column's RoPE factors first: loaded after the stores below,
+      // which may alias them as far as the compiler knows, they would make
+      // one round trip each
+      float2 rp[CW];
+#pragma unroll
+      for (int i = 0; i < CW; ++i) {
+        const int t = s_col_pos[n0 + i];
+        rp[i] = (is_v || t < 0) ? make_float2(1.f, 0.f) : __ldg(P.rope + (size_t)t * half + pi);
+      }
 #pragma unroll
       for (int i = 0; i < CW; ++i) {
         const float partner = __shfl_xor_sync(0xffffffffu, v[i], 1);
@@ -1292,7 +1340,7 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
           P.kv[s_col_kv[n] + kv_off + dim] = f2bf(v[i]);
           continue;
         }
-        const float2 cs = P.rope[(size_t)t * half + pi];
+        const float2 cs = rp[i];
         const float y0 = even ? v[i] : partner, y1 = even ? partner : v[i];
         const float o = even ? (y0 * cs.x - y1 * cs.y) : (y1 * cs.x + y0 * cs.y);
         if (is_q)
@@ -1396,49 +1444,52 @@ __device__ void rowblock_done(const KParams& P, const Tile& T) {
   if (threadIdx.x < nb) atomicAdd(P.ss + (size_t)nidx * N + threadIdx.x, s_sq[threadIdx.x]);
 }
 
-// Tensor-core tile: D[128 features][128 tokens] = W . (a_hi + a_lo)^T over the
-// tile's K chunks.  Thread 0 issues the MMAs as chunks land and commits each
-// stage back to the producer; all compute warps then read TMEM.
+// Issues the MMAs of one tensor-core tile (D[128 features][128 tokens] =
+// W . (a_hi + a_lo)^T over its K chunks) into the accumulator buffer at TMEM
+// column `tmem`, committing each stage back to the producer as its MMAs
+// complete.  The hi and lo activation rows sit back to back in the stage, so
+// one MMA with N' = 2N covers both: columns [0, N) get W . hi, [N, 2N) W . lo.
+// Successive K-steps rotate over the buffer's NA accumulators (2N columns
+// each), so that small-N MMAs do not wait on one another.  Run by the issuer
+// warp's lane 0; `c` is the tile's first chunk.
+__device__ bool issue_tile_mmas(const KParams& P, const Tile& T, const Shared& S, uint32_t c, int n_chunks,
+                                uint32_t tmem, volatile int* abort, uint32_t tile) {
+  const int N = P.mma_n, NA = P.mma_acc;
+  const uint32_t idesc = idesc_f16(128, 2 * N, true);
+  uint32_t mi = 0;  // MMAs issued for this tile
+  for (int k = 0; k < n_chunks; ++k, ++c) {  // one unit of K chunks per stage
+    const int st = c % P.n_stages;
+    if (!wait_phase(P, &S.full[st], (c / P.n_stages) & 1u, abort, tile)) return false;
+    tc_fence_after();
+    const uint32_t base = smem_u32(S.ring + (size_t)st * P.stage_bytes);
+    const uint32_t act = base + (uint32_t)P.mma_cps * kMmaChunkBytes;
+    const int nc = mma_unit(P, T, k).nc;
+    for (int j = 0; j < nc; ++j) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk, ++mi) {
+        const int a = (int)(mi % (uint32_t)NA);
+        umma_f16(tmem + (uint32_t)(a * 2 * N), sdesc_k_sw128(base + j * kMmaChunkBytes + kk * 32),
+                 sdesc_k_sw128(act + j * 2 * P.act_chunk + kk * 32), idesc, mi >= (uint32_t)NA ? 1u : 0u);
+      }
+    }
+    umma_commit(&S.empty[st]);
+  }
+  return true;
+}
+
+// Tensor-core tile, consumer side: the issuer warp has issued (or is issuing)
+// the tile's MMAs into accumulator buffer n_mma % 2; the compute warps build
+// the epilogue's tables meanwhile, wait for the accumulators, read TMEM and
+// hand the buffer back.
 __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
                          ConsumerState& cs, volatile int* abort, uint32_t tile) {
-  const uint32_t tmem = s_tmem;
   const int N = P.mma_n, NA = P.mma_acc;
-  if (threadIdx.x == 0) {
-    // The hi and lo activation rows sit back to back in the stage, so one MMA
-    // with N' = 2N covers both: columns [0, N) get W . hi, [N, 2N) W . lo.
-    // Successive K-steps rotate over NA accumulators (2N columns each), so the
-    // MMAs of a chunk do not wait on one another.
-    bool ok = true;
-    uint32_t cc = cur.c;
-    const uint32_t idesc = idesc_f16(128, 2 * N, true);
-    uint32_t mi = 0;  // MMAs issued for this tile
-    for (int k = 0; k < n_chunks; ++k, ++cc) {  // one unit of K chunks per stage
-      const int st = cc % P.n_stages;
-      if (!wait_phase(P, &S.full[st], (cc / P.n_stages) & 1u, abort, tile)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t base = smem_u32(S.ring + (size_t)st * P.stage_bytes);
-      const uint32_t act = base + (uint32_t)P.mma_cps * kMmaChunkBytes;
-      const int nc = mma_unit(P, T, k).nc;
-      for (int j = 0; j < nc; ++j) {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk, ++mi) {
-          const int a = (int)(mi % (uint32_t)NA);
-          umma_f16(tmem + (uint32_t)(a * 2 * N), sdesc_k_sw128(base + j * kMmaChunkBytes + kk * 32),
-                   sdesc_k_sw128(act + j * 2 * P.act_chunk + kk * 32), idesc, mi >= (uint32_t)NA ? 1u : 0u);
-        }
-      }
-      umma_commit(&S.empty[st]);
-    }
-    umma_commit(S.acc);
-    s_mma_ok = ok;
-  }
-  // QKV tiles: the per-column position / KV-row table (threads 32.. while
-  // thread 0 issues the MMAs)
+  const int buf = (int)(cs.n_mma & 1u);
+  const uint32_t use = cs.n_mma >> 1;
+  const uint32_t tmem = s_tmem + (uint32_t)(buf * P.mma_buf_cols);
+  // QKV tiles: the per-column position / KV-row table
   if (T.op == OP_BQKV || T.op == OP_MQKV) {
-    const int n = (int)threadIdx.x - 32;
+    const int n = (int)threadIdx.x;
     if (n >= 0 && n < N) {
       if (T.op == OP_BQKV) {
         s_col_pos[n] = (n < active_batch(P) && slot_on(P, n)) ? P.seqlen[n] : 0;
@@ -1464,10 +1515,11 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
     if (threadIdx.x < N) s_best[threadIdx.x] = 0ull;
   }
   cbar();
-  bool ok = s_mma_ok;
-  if (!wait_phase(P, S.acc, cs.acc_phase, abort, tile)) ok = false;
+  bool ok = true;
+  // (slack: the wait covers the tile's whole mainloop)
+  if (!wait_phase(P, &s_accf[buf], use & 1u, abort, tile, 4)) ok = false;
   if (P.trace && threadIdx.x == 0) s_t_data = globaltimer();  // the accumulators are complete
-  cs.acc_phase ^= 1u;
+  ++cs.n_mma;
   cur.c += n_chunks;
   if (!cbar_and(ok)) return false;
   tc_fence_after();
@@ -1497,6 +1549,7 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
   }
   tc_fence_before();
   cbar();
+  if (threadIdx.x == 0) mbar_arrive(&s_acce[buf]);  // the buffer's TMEM has been read
   if (T.op == OP_BO || T.op == OP_BDOWN) {
     rowblock_done(P, T);
   } else if (T.op == OP_BLM) {
@@ -1509,22 +1562,26 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
 // Causal GQA attention for the queries [t0, t1) of sequence b and the query
 // heads of kv head g, on the tensor cores.  The tile's 128 rows (query qi and
 // head hh at row qi * group + hh) are the MMA's M and TMEM lanes 0-127; warps
-// 0-3 own one row per thread.  Per staged KV page of 64 keys:
+// w and w + 4 share TMEM lanes 32 (w % 4) ..: each thread owns one row and one
+// half of its keys and of its output dims.  Per staged KV page of 64 keys:
 //   1. all warps build, in the stage, the page's K rows and its V transposed
 //      ([dim][key]) as K-major operands with the 128-byte swizzle;
-//   2. S = (Q_hi + Q_lo) K^T on the tensor cores, Q (scaled by 1/sqrt(d))
-//      split into bf16 hi and lo halves held in TMEM;
-//   3. each row's online softmax over S (causal mask key <= query), the
-//      probabilities split into bf16 hi and lo written to TMEM;
+//   2. S = (Q_hi + Q_lo) K^T on the tensor cores, Q (scaled by log2(e) /
+//      sqrt(d), so that the softmax runs in base 2) split into bf16 hi and lo
+//      halves held in TMEM;
+//   3. each row's online softmax over S (causal mask key <= query), the two
+//      halves exchanging their maxima and sums through shared memory; the
+//      probabilities split into bf16 hi and lo, written to TMEM;
 //   4. O_page = (P_hi + P_lo) V^T on the tensor cores, added into the row's
 //      fp32 output registers.
 // The hi/lo splits keep q and p to about 16 significant bits; K and V are
-// the cache's bf16 values; every product accumulates in fp32.  A key split
-// (pattn_ks) writes its (m, l, o) partial and the last split to finish
-// combines them, as the decode attention does.
+// the cache's bf16 values; every product accumulates in fp32.  A query block
+// split along the keys (pattn_ks) writes each split's (m, l, o) partial and
+// the last split to finish combines them, as the decode attention does.
 namespace pattn {
 constexpr uint32_t kS = 0, kO = 64, kQh = 128, kQl = 160, kPh = 192, kPl = 224;  // TMEM columns
 constexpr int kKRows = 16384, kVt = 24576;  // stage offsets of the swizzled K rows and V transposed
+constexpr float kQScale = 0.125f * 1.44269504088896341f;  // log2(e) / sqrt(64)
 }
 
 __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks,
@@ -1534,26 +1591,32 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
   pattn_span(P, T, &t0, &t1);
   pattn_keys(P, T, t1, &k_first, &k_end);
   k_first = k_first / P.page_tokens * P.page_tokens;  // splits start on a page
-  const int warp = threadIdx.x >> 5;
-  const bool row_thread = warp < 4;  // warps 0-3: one tile row (TMEM lane) each
-  const int r = threadIdx.x;         // the row, for row threads
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hw = warp >> 2;                // key half (S columns) and dim half (O columns)
+  const int r = 32 * (warp & 3) + lane;    // the row: TMEM lane
   const int qi = r / grp, hh = r % grp;
   const int t = t0 + qi;
-  const bool valid = row_thread && t < t1;
+  const bool valid = t < t1;
   const int m = b * P.T + (valid ? t : t0);
   const int head = g * grp + hh;
   const uint32_t tmem = s_tmem;
   const uint32_t lane_addr = ((uint32_t)(32 * (warp & 3)) << 16);
-  // Q row -> TMEM (hi, lo), scaled by 1/sqrt(64) = 1/8 (exact in bf16)
-  if (row_thread) {
-    const float4* qs = reinterpret_cast<const float4*>(P.pq + (size_t)m * P.q_rows + head * hd);
+  // the two halves' row maxima and sums: red[max or sum][key half][row], in
+  // the activation buffer (the program's GEMV tiles restage it)
+  float(*red)[2][128] = reinterpret_cast<float(*)[2][128]>(S.act);
+  // Q row -> TMEM (hi, lo): dims [32 hw, 32 hw + 32), all loads first
+  {
+    const float4* qs = reinterpret_cast<const float4*>(P.pq + (size_t)m * P.q_rows + head * hd + 32 * hw);
+    float4 q4[8];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {  // 16 dims = 8 columns per store
+    for (int e = 0; e < 8; ++e) q4[e] = __ldcg(qs + e);
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {  // 16 dims = 8 columns per store
       uint32_t hi[8], lo[8];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float4 q4 = __ldcg(qs + 4 * c + e);
-        const float qv[4] = {q4.x * 0.125f, q4.y * 0.125f, q4.z * 0.125f, q4.w * 0.125f};
+        const float4 x = q4[4 * c + e];
+        const float qv[4] = {x.x * pattn::kQScale, x.y * pattn::kQScale, x.z * pattn::kQScale, x.w * pattn::kQScale};
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const __nv_bfloat162 hv = __floats2bfloat162_rn(qv[2 * h2], qv[2 * h2 + 1]);
@@ -1561,15 +1624,15 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
           lo[2 * e + h2] = pack_bf16x2(qv[2 * h2] - __bfloat162float(hv.x), qv[2 * h2 + 1] - __bfloat162float(hv.y));
         }
       }
-      tmem_st8(tmem + lane_addr + pattn::kQh + 8 * c, hi);
-      tmem_st8(tmem + lane_addr + pattn::kQl + 8 * c, lo);
+      tmem_st8(tmem + lane_addr + pattn::kQh + 16 * hw + 8 * c, hi);
+      tmem_st8(tmem + lane_addr + pattn::kQl + 16 * hw + 8 * c, lo);
     }
     tmem_st_wait();
   }
-  float o[64];
+  float o[32];  // output dims [32 hw, 32 hw + 32) of the row
 #pragma unroll
-  for (int d = 0; d < 64; ++d) o[d] = 0.f;
-  float mrun = -INFINITY, lrun = 0.f;
+  for (int d = 0; d < 32; ++d) o[d] = 0.f;
+  float mrun = -INFINITY, lrun = 0.f;  // base-2 running max and sum (identical in both halves)
   const uint32_t idesc = idesc_f16(128, 64, true);
   bool ok = true;
   for (int k = 0; k < n_chunks; ++k) {
@@ -1618,53 +1681,45 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     cs.acc_phase ^= 1u;
     if (!cbar_and(ok)) return false;
     tc_fence_after();
-    // 3. online softmax of the row over the page's keys; P (hi, lo) -> TMEM
-    float corr = 1.f;
-    if (row_thread) {
-      float mx = -INFINITY;
+    // 3. online softmax of the row over the page's keys [32 hw, 32 hw + 32)
+    float sv[32];
+    tmem_ld16x2(tmem + lane_addr + pattn::kS + 32 * hw, sv);
+    float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float sv[16];
-        tmem_ld16(tmem + lane_addr + pattn::kS + 16 * c, sv);
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int key = kp + 16 * c + jj;
-          if (valid && 16 * c + jj < rows && key <= t) mx = fmaxf(mx, sv[jj]);
-        }
-      }
-      const float mnew = fmaxf(mrun, mx);
-      if (mnew != -INFINITY) {
-        corr = mrun == -INFINITY ? 0.f : expf(mrun - mnew);
-        mrun = mnew;
-      }
-      float psum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float sv[16];
-        tmem_ld16(tmem + lane_addr + pattn::kS + 16 * c, sv);
-        uint32_t hi[8], lo[8];
-#pragma unroll
-        for (int jj = 0; jj < 16; jj += 2) {
-          float pv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int key = kp + 16 * c + jj + e;
-            pv[e] = (valid && 16 * c + jj + e < rows && key <= t) ? expf(sv[jj + e] - mrun) : 0.f;
-            psum += pv[e];
-          }
-          const __nv_bfloat162 hv = __floats2bfloat162_rn(pv[0], pv[1]);
-          hi[jj / 2] = *reinterpret_cast<const uint32_t*>(&hv);
-          lo[jj / 2] = pack_bf16x2(pv[0] - __bfloat162float(hv.x), pv[1] - __bfloat162float(hv.y));
-        }
-        tmem_st8(tmem + lane_addr + pattn::kPh + 8 * c, hi);
-        tmem_st8(tmem + lane_addr + pattn::kPl + 8 * c, lo);
-      }
-      tmem_st_wait();
-      lrun = lrun * corr + psum;
+    for (int jj = 0; jj < 32; ++jj) {
+      const int j = 32 * hw + jj;
+      const bool live = valid && j < rows && kp + j <= t;
+      sv[jj] = live ? sv[jj] : -INFINITY;
+      mx = fmaxf(mx, sv[jj]);
     }
+    red[0][hw][r] = mx;
+    cbar();
+    const float mnew = fmaxf(mrun, fmaxf(mx, red[0][hw ^ 1][r]));
+    // (a row with no live key yet keeps m = -inf, its p = 0 and corr = 1)
+    const float corr = mnew == -INFINITY ? 1.f : (mrun == -INFINITY ? 0.f : exp2f(mrun - mnew));
+    float psum = 0.f;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int jj = 0; jj < 16; jj += 2) {
+        const float p0 = sv[16 * c + jj] == -INFINITY ? 0.f : exp2f(sv[16 * c + jj] - mnew);
+        const float p1 = sv[16 * c + jj + 1] == -INFINITY ? 0.f : exp2f(sv[16 * c + jj + 1] - mnew);
+        psum += p0 + p1;
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+        hi[jj / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+        lo[jj / 2] = pack_bf16x2(p0 - __bfloat162float(hv.x), p1 - __bfloat162float(hv.y));
+      }
+      tmem_st8(tmem + lane_addr + pattn::kPh + 16 * hw + 8 * c, hi);
+      tmem_st8(tmem + lane_addr + pattn::kPl + 16 * hw + 8 * c, lo);
+    }
+    red[1][hw][r] = psum;
+    tmem_st_wait();
     tc_fence_before();
     cbar();
     tc_fence_after();
+    lrun = lrun * corr + (psum + red[1][hw ^ 1][r]);
+    mrun = mnew;
     // 4. O_page = P V^T
     if (threadIdx.x == 0) {
       const uint32_t vb = smem_u32(stage + pattn::kVt);
@@ -1679,14 +1734,11 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     cs.acc_phase ^= 1u;
     if (!cbar_and(ok)) return false;
     tc_fence_after();
-    if (row_thread) {
+    {
+      float ov[32];
+      tmem_ld16x2(tmem + lane_addr + pattn::kO + 32 * hw, ov);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float ov[16];
-        tmem_ld16(tmem + lane_addr + pattn::kO + 16 * c, ov);
-#pragma unroll
-        for (int d = 0; d < 16; ++d) o[16 * c + d] = fmaf(o[16 * c + d], corr, ov[d]);
-      }
+      for (int d = 0; d < 32; ++d) o[d] = fmaf(o[d], corr, ov[d]);
     }
     // the stage and the TMEM operands are free again: hand the stage back
     tc_fence_before();
@@ -1694,17 +1746,18 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     if (threadIdx.x == 0) mbar_arrive(&S.empty[st]);
     ++cur.c;
   }
-  if (P.pattn_ks) {
+  const int n_ks = P.pattn_ks ? (t1 + P.pattn_ks - 1) / P.pattn_ks : 1;
+  if (n_ks > 1) {
     // a key split: store this split's (m, l, o) of every row; the last split
     // of the (sequence, kv head, query block) to arrive combines them
-    const int n_ks = (t1 + P.pattn_ks - 1) / P.pattn_ks;
     const int n_qb = (P.T + kTokBlock / grp - 1) / (kTokBlock / grp);
     const int idx = (b * P.n_kv + g) * n_qb + T.a2;
     float* base = P.ppart + (size_t)idx * kMaxKeySplits * 128 * (2 + kHeadDim);
-    if (row_thread) {
-      float* mine = base + ((size_t)T.a3 * 128 + r) * (2 + kHeadDim);
+    float* mine = base + ((size_t)T.a3 * 128 + r) * (2 + kHeadDim);
 #pragma unroll
-      for (int d = 0; d < 64; d += 2) *reinterpret_cast<float2*>(mine + 2 + d) = make_float2(o[d], o[d + 1]);
+    for (int d = 0; d < 32; d += 2)  // records are 66 floats: 8-byte aligned
+      *reinterpret_cast<float2*>(mine + 2 + 32 * hw + d) = make_float2(o[d], o[d + 1]);
+    if (hw == 0) {
       mine[0] = mrun;  // -inf with l = 0 when no key of the split is at or before the query
       mine[1] = lrun;
     }
@@ -1719,22 +1772,20 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     }
     cbar();
     if (!s_last_split) return true;
-    if (row_thread) {
-      float M = -INFINITY;
-      for (int j = 0; j < n_ks; ++j) M = fmaxf(M, __ldcg(base + ((size_t)j * 128 + r) * (2 + kHeadDim)));
-      lrun = 0.f;
+    float M = -INFINITY;
+    for (int j = 0; j < n_ks; ++j) M = fmaxf(M, __ldcg(base + ((size_t)j * 128 + r) * (2 + kHeadDim)));
+    lrun = 0.f;
 #pragma unroll
-      for (int d = 0; d < 64; ++d) o[d] = 0.f;
-      for (int j = 0; j < n_ks; ++j) {
-        const float* w = base + ((size_t)j * 128 + r) * (2 + kHeadDim);
-        const float f = M == -INFINITY ? 0.f : expf(__ldcg(w) - M);
-        lrun = fmaf(__ldcg(w + 1), f, lrun);
+    for (int d = 0; d < 32; ++d) o[d] = 0.f;
+    for (int j = 0; j < n_ks; ++j) {
+      const float* w = base + ((size_t)j * 128 + r) * (2 + kHeadDim);
+      const float f = M == -INFINITY ? 0.f : exp2f(__ldcg(w) - M);
+      lrun = fmaf(__ldcg(w + 1), f, lrun);
 #pragma unroll
-        for (int d = 0; d < 64; d += 2) {  // records are 66 floats: 8-byte aligned
-          const float2 x = __ldcg(reinterpret_cast<const float2*>(w + 2 + d));
-          o[d] = fmaf(x.x, f, o[d]);
-          o[d + 1] = fmaf(x.y, f, o[d + 1]);
-        }
+      for (int d = 0; d < 32; d += 2) {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(w + 2 + 32 * hw + d));
+        o[d] = fmaf(x.x, f, o[d]);
+        o[d + 1] = fmaf(x.y, f, o[d + 1]);
       }
     }
   }
@@ -1743,7 +1794,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
     const int tb = m / kTokBlock, n = m % kTokBlock, nkc = P.q_rows / 64;
     const size_t blk = ((size_t)tb * nkc + head) * P.img_stride;  // 64-column chunk == one head
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 4; ++u) {
       uint32_t ph[4], pl[4];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
@@ -1752,7 +1803,7 @@ __device__ bool body_pattn(const KParams& P, const Tile& T, const Shared& S, Cur
         ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hv);
         pl[e / 2] = pack_bf16x2(a0 - __bfloat162float(hv.x), a1 - __bfloat162float(hv.y));
       }
-      const uint32_t off = sw128_offset(n, 8 * u);
+      const uint32_t off = sw128_offset(n, 32 * hw + 8 * u);
       *reinterpret_cast<uint4*>(P.att_img[0] + blk + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
       *reinterpret_cast<uint4*>(P.att_img[1] + blk + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
     }
@@ -1942,13 +1993,20 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < P.n_stages; ++i) {
       mbar_init(&S.full[i], 1);
-      mbar_init(&S.empty[i], 1);
+      mbar_init(&S.empty[i], (uint32_t)P.gemv_cps);
     }
     for (int i = 0; i < kMaxQueue; ++i) {
       mbar_init(&S.tq_full[i], 1);
-      mbar_init(&S.tq_empty[i], 1);
+      // released by the consumers, and in tensor-core programs by the issuer
+      mbar_init(&S.tq_empty[i], kProg == kProgGemv ? 1 : 2);
     }
     mbar_init(S.acc, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_accf[i], 1);
+      mbar_init(&s_acce[i], 1);
+    }
+    mbar_init(&s_mma_fin, 1);
+    s_cons_tiles = 0;
     for (int i = 0; i < kSigQueue; ++i) {
       mbar_init(&S.sig_full[i], 1);
       mbar_init(&S.sig_empty[i], 1);
@@ -2082,10 +2140,65 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         if (stop) break;
       }
     }
+  } else if (warp == kWarps + 1) {
+    // ------------------------------------------------- tensor-core issuer
+    // Walks the tile queue in the consumers' order and issues each
+    // tensor-core tile's MMAs into one of two TMEM accumulator buffers, so
+    // the consumers' epilogue of one tile overlaps the next tile's mainloop.
+    if constexpr (kProg != kProgGemv) {
+      if ((threadIdx.x & 31) == 0) {
+        const int Q = P.per_op ? 1 : P.lookahead;
+        uint32_t c = 0;       // the consumers' chunk cursor, mirrored
+        uint32_t n_mma = 0;   // tensor-core tiles issued
+        uint32_t other = 0;   // 1 + queue position of the last other tile that takes chunks
+        bool issued = false;
+        for (uint32_t i = 0;; ++i) {
+          const int slot = i % Q;
+          if (!wait_phase(P, &S.tq_full[slot], (i / Q) & 1u, &s_abort, 0xFFFFFFFFu, 2)) break;
+          const TQEntry& e = S.tq[slot];
+          const bool valid = e.valid != 0;
+          const Tile T = e.tile;
+          const uint32_t t = e.ticket;
+          const int nch = e.n_chunks;
+          mbar_arrive(&S.tq_empty[slot]);  // the issuer's share of the slot's release
+          if (!valid) break;
+          if (!is_mma_op(T.op)) {
+            c += nch;
+            // (prefill attention also issues its own MMAs into TMEM)
+            if (nch > 0 || T.op == OP_PATTN) other = i + 1;
+            continue;
+          }
+          // The consumers take the chunks of other tiles.  A parity wait
+          // only tells a phase from the one before it, so every earlier
+          // chunk must have landed before this tile's stages are waited for.
+          if (other && !wait_count(P, &s_cons_tiles, other, &s_abort, t)) break;
+          const int b = (int)(n_mma & 1u);
+          const uint32_t use = n_mma >> 1;
+          // the buffer's previous tile has been read out
+          if (use >= 1 && !wait_phase(P, &s_acce[b], (use - 1) & 1u, &s_abort, t, 4)) break;
+          tc_fence_after();
+          issued = true;
+          if (!issue_tile_mmas(P, T, S, c, nch, s_tmem + (uint32_t)(b * P.mma_buf_cols), &s_abort, t)) break;
+          umma_commit(&s_accf[b]);
+          c += nch;
+          ++n_mma;
+        }
+        if (issued) {
+          // every MMA issued has completed before TMEM is released (bounded)
+          umma_commit(&s_mma_fin);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&s_mma_fin, 0u))
+            if (globaltimer() - t0 > P.timeout_ns) {
+              record_error(P, WPK_ERR_TIMEOUT, 0xFFFFFFFDu, kNoCounter, n_mma, 0);
+              break;
+            }
+        }
+      }
+    }
   } else {
     // ----------------------------------------------------------- consumers
     Cursor cur{0};
-    ConsumerState cs{kNoAct, kNoCounter, 0u, 0u, 0u};
+    ConsumerState cs{kNoAct, kNoCounter, 0u, 0u, 0u, 0u};
     uint32_t n_sig = 0;  // requests pushed to the signaller (thread 0)
     const int Q = P.per_op ? 1 : P.lookahead;
     __shared__ int s_fail;
@@ -2188,7 +2301,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
         }
         // attention tiles use the activation buffer as scratch; the gather
         // rewrites the LM head's input
-        if (T.op == OP_ATTN || T.op == OP_GATHER) cs.act_key = kNoAct;
+        if (T.op == OP_ATTN || T.op == OP_PATTN || T.op == OP_GATHER) cs.act_key = kNoAct;
       }
       ok = cbar_and(ok);
       if (!ok) {
@@ -2223,6 +2336,7 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
             ++n_sig;
           }
         }
+        s_cons_tiles = i + 1;
         mbar_arrive(&S.tq_empty[slot]);
       }
     }

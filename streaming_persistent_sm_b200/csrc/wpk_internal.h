@@ -11,11 +11,25 @@ namespace wpk {
 constexpr uint32_t kNoCounter = 0xFFFFFFFFu;
 constexpr int kThreads = 256;          // consumer (compute) threads per worker CTA
 constexpr int kWarps = kThreads / 32;
-constexpr int kCtaThreads = kThreads + 32;  // + one producer warp
+constexpr int kCtaThreads = kThreads + 64;  // + the producer warp + the tensor-core issuer warp
 constexpr int kStageBytes = 16384;     // one chunk stage of the staging ring
 constexpr int kMaxStages = 13;         // ring stages per worker
+// GEMV chunks (kStageBytes each) per ring stage of a staging slot of `slot`
+// bytes: two per stage, one copy each, when the slot holds two (a worker
+// issues and completes about one stage per half microsecond whatever its
+// size, so 16 KB stages cap a worker near 30 GB/s), and the chunks the slot
+// holds at once in whole stages.
+inline int gemv_chunks_per_stage(int slot) { return slot >= 2 * kStageBytes ? 2 : 1; }
+inline int gemv_ring_chunks(int slot) {
+  const int c = gemv_chunks_per_stage(slot);
+  return slot / (c * kStageBytes) * c;
+}
 constexpr int kMaxQueue = 8;           // tiles a worker may hold (lookahead)
 constexpr int kMaxGemvBatch = 8;       // token rows per GEMV pass
+// largest batch the automatic choice decodes on CUDA cores (B200, 1B shape:
+// the GEMV step at 4 sequences matches the tensor-core step, at 8 it takes
+// twice as long)
+constexpr int kAutoGemvBatch = 4;
 constexpr int kMaxTileRows = 128;      // rows per GEMV tile (partial-output buffer)
 constexpr int kMaxGroup = 8;           // q heads per kv head handled by one attention tile
 constexpr int kHeadDim = 64;           // the head dimension the attention tiles are written for
@@ -38,7 +52,7 @@ enum Op : uint16_t {
   OP_MO = 11,      // X += Wo . attn on tensor cores
   OP_MGU = 12,     // gate/up on tensor cores, SwiGLU -> hi/lo image of h
   OP_MDOWN = 13,   // X += Wd . h on tensor cores
-  OP_PATTN = 14,   // causal GQA attention of one query block (CUDA cores)
+  OP_PATTN = 14,   // causal GQA attention of one query block (tensor cores)
   OP_GATHER = 15,  // xa[b] = X[last prompt position of b]
   // batched decode program (the step's tokens are the MMA N dimension)
   OP_BQKV = 16,    // [q;k;v] partial over a K range on tensor cores, RoPE, summed into acc
@@ -187,6 +201,11 @@ struct KParams {
   ResCtl* ctl;               // resident: control block (device view of mapped memory)
   ResDev* rdev;              // resident: its device-memory copy
   int stage_bytes;           // bytes per staging-ring stage
+  // GEMV chunks per stage: a GEMV tile's rows are cut into chunks of
+  // stage_bytes / gemv_cps bytes (one warp each), gemv_cps consecutive
+  // chunks staged with one copy; the stage's empty barrier takes gemv_cps
+  // arrivals in the GEMV decode program (1 elsewhere)
+  int gemv_cps;
   int uses_tmem;             // the program has tensor-core tiles
   // prefill program (token rows m = b * T + t, M = B * T, blocks of 128)
   int M, T, n_tb;
@@ -211,9 +230,11 @@ struct KParams {
   // prefill: the hi and lo images are separate, one chunk apart), and the K
   // chunks a tensor-core tile stages per ring stage (1 or 2)
   int img_stride, mma_cps;
-  // accumulators a tile rotates its K-steps over (2 mma_n TMEM columns each)
-  // and the TMEM columns a worker allocates (a power of two >= 2 mma_n mma_acc)
-  int mma_acc, tmem_cols;
+  // accumulators a tile rotates its K-steps over (2 mma_n TMEM columns each),
+  // the columns of one tile's accumulator buffer (2 mma_n mma_acc; a worker
+  // holds two, so that one tile's epilogue overlaps the next tile's MMAs) and
+  // the TMEM columns a worker allocates (a power of two >= 2 mma_buf_cols)
+  int mma_acc, mma_buf_cols, tmem_cols;
   // batched decode program (dec_mma = 1).  Token n of the step is MMA column n;
   // columns >= the active batch hold zeros.  Images are [K/64][act_chunk].
   int dec_mma;

@@ -252,7 +252,7 @@ def test_batched_decode_k_split_edges(lib):
 
 
 def test_decode_mode_selection(lib):
-    for B, want in ((8, "lm_head"), (9, "b_lm_head"), (48, "b_lm_head")):
+    for B, want in ((4, "lm_head"), (5, "b_lm_head"), (48, "b_lm_head")):
         h = _graph(max_batch=B, max_context=64)
         try:
             _, names = _ops(h)
@@ -340,7 +340,8 @@ def test_two_stage_chunked_frame_host_side(lib):
     """frame_chunks = C builds C backbone + head pairs of ceil(B / C) sequences
     over one weight image; KV and scratch are the pairs' sums."""
     s = synth.TINY_TWO_STAGE
-    one = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16))
+    # (the pairs of three decode on CUDA cores; so does the reference plan)
+    one = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16, decode=W.WPK_DECODE_GEMV))
     per3 = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(3, 64, n_workers=12))
     h = W.wpk_build_graph(W.model_cfg(s), W.plan_cfg(5, 64, n_workers=16, frame_chunks=2, head_workers=4))
     try:
@@ -399,3 +400,20 @@ def test_team_schedule_is_one_region_launched_per_step(lib):
         with pytest.raises(W.WpkError) as ei:
             _graph(schedule=W.WPK_SCHED_TEAMS, **kw)
         assert ei.value.code == W.WPK_ERR_UNSUPPORTED
+
+
+def test_two_pass_gemv_tiles_fit_the_ring_in_whole_stages(lib):
+    # Above 8 sequences a GEMV tile is read in several passes, so all its
+    # chunks must be staged at once.  GEMV stages hold two 16 KB chunks: a
+    # slot of nine chunks holds four stages, eight chunks.
+    h = _graph(synth.LLAMA_1B, max_batch=16, max_context=640, decode=W.WPK_DECODE_GEMV, slot_bytes=9 * 16384)
+    try:
+        st = W.wpk_graph_stats_get(h)
+        ops = W.wpk_get_tile_ops(h, st["n_tiles"])
+        nbytes = W.wpk_get_tile_bytes(h, st["n_tiles"])
+        gemv = np.isin(ops, [W.OP_NAMES.index(n) for n in ("qkv", "o", "gate_up", "down", "lm_head")])
+        assert gemv.sum() > 0
+        # every 1B GEMV row is 4 KB, so a chunk is exactly 16 KB
+        assert nbytes[gemv].max() == 8 * 16384
+    finally:
+        W.wpk_destroy(h)
