@@ -24,6 +24,7 @@ size_t worker_smem_bytes(int n_stages, int stage_bytes, int act_bytes);
 const void* persistent_kernel_ptr(bool mma);  // decode on tensor cores (mma) or CUDA cores
 const void* per_op_kernel_ptr(bool mma);
 const void* prefill_kernel_ptr();
+int cta_threads(const void* fn);
 const void* prefill_op_kernel_ptr();
 }  // namespace wpk
 
@@ -359,8 +360,8 @@ void scratch_layout(wpk_handle* h) {
 // A worker grid: cooperative, so that all its CTAs are co-resident, unless
 // the handle runs beside another persistent grid (plain_launch).
 cudaError_t launch_grid(const wpk_handle* h, const void* fn, void** args, size_t smem, cudaStream_t s) {
-  if (h->plain_launch) return cudaLaunchKernel(fn, dim3(h->n_workers), dim3(kCtaThreads), args, smem, s);
-  return cudaLaunchCooperativeKernel(fn, dim3(h->n_workers), dim3(kCtaThreads), args, smem, s);
+  if (h->plain_launch) return cudaLaunchKernel(fn, dim3(h->n_workers), dim3(cta_threads(fn)), args, smem, s);
+  return cudaLaunchCooperativeKernel(fn, dim3(h->n_workers), dim3(cta_threads(fn)), args, smem, s);
 }
 
 int launch_megakernel(wpk_handle* h, const KParams& base, cudaStream_t s) {
@@ -397,7 +398,7 @@ int capture_per_op(wpk_handle* h, int32_t* out_tok, float* logits, GraphEntry* o
       P.n_stages = g.plan.per_op_slot / P.stage_bytes;
     }
     void* args[] = {&P};
-    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(og.end - og.begin), dim3(kCtaThreads), args,
+    cudaError_t e = cudaLaunchKernel(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(og.end - og.begin), dim3(cta_threads(per_op_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA))), args,
                                      h->smem_per_op, h->capture_stream);
     if (e != cudaSuccess) {
       cudaGraph_t junk = nullptr;
@@ -445,7 +446,7 @@ int res_launch(wpk_handle* h) {
   P.t_end = (uint32_t)g.tiles.size();
   P.region = 0;
   void* args[] = {&P};
-  CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(h->n_workers), dim3(kCtaThreads), args,
+  CUDA_TRY(h, cudaLaunchCooperativeKernel(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), dim3(h->n_workers), dim3(cta_threads(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA))), args,
                                           h->smem, h->res_stream));
   h->res_live = true;
   h->res_epoch = 0;
@@ -645,7 +646,7 @@ int launch_prefill(wpk_handle* h, PrefillProgram* prog, const int32_t* tokens, i
       P.t_end = og.end;
       P.per_op = 1;
       void* args[] = {&P};
-      cudaError_t err = cudaLaunchKernel(prefill_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreads), args,
+      cudaError_t err = cudaLaunchKernel(prefill_op_kernel_ptr(), dim3(og.end - og.begin), dim3(kCtaThreadsTc), args,
                                          h->smem_prefill, h->capture_stream);
       if (err != cudaSuccess) {
         cudaGraph_t junk = nullptr;
@@ -718,12 +719,12 @@ static int setup_device(wpk_handle* h) {
     CUDA_TRY(h, raise_smem_limit(prefill_kernel_ptr(), h->smem_prefill));
     CUDA_TRY(h, raise_smem_limit(prefill_op_kernel_ptr(), h->smem_prefill));
     int per_sm_p = 0;
-    CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreads,
+    CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreadsTc,
                                                               h->smem_prefill));
     if (per_sm_p < 1) return fail(h, WPK_ERR_UNSUPPORTED, "the prefill worker does not fit an SM");
   }
   int per_sm = 0;
-  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), kCtaThreads, smem_max));
+  CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), cta_threads(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA)), smem_max));
   h->per_sm = per_sm;
   {
     // tcgen05.alloc waits until the SM has free TMEM columns: workers that
@@ -738,7 +739,7 @@ static int setup_device(wpk_handle* h) {
       pp.mma_n = kTokBlock;
       set_mma_geometry(&pp);
       int per_sm_p = 0;
-      CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreads,
+      CUDA_TRY(h, cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_p, prefill_kernel_ptr(), kCtaThreadsTc,
                                                                 h->smem_prefill));
       h->per_sm_prefill = per_sm_p;
       if (per_sm_p * pp.tmem_cols > 512)

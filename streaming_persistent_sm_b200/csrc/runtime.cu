@@ -1232,8 +1232,36 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
 // Tensor-core tile epilogue for CW token columns n0..n0+CW-1 of feature row fl
 // (CW = 8 for the batched decode, whose few columns are split finer so that all
 // eight warps share the work; 16 for the prefill).
+// Gate/up epilogue output: the even lanes of a warp hold h of its 16
+// features (lane / 2) for tokens n0 .. n0 + CW.  The values go through the
+// warp's shared scratch ([hi, lo][CW tokens][16 features] bf16) so that the
+// image takes 16-byte stores of 8 consecutive features of one token.
 template <int CW>
-__device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, const float* v) {
+__device__ __forceinline__ void store_h_units(uint8_t* hi, uint8_t* lo, int col0, int n0, const float* hv,
+                                              uint16_t* scratch) {
+  const int lane = threadIdx.x & 31;
+  if ((lane & 1) == 0) {
+    const int m = lane >> 1;
+#pragma unroll
+    for (int i = 0; i < CW; ++i) {
+      const __nv_bfloat16 hb = __float2bfloat16_rn(hv[i]);
+      const __nv_bfloat16 lb = __float2bfloat16_rn(hv[i] - __bfloat162float(hb));
+      scratch[i * 16 + m] = *reinterpret_cast<const uint16_t*>(&hb);
+      scratch[(CW + i) * 16 + m] = *reinterpret_cast<const uint16_t*>(&lb);
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = lane; u < 4 * CW; u += 32) {  // (hi or lo, token, feature half)
+    const int part = u / (2 * CW), rem = u % (2 * CW), i = rem >> 1, fh = rem & 1;
+    const uint4 x = *reinterpret_cast<const uint4*>(scratch + (part * CW + i) * 16 + 8 * fh);
+    *reinterpret_cast<uint4*>((part ? lo : hi) + sw128_offset(n0 + i, col0 + 8 * fh)) = x;
+  }
+  __syncwarp();
+}
+
+template <int CW>
+__device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, const float* v, uint16_t* scratch) {
   const int f = T.a0 * 128 + fl;
   const int tb = T.a1;
   const int lane = threadIdx.x & 31;
@@ -1275,21 +1303,17 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       break;
     case OP_BGU: {
       const int nb = active_batch(P);
-      const int col = fl / 2;  // h feature 64 * a0 + col
+      // h features 64 a0 + fl / 2; the warp's 16 start at column (fl - lane) / 2
       uint8_t* hi = P.h_img[0] + (size_t)T.a0 * P.img_stride;
       uint8_t* lo = P.h_img[1] + (size_t)T.a0 * P.img_stride;
+      float hv[CW];
 #pragma unroll
       for (int i = 0; i < CW; ++i) {
         const float g = v[i] * s_rn[n0 + i];
         const float up = __shfl_xor_sync(0xffffffffu, g, 1);
-        if (lane & 1) continue;
-        const int n = n0 + i;
-        const float hv = (n < nb) ? g / (1.0f + expf(-g)) * up : 0.f;
-        const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
-        const uint32_t off = sw128_offset(n, col);
-        *reinterpret_cast<__nv_bfloat16*>(hi + off) = hb;
-        *reinterpret_cast<__nv_bfloat16*>(lo + off) = __float2bfloat16_rn(hv - __bfloat162float(hb));
+        hv[i] = (n0 + i < nb) ? g / (1.0f + expf(-g)) * up : 0.f;  // even lanes: gate, odd: up
       }
+      store_h_units<CW>(hi, lo, (fl - lane) / 2, n0, hv, scratch);
       break;
     }
     case OP_BLM: {
@@ -1360,23 +1384,18 @@ __device__ void mma_epilogue(const KParams& P, const Tile& T, int fl, int n0, co
       break;
     }
     case OP_MGU: {
-      const int j = f / 2, c = j / 64, col = j % 64, nkc = P.ffn / 64;
+      // the warp's 16 h features start at j0 (a multiple of 16: one chunk)
+      const int j0 = (f - lane) / 2, c = j0 / 64, nkc = P.ffn / 64;
       uint8_t* hi = P.h_img[0] + ((size_t)tb * nkc + c) * P.img_stride;
       uint8_t* lo = P.h_img[1] + ((size_t)tb * nkc + c) * P.img_stride;
+      float hv[CW];
 #pragma unroll
       for (int i = 0; i < CW; ++i) {
         const float up = __shfl_xor_sync(0xffffffffu, v[i], 1);
-        if (lane & 1) continue;
-        const int n = n0 + i;
-        const int m = tb * kTokBlock + n;
         const float g = v[i];
-        const float hv = (m < P.M) ? g / (1.0f + expf(-g)) * up : 0.f;
-        const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
-        const __nv_bfloat16 lb = __float2bfloat16_rn(hv - __bfloat162float(hb));
-        const uint32_t off = sw128_offset(n, col);
-        *reinterpret_cast<__nv_bfloat16*>(hi + off) = hb;
-        *reinterpret_cast<__nv_bfloat16*>(lo + off) = lb;
+        hv[i] = (tb * kTokBlock + n0 + i < P.M) ? g / (1.0f + expf(-g)) * up : 0.f;  // even lanes: gate, odd: up
       }
+      store_h_units<CW>(hi, lo, j0 % 64, n0, hv, scratch);
       break;
     }
     default:
@@ -1526,6 +1545,9 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, half = warp >> 2;
   const int fl = 32 * q + lane;
+  // the warp's shared scratch for the gate/up output (the activation buffer:
+  // no other tile body uses it while this one runs)
+  uint16_t* scratch = reinterpret_cast<uint16_t*>(S.act) + warp * (2 * 16 * 16);
   if (P.dec_mma) {
     for (int cg = half; cg < N / 8; cg += 2) {  // 8-column groups alternate between the two warp halves
       float v[8];
@@ -1534,7 +1556,7 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
       const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(8 * cg);
       for (int a = 0; a < NA; ++a)  // hi and lo parts of every accumulator
         tmem_add8x2(lane_base + (uint32_t)(a * 2 * N), lane_base + (uint32_t)(a * 2 * N + N), v);
-      mma_epilogue<8>(P, T, fl, 8 * cg, v);
+      mma_epilogue<8>(P, T, fl, 8 * cg, v, scratch);
     }
   } else {
     for (int cg = half; cg < N / 16; cg += 2) {  // 16-column groups alternate between the two warp halves
@@ -1544,7 +1566,7 @@ __device__ bool body_mma(const KParams& P, const Tile& T, const Shared& S, Curso
       const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(16 * cg);
       for (int a = 0; a < NA; ++a)  // hi and lo parts of every accumulator
         tmem_add16x2(lane_base + (uint32_t)(a * 2 * N), lane_base + (uint32_t)(a * 2 * N + N), v);
-      mma_epilogue<16>(P, T, fl, 16 * cg, v);
+      mma_epilogue<16>(P, T, fl, 16 * cg, v, scratch);
     }
   }
   tc_fence_before();
@@ -2299,9 +2321,9 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
           if (threadIdx.x == 0) record_error(P, WPK_ERR_UNSUPPORTED, t, kNoCounter, T.op, (uint32_t)kProg);
           ok = false;
         }
-        // attention tiles use the activation buffer as scratch; the gather
-        // rewrites the LM head's input
-        if (T.op == OP_ATTN || T.op == OP_PATTN || T.op == OP_GATHER) cs.act_key = kNoAct;
+        // attention and tensor-core tiles use the activation buffer as
+        // scratch; the gather rewrites the LM head's input
+        if (T.op == OP_ATTN || T.op == OP_PATTN || T.op == OP_GATHER || is_mma_op(T.op)) cs.act_key = kNoAct;
       }
       ok = cbar_and(ok);
       if (!ok) {
@@ -2386,34 +2408,34 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
 
 // Decode on CUDA cores: the persistent worker grid (one cooperative launch per
 // region per step, or one for many steps when resident).
-__global__ void __launch_bounds__(kCtaThreads, 1) wpk_persistent_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreadsGemv, 1) wpk_persistent_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   worker<kProgGemv>(P, smem_raw);
 }
 
 // Per-op launch: one CTA per tile of one op group; stream order replaces the
 // counters.  Used for the CUDA-Graph comparator.
-__global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreadsGemv, 1) wpk_per_op_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   worker<kProgGemv>(P, smem_raw);
 }
 
 // Batched decode on tensor cores: the same two launch forms.
-__global__ void __launch_bounds__(kCtaThreads, 1) wpk_persistent_mma_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreadsTc, 1) wpk_persistent_mma_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   worker<kProgMma>(P, smem_raw);
 }
-__global__ void __launch_bounds__(kCtaThreads, 1) wpk_per_op_mma_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreadsTc, 1) wpk_per_op_mma_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   worker<kProgMma>(P, smem_raw);
 }
 
 // The prefill program.
-__global__ void __launch_bounds__(kCtaThreads, 1) wpk_prefill_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreadsTc, 1) wpk_prefill_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   worker<kProgPrefill>(P, smem_raw);
 }
-__global__ void __launch_bounds__(kCtaThreads, 1) wpk_prefill_op_kernel(const KParams P) {
+__global__ void __launch_bounds__(kCtaThreadsTc, 1) wpk_prefill_op_kernel(const KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   worker<kProgPrefill>(P, smem_raw);
 }
@@ -2431,6 +2453,12 @@ const void* per_op_kernel_ptr(bool mma) {
   return mma ? reinterpret_cast<const void*>(&wpk_per_op_mma_kernel) : reinterpret_cast<const void*>(&wpk_per_op_kernel);
 }
 const void* prefill_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_prefill_kernel); }
+int cta_threads(const void* fn) {
+  return (fn == reinterpret_cast<const void*>(&wpk_persistent_kernel) ||
+          fn == reinterpret_cast<const void*>(&wpk_per_op_kernel))
+             ? kCtaThreadsGemv
+             : kCtaThreadsTc;
+}
 const void* prefill_op_kernel_ptr() { return reinterpret_cast<const void*>(&wpk_prefill_op_kernel); }
 
 }  // namespace wpk

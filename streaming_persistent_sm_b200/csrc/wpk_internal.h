@@ -11,7 +11,8 @@ namespace wpk {
 constexpr uint32_t kNoCounter = 0xFFFFFFFFu;
 constexpr int kThreads = 256;          // consumer (compute) threads per worker CTA
 constexpr int kWarps = kThreads / 32;
-constexpr int kCtaThreads = kThreads + 64;  // + the producer warp + the tensor-core issuer warp
+constexpr int kCtaThreadsGemv = kThreads + 32;  // + the producer warp
+constexpr int kCtaThreadsTc = kThreads + 64;    // + the producer warp + the tensor-core issuer warp
 constexpr int kStageBytes = 16384;     // one chunk stage of the staging ring
 constexpr int kMaxStages = 13;         // ring stages per worker
 // GEMV chunks (kStageBytes each) per ring stage of a staging slot of `slot`
