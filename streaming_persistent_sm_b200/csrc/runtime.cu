@@ -693,8 +693,9 @@ __device__ bool wait_seen(const KParams& P, int st, uint32_t target, volatile in
 // for that stage only, computes its rows and hands the stage back at once, so
 // a tile of any size streams through the ring and no block barrier is taken
 // per chunk.  Returns false on a wait failure.
-__device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks, int rpc,
-                          ConsumerState& cs, volatile int* abort) {
+template <int CPS>
+__device__ bool body_gemv_t(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks, int rpc,
+                            ConsumerState& cs, volatile int* abort) {
   const int K = T.a3, R = T.a1;
   const int nb = active_batch(P);
   const LayerDev* L = P.layers + (T.op == OP_LMHEAD ? 0 : T.layer);
@@ -710,7 +711,10 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
   }
   int bgmax = P.act_bytes / (act_stride(K) * 4);
   if (bgmax > kMaxGemvBatch) bgmax = kMaxGemvBatch;
-  const int cps = P.gemv_cps, n_real = (R + rpc - 1) / rpc;  // chunks: gemv_cps per stage
+  // chunks, CPS (= gemv_cps, a constant: the per-chunk divisions by a
+  // run-time value cost the b1 step 16 us) per stage
+  constexpr int cps = CPS;
+  const int n_real = (R + rpc - 1) / rpc;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   bool ok = true;
   for (int b0 = 0; b0 < nb || (nb == 0 && b0 == 0); b0 += bgmax) {
@@ -771,6 +775,12 @@ __device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Curs
   }
   cur.c += n_chunks;
   return true;
+}
+
+__device__ bool body_gemv(const KParams& P, const Tile& T, const Shared& S, Cursor& cur, int n_chunks, int rpc,
+                          ConsumerState& cs, volatile int* abort) {
+  return P.gemv_cps == 2 ? body_gemv_t<2>(P, T, S, cur, n_chunks, rpc, cs, abort)
+                         : body_gemv_t<1>(P, T, S, cur, n_chunks, rpc, cs, abort);
 }
 
 // ---------------------------------------------------------------------------
@@ -2313,7 +2323,10 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
             else known = false;
             break;
           default:  // GEMV tiles (decode ops, and the prefill's LM head)
-            if constexpr (kProg != kProgMma) ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort);
+            if constexpr (kProg == kProgPrefill)  // (one chunk per stage there)
+              ok = body_gemv_t<1>(P, T, S, cur, n_chunks, rpc, cs, &s_abort);
+            else if constexpr (kProg != kProgMma)
+              ok = body_gemv(P, T, S, cur, n_chunks, rpc, cs, &s_abort);
             else known = false;
             break;
         }
