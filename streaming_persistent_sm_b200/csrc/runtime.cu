@@ -345,33 +345,63 @@ __device__ void issue_mma_act(const KParams& P, const Tile& T, int u, uint8_t* d
   }
 }
 
-// Copies of chunk `k` of tile T into `dst`; arms `bar` with their bytes.
-__device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uint8_t* dst, uint64_t* bar) {
-  if (T.op == OP_PATTN || T.op == OP_ATTN) {
-    // whole KV pages - a page's K rows, then its V rows at page * head_dim -
-    // one copy each (rows past the span are never read); prefill attention:
-    // page k of sequence a0, kv head a1; decode: pages k * attn_pps .. of the
-    // split, packed into the stage
-    const uint32_t bytes = 2u * (uint32_t)P.page_tokens * (uint32_t)P.head_dim * 2u;
-    if (T.op == OP_PATTN) {
-      int t0, t1, k0, k1;
-      pattn_span(P, T, &t0, &t1);
-      pattn_keys(P, T, t1, &k0, &k1);
-      const int blk = P.block_table[(P.slot0 + T.a0) * P.max_blocks + k0 / P.page_tokens + k];
-      mbar_arrive_expect_tx(bar, bytes);
-      bulk_g2s(dst, P.kv + kv_index(P, T.layer, blk, 0, T.a1, 0), bytes, bar);
-      return;
-    }
-    const AttnSpan s = attn_span(P, T);
-    const int first = s.t0 / P.page_tokens + k * attn_pps(P);
-    const int n = min(attn_pps(P), (s.t1 - 1) / P.page_tokens + 1 - first);
-    mbar_arrive_expect_tx(bar, (uint32_t)n * bytes);
-    for (int j = 0; j < n; ++j) {
-      const int blk = P.block_table[s.b * P.max_blocks + first + j];
-      bulk_g2s(dst + (size_t)j * bytes, P.kv + kv_index(P, T.layer, blk, 0, s.g, 0), bytes, bar);
-    }
-    return;
+// The KV pages an attention tile stages: whole pages (a page's K rows, then
+// its V rows at page * head_dim), one copy each, pps per ring stage; prefill
+// attention: pages of sequence a0, kv head a1 over the tile's keys, one per
+// stage; decode: the split's pages, packed into the stages.  Computed once per
+// tile by the producer.
+struct PageWalk {
+  const int32_t* row;  // the sequence's block-table row
+  int first, n_pages, pps, g;
+};
+__device__ PageWalk page_walk(const KParams& P, const Tile& T) {
+  PageWalk w;
+  if (T.op == OP_PATTN) {
+    int t0, t1, k0, k1;
+    pattn_span(P, T, &t0, &t1);
+    pattn_keys(P, T, t1, &k0, &k1);
+    w.row = P.block_table + (size_t)(P.slot0 + T.a0) * P.max_blocks;
+    w.first = k0 / P.page_tokens;
+    w.n_pages = (k1 - 1) / P.page_tokens - w.first + 1;
+    w.pps = 1;
+    w.g = T.a1;
+  } else {
+    const AttnSpan sp = attn_span(P, T);
+    w.row = P.block_table + (size_t)sp.b * P.max_blocks;
+    w.first = sp.t0 / P.page_tokens;
+    w.n_pages = sp.t1 > sp.t0 ? (sp.t1 - 1) / P.page_tokens + 1 - w.first : 0;
+    w.pps = attn_pps(P);
+    w.g = sp.g;
   }
+  return w;
+}
+
+// Block ids of the first kPagePrefetch pages of stage k, loaded together (the
+// producer loads them before it waits for the stage: one dependent L2 round
+// trip per page took a b16 attention tile's four stages 14 us to issue).
+constexpr int kPagePrefetch = 8;
+__device__ __forceinline__ void page_blocks(const PageWalk& w, int k, int* blk) {
+  const int p0 = w.first + k * w.pps, n = min(w.pps, w.n_pages - k * w.pps);
+#pragma unroll
+  for (int j = 0; j < kPagePrefetch; ++j) blk[j] = j < n ? __ldcg(w.row + p0 + j) : 0;
+}
+
+// Copies of stage k of an attention tile into `dst`; arms `bar` with their
+// bytes.  blk holds the stage's first block ids (page_blocks).
+__device__ void issue_pages(const KParams& P, const Tile& T, const PageWalk& w, int k, const int* blk, uint8_t* dst,
+                            uint64_t* bar) {
+  const uint32_t bytes = 2u * (uint32_t)P.page_tokens * (uint32_t)P.head_dim * 2u;
+  const int p0 = w.first + k * w.pps, n = min(w.pps, w.n_pages - k * w.pps);
+  mbar_arrive_expect_tx(bar, (uint32_t)n * bytes);
+#pragma unroll
+  for (int j = 0; j < kPagePrefetch; ++j)
+    if (j < n) bulk_g2s(dst + (size_t)j * bytes, P.kv + kv_index(P, T.layer, blk[j], 0, w.g, 0), bytes, bar);
+  for (int j = kPagePrefetch; j < n; ++j)
+    bulk_g2s(dst + (size_t)j * bytes, P.kv + kv_index(P, T.layer, __ldcg(w.row + p0 + j), 0, w.g, 0), bytes, bar);
+}
+
+// Copies of GEMV stage k of tile T into `dst`; arms `bar` with their bytes.
+__device__ void issue_chunk(const KParams& P, const Tile& T, int k, int rpc, uint8_t* dst, uint64_t* bar) {
   // GEMV stage k: chunks k gemv_cps .. (consecutive rows), one copy
   const size_t row_bytes = (size_t)T.a3 * 2;
   const int r0 = k * P.gemv_cps * rpc;
@@ -2160,9 +2190,19 @@ __device__ void worker(const KParams& P, uint8_t* smem_raw) {
             if (!P.per_op && !wait_counter(P, T, t, e.epoch, &s_abort)) stop = true;
             else fence_proxy_async_global();
           }
-          for (int k = 0; k < nch && !stop; ++k, ++c) {
-            if (!free_stage(c)) { stop = true; break; }
-            issue_chunk(P, T, k, rpc, stage_ptr(c), &S.full[c % P.n_stages]);
+          if (T.op == OP_ATTN || T.op == OP_PATTN) {
+            const PageWalk w = page_walk(P, T);
+            for (int k = 0; k < nch && !stop; ++k, ++c) {
+              int blk[kPagePrefetch];
+              page_blocks(w, k, blk);
+              if (!free_stage(c)) { stop = true; break; }
+              issue_pages(P, T, w, k, blk, stage_ptr(c), &S.full[c % P.n_stages]);
+            }
+          } else {
+            for (int k = 0; k < nch && !stop; ++k, ++c) {
+              if (!free_stage(c)) { stop = true; break; }
+              issue_chunk(P, T, k, rpc, stage_ptr(c), &S.full[c % P.n_stages]);
+            }
           }
         }
         // the entry is still owned by the consumers until they release it;
