@@ -108,6 +108,7 @@ struct wpk_handle {
   size_t off_px = 0, off_pq = 0, off_xn = 0, off_att = 0, off_hi = 0, off_ppart = 0;
   int64_t prefill_max_tokens = 0;
   int prefill_stages = 0;
+  int prefill_cps = 1;  // K chunks per prefill ring stage
   size_t smem_prefill = 0;
   // program the inspection calls refer to (nullptr = the decode program)
   PrefillProgram* selected = nullptr;
@@ -582,7 +583,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.sig = prog->d_sig;
   P.ctr = prog->d_ctr;
   P.trace_buf = prog->d_trace;
-  P.stage_bytes = 3 * kMmaChunkBytes;
+  P.stage_bytes = h->prefill_cps * 3 * kMmaChunkBytes;
   P.n_stages = h->prefill_stages;
   P.gemv_cps = 1;
   P.uses_tmem = 1;
@@ -592,7 +593,7 @@ KParams prefill_params(const wpk_handle* h, const PrefillProgram* prog, const in
   P.mma_n = kTokBlock;
   P.act_chunk = kMmaChunkBytes;
   P.img_stride = 2 * kMmaChunkBytes;  // hi and lo halves of a chunk adjacent
-  P.mma_cps = 1;
+  P.mma_cps = h->prefill_cps;
   set_mma_geometry(&P);
   P.M = g.M;
   P.T = g.T;
@@ -708,9 +709,16 @@ static int setup_device(wpk_handle* h) {
     CUDA_TRY(h, cudaFuncGetAttributes(&fa, prefill_kernel_ptr()));
     const size_t fixed = worker_smem_bytes(0, 0, p.act_bytes) + fa.sharedSizeBytes;
     if (fixed >= (size_t)kMaxSmem) return fail(h, WPK_ERR_UNSUPPORTED, "no room for the prefill staging ring");
-    h->prefill_stages = (int)std::min<size_t>(kMaxStages, ((size_t)kMaxSmem - fixed) / (3 * kMmaChunkBytes));
+    // a stage holds cps K chunks of weights (16 KB each) and their 128
+    // tokens' hi and lo rows (32 KB each): two chunks per stage when two such
+    // stages fit, since a worker completes about one stage per half
+    // microsecond whatever its size
+    const size_t room = (size_t)kMaxSmem - fixed;
+    h->prefill_cps = room / (2 * 3 * kMmaChunkBytes) >= 2 ? 2 : 1;
+    const size_t stage = (size_t)h->prefill_cps * 3 * kMmaChunkBytes;
+    h->prefill_stages = (int)std::min<size_t>(kMaxStages, room / stage);
     if (h->prefill_stages < 2) return fail(h, WPK_ERR_UNSUPPORTED, "no room for the prefill staging ring");
-    h->smem_prefill = worker_smem_bytes(h->prefill_stages, 3 * kMmaChunkBytes, p.act_bytes);
+    h->smem_prefill = worker_smem_bytes(h->prefill_stages, (int)stage, p.act_bytes);
   }
   const size_t smem_max = h->smem;
   CUDA_TRY(h, raise_smem_limit(persistent_kernel_ptr(h->g.plan.decode_mode == WPK_DECODE_MMA), smem_max));
